@@ -1,0 +1,296 @@
+"""Seeded synthetic inputs for the one-GPU MoE layer forward.
+
+This module is the only code that both the CUDA path's tests/bench and the
+CPU oracle consume.  It draws random numbers and lays them out in the byte
+formats the layer takes; it holds none of the layer's arithmetic (no logits,
+no top-k, no softmax, no permutation, no matmul).
+
+Workloads (the five shapes the layer is measured and checked on):
+
+* ``fp32_n256_d256_e8_k2_f1024_relu``      fp32, ReLU FFN d->1024->d
+* ``bf16_n4096_d2048_e8_k2_f8192_swiglu``   bf16, SwiGLU FFN, ~uniform routing
+* ``bf16_n64_d4096_e64_k8_f1408_swiglu``    bf16, decode-shaped (weight streaming)
+* ``bf16_n16384_d2048_e128_k8_f768_swiglu_zipf``  bf16, fine-grained experts,
+  router bias 1.2*ln(1/rank) (Zipf-like skew, some experts empty)
+* ``e4m3_n8192_h7168_e256_k8_n2048_gmm``    fp8 e4m3 per-tensor grouped matmul
+  + token-major unpermute, plus a shared-expert matmul (8192x7168)@(7168x2048)
+
+Value recipe: x ~ N(0,1); router and expert weights ~ N(0, 1/fan_in)
+(fan_in = d for the router and the first FFN matrices, F for the second);
+for the fp8 workload x and W ~ N(0,1) quantised with one amax scale per
+tensor (scale = amax/448, e4m3 round-to-nearest-even, saturating).  Routing
+for the fp8 workload is an ordered set of K distinct experts per token, drawn
+uniformly (the same law as the top-K of iid N(0,1) logits).
+
+Physical weight layout: every expert matrix is stored output-major,
+``(E, d_out, d_in)`` row-major (the layout of a Linear layer's weight), i.e.
+the per-expert transpose of the logical ``(e, H1, N1)`` gmmWeight shape of the
+Ascend grouped-matmul page ("aclnnQuantGroupedMatMulAlltoAllv", parameter
+constraints).  The router weight is ``(d, E)`` row-major fp32.
+
+Random streams: numpy Philox bit generators seeded from
+``SeedSequence([seed, stream_id])`` and spawned per 16 Mi-element chunk, so
+the bytes are independent of the thread count.
+"""
+from __future__ import annotations
+
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, field, replace
+
+import numpy as np
+import torch
+
+DTYPE_F32 = "f32"
+DTYPE_BF16 = "bf16"
+DTYPE_E4M3 = "e4m3"
+
+ACT_NONE = "none"
+ACT_RELU = "relu"
+ACT_SWIGLU = "swiglu"
+
+SEED_BASE = 0x4D6F45
+_CHUNK = 1 << 24
+
+
+@dataclass(frozen=True)
+class MoEConfig:
+    """Shape of one MoE layer workload.
+
+    For the fp8 grouped-matmul workload ``d`` is H1 (the routed experts'
+    input width), ``F`` is N1 (their output width) and ``shared`` holds
+    (H2, N2) of the shared expert.
+    """
+    name: str
+    dtype: str
+    N: int
+    d: int
+    E: int
+    K: int
+    F: int
+    act: str
+    index: int = 0
+    zipf_bias: float = 0.0          # router bias b_e = zipf_bias * ln(1/(e+1)); 0 = no bias
+    shared: tuple | None = None     # (H2, N2) shared-expert matmul, fp8 workload only
+    routing: str = "router"         # "router" (logits from x @ W_r) or "given" (drawn ids)
+
+    @property
+    def d_out(self) -> int:
+        return self.F if self.act == ACT_NONE else self.d
+
+    @property
+    def R(self) -> int:
+        return self.N * self.K
+
+    def scaled(self, **kw) -> "MoEConfig":
+        return replace(self, **kw)
+
+
+CONFIGS: dict[str, MoEConfig] = {}
+
+
+def _reg(cfg: MoEConfig) -> MoEConfig:
+    CONFIGS[cfg.name] = cfg
+    return cfg
+
+
+FP32_RELU = _reg(MoEConfig("fp32_n256_d256_e8_k2_f1024_relu", DTYPE_F32, 256, 256, 8, 2, 1024,
+                           ACT_RELU, index=0))
+BF16_PREFILL = _reg(MoEConfig("bf16_n4096_d2048_e8_k2_f8192_swiglu", DTYPE_BF16, 4096, 2048, 8, 2,
+                              8192, ACT_SWIGLU, index=1))
+BF16_DECODE = _reg(MoEConfig("bf16_n64_d4096_e64_k8_f1408_swiglu", DTYPE_BF16, 64, 4096, 64, 8,
+                             1408, ACT_SWIGLU, index=2))
+BF16_FINEGRAINED = _reg(MoEConfig("bf16_n16384_d2048_e128_k8_f768_swiglu_zipf", DTYPE_BF16, 16384,
+                                  2048, 128, 8, 768, ACT_SWIGLU, index=3, zipf_bias=1.2))
+FP8_GMM = _reg(MoEConfig("e4m3_n8192_h7168_e256_k8_n2048_gmm", DTYPE_E4M3, 8192, 7168, 256, 8, 2048,
+                         ACT_NONE, index=4, shared=(7168, 2048), routing="given"))
+
+
+# ----------------------------------------------------------------------------
+# random streams
+# ----------------------------------------------------------------------------
+
+def _threads() -> int:
+    return max(1, min(32, os.cpu_count() or 1))
+
+
+def normal_f32(seed: int, stream: int, n: int, std: float = 1.0) -> np.ndarray:
+    """n iid N(0, std^2) float32 values, chunked Philox streams."""
+    out = np.empty(n, np.float32)
+    nchunks = max(1, (n + _CHUNK - 1) // _CHUNK)
+    children = np.random.SeedSequence([seed, stream]).spawn(nchunks)
+
+    def work(i):
+        lo, hi = i * _CHUNK, min(n, (i + 1) * _CHUNK)
+        g = np.random.Generator(np.random.Philox(children[i]))
+        v = g.standard_normal(hi - lo, dtype=np.float32)
+        if std != 1.0:
+            v *= np.float32(std)
+        out[lo:hi] = v
+
+    if nchunks == 1:
+        work(0)
+    else:
+        with ThreadPoolExecutor(_threads()) as ex:
+            list(ex.map(work, range(nchunks)))
+    return out
+
+
+def uniform_u64(seed: int, stream: int, n: int) -> np.ndarray:
+    g = np.random.Generator(np.random.Philox(np.random.SeedSequence([seed, stream])))
+    return g.integers(0, np.iinfo(np.uint64).max, size=n, dtype=np.uint64, endpoint=True)
+
+
+# ----------------------------------------------------------------------------
+# storage formats (input preparation only)
+# ----------------------------------------------------------------------------
+
+def to_bf16(a: np.ndarray) -> torch.Tensor:
+    """float32 -> bf16 (round to nearest even), as a torch CPU tensor."""
+    return torch.from_numpy(a).to(torch.bfloat16)
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """Encode float values as OCP FP8 E4M3 ("FN": bias 7, max 448, no inf)
+    bytes, round-to-nearest-even, saturating to +-448.  Input preparation for
+    the pre-quantised fp8 workload (the grouped matmul consumes codes and
+    scales, as the Ascend page's gmmX/gmmWeight do)."""
+    v = np.asarray(v, np.float64)
+    sign = (np.signbit(v)).astype(np.uint8) << 7
+    a = np.minimum(np.abs(v), 448.0)
+    code = np.zeros(a.shape, np.int64)
+    sub = a < 2.0 ** -6
+    # subnormal grid: step 2^-9; q == 8 lands exactly on the smallest normal code 0x08
+    code[sub] = np.rint(a[sub] * 2.0 ** 9).astype(np.int64)
+    nrm = ~sub
+    if np.any(nrm):
+        an = a[nrm]
+        m, ex = np.frexp(an)            # an = m * 2^ex, m in [0.5, 1)
+        e = ex - 1                      # an = s * 2^e, s in [1, 2)
+        s = an / np.ldexp(1.0, e)
+        q = np.rint((s - 1.0) * 8.0).astype(np.int64)
+        carry = q == 8
+        e = e + carry
+        q = np.where(carry, 0, q)
+        code[nrm] = ((e + 7) << 3) | q
+    return (code.astype(np.uint8) | sign)
+
+
+def quantize_e4m3_per_tensor(a: np.ndarray) -> tuple[np.ndarray, float]:
+    """(codes, scale) with scale = amax/448 and codes = e4m3(a / scale)."""
+    amax = float(np.max(np.abs(a))) if a.size else 1.0
+    scale = amax / 448.0 if amax > 0 else 1.0
+    scale = float(np.float32(scale))
+    out = np.empty(a.shape, np.uint8)
+    flat_in, flat_out = a.reshape(-1), out.reshape(-1)
+    n = flat_in.size
+    nchunks = max(1, (n + _CHUNK - 1) // _CHUNK)
+
+    def work(i):
+        lo, hi = i * _CHUNK, min(n, (i + 1) * _CHUNK)
+        flat_out[lo:hi] = e4m3_encode(flat_in[lo:hi].astype(np.float64) / scale)
+
+    if nchunks == 1:
+        work(0)
+    else:
+        with ThreadPoolExecutor(_threads()) as ex:
+            list(ex.map(work, range(nchunks)))
+    return out, scale
+
+
+# ----------------------------------------------------------------------------
+# the workload
+# ----------------------------------------------------------------------------
+
+@dataclass
+class MoEInputs:
+    """Host (CPU) tensors of one workload.
+
+    ``x``       (N, d) in the workload dtype (f32 / bf16 / uint8 e4m3 codes)
+    ``w_r``     (d, E) float32, or None when routing is given
+    ``bias``    (E,) float32 or None
+    ``w1``      (E, F, d)  first matrix (ReLU W1, SwiGLU gate, or the single fp8 matrix)
+    ``w3``      (E, F, d)  SwiGLU up matrix, else None
+    ``w2``      (E, d, F)  second matrix, None for the single-matrix workload
+    ``ids``     (N, K) int32 routing given to the fp8 workload, else None
+    ``x_scale``, ``w_scale``  per-tensor fp32 scales (fp8 workload), else 1.0
+    ``w_sh``    (N2, H2) e4m3 shared-expert weight (output-major), ``w_sh_scale``
+    """
+    cfg: MoEConfig
+    x: torch.Tensor
+    w_r: torch.Tensor | None
+    bias: torch.Tensor | None
+    w1: torch.Tensor
+    w3: torch.Tensor | None
+    w2: torch.Tensor | None
+    ids: torch.Tensor | None = None
+    x_scale: float = 1.0
+    w_scale: float = 1.0
+    w_sh: torch.Tensor | None = None
+    w_sh_scale: float = 1.0
+    extra: dict = field(default_factory=dict)
+
+
+def zipf_bias(E: int, strength: float) -> np.ndarray:
+    """b_e = strength * ln(1/rank), rank = e + 1 (natural log), float32."""
+    return np.array([strength * math.log(1.0 / (e + 1)) for e in range(E)], np.float32)
+
+
+def given_routing(seed: int, N: int, E: int, K: int) -> np.ndarray:
+    """(N, K) int32: per token an ordered set of K distinct experts, uniform.
+
+    Partial Fisher-Yates per token driven by 64-bit uniforms (bias of the
+    modulo reduction is < E/2^64, immaterial)."""
+    u = uniform_u64(seed, 91, N * K).reshape(N, K)
+    ids = np.empty((N, K), np.int32)
+    base = np.arange(E, dtype=np.int32)
+    for t in range(N):
+        perm = base.copy()
+        for j in range(K):
+            r = j + int(u[t, j] % np.uint64(E - j))
+            perm[j], perm[r] = perm[r], perm[j]
+        ids[t] = perm[:K]
+    return ids
+
+
+def make_inputs(cfg: MoEConfig, seed: int | None = None) -> MoEInputs:
+    """Draw the workload's inputs.  Deterministic in (cfg shape, seed)."""
+    if seed is None:
+        seed = SEED_BASE + cfg.index
+    N, d, E, K, F = cfg.N, cfg.d, cfg.E, cfg.K, cfg.F
+    if cfg.dtype == DTYPE_E4M3:
+        xf = normal_f32(seed, 1, N * d).reshape(N, d)
+        xq, xs = quantize_e4m3_per_tensor(xf)
+        wf = normal_f32(seed, 2, E * F * d).reshape(E, F, d)
+        wq, ws = quantize_e4m3_per_tensor(wf)
+        del wf
+        inp = MoEInputs(cfg, torch.from_numpy(xq), None, None, torch.from_numpy(wq), None, None,
+                        ids=torch.from_numpy(given_routing(seed, N, E, K)), x_scale=xs, w_scale=ws)
+        if cfg.shared is not None:
+            H2, N2 = cfg.shared
+            assert H2 == d, "the shared expert reads the same token matrix"
+            shf = normal_f32(seed, 3, N2 * H2).reshape(N2, H2)
+            shq, shs = quantize_e4m3_per_tensor(shf)
+            inp.w_sh, inp.w_sh_scale = torch.from_numpy(shq), shs
+        return inp
+
+    conv = (lambda a: torch.from_numpy(a)) if cfg.dtype == DTYPE_F32 else to_bf16
+    x = conv(normal_f32(seed, 1, N * d).reshape(N, d))
+    w_r = torch.from_numpy(normal_f32(seed, 4, d * E, 1.0 / math.sqrt(d)).reshape(d, E))
+    bias = torch.from_numpy(zipf_bias(E, cfg.zipf_bias)) if cfg.zipf_bias else None
+    w1 = conv(normal_f32(seed, 2, E * F * d, 1.0 / math.sqrt(d)).reshape(E, F, d))
+    w3 = None
+    if cfg.act == ACT_SWIGLU:
+        w3 = conv(normal_f32(seed, 5, E * F * d, 1.0 / math.sqrt(d)).reshape(E, F, d))
+    w2 = conv(normal_f32(seed, 6, E * d * F, 1.0 / math.sqrt(F)).reshape(E, d, F))
+    return MoEInputs(cfg, x, w_r, bias, w1, w3, w2)
+
+
+def small_variant(cfg: MoEConfig, **kw) -> MoEConfig:
+    """A reduced copy of a workload (same dtype/act/routing law) for tests."""
+    return replace(cfg, name=cfg.name + "_small", **kw)
+
+
+def dtype_bytes(dtype: str) -> int:
+    return {DTYPE_F32: 4, DTYPE_BF16: 2, DTYPE_E4M3: 1}[dtype]
