@@ -1,0 +1,384 @@
+"""Benchmark of the one-GPU MoE layer forward (router -> permute -> grouped
+FFN -> combine) on the bf16 prefill workload: N=4096 tokens, d=2048, E=8
+experts, top-2, SwiGLU FFN d->8192->d, fp32 router; seeded synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0.  ``value`` is whole-job tokens/s from CUDA events on
+the launching stream (max over ranks), inputs resident in HBM, L2 flushed
+(a 256 MiB write) before every step.  ``e2e`` is the same metric through the
+host-buffer entry point (moe_forward_host: pinned H2D of x, the layer, D2H of
+y).  ``roofline`` reports the dominant kernel (the fused gate/up SwiGLU grouped
+GEMM) against the measured bf16 tensor peak.  ``cpu_baseline`` times the CPU
+oracle on a bounded sample of the same workload.  Under torchrun (N > 1) every
+rank runs an independent replica of the layer on its own GPU (the layer needs
+no exchange between GPUs: weak scaling).
+
+``--impl reference`` times the CPU oracle itself (the reference arm: it is
+the plain fp64 restatement of the method), on the host cores, one bounded
+token sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s and grouped-GEMM TFLOP/s (% of tensor/HBM roofline), 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="bf16_n4096_d2048_e8_k2_f8192_swiglu")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("gemm_tc.cu", "kernels.h", "common.cuh"):
+        with open(os.path.join(ROOT, "top_routing_grouped_gemv_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if
+    it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_sha = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_b or m_sha.group(1) != kernel_source_hash():
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """NVML sampling of SM clock and throttle reasons on this process's GPU."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            except Exception:
+                pass
+            h = None
+            if uuid:
+                for i in range(pynvml.nvmlDeviceGetCount()):
+                    hh = pynvml.nvmlDeviceGetHandleByIndex(i)
+                    u = pynvml.nvmlDeviceGetUUID(hh)
+                    u = u.decode() if isinstance(u, bytes) else u
+                    if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                        h = hh
+            self.h = h or pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, keep going
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.stop = threading.Event()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def gemm_flops(cfg, rows: int):
+    """Algorithmic FLOPs of the grouped FFN over the actual routed rows."""
+    if cfg.act == "swiglu":
+        return 2.0 * rows * cfg.d * 2 * cfg.F, 2.0 * rows * cfg.F * cfg.d
+    if cfg.act == "relu":
+        return 2.0 * rows * cfg.d * cfg.F, 2.0 * rows * cfg.F * cfg.d
+    return 2.0 * rows * cfg.d * cfg.F, 0.0
+
+
+def oracle_sample_tokens(cfg, inp, target_s: float, max_tokens: int | None = None):
+    """Time the oracle's whole-layer forward on a token sample sized to take
+    about target_s seconds; returns (tokens, seconds, threads)."""
+    import numpy as np
+    import oracle
+    threads = oracle.num_threads()
+    n = max(1, threads)
+    t0 = time.perf_counter()
+    oracle.forward_tokens(inp, np.arange(n))
+    dt = time.perf_counter() - t0
+    n2 = int(min(max_tokens or cfg.N, max(n, n * target_s / max(dt, 1e-6))))
+    n2 = max(threads, n2 // threads * threads) if n2 >= threads else n2
+    rng = np.random.default_rng(17)
+    tok = np.sort(rng.choice(cfg.N, size=min(n2, cfg.N), replace=False))
+    t0 = time.perf_counter()
+    oracle.forward_tokens(inp, tok)
+    return len(tok), time.perf_counter() - t0, threads
+
+
+def run_reference(args, rank: int):
+    import numpy as np
+    import oracle
+    import synth
+    cfg = synth.CONFIGS[args.workload]
+    if rank != 0:
+        return
+    oracle.build()
+    inp = synth.make_inputs(cfg)
+    threads = oracle.num_threads()
+    per = max(1, threads)
+    rng = np.random.default_rng(23)
+    for _ in range(args.warmup):
+        oracle.forward_tokens(inp, rng.choice(cfg.N, size=per, replace=False))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward_tokens(inp, rng.choice(cfg.N, size=per, replace=False))
+    dt = time.perf_counter() - t0
+    value = per * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "N": cfg.N, "d": cfg.d, "E": cfg.E, "K": cfg.K,
+                   "F": cfg.F, "act": cfg.act, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{per} random tokens of the {cfg.N}-token batch per step "
+                                   "(route, K experts, combine), fp64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import numpy as np
+    import torch
+    import synth
+    import top_routing_grouped_gemv_b200 as moe
+
+    assert torch.cuda.is_available(), "bench needs a CUDA device"
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    moe.build()
+    moe.load()
+
+    cfg = synth.CONFIGS[args.workload]
+    inp = synth.make_inputs(cfg)
+    w = {"w1": inp.w1.cuda(), "w_scale": inp.w_scale}
+    for k, t in (("w3", inp.w3), ("w2", inp.w2), ("w_r", inp.w_r), ("bias", inp.bias)):
+        if t is not None:
+            w[k] = t.cuda()
+    plan = moe.Plan(cfg.N, cfg.d, cfg.E, cfg.K, cfg.F, cfg.dtype, cfg.act, w)
+    ws = plan.new_workspace()
+    x = inp.x.cuda()
+    ydt = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
+    y = torch.empty(cfg.N, cfg.d_out, dtype=ydt, device="cuda")
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        plan.forward(x, y, ws)
+
+    # warm-up
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert plan.read_device_status(ws) == 0, "device status after warm-up"
+    launches_per_step = plan.last_launch_count()
+
+    # timed region: K steps back to back (the host runs ahead of the GPU),
+    # CUDA events around every step on the launching stream
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+        # per-kernel durations: the library records events between its
+        # kernels; a short GPU sleep before each step lets the host enqueue
+        # the whole step first, so no launch gap lands inside a kernel's span
+        plan.profile(True)
+        per_kernel: dict[str, list[float]] = {}
+        for i in range(min(args.steps, 50)):
+            flush.zero_()
+            torch.cuda._sleep(400_000)
+            step()
+            for name, ms in plan.profile_read():
+                per_kernel.setdefault(name, []).append(ms)
+        plan.profile(False)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    assert plan.read_device_status(ws) == 0, "device status after timing"
+    value = world * cfg.N * args.steps / (total_ms / 1e3)
+
+    # end to end through the host-buffer entry point
+    e2e = None
+    if not args.no_e2e:
+        xh = inp.x.clone().pin_memory()
+        yh = torch.empty(cfg.N, cfg.d_out, dtype=ydt).pin_memory()
+        for _ in range(min(args.warmup, 3)):
+            plan.forward_host(xh, yh, ws)
+        n_e2e = max(1, min(args.steps, 200))
+        e_ms = 0.0
+        if dist:
+            dist.barrier()
+        for _ in range(n_e2e):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            plan.forward_host(xh, yh, ws)
+            b.record(stream)
+            b.synchronize()
+            e_ms += a.elapsed_time(b)
+        if dist:
+            t = torch.tensor([e_ms], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * cfg.N * n_e2e / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+               "d2h_bytes_per_step": yh.numel() * yh.element_size(), "steps": n_e2e}
+
+    # roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    R = cfg.N * cfg.K
+    f1, f2 = gemm_flops(cfg, R)
+    k1 = "ffn1_swiglu_tc" if cfg.act == "swiglu" else ("gmm_tc" if cfg.act == "none" else "ffn1_simt_f32")
+    stage_us = {k: 1e3 * statistics.mean(v) for k, v in per_kernel.items()}
+    sustained = wall > 2.0
+    peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    t1 = stage_us.get(k1, float("nan")) * 1e-6
+    achieved = f1 / t1 / 1e12
+    traffic = profiled_traffic(cfg.name, k1)
+    roofline = {"bound": "tensor", "kernel": k1, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'}",
+                "algorithmic_flop_per_launch": f1}
+    ffn_keys = [k for k in stage_us if k.startswith("ffn") or k.startswith("gmm")]
+    ffn_s = sum(stage_us[k] for k in ffn_keys) * 1e-6
+    gemm = {"tflops": (f1 + f2) / ffn_s / 1e12, "frac_of_peak": (f1 + f2) / ffn_s / 1e12 / peak,
+            "flop_per_step": f1 + f2}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        n_tok, secs, threads = oracle_sample_tokens(cfg, inp, args.cpu_seconds)
+        cpu = {"value": n_tok / secs, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n_tok} random tokens of the {cfg.N}-token batch (route, K experts, "
+                         f"combine; fp64), {secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": cfg.name, "N": cfg.N, "d": cfg.d, "E": cfg.E, "K": cfg.K,
+                       "F": cfg.F, "act": cfg.act, "router": "fp32",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed (256 MiB write) before every step",
+                       "inputs": "seeded synthetic, resident in HBM"},
+            "roofline": roofline, "gemm": gemm,
+            "stages_us": {k: round(v, 2) for k, v in stage_us.items()},
+            "cpu_baseline": cpu, "clocks": clk.summary(), "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    del plan
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

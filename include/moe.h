@@ -1,0 +1,222 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) Mixture-of-Experts layer forward.
+ *
+ * One MoE layer forward on one GPU, in four stages, each a hand-written CUDA
+ * kernel (or a short chain of them) behind one entry point:
+ *
+ *   moe_router_topk        router logits, top-K, softmax over the kept K
+ *   moe_permute            expert histogram, prefix scan, stable gather
+ *   moe_grouped_ffn        every expert's FFN as one grouped GEMM launch chain
+ *   moe_unpermute_combine  y = sum_j g_j * E_j(x)  (or a pure unpermute)
+ *   moe_forward            all four, one stream, no host synchronisation
+ *
+ * Sources (web pages): "Advanced GPU Optimization: How to tech an LLM with
+ * CUDA and ROCm? - Part 5" sections 1.1 (router kernel, top-2, sparse softmax)
+ * and 1.2 (tokens grouped by destination expert, local expert FFNs);
+ * "aclnnQuantGroupedMatMulAlltoAllv" (Ascend CANN) function/formula sections
+ * (gmmY = (gmmX @ gmmWeight) * gmmXScale * gmmWeightScale, Unpermute, the
+ * parallel shared-expert matmul, quant modes 0 = none / 1 = per-tensor), its
+ * return-value section (two-phase interface: validate and size the workspace
+ * first, then execute) and constraints (K in [2, 8], e*epWorldSize <= 256,
+ * H1, N1 < 65536, deterministic by default); zyxy.net "SpMM ... MoE" MoE
+ * structure section (y = sum_i g_i(x) E_i(x), gating (N,E), top-K (N,K)).
+ *
+ * Conventions for every call
+ *  - Pointers named *_host are host memory; every other data pointer is
+ *    device memory of the plan's device.  The caller allocates and frees all
+ *    of them.  The library allocates no device memory (not in
+ *    moe_plan_create either); it never frees caller memory.
+ *  - Launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  Only moe_read_device_status, moe_forward_host and
+ *    moe_profile_read synchronise.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    failed validation returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED /
+ *    MOE_ERR_WORKSPACE_TOO_SMALL and launches nothing.
+ *  - Errors found on the device (an expert id outside [0, E), a permutation
+ *    index outside [0, N*K), a pipeline wait that ran out of time) are
+ *    recorded in a sticky status word at the start of the workspace; the
+ *    kernel skips the offending access and finishes.  Read (and clear) it
+ *    with moe_read_device_status.
+ *  - Results are deterministic: the same inputs give the same bytes (no
+ *    floating-point atomics, fixed summation orders, stable permutation).
+ *  - All row pointers must be 16-byte aligned and every row a multiple of
+ *    16 bytes (d * sizeof(dtype) % 16 == 0).
+ *
+ * Layouts (row-major throughout)
+ *  x          (N, d)        dtype (fp32, bf16 or e4m3 codes)
+ *  w_r        (d, E)        fp32 router weight
+ *  router_bias(E)           fp32 or NULL
+ *  w1         (E, F, d)     ReLU W1 / SwiGLU gate / the single fp8 matrix;
+ *                           each expert output-major (the transpose of the
+ *                           Ascend page's logical (e, H1, N1)), like a Linear
+ *                           layer's weight
+ *  w3         (E, F, d)     SwiGLU up matrix (NULL otherwise)
+ *  w2         (E, d, F)     second matrix (NULL for MOE_ACT_NONE)
+ *  topk_ids   (N, K) int32, topk_gates (N, K) fp32, slots in descending logit
+ *  counts     (E) int32, offsets (E+1) int32 (offsets[E] = N*K)
+ *  perm_pos   (N*K) int32: row of x_perm that holds (token t, slot j)
+ *  perm_src   (N*K) int32: token of each x_perm row
+ *  x_perm     (N*K, d) dtype, expert-contiguous, stable within an expert
+ *  y_perm     (N*K, d_out)  d_out = d, or F for MOE_ACT_NONE; dtype = x's
+ *                           for fp32/bf16 layers, bf16 for e4m3 layers
+ *  y          (N, d_out), or (N*K, F) token-major for the pure unpermute
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,         /* bad pointer, size, alignment or limit */
+  MOE_ERR_UNSUPPORTED = 2,         /* valid but not built: dtype/act/quant combination */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below moe_workspace_size */
+  MOE_ERR_CUDA = 4,                /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE_BAD_INDEX = 5,    /* device: expert id or permutation index out of range */
+  MOE_ERR_DEVICE_TIMEOUT = 6       /* device: a bounded pipeline wait gave up */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
+
+/* Expert FFN form.  NONE: one matrix per expert, y = x W1^T (the grouped
+ * matmul of the Ascend page).  RELU: y = relu(x W1^T) W2^T.
+ * SWIGLU: y = (silu(x W1^T) * (x W3^T)) W2^T, silu(z) = z / (1 + exp(-z)). */
+typedef enum { MOE_ACT_NONE = 0, MOE_ACT_RELU = 1, MOE_ACT_SWIGLU = 2 } moe_act;
+
+/* Scale granularity; values equal the Ascend page's quant-mode enumeration
+ * (0 = not quantised, 1 = per-tensor).  Finer modes are not built. */
+typedef enum { MOE_QUANT_NONE = 0, MOE_QUANT_PER_TENSOR = 1 } moe_quant;
+
+typedef struct {
+  int32_t N;      /* tokens per call, >= 1 */
+  int32_t d;      /* token width (H1 of the grouped matmul), < 65536 */
+  int32_t E;      /* experts, 1..256 */
+  int32_t K;      /* experts kept per token, 1..8 and <= E */
+  int32_t F;      /* FFN inner width; for MOE_ACT_NONE the output width N1; < 65536 */
+  moe_dtype dtype;/* of x and the expert weights */
+  moe_act act;
+  moe_quant quant;/* MOE_QUANT_PER_TENSOR requires dtype MOE_E4M3, and vice versa */
+} moe_layer_desc;
+
+typedef struct {
+  const float* w_r;         /* (d, E) fp32; NULL if the caller always supplies routing */
+  const float* router_bias; /* (E) fp32 added to the logits before top-K, or NULL */
+  const void* w1;           /* (E, F, d) */
+  const void* w3;           /* (E, F, d) for SWIGLU, else NULL */
+  const void* w2;           /* (E, d, F) for RELU / SWIGLU, else NULL */
+  float w_scale;            /* per-tensor weight scale (gmmWeightScale) for e4m3, else ignored */
+} moe_layer_weights;
+
+typedef struct moe_plan_s* moe_plan;
+
+/* ---- phase 1: validate, build the executor, size the workspace ---------- */
+
+/* Validates desc and weights, records the weight pointers (not owned: they
+ * must stay valid while the plan is used) and encodes the TMA descriptors of
+ * the weights for the current CUDA device.  Allocates host memory only. */
+moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* weights,
+                           moe_plan* out);
+moe_status moe_plan_destroy(moe_plan plan);
+
+/* Bytes of device workspace that every call below accepts (the largest
+ * need, that of moe_forward_host).  Workspace base must be 256-byte aligned. */
+moe_status moe_workspace_size(moe_plan plan, size_t* bytes);
+
+/* Clears the device status word of a fresh workspace (stream-ordered). */
+moe_status moe_workspace_init(moe_plan plan, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---- phase 2: execute --------------------------------------------------- */
+
+/* Router (page 1 section 1.1; zyxy MoE expert-selection section).  For each
+ * token t: l[e] = sum_k x[t,k] * w_r[k,e] (+ router_bias[e]) in fp32; keep
+ * the K largest (descending, equal logits -> lower expert index); gates =
+ * softmax over the kept K only.  margin_or_null (N) receives l_(K) - l_(K+1)
+ * (+inf when K == E).  x dtype fp32 or bf16.  Needs plan weights.w_r. */
+moe_status moe_router_topk(moe_plan plan, const void* x, int32_t* topk_ids, float* topk_gates,
+                           float* margin_or_null, moe_stream_t stream);
+
+/* Permute / dispatch (page 1 section 1.2 token dispatch, local form; Ascend
+ * page sendCounts).  counts[e] = #{(t,j): ids[t,j] = e}; offsets = exclusive
+ * scan; perm_pos[t*K+j] = offsets[e] + #{(t',j') before (t,j) in (token,
+ * slot) order with the same expert}; perm_src[perm_pos] = t;
+ * x_perm[perm_pos[t*K+j]] = x[t] (byte copy).  Ids outside [0, E) set
+ * MOE_ERR_DEVICE_BAD_INDEX and are skipped.  Uses workspace scratch. */
+moe_status moe_permute(moe_plan plan, const void* x, const int32_t* topk_ids, int32_t* counts,
+                       int32_t* offsets, int32_t* perm_pos, int32_t* perm_src, void* x_perm,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped FFN (page 1 section 1.2 local expert execution; Ascend formula
+ * gmmY).  Rows [offsets[e], offsets[e+1]) of x_perm go through expert e; the
+ * result goes to the same rows of y_perm.  For e4m3: y_perm = (x_perm @
+ * W_e) * x_scale * w_scale in fp32, rounded once to bf16.  x_scale is the
+ * per-tensor gmmXScale (ignored unless e4m3).  offsets must be a valid
+ * non-decreasing prefix with offsets[E] = N*K (as moe_permute writes it).
+ * Uses workspace scratch (the SwiGLU/ReLU hidden activations). */
+moe_status moe_grouped_ffn(moe_plan plan, const void* x_perm, const int32_t* offsets,
+                           float x_scale, void* y_perm, void* ws, size_t ws_bytes,
+                           moe_stream_t stream);
+
+/* Unpermute + combine (zyxy MoE structure: y = sum_i g_i E_i(x); Ascend
+ * Unpermute).  topk_gates != NULL: y[t] = sum_{j<K} gates[t,j] *
+ * y_perm[perm_pos[t,j]], fp32 in slot order, one rounding to y's dtype.
+ * topk_gates == NULL: y[t*K+j] = y_perm[perm_pos[t*K+j]] (pure reorder,
+ * (N*K, d_out)).  Indices outside [0, N*K) set MOE_ERR_DEVICE_BAD_INDEX. */
+moe_status moe_unpermute_combine(moe_plan plan, const void* y_perm, const int32_t* perm_pos,
+                                 const float* topk_gates_or_null, void* y, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream);
+
+/* Shared-expert matmul run beside the routed experts (Ascend formula mmY =
+ * (mmX @ mmWeight) * mmXScale * mmWeightScale).  x (M, H) e4m3, w (N2, H)
+ * e4m3 output-major, y (M, N2) bf16.  Plan dtype must be e4m3.  Limits: H
+ * a multiple of 16 and <= 12288, N2 < 65536. */
+moe_status moe_shared_matmul(moe_plan plan, const void* x, int32_t M, int32_t H, const void* w,
+                             int32_t N2, float x_scale, float w_scale, void* y,
+                             moe_stream_t stream);
+
+/* Whole layer: router -> permute -> grouped FFN -> combine, on one stream,
+ * with every intermediate in the workspace.  Needs plan weights.w_r (use
+ * moe_forward_routed for caller-supplied routing). */
+moe_status moe_forward(moe_plan plan, const void* x, void* y, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* Layer with caller-supplied routing: permute -> grouped FFN -> unpermute.
+ * topk_gates_or_null selects combine (gates) or pure reorder (NULL; y is
+ * (N*K, d_out)).  x_scale as in moe_grouped_ffn. */
+moe_status moe_forward_routed(moe_plan plan, const void* x, const int32_t* topk_ids,
+                              const float* topk_gates_or_null, float x_scale, void* y, void* ws,
+                              size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward from host buffers: copies x_host (N, d) in, runs the layer,
+ * copies y back to y_host (N, d_out) and synchronises the stream.  Pinned
+ * host memory gives asynchronous copies; pageable memory works too. */
+moe_status moe_forward_host(moe_plan plan, const void* x_host, void* y_host, void* ws,
+                            size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronises `stream`, returns the sticky device status of the workspace
+ * (MOE_OK if clean) and clears it. */
+moe_status moe_read_device_status(moe_plan plan, void* ws, moe_stream_t stream);
+
+/* Stage timing: when enabled, moe_forward / moe_forward_routed record CUDA
+ * events between their kernels.  moe_profile_read synchronises the last
+ * recorded forward and writes per-kernel milliseconds in launch order;
+ * names_or_null receives static kernel names. */
+moe_status moe_profile_enable(moe_plan plan, int enable);
+moe_status moe_profile_read(moe_plan plan, float* ms, const char** names_or_null, int capacity,
+                            int* count);
+
+/* Number of kernels the last moe_forward / moe_forward_routed launched. */
+int moe_last_launch_count(moe_plan plan);
+
+const char* moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

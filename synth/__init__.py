@@ -152,36 +152,40 @@ def to_bf16(a: np.ndarray) -> torch.Tensor:
 
 
 def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """Encode float values as e4m3 codes (see _e4m3_encode_block), in
+    cache-sized blocks."""
+    v = np.asarray(v, np.float64)
+    flat = v.reshape(-1)
+    out = np.empty(flat.shape, np.uint8)
+    blk = 1 << 18
+    for lo in range(0, flat.size, blk):
+        out[lo:lo + blk] = _e4m3_encode_block(flat[lo:lo + blk])
+    return out.reshape(v.shape)
+
+
+def _e4m3_encode_block(v: np.ndarray) -> np.ndarray:
     """Encode float values as OCP FP8 E4M3 ("FN": bias 7, max 448, no inf)
     bytes, round-to-nearest-even, saturating to +-448.  Input preparation for
     the pre-quantised fp8 workload (the grouped matmul consumes codes and
     scales, as the Ascend page's gmmX/gmmWeight do)."""
     v = np.asarray(v, np.float64)
-    sign = (np.signbit(v)).astype(np.uint8) << 7
+    sign = (v.view(np.uint64) >> np.uint64(63)).astype(np.uint8) << np.uint8(7)
     a = np.minimum(np.abs(v), 448.0)
-    code = np.zeros(a.shape, np.int64)
-    sub = a < 2.0 ** -6
-    # subnormal grid: step 2^-9; q == 8 lands exactly on the smallest normal code 0x08
-    code[sub] = np.rint(a[sub] * 2.0 ** 9).astype(np.int64)
-    nrm = ~sub
-    if np.any(nrm):
-        an = a[nrm]
-        m, ex = np.frexp(an)            # an = m * 2^ex, m in [0.5, 1)
-        e = ex - 1                      # an = s * 2^e, s in [1, 2)
-        s = an / np.ldexp(1.0, e)
-        q = np.rint((s - 1.0) * 8.0).astype(np.int64)
-        carry = q == 8
-        e = e + carry
-        q = np.where(carry, 0, q)
-        code[nrm] = ((e + 7) << 3) | q
-    return (code.astype(np.uint8) | sign)
+    bits = a.view(np.int64)
+    e = (bits >> 52) - 1023                      # unbiased exponent
+    m = bits & ((1 << 52) - 1)                   # 52 fraction bits
+    # keep 3 fraction bits, round to nearest even; q == 8 carries into e
+    q = (m + ((1 << 48) - 1) + ((m >> 49) & 1)) >> 49
+    code = ((e + 7) << 3) + q
+    # below the smallest normal (2^-6) the grid step is 2^-9
+    code = np.where(a < 2.0 ** -6, np.rint(a * 512.0).astype(np.int64), code)
+    return code.astype(np.uint8) | sign
 
 
 def quantize_e4m3_per_tensor(a: np.ndarray) -> tuple[np.ndarray, float]:
     """(codes, scale) with scale = amax/448 and codes = e4m3(a / scale)."""
     amax = float(np.max(np.abs(a))) if a.size else 1.0
-    scale = amax / 448.0 if amax > 0 else 1.0
-    scale = float(np.float32(scale))
+    scale = float(np.float32(amax / 448.0)) if amax > 0 else 1.0
     out = np.empty(a.shape, np.uint8)
     flat_in, flat_out = a.reshape(-1), out.reshape(-1)
     n = flat_in.size
@@ -191,12 +195,47 @@ def quantize_e4m3_per_tensor(a: np.ndarray) -> tuple[np.ndarray, float]:
         lo, hi = i * _CHUNK, min(n, (i + 1) * _CHUNK)
         flat_out[lo:hi] = e4m3_encode(flat_in[lo:hi].astype(np.float64) / scale)
 
+    _run(work, nchunks)
+    return out, scale
+
+
+def normal_e4m3(seed: int, stream: int, n: int) -> tuple[np.ndarray, float]:
+    """n iid N(0,1) draws quantised per tensor to e4m3, without holding the
+    float draws: pass 1 finds amax chunk by chunk, pass 2 redraws each chunk
+    (same stream) and encodes it.  Same bytes as
+    quantize_e4m3_per_tensor(normal_f32(seed, stream, n))."""
+    nchunks = max(1, (n + _CHUNK - 1) // _CHUNK)
+    children = np.random.SeedSequence([seed, stream]).spawn(nchunks)
+
+    def draw(i):
+        lo, hi = i * _CHUNK, min(n, (i + 1) * _CHUNK)
+        return lo, hi, np.random.Generator(np.random.Philox(children[i])).standard_normal(
+            hi - lo, dtype=np.float32)
+
+    amax = np.zeros(nchunks)
+
+    def pass1(i):
+        amax[i] = float(np.max(np.abs(draw(i)[2])))
+
+    _run(pass1, nchunks)
+    a = float(amax.max())
+    scale = float(np.float32(a / 448.0)) if a > 0 else 1.0
+    out = np.empty(n, np.uint8)
+
+    def pass2(i):
+        lo, hi, v = draw(i)
+        out[lo:hi] = e4m3_encode(v.astype(np.float64) / scale)
+
+    _run(pass2, nchunks)
+    return out, scale
+
+
+def _run(fn, nchunks):
     if nchunks == 1:
-        work(0)
+        fn(0)
     else:
         with ThreadPoolExecutor(_threads()) as ex:
-            list(ex.map(work, range(nchunks)))
-    return out, scale
+            list(ex.map(fn, range(nchunks)))
 
 
 # ----------------------------------------------------------------------------
@@ -260,19 +299,16 @@ def make_inputs(cfg: MoEConfig, seed: int | None = None) -> MoEInputs:
         seed = SEED_BASE + cfg.index
     N, d, E, K, F = cfg.N, cfg.d, cfg.E, cfg.K, cfg.F
     if cfg.dtype == DTYPE_E4M3:
-        xf = normal_f32(seed, 1, N * d).reshape(N, d)
-        xq, xs = quantize_e4m3_per_tensor(xf)
-        wf = normal_f32(seed, 2, E * F * d).reshape(E, F, d)
-        wq, ws = quantize_e4m3_per_tensor(wf)
-        del wf
-        inp = MoEInputs(cfg, torch.from_numpy(xq), None, None, torch.from_numpy(wq), None, None,
+        xq, xs = normal_e4m3(seed, 1, N * d)
+        wq, ws = normal_e4m3(seed, 2, E * F * d)
+        inp = MoEInputs(cfg, torch.from_numpy(xq.reshape(N, d)), None, None,
+                        torch.from_numpy(wq.reshape(E, F, d)), None, None,
                         ids=torch.from_numpy(given_routing(seed, N, E, K)), x_scale=xs, w_scale=ws)
         if cfg.shared is not None:
             H2, N2 = cfg.shared
             assert H2 == d, "the shared expert reads the same token matrix"
-            shf = normal_f32(seed, 3, N2 * H2).reshape(N2, H2)
-            shq, shs = quantize_e4m3_per_tensor(shf)
-            inp.w_sh, inp.w_sh_scale = torch.from_numpy(shq), shs
+            shq, shs = normal_e4m3(seed, 3, N2 * H2)
+            inp.w_sh, inp.w_sh_scale = torch.from_numpy(shq.reshape(N2, H2)), shs
         return inp
 
     conv = (lambda a: torch.from_numpy(a)) if cfg.dtype == DTYPE_F32 else to_bf16
@@ -283,7 +319,9 @@ def make_inputs(cfg: MoEConfig, seed: int | None = None) -> MoEInputs:
     w3 = None
     if cfg.act == ACT_SWIGLU:
         w3 = conv(normal_f32(seed, 5, E * F * d, 1.0 / math.sqrt(d)).reshape(E, F, d))
-    w2 = conv(normal_f32(seed, 6, E * d * F, 1.0 / math.sqrt(F)).reshape(E, d, F))
+    w2 = None
+    if cfg.act != ACT_NONE:
+        w2 = conv(normal_f32(seed, 6, E * d * F, 1.0 / math.sqrt(F)).reshape(E, d, F))
     return MoEInputs(cfg, x, w_r, bias, w1, w3, w2)
 
 

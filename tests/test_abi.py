@@ -1,0 +1,71 @@
+"""CPU checks of the C ABI: the library loads, exports every function that
+include/moe.h declares, and rejects invalid arguments on the host before any
+CUDA call."""
+import ctypes
+
+import pytest
+
+import top_routing_grouped_gemv_b200 as moe
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moe.build()
+    return moe.load()
+
+
+def test_header_declares_the_stage_entry_points():
+    names = set(moe.header_functions())
+    for n in ("moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine",
+              "moe_forward", "moe_plan_create", "moe_workspace_size", "moe_read_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_header_symbol(lib):
+    missing = [n for n in moe.header_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_struct_layouts_match_header():
+    assert ctypes.sizeof(moe.LayerDesc) == 32
+    assert ctypes.sizeof(moe.LayerWeights) == 48
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.moe_status_string(code)
+
+
+def _create(lib, N=64, d=64, E=8, K=2, F=64, dtype=moe.MOE_BF16, act=moe.ACT_SWIGLU,
+            quant=moe.QUANT_NONE, w1=0x1000, w3=0x2000, w2=0x3000, w_r=0x4000):
+    desc = moe.LayerDesc(N, d, E, K, F, dtype, act, quant)
+    w = moe.LayerWeights(w_r, None, w1, w3, w2, 1.0)
+    h = ctypes.c_void_p()
+    rc = lib.moe_plan_create(ctypes.byref(desc), ctypes.byref(w), ctypes.byref(h))
+    if rc == 0:
+        lib.moe_plan_destroy(h)
+    return rc
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=0), 1), (dict(K=0), 1), (dict(K=9, E=16), 1), (dict(K=4, E=2), 1),
+    (dict(E=257), 1), (dict(d=65536), 1), (dict(F=70000), 1),
+    (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None), 2),   # e4m3 needs per-tensor
+    (dict(quant=moe.QUANT_PER_TENSOR), 2),                                 # per-tensor needs e4m3
+    (dict(dtype=moe.MOE_E4M3, act=moe.ACT_SWIGLU, quant=moe.QUANT_PER_TENSOR), 2),
+    (dict(dtype=moe.MOE_BF16, act=moe.ACT_RELU, w3=None), 2),
+    (dict(w3=None), 1),                                                    # SwiGLU needs w3
+    (dict(act=moe.ACT_NONE), 1),                                           # NONE takes no w2/w3
+    (dict(w1=0x1008), 1),                                                  # misaligned weights
+    (dict(d=60), 1),                                                       # 120-byte rows
+])
+def test_plan_validation_rejects(lib, kw, code):
+    assert _create(lib, **kw) == code
+
+
+def test_null_arguments(lib):
+    assert lib.moe_plan_create(None, None, None) == 1
+    assert lib.moe_plan_destroy(None) == 1
+    assert lib.moe_workspace_size(None, None) == 1
+    assert lib.moe_forward(None, None, None, None, 0, None) == 1
+    assert lib.moe_last_launch_count(None) == -1

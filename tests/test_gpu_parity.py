@@ -1,0 +1,306 @@
+"""GPU parity of every stage of the MoE layer forward against the fp64 oracle,
+called through the C ABI (libmoe.so via the ctypes binding).
+
+Bars: routing ids, counts, offsets, permutation and x_perm bit-exact (near-tie
+tokens reported separately); floats within the normwise tolerance of their
+dtype (fp32 1e-5, bf16 2e-2, fp8 6e-2).  Each stage is fed the same inputs as
+the oracle stage it is compared with, so a routing near tie cannot hide an
+FFN or combine error.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests._util import TOL, check_routing, f64, make_plan, near_tie_tokens, rel_err, to_gpu
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "f32_relu_n256": synth.FP32_RELU,
+    "f32_relu_ragged": synth.small_variant(synth.FP32_RELU, N=77, d=64, E=5, K=2, F=96),
+    "f32_swiglu": synth.MoEConfig("f32_swiglu", "f32", 100, 128, 6, 3, 64, "swiglu"),
+    "f32_none": synth.MoEConfig("f32_none", "f32", 50, 64, 4, 2, 40, "none"),
+    "bf16_swiglu_ragged": synth.small_variant(synth.BF16_PREFILL, N=300, d=256, E=8, K=2, F=384),
+    "bf16_swiglu_k4": synth.small_variant(synth.BF16_PREFILL, N=200, d=512, E=16, K=4, F=256),
+    "bf16_decode": synth.small_variant(synth.BF16_DECODE, N=8, d=1024, E=64, K=8, F=256),
+    "bf16_zipf": synth.small_variant(synth.BF16_FINEGRAINED, N=1000, d=256, E=64, K=8, F=128),
+    "bf16_k1": synth.small_variant(synth.BF16_PREFILL, N=130, d=128, E=4, K=1, F=128),
+    "bf16_f_not_tile": synth.small_variant(synth.BF16_PREFILL, N=160, d=192, E=3, K=2, F=200),
+    "e4m3_gmm": synth.small_variant(synth.FP8_GMM, N=256, d=512, E=16, K=4, F=512,
+                                    shared=(512, 384)),
+    "e4m3_gmm_ragged": synth.small_variant(synth.FP8_GMM, N=45, d=256, E=40, K=8, F=96,
+                                           shared=(256, 136)),
+}
+
+_cache = {}
+
+
+def setup_module(module):
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import top_routing_grouped_gemv_b200 as moe
+    moe.build()
+    moe.load()
+
+
+def case(name):
+    if name not in _cache:
+        cfg = SMALL[name]
+        inp = synth.make_inputs(cfg, seed=1234 + sum(map(ord, name)))
+        plan, w = make_plan(inp)
+        _cache[name] = (inp, plan, w)
+    return _cache[name]
+
+
+def ref_routing(inp):
+    """Oracle routing: (ids, gates, logits) -- given ids for the fp8 workload."""
+    if inp.ids is not None:
+        ids = inp.ids.numpy()
+        return ids, np.ones(ids.shape), None
+    ids, gates, margin, logits = oracle.router(inp.x, oracle.DTYPE[inp.cfg.dtype], inp.w_r,
+                                               inp.bias, inp.cfg.K, want_logits=True)
+    return ids, gates, logits
+
+
+ROUTED = [n for n in SMALL if SMALL[n].routing == "router"]
+
+
+@pytest.mark.parametrize("name", ROUTED)
+def test_router_parity(name):
+    inp, plan, w = case(name)
+    c = inp.cfg
+    x = inp.x.cuda()
+    ids = torch.empty(c.N, c.K, dtype=torch.int32, device="cuda")
+    gates = torch.empty(c.N, c.K, dtype=torch.float32, device="cuda")
+    margin = torch.empty(c.N, dtype=torch.float32, device="cuda")
+    plan.router_topk(x, ids, gates, margin)
+    torch.cuda.synchronize()
+    rid, rg, logits = ref_routing(inp)
+    ties, diff = check_routing(ids.cpu().numpy(), gates.cpu().double().numpy(), logits, rid, rg)
+    # margin: K-th minus (K+1)-th logit, fp32 logits vs fp64
+    _, _, rmargin, _ = oracle.router(inp.x, oracle.DTYPE[c.dtype], inp.w_r, inp.bias, c.K)
+    m = margin.cpu().double().numpy()
+    if c.K == c.E:
+        assert np.all(np.isinf(m))
+    else:
+        ok = np.setdiff1d(np.arange(c.N), diff)
+        assert np.abs(m[ok] - rmargin[ok]).max() < 1e-4
+    print(f"{name}: near-tie tokens {len(ties)}, differing ids {len(diff)}")
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_permute_parity(name):
+    inp, plan, w = case(name)
+    c = inp.cfg
+    rid, _, _ = ref_routing(inp)
+    ids = torch.from_numpy(np.ascontiguousarray(rid)).cuda()
+    x = inp.x.cuda()
+    R = c.N * c.K
+    counts = torch.empty(c.E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(c.E + 1, dtype=torch.int32, device="cuda")
+    pos = torch.empty(R, dtype=torch.int32, device="cuda")
+    src = torch.empty(R, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty((R,) + tuple(inp.x.shape[1:]), dtype=inp.x.dtype, device="cuda")
+    ws = plan.new_workspace()
+    plan.permute(x, ids, counts, offsets, pos, src, x_perm, ws)
+    assert plan.read_device_status(ws) == 0
+    rc, ro, rp, rs, rx = oracle.permute(rid, c.E, inp.x)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(pos.cpu().numpy(), rp)
+    assert np.array_equal(src.cpu().numpy(), rs)
+    xp = x_perm.cpu()
+    if xp.dtype == torch.bfloat16:
+        xp = xp.view(torch.int16)
+    assert np.array_equal(xp.numpy().view(np.uint8), np.ascontiguousarray(rx).view(np.uint8))
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_grouped_ffn_parity(name):
+    inp, plan, w = case(name)
+    c = inp.cfg
+    rid, _, _ = ref_routing(inp)
+    rc, ro, rp, rs, rx = oracle.permute(rid, c.E, inp.x)
+    xp_cpu = torch.from_numpy(rx) if isinstance(rx, np.ndarray) else rx
+    if c.dtype == "bf16":
+        xp_cpu = torch.from_numpy(np.ascontiguousarray(rx)).view(torch.bfloat16)
+    x_perm = xp_cpu.cuda()
+    offsets = torch.from_numpy(ro).cuda()
+    R = c.N * c.K
+    ydt = torch.float32 if c.dtype == "f32" else torch.bfloat16
+    y_perm = torch.full((R, c.d_out), float("nan"), dtype=ydt, device="cuda")
+    ws = plan.new_workspace()
+    plan.grouped_ffn(x_perm, offsets, y_perm, ws, x_scale=inp.x_scale)
+    assert plan.read_device_status(ws) == 0
+    row_e = np.repeat(np.arange(c.E), rc).astype(np.int32)
+    dt = oracle.DTYPE[c.dtype]
+    ref = oracle.expert_rows(row_e, rx, dt, c.act, inp.w1, inp.w3, inp.w2, dt, inp.x_scale,
+                             inp.w_scale)
+    got = f64(y_perm)
+    assert np.isfinite(got).all()
+    err = rel_err(got, ref)
+    assert err <= TOL[c.dtype], err
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_combine_parity(name):
+    """Combine fed a synthetic y_perm of the layer's dtype and the oracle's
+    pos/gates; compared with the oracle combine of the same values."""
+    inp, plan, w = case(name)
+    c = inp.cfg
+    rid, rg, _ = ref_routing(inp)
+    rc, ro, rp, rs, _ = oracle.permute(rid, c.E)
+    R = c.N * c.K
+    ydt = torch.float32 if c.dtype == "f32" else torch.bfloat16
+    yp = torch.from_numpy(synth.normal_f32(77, 9, R * c.d_out).reshape(R, c.d_out)).to(ydt)
+    gated = c.act != "none"
+    gates = torch.from_numpy(rg.astype(np.float32)) if gated else None
+    rows = c.N if gated else R
+    y = torch.empty(rows, c.d_out, dtype=ydt, device="cuda")
+    ws = plan.new_workspace()
+    plan.unpermute_combine(yp.cuda(), torch.from_numpy(rp).cuda(),
+                           gates.cuda() if gated else None, y, ws)
+    assert plan.read_device_status(ws) == 0
+    ref = oracle.combine(rp, gates.double().numpy() if gated else None, yp.double().numpy(), c.N,
+                         c.K)
+    got = f64(y)
+    if gated:
+        # one fp32 accumulation in slot order, one rounding to the output dtype
+        assert rel_err(got, ref) <= (1e-6 if c.dtype == "f32" else 8e-3)
+    else:
+        assert np.array_equal(got, ref)  # pure reorder: exact
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_end_to_end(name):
+    inp, plan, w = case(name)
+    c = inp.cfg
+    x = inp.x.cuda()
+    ws = plan.new_workspace()
+    ydt = torch.float32 if c.dtype == "f32" else torch.bfloat16
+    if c.routing == "router":
+        y = torch.empty(c.N, c.d_out, dtype=ydt, device="cuda")
+        plan.forward(x, y, ws)
+        gate_mode = 1
+    else:
+        y = torch.empty(c.N * c.K, c.d_out, dtype=ydt, device="cuda")
+        plan.forward_routed(x, inp.ids.cuda(), None, y, ws, x_scale=inp.x_scale)
+        gate_mode = 0
+    assert plan.read_device_status(ws) == 0
+    assert plan.last_launch_count() >= 5
+    ref, rids, _, _ = oracle.forward_tokens(inp, np.arange(c.N), gates_mode=gate_mode)
+    got = f64(y)
+    if c.routing == "router":
+        # exclude near-tie tokens whose routing differs (their y is a different sum)
+        ids = torch.empty(c.N, c.K, dtype=torch.int32, device="cuda")
+        gates = torch.empty(c.N, c.K, dtype=torch.float32, device="cuda")
+        plan.router_topk(x, ids, gates)
+        rid, rg, logits = ref_routing(inp)
+        ties, diff = check_routing(ids.cpu().numpy(), gates.cpu().double().numpy(), logits, rid, rg)
+        keep = np.setdiff1d(np.arange(c.N), diff)
+        assert len(keep) >= 0.9 * c.N
+        err = rel_err(got[keep], ref[keep])
+    else:
+        err = rel_err(got, ref)
+    assert err <= TOL[c.dtype], err
+
+
+@pytest.mark.parametrize("name", ["bf16_zipf", "f32_relu_n256", "e4m3_gmm"])
+def test_forward_deterministic(name):
+    inp, plan, w = case(name)
+    c = inp.cfg
+    x = inp.x.cuda()
+    ws = plan.new_workspace()
+    outs = []
+    for _ in range(3):
+        if c.routing == "router":
+            y = torch.empty(c.N, c.d_out, dtype=torch.float32 if c.dtype == "f32" else torch.bfloat16,
+                            device="cuda")
+            plan.forward(x, y, ws)
+        else:
+            y = torch.empty(c.N * c.K, c.d_out, dtype=torch.bfloat16, device="cuda")
+            plan.forward_routed(x, inp.ids.cuda(), None, y, ws, x_scale=inp.x_scale)
+        torch.cuda.synchronize()
+        outs.append(y.cpu().view(torch.uint8 if y.dtype == torch.float32 else torch.int16).clone())
+    assert all(torch.equal(outs[0], o) for o in outs[1:])
+
+
+@pytest.mark.parametrize("name", ["e4m3_gmm", "e4m3_gmm_ragged"])
+def test_shared_expert_matmul(name):
+    inp, plan, w = case(name)
+    c = inp.cfg
+    H2, N2 = c.shared
+    x = inp.x.cuda()
+    wsh = inp.w_sh.cuda()
+    y = torch.empty(c.N, N2, dtype=torch.bfloat16, device="cuda")
+    plan.shared_matmul(x, wsh, inp.x_scale, inp.w_sh_scale, y)
+    torch.cuda.synchronize()
+    ref = oracle.expert_rows(np.zeros(c.N, np.int32), inp.x, oracle.E4M3, "none",
+                             inp.w_sh.reshape(1, N2, H2), None, None, oracle.E4M3, inp.x_scale,
+                             inp.w_sh_scale)
+    assert rel_err(f64(y), ref) <= TOL["e4m3"]
+
+
+def test_forward_host_matches_device():
+    inp, plan, w = case("bf16_swiglu_ragged")
+    c = inp.cfg
+    ws = plan.new_workspace()
+    y_dev = torch.empty(c.N, c.d_out, dtype=torch.bfloat16, device="cuda")
+    plan.forward(inp.x.cuda(), y_dev, ws)
+    x_host = inp.x.clone().pin_memory()
+    y_host = torch.empty(c.N, c.d_out, dtype=torch.bfloat16).pin_memory()
+    plan.forward_host(x_host, y_host, ws)
+    assert torch.equal(y_host.view(torch.int16), y_dev.cpu().view(torch.int16))
+
+
+def test_bad_expert_ids_set_device_status():
+    inp, plan, w = case("bf16_k1")
+    c = inp.cfg
+    ids = torch.zeros(c.N, c.K, dtype=torch.int32)
+    ids[5, 0] = c.E        # out of range
+    ids[7, 0] = -3
+    R = c.N * c.K
+    ws = plan.new_workspace()
+    out = [torch.empty(c.E, dtype=torch.int32, device="cuda"),
+           torch.empty(c.E + 1, dtype=torch.int32, device="cuda"),
+           torch.empty(R, dtype=torch.int32, device="cuda"),
+           torch.empty(R, dtype=torch.int32, device="cuda"),
+           torch.empty(R, c.d, dtype=torch.bfloat16, device="cuda")]
+    plan.permute(inp.x.cuda(), ids.cuda(), *out, ws)
+    import top_routing_grouped_gemv_b200 as moe
+    assert plan.read_device_status(ws) == 5
+    assert plan.read_device_status(ws) == 0          # read clears it
+    assert out[2].cpu()[5].item() == -1              # skipped, not written elsewhere
+    assert int(out[1].cpu()[c.E]) == R - 2
+
+
+def test_workspace_too_small_and_misaligned():
+    import top_routing_grouped_gemv_b200 as moe
+    inp, plan, w = case("bf16_k1")
+    c = inp.cfg
+    ws = plan.new_workspace()
+    small = ws[: 1024]
+    y = torch.empty(c.N, c.d, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(moe.MoEError) as e:
+        plan.forward(inp.x.cuda(), y, small)
+    assert e.value.code == 3
+    with pytest.raises(moe.MoEError) as e:
+        plan.forward(inp.x.cuda(), y, ws[16:])
+    assert e.value.code == 1
+
+
+def test_stage_profile_names():
+    inp, plan, w = case("bf16_swiglu_ragged")
+    c = inp.cfg
+    ws = plan.new_workspace()
+    y = torch.empty(c.N, c.d, dtype=torch.bfloat16, device="cuda")
+    plan.profile(True)
+    plan.forward(inp.x.cuda(), y, ws)
+    prof = plan.profile_read()
+    plan.profile(False)
+    names = [n for n, _ in prof]
+    assert names == ["router_topk", "permute_count", "permute_scan", "permute_gather",
+                     "ffn1_swiglu_tc", "ffn2_tc", "combine"]
+    assert all(ms >= 0 for _, ms in prof)
+    assert plan.last_launch_count() == 7

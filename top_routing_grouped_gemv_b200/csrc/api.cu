@@ -1,0 +1,509 @@
+// C ABI of the MoE layer forward (include/moe.h): the two-phase interface of
+// aclnnQuantGroupedMatMulAlltoAllv (return-value section: phase 1 validates
+// the parameters and sizes the workspace and the executor, phase 2 runs),
+// argument validation against that page's constraints, the workspace layout
+// and the launch sequence of each stage.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "../../include/moe.h"
+#include "kernels.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+constexpr int kMaxEvents = 16;
+
+struct Layout {
+  size_t status = 0, chunk_counts = 0, h = 0, h_end = 0;
+  size_t ids = 0, gates = 0, pos = 0, src = 0, counts = 0, offsets = 0, x_perm = 0, y_perm = 0;
+  size_t fwd_end = 0, x_stage = 0, y_stage = 0, total = 0;
+  size_t permute_end = 0;
+};
+
+}  // namespace
+
+struct moe_plan_s {
+  moe_layer_desc desc;
+  moe_layer_weights w;
+  int device;
+  int ex, eh, ey;  // element bytes of x / hidden / y
+  int dout;
+  CUtensorMap tmW1, tmW3, tmW2;
+  Layout L;
+  bool profile;
+  cudaEvent_t ev[kMaxEvents];
+  const char* ev_name[kMaxEvents];
+  int nev;
+  int launches;
+};
+
+namespace {
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Stage boundary marker for the optional per-kernel timing.
+void mark(moe_plan p, cudaStream_t s, const char* name_of_next) {
+  if (!p->profile || p->nev >= kMaxEvents) return;
+  cudaEventRecord(p->ev[p->nev], s);
+  p->ev_name[p->nev] = name_of_next;
+  p->nev++;
+}
+
+void layout(moe_plan p) {
+  const moe_layer_desc& d = p->desc;
+  const long long R = static_cast<long long>(d.N) * d.K;
+  Layout L;
+  size_t off = 0;
+  L.status = off; off = align_up(off + 4);
+  L.chunk_counts = off; off = align_up(off + static_cast<size_t>(permute_chunks(d.N)) * d.E * 4);
+  L.permute_end = off;
+  L.h = off;
+  if (d.act != MOE_ACT_NONE) off = align_up(off + static_cast<size_t>(R) * d.F * p->eh);
+  L.h_end = off;
+  L.ids = off; off = align_up(off + static_cast<size_t>(R) * 4);
+  L.gates = off; off = align_up(off + static_cast<size_t>(R) * 4);
+  L.pos = off; off = align_up(off + static_cast<size_t>(R) * 4);
+  L.src = off; off = align_up(off + static_cast<size_t>(R) * 4);
+  L.counts = off; off = align_up(off + static_cast<size_t>(d.E) * 4);
+  L.offsets = off; off = align_up(off + static_cast<size_t>(d.E + 1) * 4);
+  L.x_perm = off; off = align_up(off + static_cast<size_t>(R) * d.d * p->ex);
+  L.y_perm = off; off = align_up(off + static_cast<size_t>(R) * p->dout * p->ey);
+  L.fwd_end = off;
+  L.x_stage = off; off = align_up(off + static_cast<size_t>(d.N) * d.d * p->ex);
+  L.y_stage = off;
+  const long long yrows = (d.act == MOE_ACT_NONE) ? R : d.N;
+  off = align_up(off + static_cast<size_t>(yrows) * p->dout * p->ey);
+  L.total = off;
+  p->L = L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+moe_status check_ws(moe_plan p, void* ws, size_t ws_bytes, size_t need) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  (void)p;
+  return MOE_OK;
+}
+
+bool uses_tensor_cores(const moe_layer_desc& d) { return d.dtype != MOE_F32; }
+
+moe_status run_router(moe_plan p, const void* x, int32_t* ids, float* gates, float* margin,
+                      cudaStream_t s) {
+  const moe_layer_desc& d = p->desc;
+  mark(p, s, "router_topk");
+  p->launches += 1;
+  return cuda_status(launch_router(x, d.dtype, p->w.w_r, p->w.router_bias, d.N, d.d, d.E, d.K, ids,
+                                   gates, margin, s));
+}
+
+moe_status run_permute(moe_plan p, const void* x, const int32_t* ids, int32_t* counts,
+                       int32_t* offsets, int32_t* pos, int32_t* src, void* x_perm, void* ws,
+                       cudaStream_t s) {
+  const moe_layer_desc& d = p->desc;
+  int* status = at<int>(ws, p->L.status);
+  int32_t* cc = at<int32_t>(ws, p->L.chunk_counts);
+  mark(p, s, "permute_count");
+  if (launch_permute_count(ids, d.N, d.K, d.E, cc, status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(p, s, "permute_scan");
+  if (launch_permute_scan(cc, permute_chunks(d.N), d.E, counts, offsets, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  mark(p, s, "permute_gather");
+  if (launch_permute_gather(x, d.d * p->ex, ids, d.N, d.K, d.E, cc, pos, src, x_perm, status, s) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  p->launches += 3;
+  return MOE_OK;
+}
+
+moe_status run_ffn(moe_plan p, const void* x_perm, const int32_t* offsets, float x_scale,
+                   void* y_perm, void* ws, cudaStream_t s) {
+  const moe_layer_desc& d = p->desc;
+  const int R = d.N * d.K;
+  int* status = at<int>(ws, p->L.status);
+  void* h = at<void>(ws, p->L.h);
+  if (!uses_tensor_cores(d)) {
+    const float* A = static_cast<const float*>(x_perm);
+    if (d.act == MOE_ACT_NONE) {
+      mark(p, s, "ffn_simt_f32");
+      p->launches += 1;
+      return cuda_status(launch_gemm_simt_f32(A, d.d, static_cast<const float*>(p->w.w1), nullptr,
+                                              d.F, kActNone, 1.f, offsets, d.E, R,
+                                              static_cast<float*>(y_perm), s));
+    }
+    mark(p, s, "ffn1_simt_f32");
+    if (launch_gemm_simt_f32(A, d.d, static_cast<const float*>(p->w.w1),
+                             static_cast<const float*>(p->w.w3), d.F, d.act, 1.f, offsets, d.E, R,
+                             static_cast<float*>(h), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    mark(p, s, "ffn2_simt_f32");
+    p->launches += 2;
+    return cuda_status(launch_gemm_simt_f32(static_cast<const float*>(h), d.F,
+                                            static_cast<const float*>(p->w.w2), nullptr, d.d,
+                                            kActNone, 1.f, offsets, d.E, R,
+                                            static_cast<float*>(y_perm), s));
+  }
+  TcGemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.offsets = offsets;
+  a.groups = d.E;
+  a.m_total = R;
+  a.status = status;
+  if (d.act == MOE_ACT_NONE) {
+    if (!encode_kmajor_map(&a.tmA, x_perm, p->ex, R, d.d, kTcBlockM)) return MOE_ERR_CUDA;
+    a.tmB0 = p->tmW1;
+    a.tmB1 = p->tmW1;
+    a.kdim = d.d;
+    a.n_out = d.F;
+    a.n_tiles = (d.F + kTcBlockN - 1) / kTcBlockN;
+    a.out = y_perm;
+    a.ldo = d.F;
+    a.scale = d.quant == MOE_QUANT_PER_TENSOR ? x_scale * p->w.w_scale : 1.f;
+    mark(p, s, "gmm_tc");
+    p->launches += 1;
+    return cuda_status(launch_gemm_tc(a, d.dtype, kEpiStore, R, s));
+  }
+  // SwiGLU: gate/up GEMM with the activation fused into its epilogue, then down
+  if (!encode_kmajor_map(&a.tmA, x_perm, p->ex, R, d.d, kTcBlockM)) return MOE_ERR_CUDA;
+  a.tmB0 = p->tmW1;
+  a.tmB1 = p->tmW3;
+  a.kdim = d.d;
+  a.n_out = d.F;
+  a.n_tiles = (d.F + kTcBlockN / 2 - 1) / (kTcBlockN / 2);
+  a.out = h;
+  a.ldo = d.F;
+  a.scale = 1.f;
+  mark(p, s, "ffn1_swiglu_tc");
+  if (launch_gemm_tc(a, d.dtype, kEpiSwiglu, R, s) != cudaSuccess) return MOE_ERR_CUDA;
+  TcGemmArgs b = a;
+  if (!encode_kmajor_map(&b.tmA, h, p->eh, R, d.F, kTcBlockM)) return MOE_ERR_CUDA;
+  b.tmB0 = p->tmW2;
+  b.tmB1 = p->tmW2;
+  b.kdim = d.F;
+  b.n_out = d.d;
+  b.n_tiles = (d.d + kTcBlockN - 1) / kTcBlockN;
+  b.out = y_perm;
+  b.ldo = d.d;
+  mark(p, s, "ffn2_tc");
+  p->launches += 2;
+  return cuda_status(launch_gemm_tc(b, d.dtype, kEpiStore, R, s));
+}
+
+moe_status run_combine(moe_plan p, const void* y_perm, const int32_t* pos, const float* gates,
+                       void* y, void* ws, cudaStream_t s) {
+  const moe_layer_desc& d = p->desc;
+  mark(p, s, gates ? "combine" : "unpermute");
+  p->launches += 1;
+  const int ydt = d.dtype == MOE_F32 ? kF32 : kBF16;
+  return cuda_status(launch_combine(y_perm, ydt, p->dout, pos, gates, d.N, d.K, y,
+                                    at<int>(ws, p->L.status), s));
+}
+
+void begin(moe_plan p) {
+  p->nev = 0;
+  p->launches = 0;
+}
+void end(moe_plan p, cudaStream_t s) { mark(p, s, nullptr); }
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status st) {
+  switch (st) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_BAD_INDEX: return "device: index out of range";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device: pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* w, moe_plan* out) {
+  if (!desc || !w || !out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const moe_layer_desc d = *desc;
+  // limits of the Ascend page (K in [2, 8] widened to [1, 8]; experts <= 256;
+  // H1, N1 < 65536)
+  if (d.N < 1 || d.d < 1 || d.d >= 65536 || d.E < 1 || d.E > 256 || d.K < 1 || d.K > 8 ||
+      d.K > d.E || d.F < 1 || d.F >= 65536)
+    return MOE_ERR_INVALID_ARG;
+  if (static_cast<long long>(d.N) * d.K >= (1LL << 31)) return MOE_ERR_INVALID_ARG;
+  if (d.dtype < MOE_F32 || d.dtype > MOE_E4M3 || d.act < MOE_ACT_NONE || d.act > MOE_ACT_SWIGLU ||
+      d.quant < MOE_QUANT_NONE || d.quant > MOE_QUANT_PER_TENSOR)
+    return MOE_ERR_INVALID_ARG;
+  if ((d.quant == MOE_QUANT_PER_TENSOR) != (d.dtype == MOE_E4M3)) return MOE_ERR_UNSUPPORTED;
+  if (d.dtype == MOE_E4M3 && d.act != MOE_ACT_NONE) return MOE_ERR_UNSUPPORTED;
+  if (d.dtype == MOE_BF16 && d.act == MOE_ACT_RELU) return MOE_ERR_UNSUPPORTED;
+  if (!w->w1 || (d.act == MOE_ACT_SWIGLU) != (w->w3 != nullptr) ||
+      (d.act != MOE_ACT_NONE) != (w->w2 != nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->w1) || (w->w3 && !aligned16(w->w3)) || (w->w2 && !aligned16(w->w2)))
+    return MOE_ERR_INVALID_ARG;
+
+  moe_plan p = new (std::nothrow) moe_plan_s;
+  if (!p) return MOE_ERR_CUDA;
+  memset(static_cast<void*>(p), 0, sizeof(*p));
+  p->desc = d;
+  p->w = *w;
+  p->ex = dtype_bytes(d.dtype);
+  p->eh = d.dtype == MOE_F32 ? 4 : 2;
+  p->ey = d.dtype == MOE_F32 ? 4 : 2;
+  p->dout = d.act == MOE_ACT_NONE ? d.F : d.d;
+  // every row that a kernel moves with 16-byte vectors or TMA is a multiple
+  // of 16 bytes
+  if ((static_cast<long long>(d.d) * p->ex) % 16 || (static_cast<long long>(p->dout) * p->ey) % 16 ||
+      (d.act != MOE_ACT_NONE && (static_cast<long long>(d.F) * p->eh) % 16)) {
+    delete p;
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (cudaGetDevice(&p->device) != cudaSuccess) {
+    delete p;
+    return MOE_ERR_CUDA;
+  }
+  if (uses_tensor_cores(d)) {
+    bool ok = true;
+    if (d.act == MOE_ACT_NONE) {
+      ok = encode_kmajor_map(&p->tmW1, w->w1, p->ex, static_cast<long long>(d.E) * d.F, d.d,
+                             kTcBlockN);
+    } else {
+      ok = encode_kmajor_map(&p->tmW1, w->w1, p->ex, static_cast<long long>(d.E) * d.F, d.d,
+                             kTcBlockN / 2) &&
+           encode_kmajor_map(&p->tmW3, w->w3, p->ex, static_cast<long long>(d.E) * d.F, d.d,
+                             kTcBlockN / 2) &&
+           encode_kmajor_map(&p->tmW2, w->w2, p->ex, static_cast<long long>(d.E) * d.d, d.F,
+                             kTcBlockN);
+    }
+    if (!ok) {
+      delete p;
+      return MOE_ERR_CUDA;
+    }
+  }
+  for (int i = 0; i < kMaxEvents; ++i) p->ev[i] = nullptr;
+  layout(p);
+  *out = p;
+  return MOE_OK;
+}
+
+moe_status moe_plan_destroy(moe_plan p) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < kMaxEvents; ++i)
+    if (p->ev[i]) cudaEventDestroy(p->ev[i]);
+  delete p;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_size(moe_plan p, size_t* bytes) {
+  if (!p || !bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = p->L.total;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(moe_plan p, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.chunk_counts);
+  if (st != MOE_OK) return st;
+  return cuda_status(cudaMemsetAsync(ws, 0, 4, stream));
+}
+
+moe_status moe_router_topk(moe_plan p, const void* x, int32_t* ids, float* gates, float* margin,
+                           moe_stream_t stream) {
+  if (!p || !x || !ids || !gates || !p->w.w_r) return MOE_ERR_INVALID_ARG;
+  if (p->desc.dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  begin(p);
+  moe_status st = run_router(p, x, ids, gates, margin, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_permute(moe_plan p, const void* x, const int32_t* ids, int32_t* counts,
+                       int32_t* offsets, int32_t* pos, int32_t* src, void* x_perm, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !x || !ids || !counts || !offsets || !pos || !src || !x_perm) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.permute_end);
+  if (st != MOE_OK) return st;
+  begin(p);
+  st = run_permute(p, x, ids, counts, offsets, pos, src, x_perm, ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_grouped_ffn(moe_plan p, const void* x_perm, const int32_t* offsets, float x_scale,
+                           void* y_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !x_perm || !offsets || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_perm) || !aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.h_end);
+  if (st != MOE_OK) return st;
+  begin(p);
+  st = run_ffn(p, x_perm, offsets, x_scale, y_perm, ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_unpermute_combine(moe_plan p, const void* y_perm, const int32_t* pos,
+                                 const float* gates, void* y, void* ws, size_t ws_bytes,
+                                 moe_stream_t stream) {
+  if (!p || !y_perm || !pos || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.chunk_counts);
+  if (st != MOE_OK) return st;
+  begin(p);
+  st = run_combine(p, y_perm, pos, gates, y, ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_shared_matmul(moe_plan p, const void* x, int32_t M, int32_t H, const void* w,
+                             int32_t N2, float x_scale, float w_scale, void* y,
+                             moe_stream_t stream) {
+  if (!p || !x || !w || !y || M < 1 || H < 16 || H > 12288 || H % 16 || N2 < 1 || N2 >= 65536 ||
+      N2 % 8)
+    return MOE_ERR_INVALID_ARG;
+  if (p->desc.dtype != MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  TcGemmArgs a;
+  memset(&a, 0, sizeof(a));
+  if (!encode_kmajor_map(&a.tmA, x, 1, M, H, kTcBlockM) ||
+      !encode_kmajor_map(&a.tmB0, w, 1, N2, H, kTcBlockN))
+    return MOE_ERR_CUDA;
+  a.tmB1 = a.tmB0;
+  a.offsets = nullptr;
+  a.groups = 1;
+  a.m_total = M;
+  a.kdim = H;
+  a.n_out = N2;
+  a.n_tiles = (N2 + kTcBlockN - 1) / kTcBlockN;
+  a.out = y;
+  a.ldo = N2;
+  a.scale = x_scale * w_scale;
+  a.status = nullptr;
+  return cuda_status(launch_gemm_tc(a, kE4M3, kEpiStore, M, stream));
+}
+
+moe_status moe_forward_routed(moe_plan p, const void* x, const int32_t* ids, const float* gates,
+                              float x_scale, void* y, void* ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+  if (!p || !x || !ids || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.fwd_end);
+  if (st != MOE_OK) return st;
+  const Layout& L = p->L;
+  begin(p);
+  st = run_permute(p, x, ids, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
+                   at<int32_t>(ws, L.pos), at<int32_t>(ws, L.src), at<void>(ws, L.x_perm), ws,
+                   stream);
+  if (st == MOE_OK)
+    st = run_ffn(p, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), x_scale,
+                 at<void>(ws, L.y_perm), ws, stream);
+  if (st == MOE_OK)
+    st = run_combine(p, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_forward(moe_plan p, const void* x, void* y, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+  if (!p || !x || !y || !p->w.w_r) return MOE_ERR_INVALID_ARG;
+  if (p->desc.dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.fwd_end);
+  if (st != MOE_OK) return st;
+  const Layout& L = p->L;
+  begin(p);
+  st = run_router(p, x, at<int32_t>(ws, L.ids), at<float>(ws, L.gates), nullptr, stream);
+  if (st == MOE_OK)
+    st = run_permute(p, x, at<int32_t>(ws, L.ids), at<int32_t>(ws, L.counts),
+                     at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.pos), at<int32_t>(ws, L.src),
+                     at<void>(ws, L.x_perm), ws, stream);
+  if (st == MOE_OK)
+    st = run_ffn(p, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), 1.f,
+                 at<void>(ws, L.y_perm), ws, stream);
+  if (st == MOE_OK)
+    st = run_combine(p, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), at<float>(ws, L.gates), y,
+                     ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_forward_host(moe_plan p, const void* x_host, void* y_host, void* ws,
+                            size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !x_host || !y_host) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.total);
+  if (st != MOE_OK) return st;
+  const moe_layer_desc& d = p->desc;
+  void* xs = at<void>(ws, p->L.x_stage);
+  void* ys = at<void>(ws, p->L.y_stage);
+  const size_t xb = static_cast<size_t>(d.N) * d.d * p->ex;
+  const size_t yb = static_cast<size_t>(d.N) * p->dout * p->ey;
+  if (cudaMemcpyAsync(xs, x_host, xb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  st = moe_forward(p, xs, ys, ws, ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(y_host, ys, yb, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cuda_status(cudaStreamSynchronize(stream));
+}
+
+moe_status moe_read_device_status(moe_plan p, void* ws, moe_stream_t stream) {
+  if (!p || !ws) return MOE_ERR_INVALID_ARG;
+  int v = 0;
+  if (cudaMemcpyAsync(&v, at<int>(ws, p->L.status), 4, cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (v != 0) {
+    if (cudaMemsetAsync(at<int>(ws, p->L.status), 0, 4, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  return static_cast<moe_status>(v);
+}
+
+moe_status moe_profile_enable(moe_plan p, int enable) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (enable && !p->ev[0]) {
+    for (int i = 0; i < kMaxEvents; ++i)
+      if (cudaEventCreate(&p->ev[i]) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  p->profile = enable != 0;
+  p->nev = 0;
+  return MOE_OK;
+}
+
+moe_status moe_profile_read(moe_plan p, float* ms, const char** names, int capacity, int* count) {
+  if (!p || !count) return MOE_ERR_INVALID_ARG;
+  *count = 0;
+  if (!p->profile || p->nev < 2) return MOE_OK;
+  if (cudaEventSynchronize(p->ev[p->nev - 1]) != cudaSuccess) return MOE_ERR_CUDA;
+  int n = 0;
+  for (int i = 0; i + 1 < p->nev && n < capacity; ++i, ++n) {
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, p->ev[i], p->ev[i + 1]) != cudaSuccess) return MOE_ERR_CUDA;
+    if (ms) ms[n] = t;
+    if (names) names[n] = p->ev_name[i];
+  }
+  *count = n;
+  return MOE_OK;
+}
+
+int moe_last_launch_count(moe_plan p) { return p ? p->launches : -1; }
+
+}  // extern "C"

@@ -1,0 +1,141 @@
+// Grouped expert GEMM for fp32 layers on the FP32 FMA pipes ("Advanced GPU
+// Optimization ... Part 5", section 1.2 step 2: every expert's FFN on the
+// tokens routed to it).  The fp32 path needs fp32-exact products (tf32
+// tensor cores round the operands to 10 mantissa bits), so it runs on the
+// SIMT pipes: 64x64 output tiles, k staged through shared memory in slices
+// of 16, a 4x4 register micro-tile per thread, k summed in ascending order.
+//
+// Tile schedule: blockIdx.y enumerates the 64-row tiles of all experts in
+// expert order (empty experts own none); the CTA finds its expert from the
+// device-side offsets, so no host round trip is needed.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 64, BN = 64, BK = 16;
+
+template <int ACT>
+__global__ void __launch_bounds__(256)
+gemm_simt_f32_kernel(const float* __restrict__ A, int kdim, const float* __restrict__ W,
+                     const float* __restrict__ W3, int ncols, float scale,
+                     const int32_t* __restrict__ offsets, int E, float* __restrict__ out) {
+  __shared__ __align__(16) float As[BK][BM + 4];
+  __shared__ __align__(16) float Bs[BK][BN + 4];
+  __shared__ __align__(16) float Us[BK][BN + 4];
+  __shared__ int s_e, s_row0, s_row1;
+
+  if (threadIdx.x == 0) {
+    int tile = blockIdx.y, run = 0, found = -1;
+    for (int e = 0; e < E; ++e) {
+      int r0 = offsets[e], r1 = offsets[e + 1];
+      int mt = (r1 - r0 + BM - 1) / BM;
+      if (tile < run + mt) {
+        found = e;
+        s_row0 = r0 + (tile - run) * BM;
+        s_row1 = r1;
+        break;
+      }
+      run += mt;
+    }
+    s_e = found;
+  }
+  __syncthreads();
+  const int e = s_e;
+  if (e < 0) return;  // fewer tiles than the grid's upper bound
+  const int row0 = s_row0, row1 = s_row1;
+  const int col0 = blockIdx.x * BN;
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  const float* We = W + (long long)e * ncols * kdim;
+  const float* Ue = ACT == kActSwiglu ? W3 + (long long)e * ncols * kdim : nullptr;
+
+  float acc[4][4], accu[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = accu[i][j] = 0.f;
+
+  const int lr = tid / 4, lk = (tid % 4) * 4;  // loader: row/col within tile, k offset
+  for (int k0 = 0; k0 < kdim; k0 += BK) {
+    {
+      int r = row0 + lr, k = k0 + lk;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < row1 && k < kdim) a = *reinterpret_cast<const float4*>(A + (long long)r * kdim + k);
+      As[lk + 0][lr] = a.x; As[lk + 1][lr] = a.y; As[lk + 2][lr] = a.z; As[lk + 3][lr] = a.w;
+      int n = col0 + lr;
+      float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (n < ncols && k < kdim) b = *reinterpret_cast<const float4*>(We + (long long)n * kdim + k);
+      Bs[lk + 0][lr] = b.x; Bs[lk + 1][lr] = b.y; Bs[lk + 2][lr] = b.z; Bs[lk + 3][lr] = b.w;
+      if (ACT == kActSwiglu) {
+        float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (n < ncols && k < kdim) u = *reinterpret_cast<const float4*>(Ue + (long long)n * kdim + k);
+        Us[lk + 0][lr] = u.x; Us[lk + 1][lr] = u.y; Us[lk + 2][lr] = u.z; Us[lk + 3][lr] = u.w;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < BK; ++kk) {
+      float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      if (ACT == kActSwiglu) {
+        float4 u = *reinterpret_cast<const float4*>(&Us[kk][tx * 4]);
+        float uv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) accu[i][j] = fmaf(av[i], uv[j], accu[i][j]);
+      }
+    }
+    __syncthreads();
+  }
+
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int r = row0 + ty * 4 + i;
+    if (r >= row1 || r >= row0 + BM) continue;
+    float o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float v = acc[i][j];
+      if (ACT == kActRelu) v = fmaxf(v, 0.f);
+      else if (ACT == kActSwiglu) v = (v / (1.f + expf(-v))) * accu[i][j];
+      else v *= scale;
+      o[j] = v;
+    }
+    int n = col0 + tx * 4;
+    if (n + 3 < ncols) {
+      *reinterpret_cast<float4*>(out + (long long)r * ncols + n) = make_float4(o[0], o[1], o[2], o[3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (n + j < ncols) out[(long long)r * ncols + n + j] = o[j];
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_simt_f32(const float* A, int kdim, const float* W, const float* W3,
+                                 int ncols, int act, float scale, const int32_t* offsets, int E,
+                                 int R, float* out, cudaStream_t stream) {
+  if (R == 0) return cudaSuccess;
+  dim3 grid((ncols + BN - 1) / BN, (R + BM - 1) / BM + E);
+  if (act == kActRelu)
+    gemm_simt_f32_kernel<kActRelu><<<grid, 256, 0, stream>>>(A, kdim, W, W3, ncols, scale, offsets,
+                                                             E, out);
+  else if (act == kActSwiglu)
+    gemm_simt_f32_kernel<kActSwiglu><<<grid, 256, 0, stream>>>(A, kdim, W, W3, ncols, scale,
+                                                               offsets, E, out);
+  else
+    gemm_simt_f32_kernel<kActNone><<<grid, 256, 0, stream>>>(A, kdim, W, W3, ncols, scale, offsets,
+                                                             E, out);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,534 @@
+// Grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// What it computes ("Advanced GPU Optimization ... Part 5", section 1.2
+// step 2, local expert FFNs; aclnnQuantGroupedMatMulAlltoAllv formula:
+// gmmY = (gmmX @ gmmWeight) * gmmXScale * gmmWeightScale, and the shared
+// expert mmY = (mmX @ mmWeight) * ...): for every group g (expert), the rows
+// [offsets[g], offsets[g+1]) of A times the transpose of the group's
+// weight block W_g (n_out x kdim, K-major), fp32 accumulation, then either
+//   kEpiStore : out = bf16(acc * scale)
+//   kEpiSwiglu: out = bf16(silu(acc_gate) * acc_up)  (the weight tile holds
+//               128 gate rows followed by 128 up rows of the same outputs)
+//
+// Structure (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: 128-byte-swizzled K-major tiles of A (128 rows)
+//               and W (256 rows) into a 4-stage shared-memory ring
+//   warp 1      owns the 512 TMEM columns; lane 0 issues tcgen05.mma
+//               (M=128, N=256, K=16 bf16 / K=32 e4m3 per instruction) into
+//               one of two fp32 accumulators, and tcgen05.commit releases
+//               ring slots and hands finished accumulators to the epilogue
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows of their TMEM
+//               lane quadrant, activation/scale, bf16, 16-byte stores;
+//               overlaps the next tile's MMAs (double-buffered TMEM)
+// The tile list (group, row tile, column tile) is derived on the device
+// from the offsets, so no host synchronisation is needed; empty groups own
+// no tiles, and rows past a group's end are computed but never stored.
+//
+// Every mbarrier wait is bounded (1 s): on expiry the CTA records
+// MOE_ERR_DEVICE_TIMEOUT, the other roles leave their loops, in-flight
+// copies and MMAs are drained (bounded) and TMEM is freed before exit.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = kTcBlockM;     // 128 rows per tile
+constexpr int BN = kTcBlockN;     // 256 accumulator columns per tile
+constexpr int ROWB = 128;         // bytes of K per row per stage (one swizzle atom)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * ROWB;
+constexpr int B_BYTES = BN * ROWB;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 2 * BN;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr int kMaxGroups = 256;
+
+// shared-memory map past the stage ring
+constexpr int kBarFull = 0, kBarEmpty = STAGES, kBarTFull = 2 * STAGES, kBarTEmpty = 2 * STAGES + 2,
+              kBarDrain = 2 * STAGES + 4, kNumBars = 2 * STAGES + 5;
+constexpr int kSmemBytes = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + kNumBars * 8 + 16 +
+                           2 * (kMaxGroups + 1) * 4;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- mbarrier -----------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase of parity `parity` to complete.  Gives up (false) when
+// another role raised the abort flag or after kWaitLimitNs, raising it.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 127) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+// Bounded wait that ignores the abort flag (used while draining).
+__device__ __noinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  return true;
+}
+
+// ---- TMA ----------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---- tcgen05 ------------------------------------------------------------------
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+template <bool kFp8>
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  if constexpr (kFp8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+// 32 lanes x 32 consecutive fp32 columns: thread i of the warp gets row
+// (quadrant*32 + i), columns [col, col+32).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with
+// 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
+//   [0,14) start >> 4 | [16,30) leading offset (unused here: 16 B)
+//   [32,46) stride offset 1024 >> 4 | [46,48) version 1 | [61,64) swizzle-128B (2)
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (1ull << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor: fp32 accumulator (bit 4), A/B format at [7,10) and
+// [10,13) (bf16 = 1 for kind::f16, e4m3 = 0 for kind::f8f6f4), both K-major,
+// N >> 3 at [17,23), M >> 4 at [24,29).
+template <bool kFp8>
+constexpr uint32_t make_idesc() {
+  return (1u << 4) | ((kFp8 ? 0u : 1u) << 7) | ((kFp8 ? 0u : 1u) << 10) |
+         (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+}
+
+struct TileCoord {
+  int g, m_row0, n_tile;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(int T, const int* s_pref, const int* s_off,
+                                                 int G) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (s_pref[mid] <= T) lo = mid; else hi = mid - 1;
+  }
+  TileCoord c;
+  c.g = lo;
+  const int local = T - s_pref[lo];
+  const int mt = (s_off[lo + 1] - s_off[lo] + BM - 1) / BM;
+  c.n_tile = local / mt;
+  c.m_row0 = s_off[lo] + (local - c.n_tile * mt) * BM;
+  return c;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.f + __expf(-g)) * u; }
+
+template <bool kFp8, int kEpi>
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ TcGemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  const uint32_t bar0 = smem_u32(bars);
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_pref = reinterpret_cast<int*>(tmem_slot + 4);
+  int* s_off = s_pref + (kMaxGroups + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = args.groups;
+
+  // Per-group tile counts -> exclusive prefix (warp 0), group row offsets.
+  if (warp == 0) {
+    const int per = (G + 31) / 32;
+    const int b0 = min(G, lane * per), b1 = min(G, b0 + per);
+    int local = 0;
+    for (int q = b0; q < b1; ++q) {
+      int o0 = args.offsets ? args.offsets[q] : 0;
+      int o1 = args.offsets ? args.offsets[q + 1] : args.m_total;
+      s_off[q] = o0;
+      int cnt = max(0, o1 - o0);
+      int t = (cnt + BM - 1) / BM * args.n_tiles;
+      s_pref[q] = t;
+      local += t;
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int run = incl - local;
+    for (int q = b0; q < b1; ++q) {
+      int t = s_pref[q];
+      s_pref[q] = run;
+      run += t;
+    }
+    if (lane == 31) {
+      s_pref[G] = incl;
+      s_off[G] = args.offsets ? args.offsets[G] : args.m_total;
+    }
+  }
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar(kBarFull + s), 1);
+      mbar_init(bar(kBarEmpty + s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar(kBarTFull + a), 1);
+      mbar_init(bar(kBarTEmpty + a), 4);
+    }
+    mbar_init(bar(kBarDrain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&args.tmA);
+    tma_prefetch_desc(&args.tmB0);
+    if (kEpi == kEpiSwiglu) tma_prefetch_desc(&args.tmB1);
+  }
+  if (warp == 1) {
+    __syncwarp();  // tcgen05.alloc is .sync.aligned: converge after thread 32's branch
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_pref[G];
+  constexpr int kElems = kFp8 ? 128 : 64;  // K elements per stage
+  const int num_kb = (args.kdim + kElems - 1) / kElems;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool aborted = false;
+      uint32_t issued = 0, issued_ph = 0;  // per-stage bits: loaded at least once / its parity
+      for (int T = blockIdx.x; T < total && !aborted; T += gridDim.x) {
+        const TileCoord c = decode_tile(T, s_pref, s_off, G);
+        const int brow = c.g * args.n_out + c.n_tile * (kEpi == kEpiSwiglu ? BN / 2 : BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(bar(kBarEmpty + s), ph ^ 1u, abort_flag)) { aborted = true; break; }
+          mbar_expect_tx(bar(kBarFull + s), STAGE_BYTES);
+          const int kx = kb * kElems;
+          tma_load_2d(sA + s * A_BYTES, &args.tmA, kx, c.m_row0, bar(kBarFull + s));
+          if (kEpi == kEpiSwiglu) {
+            tma_load_2d(sB + s * B_BYTES, &args.tmB0, kx, brow, bar(kBarFull + s));
+            tma_load_2d(sB + s * B_BYTES + (BN / 2) * ROWB, &args.tmB1, kx, brow, bar(kBarFull + s));
+          } else {
+            tma_load_2d(sB + s * B_BYTES, &args.tmB0, kx, brow, bar(kBarFull + s));
+          }
+          issued |= 1u << s;
+          issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (aborted) {
+        set_status(args.status, kStatusTimeout);
+        // let copies already in flight land before the CTA's memory is reused
+        for (int i = 0; i < STAGES; ++i)
+          if ((issued >> i) & 1u) mbar_wait_drain(bar(kBarFull + i), (issued_ph >> i) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc<kFp8>();
+      int s = 0;
+      uint32_t ph = 0;
+      bool aborted = false;
+      int i = 0;
+      for (int T = blockIdx.x; T < total; T += gridDim.x, ++i) {
+        const int acc = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        if (!mbar_wait(bar(kBarTEmpty + acc), aph ^ 1u, abort_flag)) { aborted = true; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(bar(kBarFull + s), ph, abort_flag)) { aborted = true; break; }
+          tc_fence_after();
+          const uint32_t a0 = sA + s * A_BYTES, b0 = sB + s * B_BYTES;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma<kFp8>(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc,
+                         (kb | k) != 0 ? 1u : 0u);
+          tc_commit(bar(kBarEmpty + s));
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+        if (aborted) break;
+        tc_commit(bar(kBarTFull + acc));
+      }
+      if (aborted) {
+        set_status(args.status, kStatusTimeout);
+        tc_commit(bar(kBarDrain));  // arrives once every MMA issued so far has finished
+        mbar_wait_drain(bar(kBarDrain), 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;
+    int i = 0;
+    for (int T = blockIdx.x; T < total; T += gridDim.x, ++i) {
+      const int acc = i & 1;
+      const uint32_t aph = (i >> 1) & 1;
+      // every lane polls; lane 0's answer is taken by all (and converges the warp
+      // before the .sync.aligned TMEM loads)
+      const bool ok = __shfl_sync(0xffffffffu, mbar_wait(bar(kBarTFull + acc), aph, abort_flag), 0);
+      if (!ok) {
+        set_status(args.status, kStatusTimeout);
+        break;
+      }
+      tc_fence_after();
+      const TileCoord c = decode_tile(T, s_pref, s_off, G);
+      const long long grow = static_cast<long long>(c.m_row0) + row;
+      const bool valid = grow < s_off[c.g + 1] && grow < args.m_total && grow >= 0;
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + grow * args.ldo;
+      if (kEpi == kEpiSwiglu) {
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 2; cc += 32) {
+          uint32_t gr[32], ur[32];
+          __syncwarp();
+          tmem_ld32(tbase + cc, gr);
+          tmem_ld32(tbase + BN / 2 + cc, ur);
+          tmem_ld_wait();
+          const int col = c.n_tile * (BN / 2) + cc;
+          if (valid && col < args.n_out) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              pk[j] = pack_bf16x2(silu_mul(__uint_as_float(gr[2 * j]), __uint_as_float(ur[2 * j])),
+                                  silu_mul(__uint_as_float(gr[2 * j + 1]),
+                                           __uint_as_float(ur[2 * j + 1])));
+            if (col + 32 <= args.n_out) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col + j < args.n_out)
+                  orow[col + j] = __float2bfloat16_rn(
+                      silu_mul(__uint_as_float(gr[j]), __uint_as_float(ur[j])));
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < BN; cc += 32) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(tbase + cc, v);
+          tmem_ld_wait();
+          const int col = c.n_tile * BN + cc;
+          if (valid && col < args.n_out) {
+            const float sc = args.scale;
+            if (col + 32 <= args.n_out) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(
+                    pack_bf16x2(__uint_as_float(v[8 * j + 0]) * sc, __uint_as_float(v[8 * j + 1]) * sc),
+                    pack_bf16x2(__uint_as_float(v[8 * j + 2]) * sc, __uint_as_float(v[8 * j + 3]) * sc),
+                    pack_bf16x2(__uint_as_float(v[8 * j + 4]) * sc, __uint_as_float(v[8 * j + 5]) * sc),
+                    pack_bf16x2(__uint_as_float(v[8 * j + 6]) * sc, __uint_as_float(v[8 * j + 7]) * sc));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col + j < args.n_out) orow[col + j] = __float2bfloat16_rn(__uint_as_float(v[j]) * sc);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarTEmpty + acc));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+template <bool kFp8, int kEpi>
+cudaError_t launch_t(const TcGemmArgs& args, int grid, cudaStream_t stream) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kFp8, kEpi>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  gemm_tc_kernel<kFp8, kEpi><<<grid, kThreads, kSmemBytes, stream>>>(args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool encode_kmajor_map(CUtensorMap* map, const void* base, int elem_bytes, long long rows,
+                       long long kdim, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows <= 0 || kdim <= 0) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kdim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kdim * elem_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(ROWB / elem_bytes), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUtensorMapDataType dt =
+      elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gemm_tc(const TcGemmArgs& args, int dtype, int epilogue, int rows_upper,
+                           cudaStream_t stream) {
+  if (args.groups < 1 || args.groups > kMaxGroups) return cudaErrorInvalidValue;
+  long long max_tiles = (static_cast<long long>(rows_upper) / BM + args.groups) * args.n_tiles;
+  if (max_tiles <= 0) return cudaSuccess;
+  int grid = static_cast<int>(max_tiles < device_sm_count() ? max_tiles : device_sm_count());
+  const bool fp8 = dtype == kE4M3;
+  if (fp8) {
+    if (epilogue == kEpiSwiglu) return launch_t<true, kEpiSwiglu>(args, grid, stream);
+    return launch_t<true, kEpiStore>(args, grid, stream);
+  }
+  if (epilogue == kEpiSwiglu) return launch_t<false, kEpiSwiglu>(args, grid, stream);
+  return launch_t<false, kEpiStore>(args, grid, stream);
+}
+
+int device_sm_count() {
+  static int count[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (count[dev] == 0) {
+    int c = 0;
+    cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev);
+    count[dev] = c > 0 ? c : 148;
+  }
+  return count[dev];
+}
+
+}  // namespace moe

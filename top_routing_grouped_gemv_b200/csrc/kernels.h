@@ -1,0 +1,80 @@
+// Internal launchers of the MoE layer kernels.  Host-side C++ only; the
+// public surface is the C ABI in include/moe.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+enum DType { kF32 = 0, kBF16 = 1, kE4M3 = 2 };
+enum Act { kActNone = 0, kActRelu = 1, kActSwiglu = 2 };
+
+inline int dtype_bytes(int dt) { return dt == kF32 ? 4 : dt == kBF16 ? 2 : 1; }
+
+// ---- router -----------------------------------------------------------------
+cudaError_t launch_router(const void* x, int x_dtype, const float* w_r, const float* bias, int N,
+                          int d, int E, int K, int32_t* ids, float* gates, float* margin,
+                          cudaStream_t stream);
+
+// ---- permute ----------------------------------------------------------------
+constexpr int kPermuteChunk = 32;  // tokens per chunk of the stable counting pass
+inline int permute_chunks(int N) { return (N + kPermuteChunk - 1) / kPermuteChunk; }
+
+cudaError_t launch_permute_count(const int32_t* ids, int N, int K, int E, int32_t* chunk_counts,
+                                 int* status, cudaStream_t stream);
+cudaError_t launch_permute_scan(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
+                                int32_t* offsets, cudaStream_t stream);
+cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* ids, int N, int K,
+                                  int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
+                                  void* x_perm, int* status, cudaStream_t stream);
+
+// ---- combine / unpermute ----------------------------------------------------
+// y_dtype: kF32 or kBF16 (the dtype of y_perm and y).
+cudaError_t launch_combine(const void* y_perm, int y_dtype, int dout, const int32_t* pos,
+                           const float* gates, int N, int K, void* y, int* status,
+                           cudaStream_t stream);
+
+// ---- grouped FFN, fp32 SIMT path --------------------------------------------
+// C[r, n] for rows of expert e: act(A[r,:] . W[e][n,:]) with A (R, kdim),
+// W (E, ncols, kdim); SwiGLU uses W3 as the up matrix.  out (R, ncols) fp32.
+cudaError_t launch_gemm_simt_f32(const float* A, int kdim, const float* W, const float* W3,
+                                 int ncols, int act, float scale, const int32_t* offsets, int E,
+                                 int R, float* out, cudaStream_t stream);
+
+// ---- grouped GEMM on tcgen05 tensor cores -----------------------------------
+enum TcEpilogue { kEpiStore = 0, kEpiSwiglu = 1 };
+
+struct TcGemmArgs {
+  CUtensorMap tmA;   // activations: rows (R), cols kdim
+  CUtensorMap tmB0;  // weights: rows (groups * n_out), cols kdim (gate / single matrix)
+  CUtensorMap tmB1;  // SwiGLU up matrix, same shape as tmB0
+  const int32_t* offsets;  // (groups + 1) row offsets of A, device; NULL: one group of m_total
+  int groups;              // experts (1 for a plain matmul)
+  int m_total;             // rows of A and out; rows at or past it are never stored
+  int kdim;
+  int n_out;               // output columns per group
+  int n_tiles;             // output column tiles per group
+  void* out;               // bf16 (rows, ldo)
+  long long ldo;           // elements
+  float scale;             // multiplies the fp32 accumulator before rounding
+  int* status;
+};
+
+// Host: encode a 2-D K-major tile map over a (rows, kdim) row-major matrix of
+// elem_bytes-wide elements; box = (128 bytes of K) x box_rows, 128-B swizzle.
+bool encode_kmajor_map(CUtensorMap* map, const void* base, int elem_bytes, long long rows,
+                       long long kdim, int box_rows);
+
+// dtype kBF16 or kE4M3.  offsets on device; rows_upper = upper bound of the
+// number of A rows (to size the grid).
+cudaError_t launch_gemm_tc(const TcGemmArgs& args, int dtype, int epilogue, int rows_upper,
+                           cudaStream_t stream);
+constexpr int kTcBlockM = 128;
+constexpr int kTcBlockN = 256;  // accumulator columns; SwiGLU: 128 gate + 128 up
+
+int device_sm_count();
+
+}  // namespace moe

@@ -1,0 +1,228 @@
+// Permute / dispatch: expert histogram, prefix scan and a stable gather of
+// token rows into expert-contiguous order ("Advanced GPU Optimization ...
+// Part 5", section 1.2 step 1, token dispatch: a buffer per destination built
+// from the routing decisions, here local; aclnnQuantGroupedMatMulAlltoAllv
+// constraints: sendCounts per expert; determinism by default).
+//
+// Stable order: within expert e the rows appear in (token, slot) order, so
+//   pos[t,j] = offsets[e] + #{(t',j') before (t,j) with ids[t',j'] = e}.
+// Tokens are cut into chunks of kPermuteChunk (32).  Three launches:
+//   1. count:  per-chunk expert histogram in shared memory -> chunk_counts
+//   2. scan:   one CTA turns chunk_counts into per-(chunk, expert) bases
+//              (offsets[e] + rows of e in earlier chunks), counts, offsets
+//   3. gather: one warp ranks the chunk's (t, j) pairs with shuffles (no
+//              atomics, so the order is fixed), then all warps copy each
+//              token row once from HBM into its K destination rows with
+//              16-byte vector loads/stores.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int CH = kPermuteChunk;
+
+__global__ void __launch_bounds__(128)
+permute_count_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
+                     int32_t* __restrict__ chunk_counts, int* status) {
+  __shared__ int hist[256];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const long long base = (long long)blockIdx.x * CH * K;
+  const long long end = min((long long)N * K, base + (long long)CH * K);
+  for (long long i = base + threadIdx.x; i < end; i += blockDim.x) {
+    int e = ids[i];
+    if (e < 0 || e >= E) {
+      set_status(status, kStatusBadIndex);
+      continue;
+    }
+    atomicAdd(&hist[e], 1);  // integer counts: order-independent
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    chunk_counts[(long long)blockIdx.x * E + e] = hist[e];
+}
+
+// One CTA of 1024 threads.  Thread (e, s) owns expert e and a contiguous
+// slice s of the chunks.  Afterwards chunk_counts[c][e] holds the first
+// destination row of chunk c's rows of expert e.
+__global__ void __launch_bounds__(1024)
+permute_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
+                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  __shared__ int part[1024];
+  __shared__ int total[257];
+  int Ep = 1;
+  while (Ep < E) Ep <<= 1;
+  const int S = 1024 / Ep;                 // slices per expert (>= 4 for E <= 256)
+  const int e = threadIdx.x % Ep, s = threadIdx.x / Ep;
+  const int cs = (nchunks + S - 1) / S;
+  const int c0 = s * cs, c1 = min(nchunks, c0 + cs);
+  int sum = 0;
+  if (e < E)
+    for (int c = c0; c < c1; ++c) sum += chunk_counts[(long long)c * E + e];
+  part[threadIdx.x] = sum;
+  __syncthreads();
+  // exclusive scan over the slices of each expert
+  if (threadIdx.x < E) {
+    int run = 0;
+    for (int q = 0; q < S; ++q) {
+      int v = part[q * Ep + threadIdx.x];
+      part[q * Ep + threadIdx.x] = run;
+      run += v;
+    }
+    total[threadIdx.x] = run;
+  }
+  __syncthreads();
+  // exclusive scan over experts (warp 0; E <= 256 -> up to 8 per lane)
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int per = (E + 31) / 32;
+    const int b0 = lane * per, b1 = min(E, b0 + per);
+    int local = 0;
+    for (int q = b0; q < b1; ++q) local += total[q];
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int run = incl - local;
+    for (int q = b0; q < b1; ++q) {
+      int c = total[q];
+      counts[q] = c;
+      offsets[q] = run;
+      total[q] = run;
+      run += c;
+    }
+    if (lane == 31) offsets[E] = incl;
+  }
+  __syncthreads();
+  if (e < E) {
+    int run = total[e] + part[s * Ep + e];
+    for (int c = c0; c < c1; ++c) {
+      int v = chunk_counts[(long long)c * E + e];
+      chunk_counts[(long long)c * E + e] = run;
+      run += v;
+    }
+  }
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(256)
+permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* __restrict__ ids,
+                      int N, int K, int E, const int32_t* __restrict__ chunk_base,
+                      int32_t* __restrict__ pos, int32_t* __restrict__ src, uint4* __restrict__ x_perm,
+                      int* status) {
+  __shared__ int spos[CH][KMAX];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = blockIdx.x;
+  if (warp == 0) {
+    const int t = c * CH + lane;
+    int my[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      my[j] = -1;
+      if (j < K && t < N) {
+        int e = ids[(long long)t * K + j];
+        if (e >= 0 && e < E) my[j] = e;  // bad ids were flagged by the count pass
+      }
+    }
+    // rank of (t, j): earlier slots of t with the same expert ...
+    int rank[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      rank[j] = 0;
+#pragma unroll
+      for (int jj = 0; jj < KMAX; ++jj)
+        if (jj < j && my[jj] == my[j]) rank[j]++;
+    }
+    // ... plus every slot of the earlier tokens of this chunk with that expert
+#pragma unroll
+    for (int jj = 0; jj < KMAX; ++jj) {
+      if (jj >= K) break;
+      for (int sl = 0; sl < 31; ++sl) {
+        int v = __shfl_sync(0xffffffffu, my[jj], sl);
+        if (sl < lane) {
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j)
+            if (v == my[j] && v >= 0) rank[j]++;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j >= K) break;
+      int p = -1;
+      if (my[j] >= 0) {
+        p = chunk_base[(long long)c * E + my[j]] + rank[j];
+        src[p] = t;
+      }
+      if (t < N) pos[(long long)t * K + j] = p;
+      spos[lane][j] = p;
+    }
+  }
+  __syncthreads();
+  // copy: each warp owns tokens warp, warp+8, ...; a row is read once
+  for (int tt = warp; tt < CH; tt += 8) {
+    const int t = c * CH + tt;
+    if (t >= N) break;
+    const uint4* srow = x + (long long)t * row_vecs;
+    int p[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) p[j] = j < K ? spos[tt][j] : -1;
+    int v = lane;
+    for (; v + 96 < row_vecs; v += 128) {
+      uint4 a0 = srow[v], a1 = srow[v + 32], a2 = srow[v + 64], a3 = srow[v + 96];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (p[j] < 0) continue;
+        uint4* drow = x_perm + (long long)p[j] * row_vecs;
+        drow[v] = a0; drow[v + 32] = a1; drow[v + 64] = a2; drow[v + 96] = a3;
+      }
+    }
+    for (; v < row_vecs; v += 32) {
+      uint4 a0 = srow[v];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (p[j] >= 0) x_perm[(long long)p[j] * row_vecs + v] = a0;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_permute_count(const int32_t* ids, int N, int K, int E, int32_t* chunk_counts,
+                                 int* status, cudaStream_t stream) {
+  int nchunks = permute_chunks(N);
+  if (nchunks == 0) return cudaSuccess;
+  permute_count_kernel<<<nchunks, 128, 0, stream>>>(ids, N, K, E, chunk_counts, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_scan(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
+                                int32_t* offsets, cudaStream_t stream) {
+  permute_scan_kernel<<<1, 1024, 0, stream>>>(chunk_counts, nchunks, E, counts, offsets);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* ids, int N, int K,
+                                  int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
+                                  void* x_perm, int* status, cudaStream_t stream) {
+  int nchunks = permute_chunks(N);
+  if (nchunks == 0) return cudaSuccess;
+  int row_vecs = row_bytes / 16;
+  auto xv = static_cast<const uint4*>(x);
+  auto xp = static_cast<uint4*>(x_perm);
+  if (K <= 2)
+    permute_gather_kernel<2><<<nchunks, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base,
+                                                          pos, src, xp, status);
+  else if (K <= 4)
+    permute_gather_kernel<4><<<nchunks, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base,
+                                                          pos, src, xp, status);
+  else
+    permute_gather_kernel<8><<<nchunks, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base,
+                                                          pos, src, xp, status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
