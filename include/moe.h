@@ -25,7 +25,9 @@
  *  - Pointers named *_host are host memory; every other data pointer is
  *    device memory of the plan's device.  The caller allocates and frees all
  *    of them.  The library allocates no device memory (not in
- *    moe_plan_create either); it never frees caller memory.
+ *    moe_plan_create either); it never frees caller memory.  Its only
+ *    device memory of its own is the static scratch array of
+ *    moe_permute_noalloc.
  *  - Launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *    default stream).  Only moe_read_device_status, moe_forward_host and
  *    moe_profile_read synchronise.
@@ -151,6 +153,29 @@ moe_status moe_router_topk(moe_plan plan, const void* x, int32_t* topk_ids, floa
 moe_status moe_permute(moe_plan plan, const void* x, const int32_t* topk_ids, int32_t* counts,
                        int32_t* offsets, int32_t* perm_pos, int32_t* perm_src, void* x_perm,
                        void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_permute for callers that cannot allocate device memory: the pages
+ * have no counterpart of this entry point.  Some callers cannot call
+ * cudaMalloc: code running inside a host framework that owns every device
+ * allocation and passes an operator only its inputs and outputs (a plugin
+ * of an inference engine), or latency-critical code that must not risk the
+ * device-wide synchronisation a cudaMalloc / cudaFree can cause.  This
+ * variant takes no workspace and allocates nothing: its scratch (the
+ * per-chunk expert counts) is a 1 MiB array in the library's static device
+ * memory, held by every GPU that loads the library until the process exits.
+ * Same outputs as moe_permute.  device_status_or_null (device int32, may be
+ * NULL; the caller zeroes it) receives MOE_ERR_DEVICE_BAD_INDEX if an id is
+ * outside [0, E).  Limit: ceil(N/32) * E * 4 bytes <= 1 MiB (e.g. N = 32768
+ * with E = 256); a larger plan is refused with MOE_ERR_WORKSPACE_TOO_SMALL
+ * and nothing is launched.  The first call on each device looks up the
+ * array's device address (with that device current), so make that first
+ * call before any stream capture.  All calls share the one array: calls
+ * whose kernels overlap on the GPU (different streams, or several threads)
+ * race on it; serialise them. */
+moe_status moe_permute_noalloc(moe_plan plan, const void* x, const int32_t* topk_ids,
+                               int32_t* counts, int32_t* offsets, int32_t* perm_pos,
+                               int32_t* perm_src, void* x_perm, int32_t* device_status_or_null,
+                               moe_stream_t stream);
 
 /* Grouped FFN (page 1 section 1.2 local expert execution; Ascend formula
  * gmmY).  Rows [offsets[e], offsets[e+1]) of x_perm go through expert e; the

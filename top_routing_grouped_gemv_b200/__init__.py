@@ -77,6 +77,7 @@ def load(path: str = LIB_PATH):
         "moe_workspace_init": ([P, P, sz, P], ctypes.c_int),
         "moe_router_topk": ([P, P, P, P, P, P], ctypes.c_int),
         "moe_permute": ([P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_permute_noalloc": ([P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
         "moe_grouped_ffn": ([P, P, P, f32, P, P, sz, P], ctypes.c_int),
         "moe_unpermute_combine": ([P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_shared_matmul": ([P, P, i32, i32, P, i32, f32, f32, P, P], ctypes.c_int),
@@ -169,6 +170,15 @@ class Plan:
         _check(self.lib.moe_permute(self.handle, _ptr(x), _ptr(ids), _ptr(counts), _ptr(offsets),
                                     _ptr(pos), _ptr(src), _ptr(x_perm), _ptr(ws), ws.numel(),
                                     _stream(stream)), "moe_permute")
+
+    def permute_noalloc(self, x, ids, counts, offsets, pos, src, x_perm, device_status=None,
+                        stream=None):
+        """moe_permute without a workspace (scratch in the library's static
+        device memory; see include/moe.h)."""
+        _check(self.lib.moe_permute_noalloc(self.handle, _ptr(x), _ptr(ids), _ptr(counts),
+                                            _ptr(offsets), _ptr(pos), _ptr(src), _ptr(x_perm),
+                                            _ptr(device_status), _stream(stream)),
+               "moe_permute_noalloc")
 
     def grouped_ffn(self, x_perm, offsets, y_perm, ws, x_scale: float = 1.0, stream=None):
         _check(self.lib.moe_grouped_ffn(self.handle, _ptr(x_perm), _ptr(offsets), x_scale,

@@ -507,3 +507,14 @@ moe_status moe_profile_read(moe_plan p, float* ms, const char** names, int capac
 int moe_last_launch_count(moe_plan p) { return p ? p->launches : -1; }
 
 }  // extern "C"
+
+bool moe::plan_permute_shape(const moe_plan_s* p, int* N, int* d, int* E, int* K,
+                             int* row_bytes) {
+  if (!p) return false;
+  *N = p->desc.N;
+  *d = p->desc.d;
+  *E = p->desc.E;
+  *K = p->desc.K;
+  *row_bytes = p->desc.d * p->ex;
+  return true;
+}

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+struct moe_plan_s;  // the C ABI's plan (include/moe.h)
+
 namespace moe {
 
 enum DType { kF32 = 0, kBF16 = 1, kE4M3 = 2 };
@@ -76,5 +78,11 @@ constexpr int kTcBlockM = 128;
 constexpr int kTcBlockN = 256;  // accumulator columns; SwiGLU: 128 gate + 128 up
 
 int device_sm_count();
+
+// Shape of a plan for code outside the plan's translation unit: tokens,
+// token width, experts, experts per token and bytes per token row of x.
+// Returns false for a null plan.
+bool plan_permute_shape(const ::moe_plan_s* plan, int* N, int* d, int* E, int* K,
+                        int* row_bytes);
 
 }  // namespace moe

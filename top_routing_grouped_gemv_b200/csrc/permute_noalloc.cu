@@ -1,0 +1,77 @@
+// moe_permute_noalloc: the permute stage for callers that cannot allocate
+// device memory.  Such callers run inside a host framework that owns every
+// device allocation and hands a kernel only its inputs and outputs (an
+// operator plugin of an inference engine, for example), or sit on a
+// latency-critical path where a cudaMalloc / cudaFree, which can synchronise
+// the whole device, is not acceptable.  The per-chunk expert counts that
+// moe_permute keeps in the caller's workspace live here in a file-scope
+// device array instead; nothing is allocated by this entry point.
+//
+// The array is a module-scope __device__ variable: every GPU that loads the
+// library holds its 1 MiB until the process exits.  Its host-side name is
+// only a stand-in for the symbol, so the device address is looked up with
+// cudaGetSymbolAddress once per device (on the first call made with that
+// device current) and cached.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "kernels.h"
+
+namespace {
+
+constexpr size_t kScratchBytes = size_t(1) << 20;
+constexpr int kMaxDevices = 64;
+
+// Per-chunk expert counts, then (after the scan) per-chunk expert bases.
+// Every call writes all ceil(N/32)*E entries it later reads, so no entry has
+// to start at zero.
+static __device__ __align__(256) int32_t g_permute_scratch[kScratchBytes / sizeof(int32_t)];
+
+std::mutex g_mutex;
+int32_t* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_permute_scratch on the current device.
+moe_status scratch_on_current_device(int32_t** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr)
+      return MOE_ERR_CUDA;
+    g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_scratch_ptr[dev];
+  return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" moe_status moe_permute_noalloc(moe_plan plan, const void* x, const int32_t* topk_ids,
+                                          int32_t* counts, int32_t* offsets, int32_t* perm_pos,
+                                          int32_t* perm_src, void* x_perm,
+                                          int32_t* device_status_or_null, moe_stream_t stream) {
+  int N = 0, d = 0, E = 0, K = 0, row_bytes = 0;
+  if (!moe::plan_permute_shape(plan, &N, &d, &E, &K, &row_bytes)) return MOE_ERR_INVALID_ARG;
+  if (!x || !topk_ids || !counts || !offsets || !perm_pos || !perm_src || !x_perm)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+  const int nchunks = moe::permute_chunks(N);
+  if (static_cast<size_t>(nchunks) * E * sizeof(int32_t) > kScratchBytes)
+    return MOE_ERR_WORKSPACE_TOO_SMALL;
+  int32_t* scratch = nullptr;
+  moe_status st = scratch_on_current_device(&scratch);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = stream;
+  int* status = device_status_or_null;
+  if (moe::launch_permute_count(topk_ids, N, K, E, scratch, status, s) != cudaSuccess ||
+      moe::launch_permute_scan(scratch, nchunks, E, counts, offsets, s) != cudaSuccess ||
+      moe::launch_permute_gather(x, row_bytes, topk_ids, N, K, E, scratch, perm_pos, perm_src,
+                                 x_perm, status, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
