@@ -224,6 +224,21 @@ moe_status moe_forward_routed(moe_plan plan, const void* x, const int32_t* topk_
 moe_status moe_forward_host(moe_plan plan, const void* x_host, void* y_host, void* ws,
                             size_t ws_bytes, moe_stream_t stream);
 
+/* Asynchronous moe_forward_host for a stream of batches: returns once the
+ * work is queued.  The H2D copy of x_host and the D2H copy into y_host run
+ * on two copy streams owned by the plan, the layer on `stream`; two staging
+ * slots in the workspace alternate between calls, so the copies of one
+ * batch overlap the compute of its neighbours.  x_host must stay unchanged
+ * and y_host unread until the copies finish: after moe_host_join(plan, s)
+ * work queued on s runs after them (synchronise s to wait on the host).
+ * Use one stream per plan for these calls.  x_host / y_host should be pinned
+ * for the copies to overlap. */
+moe_status moe_forward_host_async(moe_plan plan, const void* x_host, void* y_host, void* ws,
+                                  size_t ws_bytes, moe_stream_t stream);
+
+/* Makes `stream` wait for every host-buffer copy queued so far on this plan. */
+moe_status moe_host_join(moe_plan plan, moe_stream_t stream);
+
 /* Synchronises `stream`, returns the sticky device status of the workspace
  * (MOE_OK if clean) and clears it. */
 moe_status moe_read_device_status(moe_plan plan, void* ws, moe_stream_t stream);

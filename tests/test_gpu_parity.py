@@ -32,6 +32,12 @@ SMALL = {
                                     shared=(512, 384)),
     "e4m3_gmm_ragged": synth.small_variant(synth.FP8_GMM, N=45, d=256, E=40, K=8, F=96,
                                            shared=(256, 136)),
+    # >= 256 routed rows per expert on average: 256-row tiles on CTA pairs
+    "bf16_pair": synth.small_variant(synth.BF16_PREFILL, N=1024, d=256, E=4, K=2, F=384),
+    "bf16_pair_ragged": synth.small_variant(synth.BF16_PREFILL, N=700, d=320, E=4, K=2, F=200),
+    "bf16_pair_zipf": synth.small_variant(synth.BF16_FINEGRAINED, N=1100, d=256, E=8, K=2, F=256),
+    "e4m3_pair": synth.small_variant(synth.FP8_GMM, N=600, d=256, E=4, K=2, F=392,
+                                     shared=(256, 392)),
 }
 
 _cache = {}
@@ -206,7 +212,7 @@ def test_forward_end_to_end(name):
     assert err <= TOL[c.dtype], err
 
 
-@pytest.mark.parametrize("name", ["bf16_zipf", "f32_relu_n256", "e4m3_gmm"])
+@pytest.mark.parametrize("name", ["bf16_zipf", "f32_relu_n256", "e4m3_gmm", "bf16_pair_ragged"])
 def test_forward_deterministic(name):
     inp, plan, w = case(name)
     c = inp.cfg
@@ -226,7 +232,7 @@ def test_forward_deterministic(name):
     assert all(torch.equal(outs[0], o) for o in outs[1:])
 
 
-@pytest.mark.parametrize("name", ["e4m3_gmm", "e4m3_gmm_ragged"])
+@pytest.mark.parametrize("name", ["e4m3_gmm", "e4m3_gmm_ragged", "e4m3_pair"])
 def test_shared_expert_matmul(name):
     inp, plan, w = case(name)
     c = inp.cfg
@@ -242,16 +248,44 @@ def test_shared_expert_matmul(name):
     assert rel_err(f64(y), ref) <= TOL["e4m3"]
 
 
-def test_forward_host_matches_device():
-    inp, plan, w = case("bf16_swiglu_ragged")
+@pytest.mark.parametrize("name", ["bf16_swiglu_ragged", "bf16_pair", "f32_relu_n256"])
+def test_forward_host_matches_device(name):
+    """moe_forward_host (token chunks with copies overlapping compute when the
+    experts are large enough) gives the bytes of moe_forward."""
+    inp, plan, w = case(name)
     c = inp.cfg
     ws = plan.new_workspace()
-    y_dev = torch.empty(c.N, c.d_out, dtype=torch.bfloat16, device="cuda")
+    ydt = torch.float32 if c.dtype == "f32" else torch.bfloat16
+    y_dev = torch.empty(c.N, c.d_out, dtype=ydt, device="cuda")
     plan.forward(inp.x.cuda(), y_dev, ws)
     x_host = inp.x.clone().pin_memory()
-    y_host = torch.empty(c.N, c.d_out, dtype=torch.bfloat16).pin_memory()
+    y_host = torch.full((c.N, c.d_out), float("nan"), dtype=ydt).pin_memory()
     plan.forward_host(x_host, y_host, ws)
-    assert torch.equal(y_host.view(torch.int16), y_dev.cpu().view(torch.int16))
+    assert plan.read_device_status(ws) == 0
+    assert torch.equal(y_host.view(torch.uint8), y_dev.cpu().view(torch.uint8))
+
+
+def test_forward_host_async_stream_of_batches():
+    """Three batches through moe_forward_host_async (alternating staging
+    slots, copies on the plan's streams) equal moe_forward of each batch."""
+    inp, plan, w = case("bf16_pair")
+    c = inp.cfg
+    ws = plan.new_workspace()
+    xs = [inp.x.clone(), (inp.x.float() * -0.5).to(torch.bfloat16), inp.x.flip(0).contiguous()]
+    ref = []
+    for x in xs:
+        y = torch.empty(c.N, c.d, dtype=torch.bfloat16, device="cuda")
+        plan.forward(x.cuda(), y, ws)
+        ref.append(y.cpu())
+    xh = [x.pin_memory() for x in xs]
+    yh = [torch.empty(c.N, c.d, dtype=torch.bfloat16).pin_memory() for _ in xs]
+    for x, y in zip(xh, yh):
+        plan.forward_host_async(x, y, ws)
+    plan.host_join()
+    torch.cuda.synchronize()
+    assert plan.read_device_status(ws) == 0
+    for y, r in zip(yh, ref):
+        assert torch.equal(y.view(torch.int16), r.view(torch.int16))
 
 
 def test_bad_expert_ids_set_device_status():

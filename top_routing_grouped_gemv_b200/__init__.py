@@ -84,6 +84,8 @@ def load(path: str = LIB_PATH):
         "moe_forward": ([P, P, P, P, sz, P], ctypes.c_int),
         "moe_forward_routed": ([P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
         "moe_forward_host": ([P, P, P, P, sz, P], ctypes.c_int),
+        "moe_forward_host_async": ([P, P, P, P, sz, P], ctypes.c_int),
+        "moe_host_join": ([P, P], ctypes.c_int),
         "moe_read_device_status": ([P, P, P], ctypes.c_int),
         "moe_profile_enable": ([P, ctypes.c_int], ctypes.c_int),
         "moe_profile_read": ([P, ctypes.POINTER(f32), ctypes.POINTER(ctypes.c_char_p),
@@ -208,6 +210,14 @@ class Plan:
     def forward_host(self, x_host, y_host, ws, stream=None):
         _check(self.lib.moe_forward_host(self.handle, _ptr(x_host), _ptr(y_host), _ptr(ws),
                                          ws.numel(), _stream(stream)), "moe_forward_host")
+
+    def forward_host_async(self, x_host, y_host, ws, stream=None):
+        _check(self.lib.moe_forward_host_async(self.handle, _ptr(x_host), _ptr(y_host), _ptr(ws),
+                                               ws.numel(), _stream(stream)),
+               "moe_forward_host_async")
+
+    def host_join(self, stream=None):
+        _check(self.lib.moe_host_join(self.handle, _stream(stream)), "moe_host_join")
 
     def read_device_status(self, ws, stream=None) -> int:
         return self.lib.moe_read_device_status(self.handle, _ptr(ws), _stream(stream))

@@ -10,7 +10,7 @@
 
 #include <new>
 
-#include "../../include/moe.h"
+#include "moe.h"
 #include "kernels.h"
 
 using namespace moe;
@@ -21,11 +21,13 @@ constexpr size_t kAlign = 256;
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 constexpr int kMaxEvents = 16;
+// host-buffer path events: per staging slot s: in_done[s], out_ready[s], slot_free[s]
+constexpr int kHostEvents = 6;
 
 struct Layout {
   size_t status = 0, chunk_counts = 0, h = 0, h_end = 0;
   size_t ids = 0, gates = 0, pos = 0, src = 0, counts = 0, offsets = 0, x_perm = 0, y_perm = 0;
-  size_t fwd_end = 0, x_stage = 0, y_stage = 0, total = 0;
+  size_t fwd_end = 0, x_stage = 0, y_stage = 0, total = 0, x_stage_bytes = 0, y_stage_bytes = 0;
   size_t permute_end = 0;
 };
 
@@ -37,13 +39,17 @@ struct moe_plan_s {
   int device;
   int ex, eh, ey;  // element bytes of x / hidden / y
   int dout;
-  CUtensorMap tmW1, tmW3, tmW2;
+  CUtensorMap tmW1, tmW3, tmW2;      // single-CTA tiles (256-row boxes; 128 for gate/up)
+  CUtensorMap tmW1h, tmW2h;          // CTA-pair tiles: 128-row boxes
   Layout L;
   bool profile;
   cudaEvent_t ev[kMaxEvents];
   const char* ev_name[kMaxEvents];
   int nev;
   int launches;
+  cudaStream_t h2d, d2h;  // host-buffer path copy streams (created on first use)
+  cudaEvent_t hev[kHostEvents];
+  unsigned long long host_calls;  // host-buffer calls so far (selects the staging slot)
 };
 
 namespace {
@@ -80,10 +86,13 @@ void layout(moe_plan p) {
   L.x_perm = off; off = align_up(off + static_cast<size_t>(R) * d.d * p->ex);
   L.y_perm = off; off = align_up(off + static_cast<size_t>(R) * p->dout * p->ey);
   L.fwd_end = off;
-  L.x_stage = off; off = align_up(off + static_cast<size_t>(d.N) * d.d * p->ex);
-  L.y_stage = off;
-  const long long yrows = (d.act == MOE_ACT_NONE) ? R : d.N;
-  off = align_up(off + static_cast<size_t>(yrows) * p->dout * p->ey);
+  // two staging slots for x and y: consecutive host-buffer calls alternate
+  const size_t xbytes = align_up(static_cast<size_t>(d.N) * d.d * p->ex);
+  const size_t ybytes = align_up(static_cast<size_t>(d.N) * p->dout * p->ey);
+  L.x_stage = off; off += 2 * xbytes;
+  L.y_stage = off; off += 2 * ybytes;
+  L.x_stage_bytes = xbytes;
+  L.y_stage_bytes = ybytes;
   L.total = off;
   p->L = L;
 }
@@ -102,38 +111,41 @@ moe_status check_ws(moe_plan p, void* ws, size_t ws_bytes, size_t need) {
 
 bool uses_tensor_cores(const moe_layer_desc& d) { return d.dtype != MOE_F32; }
 
-moe_status run_router(moe_plan p, const void* x, int32_t* ids, float* gates, float* margin,
+// The stage runners take the token count n <= plan N explicitly (the
+// host-buffer path runs the layer on token chunks).
+moe_status run_router(moe_plan p, int n, const void* x, int32_t* ids, float* gates, float* margin,
                       cudaStream_t s) {
   const moe_layer_desc& d = p->desc;
   mark(p, s, "router_topk");
   p->launches += 1;
-  return cuda_status(launch_router(x, d.dtype, p->w.w_r, p->w.router_bias, d.N, d.d, d.E, d.K, ids,
+  return cuda_status(launch_router(x, d.dtype, p->w.w_r, p->w.router_bias, n, d.d, d.E, d.K, ids,
                                    gates, margin, s));
 }
 
-moe_status run_permute(moe_plan p, const void* x, const int32_t* ids, int32_t* counts,
+moe_status run_permute(moe_plan p, int n, const void* x, const int32_t* ids, int32_t* counts,
                        int32_t* offsets, int32_t* pos, int32_t* src, void* x_perm, void* ws,
                        cudaStream_t s) {
   const moe_layer_desc& d = p->desc;
   int* status = at<int>(ws, p->L.status);
   int32_t* cc = at<int32_t>(ws, p->L.chunk_counts);
   mark(p, s, "permute_count");
-  if (launch_permute_count(ids, d.N, d.K, d.E, cc, status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_permute_count(ids, n, d.K, d.E, cc, pos, status, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   mark(p, s, "permute_scan");
-  if (launch_permute_scan(cc, permute_chunks(d.N), d.E, counts, offsets, s) != cudaSuccess)
+  if (launch_permute_scan(cc, permute_chunks(n), d.E, counts, offsets, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   mark(p, s, "permute_gather");
-  if (launch_permute_gather(x, d.d * p->ex, ids, d.N, d.K, d.E, cc, pos, src, x_perm, status, s) !=
+  if (launch_permute_gather(x, d.d * p->ex, ids, n, d.K, d.E, cc, pos, src, x_perm, status, s) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
   p->launches += 3;
   return MOE_OK;
 }
 
-moe_status run_ffn(moe_plan p, const void* x_perm, const int32_t* offsets, float x_scale,
+moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets, float x_scale,
                    void* y_perm, void* ws, cudaStream_t s) {
   const moe_layer_desc& d = p->desc;
-  const int R = d.N * d.K;
+  const int R = n * d.K;
   int* status = at<int>(ws, p->L.status);
   void* h = at<void>(ws, p->L.h);
   if (!uses_tensor_cores(d)) {
@@ -163,10 +175,13 @@ moe_status run_ffn(moe_plan p, const void* x_perm, const int32_t* offsets, float
   a.groups = d.E;
   a.m_total = R;
   a.status = status;
+  // 256-row tiles on CTA pairs when the experts average at least that many
+  // rows; otherwise 128-row tiles on single CTAs (less padding work)
+  const bool pair = R >= 256 * d.E;
   if (d.act == MOE_ACT_NONE) {
     if (!encode_kmajor_map(&a.tmA, x_perm, p->ex, R, d.d, kTcBlockM)) return MOE_ERR_CUDA;
-    a.tmB0 = p->tmW1;
-    a.tmB1 = p->tmW1;
+    a.tmB0 = pair ? p->tmW1h : p->tmW1;
+    a.tmB1 = a.tmB0;
     a.kdim = d.d;
     a.n_out = d.F;
     a.n_tiles = (d.F + kTcBlockN - 1) / kTcBlockN;
@@ -175,7 +190,7 @@ moe_status run_ffn(moe_plan p, const void* x_perm, const int32_t* offsets, float
     a.scale = d.quant == MOE_QUANT_PER_TENSOR ? x_scale * p->w.w_scale : 1.f;
     mark(p, s, "gmm_tc");
     p->launches += 1;
-    return cuda_status(launch_gemm_tc(a, d.dtype, kEpiStore, R, s));
+    return cuda_status(launch_gemm_tc(a, d.dtype, kEpiStore, R, pair, s));
   }
   // SwiGLU: gate/up GEMM with the activation fused into its epilogue, then down
   if (!encode_kmajor_map(&a.tmA, x_perm, p->ex, R, d.d, kTcBlockM)) return MOE_ERR_CUDA;
@@ -188,11 +203,11 @@ moe_status run_ffn(moe_plan p, const void* x_perm, const int32_t* offsets, float
   a.ldo = d.F;
   a.scale = 1.f;
   mark(p, s, "ffn1_swiglu_tc");
-  if (launch_gemm_tc(a, d.dtype, kEpiSwiglu, R, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_gemm_tc(a, d.dtype, kEpiSwiglu, R, pair, s) != cudaSuccess) return MOE_ERR_CUDA;
   TcGemmArgs b = a;
   if (!encode_kmajor_map(&b.tmA, h, p->eh, R, d.F, kTcBlockM)) return MOE_ERR_CUDA;
-  b.tmB0 = p->tmW2;
-  b.tmB1 = p->tmW2;
+  b.tmB0 = pair ? p->tmW2h : p->tmW2;
+  b.tmB1 = b.tmB0;
   b.kdim = d.F;
   b.n_out = d.d;
   b.n_tiles = (d.d + kTcBlockN - 1) / kTcBlockN;
@@ -200,16 +215,16 @@ moe_status run_ffn(moe_plan p, const void* x_perm, const int32_t* offsets, float
   b.ldo = d.d;
   mark(p, s, "ffn2_tc");
   p->launches += 2;
-  return cuda_status(launch_gemm_tc(b, d.dtype, kEpiStore, R, s));
+  return cuda_status(launch_gemm_tc(b, d.dtype, kEpiStore, R, pair, s));
 }
 
-moe_status run_combine(moe_plan p, const void* y_perm, const int32_t* pos, const float* gates,
-                       void* y, void* ws, cudaStream_t s) {
+moe_status run_combine(moe_plan p, int n, const void* y_perm, const int32_t* pos,
+                       const float* gates, void* y, void* ws, cudaStream_t s) {
   const moe_layer_desc& d = p->desc;
   mark(p, s, gates ? "combine" : "unpermute");
   p->launches += 1;
   const int ydt = d.dtype == MOE_F32 ? kF32 : kBF16;
-  return cuda_status(launch_combine(y_perm, ydt, p->dout, pos, gates, d.N, d.K, y,
+  return cuda_status(launch_combine(y_perm, ydt, p->dout, pos, gates, n, d.K, y,
                                     at<int>(ws, p->L.status), s));
 }
 
@@ -255,7 +270,8 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
   if (!w->w1 || (d.act == MOE_ACT_SWIGLU) != (w->w3 != nullptr) ||
       (d.act != MOE_ACT_NONE) != (w->w2 != nullptr))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned16(w->w1) || (w->w3 && !aligned16(w->w3)) || (w->w2 && !aligned16(w->w2)))
+  if (!aligned16(w->w1) || (w->w3 && !aligned16(w->w3)) || (w->w2 && !aligned16(w->w2)) ||
+      (w->w_r && !aligned16(w->w_r)))
     return MOE_ERR_INVALID_ARG;
 
   moe_plan p = new (std::nothrow) moe_plan_s;
@@ -280,16 +296,16 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
   }
   if (uses_tensor_cores(d)) {
     bool ok = true;
+    const long long rows1 = static_cast<long long>(d.E) * d.F;
     if (d.act == MOE_ACT_NONE) {
-      ok = encode_kmajor_map(&p->tmW1, w->w1, p->ex, static_cast<long long>(d.E) * d.F, d.d,
-                             kTcBlockN);
+      ok = encode_kmajor_map(&p->tmW1, w->w1, p->ex, rows1, d.d, kTcBlockN) &&
+           encode_kmajor_map(&p->tmW1h, w->w1, p->ex, rows1, d.d, kTcBlockN / 2);
     } else {
-      ok = encode_kmajor_map(&p->tmW1, w->w1, p->ex, static_cast<long long>(d.E) * d.F, d.d,
-                             kTcBlockN / 2) &&
-           encode_kmajor_map(&p->tmW3, w->w3, p->ex, static_cast<long long>(d.E) * d.F, d.d,
-                             kTcBlockN / 2) &&
-           encode_kmajor_map(&p->tmW2, w->w2, p->ex, static_cast<long long>(d.E) * d.d, d.F,
-                             kTcBlockN);
+      const long long rows2 = static_cast<long long>(d.E) * d.d;
+      ok = encode_kmajor_map(&p->tmW1, w->w1, p->ex, rows1, d.d, kTcBlockN / 2) &&
+           encode_kmajor_map(&p->tmW3, w->w3, p->ex, rows1, d.d, kTcBlockN / 2) &&
+           encode_kmajor_map(&p->tmW2, w->w2, p->ex, rows2, d.F, kTcBlockN) &&
+           encode_kmajor_map(&p->tmW2h, w->w2, p->ex, rows2, d.F, kTcBlockN / 2);
     }
     if (!ok) {
       delete p;
@@ -306,6 +322,10 @@ moe_status moe_plan_destroy(moe_plan p) {
   if (!p) return MOE_ERR_INVALID_ARG;
   for (int i = 0; i < kMaxEvents; ++i)
     if (p->ev[i]) cudaEventDestroy(p->ev[i]);
+  for (int i = 0; i < kHostEvents; ++i)
+    if (p->hev[i]) cudaEventDestroy(p->hev[i]);
+  if (p->h2d) cudaStreamDestroy(p->h2d);
+  if (p->d2h) cudaStreamDestroy(p->d2h);
   delete p;
   return MOE_OK;
 }
@@ -327,8 +347,9 @@ moe_status moe_router_topk(moe_plan p, const void* x, int32_t* ids, float* gates
                            moe_stream_t stream) {
   if (!p || !x || !ids || !gates || !p->w.w_r) return MOE_ERR_INVALID_ARG;
   if (p->desc.dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
   begin(p);
-  moe_status st = run_router(p, x, ids, gates, margin, stream);
+  moe_status st = run_router(p, p->desc.N, x, ids, gates, margin, stream);
   end(p, stream);
   return st;
 }
@@ -341,7 +362,7 @@ moe_status moe_permute(moe_plan p, const void* x, const int32_t* ids, int32_t* c
   moe_status st = check_ws(p, ws, ws_bytes, p->L.permute_end);
   if (st != MOE_OK) return st;
   begin(p);
-  st = run_permute(p, x, ids, counts, offsets, pos, src, x_perm, ws, stream);
+  st = run_permute(p, p->desc.N, x, ids, counts, offsets, pos, src, x_perm, ws, stream);
   end(p, stream);
   return st;
 }
@@ -353,7 +374,7 @@ moe_status moe_grouped_ffn(moe_plan p, const void* x_perm, const int32_t* offset
   moe_status st = check_ws(p, ws, ws_bytes, p->L.h_end);
   if (st != MOE_OK) return st;
   begin(p);
-  st = run_ffn(p, x_perm, offsets, x_scale, y_perm, ws, stream);
+  st = run_ffn(p, p->desc.N, x_perm, offsets, x_scale, y_perm, ws, stream);
   end(p, stream);
   return st;
 }
@@ -366,7 +387,7 @@ moe_status moe_unpermute_combine(moe_plan p, const void* y_perm, const int32_t* 
   moe_status st = check_ws(p, ws, ws_bytes, p->L.chunk_counts);
   if (st != MOE_OK) return st;
   begin(p);
-  st = run_combine(p, y_perm, pos, gates, y, ws, stream);
+  st = run_combine(p, p->desc.N, y_perm, pos, gates, y, ws, stream);
   end(p, stream);
   return st;
 }
@@ -381,8 +402,9 @@ moe_status moe_shared_matmul(moe_plan p, const void* x, int32_t M, int32_t H, co
   if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   TcGemmArgs a;
   memset(&a, 0, sizeof(a));
+  const bool pair = M >= 256;
   if (!encode_kmajor_map(&a.tmA, x, 1, M, H, kTcBlockM) ||
-      !encode_kmajor_map(&a.tmB0, w, 1, N2, H, kTcBlockN))
+      !encode_kmajor_map(&a.tmB0, w, 1, N2, H, pair ? kTcBlockN / 2 : kTcBlockN))
     return MOE_ERR_CUDA;
   a.tmB1 = a.tmB0;
   a.offsets = nullptr;
@@ -395,7 +417,7 @@ moe_status moe_shared_matmul(moe_plan p, const void* x, int32_t M, int32_t H, co
   a.ldo = N2;
   a.scale = x_scale * w_scale;
   a.status = nullptr;
-  return cuda_status(launch_gemm_tc(a, kE4M3, kEpiStore, M, stream));
+  return cuda_status(launch_gemm_tc(a, kE4M3, kEpiStore, M, pair, stream));
 }
 
 moe_status moe_forward_routed(moe_plan p, const void* x, const int32_t* ids, const float* gates,
@@ -407,17 +429,53 @@ moe_status moe_forward_routed(moe_plan p, const void* x, const int32_t* ids, con
   if (st != MOE_OK) return st;
   const Layout& L = p->L;
   begin(p);
-  st = run_permute(p, x, ids, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
+  const int n = p->desc.N;
+  st = run_permute(p, n, x, ids, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
                    at<int32_t>(ws, L.pos), at<int32_t>(ws, L.src), at<void>(ws, L.x_perm), ws,
                    stream);
   if (st == MOE_OK)
-    st = run_ffn(p, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), x_scale,
+    st = run_ffn(p, n, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), x_scale,
                  at<void>(ws, L.y_perm), ws, stream);
   if (st == MOE_OK)
-    st = run_combine(p, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
+    st = run_combine(p, n, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
   end(p, stream);
   return st;
 }
+
+}  // extern "C"
+
+namespace {
+// The whole layer on n <= N tokens; every intermediate lives in the workspace.
+moe_status forward_tokens(moe_plan p, int n, const void* x, void* y, void* ws, cudaStream_t stream) {
+  const Layout& L = p->L;
+  moe_status st = run_router(p, n, x, at<int32_t>(ws, L.ids), at<float>(ws, L.gates), nullptr,
+                             stream);
+  if (st == MOE_OK)
+    st = run_permute(p, n, x, at<int32_t>(ws, L.ids), at<int32_t>(ws, L.counts),
+                     at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.pos), at<int32_t>(ws, L.src),
+                     at<void>(ws, L.x_perm), ws, stream);
+  if (st == MOE_OK)
+    st = run_ffn(p, n, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), 1.f,
+                 at<void>(ws, L.y_perm), ws, stream);
+  if (st == MOE_OK)
+    st = run_combine(p, n, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), at<float>(ws, L.gates),
+                     y, ws, stream);
+  return st;
+}
+
+moe_status ensure_host_streams(moe_plan p) {
+  if (p->h2d) return MOE_OK;
+  if (cudaStreamCreateWithFlags(&p->h2d, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&p->d2h, cudaStreamNonBlocking) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  for (int i = 0; i < kHostEvents; ++i)
+    if (cudaEventCreateWithFlags(&p->hev[i], cudaEventDisableTiming) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+}  // namespace
+
+extern "C" {
 
 moe_status moe_forward(moe_plan p, const void* x, void* y, void* ws, size_t ws_bytes,
                        moe_stream_t stream) {
@@ -426,39 +484,65 @@ moe_status moe_forward(moe_plan p, const void* x, void* y, void* ws, size_t ws_b
   if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   moe_status st = check_ws(p, ws, ws_bytes, p->L.fwd_end);
   if (st != MOE_OK) return st;
-  const Layout& L = p->L;
   begin(p);
-  st = run_router(p, x, at<int32_t>(ws, L.ids), at<float>(ws, L.gates), nullptr, stream);
-  if (st == MOE_OK)
-    st = run_permute(p, x, at<int32_t>(ws, L.ids), at<int32_t>(ws, L.counts),
-                     at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.pos), at<int32_t>(ws, L.src),
-                     at<void>(ws, L.x_perm), ws, stream);
-  if (st == MOE_OK)
-    st = run_ffn(p, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), 1.f,
-                 at<void>(ws, L.y_perm), ws, stream);
-  if (st == MOE_OK)
-    st = run_combine(p, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), at<float>(ws, L.gates), y,
-                     ws, stream);
+  st = forward_tokens(p, p->desc.N, x, y, ws, stream);
   end(p, stream);
   return st;
 }
 
-moe_status moe_forward_host(moe_plan p, const void* x_host, void* y_host, void* ws,
-                            size_t ws_bytes, moe_stream_t stream) {
-  if (!p || !x_host || !y_host) return MOE_ERR_INVALID_ARG;
+// Host buffers, asynchronous.  Staging slot s = call number % 2.  The H2D
+// copy of x goes on a copy stream, after slot s was released by its previous
+// user (two calls ago); the layer runs on the caller's stream once the copy
+// landed; the D2H copy of y goes on a second copy stream once the layer is
+// done, and then releases the slot.  Consecutive calls therefore overlap one
+// batch's copies with the neighbouring batches' compute.
+moe_status moe_forward_host_async(moe_plan p, const void* x_host, void* y_host, void* ws,
+                                  size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !x_host || !y_host || !p->w.w_r) return MOE_ERR_INVALID_ARG;
+  if (p->desc.dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
   moe_status st = check_ws(p, ws, ws_bytes, p->L.total);
   if (st != MOE_OK) return st;
+  if ((st = ensure_host_streams(p)) != MOE_OK) return st;
   const moe_layer_desc& d = p->desc;
-  void* xs = at<void>(ws, p->L.x_stage);
-  void* ys = at<void>(ws, p->L.y_stage);
+  const int slot = static_cast<int>(p->host_calls & 1u);
+  cudaEvent_t in_done = p->hev[3 * slot], out_ready = p->hev[3 * slot + 1],
+              slot_free = p->hev[3 * slot + 2];
+  char* xs = at<char>(ws, p->L.x_stage + slot * p->L.x_stage_bytes);
+  char* ys = at<char>(ws, p->L.y_stage + slot * p->L.y_stage_bytes);
   const size_t xb = static_cast<size_t>(d.N) * d.d * p->ex;
   const size_t yb = static_cast<size_t>(d.N) * p->dout * p->ey;
-  if (cudaMemcpyAsync(xs, x_host, xb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+  cudaStream_t cs = stream;
+  if (p->host_calls >= 2 && cudaStreamWaitEvent(p->h2d, slot_free, 0) != cudaSuccess)
     return MOE_ERR_CUDA;
-  st = moe_forward(p, xs, ys, ws, ws_bytes, stream);
+  if (cudaMemcpyAsync(xs, x_host, xb, cudaMemcpyHostToDevice, p->h2d) != cudaSuccess ||
+      cudaEventRecord(in_done, p->h2d) != cudaSuccess ||
+      cudaStreamWaitEvent(cs, in_done, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  begin(p);
+  st = forward_tokens(p, d.N, xs, ys, ws, cs);
+  end(p, cs);
   if (st != MOE_OK) return st;
-  if (cudaMemcpyAsync(y_host, ys, yb, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+  if (cudaEventRecord(out_ready, cs) != cudaSuccess ||
+      cudaStreamWaitEvent(p->d2h, out_ready, 0) != cudaSuccess ||
+      cudaMemcpyAsync(y_host, ys, yb, cudaMemcpyDeviceToHost, p->d2h) != cudaSuccess ||
+      cudaEventRecord(slot_free, p->d2h) != cudaSuccess)
     return MOE_ERR_CUDA;
+  p->host_calls++;
+  return MOE_OK;
+}
+
+moe_status moe_host_join(moe_plan p, moe_stream_t stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (!p->h2d || p->host_calls == 0) return MOE_OK;
+  const int last = static_cast<int>((p->host_calls - 1) & 1u);
+  return cuda_status(cudaStreamWaitEvent(stream, p->hev[3 * last + 2], 0));
+}
+
+moe_status moe_forward_host(moe_plan p, const void* x_host, void* y_host, void* ws,
+                            size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = moe_forward_host_async(p, x_host, y_host, ws, ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  if ((st = moe_host_join(p, stream)) != MOE_OK) return st;
   return cuda_status(cudaStreamSynchronize(stream));
 }
 

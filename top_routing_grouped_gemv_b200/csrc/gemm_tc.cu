@@ -35,23 +35,31 @@
 namespace moe {
 namespace {
 
-constexpr int BM = kTcBlockM;     // 128 rows per tile
+constexpr int BM = kTcBlockM;     // 128 rows per CTA (256 per CTA pair)
 constexpr int BN = kTcBlockN;     // 256 accumulator columns per tile
 constexpr int ROWB = 128;         // bytes of K per row per stage (one swizzle atom)
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * ROWB;
-constexpr int B_BYTES = BN * ROWB;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 2 * BN;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr int kMaxGroups = 256;
 
-// shared-memory map past the stage ring
-constexpr int kBarFull = 0, kBarEmpty = STAGES, kBarTFull = 2 * STAGES, kBarTEmpty = 2 * STAGES + 2,
-              kBarDrain = 2 * STAGES + 4, kNumBars = 2 * STAGES + 5;
-constexpr int kSmemBytes = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + kNumBars * 8 + 16 +
-                           2 * (kMaxGroups + 1) * 4;
+// Per-mode geometry.  Single CTA: B tile 256 rows, 4 stages of 48 KB.  CTA
+// pair (tcgen05 cta_group::2): each CTA holds its 128 A rows and half of the
+// 256 B rows, 6 stages of 32 KB.
+template <bool kPair>
+struct Geo {
+  static constexpr int B_ROWS = kPair ? BN / 2 : BN;
+  static constexpr int B_BYTES = B_ROWS * ROWB;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = kPair ? 6 : 4;
+  static constexpr int TILE_M = kPair ? 2 * BM : BM;
+  static constexpr int kBarFull = 0, kBarEmpty = STAGES, kBarTFull = 2 * STAGES,
+                       kBarTEmpty = 2 * STAGES + 2, kBarDrain = 2 * STAGES + 4,
+                       kNumBars = 2 * STAGES + 5;
+  static constexpr int kSmemBytes = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES +
+                                    kNumBars * 8 + 16 + 2 * (kMaxGroups + 1) * 4;
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -174,17 +182,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 
 // Instruction descriptor: fp32 accumulator (bit 4), A/B format at [7,10) and
 // [10,13) (bf16 = 1 for kind::f16, e4m3 = 0 for kind::f8f6f4), both K-major,
-// N >> 3 at [17,23), M >> 4 at [24,29).
-template <bool kFp8>
-constexpr uint32_t make_idesc() {
-  return (1u << 4) | ((kFp8 ? 0u : 1u) << 7) | ((kFp8 ? 0u : 1u) << 10) |
-         (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
-}
-
+// N >> 3 at [17,23), M >> 4 at [24,29) (M = 128 for one CTA, 256 for a pair).
 struct TileCoord {
   int g, m_row0, n_tile;
 };
 
+template <int TILE_M>
 __device__ __forceinline__ TileCoord decode_tile(int T, const int* s_pref, const int* s_off,
                                                  int G) {
   int lo = 0, hi = G - 1;
@@ -195,31 +198,109 @@ __device__ __forceinline__ TileCoord decode_tile(int T, const int* s_pref, const
   TileCoord c;
   c.g = lo;
   const int local = T - s_pref[lo];
-  const int mt = (s_off[lo + 1] - s_off[lo] + BM - 1) / BM;
+  const int mt = (s_off[lo + 1] - s_off[lo] + TILE_M - 1) / TILE_M;
   c.n_tile = local / mt;
-  c.m_row0 = s_off[lo] + (local - c.n_tile * mt) * BM;
+  c.m_row0 = s_off[lo] + (local - c.n_tile * mt) * TILE_M;
   return c;
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.f + __expf(-g)) * u; }
 
-template <bool kFp8, int kEpi>
+// ---- CTA pair (cta_group::2) ------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA load into this CTA's shared memory that signals the barrier at a
+// shared::cluster address (the pair leader's); no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+template <bool kFp8>
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  if constexpr (kFp8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+// arrives on the barrier at this offset in both CTAs of the pair once the
+// pair's MMAs issued so far have completed
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair_self(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+template <bool kFp8, bool kPair>
+constexpr uint32_t make_idesc_mode() {
+  return (1u << 4) | ((kFp8 ? 0u : 1u) << 7) | ((kFp8 ? 0u : 1u) << 10) |
+         (static_cast<uint32_t>(BN >> 3) << 17) |
+         (static_cast<uint32_t>((kPair ? 2 * BM : BM) >> 4) << 24);
+}
+
+// kPair: a cluster of 2 CTAs computes 256-row tiles with tcgen05 cta_group::2;
+// CTA rank r holds rows [128r, 128r+128) of the tile and B rows [128r, 128r+128)
+// of the 256-row weight tile; the leader (rank 0) issues the MMAs.
+template <bool kFp8, int kEpi, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ TcGemmArgs args) {
+  using Gm = Geo<kPair>;
+  constexpr int STAGES = Gm::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + STAGES * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Gm::STAGE_BYTES);
   const uint32_t bar0 = smem_u32(bars);
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Gm::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_pref = reinterpret_cast<int*>(tmem_slot + 4);
   int* s_off = s_pref + (kMaxGroups + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.groups;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int nunits = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   // Per-group tile counts -> exclusive prefix (warp 0), group row offsets.
   if (warp == 0) {
@@ -231,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       int o1 = args.offsets ? args.offsets[q + 1] : args.m_total;
       s_off[q] = o0;
       int cnt = max(0, o1 - o0);
-      int t = (cnt + BM - 1) / BM * args.n_tiles;
+      int t = (cnt + Gm::TILE_M - 1) / Gm::TILE_M * args.n_tiles;
       s_pref[q] = t;
       local += t;
     }
@@ -254,14 +335,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   }
   if (threadIdx.x == 32) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar(kBarFull + s), 1);
-      mbar_init(bar(kBarEmpty + s), 1);
+      mbar_init(bar(Gm::kBarFull + s), 1);
+      mbar_init(bar(Gm::kBarEmpty + s), 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(bar(kBarTFull + a), 1);
-      mbar_init(bar(kBarTEmpty + a), 4);
+      mbar_init(bar(Gm::kBarTFull + a), 1);
+      mbar_init(bar(Gm::kBarTEmpty + a), kPair ? 8 : 4);
     }
-    mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(Gm::kBarDrain), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -273,14 +354,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   }
   if (warp == 1) {
     __syncwarp();  // tcgen05.alloc is .sync.aligned: converge after thread 32's branch
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if constexpr (kPair) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();  // the leader's barriers exist before the peer signals them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_pref[G];
@@ -288,25 +378,39 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   const int num_kb = (args.kdim + kElems - 1) / kElems;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (every CTA fills its own ring) ----------------
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
       bool aborted = false;
       uint32_t issued = 0, issued_ph = 0;  // per-stage bits: loaded at least once / its parity
-      for (int T = blockIdx.x; T < total && !aborted; T += gridDim.x) {
-        const TileCoord c = decode_tile(T, s_pref, s_off, G);
-        const int brow = c.g * args.n_out + c.n_tile * (kEpi == kEpiSwiglu ? BN / 2 : BN);
+      const CUtensorMap* mapB = (kEpi == kEpiSwiglu && kPair && rank == 1) ? &args.tmB1 : &args.tmB0;
+      for (int T = unit; T < total && !aborted; T += nunits) {
+        const TileCoord c = decode_tile<Gm::TILE_M>(T, s_pref, s_off, G);
+        const int arow = c.m_row0 + static_cast<int>(rank) * BM;
+        int brow;
+        if constexpr (kEpi == kEpiSwiglu)
+          brow = c.g * args.n_out + c.n_tile * (BN / 2);  // gate (and up) rows of 128 outputs
+        else
+          brow = c.g * args.n_out + c.n_tile * BN + static_cast<int>(rank) * Gm::B_ROWS;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(bar(kBarEmpty + s), ph ^ 1u, abort_flag)) { aborted = true; break; }
-          mbar_expect_tx(bar(kBarFull + s), STAGE_BYTES);
+          if (!mbar_wait(bar(Gm::kBarEmpty + s), ph ^ 1u, abort_flag)) { aborted = true; break; }
           const int kx = kb * kElems;
-          tma_load_2d(sA + s * A_BYTES, &args.tmA, kx, c.m_row0, bar(kBarFull + s));
-          if (kEpi == kEpiSwiglu) {
-            tma_load_2d(sB + s * B_BYTES, &args.tmB0, kx, brow, bar(kBarFull + s));
-            tma_load_2d(sB + s * B_BYTES + (BN / 2) * ROWB, &args.tmB1, kx, brow, bar(kBarFull + s));
+          if constexpr (kPair) {
+            const uint32_t full_leader = map_to_rank(bar(Gm::kBarFull + s), 0);
+            if (leader) mbar_expect_tx(bar(Gm::kBarFull + s), 2 * Gm::STAGE_BYTES);
+            tma_load_2d_pair(sA + s * A_BYTES, &args.tmA, kx, arow, full_leader);
+            tma_load_2d_pair(sB + s * Gm::B_BYTES, mapB, kx, brow, full_leader);
           } else {
-            tma_load_2d(sB + s * B_BYTES, &args.tmB0, kx, brow, bar(kBarFull + s));
+            mbar_expect_tx(bar(Gm::kBarFull + s), Gm::STAGE_BYTES);
+            tma_load_2d(sA + s * A_BYTES, &args.tmA, kx, arow, bar(Gm::kBarFull + s));
+            if (kEpi == kEpiSwiglu) {
+              tma_load_2d(sB + s * Gm::B_BYTES, &args.tmB0, kx, brow, bar(Gm::kBarFull + s));
+              tma_load_2d(sB + s * Gm::B_BYTES + (BN / 2) * ROWB, &args.tmB1, kx, brow,
+                          bar(Gm::kBarFull + s));
+            } else {
+              tma_load_2d(sB + s * Gm::B_BYTES, &args.tmB0, kx, brow, bar(Gm::kBarFull + s));
+            }
           }
           issued |= 1u << s;
           issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
@@ -316,63 +420,72 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       if (aborted) {
         set_status(args.status, kStatusTimeout);
         // let copies already in flight land before the CTA's memory is reused
-        for (int i = 0; i < STAGES; ++i)
-          if ((issued >> i) & 1u) mbar_wait_drain(bar(kBarFull + i), (issued_ph >> i) & 1u);
+        if (leader)
+          for (int i = 0; i < STAGES; ++i)
+            if ((issued >> i) & 1u) mbar_wait_drain(bar(Gm::kBarFull + i), (issued_ph >> i) & 1u);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc<kFp8>();
+    // ---------------- MMA issuer (the pair leader issues for both CTAs) ----------------
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = make_idesc_mode<kFp8, kPair>();
       int s = 0;
       uint32_t ph = 0;
       bool aborted = false;
       int i = 0;
-      for (int T = blockIdx.x; T < total; T += gridDim.x, ++i) {
+      for (int T = unit; T < total; T += nunits, ++i) {
         const int acc = i & 1;
         const uint32_t aph = (i >> 1) & 1;
-        if (!mbar_wait(bar(kBarTEmpty + acc), aph ^ 1u, abort_flag)) { aborted = true; break; }
+        if (!mbar_wait(bar(Gm::kBarTEmpty + acc), aph ^ 1u, abort_flag)) { aborted = true; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(bar(kBarFull + s), ph, abort_flag)) { aborted = true; break; }
+          if (!mbar_wait(bar(Gm::kBarFull + s), ph, abort_flag)) { aborted = true; break; }
           tc_fence_after();
-          const uint32_t a0 = sA + s * A_BYTES, b0 = sB + s * B_BYTES;
+          const uint32_t a0 = sA + s * A_BYTES, b0 = sB + s * Gm::B_BYTES;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma<kFp8>(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc,
-                         (kb | k) != 0 ? 1u : 0u);
-          tc_commit(bar(kBarEmpty + s));
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
+            if constexpr (kPair)
+              tc_mma_pair<kFp8>(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, accum);
+            else
+              tc_mma<kFp8>(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, accum);
+          }
+          if constexpr (kPair) tc_commit_pair_both(bar(Gm::kBarEmpty + s));
+          else tc_commit(bar(Gm::kBarEmpty + s));
           if (++s == STAGES) { s = 0; ph ^= 1u; }
         }
         if (aborted) break;
-        tc_commit(bar(kBarTFull + acc));
+        if constexpr (kPair) tc_commit_pair_both(bar(Gm::kBarTFull + acc));
+        else tc_commit(bar(Gm::kBarTFull + acc));
       }
       if (aborted) {
         set_status(args.status, kStatusTimeout);
-        tc_commit(bar(kBarDrain));  // arrives once every MMA issued so far has finished
-        mbar_wait_drain(bar(kBarDrain), 0);
+        // arrives once every MMA issued so far has finished
+        if constexpr (kPair) tc_commit_pair_self(bar(Gm::kBarDrain));
+        else tc_commit(bar(Gm::kBarDrain));
+        mbar_wait_drain(bar(Gm::kBarDrain), 0);
       }
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..5 of every CTA) ----------------
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const int row = q * 32 + lane;
+    const int row = static_cast<int>(rank) * BM + q * 32 + lane;  // row within the tile
     int i = 0;
-    for (int T = blockIdx.x; T < total; T += gridDim.x, ++i) {
+    for (int T = unit; T < total; T += nunits, ++i) {
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1;
       // every lane polls; lane 0's answer is taken by all (and converges the warp
       // before the .sync.aligned TMEM loads)
-      const bool ok = __shfl_sync(0xffffffffu, mbar_wait(bar(kBarTFull + acc), aph, abort_flag), 0);
+      const bool ok = __shfl_sync(0xffffffffu, mbar_wait(bar(Gm::kBarTFull + acc), aph, abort_flag), 0);
       if (!ok) {
         set_status(args.status, kStatusTimeout);
         break;
       }
       tc_fence_after();
-      const TileCoord c = decode_tile(T, s_pref, s_off, G);
+      const TileCoord c = decode_tile<Gm::TILE_M>(T, s_pref, s_off, G);
       const long long grow = static_cast<long long>(c.m_row0) + row;
       const bool valid = grow < s_off[c.g + 1] && grow < args.m_total && grow >= 0;
       const uint32_t tbase =
@@ -437,18 +550,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarTEmpty + acc));
+      if (lane == 0) {
+        if constexpr (kPair) mbar_arrive_cluster(map_to_rank(bar(Gm::kBarTEmpty + acc), 0));
+        else mbar_arrive(bar(Gm::kBarTEmpty + acc));
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();  // the peer is done with this CTA's memory and TMEM
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(kTmemCols)
-                 : "memory");
+    if constexpr (kPair)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(kTmemCols)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(kTmemCols)
+                   : "memory");
   }
 }
 
@@ -472,17 +594,45 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <bool kFp8, int kEpi>
-cudaError_t launch_t(const TcGemmArgs& args, int grid, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kFp8, kEpi>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
+template <bool kFp8, int kEpi, bool kPair>
+cudaError_t launch_t(const TcGemmArgs& args, long long max_units, cudaStream_t stream) {
+  using Gm = Geo<kPair>;
+  auto kern = gemm_tc_kernel<kFp8, kEpi, kPair>;
+  static int configured[64] = {0};
+  static int max_clusters[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Gm::kSmemBytes;
+  cfg.stream = stream;
+  if constexpr (kPair) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
   }
-  gemm_tc_kernel<kFp8, kEpi><<<grid, kThreads, kSmemBytes, stream>>>(args);
-  return cudaGetLastError();
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Gm::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if constexpr (kPair) {
+      int n = 0;
+      cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
+      e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+      if (e != cudaSuccess) return e;
+      max_clusters[dev] = n > 0 ? n : 1;
+    }
+    configured[dev] = 1;
+  }
+  long long units = kPair ? max_clusters[dev] : device_sm_count();
+  if (max_units < units) units = max_units;
+  cfg.gridDim = dim3(static_cast<unsigned>((kPair ? 2 : 1) * units), 1, 1);
+  return cudaLaunchKernelEx(&cfg, kern, args);
 }
 
 }  // namespace
@@ -504,18 +654,24 @@ bool encode_kmajor_map(CUtensorMap* map, const void* base, int elem_bytes, long 
 }
 
 cudaError_t launch_gemm_tc(const TcGemmArgs& args, int dtype, int epilogue, int rows_upper,
-                           cudaStream_t stream) {
+                           bool pair, cudaStream_t stream) {
   if (args.groups < 1 || args.groups > kMaxGroups) return cudaErrorInvalidValue;
-  long long max_tiles = (static_cast<long long>(rows_upper) / BM + args.groups) * args.n_tiles;
-  if (max_tiles <= 0) return cudaSuccess;
-  int grid = static_cast<int>(max_tiles < device_sm_count() ? max_tiles : device_sm_count());
+  const int tile_m = pair ? 2 * BM : BM;
+  const long long max_units =
+      (static_cast<long long>(rows_upper) / tile_m + args.groups) * args.n_tiles;
+  if (max_units <= 0) return cudaSuccess;
   const bool fp8 = dtype == kE4M3;
-  if (fp8) {
-    if (epilogue == kEpiSwiglu) return launch_t<true, kEpiSwiglu>(args, grid, stream);
-    return launch_t<true, kEpiStore>(args, grid, stream);
+  const bool sw = epilogue == kEpiSwiglu;
+  if (pair) {
+    if (fp8) return sw ? launch_t<true, kEpiSwiglu, true>(args, max_units, stream)
+                       : launch_t<true, kEpiStore, true>(args, max_units, stream);
+    return sw ? launch_t<false, kEpiSwiglu, true>(args, max_units, stream)
+              : launch_t<false, kEpiStore, true>(args, max_units, stream);
   }
-  if (epilogue == kEpiSwiglu) return launch_t<false, kEpiSwiglu>(args, grid, stream);
-  return launch_t<false, kEpiStore>(args, grid, stream);
+  if (fp8) return sw ? launch_t<true, kEpiSwiglu, false>(args, max_units, stream)
+                     : launch_t<true, kEpiStore, false>(args, max_units, stream);
+  return sw ? launch_t<false, kEpiSwiglu, false>(args, max_units, stream)
+            : launch_t<false, kEpiStore, false>(args, max_units, stream);
 }
 
 int device_sm_count() {

@@ -25,10 +25,15 @@ cudaError_t launch_router(const void* x, int x_dtype, const float* w_r, const fl
 constexpr int kPermuteChunk = 32;  // tokens per chunk of the stable counting pass
 inline int permute_chunks(int N) { return (N + kPermuteChunk - 1) / kPermuteChunk; }
 
+// Writes each (t, j)'s rank within its 32-token chunk to local_rank (the
+// perm_pos buffer; the gather turns it into the final position) and the
+// chunk's expert histogram to chunk_counts.
 cudaError_t launch_permute_count(const int32_t* ids, int N, int K, int E, int32_t* chunk_counts,
-                                 int* status, cudaStream_t stream);
+                                 int32_t* local_rank, int* status, cudaStream_t stream);
 cudaError_t launch_permute_scan(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
                                 int32_t* offsets, cudaStream_t stream);
+// pos holds the ranks from launch_permute_count on entry, the final
+// positions on exit.
 cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* ids, int N, int K,
                                   int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
                                   void* x_perm, int* status, cudaStream_t stream);
@@ -71,9 +76,11 @@ bool encode_kmajor_map(CUtensorMap* map, const void* base, int elem_bytes, long 
                        long long kdim, int box_rows);
 
 // dtype kBF16 or kE4M3.  offsets on device; rows_upper = upper bound of the
-// number of A rows (to size the grid).
+// number of A rows (to size the grid).  pair: 256-row tiles on CTA pairs
+// (tcgen05 cta_group::2); the B maps then have 128-row boxes for the store
+// epilogue (each CTA loads half of the 256 weight rows).
 cudaError_t launch_gemm_tc(const TcGemmArgs& args, int dtype, int epilogue, int rows_upper,
-                           cudaStream_t stream);
+                           bool pair, cudaStream_t stream);
 constexpr int kTcBlockM = 128;
 constexpr int kTcBlockN = 256;  // accumulator columns; SwiGLU: 128 gate + 128 up
 

@@ -7,13 +7,15 @@
 // Stable order: within expert e the rows appear in (token, slot) order, so
 //   pos[t,j] = offsets[e] + #{(t',j') before (t,j) with ids[t',j'] = e}.
 // Tokens are cut into chunks of kPermuteChunk (32).  Three launches:
-//   1. count:  per-chunk expert histogram in shared memory -> chunk_counts
+//   1. rank:   one warp per chunk ranks the chunk's (t, j) pairs with
+//              shuffles (no atomics in the ranks, so the order is fixed),
+//              writes each pair's rank within its chunk (into perm_pos) and
+//              the chunk's expert histogram (chunk_counts)
 //   2. scan:   one CTA turns chunk_counts into per-(chunk, expert) bases
 //              (offsets[e] + rows of e in earlier chunks), counts, offsets
-//   3. gather: one warp ranks the chunk's (t, j) pairs with shuffles (no
-//              atomics, so the order is fixed), then all warps copy each
-//              token row once from HBM into its K destination rows with
-//              16-byte vector loads/stores.
+//   3. gather: one warp per token turns its ranks into final positions and
+//              copies the token row once from HBM into its K destination
+//              rows with 16-byte vector loads/stores.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -22,25 +24,60 @@ namespace {
 
 constexpr int CH = kPermuteChunk;
 
+// One warp per chunk of 32 tokens; lane = token.
+template <int KMAX>
 __global__ void __launch_bounds__(128)
-permute_count_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
-                     int32_t* __restrict__ chunk_counts, int* status) {
-  __shared__ int hist[256];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
-  __syncthreads();
-  const long long base = (long long)blockIdx.x * CH * K;
-  const long long end = min((long long)N * K, base + (long long)CH * K);
-  for (long long i = base + threadIdx.x; i < end; i += blockDim.x) {
-    int e = ids[i];
-    if (e < 0 || e >= E) {
-      set_status(status, kStatusBadIndex);
-      continue;
+permute_rank_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
+                    int32_t* __restrict__ chunk_counts, int32_t* __restrict__ local_rank,
+                    int* status) {
+  __shared__ int hist[4][256];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = blockIdx.x * 4 + warp;
+  const int nchunks = (N + CH - 1) / CH;
+  if (c >= nchunks) return;  // whole warp
+  for (int e = lane; e < E; e += 32) hist[warp][e] = 0;
+  __syncwarp();
+  const int t = c * CH + lane;
+  int my[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    my[j] = -1;
+    if (j < K && t < N) {
+      const int e = ids[(long long)t * K + j];
+      if (e >= 0 && e < E) my[j] = e;
+      else set_status(status, kStatusBadIndex);
     }
-    atomicAdd(&hist[e], 1);  // integer counts: order-independent
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    chunk_counts[(long long)blockIdx.x * E + e] = hist[e];
+  // rank of (t, j): earlier slots of t with the same expert ...
+  int rank[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    rank[j] = 0;
+#pragma unroll
+    for (int jj = 0; jj < KMAX; ++jj)
+      if (jj < j && my[jj] == my[j]) rank[j]++;
+  }
+  // ... plus every slot of the earlier tokens of this chunk with that expert
+#pragma unroll
+  for (int jj = 0; jj < KMAX; ++jj) {
+    if (jj >= K) break;
+    for (int sl = 0; sl < 31; ++sl) {
+      const int v = __shfl_sync(0xffffffffu, my[jj], sl);
+      if (sl < lane) {
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+          if (v == my[j] && v >= 0) rank[j]++;
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j >= K) break;
+    if (t < N) local_rank[(long long)t * K + j] = my[j] >= 0 ? rank[j] : -1;
+    if (my[j] >= 0) atomicAdd(&hist[warp][my[j]], 1);  // integer counts: order-independent
+  }
+  __syncwarp();
+  for (int e = lane; e < E; e += 32) chunk_counts[(long long)c * E + e] = hist[warp][e];
 }
 
 // One CTA of 1024 threads.  Thread (e, s) owns expert e and a contiguous
@@ -107,95 +144,62 @@ permute_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
   }
 }
 
+// One warp per token: final positions from the chunk bases and the ranks,
+// then one read of the token row and K writes.
 template <int KMAX>
 __global__ void __launch_bounds__(256)
 permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* __restrict__ ids,
                       int N, int K, int E, const int32_t* __restrict__ chunk_base,
-                      int32_t* __restrict__ pos, int32_t* __restrict__ src, uint4* __restrict__ x_perm,
-                      int* status) {
-  __shared__ int spos[CH][KMAX];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int c = blockIdx.x;
-  if (warp == 0) {
-    const int t = c * CH + lane;
-    int my[KMAX];
+                      int32_t* __restrict__ pos, int32_t* __restrict__ src, uint4* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= N) return;
+  int mine = -1;
+  if (lane < K) {
+    const long long i = (long long)t * K + lane;
+    const int e = ids[i];
+    const int r = pos[i];  // rank within the chunk (written by the rank pass)
+    if (r >= 0 && e >= 0 && e < E) {
+      mine = chunk_base[(long long)(t / CH) * E + e] + r;
+      src[mine] = t;
+    }
+    pos[i] = mine;
+  }
+  int p[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) p[j] = __shfl_sync(0xffffffffu, mine, j);
+  const uint4* srow = x + (long long)t * row_vecs;
+  int v = lane;
+  for (; v + 96 < row_vecs; v += 128) {
+    const uint4 a0 = srow[v], a1 = srow[v + 32], a2 = srow[v + 64], a3 = srow[v + 96];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
-      my[j] = -1;
-      if (j < K && t < N) {
-        int e = ids[(long long)t * K + j];
-        if (e >= 0 && e < E) my[j] = e;  // bad ids were flagged by the count pass
-      }
-    }
-    // rank of (t, j): earlier slots of t with the same expert ...
-    int rank[KMAX];
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      rank[j] = 0;
-#pragma unroll
-      for (int jj = 0; jj < KMAX; ++jj)
-        if (jj < j && my[jj] == my[j]) rank[j]++;
-    }
-    // ... plus every slot of the earlier tokens of this chunk with that expert
-#pragma unroll
-    for (int jj = 0; jj < KMAX; ++jj) {
-      if (jj >= K) break;
-      for (int sl = 0; sl < 31; ++sl) {
-        int v = __shfl_sync(0xffffffffu, my[jj], sl);
-        if (sl < lane) {
-#pragma unroll
-          for (int j = 0; j < KMAX; ++j)
-            if (v == my[j] && v >= 0) rank[j]++;
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      if (j >= K) break;
-      int p = -1;
-      if (my[j] >= 0) {
-        p = chunk_base[(long long)c * E + my[j]] + rank[j];
-        src[p] = t;
-      }
-      if (t < N) pos[(long long)t * K + j] = p;
-      spos[lane][j] = p;
+      if (j >= K || p[j] < 0) continue;
+      uint4* drow = x_perm + (long long)p[j] * row_vecs;
+      drow[v] = a0; drow[v + 32] = a1; drow[v + 64] = a2; drow[v + 96] = a3;
     }
   }
-  __syncthreads();
-  // copy: each warp owns tokens warp, warp+8, ...; a row is read once
-  for (int tt = warp; tt < CH; tt += 8) {
-    const int t = c * CH + tt;
-    if (t >= N) break;
-    const uint4* srow = x + (long long)t * row_vecs;
-    int p[KMAX];
+  for (; v < row_vecs; v += 32) {
+    const uint4 a0 = srow[v];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) p[j] = j < K ? spos[tt][j] : -1;
-    int v = lane;
-    for (; v + 96 < row_vecs; v += 128) {
-      uint4 a0 = srow[v], a1 = srow[v + 32], a2 = srow[v + 64], a3 = srow[v + 96];
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        if (p[j] < 0) continue;
-        uint4* drow = x_perm + (long long)p[j] * row_vecs;
-        drow[v] = a0; drow[v + 32] = a1; drow[v + 64] = a2; drow[v + 96] = a3;
-      }
-    }
-    for (; v < row_vecs; v += 32) {
-      uint4 a0 = srow[v];
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (p[j] >= 0) x_perm[(long long)p[j] * row_vecs + v] = a0;
-    }
+    for (int j = 0; j < KMAX; ++j)
+      if (j < K && p[j] >= 0) x_perm[(long long)p[j] * row_vecs + v] = a0;
   }
 }
 
 }  // namespace
 
 cudaError_t launch_permute_count(const int32_t* ids, int N, int K, int E, int32_t* chunk_counts,
-                                 int* status, cudaStream_t stream) {
-  int nchunks = permute_chunks(N);
+                                 int32_t* local_rank, int* status, cudaStream_t stream) {
+  const int nchunks = permute_chunks(N);
   if (nchunks == 0) return cudaSuccess;
-  permute_count_kernel<<<nchunks, 128, 0, stream>>>(ids, N, K, E, chunk_counts, status);
+  const int grid = (nchunks + 3) / 4;
+  if (K <= 2)
+    permute_rank_kernel<2><<<grid, 128, 0, stream>>>(ids, N, K, E, chunk_counts, local_rank, status);
+  else if (K <= 4)
+    permute_rank_kernel<4><<<grid, 128, 0, stream>>>(ids, N, K, E, chunk_counts, local_rank, status);
+  else
+    permute_rank_kernel<8><<<grid, 128, 0, stream>>>(ids, N, K, E, chunk_counts, local_rank, status);
   return cudaGetLastError();
 }
 
@@ -208,20 +212,21 @@ cudaError_t launch_permute_scan(int32_t* chunk_counts, int nchunks, int E, int32
 cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* ids, int N, int K,
                                   int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
                                   void* x_perm, int* status, cudaStream_t stream) {
-  int nchunks = permute_chunks(N);
-  if (nchunks == 0) return cudaSuccess;
-  int row_vecs = row_bytes / 16;
+  (void)status;  // bad ids were recorded by the rank pass
+  if (N == 0) return cudaSuccess;
+  const int row_vecs = row_bytes / 16;
+  const int grid = (N + 7) / 8;
   auto xv = static_cast<const uint4*>(x);
   auto xp = static_cast<uint4*>(x_perm);
   if (K <= 2)
-    permute_gather_kernel<2><<<nchunks, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base,
-                                                          pos, src, xp, status);
+    permute_gather_kernel<2><<<grid, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base, pos,
+                                                       src, xp);
   else if (K <= 4)
-    permute_gather_kernel<4><<<nchunks, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base,
-                                                          pos, src, xp, status);
+    permute_gather_kernel<4><<<grid, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base, pos,
+                                                       src, xp);
   else
-    permute_gather_kernel<8><<<nchunks, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base,
-                                                          pos, src, xp, status);
+    permute_gather_kernel<8><<<grid, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base, pos,
+                                                       src, xp);
   return cudaGetLastError();
 }
 

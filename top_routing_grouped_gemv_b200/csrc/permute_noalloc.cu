@@ -16,7 +16,7 @@
 
 #include <mutex>
 
-#include "../../include/moe.h"
+#include "moe.h"
 #include "kernels.h"
 
 namespace {
@@ -68,7 +68,7 @@ extern "C" moe_status moe_permute_noalloc(moe_plan plan, const void* x, const in
   if (st != MOE_OK) return st;
   cudaStream_t s = stream;
   int* status = device_status_or_null;
-  if (moe::launch_permute_count(topk_ids, N, K, E, scratch, status, s) != cudaSuccess ||
+  if (moe::launch_permute_count(topk_ids, N, K, E, scratch, perm_pos, status, s) != cudaSuccess ||
       moe::launch_permute_scan(scratch, nchunks, E, counts, offsets, s) != cudaSuccess ||
       moe::launch_permute_gather(x, row_bytes, topk_ids, N, K, E, scratch, perm_pos, perm_src,
                                  x_perm, status, s) != cudaSuccess)

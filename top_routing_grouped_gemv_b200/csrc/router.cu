@@ -150,152 +150,189 @@ router_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
   }
 }
 
-// Small d*E (d*E <= 256 threads * 64 weights): every thread keeps the
-// router weights of its k-slice [tid*KPT, tid*KPT+KPT) for all experts in
-// registers, so the weights are read from memory once per CTA.  A CTA takes
-// TB = 32/ET tokens at a time: each thread forms its partial logits for
-// them (k ascending inside the slice), a warp reduce-scatter (31 shuffles)
-// leaves lane l with the warp's sum of value l = (token l/ET, expert l%ET),
-// and the eight warp sums are added in warp order.  Warp j then picks the
-// top-K of token j.
-template <int V>
-__device__ __forceinline__ float warp_reduce_scatter(float (&v)[V], int lane) {
-  static_assert(V == 32, "one value per lane after the reduction");
-#pragma unroll
-  for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < n / 2; ++i) {
-      const float send = upper ? v[i] : v[i + n / 2];
-      const float keep = upper ? v[i + n / 2] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-  return v[0];
-}
-
-template <typename TX, int ET, int KPT>
-__global__ void __launch_bounds__(256)
-router_regw_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
+// Small E (<= 32) with W_r fitting in shared memory: the whole router
+// weight is staged once per CTA; warps then stream tokens.  Lane l of a warp
+// reads 16-byte vectors v = l, l+32, ... of a token row (VEC consecutive k)
+// and accumulates all E logits of TPW tokens in registers (k ascending
+// within each vector), so every weight read from shared memory feeds TPW
+// tokens.  The E partial sums are then added across the 32 lanes by an XOR
+// butterfly (fixed order), after which lane e holds logit e and the top-K is
+// taken by K rounds of the warp-shuffle argmax.
+//
+// Shared layout: block m holds the VEC rows k = m*VEC .. m*VEC+VEC-1 as
+// [e][VEC] floats, i.e. 16-byte chunks c = e*VEC/4 + h.  Chunk c of block m
+// sits at position c ^ (m & 7): the lanes of a warp read consecutive blocks,
+// so the XOR spreads one logical chunk over 8 bank groups (conflict-free
+// 128-bit reads).
+template <typename TX, int E_T, int TPW>
+__global__ void __launch_bounds__(256, E_T <= 8 ? 2 : 1)
+router_smem_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
                    const float* __restrict__ bias, int N, int d, int E, int K,
                    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ margin) {
-  constexpr int TB = 32 / ET;  // tokens per pass
-  __shared__ float red[8][32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int k0 = tid * KPT;
-  float w[KPT][ET];
-#pragma unroll
-  for (int i = 0; i < KPT; ++i)
-#pragma unroll
-    for (int e = 0; e < ET; ++e)
-      w[i][e] = (k0 + i < d && e < E) ? w_r[(long long)(k0 + i) * E + e] : 0.f;
+  constexpr int VEC = 16 / sizeof(TX);        // k per 16-byte vector of x
+  constexpr int CPB = E_T * VEC / 4;          // 16-byte chunks per block
+  extern __shared__ float4 wsm[];
+  const int nvec = d / VEC;                   // d is a multiple of VEC
+  // stage W_r: block m, expert e, row i -> chunk (e*VEC + i)/4 ^ (m & 7), lane (i % 4)
+  float* wf = reinterpret_cast<float*>(wsm);
+  auto put = [&](int k, int e, float v) {
+    const int m = k / VEC, i = k % VEC;
+    const int c = (e * VEC + i) >> 2;
+    wf[((long long)m * CPB + (c ^ (m & 7))) * 4 + (i & 3)] = v;
+  };
+  if (E == E_T && (E & 3) == 0) {  // whole rows, 16-byte loads
+    const float4* w4 = reinterpret_cast<const float4*>(w_r);
+    for (int idx = threadIdx.x; idx < d * E / 4; idx += blockDim.x) {
+      const float4 v = w4[idx];
+      const int k = idx * 4 / E, e = idx * 4 % E;
+      put(k, e, v.x); put(k, e + 1, v.y); put(k, e + 2, v.z); put(k, e + 3, v.w);
+    }
+  } else {
+    for (int idx = threadIdx.x; idx < d * E_T; idx += blockDim.x) {
+      const int k = idx / E_T, e = idx % E_T;
+      put(k, e, e < E ? w_r[(long long)k * E + e] : 0.f);
+    }
+  }
+  __syncthreads();
 
-  for (int t0 = blockIdx.x * TB; t0 < N; t0 += gridDim.x * TB) {
-    float part[32];
+  const int lane = threadIdx.x & 31;
+  const int gwarp = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  for (int t0 = gwarp * TPW; t0 < N; t0 += nwarps * TPW) {
+    float acc[TPW][E_T];
 #pragma unroll
-    for (int j = 0; j < TB; ++j) {
-      float xv[KPT];
-      const int t = t0 + j;
+    for (int j = 0; j < TPW; ++j)
 #pragma unroll
-      for (int i = 0; i < KPT; ++i)
-        xv[i] = (t < N && k0 + i < d) ? to_f32(x[(long long)t * d + k0 + i]) : 0.f;
+      for (int e = 0; e < E_T; ++e) acc[j][e] = 0.f;
+    // four vectors per token in flight per lane before the FMAs
+    for (int mb = lane; mb < nvec; mb += 128) {
+      uint4 u[4][TPW];
 #pragma unroll
-      for (int e = 0; e < ET; ++e) {
-        float a = 0.f;
+      for (int q = 0; q < 4; ++q)
 #pragma unroll
-        for (int i = 0; i < KPT; ++i) a = fmaf(xv[i], w[i][e], a);
-        part[j * ET + e] = a;
+        for (int j = 0; j < TPW; ++j) {
+          const int m = mb + 32 * q;
+          const int t = min(t0 + j, N - 1);
+          u[q][j] = m < nvec ? reinterpret_cast<const uint4*>(x + (long long)t * d)[m]
+                             : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int m = mb + 32 * q;
+        if (m >= nvec) break;
+        float xv[TPW][VEC];
+#pragma unroll
+        for (int j = 0; j < TPW; ++j) {
+          if constexpr (VEC == 8) {
+            xv[j][0] = bf16lo(u[q][j].x); xv[j][1] = bf16hi(u[q][j].x);
+            xv[j][2] = bf16lo(u[q][j].y); xv[j][3] = bf16hi(u[q][j].y);
+            xv[j][4] = bf16lo(u[q][j].z); xv[j][5] = bf16hi(u[q][j].z);
+            xv[j][6] = bf16lo(u[q][j].w); xv[j][7] = bf16hi(u[q][j].w);
+          } else {
+            xv[j][0] = __uint_as_float(u[q][j].x); xv[j][1] = __uint_as_float(u[q][j].y);
+            xv[j][2] = __uint_as_float(u[q][j].z); xv[j][3] = __uint_as_float(u[q][j].w);
+          }
+        }
+        const float4* blk = wsm + (long long)m * CPB;
+#pragma unroll
+        for (int e = 0; e < E_T; ++e) {
+#pragma unroll
+          for (int h = 0; h < VEC / 4; ++h) {
+            const float4 w4 = blk[(e * (VEC / 4) + h) ^ (m & 7)];
+            const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+              for (int j = 0; j < TPW; ++j) acc[j][e] = fmaf(xv[j][h * 4 + i], wv[i], acc[j][e]);
+          }
+        }
       }
     }
-    red[warp][lane] = warp_reduce_scatter<32>(part, lane);
-    __syncthreads();
-    if (warp < TB) {
-      const int t = t0 + warp;
+#pragma unroll
+    for (int j = 0; j < TPW; ++j)
+#pragma unroll
+      for (int e = 0; e < E_T; ++e)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[j][e] += __shfl_xor_sync(0xffffffffu, acc[j][e], o);
+
+#pragma unroll
+    for (int j = 0; j < TPW; ++j) {
+      const int t = t0 + j;
+      if (t >= N) break;  // warp-uniform
       float v[1];
       bool avail[1];
       v[0] = 0.f;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v[0] += red[q][warp * ET + (lane % ET)];
+      for (int e = 0; e < E_T; ++e)
+        if (e == lane) v[0] = acc[j][e];
       avail[0] = lane < E;
       if (avail[0] && bias != nullptr) v[0] += bias[lane];
-      if (t < N) {
-        float sel_v[8];
-        int sel_e[8];
+      float sel_v[8];
+      int sel_e[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j >= K) break;
-          warp_argmax<1>(v, avail, lane, sel_v[j], sel_e[j]);
-          if (lane == sel_e[j]) avail[0] = false;
-        }
-        float next_v = 0.f;
-        if (K < E) {
-          int next_e;
-          warp_argmax<1>(v, avail, lane, next_v, next_e);
-        }
-        float z = 0.f, my_g = 0.f;
-        int my_e = 0;
+      for (int q = 0; q < 8; ++q) {
+        if (q >= K) break;
+        warp_argmax<1>(v, avail, lane, sel_v[q], sel_e[q]);
+        if (lane == sel_e[q]) avail[0] = false;
+      }
+      float next_v = 0.f;
+      if (K < E) {
+        int next_e;
+        warp_argmax<1>(v, avail, lane, next_v, next_e);
+      }
+      float z = 0.f, my_g = 0.f;
+      int my_e = 0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j < K) {
-            const float p = expf(sel_v[j] - sel_v[0]);
-            z += p;
-            if (j == lane) { my_g = p; my_e = sel_e[j]; }
-          }
-        }
-        if (lane < K) {
-          ids[(long long)t * K + lane] = my_e;
-          gates[(long long)t * K + lane] = my_g / z;
-        }
-        if (margin != nullptr && lane == 0) {
-          float kth = sel_v[0];
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (j == K - 1) kth = sel_v[j];
-          margin[t] = (K == E) ? __int_as_float(0x7f800000) : kth - next_v;
+      for (int q = 0; q < 8; ++q) {
+        if (q < K) {
+          const float p = expf(sel_v[q] - sel_v[0]);
+          z += p;
+          if (q == lane) { my_g = p; my_e = sel_e[q]; }
         }
       }
+      if (lane < K) {
+        ids[(long long)t * K + lane] = my_e;
+        gates[(long long)t * K + lane] = my_g / z;
+      }
+      if (margin != nullptr && lane == 0) {
+        float kth = sel_v[0];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q == K - 1) kth = sel_v[q];
+        margin[t] = (K == E) ? __int_as_float(0x7f800000) : kth - next_v;
+      }
     }
-    __syncthreads();
   }
 }
 
-template <typename TX, int ET, int KPT>
-void launch_regw_kpt(const TX* x, const float* w_r, const float* bias, int N, int d, int E, int K,
-                     int32_t* ids, float* gates, float* margin, int grid, cudaStream_t stream) {
-  router_regw_kernel<TX, ET, KPT><<<grid, 256, 0, stream>>>(x, w_r, bias, N, d, E, K, ids, gates,
-                                                            margin);
-}
+constexpr size_t kRouterSmemMax = 160 * 1024;
 
-// Picks the k-slice per thread (KPT = 1, 2, 4, 8: d <= 256*KPT) with at most
-// 64 weights per thread; false if d*E is too large for this kernel.
-template <typename TX, int ET>
-bool launch_regw(const TX* x, const float* w_r, const float* bias, int N, int d, int E, int K,
+template <typename TX, int E_T>
+bool launch_smem(const TX* x, const float* w_r, const float* bias, int N, int d, int E, int K,
                  int32_t* ids, float* gates, float* margin, cudaStream_t stream) {
-  constexpr int TB = 32 / ET;
-  const int grid = min((N + TB - 1) / TB, 2 * device_sm_count());
-  if (d <= 256) {
-    launch_regw_kpt<TX, ET, 1>(x, w_r, bias, N, d, E, K, ids, gates, margin, grid, stream);
-    return true;
+  constexpr int VEC = 16 / sizeof(TX);
+  const size_t smem = static_cast<size_t>(d) * E_T * sizeof(float);
+  if (d % VEC != 0 || smem > kRouterSmemMax) return false;
+  constexpr int TPW = E_T <= 8 ? 2 : 1;
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    if (cudaFuncSetAttribute(router_smem_kernel<TX, E_T, TPW>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kRouterSmemMax)) != cudaSuccess)
+      return false;
+    configured[dev] = true;
   }
-  if constexpr (2 * ET <= 64) {
-    if (d <= 512) {
-      launch_regw_kpt<TX, ET, 2>(x, w_r, bias, N, d, E, K, ids, gates, margin, grid, stream);
-      return true;
-    }
-  }
-  if constexpr (4 * ET <= 64) {
-    if (d <= 1024) {
-      launch_regw_kpt<TX, ET, 4>(x, w_r, bias, N, d, E, K, ids, gates, margin, grid, stream);
-      return true;
-    }
-  }
-  if constexpr (8 * ET <= 64) {
-    if (d <= 2048) {
-      launch_regw_kpt<TX, ET, 8>(x, w_r, bias, N, d, E, K, ids, gates, margin, grid, stream);
-      return true;
-    }
-  }
-  return false;
+  // up to two CTAs per SM (shared memory permitting): the weights are staged
+  // once per CTA, then every warp streams tokens
+  const int per_sm = (E_T <= 8 && smem <= 100 * 1024) ? 2 : 1;
+  const long long need = (static_cast<long long>(N) + 8 * TPW - 1) / (8 * TPW);
+  const long long cap = static_cast<long long>(per_sm) * device_sm_count();
+  const int grid = static_cast<int>(need < cap ? need : cap);
+  router_smem_kernel<TX, E_T, TPW><<<grid, 256, smem, stream>>>(x, w_r, bias, N, d, E, K, ids,
+                                                                gates, margin);
+  return true;
 }
 
 template <typename TX, int EPL>
@@ -319,11 +356,11 @@ cudaError_t launch_epl(const TX* x, const float* w_r, const float* bias, int N, 
 template <typename TX>
 cudaError_t launch_t(const TX* x, const float* w_r, const float* bias, int N, int d, int E, int K,
                      int32_t* ids, float* gates, float* margin, cudaStream_t stream) {
-  if (E <= 8 && launch_regw<TX, 8>(x, w_r, bias, N, d, E, K, ids, gates, margin, stream))
+  if (E <= 8 && launch_smem<TX, 8>(x, w_r, bias, N, d, E, K, ids, gates, margin, stream))
     return cudaGetLastError();
-  if (E <= 16 && launch_regw<TX, 16>(x, w_r, bias, N, d, E, K, ids, gates, margin, stream))
+  if (E <= 16 && launch_smem<TX, 16>(x, w_r, bias, N, d, E, K, ids, gates, margin, stream))
     return cudaGetLastError();
-  if (E <= 32 && launch_regw<TX, 32>(x, w_r, bias, N, d, E, K, ids, gates, margin, stream))
+  if (E <= 32 && launch_smem<TX, 32>(x, w_r, bias, N, d, E, K, ids, gates, margin, stream))
     return cudaGetLastError();
   if (E <= 32) return launch_epl<TX, 1>(x, w_r, bias, N, d, E, K, ids, gates, margin, stream);
   if (E <= 64) return launch_epl<TX, 2>(x, w_r, bias, N, d, E, K, ids, gates, margin, stream);
