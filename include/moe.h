@@ -137,12 +137,16 @@ moe_status moe_workspace_init(moe_plan plan, void* ws, size_t ws_bytes, moe_stre
 /* ---- phase 2: execute --------------------------------------------------- */
 
 /* Router (page 1 section 1.1; zyxy MoE expert-selection section).  For each
- * token t: l[e] = sum_k x[t,k] * w_r[k,e] (+ router_bias[e]) in fp32; keep
- * the K largest (descending, equal logits -> lower expert index); gates =
- * softmax over the kept K only.  margin_or_null (N) receives l_(K) - l_(K+1)
- * (+inf when K == E).  x dtype fp32 or bf16.  Needs plan weights.w_r. */
+ * token t: l[e] = sum_k x[t,k] * w_r[k,e] (+ router_bias[e]) with fp32
+ * accuracy; keep the K largest (descending, equal logits -> lower expert
+ * index); gates = softmax over the kept K only.  margin_or_null (N)
+ * receives l_(K) - l_(K+1) (+inf when K == E).  x dtype fp32 or bf16.
+ * Needs plan weights.w_r.  bf16 layers with more than 32 experts compute the
+ * logits on the tensor cores from an exact three-part bf16 split of w_r,
+ * written to workspace scratch on every call (so w_r may change between
+ * calls). */
 moe_status moe_router_topk(moe_plan plan, const void* x, int32_t* topk_ids, float* topk_gates,
-                           float* margin_or_null, moe_stream_t stream);
+                           float* margin_or_null, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Permute / dispatch (page 1 section 1.2 token dispatch, local form; Ascend
  * page sendCounts).  counts[e] = #{(t,j): ids[t,j] = e}; offsets = exclusive

@@ -56,7 +56,7 @@ def run_routed_layer(cfg: synth.MoEConfig, n_tok_sample: int):
     # routing, full
     ids = torch.empty(c.N, c.K, dtype=torch.int32, device="cuda")
     gates = torch.empty(c.N, c.K, dtype=torch.float32, device="cuda")
-    plan.router_topk(x, ids, gates)
+    plan.router_topk(x, ids, gates, ws)
     rid, rg, _, logits = oracle.router(inp.x, dt, inp.w_r, inp.bias, c.K, want_logits=True)
     ids_g = ids.cpu().numpy()
     ties, diff = check_routing(ids_g, gates.cpu().double().numpy(), logits, rid, rg)

@@ -32,11 +32,16 @@ SMALL = {
                                     shared=(512, 384)),
     "e4m3_gmm_ragged": synth.small_variant(synth.FP8_GMM, N=45, d=256, E=40, K=8, F=96,
                                            shared=(256, 136)),
-    # >= 256 routed rows per expert on average: 256-row tiles on CTA pairs
+    # > 32 experts with bf16 tokens: router logits on the tensor cores
+    "bf16_tc_router_e64": synth.small_variant(synth.BF16_DECODE, N=200, d=512, E=64, K=8, F=128),
+    "bf16_tc_router_e100_k3": synth.MoEConfig("tc_e100", "bf16", 333, 256, 100, 3, 128, "swiglu",
+                                              zipf_bias=1.2),
+    "bf16_tc_router_e256_k1": synth.MoEConfig("tc_e256", "bf16", 130, 128, 256, 1, 64, "swiglu"),
+    # >= 512 routed rows per expert on average: 256-row tiles on CTA pairs
     "bf16_pair": synth.small_variant(synth.BF16_PREFILL, N=1024, d=256, E=4, K=2, F=384),
-    "bf16_pair_ragged": synth.small_variant(synth.BF16_PREFILL, N=700, d=320, E=4, K=2, F=200),
-    "bf16_pair_zipf": synth.small_variant(synth.BF16_FINEGRAINED, N=1100, d=256, E=8, K=2, F=256),
-    "e4m3_pair": synth.small_variant(synth.FP8_GMM, N=600, d=256, E=4, K=2, F=392,
+    "bf16_pair_ragged": synth.small_variant(synth.BF16_PREFILL, N=1300, d=320, E=4, K=2, F=200),
+    "bf16_pair_zipf": synth.small_variant(synth.BF16_FINEGRAINED, N=2100, d=256, E=8, K=2, F=256),
+    "e4m3_pair": synth.small_variant(synth.FP8_GMM, N=1100, d=256, E=4, K=2, F=392,
                                      shared=(256, 392)),
 }
 
@@ -80,7 +85,8 @@ def test_router_parity(name):
     ids = torch.empty(c.N, c.K, dtype=torch.int32, device="cuda")
     gates = torch.empty(c.N, c.K, dtype=torch.float32, device="cuda")
     margin = torch.empty(c.N, dtype=torch.float32, device="cuda")
-    plan.router_topk(x, ids, gates, margin)
+    ws = plan.new_workspace()
+    plan.router_topk(x, ids, gates, ws, margin)
     torch.cuda.synchronize()
     rid, rg, logits = ref_routing(inp)
     ties, diff = check_routing(ids.cpu().numpy(), gates.cpu().double().numpy(), logits, rid, rg)
@@ -201,7 +207,7 @@ def test_forward_end_to_end(name):
         # exclude near-tie tokens whose routing differs (their y is a different sum)
         ids = torch.empty(c.N, c.K, dtype=torch.int32, device="cuda")
         gates = torch.empty(c.N, c.K, dtype=torch.float32, device="cuda")
-        plan.router_topk(x, ids, gates)
+        plan.router_topk(x, ids, gates, ws)
         rid, rg, logits = ref_routing(inp)
         ties, diff = check_routing(ids.cpu().numpy(), gates.cpu().double().numpy(), logits, rid, rg)
         keep = np.setdiff1d(np.arange(c.N), diff)

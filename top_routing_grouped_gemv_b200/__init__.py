@@ -75,7 +75,7 @@ def load(path: str = LIB_PATH):
         "moe_plan_destroy": ([P], ctypes.c_int),
         "moe_workspace_size": ([P, ctypes.POINTER(sz)], ctypes.c_int),
         "moe_workspace_init": ([P, P, sz, P], ctypes.c_int),
-        "moe_router_topk": ([P, P, P, P, P, P], ctypes.c_int),
+        "moe_router_topk": ([P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_permute": ([P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_permute_noalloc": ([P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
         "moe_grouped_ffn": ([P, P, P, f32, P, P, sz, P], ctypes.c_int),
@@ -164,9 +164,10 @@ class Plan:
         return ws
 
     # -- stages ------------------------------------------------------------
-    def router_topk(self, x, ids, gates, margin=None, stream=None):
+    def router_topk(self, x, ids, gates, ws, margin=None, stream=None):
         _check(self.lib.moe_router_topk(self.handle, _ptr(x), _ptr(ids), _ptr(gates),
-                                        _ptr(margin), _stream(stream)), "moe_router_topk")
+                                        _ptr(margin), _ptr(ws), ws.numel(), _stream(stream)),
+               "moe_router_topk")
 
     def permute(self, x, ids, counts, offsets, pos, src, x_perm, ws, stream=None):
         _check(self.lib.moe_permute(self.handle, _ptr(x), _ptr(ids), _ptr(counts), _ptr(offsets),

@@ -28,7 +28,7 @@ struct Layout {
   size_t status = 0, chunk_counts = 0, h = 0, h_end = 0;
   size_t ids = 0, gates = 0, pos = 0, src = 0, counts = 0, offsets = 0, x_perm = 0, y_perm = 0;
   size_t fwd_end = 0, x_stage = 0, y_stage = 0, total = 0, x_stage_bytes = 0, y_stage_bytes = 0;
-  size_t permute_end = 0;
+  size_t permute_end = 0, router_w3 = 0, router_end = 0;
 };
 
 }  // namespace
@@ -66,6 +66,10 @@ void mark(moe_plan p, cudaStream_t s, const char* name_of_next) {
   p->nev++;
 }
 
+bool router_on_tensor_cores(const moe_layer_desc& d) {
+  return d.dtype == MOE_BF16 && d.E >= kRouterTcMinExperts;
+}
+
 void layout(moe_plan p) {
   const moe_layer_desc& d = p->desc;
   const long long R = static_cast<long long>(d.N) * d.K;
@@ -74,6 +78,9 @@ void layout(moe_plan p) {
   L.status = off; off = align_up(off + 4);
   L.chunk_counts = off; off = align_up(off + static_cast<size_t>(permute_chunks(d.N)) * d.E * 4);
   L.permute_end = off;
+  L.router_w3 = off;
+  if (router_on_tensor_cores(d)) off = align_up(off + router_tc_scratch_bytes(d.d, d.E));
+  L.router_end = off;
   L.h = off;
   if (d.act != MOE_ACT_NONE) off = align_up(off + static_cast<size_t>(R) * d.F * p->eh);
   L.h_end = off;
@@ -114,8 +121,15 @@ bool uses_tensor_cores(const moe_layer_desc& d) { return d.dtype != MOE_F32; }
 // The stage runners take the token count n <= plan N explicitly (the
 // host-buffer path runs the layer on token chunks).
 moe_status run_router(moe_plan p, int n, const void* x, int32_t* ids, float* gates, float* margin,
-                      cudaStream_t s) {
+                      void* ws, cudaStream_t s) {
   const moe_layer_desc& d = p->desc;
+  if (router_on_tensor_cores(d)) {
+    mark(p, s, "router_tc");
+    p->launches += 2;  // weight split + logits/top-K
+    return cuda_status(launch_router_tc(x, p->w.w_r, p->w.router_bias, n, d.d, d.E, d.K, ids, gates,
+                                        margin, at<void>(ws, p->L.router_w3),
+                                        at<int>(ws, p->L.status), s));
+  }
   mark(p, s, "router_topk");
   p->launches += 1;
   return cuda_status(launch_router(x, d.dtype, p->w.w_r, p->w.router_bias, n, d.d, d.E, d.K, ids,
@@ -175,9 +189,10 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
   a.groups = d.E;
   a.m_total = R;
   a.status = status;
-  // 256-row tiles on CTA pairs when the experts average at least that many
-  // rows; otherwise 128-row tiles on single CTAs (less padding work)
-  const bool pair = R >= 256 * d.E;
+  // 256-row tiles on CTA pairs when the experts average at least 512 routed
+  // rows; below that the last, partly empty row tile of each expert wastes
+  // too much MMA work and 128-row tiles on single CTAs win
+  const bool pair = R >= 512 * d.E;
   if (d.act == MOE_ACT_NONE) {
     if (!encode_kmajor_map(&a.tmA, x_perm, p->ex, R, d.d, kTcBlockM)) return MOE_ERR_CUDA;
     a.tmB0 = pair ? p->tmW1h : p->tmW1;
@@ -344,12 +359,14 @@ moe_status moe_workspace_init(moe_plan p, void* ws, size_t ws_bytes, moe_stream_
 }
 
 moe_status moe_router_topk(moe_plan p, const void* x, int32_t* ids, float* gates, float* margin,
-                           moe_stream_t stream) {
+                           void* ws, size_t ws_bytes, moe_stream_t stream) {
   if (!p || !x || !ids || !gates || !p->w.w_r) return MOE_ERR_INVALID_ARG;
   if (p->desc.dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
   if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
+  moe_status st0 = check_ws(p, ws, ws_bytes, p->L.router_end);
+  if (st0 != MOE_OK) return st0;
   begin(p);
-  moe_status st = run_router(p, p->desc.N, x, ids, gates, margin, stream);
+  moe_status st = run_router(p, p->desc.N, x, ids, gates, margin, ws, stream);
   end(p, stream);
   return st;
 }
@@ -449,7 +466,7 @@ namespace {
 moe_status forward_tokens(moe_plan p, int n, const void* x, void* y, void* ws, cudaStream_t stream) {
   const Layout& L = p->L;
   moe_status st = run_router(p, n, x, at<int32_t>(ws, L.ids), at<float>(ws, L.gates), nullptr,
-                             stream);
+                             ws, stream);
   if (st == MOE_OK)
     st = run_permute(p, n, x, at<int32_t>(ws, L.ids), at<int32_t>(ws, L.counts),
                      at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.pos), at<int32_t>(ws, L.src),

@@ -3,7 +3,8 @@
 // tokens routed to it).  The fp32 path needs fp32-exact products (tf32
 // tensor cores round the operands to 10 mantissa bits), so it runs on the
 // SIMT pipes: 64x64 output tiles, k staged through shared memory in slices
-// of 16, a 4x4 register micro-tile per thread, k summed in ascending order.
+// of 16 (the next slice prefetched into registers), a 4x4 register
+// micro-tile per thread, k summed in ascending order.
 //
 // Tile schedule: blockIdx.y enumerates the 64-row tiles of all experts in
 // expert order (empty experts own none); the CTA finds its expert from the
@@ -57,23 +58,28 @@ gemm_simt_f32_kernel(const float* __restrict__ A, int kdim, const float* __restr
     for (int j = 0; j < 4; ++j) acc[i][j] = accu[i][j] = 0.f;
 
   const int lr = tid / 4, lk = (tid % 4) * 4;  // loader: row/col within tile, k offset
+  // the next k-slice is fetched into registers while the current one is
+  // multiplied out of shared memory
+  float4 na, nb, nu;
+  auto fetch = [&](int k0) {
+    const int r = row0 + lr, k = k0 + lk, n = col0 + lr;
+    na = (r < row1 && k < kdim) ? *reinterpret_cast<const float4*>(A + (long long)r * kdim + k)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+    nb = (n < ncols && k < kdim) ? *reinterpret_cast<const float4*>(We + (long long)n * kdim + k)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (ACT == kActSwiglu)
+      nu = (n < ncols && k < kdim) ? *reinterpret_cast<const float4*>(Ue + (long long)n * kdim + k)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  fetch(0);
   for (int k0 = 0; k0 < kdim; k0 += BK) {
-    {
-      int r = row0 + lr, k = k0 + lk;
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < row1 && k < kdim) a = *reinterpret_cast<const float4*>(A + (long long)r * kdim + k);
-      As[lk + 0][lr] = a.x; As[lk + 1][lr] = a.y; As[lk + 2][lr] = a.z; As[lk + 3][lr] = a.w;
-      int n = col0 + lr;
-      float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (n < ncols && k < kdim) b = *reinterpret_cast<const float4*>(We + (long long)n * kdim + k);
-      Bs[lk + 0][lr] = b.x; Bs[lk + 1][lr] = b.y; Bs[lk + 2][lr] = b.z; Bs[lk + 3][lr] = b.w;
-      if (ACT == kActSwiglu) {
-        float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (n < ncols && k < kdim) u = *reinterpret_cast<const float4*>(Ue + (long long)n * kdim + k);
-        Us[lk + 0][lr] = u.x; Us[lk + 1][lr] = u.y; Us[lk + 2][lr] = u.z; Us[lk + 3][lr] = u.w;
-      }
+    As[lk + 0][lr] = na.x; As[lk + 1][lr] = na.y; As[lk + 2][lr] = na.z; As[lk + 3][lr] = na.w;
+    Bs[lk + 0][lr] = nb.x; Bs[lk + 1][lr] = nb.y; Bs[lk + 2][lr] = nb.z; Bs[lk + 3][lr] = nb.w;
+    if (ACT == kActSwiglu) {
+      Us[lk + 0][lr] = nu.x; Us[lk + 1][lr] = nu.y; Us[lk + 2][lr] = nu.z; Us[lk + 3][lr] = nu.w;
     }
     __syncthreads();
+    if (k0 + BK < kdim) fetch(k0 + BK);
 #pragma unroll
     for (int kk = 0; kk < BK; ++kk) {
       float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);

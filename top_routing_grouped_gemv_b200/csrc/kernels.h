@@ -21,6 +21,16 @@ cudaError_t launch_router(const void* x, int x_dtype, const float* w_r, const fl
                           int d, int E, int K, int32_t* ids, float* gates, float* margin,
                           cudaStream_t stream);
 
+// Tensor-core router (bf16 x): splits w_r into three bf16 parts in `scratch`
+// (router_tc_scratch_bytes) and runs the logits on tcgen05; top-K and the
+// softmax in the epilogue.
+size_t router_tc_scratch_bytes(int d, int E);
+cudaError_t launch_router_tc(const void* x, const float* w_r, const float* bias, int N, int d,
+                             int E, int K, int32_t* ids, float* gates, float* margin,
+                             void* scratch, int* status, cudaStream_t stream);
+// Experts above which bf16 routers run on the tensor cores.
+constexpr int kRouterTcMinExperts = 33;
+
 // ---- permute ----------------------------------------------------------------
 constexpr int kPermuteChunk = 32;  // tokens per chunk of the stable counting pass
 inline int permute_chunks(int N) { return (N + kPermuteChunk - 1) / kPermuteChunk; }
