@@ -330,10 +330,11 @@ def main():
         n_e2e = max(1, args.steps)
         if dist:
             dist.barrier()
+        # no L2 flush in this loop: every step's x arrives fresh from the host
+        # and the expert weights (> L2) are re-read each step anyway
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for i in range(n_e2e):
-            flush.zero_()
             plan.forward_host_async(xh[i % 2], yh[i % 2], ws)
         plan.host_join()
         b.record(stream)
@@ -387,7 +388,8 @@ def main():
             "config": {"workload": cfg.name, "N": cfg.N, "d": cfg.d, "E": cfg.E, "K": cfg.K,
                        "F": cfg.F, "act": cfg.act, "router": "fp32",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "flushed (256 MiB write) before every step",
+                       "l2": "value: flushed (256 MiB write) before every step; e2e: inputs "
+                             "larger than L2 (805 MB of expert weights), no flush",
                        "inputs": "seeded synthetic, resident in HBM"},
             "roofline": roofline, "gemm": gemm,
             "stages_us": {k: round(v, 2) for k, v in stage_us.items()},

@@ -43,6 +43,9 @@ __global__ void __launch_bounds__(256)
 combine_kernel(const uint4* __restrict__ y_perm, int row_vecs, const int32_t* __restrict__ pos,
                const float* __restrict__ gates, int N, int K, int R, uint4* __restrict__ y,
                int* status) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= N) return;
@@ -88,6 +91,9 @@ combine_kernel(const uint4* __restrict__ y_perm, int row_vecs, const int32_t* __
 __global__ void __launch_bounds__(256)
 unpermute_kernel(const uint4* __restrict__ y_perm, int row_vecs, const int32_t* __restrict__ pos,
                  int R, uint4* __restrict__ y, int* status) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
   const int lane = threadIdx.x & 31;
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (r >= R) return;
@@ -111,11 +117,11 @@ void launch_gated(const uint4* yp, int row_vecs, const int32_t* pos, const float
                   int K, int R, uint4* y, int* status, cudaStream_t stream) {
   int grid = (N + 7) / 8;
   if (K <= 2)
-    combine_kernel<T, 2><<<grid, 256, 0, stream>>>(yp, row_vecs, pos, gates, N, K, R, y, status);
+    launch_pdl(combine_kernel<T, 2>, dim3(grid), dim3(256), 0, stream, yp, row_vecs, pos, gates, N, K, R, y, status);
   else if (K <= 4)
-    combine_kernel<T, 4><<<grid, 256, 0, stream>>>(yp, row_vecs, pos, gates, N, K, R, y, status);
+    launch_pdl(combine_kernel<T, 4>, dim3(grid), dim3(256), 0, stream, yp, row_vecs, pos, gates, N, K, R, y, status);
   else
-    combine_kernel<T, 8><<<grid, 256, 0, stream>>>(yp, row_vecs, pos, gates, N, K, R, y, status);
+    launch_pdl(combine_kernel<T, 8>, dim3(grid), dim3(256), 0, stream, yp, row_vecs, pos, gates, N, K, R, y, status);
 }
 
 }  // namespace
@@ -129,7 +135,7 @@ cudaError_t launch_combine(const void* y_perm, int y_dtype, int dout, const int3
   auto yp = static_cast<const uint4*>(y_perm);
   auto yo = static_cast<uint4*>(y);
   if (gates == nullptr) {
-    unpermute_kernel<<<(R + 7) / 8, 256, 0, stream>>>(yp, row_vecs, pos, R, yo, status);
+    launch_pdl(unpermute_kernel, dim3((R + 7) / 8), dim3(256), 0, stream, yp, row_vecs, pos, R, yo, status);
   } else if (y_dtype == kF32) {
     launch_gated<float>(yp, row_vecs, pos, gates, N, K, R, yo, status, stream);
   } else {

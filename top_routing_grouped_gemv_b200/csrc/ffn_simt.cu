@@ -22,6 +22,9 @@ __global__ void __launch_bounds__(256)
 gemm_simt_f32_kernel(const float* __restrict__ A, int kdim, const float* __restrict__ W,
                      const float* __restrict__ W3, int ncols, float scale,
                      const int32_t* __restrict__ offsets, int E, float* __restrict__ out) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
   __shared__ __align__(16) float As[BK][BM + 4];
   __shared__ __align__(16) float Bs[BK][BN + 4];
   __shared__ __align__(16) float Us[BK][BN + 4];
@@ -133,13 +136,13 @@ cudaError_t launch_gemm_simt_f32(const float* A, int kdim, const float* W, const
   if (R == 0) return cudaSuccess;
   dim3 grid((ncols + BN - 1) / BN, (R + BM - 1) / BM + E);
   if (act == kActRelu)
-    gemm_simt_f32_kernel<kActRelu><<<grid, 256, 0, stream>>>(A, kdim, W, W3, ncols, scale, offsets,
+    launch_pdl(gemm_simt_f32_kernel<kActRelu>, dim3(grid), dim3(256), 0, stream, A, kdim, W, W3, ncols, scale, offsets,
                                                              E, out);
   else if (act == kActSwiglu)
-    gemm_simt_f32_kernel<kActSwiglu><<<grid, 256, 0, stream>>>(A, kdim, W, W3, ncols, scale,
+    launch_pdl(gemm_simt_f32_kernel<kActSwiglu>, dim3(grid), dim3(256), 0, stream, A, kdim, W, W3, ncols, scale,
                                                                offsets, E, out);
   else
-    gemm_simt_f32_kernel<kActNone><<<grid, 256, 0, stream>>>(A, kdim, W, W3, ncols, scale, offsets,
+    launch_pdl(gemm_simt_f32_kernel<kActNone>, dim3(grid), dim3(256), 0, stream, A, kdim, W, W3, ncols, scale, offsets,
                                                              E, out);
   return cudaGetLastError();
 }

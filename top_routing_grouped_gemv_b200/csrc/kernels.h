@@ -7,9 +7,29 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 struct moe_plan_s;  // the C ABI's plan (include/moe.h)
 
 namespace moe {
+
+// Launch with programmatic stream serialization (the kernel must call
+// griddep_wait before reading its predecessor's output).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 enum DType { kF32 = 0, kBF16 = 1, kE4M3 = 2 };
 enum Act { kActNone = 0, kActRelu = 1, kActSwiglu = 2 };

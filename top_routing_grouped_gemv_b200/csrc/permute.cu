@@ -30,6 +30,9 @@ __global__ void __launch_bounds__(128)
 permute_rank_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
                     int32_t* __restrict__ chunk_counts, int32_t* __restrict__ local_rank,
                     int* status) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
   __shared__ int hist[4][256];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int c = blockIdx.x * 4 + warp;
@@ -86,6 +89,9 @@ permute_rank_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
 __global__ void __launch_bounds__(1024)
 permute_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
   __shared__ int part[1024];
   __shared__ int total[257];
   int Ep = 1;
@@ -151,6 +157,9 @@ __global__ void __launch_bounds__(256)
 permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* __restrict__ ids,
                       int N, int K, int E, const int32_t* __restrict__ chunk_base,
                       int32_t* __restrict__ pos, int32_t* __restrict__ src, uint4* __restrict__ x_perm) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= N) return;
@@ -195,17 +204,17 @@ cudaError_t launch_permute_count(const int32_t* ids, int N, int K, int E, int32_
   if (nchunks == 0) return cudaSuccess;
   const int grid = (nchunks + 3) / 4;
   if (K <= 2)
-    permute_rank_kernel<2><<<grid, 128, 0, stream>>>(ids, N, K, E, chunk_counts, local_rank, status);
+    launch_pdl(permute_rank_kernel<2>, dim3(grid), dim3(128), 0, stream, ids, N, K, E, chunk_counts, local_rank, status);
   else if (K <= 4)
-    permute_rank_kernel<4><<<grid, 128, 0, stream>>>(ids, N, K, E, chunk_counts, local_rank, status);
+    launch_pdl(permute_rank_kernel<4>, dim3(grid), dim3(128), 0, stream, ids, N, K, E, chunk_counts, local_rank, status);
   else
-    permute_rank_kernel<8><<<grid, 128, 0, stream>>>(ids, N, K, E, chunk_counts, local_rank, status);
+    launch_pdl(permute_rank_kernel<8>, dim3(grid), dim3(128), 0, stream, ids, N, K, E, chunk_counts, local_rank, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_permute_scan(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
                                 int32_t* offsets, cudaStream_t stream) {
-  permute_scan_kernel<<<1, 1024, 0, stream>>>(chunk_counts, nchunks, E, counts, offsets);
+  launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, stream, chunk_counts, nchunks, E, counts, offsets);
   return cudaGetLastError();
 }
 
@@ -219,13 +228,13 @@ cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* i
   auto xv = static_cast<const uint4*>(x);
   auto xp = static_cast<uint4*>(x_perm);
   if (K <= 2)
-    permute_gather_kernel<2><<<grid, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base, pos,
+    launch_pdl(permute_gather_kernel<2>, dim3(grid), dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos,
                                                        src, xp);
   else if (K <= 4)
-    permute_gather_kernel<4><<<grid, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base, pos,
+    launch_pdl(permute_gather_kernel<4>, dim3(grid), dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos,
                                                        src, xp);
   else
-    permute_gather_kernel<8><<<grid, 256, 0, stream>>>(xv, row_vecs, ids, N, K, E, chunk_base, pos,
+    launch_pdl(permute_gather_kernel<8>, dim3(grid), dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos,
                                                        src, xp);
   return cudaGetLastError();
 }

@@ -56,6 +56,9 @@ __global__ void __launch_bounds__(kWarps * 32)
 router_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
               const float* __restrict__ bias, int N, int d, int E, int K,
               int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ margin) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
   constexpr int TM = kWarps * TPW;  // tokens per CTA
   constexpr int EP = EPL * 32;      // padded experts
   __shared__ float xs[kKC][TM + 1];  // +1: conflict-free transposed stores
@@ -169,6 +172,9 @@ __global__ void __launch_bounds__(256, E_T <= 8 ? 2 : 1)
 router_smem_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
                    const float* __restrict__ bias, int N, int d, int E, int K,
                    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ margin) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
   constexpr int VEC = 16 / sizeof(TX);        // k per 16-byte vector of x
   constexpr int CPB = E_T * VEC / 4;          // 16-byte chunks per block
   extern __shared__ float4 wsm[];
@@ -330,7 +336,7 @@ bool launch_smem(const TX* x, const float* w_r, const float* bias, int N, int d,
   const long long need = (static_cast<long long>(N) + 8 * TPW - 1) / (8 * TPW);
   const long long cap = static_cast<long long>(per_sm) * device_sm_count();
   const int grid = static_cast<int>(need < cap ? need : cap);
-  router_smem_kernel<TX, E_T, TPW><<<grid, 256, smem, stream>>>(x, w_r, bias, N, d, E, K, ids,
+  launch_pdl(router_smem_kernel<TX, E_T, TPW>, dim3(grid), dim3(256), smem, stream, x, w_r, bias, N, d, E, K, ids,
                                                                 gates, margin);
   return true;
 }
@@ -343,11 +349,11 @@ cudaError_t launch_epl(const TX* x, const float* w_r, const float* bias, int N, 
   int sms = device_sm_count();
   if ((long long)N >= 64LL * 2 * sms) {
     int grid = (N + 63) / 64;
-    router_kernel<TX, EPL, 8><<<grid, kWarps * 32, 0, stream>>>(x, w_r, bias, N, d, E, K, ids,
+    launch_pdl(router_kernel<TX, EPL, 8>, dim3(grid), dim3(kWarps * 32), 0, stream, x, w_r, bias, N, d, E, K, ids,
                                                                  gates, margin);
   } else {
     int grid = (N + 15) / 16;
-    router_kernel<TX, EPL, 2><<<grid, kWarps * 32, 0, stream>>>(x, w_r, bias, N, d, E, K, ids,
+    launch_pdl(router_kernel<TX, EPL, 2>, dim3(grid), dim3(kWarps * 32), 0, stream, x, w_r, bias, N, d, E, K, ids,
                                                                  gates, margin);
   }
   return cudaGetLastError();

@@ -57,6 +57,9 @@ constexpr uint32_t kRouterIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
 __global__ void __launch_bounds__(256)
 router_split_kernel(const float* __restrict__ w_r, int d, int E, int nchunks,
                     __nv_bfloat16* __restrict__ w3) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
   const long long total = static_cast<long long>(nchunks) * REC * d;
   for (long long idx = blockIdx.x * 256ll + threadIdx.x; idx < total; idx += 256ll * gridDim.x) {
     const int e = static_cast<int>(idx / d), k = static_cast<int>(idx % d);
@@ -86,6 +89,9 @@ struct RouterTcArgs {
 };
 
 __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(const __grid_constant__ RouterTcArgs args) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -295,8 +301,9 @@ cudaError_t launch_router_tc(const void* x, const float* w_r, const float* bias,
     const long long total = static_cast<long long>(nchunks) * REC * d;
     long long blocks = (total + 255) / 256;
     if (blocks > 4LL * device_sm_count()) blocks = 4LL * device_sm_count();
-    router_split_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(w_r, d, E, nchunks, w3);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(router_split_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                               stream, w_r, d, E, nchunks, w3);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   RouterTcArgs a;
@@ -325,7 +332,7 @@ cudaError_t launch_router_tc(const void* x, const float* w_r, const float* bias,
   }
   const int ntiles = (N + RM - 1) / RM;
   const int grid = ntiles < device_sm_count() ? ntiles : device_sm_count();
-  router_tc_kernel<<<grid, kRThreads, kRSmemBytes, stream>>>(a);
+  launch_pdl(router_tc_kernel, dim3(grid), dim3(kRThreads), kRSmemBytes, stream, a);
   return cudaGetLastError();
 }
 
