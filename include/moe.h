@@ -92,9 +92,16 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
  * SWIGLU: y = (silu(x W1^T) * (x W3^T)) W2^T, silu(z) = z / (1 + exp(-z)). */
 typedef enum { MOE_ACT_NONE = 0, MOE_ACT_RELU = 1, MOE_ACT_SWIGLU = 2 } moe_act;
 
-/* Scale granularity; values equal the Ascend page's quant-mode enumeration
- * (0 = not quantised, 1 = per-tensor).  Finer modes are not built. */
-typedef enum { MOE_QUANT_NONE = 0, MOE_QUANT_PER_TENSOR = 1 } moe_quant;
+/* Scale granularity of the expert weights; values equal the Ascend page's
+ * quant-mode enumeration (0 = not quantised, 1 = per-tensor, 2 =
+ * per-channel: one scale per output column of each expert).  Per-token
+ * activation scales (mode 3) are a per-call argument (x_token_scales).
+ * Group, block and mx modes are not built. */
+typedef enum {
+  MOE_QUANT_NONE = 0,
+  MOE_QUANT_PER_TENSOR = 1,
+  MOE_QUANT_PER_CHANNEL = 2
+} moe_quant;
 
 typedef struct {
   int32_t N;      /* tokens per call, >= 1 */
@@ -104,7 +111,7 @@ typedef struct {
   int32_t F;      /* FFN inner width; for MOE_ACT_NONE the output width N1; < 65536 */
   moe_dtype dtype;/* of x and the expert weights */
   moe_act act;
-  moe_quant quant;/* MOE_QUANT_PER_TENSOR requires dtype MOE_E4M3, and vice versa */
+  moe_quant quant;/* PER_TENSOR or PER_CHANNEL for dtype MOE_E4M3; NONE otherwise */
 } moe_layer_desc;
 
 typedef struct {
@@ -113,7 +120,8 @@ typedef struct {
   const void* w1;           /* (E, F, d) */
   const void* w3;           /* (E, F, d) for SWIGLU, else NULL */
   const void* w2;           /* (E, d, F) for RELU / SWIGLU, else NULL */
-  float w_scale;            /* per-tensor weight scale (gmmWeightScale) for e4m3, else ignored */
+  float w_scale;            /* per-tensor weight scale (gmmWeightScale), e4m3 PER_TENSOR */
+  const float* w_channel_scales; /* (E, F) fp32 per output channel, e4m3 PER_CHANNEL, else NULL */
 } moe_layer_weights;
 
 typedef struct moe_plan_s* moe_plan;
@@ -183,14 +191,17 @@ moe_status moe_permute_noalloc(moe_plan plan, const void* x, const int32_t* topk
 
 /* Grouped FFN (page 1 section 1.2 local expert execution; Ascend formula
  * gmmY).  Rows [offsets[e], offsets[e+1]) of x_perm go through expert e; the
- * result goes to the same rows of y_perm.  For e4m3: y_perm = (x_perm @
- * W_e) * x_scale * w_scale in fp32, rounded once to bf16.  x_scale is the
- * per-tensor gmmXScale (ignored unless e4m3).  offsets must be a valid
- * non-decreasing prefix with offsets[E] = N*K (as moe_permute writes it).
- * Uses workspace scratch (the SwiGLU/ReLU hidden activations). */
+ * result goes to the same rows of y_perm.  For e4m3: y_perm[r][n] =
+ * (x_perm[r] . W_e[n]) * xs(r) * ws(e, n) in fp32, rounded once to bf16, with
+ * xs(r) = x_row_scales[r] (per-token mode: one scale per permuted row) or the
+ * per-tensor x_scale when x_row_scales_or_null is NULL, and ws(e, n) the
+ * plan's per-channel scale or per-tensor w_scale.  Scales are ignored for
+ * bf16/fp32 layers.  offsets must be a valid non-decreasing prefix with
+ * offsets[E] = N*K (as moe_permute writes it).  Uses workspace scratch (the
+ * SwiGLU/ReLU hidden activations). */
 moe_status moe_grouped_ffn(moe_plan plan, const void* x_perm, const int32_t* offsets,
-                           float x_scale, void* y_perm, void* ws, size_t ws_bytes,
-                           moe_stream_t stream);
+                           float x_scale, const float* x_row_scales_or_null, void* y_perm,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Unpermute + combine (zyxy MoE structure: y = sum_i g_i E_i(x); Ascend
  * Unpermute).  topk_gates != NULL: y[t] = sum_{j<K} gates[t,j] *
@@ -203,10 +214,13 @@ moe_status moe_unpermute_combine(moe_plan plan, const void* y_perm, const int32_
 
 /* Shared-expert matmul run beside the routed experts (Ascend formula mmY =
  * (mmX @ mmWeight) * mmXScale * mmWeightScale).  x (M, H) e4m3, w (N2, H)
- * e4m3 output-major, y (M, N2) bf16.  Plan dtype must be e4m3.  Limits: H
- * a multiple of 16 and <= 12288, N2 < 65536. */
+ * e4m3 output-major, y (M, N2) bf16.  Scales: x_token_scales_or_null (M,
+ * per-token) else x_scale; w_channel_scales_or_null (N2, per-channel) else
+ * w_scale.  Plan dtype must be e4m3.  Limits: H a multiple of 16 and
+ * <= 12288, N2 < 65536. */
 moe_status moe_shared_matmul(moe_plan plan, const void* x, int32_t M, int32_t H, const void* w,
-                             int32_t N2, float x_scale, float w_scale, void* y,
+                             int32_t N2, float x_scale, const float* x_token_scales_or_null,
+                             float w_scale, const float* w_channel_scales_or_null, void* y,
                              moe_stream_t stream);
 
 /* Whole layer: router -> permute -> grouped FFN -> combine, on one stream,
@@ -217,9 +231,11 @@ moe_status moe_forward(moe_plan plan, const void* x, void* y, void* ws, size_t w
 
 /* Layer with caller-supplied routing: permute -> grouped FFN -> unpermute.
  * topk_gates_or_null selects combine (gates) or pure reorder (NULL; y is
- * (N*K, d_out)).  x_scale as in moe_grouped_ffn. */
+ * (N*K, d_out)).  For e4m3: x_token_scales_or_null (N, per-token mode) gives
+ * each token's scale (applied to its K permuted rows), else x_scale. */
 moe_status moe_forward_routed(moe_plan plan, const void* x, const int32_t* topk_ids,
-                              const float* topk_gates_or_null, float x_scale, void* y, void* ws,
+                              const float* topk_gates_or_null, float x_scale,
+                              const float* x_token_scales_or_null, void* y, void* ws,
                               size_t ws_bytes, moe_stream_t stream);
 
 /* moe_forward from host buffers: copies x_host (N, d) in, runs the layer,
@@ -246,6 +262,19 @@ moe_status moe_host_join(moe_plan plan, moe_stream_t stream);
 /* Synchronises `stream`, returns the sticky device status of the workspace
  * (MOE_OK if clean) and clears it. */
 moe_status moe_read_device_status(moe_plan plan, void* ws, moe_stream_t stream);
+
+/* Diagnostic of the device-side failure path (the pages have no counterpart):
+ * launches one CTA that waits, with the same bounded mbarrier wait the
+ * tensor-core kernels use but a limit of limit_us microseconds (1..1e6), on
+ * a barrier nothing arrives at, while a second warp waits on it with the
+ * kernels' default limit.  The first wait gives up and records
+ * MOE_ERR_DEVICE_TIMEOUT in the status word at the start of `ws` (read it
+ * with moe_read_device_status); the second leaves through the shared abort
+ * flag.  leave_order_or_null (device int32[2], caller-initialised) receives
+ * the order in which the two warps left.  No trap, fault or hang: the
+ * context stays usable. */
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t limit_us,
+                                     int32_t* leave_order_or_null, moe_stream_t stream);
 
 /* Stage timing: when enabled, moe_forward / moe_forward_routed record CUDA
  * events between their kernels.  moe_profile_read synchronises the last

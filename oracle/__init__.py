@@ -41,10 +41,15 @@ _lib = None
 
 
 def lib():
+    """The oracle library; ORACLE_LIB may name another build of moe_oracle.c
+    (the mutation tests point it at deliberately broken copies)."""
     global _lib
     if _lib is None:
-        build()
-        L = ctypes.CDLL(_LIB)
+        path = os.environ.get("ORACLE_LIB")
+        if not path:
+            build()
+            path = _LIB
+        L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         i, i64, d = ctypes.c_int, ctypes.c_int64, ctypes.c_double
         L.orc_router.argtypes = [i, i, i, i, i, P, P, P, P, P, P, P]
@@ -52,6 +57,7 @@ def lib():
         L.orc_permute.argtypes = [i, i, i, P, P, i64, P, P, P, P, P]
         L.orc_expert_rows.argtypes = [i, P, i, i, i, P, i, i, i, P, P, P, d, d, P]
         L.orc_combine.argtypes = [i, i, i, P, P, P, P]
+        L.orc_expert_rows_scaled.argtypes = [i, P, i, i, i, P, i, i, P, d, P, d, P, P]
         L.orc_forward_tokens.argtypes = [i, P, i, i, i, i, i, P, P, P, P, i, i, i, P, P, P, d, d,
                                          i, P, P, P, P]
         L.orc_dense_masked.argtypes = [i, i, i, i, P, P, i, i, i, P, P, P, d, d, P]
@@ -174,6 +180,23 @@ def expert_rows(row_expert, xrows, x_dtype: int, act: str, w1, w3, w2, w_dtype: 
     _check(lib().orc_expert_rows(len(row_expert), _p(row_expert), E, din, x_dtype, _p(xr), ACT[act],
                                  F, w_dtype, _p(w1n), _p(w3n), _p(w2n), x_scale, w_scale, _p(y)),
            "expert_rows")
+    return y
+
+
+def expert_rows_scaled(row_expert, xrows, x_dtype: int, w1, w_dtype: int, x_scale: float = 1.0,
+                       x_row_scales=None, w_scale: float = 1.0, w_channel_scales=None):
+    """Single-matrix experts with per-row x scales and per-(expert, output
+    channel) weight scales (NULL -> the per-tensor scalar)."""
+    row_expert = np.ascontiguousarray(row_expert, np.int32)
+    xr = _np(xrows)
+    w1n = _np(w1)
+    E, F, din = w1n.shape
+    xs = None if x_row_scales is None else np.ascontiguousarray(x_row_scales, np.float64)
+    ws = None if w_channel_scales is None else np.ascontiguousarray(w_channel_scales, np.float64)
+    y = np.full((len(row_expert), F), np.nan)
+    _check(lib().orc_expert_rows_scaled(len(row_expert), _p(row_expert), E, din, x_dtype, _p(xr), F,
+                                        w_dtype, _p(w1n), x_scale, _p(xs), w_scale, _p(ws), _p(y)),
+           "expert_rows_scaled")
     return y
 
 

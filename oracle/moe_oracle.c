@@ -339,6 +339,36 @@ int orc_expert_rows(int nrows, const int32_t* row_expert, int E, int din, int x_
     return ORC_OK;
 }
 
+/* Single-matrix experts with finer scales (Ascend quant modes 2 = per-channel
+ * for the weights, 3 = per-token for the activations):
+ *   y[r][n] = (sum_k x[r][k] W[e][n][k]) * xs[r] * ws[e][n]
+ * xs: one scale per input row (NULL: x_scale for all); ws: (E, F) per output
+ * channel of each expert (NULL: w_scale for all). */
+int orc_expert_rows_scaled(int nrows, const int32_t* row_expert, int E, int din, int x_dtype,
+                           const void* xrows, int F, int w_dtype, const void* w1, double x_scale,
+                           const double* xs, double w_scale, const double* ws, double* y) {
+    if (nrows < 0 || !row_expert || !xrows || !y || !w1 || din <= 0 || F <= 0) return ORC_ERR_ARG;
+    for (int r = 0; r < nrows; ++r)
+        if (row_expert[r] >= E) return ORC_ERR_INDEX;
+#pragma omp parallel
+    {
+        double* xr = (double*)malloc(sizeof(double) * (size_t)din);
+#pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < nrows; ++r) {
+            int e = row_expert[r];
+            if (e < 0) continue;
+            orc_to_f64(xrows, x_dtype, (int64_t)r * din, din, xr);
+            double sx = xs ? xs[r] : x_scale;
+            for (int n = 0; n < F; ++n) {
+                double sw = ws ? ws[(int64_t)e * F + n] : w_scale;
+                y[(int64_t)r * F + n] = dot_row(din, xr, w1, w_dtype, (int64_t)e * F + n) * sx * sw;
+            }
+        }
+        free(xr);
+    }
+    return ORC_OK;
+}
+
 /* ------------------------------------------------------------------------ */
 /* unpermute / combine                                                      */
 /* ------------------------------------------------------------------------ */

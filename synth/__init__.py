@@ -199,6 +199,15 @@ def quantize_e4m3_per_tensor(a: np.ndarray) -> tuple[np.ndarray, float]:
     return out, scale
 
 
+def quantize_e4m3_rows(a: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row e4m3 quantisation of a 2-D array: scale[i] = amax(|a[i]|)/448
+    (1 for an all-zero row), codes[i] = e4m3(a[i] / scale[i])."""
+    amax = np.max(np.abs(a), axis=1).astype(np.float64)
+    scale = np.where(amax > 0, amax / 448.0, 1.0).astype(np.float32)
+    codes = e4m3_encode(a.astype(np.float64) / scale.astype(np.float64)[:, None])
+    return codes, scale
+
+
 def normal_e4m3(seed: int, stream: int, n: int) -> tuple[np.ndarray, float]:
     """n iid N(0,1) draws quantised per tensor to e4m3, without holding the
     float draws: pass 1 finds amax chunk by chunk, pass 2 redraws each chunk

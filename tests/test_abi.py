@@ -28,7 +28,7 @@ def test_library_exports_every_header_symbol(lib):
 
 def test_struct_layouts_match_header():
     assert ctypes.sizeof(moe.LayerDesc) == 32
-    assert ctypes.sizeof(moe.LayerWeights) == 48
+    assert ctypes.sizeof(moe.LayerWeights) == 56
 
 
 def test_status_strings(lib):
@@ -39,7 +39,7 @@ def test_status_strings(lib):
 def _create(lib, N=64, d=64, E=8, K=2, F=64, dtype=moe.MOE_BF16, act=moe.ACT_SWIGLU,
             quant=moe.QUANT_NONE, w1=0x1000, w3=0x2000, w2=0x3000, w_r=0x4000):
     desc = moe.LayerDesc(N, d, E, K, F, dtype, act, quant)
-    w = moe.LayerWeights(w_r, None, w1, w3, w2, 1.0)
+    w = moe.LayerWeights(w_r, None, w1, w3, w2, 1.0, None)
     h = ctypes.c_void_p()
     rc = lib.moe_plan_create(ctypes.byref(desc), ctypes.byref(w), ctypes.byref(h))
     if rc == 0:
@@ -52,6 +52,9 @@ def _create(lib, N=64, d=64, E=8, K=2, F=64, dtype=moe.MOE_BF16, act=moe.ACT_SWI
     (dict(E=257), 1), (dict(d=65536), 1), (dict(F=70000), 1),
     (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None), 2),   # e4m3 needs per-tensor
     (dict(quant=moe.QUANT_PER_TENSOR), 2),                                 # per-tensor needs e4m3
+    (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None,
+          quant=moe.QUANT_PER_CHANNEL), 1),                                # per-channel needs scales
+    (dict(quant=7), 1),                                                    # mode not built
     (dict(dtype=moe.MOE_E4M3, act=moe.ACT_SWIGLU, quant=moe.QUANT_PER_TENSOR), 2),
     (dict(dtype=moe.MOE_BF16, act=moe.ACT_RELU, w3=None), 2),
     (dict(w3=None), 1),                                                    # SwiGLU needs w3

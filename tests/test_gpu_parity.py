@@ -344,3 +344,72 @@ def test_stage_profile_names():
                      "ffn1_swiglu_tc", "ffn2_tc", "combine"]
     assert all(ms >= 0 for _, ms in prof)
     assert plan.last_launch_count() == 7
+
+
+def test_bounded_wait_timeout_sets_status_and_context_survives():
+    """A wait on a barrier that nothing arrives at gives up after its limit,
+    records MOE_ERR_DEVICE_TIMEOUT and the other waiter leaves through the
+    abort flag; the context keeps working afterwards."""
+    import time
+    import top_routing_grouped_gemv_b200 as moe
+    inp, plan, w = case("bf16_k1")
+    c = inp.cfg
+    ws = plan.new_workspace()
+    order = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    moe.selftest_wait_timeout(ws, 20_000, order)          # 20 ms limit
+    assert plan.read_device_status(ws) == 6               # MOE_ERR_DEVICE_TIMEOUT
+    elapsed = time.perf_counter() - t0
+    assert 0.015 < elapsed < 0.9                          # gave up near its own limit
+    assert sorted(order.cpu().tolist()) == [0, 1]         # both waiters left
+    assert plan.read_device_status(ws) == 0               # cleared by the read
+    y = torch.empty(c.N, c.d, dtype=torch.bfloat16, device="cuda")
+    plan.forward(inp.x.cuda(), y, ws)                     # the context still works
+    assert plan.read_device_status(ws) == 0
+    assert torch.isfinite(y.float()).all()
+
+
+@pytest.mark.parametrize("N,d,E,K,F", [(300, 256, 8, 4, 384), (1100, 256, 4, 2, 392)])
+def test_e4m3_per_channel_weights_per_token_activations(N, d, E, K, F):
+    """Ascend quant modes 2 (weights, one scale per expert output channel) and
+    3 (activations, one scale per token) on the grouped matmul, the routed
+    layer (scales follow each token to its K permuted rows) and the shared
+    expert; the second shape runs on CTA pairs."""
+    import synth as sy
+    xq, xs = sy.quantize_e4m3_rows(sy.normal_f32(31, 1, N * d).reshape(N, d))
+    wq, wsc = sy.quantize_e4m3_rows(sy.normal_f32(31, 2, E * F * d).reshape(E * F, d))
+    wq, wsc = wq.reshape(E, F, d), wsc.reshape(E, F)
+    ids = sy.given_routing(31, N, E, K)
+    import top_routing_grouped_gemv_b200 as moe
+    w = {"w1": torch.from_numpy(wq).cuda(), "w_channel_scales": torch.from_numpy(wsc).cuda()}
+    plan = moe.Plan(N, d, E, K, F, "e4m3", "none", w)
+    ws = plan.new_workspace()
+    R = N * K
+    y = torch.empty(R, F, dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed(torch.from_numpy(xq).cuda(), torch.from_numpy(ids).cuda(), None, y, ws,
+                        x_token_scales=torch.from_numpy(xs).cuda())
+    assert plan.read_device_status(ws) == 0
+    rows_tok = np.repeat(np.arange(N), K)
+    ref = oracle.expert_rows_scaled(ids.reshape(-1), xq[rows_tok], oracle.E4M3, wq, oracle.E4M3,
+                                    x_row_scales=xs[rows_tok].astype(np.float64),
+                                    w_channel_scales=wsc.astype(np.float64))
+    assert rel_err(f64(y), ref) <= TOL["e4m3"]
+    # the grouped-matmul stage with per-row scales of the permuted rows
+    rc, ro, rp, rs, rx = oracle.permute(ids, E, xq)
+    yp = torch.empty(R, F, dtype=torch.bfloat16, device="cuda")
+    plan.grouped_ffn(torch.from_numpy(rx).cuda(), torch.from_numpy(ro).cuda(), yp, ws,
+                     x_row_scales=torch.from_numpy(xs[rs]).cuda())
+    ref_p = oracle.expert_rows_scaled(np.repeat(np.arange(E), rc).astype(np.int32), rx, oracle.E4M3,
+                                      wq, oracle.E4M3, x_row_scales=xs[rs].astype(np.float64),
+                                      w_channel_scales=wsc.astype(np.float64))
+    assert rel_err(f64(yp), ref_p) <= TOL["e4m3"]
+    # shared expert with both finer scales
+    shq, shs = sy.quantize_e4m3_rows(sy.normal_f32(31, 3, 136 * d).reshape(136, d))
+    ysh = torch.empty(N, 136, dtype=torch.bfloat16, device="cuda")
+    plan.shared_matmul(torch.from_numpy(xq).cuda(), torch.from_numpy(shq).cuda(), 1.0, 1.0, ysh,
+                       x_token_scales=torch.from_numpy(xs).cuda(),
+                       w_channel_scales=torch.from_numpy(shs).cuda())
+    ref_s = oracle.expert_rows_scaled(np.zeros(N, np.int32), xq, oracle.E4M3, shq.reshape(1, 136, d),
+                                      oracle.E4M3, x_row_scales=xs.astype(np.float64),
+                                      w_channel_scales=shs.astype(np.float64).reshape(1, 136))
+    assert rel_err(f64(ysh), ref_s) <= TOL["e4m3"]

@@ -151,6 +151,18 @@ def test_router_gate_properties(orc):
     assert np.allclose(gates, 0.25, atol=0) and ids.tolist() == [[0, 1, 2, 3]] * 3
 
 
+def test_router_softmax_is_stable_for_large_logits(orc):
+    """The softmax subtracts the largest kept logit: logits far from zero give
+    finite gates equal to the closed form (K = 2: logistic of the gap)."""
+    L = np.array([[0.0, 800.0, 900.0, -50.0], [-1000.0, -999.0, -2000.0, -1500.0]])
+    ids, gates, margin = orc.topk_from_logits(L, 2)
+    assert ids.tolist() == [[2, 1], [1, 0]]
+    assert np.isfinite(gates).all()
+    assert np.allclose(gates[0], [1 / (1 + np.exp(-100.0)), 1 - 1 / (1 + np.exp(-100.0))], atol=1e-15)
+    assert np.allclose(gates[1], [1 / (1 + np.exp(-1.0)), 1 / (1 + np.exp(1.0))], atol=1e-15)
+    assert margin.tolist() == [800.0, 500.0]
+
+
 def test_router_zipf_bias_closed_form(orc):
     """x = 0 leaves only the bias 1.2*ln(1/(e+1)): ids = 0..K-1, g_j ~ (j+1)^-1.2."""
     E, K, d = 128, 8, 16
@@ -288,6 +300,47 @@ def test_fp8_grouped_matmul_exact_integers(orc):
         for n in range(F):
             exact = sum(int(Xi[r, k]) * int(Wi[rexp[r], n, k]) for k in range(din))
             assert y[r, n] == exact * xs * ws
+
+
+def test_fp8_per_channel_and_per_token_scales_exact(orc):
+    """Ascend quant modes 2 (per-channel weights) and 3 (per-token x): with
+    small-integer codes the product sums are exact, so y = (sum x w) * xs[r] *
+    ws[e][n] is checked against Python integers times the scales."""
+    rng = np.random.default_rng(13)
+    E, F, din, R = 3, 6, 10, 9
+    Xi = rng.integers(-8, 9, size=(R, din))
+    Wi = rng.integers(-8, 9, size=(E, F, din))
+    enc = np.vectorize(orc.f64_to_e4m3, otypes=[np.uint8])
+    Xq, Wq = enc(Xi.astype(np.float64)), enc(Wi.astype(np.float64))
+    rexp = rng.integers(0, E, size=R).astype(np.int32)
+    xs = 2.0 ** rng.integers(-6, 3, size=R)
+    ws = 2.0 ** rng.integers(-6, 3, size=(E, F))
+    y = orc.expert_rows_scaled(rexp, Xq, orc.E4M3, Wq, orc.E4M3, x_row_scales=xs,
+                               w_channel_scales=ws)
+    for r in range(R):
+        for n in range(F):
+            exact = sum(int(Xi[r, k]) * int(Wi[rexp[r], n, k]) for k in range(din))
+            assert y[r, n] == exact * xs[r] * ws[rexp[r], n]
+    # NULL arrays fall back to the per-tensor scalars of the plain function
+    y0 = orc.expert_rows_scaled(rexp, Xq, orc.E4M3, Wq, orc.E4M3, x_scale=0.5, w_scale=0.25)
+    y1 = orc.expert_rows(rexp, Xq, orc.E4M3, "none", Wq, None, None, orc.E4M3, 0.5, 0.25)
+    assert np.array_equal(y0, y1)
+
+
+def test_per_row_quantiser_round_trip():
+    rng = np.random.default_rng(2)
+    a = rng.standard_normal((50, 64)) * rng.uniform(0.01, 100, size=(50, 1))
+    a[3] = 0.0
+    codes, scale = synth.quantize_e4m3_rows(a)
+    import oracle as orc
+    dec = orc.to_f64(codes, orc.E4M3) * scale[:, None]
+    # each row's max maps to 448 * scale; e4m3 rounding error is <= 2^-4
+    # relative for normal codes, <= half the subnormal step 2^-10 absolute
+    bound = 2.0 ** -4 * np.abs(a) + 2.0 ** -10 * scale[:, None].astype(np.float64)
+    assert np.all(np.abs(dec - a) <= bound)
+    keep = np.arange(50) != 3
+    assert np.array_equal(np.abs(dec).max(1)[keep], 448.0 * scale.astype(np.float64)[keep])
+    assert scale[3] == 1.0 and np.all(dec[3] == 0)
 
 
 @pytest.mark.parametrize("act,dtype", [("relu", "f32"), ("swiglu", "bf16"), ("none", "e4m3")])

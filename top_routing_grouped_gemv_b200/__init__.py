@@ -20,7 +20,7 @@ HEADER = os.path.join(ROOT, "include", "moe.h")
 
 MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
 ACT_NONE, ACT_RELU, ACT_SWIGLU = 0, 1, 2
-QUANT_NONE, QUANT_PER_TENSOR = 0, 1
+QUANT_NONE, QUANT_PER_TENSOR, QUANT_PER_CHANNEL = 0, 1, 2
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
           3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_BAD_INDEX",
@@ -44,7 +44,7 @@ class LayerDesc(ctypes.Structure):
 class LayerWeights(ctypes.Structure):
     _fields_ = [("w_r", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
                 ("w1", ctypes.c_void_p), ("w3", ctypes.c_void_p), ("w2", ctypes.c_void_p),
-                ("w_scale", ctypes.c_float)]
+                ("w_scale", ctypes.c_float), ("w_channel_scales", ctypes.c_void_p)]
 
 
 _lib = None
@@ -78,11 +78,11 @@ def load(path: str = LIB_PATH):
         "moe_router_topk": ([P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_permute": ([P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_permute_noalloc": ([P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
-        "moe_grouped_ffn": ([P, P, P, f32, P, P, sz, P], ctypes.c_int),
+        "moe_grouped_ffn": ([P, P, P, f32, P, P, P, sz, P], ctypes.c_int),
         "moe_unpermute_combine": ([P, P, P, P, P, P, sz, P], ctypes.c_int),
-        "moe_shared_matmul": ([P, P, i32, i32, P, i32, f32, f32, P, P], ctypes.c_int),
+        "moe_shared_matmul": ([P, P, i32, i32, P, i32, f32, P, f32, P, P, P], ctypes.c_int),
         "moe_forward": ([P, P, P, P, sz, P], ctypes.c_int),
-        "moe_forward_routed": ([P, P, P, P, f32, P, P, sz, P], ctypes.c_int),
+        "moe_forward_routed": ([P, P, P, P, f32, P, P, P, sz, P], ctypes.c_int),
         "moe_forward_host": ([P, P, P, P, sz, P], ctypes.c_int),
         "moe_forward_host_async": ([P, P, P, P, sz, P], ctypes.c_int),
         "moe_host_join": ([P, P], ctypes.c_int),
@@ -92,6 +92,7 @@ def load(path: str = LIB_PATH):
                               ctypes.c_int, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
         "moe_last_launch_count": ([P], ctypes.c_int),
         "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "moe_selftest_wait_timeout": ([P, sz, i32, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -131,11 +132,15 @@ class Plan:
         self.dtype, self.act = dtype, act
         self.d_out = F if act == "none" else d
         self._keep = dict(weights)
-        quant = QUANT_PER_TENSOR if dtype == "e4m3" else QUANT_NONE
+        quant = QUANT_NONE
+        if dtype == "e4m3":
+            quant = QUANT_PER_CHANNEL if weights.get("w_channel_scales") is not None \
+                else QUANT_PER_TENSOR
         desc = LayerDesc(N, d, E, K, F, DTYPE_CODE[dtype], ACT_CODE[act], quant)
         w = LayerWeights(_ptr(weights.get("w_r")), _ptr(weights.get("bias")),
                          _ptr(weights.get("w1")), _ptr(weights.get("w3")),
-                         _ptr(weights.get("w2")), float(weights.get("w_scale", 1.0)))
+                         _ptr(weights.get("w2")), float(weights.get("w_scale", 1.0)),
+                         _ptr(weights.get("w_channel_scales")))
         h = ctypes.c_void_p()
         _check(self.lib.moe_plan_create(ctypes.byref(desc), ctypes.byref(w), ctypes.byref(h)),
                "moe_plan_create")
@@ -183,30 +188,34 @@ class Plan:
                                             _ptr(device_status), _stream(stream)),
                "moe_permute_noalloc")
 
-    def grouped_ffn(self, x_perm, offsets, y_perm, ws, x_scale: float = 1.0, stream=None):
+    def grouped_ffn(self, x_perm, offsets, y_perm, ws, x_scale: float = 1.0, x_row_scales=None,
+                    stream=None):
         _check(self.lib.moe_grouped_ffn(self.handle, _ptr(x_perm), _ptr(offsets), x_scale,
-                                        _ptr(y_perm), _ptr(ws), ws.numel(), _stream(stream)),
-               "moe_grouped_ffn")
+                                        _ptr(x_row_scales), _ptr(y_perm), _ptr(ws), ws.numel(),
+                                        _stream(stream)), "moe_grouped_ffn")
 
     def unpermute_combine(self, y_perm, pos, gates, y, ws, stream=None):
         _check(self.lib.moe_unpermute_combine(self.handle, _ptr(y_perm), _ptr(pos), _ptr(gates),
                                               _ptr(y), _ptr(ws), ws.numel(), _stream(stream)),
                "moe_unpermute_combine")
 
-    def shared_matmul(self, x, w, x_scale, w_scale, y, stream=None):
+    def shared_matmul(self, x, w, x_scale, w_scale, y, x_token_scales=None,
+                      w_channel_scales=None, stream=None):
         M, H = x.shape
         N2 = w.shape[0]
         _check(self.lib.moe_shared_matmul(self.handle, _ptr(x), M, H, _ptr(w), N2, x_scale,
-                                          w_scale, _ptr(y), _stream(stream)), "moe_shared_matmul")
+                                          _ptr(x_token_scales), w_scale, _ptr(w_channel_scales),
+                                          _ptr(y), _stream(stream)), "moe_shared_matmul")
 
     def forward(self, x, y, ws, stream=None):
         _check(self.lib.moe_forward(self.handle, _ptr(x), _ptr(y), _ptr(ws), ws.numel(),
                                     _stream(stream)), "moe_forward")
 
-    def forward_routed(self, x, ids, gates, y, ws, x_scale: float = 1.0, stream=None):
+    def forward_routed(self, x, ids, gates, y, ws, x_scale: float = 1.0, x_token_scales=None,
+                       stream=None):
         _check(self.lib.moe_forward_routed(self.handle, _ptr(x), _ptr(ids), _ptr(gates), x_scale,
-                                           _ptr(y), _ptr(ws), ws.numel(), _stream(stream)),
-               "moe_forward_routed")
+                                           _ptr(x_token_scales), _ptr(y), _ptr(ws), ws.numel(),
+                                           _stream(stream)), "moe_forward_routed")
 
     def forward_host(self, x_host, y_host, ws, stream=None):
         _check(self.lib.moe_forward_host(self.handle, _ptr(x_host), _ptr(y_host), _ptr(ws),
@@ -237,6 +246,13 @@ class Plan:
 
     def last_launch_count(self) -> int:
         return self.lib.moe_last_launch_count(self.handle)
+
+
+def selftest_wait_timeout(ws, limit_us: int, leave_order=None, stream=None):
+    """Run the bounded-wait failure-path self-test (see include/moe.h)."""
+    lib = load()
+    _check(lib.moe_selftest_wait_timeout(_ptr(ws), ws.numel(), int(limit_us), _ptr(leave_order),
+                                         _stream(stream)), "moe_selftest_wait_timeout")
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

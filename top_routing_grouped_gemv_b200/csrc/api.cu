@@ -156,8 +156,11 @@ moe_status run_permute(moe_plan p, int n, const void* x, const int32_t* ids, int
   return MOE_OK;
 }
 
+// x_rows: per-token activation scales indexed by row_index[row] (or by the
+// permuted row itself when row_index is NULL); NULL = the scalar x_scale.
 moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets, float x_scale,
-                   void* y_perm, void* ws, cudaStream_t s) {
+                   const float* x_rows, const int32_t* row_index, void* y_perm, void* ws,
+                   cudaStream_t s) {
   const moe_layer_desc& d = p->desc;
   const int R = n * d.K;
   int* status = at<int>(ws, p->L.status);
@@ -202,7 +205,15 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
     a.n_tiles = (d.F + kTcBlockN - 1) / kTcBlockN;
     a.out = y_perm;
     a.ldo = d.F;
-    a.scale = d.quant == MOE_QUANT_PER_TENSOR ? x_scale * p->w.w_scale : 1.f;
+    if (d.dtype == MOE_E4M3) {
+      const bool per_channel = d.quant == MOE_QUANT_PER_CHANNEL;
+      a.scale = (x_rows ? 1.f : x_scale) * (per_channel ? 1.f : p->w.w_scale);
+      a.row_scale = x_rows;
+      a.row_index = x_rows ? row_index : nullptr;
+      a.col_scale = per_channel ? p->w.w_channel_scales : nullptr;
+    } else {
+      a.scale = 1.f;
+    }
     mark(p, s, "gmm_tc");
     p->launches += 1;
     return cuda_status(launch_gemm_tc(a, d.dtype, kEpiStore, R, pair, s));
@@ -277,9 +288,12 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
     return MOE_ERR_INVALID_ARG;
   if (static_cast<long long>(d.N) * d.K >= (1LL << 31)) return MOE_ERR_INVALID_ARG;
   if (d.dtype < MOE_F32 || d.dtype > MOE_E4M3 || d.act < MOE_ACT_NONE || d.act > MOE_ACT_SWIGLU ||
-      d.quant < MOE_QUANT_NONE || d.quant > MOE_QUANT_PER_TENSOR)
+      d.quant < MOE_QUANT_NONE || d.quant > MOE_QUANT_PER_CHANNEL)
     return MOE_ERR_INVALID_ARG;
-  if ((d.quant == MOE_QUANT_PER_TENSOR) != (d.dtype == MOE_E4M3)) return MOE_ERR_UNSUPPORTED;
+  if (d.quant < MOE_QUANT_NONE || d.quant > MOE_QUANT_PER_CHANNEL) return MOE_ERR_INVALID_ARG;
+  if ((d.quant != MOE_QUANT_NONE) != (d.dtype == MOE_E4M3)) return MOE_ERR_UNSUPPORTED;
+  if ((d.quant == MOE_QUANT_PER_CHANNEL) != (w->w_channel_scales != nullptr))
+    return MOE_ERR_INVALID_ARG;
   if (d.dtype == MOE_E4M3 && d.act != MOE_ACT_NONE) return MOE_ERR_UNSUPPORTED;
   if (d.dtype == MOE_BF16 && d.act == MOE_ACT_RELU) return MOE_ERR_UNSUPPORTED;
   if (!w->w1 || (d.act == MOE_ACT_SWIGLU) != (w->w3 != nullptr) ||
@@ -385,13 +399,14 @@ moe_status moe_permute(moe_plan p, const void* x, const int32_t* ids, int32_t* c
 }
 
 moe_status moe_grouped_ffn(moe_plan p, const void* x_perm, const int32_t* offsets, float x_scale,
-                           void* y_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+                           const float* x_row_scales, void* y_perm, void* ws, size_t ws_bytes,
+                           moe_stream_t stream) {
   if (!p || !x_perm || !offsets || !y_perm) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x_perm) || !aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
   moe_status st = check_ws(p, ws, ws_bytes, p->L.h_end);
   if (st != MOE_OK) return st;
   begin(p);
-  st = run_ffn(p, p->desc.N, x_perm, offsets, x_scale, y_perm, ws, stream);
+  st = run_ffn(p, p->desc.N, x_perm, offsets, x_scale, x_row_scales, nullptr, y_perm, ws, stream);
   end(p, stream);
   return st;
 }
@@ -410,7 +425,8 @@ moe_status moe_unpermute_combine(moe_plan p, const void* y_perm, const int32_t* 
 }
 
 moe_status moe_shared_matmul(moe_plan p, const void* x, int32_t M, int32_t H, const void* w,
-                             int32_t N2, float x_scale, float w_scale, void* y,
+                             int32_t N2, float x_scale, const float* x_token_scales,
+                             float w_scale, const float* w_channel_scales, void* y,
                              moe_stream_t stream) {
   if (!p || !x || !w || !y || M < 1 || H < 16 || H > 12288 || H % 16 || N2 < 1 || N2 >= 65536 ||
       N2 % 8)
@@ -432,14 +448,16 @@ moe_status moe_shared_matmul(moe_plan p, const void* x, int32_t M, int32_t H, co
   a.n_tiles = (N2 + kTcBlockN - 1) / kTcBlockN;
   a.out = y;
   a.ldo = N2;
-  a.scale = x_scale * w_scale;
+  a.scale = (x_token_scales ? 1.f : x_scale) * (w_channel_scales ? 1.f : w_scale);
+  a.row_scale = x_token_scales;
+  a.col_scale = w_channel_scales;
   a.status = nullptr;
   return cuda_status(launch_gemm_tc(a, kE4M3, kEpiStore, M, pair, stream));
 }
 
 moe_status moe_forward_routed(moe_plan p, const void* x, const int32_t* ids, const float* gates,
-                              float x_scale, void* y, void* ws, size_t ws_bytes,
-                              moe_stream_t stream) {
+                              float x_scale, const float* x_token_scales, void* y, void* ws,
+                              size_t ws_bytes, moe_stream_t stream) {
   if (!p || !x || !ids || !y) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   moe_status st = check_ws(p, ws, ws_bytes, p->L.fwd_end);
@@ -450,9 +468,10 @@ moe_status moe_forward_routed(moe_plan p, const void* x, const int32_t* ids, con
   st = run_permute(p, n, x, ids, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
                    at<int32_t>(ws, L.pos), at<int32_t>(ws, L.src), at<void>(ws, L.x_perm), ws,
                    stream);
+  // per-token scales reach the permuted rows through the source-token index
   if (st == MOE_OK)
-    st = run_ffn(p, n, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), x_scale,
-                 at<void>(ws, L.y_perm), ws, stream);
+    st = run_ffn(p, n, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), x_scale, x_token_scales,
+                 at<int32_t>(ws, L.src), at<void>(ws, L.y_perm), ws, stream);
   if (st == MOE_OK)
     st = run_combine(p, n, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
   end(p, stream);
@@ -472,7 +491,7 @@ moe_status forward_tokens(moe_plan p, int n, const void* x, void* y, void* ws, c
                      at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.pos), at<int32_t>(ws, L.src),
                      at<void>(ws, L.x_perm), ws, stream);
   if (st == MOE_OK)
-    st = run_ffn(p, n, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), 1.f,
+    st = run_ffn(p, n, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), 1.f, nullptr, nullptr,
                  at<void>(ws, L.y_perm), ws, stream);
   if (st == MOE_OK)
     st = run_combine(p, n, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), at<float>(ws, L.gates),

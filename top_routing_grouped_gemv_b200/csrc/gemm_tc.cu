@@ -343,6 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           }
         }
       } else {
+        float rsc = args.scale;
+        if (valid && args.row_scale != nullptr)
+          rsc *= args.row_scale[args.row_index != nullptr ? args.row_index[grow] : grow];
 #pragma unroll 1
         for (int cc = 0; cc < BN; cc += 32) {
           uint32_t v[32];
@@ -351,7 +354,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           tmem_ld_wait();
           const int col = c.n_tile * BN + cc;
           if (valid && col < args.n_out) {
-            const float sc = args.scale;
+            const float sc = rsc;
+            if (args.col_scale != nullptr) {
+              // per output channel: fold the channel scale into the values
+              const float* cs = args.col_scale + static_cast<long long>(c.g) * args.n_out + col;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col + j < args.n_out) v[j] = __float_as_uint(__uint_as_float(v[j]) * cs[j]);
+            }
             if (col + 32 <= args.n_out) {
               uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll

@@ -97,6 +97,11 @@ struct TcGemmArgs {
   void* out;               // bf16 (rows, ldo)
   long long ldo;           // elements
   float scale;             // multiplies the fp32 accumulator before rounding
+  // finer scales (store epilogue): out = acc * scale * row_scale[row'] *
+  // col_scale[g * n_out + col], row' = row_index[row] (or row); NULL = 1
+  const float* row_scale;
+  const int32_t* row_index;
+  const float* col_scale;
   int* status;
 };
 

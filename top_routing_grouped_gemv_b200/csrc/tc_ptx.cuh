@@ -40,15 +40,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Waits for the phase of parity `parity` to complete.  Gives up (false) when
-// another role raised the abort flag or after kWaitLimitNs, raising it.
-__device__ __noinline__ inline bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// another role raised the abort flag or after limit_ns, raising it.
+__device__ __noinline__ inline bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 127) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         return false;
       }
