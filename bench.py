@@ -297,14 +297,14 @@ def main():
             ends[i].record(stream)
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
-        # per-kernel durations: the library records events between its
-        # kernels; a short GPU sleep before each step lets the host enqueue
-        # the whole step first, so no launch gap lands inside a kernel's span
+        # per-kernel durations: the same loop with the library recording
+        # events between its kernels (the L2 flush before each step gives the
+        # host a head start, so the GEMMs are enqueued before the GPU reaches
+        # them and no launch gap lands inside their spans)
         plan.profile(True)
         per_kernel: dict[str, list[float]] = {}
-        for i in range(min(args.steps, 50)):
+        for i in range(min(args.steps, 100)):
             flush.zero_()
-            torch.cuda._sleep(400_000)
             step()
             for name, ms in plan.profile_read():
                 per_kernel.setdefault(name, []).append(ms)

@@ -232,7 +232,11 @@ moe_status moe_forward(moe_plan plan, const void* x, void* y, void* ws, size_t w
 /* Layer with caller-supplied routing: permute -> grouped FFN -> unpermute.
  * topk_gates_or_null selects combine (gates) or pure reorder (NULL; y is
  * (N*K, d_out)).  For e4m3: x_token_scales_or_null (N, per-token mode) gives
- * each token's scale (applied to its K permuted rows), else x_scale. */
+ * each token's scale (applied to its K permuted rows), else x_scale.  The
+ * pure reorder of a single-matrix tensor-core layer (the Ascend page's fused
+ * GMM -> Unpermute) is done by the grouped GEMM's stores, row r of the
+ * result going straight to row t*K+j of y; rows of invalid (t, j) pairs are
+ * left unwritten, as moe_unpermute_combine leaves them. */
 moe_status moe_forward_routed(moe_plan plan, const void* x, const int32_t* topk_ids,
                               const float* topk_gates_or_null, float x_scale,
                               const float* x_token_scales_or_null, void* y, void* ws,

@@ -28,6 +28,8 @@ SMALL = {
     "bf16_zipf": synth.small_variant(synth.BF16_FINEGRAINED, N=1000, d=256, E=64, K=8, F=128),
     "bf16_k1": synth.small_variant(synth.BF16_PREFILL, N=130, d=128, E=4, K=1, F=128),
     "bf16_f_not_tile": synth.small_variant(synth.BF16_PREFILL, N=160, d=192, E=3, K=2, F=200),
+    # token rows not a whole number of 128-byte K blocks (partial K box)
+    "bf16_d_not_kblock": synth.small_variant(synth.BF16_PREFILL, N=150, d=200, E=5, K=2, F=136),
     "e4m3_gmm": synth.small_variant(synth.FP8_GMM, N=256, d=512, E=16, K=4, F=512,
                                     shared=(512, 384)),
     "e4m3_gmm_ragged": synth.small_variant(synth.FP8_GMM, N=45, d=256, E=40, K=8, F=96,
@@ -155,6 +157,45 @@ def test_grouped_ffn_parity(name):
     assert err <= TOL[c.dtype], err
 
 
+# Row counts per expert around the 256-row tile of the CTA-pair mode (each
+# CTA of the pair holds 128 rows of a tile): last tiles holding 128, 129, 128
+# (the whole expert) and 126 / 22 rows.
+TAIL_COUNTS = [384, 385, 128, 1151]
+
+
+@pytest.mark.parametrize("name", ["bf16_pair", "e4m3_pair"])
+def test_pair_tile_tail_boundaries(name):
+    inp, plan, w = case(name)
+    c = inp.cfg
+    R = c.N * c.K
+    assert R >= 512 * c.E and c.E == len(TAIL_COUNTS)
+    counts = np.array(TAIL_COUNTS, np.int64)
+    counts[-1] += R - counts.sum() - 1        # one row short of R: m_total > offsets[E]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    rng = np.random.default_rng(11)
+    rows = rng.integers(0, c.N, R)            # any token rows as the permuted input
+    xn = inp.x.numpy() if c.dtype == "e4m3" else inp.x.view(torch.int16).numpy()
+    xp = np.ascontiguousarray(xn[rows])
+    x_perm = torch.from_numpy(xp).cuda()
+    if c.dtype == "bf16":
+        x_perm = x_perm.view(torch.bfloat16)
+    y_perm = torch.full((R, c.d_out), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = plan.new_workspace()
+    plan.grouped_ffn(x_perm, torch.from_numpy(offsets).cuda(), y_perm, ws, x_scale=inp.x_scale)
+    assert plan.read_device_status(ws) == 0
+    used = int(offsets[-1])
+    row_e = np.repeat(np.arange(c.E), counts).astype(np.int32)
+    dt = oracle.DTYPE[c.dtype]
+    xsrc = inp.x.numpy()[rows[:used]] if c.dtype == "e4m3" else inp.x[torch.from_numpy(rows[:used])]
+    ref = oracle.expert_rows(row_e, xsrc, dt, c.act, inp.w1, inp.w3, inp.w2, dt, inp.x_scale,
+                             inp.w_scale)
+    got = f64(y_perm)
+    assert np.isnan(got[used:]).all()         # rows past offsets[E] are never stored
+    for e in range(c.E):
+        a, b = offsets[e], offsets[e + 1]
+        assert rel_err(got[a:b], ref[a:b]) <= TOL[c.dtype], e
+
+
 @pytest.mark.parametrize("name", list(SMALL))
 def test_combine_parity(name):
     """Combine fed a synthetic y_perm of the layer's dtype and the oracle's
@@ -200,7 +241,9 @@ def test_forward_end_to_end(name):
         plan.forward_routed(x, inp.ids.cuda(), None, y, ws, x_scale=inp.x_scale)
         gate_mode = 0
     assert plan.read_device_status(ws) == 0
-    assert plan.last_launch_count() >= 5
+    # router, count, scan, gather, GEMM(s), combine -- the pure
+    # unpermute of the routed single-matrix layer is done by its GEMM's stores
+    assert plan.last_launch_count() >= (5 if c.routing == "router" else 4)
     ref, rids, _, _ = oracle.forward_tokens(inp, np.arange(c.N), gates_mode=gate_mode)
     got = f64(y)
     if c.routing == "router":
@@ -328,6 +371,71 @@ def test_workspace_too_small_and_misaligned():
     with pytest.raises(moe.MoEError) as e:
         plan.forward(inp.x.cuda(), y, ws[16:])
     assert e.value.code == 1
+
+
+TC_CASES = [n for n in SMALL if SMALL[n].dtype != "f32"]
+
+
+@pytest.mark.parametrize("name", TC_CASES)
+def test_fused_forward_matches_stage_composition(name):
+    """The whole-layer calls keep their intermediates in the workspace (and,
+    for the single-matrix layer without gates, the GEMM stores its rows
+    straight to their unpermuted place); the stage calls take caller buffers.
+    Same operands, same MMA order: the results agree bit for bit."""
+    inp, plan, w = case(name)
+    c = inp.cfg
+    x = inp.x.cuda()
+    ws = plan.new_workspace()
+    R = c.N * c.K
+    ydt = torch.bfloat16
+    if c.routing == "router":
+        ids = torch.empty(c.N, c.K, dtype=torch.int32, device="cuda")
+        gates = torch.empty(c.N, c.K, dtype=torch.float32, device="cuda")
+        plan.router_topk(x, ids, gates, ws)
+        y_fused = torch.empty(c.N, c.d_out, dtype=ydt, device="cuda")
+        plan.forward(x, y_fused, ws)
+    else:
+        ids = inp.ids.cuda()
+        gates = None
+        y_fused = torch.full((R, c.d_out), float("nan"), dtype=ydt, device="cuda")
+        plan.forward_routed(x, ids, None, y_fused, ws, x_scale=inp.x_scale)
+    assert plan.read_device_status(ws) == 0
+    counts = torch.empty(c.E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(c.E + 1, dtype=torch.int32, device="cuda")
+    pos = torch.empty(R, dtype=torch.int32, device="cuda")
+    src = torch.empty(R, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty((R,) + tuple(x.shape[1:]), dtype=x.dtype, device="cuda")
+    y_perm = torch.empty(R, c.d_out, dtype=ydt, device="cuda")
+    plan.permute(x, ids, counts, offsets, pos, src, x_perm, ws)
+    plan.grouped_ffn(x_perm, offsets, y_perm, ws, x_scale=inp.x_scale)
+    y_stage = torch.empty_like(y_fused)
+    plan.unpermute_combine(y_perm, pos, gates, y_stage, ws)
+    assert plan.read_device_status(ws) == 0
+    assert torch.equal(y_fused.view(torch.int16), y_stage.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["e4m3_gmm", "e4m3_pair"])
+def test_fused_routed_with_gates_and_token_scales(name):
+    """Single-matrix layer with gates (combine as its own pass) and
+    per-token activation scales read through the source-token index."""
+    inp, plan, w = case(name)
+    c = inp.cfg
+    ws = plan.new_workspace()
+    rng = np.random.default_rng(7)
+    ids = inp.ids.numpy()
+    g = rng.random((c.N, c.K)).astype(np.float32)
+    xs = (inp.x_scale * rng.uniform(0.5, 2.0, c.N)).astype(np.float32)
+    y = torch.empty(c.N, c.d_out, dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed(inp.x.cuda(), inp.ids.cuda(), torch.from_numpy(g).cuda(), y, ws,
+                        x_scale=1.0, x_token_scales=torch.from_numpy(xs).cuda())
+    assert plan.read_device_status(ws) == 0
+    # oracle: per-row scales of the permuted rows, then the gated combine
+    _, _, rp, rs, rx = oracle.permute(ids, c.E, inp.x)
+    row_e = np.repeat(np.arange(c.E, dtype=np.int32), np.bincount(ids.ravel(), minlength=c.E))
+    yp = oracle.expert_rows_scaled(row_e, rx, oracle.E4M3, inp.w1, oracle.E4M3, x_scale=1.0,
+                                   x_row_scales=xs[rs].astype(np.float64), w_scale=inp.w_scale)
+    ref = oracle.combine(rp, g.astype(np.float64), yp, c.N, c.K)
+    assert rel_err(f64(y), ref) <= TOL["e4m3"]
 
 
 def test_stage_profile_names():

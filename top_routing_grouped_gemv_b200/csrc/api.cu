@@ -26,7 +26,8 @@ constexpr int kHostEvents = 6;
 
 struct Layout {
   size_t status = 0, chunk_counts = 0, h = 0, h_end = 0;
-  size_t ids = 0, gates = 0, pos = 0, src = 0, counts = 0, offsets = 0, x_perm = 0, y_perm = 0;
+  size_t ids = 0, gates = 0, pos = 0, src = 0, slot = 0, counts = 0, offsets = 0, x_perm = 0,
+         y_perm = 0;
   size_t fwd_end = 0, x_stage = 0, y_stage = 0, total = 0, x_stage_bytes = 0, y_stage_bytes = 0;
   size_t permute_end = 0, router_w3 = 0, router_end = 0;
 };
@@ -66,6 +67,8 @@ void mark(moe_plan p, cudaStream_t s, const char* name_of_next) {
   p->nev++;
 }
 
+bool uses_tensor_cores(const moe_layer_desc& d) { return d.dtype != MOE_F32; }
+
 bool router_on_tensor_cores(const moe_layer_desc& d) {
   return d.dtype == MOE_BF16 && d.E >= kRouterTcMinExperts;
 }
@@ -88,6 +91,7 @@ void layout(moe_plan p) {
   L.gates = off; off = align_up(off + static_cast<size_t>(R) * 4);
   L.pos = off; off = align_up(off + static_cast<size_t>(R) * 4);
   L.src = off; off = align_up(off + static_cast<size_t>(R) * 4);
+  L.slot = off; off = align_up(off + static_cast<size_t>(R) * 4);
   L.counts = off; off = align_up(off + static_cast<size_t>(d.E) * 4);
   L.offsets = off; off = align_up(off + static_cast<size_t>(d.E + 1) * 4);
   L.x_perm = off; off = align_up(off + static_cast<size_t>(R) * d.d * p->ex);
@@ -116,8 +120,6 @@ moe_status check_ws(moe_plan p, void* ws, size_t ws_bytes, size_t need) {
   return MOE_OK;
 }
 
-bool uses_tensor_cores(const moe_layer_desc& d) { return d.dtype != MOE_F32; }
-
 // The stage runners take the token count n <= plan N explicitly (the
 // host-buffer path runs the layer on token chunks).
 moe_status run_router(moe_plan p, int n, const void* x, int32_t* ids, float* gates, float* margin,
@@ -136,9 +138,11 @@ moe_status run_router(moe_plan p, int n, const void* x, int32_t* ids, float* gat
                                    gates, margin, s));
 }
 
+// slot (optional): slot[pos] = t*K + j, the destination row of a pure
+// unpermute, for a grouped FFN that stores its rows there directly.
 moe_status run_permute(moe_plan p, int n, const void* x, const int32_t* ids, int32_t* counts,
                        int32_t* offsets, int32_t* pos, int32_t* src, void* x_perm, void* ws,
-                       cudaStream_t s) {
+                       cudaStream_t s, int32_t* slot = nullptr) {
   const moe_layer_desc& d = p->desc;
   int* status = at<int>(ws, p->L.status);
   int32_t* cc = at<int32_t>(ws, p->L.chunk_counts);
@@ -149,8 +153,8 @@ moe_status run_permute(moe_plan p, int n, const void* x, const int32_t* ids, int
   if (launch_permute_scan(cc, permute_chunks(n), d.E, counts, offsets, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   mark(p, s, "permute_gather");
-  if (launch_permute_gather(x, d.d * p->ex, ids, n, d.K, d.E, cc, pos, src, x_perm, status, s) !=
-      cudaSuccess)
+  if (launch_permute_gather(x, d.d * p->ex, ids, n, d.K, d.E, cc, pos, src, slot, x_perm, status,
+                            s) != cudaSuccess)
     return MOE_ERR_CUDA;
   p->launches += 3;
   return MOE_OK;
@@ -158,9 +162,11 @@ moe_status run_permute(moe_plan p, int n, const void* x, const int32_t* ids, int
 
 // x_rows: per-token activation scales indexed by row_index[row] (or by the
 // permuted row itself when row_index is NULL); NULL = the scalar x_scale.
+// out_rows (tensor cores, single-matrix layer): result row r goes to row
+// out_rows[r] of y_perm (the pure unpermute done by the GEMM's stores).
 moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets, float x_scale,
                    const float* x_rows, const int32_t* row_index, void* y_perm, void* ws,
-                   cudaStream_t s) {
+                   cudaStream_t s, const int32_t* out_rows = nullptr) {
   const moe_layer_desc& d = p->desc;
   const int R = n * d.K;
   int* status = at<int>(ws, p->L.status);
@@ -196,14 +202,15 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
   // rows; below that the last, partly empty row tile of each expert wastes
   // too much MMA work and 128-row tiles on single CTAs win
   const bool pair = R >= 512 * d.E;
+  if (!encode_kmajor_map(&a.tmA, x_perm, p->ex, R, d.d, kTcBlockM)) return MOE_ERR_CUDA;
   if (d.act == MOE_ACT_NONE) {
-    if (!encode_kmajor_map(&a.tmA, x_perm, p->ex, R, d.d, kTcBlockM)) return MOE_ERR_CUDA;
     a.tmB0 = pair ? p->tmW1h : p->tmW1;
     a.tmB1 = a.tmB0;
     a.kdim = d.d;
     a.n_out = d.F;
     a.n_tiles = (d.F + kTcBlockN - 1) / kTcBlockN;
     a.out = y_perm;
+    a.out_rows = out_rows;
     a.ldo = d.F;
     if (d.dtype == MOE_E4M3) {
       const bool per_channel = d.quant == MOE_QUANT_PER_CHANNEL;
@@ -219,7 +226,6 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
     return cuda_status(launch_gemm_tc(a, d.dtype, kEpiStore, R, pair, s));
   }
   // SwiGLU: gate/up GEMM with the activation fused into its epilogue, then down
-  if (!encode_kmajor_map(&a.tmA, x_perm, p->ex, R, d.d, kTcBlockM)) return MOE_ERR_CUDA;
   a.tmB0 = p->tmW1;
   a.tmB1 = p->tmW3;
   a.kdim = d.d;
@@ -465,14 +471,18 @@ moe_status moe_forward_routed(moe_plan p, const void* x, const int32_t* ids, con
   const Layout& L = p->L;
   begin(p);
   const int n = p->desc.N;
+  int32_t* src = at<int32_t>(ws, L.src);
+  // a pure unpermute of the single-matrix layer on the tensor cores is done
+  // by the GEMM's stores (row r -> row slot[r] = t*K + j of y): no reorder pass
+  const bool scatter = uses_tensor_cores(p->desc) && p->desc.act == MOE_ACT_NONE && !gates;
+  int32_t* slot = scatter ? at<int32_t>(ws, L.slot) : nullptr;
   st = run_permute(p, n, x, ids, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
-                   at<int32_t>(ws, L.pos), at<int32_t>(ws, L.src), at<void>(ws, L.x_perm), ws,
-                   stream);
+                   at<int32_t>(ws, L.pos), src, at<void>(ws, L.x_perm), ws, stream, slot);
   // per-token scales reach the permuted rows through the source-token index
   if (st == MOE_OK)
-    st = run_ffn(p, n, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), x_scale, x_token_scales,
-                 at<int32_t>(ws, L.src), at<void>(ws, L.y_perm), ws, stream);
-  if (st == MOE_OK)
+    st = run_ffn(p, n, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), x_scale,
+                 x_token_scales, src, scatter ? y : at<void>(ws, L.y_perm), ws, stream, slot);
+  if (st == MOE_OK && !scatter)
     st = run_combine(p, n, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
   end(p, stream);
   return st;

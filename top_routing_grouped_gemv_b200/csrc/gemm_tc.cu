@@ -12,7 +12,8 @@
 //
 // Structure (one persistent CTA per SM, 6 warps):
 //   warp 0      TMA producer: 128-byte-swizzled K-major tiles of A (128 rows)
-//               and W (256 rows) into a 4-stage shared-memory ring
+//               and W (256 rows) into a 4-stage shared-memory ring (6
+//               stages of 128 + 128 rows per CTA in the CTA-pair mode)
 //   warp 1      owns the 512 TMEM columns; lane 0 issues tcgen05.mma
 //               (M=128, N=256, K=16 bf16 / K=32 e4m3 per instruction) into
 //               one of two fp32 accumulators, and tcgen05.commit releases
@@ -23,6 +24,9 @@
 // The tile list (group, row tile, column tile) is derived on the device
 // from the offsets, so no host synchronisation is needed; empty groups own
 // no tiles, and rows past a group's end are computed but never stored.
+//
+// Optional row scatter: result row r is stored at row out_rows[r] (the pure
+// unpermute of the single-matrix layer done by the stores).
 //
 // Every mbarrier wait is bounded (1 s): on expiry the CTA records
 // MOE_ERR_DEVICE_TIMEOUT, the other roles leave their loops, in-flight
@@ -293,7 +297,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   } else {
     // ---------------- epilogue (warps 2..5 of every CTA) ----------------
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const int row = static_cast<int>(rank) * BM + q * 32 + lane;  // row within the tile
     int i = 0;
     for (int T = unit; T < total; T += nunits, ++i) {
       const int acc = i & 1;
@@ -307,20 +310,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       }
       tc_fence_after();
       const TileCoord c = decode_tile<Gm::TILE_M>(T, s_pref, s_off, G);
+      // lane quadrant q holds rows 32q.. of this CTA's 128 rows of the tile
+      const int row = static_cast<int>(rank) * BM + q * 32 + lane;
+      constexpr int span = kEpi == kEpiSwiglu ? BN / 2 : BN;  // output columns of the tile
+      const int col0 = c.n_tile * span;
       const long long grow = static_cast<long long>(c.m_row0) + row;
       const bool valid = grow < s_off[c.g + 1] && grow < args.m_total && grow >= 0;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + grow * args.ldo;
+      long long orow_i = grow;
+      if (valid && args.out_rows != nullptr) orow_i = args.out_rows[grow];
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + orow_i * args.ldo;
       if (kEpi == kEpiSwiglu) {
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 2; cc += 32) {
+        for (int cc = 0; cc < span; cc += 32) {
           uint32_t gr[32], ur[32];
           __syncwarp();
-          tmem_ld32(tbase + cc, gr);
-          tmem_ld32(tbase + BN / 2 + cc, ur);
+          tmem_ld32(tbase + cc, gr);          // gate columns
+          tmem_ld32(tbase + span + cc, ur);   // up columns of the same outputs
           tmem_ld_wait();
-          const int col = c.n_tile * (BN / 2) + cc;
+          const int col = col0 + cc;
           if (valid && col < args.n_out) {
             uint32_t pk[16];
 #pragma unroll
@@ -347,12 +356,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         if (valid && args.row_scale != nullptr)
           rsc *= args.row_scale[args.row_index != nullptr ? args.row_index[grow] : grow];
 #pragma unroll 1
-        for (int cc = 0; cc < BN; cc += 32) {
+        for (int cc = 0; cc < span; cc += 32) {
           uint32_t v[32];
           __syncwarp();
           tmem_ld32(tbase + cc, v);
           tmem_ld_wait();
-          const int col = c.n_tile * BN + cc;
+          const int col = col0 + cc;
           if (valid && col < args.n_out) {
             const float sc = rsc;
             if (args.col_scale != nullptr) {

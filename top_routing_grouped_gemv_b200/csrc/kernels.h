@@ -63,10 +63,11 @@ cudaError_t launch_permute_count(const int32_t* ids, int N, int K, int E, int32_
 cudaError_t launch_permute_scan(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
                                 int32_t* offsets, cudaStream_t stream);
 // pos holds the ranks from launch_permute_count on entry, the final
-// positions on exit.
+// positions on exit; src[pos] = t and, when slot is non-null,
+// slot[pos] = t*K + j.
 cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* ids, int N, int K,
                                   int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
-                                  void* x_perm, int* status, cudaStream_t stream);
+                                  int32_t* slot, void* x_perm, int* status, cudaStream_t stream);
 
 // ---- combine / unpermute ----------------------------------------------------
 // y_dtype: kF32 or kBF16 (the dtype of y_perm and y).
@@ -103,6 +104,9 @@ struct TcGemmArgs {
   const int32_t* row_index;
   const float* col_scale;
   int* status;
+  // Row scatter (unpermute fused into the store): when set, row r of the
+  // result is stored at row out_rows[r] of out.
+  const int32_t* out_rows;
 };
 
 // Host: encode a 2-D K-major tile map over a (rows, kdim) row-major matrix of

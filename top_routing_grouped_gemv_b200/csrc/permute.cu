@@ -15,7 +15,9 @@
 //              (offsets[e] + rows of e in earlier chunks), counts, offsets
 //   3. gather: one warp per token turns its ranks into final positions and
 //              copies the token row once from HBM into its K destination
-//              rows with 16-byte vector loads/stores.
+//              rows with 16-byte vector loads/stores (and, on request, notes
+//              each position's flat slot t*K + j for an unpermute done by
+//              the grouped GEMM's stores).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -156,7 +158,8 @@ template <int KMAX>
 __global__ void __launch_bounds__(256)
 permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* __restrict__ ids,
                       int N, int K, int E, const int32_t* __restrict__ chunk_base,
-                      int32_t* __restrict__ pos, int32_t* __restrict__ src, uint4* __restrict__ x_perm) {
+                      int32_t* __restrict__ pos, int32_t* __restrict__ src,
+                      int32_t* __restrict__ slot, uint4* __restrict__ x_perm) {
   griddep_trigger();  // let the next kernel of the stream start launching
   griddep_wait();     // inputs written by the previous kernel are visible
 
@@ -171,6 +174,7 @@ permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* 
     if (r >= 0 && e >= 0 && e < E) {
       mine = chunk_base[(long long)(t / CH) * E + e] + r;
       src[mine] = t;
+      if (slot) slot[mine] = static_cast<int32_t>(i);
     }
     pos[i] = mine;
   }
@@ -220,7 +224,7 @@ cudaError_t launch_permute_scan(int32_t* chunk_counts, int nchunks, int E, int32
 
 cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* ids, int N, int K,
                                   int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
-                                  void* x_perm, int* status, cudaStream_t stream) {
+                                  int32_t* slot, void* x_perm, int* status, cudaStream_t stream) {
   (void)status;  // bad ids were recorded by the rank pass
   if (N == 0) return cudaSuccess;
   const int row_vecs = row_bytes / 16;
@@ -229,13 +233,13 @@ cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* i
   auto xp = static_cast<uint4*>(x_perm);
   if (K <= 2)
     launch_pdl(permute_gather_kernel<2>, dim3(grid), dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos,
-                                                       src, xp);
+                                                       src, slot, xp);
   else if (K <= 4)
     launch_pdl(permute_gather_kernel<4>, dim3(grid), dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos,
-                                                       src, xp);
+                                                       src, slot, xp);
   else
     launch_pdl(permute_gather_kernel<8>, dim3(grid), dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos,
-                                                       src, xp);
+                                                       src, slot, xp);
   return cudaGetLastError();
 }
 

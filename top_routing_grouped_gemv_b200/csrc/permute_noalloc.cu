@@ -70,7 +70,7 @@ extern "C" moe_status moe_permute_noalloc(moe_plan plan, const void* x, const in
   int* status = device_status_or_null;
   if (moe::launch_permute_count(topk_ids, N, K, E, scratch, perm_pos, status, s) != cudaSuccess ||
       moe::launch_permute_scan(scratch, nchunks, E, counts, offsets, s) != cudaSuccess ||
-      moe::launch_permute_gather(x, row_bytes, topk_ids, N, K, E, scratch, perm_pos, perm_src,
+      moe::launch_permute_gather(x, row_bytes, topk_ids, N, K, E, scratch, perm_pos, perm_src, nullptr,
                                  x_perm, status, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
