@@ -39,6 +39,12 @@ SMALL = {
     "bf16_tc_router_e100_k3": synth.MoEConfig("tc_e100", "bf16", 333, 256, 100, 3, 128, "swiglu",
                                               zipf_bias=1.2),
     "bf16_tc_router_e256_k1": synth.MoEConfig("tc_e256", "bf16", 130, 128, 256, 1, 64, "swiglu"),
+    # few tokens with long rows: split-K router (partial logits per slice of d)
+    "bf16_splitk_e8": synth.MoEConfig("sk_e8", "bf16", 40, 2048, 8, 2, 128, "swiglu"),
+    "bf16_splitk_e256_k8": synth.MoEConfig("sk_e256", "bf16", 130, 1024, 256, 8, 64, "swiglu"),
+    "bf16_splitk_e100_k3": synth.MoEConfig("sk_e100", "bf16", 33, 1536, 100, 3, 64, "swiglu",
+                                           zipf_bias=1.2),
+    "f32_splitk_e16": synth.MoEConfig("sk_f32", "f32", 50, 1024, 16, 4, 64, "relu"),
     # >= 512 routed rows per expert on average: 256-row tiles on CTA pairs
     "bf16_pair": synth.small_variant(synth.BF16_PREFILL, N=1024, d=256, E=4, K=2, F=384),
     "bf16_pair_ragged": synth.small_variant(synth.BF16_PREFILL, N=1300, d=320, E=4, K=2, F=200),

@@ -69,8 +69,12 @@ void mark(moe_plan p, cudaStream_t s, const char* name_of_next) {
 
 bool uses_tensor_cores(const moe_layer_desc& d) { return d.dtype != MOE_F32; }
 
+// Router flavour of a plan: split-K SIMT for few tokens with long rows,
+// else tensor cores for bf16 tokens and many experts, else the per-token
+// SIMT kernels.
+bool router_splitk(const moe_layer_desc& d) { return router_uses_splitk(d.N, d.d); }
 bool router_on_tensor_cores(const moe_layer_desc& d) {
-  return d.dtype == MOE_BF16 && d.E >= kRouterTcMinExperts;
+  return !router_splitk(d) && d.dtype == MOE_BF16 && d.E >= kRouterTcMinExperts;
 }
 
 void layout(moe_plan p) {
@@ -82,7 +86,8 @@ void layout(moe_plan p) {
   L.chunk_counts = off; off = align_up(off + static_cast<size_t>(permute_chunks(d.N)) * d.E * 4);
   L.permute_end = off;
   L.router_w3 = off;
-  if (router_on_tensor_cores(d)) off = align_up(off + router_tc_scratch_bytes(d.d, d.E));
+  if (router_on_tensor_cores(d)) off = align_up(off + router_tc_scratch_bytes(d.N, d.d, d.E));
+  if (router_splitk(d)) off = align_up(off + router_splitk_scratch_bytes(d.N, d.d, d.E));
   L.router_end = off;
   L.h = off;
   if (d.act != MOE_ACT_NONE) off = align_up(off + static_cast<size_t>(R) * d.F * p->eh);
@@ -127,15 +132,16 @@ moe_status run_router(moe_plan p, int n, const void* x, int32_t* ids, float* gat
   const moe_layer_desc& d = p->desc;
   if (router_on_tensor_cores(d)) {
     mark(p, s, "router_tc");
-    p->launches += 2;  // weight split + logits/top-K
+    p->launches += 3;  // weight split + logits + top-K
     return cuda_status(launch_router_tc(x, p->w.w_r, p->w.router_bias, n, d.d, d.E, d.K, ids, gates,
                                         margin, at<void>(ws, p->L.router_w3),
                                         at<int>(ws, p->L.status), s));
   }
-  mark(p, s, "router_topk");
-  p->launches += 1;
+  const bool splitk = router_splitk(d);
+  mark(p, s, splitk ? "router_splitk" : "router_topk");
+  p->launches += splitk ? 2 : 1;  // partial logits + reduction/top-K
   return cuda_status(launch_router(x, d.dtype, p->w.w_r, p->w.router_bias, n, d.d, d.E, d.K, ids,
-                                   gates, margin, s));
+                                   gates, margin, at<void>(ws, p->L.router_w3), s));
 }
 
 // slot (optional): slot[pos] = t*K + j, the destination row of a pure

@@ -37,14 +37,27 @@ enum Act { kActNone = 0, kActRelu = 1, kActSwiglu = 2 };
 inline int dtype_bytes(int dt) { return dt == kF32 ? 4 : dt == kBF16 ? 2 : 1; }
 
 // ---- router -----------------------------------------------------------------
+// SIMT router (fp32 logits, any E <= 256).  Few tokens with long rows
+// (router_uses_splitk) take the split-K form, which needs `scratch` of
+// router_splitk_scratch_bytes for its partial logits; otherwise scratch may
+// be NULL.
 cudaError_t launch_router(const void* x, int x_dtype, const float* w_r, const float* bias, int N,
                           int d, int E, int K, int32_t* ids, float* gates, float* margin,
-                          cudaStream_t stream);
+                          void* scratch, cudaStream_t stream);
+constexpr int kRouterSplitkMaxTokens = 512;
+constexpr size_t kRouterSplitkSmemMax = 96 * 1024;
+bool router_uses_splitk(int N, int d);
+int router_splitk_rows(int d, int E);
+size_t router_splitk_scratch_bytes(int N, int d, int E);
+
+// Top-K, softmax and margin of fp32 logits (N, E) in memory, plus bias.
+cudaError_t launch_logits_topk(const float* logits, const float* bias, int N, int E, int K,
+                              int32_t* ids, float* gates, float* margin, cudaStream_t stream);
 
 // Tensor-core router (bf16 x): splits w_r into three bf16 parts in `scratch`
-// (router_tc_scratch_bytes) and runs the logits on tcgen05; top-K and the
-// softmax in the epilogue.
-size_t router_tc_scratch_bytes(int d, int E);
+// (router_tc_scratch_bytes), runs the logits on tcgen05 into fp32 logits in
+// the same scratch, then the top-K and softmax (launch_logits_topk).
+size_t router_tc_scratch_bytes(int N, int d, int E);
 cudaError_t launch_router_tc(const void* x, const float* w_r, const float* bias, int N, int d,
                              int E, int K, int32_t* ids, float* gates, float* margin,
                              void* scratch, int* status, cudaStream_t stream);

@@ -51,6 +51,53 @@ __device__ __forceinline__ void warp_argmax(const float (&v)[EPL], const bool (&
   }
 }
 
+// Top-K of one token's logits held by a warp (lane l: experts l, l+32, ...;
+// avail marks the real experts), softmax over the kept K, margin = K-th
+// minus (K+1)-th logit (+inf when K = E).  Warp-uniform; writes slot j from
+// lane j.
+template <int EPL>
+__device__ __forceinline__ void write_topk(const float (&v)[EPL], bool (&avail)[EPL], int lane,
+                                           int K, int E, long long t, int32_t* __restrict__ ids,
+                                           float* __restrict__ gates, float* __restrict__ margin) {
+  float sel_v[8];
+  int sel_e[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j >= K) break;  // warp-uniform
+    warp_argmax<EPL>(v, avail, lane, sel_v[j], sel_e[j]);
+#pragma unroll
+    for (int q = 0; q < EPL; ++q)
+      if (lane + 32 * q == sel_e[j]) avail[q] = false;
+  }
+  float next_v = 0.f;
+  if (K < E) {
+    int next_e;
+    warp_argmax<EPL>(v, avail, lane, next_v, next_e);
+  }
+  // softmax over the kept logits, largest first (sel_v[0] is the max)
+  float z = 0.f, my_g = 0.f;
+  int my_e = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < K) {
+      const float p = expf(sel_v[j] - sel_v[0]);
+      z += p;
+      if (j == lane) { my_g = p; my_e = sel_e[j]; }
+    }
+  }
+  if (lane < K) {
+    ids[t * K + lane] = my_e;
+    gates[t * K + lane] = my_g / z;
+  }
+  if (margin != nullptr && lane == 0) {
+    float kth = sel_v[0];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j == K - 1) kth = sel_v[j];
+    margin[t] = (K == E) ? __int_as_float(0x7f800000) : kth - next_v;
+  }
+}
+
 template <typename TX, int EPL, int TPW>
 __global__ void __launch_bounds__(kWarps * 32)
 router_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
@@ -113,43 +160,7 @@ router_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
       avail[q] = e < E;
       v[q] = acc[i][q] + ((bias != nullptr && e < E) ? bias[e] : 0.f);
     }
-    float sel_v[8];
-    int sel_e[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j >= K) break;  // warp-uniform
-      warp_argmax<EPL>(v, avail, lane, sel_v[j], sel_e[j]);
-#pragma unroll
-      for (int q = 0; q < EPL; ++q)
-        if (lane + 32 * q == sel_e[j]) avail[q] = false;
-    }
-    float next_v = 0.f;
-    if (K < E) {
-      int next_e;
-      warp_argmax<EPL>(v, avail, lane, next_v, next_e);
-    }
-    // softmax over the kept logits, largest first (sel_v[0] is the max)
-    float z = 0.f, my_g = 0.f;
-    int my_e = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j < K) {
-        float p = expf(sel_v[j] - sel_v[0]);
-        z += p;
-        if (j == lane) { my_g = p; my_e = sel_e[j]; }
-      }
-    }
-    if (lane < K) {
-      ids[(long long)t * K + lane] = my_e;
-      gates[(long long)t * K + lane] = my_g / z;
-    }
-    if (margin != nullptr && lane == 0) {
-      float kth = sel_v[0];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (j == K - 1) kth = sel_v[j];
-      margin[t] = (K == E) ? __int_as_float(0x7f800000) : kth - next_v;
-    }
+    write_topk<EPL>(v, avail, lane, K, E, t, ids, gates, margin);
   }
 }
 
@@ -273,42 +284,183 @@ router_smem_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
         if (e == lane) v[0] = acc[j][e];
       avail[0] = lane < E;
       if (avail[0] && bias != nullptr) v[0] += bias[lane];
-      float sel_v[8];
-      int sel_e[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (q >= K) break;
-        warp_argmax<1>(v, avail, lane, sel_v[q], sel_e[q]);
-        if (lane == sel_e[q]) avail[0] = false;
-      }
-      float next_v = 0.f;
-      if (K < E) {
-        int next_e;
-        warp_argmax<1>(v, avail, lane, next_v, next_e);
-      }
-      float z = 0.f, my_g = 0.f;
-      int my_e = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (q < K) {
-          const float p = expf(sel_v[q] - sel_v[0]);
-          z += p;
-          if (q == lane) { my_g = p; my_e = sel_e[q]; }
-        }
-      }
-      if (lane < K) {
-        ids[(long long)t * K + lane] = my_e;
-        gates[(long long)t * K + lane] = my_g / z;
-      }
-      if (margin != nullptr && lane == 0) {
-        float kth = sel_v[0];
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q == K - 1) kth = sel_v[q];
-        margin[t] = (K == E) ? __int_as_float(0x7f800000) : kth - next_v;
-      }
+      write_topk<1>(v, avail, lane, K, E, t, ids, gates, margin);
     }
   }
+}
+
+// Split-K router for few tokens and long rows (decode-shaped batches): the
+// per-token kernels above give one warp (or one 128-token tile) per token
+// group and so leave most SMs idle, each streaming the whole of W_r.  Here
+// the reduction dimension is cut into S slices of ks rows: CTA (s, b) stages
+// W_r[ks*s .. ks*s+ks) and the matching x columns of 32 tokens in shared
+// memory and writes their partial logits (k ascending) to part[s][t][e];
+// a second kernel adds the S partials of each (t, e) in slice order (fixed,
+// so results are deterministic) and takes the top-K.
+constexpr int kSkTokens = 32;  // tokens per CTA of the partial kernel
+
+template <typename TX, int EPL>
+__global__ void __launch_bounds__(256)
+router_splitk_kernel(const TX* __restrict__ x, const float* __restrict__ w_r, int N, int d, int E,
+                     int ks, float* __restrict__ part) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
+  constexpr int EP = EPL * 32;
+  extern __shared__ float sk_smem[];
+  float* ws = sk_smem;                 // [ks][EP]
+  float* xs = sk_smem + ks * EP;       // [ks][kSkTokens + 1]
+  const int k0 = blockIdx.x * ks, kn = min(ks, d - k0);
+  const int t0 = blockIdx.y * kSkTokens;
+  for (int idx = threadIdx.x; idx < kn * EP; idx += 256) {
+    const int kk = idx / EP, e = idx % EP;
+    ws[idx] = e < E ? w_r[static_cast<long long>(k0 + kk) * E + e] : 0.f;
+  }
+  for (int idx = threadIdx.x; idx < kSkTokens * kn; idx += 256) {
+    const int t = idx / kn, kk = idx % kn;
+    const int gt = t0 + t;
+    xs[kk * (kSkTokens + 1) + t] = gt < N ? to_f32(x[static_cast<long long>(gt) * d + k0 + kk]) : 0.f;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int TPW = kSkTokens / 8;  // tokens per warp
+  float acc[TPW][EPL];
+#pragma unroll
+  for (int i = 0; i < TPW; ++i)
+#pragma unroll
+    for (int q = 0; q < EPL; ++q) acc[i][q] = 0.f;
+#pragma unroll 4
+  for (int kk = 0; kk < kn; ++kk) {
+    float wv[EPL];
+#pragma unroll
+    for (int q = 0; q < EPL; ++q) wv[q] = ws[kk * EP + lane + 32 * q];
+#pragma unroll
+    for (int i = 0; i < TPW; ++i) {
+      const float xv = xs[kk * (kSkTokens + 1) + warp * TPW + i];
+#pragma unroll
+      for (int q = 0; q < EPL; ++q) acc[i][q] = fmaf(xv, wv[q], acc[i][q]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) {
+    const int t = t0 + warp * TPW + i;
+    if (t >= N) break;  // warp-uniform
+    float* prow = part + (static_cast<long long>(blockIdx.x) * N + t) * E;
+#pragma unroll
+    for (int q = 0; q < EPL; ++q)
+      if (lane + 32 * q < E) prow[lane + 32 * q] = acc[i][q];
+  }
+}
+
+// One CTA of 256 threads per token: thread (g, e) adds the partials of
+// expert e over its share of the slices (slice order), the G shares are
+// added in share order, then warp 0 takes the top-K.
+template <int EPL>
+__global__ void __launch_bounds__(256)
+router_splitk_reduce_kernel(const float* __restrict__ part, const float* __restrict__ bias, int N,
+                            int E, int K, int S, int32_t* __restrict__ ids,
+                            float* __restrict__ gates, float* __restrict__ margin) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
+  constexpr int EP = EPL * 32;
+  constexpr int G = 256 / EP;  // slice shares per expert
+  __shared__ float sums[G][EP];
+  const int t = blockIdx.x;
+  const int e = threadIdx.x % EP, g = threadIdx.x / EP;
+  const int per = (S + G - 1) / G;
+  const int s0 = g * per, s1 = min(S, s0 + per);
+  float a = 0.f;
+  if (e < E) {
+    const float* p = part + static_cast<long long>(t) * E + e;
+    const long long stride = static_cast<long long>(N) * E;
+    int s = s0;
+    for (; s + 4 <= s1; s += 4) {
+      const float v0 = p[s * stride], v1 = p[(s + 1) * stride], v2 = p[(s + 2) * stride],
+                  v3 = p[(s + 3) * stride];
+      a += v0; a += v1; a += v2; a += v3;
+    }
+    for (; s < s1; ++s) a += p[s * stride];
+  }
+  sums[g][e] = a;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    float v[EPL];
+    bool avail[EPL];
+#pragma unroll
+    for (int q = 0; q < EPL; ++q) {
+      const int ee = lane + 32 * q;
+      float tot = 0.f;
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) tot += sums[gg][ee];
+      avail[q] = ee < E;
+      v[q] = tot + ((bias != nullptr && ee < E) ? bias[ee] : 0.f);
+    }
+    write_topk<EPL>(v, avail, lane, K, E, t, ids, gates, margin);
+  }
+}
+
+// Top-K of logits already in memory (the tensor-core router's output): one
+// warp per token, lane l reads experts l, l+32, ...
+template <int EPL>
+__global__ void __launch_bounds__(256)
+logits_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int N, int E,
+                   int K, int32_t* __restrict__ ids, float* __restrict__ gates,
+                   float* __restrict__ margin) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= N) return;  // whole warp
+  const float* row = logits + static_cast<long long>(t) * E;
+  float v[EPL];
+  bool avail[EPL];
+#pragma unroll
+  for (int q = 0; q < EPL; ++q) {
+    const int e = lane + 32 * q;
+    avail[q] = e < E;
+    v[q] = avail[q] ? row[e] + (bias != nullptr ? bias[e] : 0.f) : 0.f;
+  }
+  write_topk<EPL>(v, avail, lane, K, E, t, ids, gates, margin);
+}
+
+template <typename TX, int EPL>
+cudaError_t launch_splitk(const TX* x, const float* w_r, const float* bias, int N, int d, int E,
+                          int K, int32_t* ids, float* gates, float* margin, float* part,
+                          cudaStream_t stream) {
+  constexpr int EP = EPL * 32;
+  const int ks = router_splitk_rows(d, E);
+  const int S = (d + ks - 1) / ks;
+  const size_t smem = static_cast<size_t>(ks) * (EP + kSkTokens + 1) * sizeof(float);
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(router_splitk_kernel<TX, EPL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kRouterSplitkSmemMax));
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  if (smem > kRouterSplitkSmemMax) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(S), static_cast<unsigned>((N + kSkTokens - 1) / kSkTokens));
+  cudaError_t e = launch_pdl(router_splitk_kernel<TX, EPL>, grid, dim3(256), smem, stream, x, w_r,
+                             N, d, E, ks, part);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(router_splitk_reduce_kernel<EPL>, dim3(static_cast<unsigned>(N)), dim3(256), 0,
+                    stream, part, bias, N, E, K, S, ids, gates, margin);
+}
+
+template <typename TX>
+cudaError_t launch_splitk_t(const TX* x, const float* w_r, const float* bias, int N, int d, int E,
+                            int K, int32_t* ids, float* gates, float* margin, float* part,
+                            cudaStream_t stream) {
+  if (E <= 32) return launch_splitk<TX, 1>(x, w_r, bias, N, d, E, K, ids, gates, margin, part, stream);
+  if (E <= 64) return launch_splitk<TX, 2>(x, w_r, bias, N, d, E, K, ids, gates, margin, part, stream);
+  if (E <= 128) return launch_splitk<TX, 4>(x, w_r, bias, N, d, E, K, ids, gates, margin, part, stream);
+  return launch_splitk<TX, 8>(x, w_r, bias, N, d, E, K, ids, gates, margin, part, stream);
 }
 
 constexpr size_t kRouterSmemMax = 160 * 1024;
@@ -376,10 +528,51 @@ cudaError_t launch_t(const TX* x, const float* w_r, const float* bias, int N, in
 
 }  // namespace
 
+cudaError_t launch_logits_topk(const float* logits, const float* bias, int N, int E, int K,
+                              int32_t* ids, float* gates, float* margin, cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  const dim3 grid(static_cast<unsigned>((N + 7) / 8));
+  if (E <= 32)
+    return launch_pdl(logits_topk_kernel<1>, grid, dim3(256), 0, stream, logits, bias, N, E, K, ids, gates, margin);
+  if (E <= 64)
+    return launch_pdl(logits_topk_kernel<2>, grid, dim3(256), 0, stream, logits, bias, N, E, K, ids, gates, margin);
+  if (E <= 128)
+    return launch_pdl(logits_topk_kernel<4>, grid, dim3(256), 0, stream, logits, bias, N, E, K, ids, gates, margin);
+  return launch_pdl(logits_topk_kernel<8>, grid, dim3(256), 0, stream, logits, bias, N, E, K, ids, gates, margin);
+}
+
+int router_splitk_rows(int d, int E) {
+  // about 64 slices, each staging at most kRouterSplitkSmemMax of weights and
+  // token columns; a multiple of 4 rows
+  const int ep = (E + 31) / 32 * 32;
+  const int cap = static_cast<int>(kRouterSplitkSmemMax / ((ep + kSkTokens + 1) * sizeof(float)));
+  int ks = (d + 63) / 64;
+  ks = (ks + 3) / 4 * 4;
+  if (ks > cap) ks = cap / 4 * 4;
+  return ks < 4 ? 4 : ks;
+}
+
+bool router_uses_splitk(int N, int d) { return N <= kRouterSplitkMaxTokens && d >= 1024; }
+
+size_t router_splitk_scratch_bytes(int N, int d, int E) {
+  const int ks = router_splitk_rows(d, E);
+  const long long S = (d + ks - 1) / ks;
+  return static_cast<size_t>(S) * N * E * sizeof(float);
+}
+
 cudaError_t launch_router(const void* x, int x_dtype, const float* w_r, const float* bias, int N,
                           int d, int E, int K, int32_t* ids, float* gates, float* margin,
-                          cudaStream_t stream) {
+                          void* scratch, cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
+  if (router_uses_splitk(N, d)) {
+    if (scratch == nullptr) return cudaErrorInvalidValue;
+    float* part = static_cast<float*>(scratch);
+    if (x_dtype == kF32)
+      return launch_splitk_t(static_cast<const float*>(x), w_r, bias, N, d, E, K, ids, gates,
+                             margin, part, stream);
+    return launch_splitk_t(static_cast<const __nv_bfloat16*>(x), w_r, bias, N, d, E, K, ids, gates,
+                           margin, part, stream);
+  }
   if (x_dtype == kF32)
     return launch_t(static_cast<const float*>(x), w_r, bias, N, d, E, K, ids, gates, margin,
                     stream);

@@ -18,10 +18,13 @@
 // Structure: one CTA per 128-token tile (persistent), warp 0 streams x and
 // weight tiles with TMA into a 4-stage ring, warp 1 issues the MMAs into two
 // TMEM accumulators (one per expert chunk, double-buffered), warps 2..5 (one
-// token row per thread) add the three parts and the bias and keep a running
-// top-(K+1) list in registers over the chunks, expert index ascending, so
-// equal logits keep the lower index.  Then the softmax over the K kept
-// logits and the margin (K-th minus (K+1)-th logit).
+// token row per thread) add the three parts and store the fp32 logits.  A
+// warp-per-token kernel then takes the top-K (value desc, index asc), the
+// softmax over the kept K and the margin, shared with the SIMT routers.
+// (Keeping a running top-(K+1) list per thread in the epilogue instead made
+// the epilogue, one warp per SM sub-partition on serial compare chains, the
+// bound: 116 us against 44 us without it on the 16384-token, 128-expert
+// workload.)
 #include <float.h>
 #include <limits.h>
 #include <string.h>
@@ -80,11 +83,8 @@ router_split_kernel(const float* __restrict__ w_r, int d, int E, int nchunks,
 struct RouterTcArgs {
   CUtensorMap tmX;  // x: rows N, cols d, 128-row boxes
   CUtensorMap tmW;  // split weights: rows nchunks*256, cols d, 256-row boxes
-  int N, d, E, K, nchunks;
-  const float* bias;
-  int32_t* ids;
-  float* gates;
-  float* margin;
+  int N, d, E, nchunks;
+  float* logits;  // (N, E) fp32
   int* status;
 };
 
@@ -136,6 +136,10 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(const __grid_co
   const int ntiles = (args.N + RM - 1) / RM;
   const int num_kb = (args.d + 63) / 64;
   const int nchunks = args.nchunks;
+  // Every CTA reads the same split-weight tiles; starting each CTA's k loop
+  // at a different block (rotated order) spreads those reads over the L2
+  // instead of sending all CTAs to the same lines at once.
+  const int kb_first = static_cast<int>(blockIdx.x % static_cast<unsigned>(num_kb));
 
   if (warp == 0) {
     if (lane == 0) {  // ---- TMA producer ----
@@ -144,7 +148,8 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(const __grid_co
       bool aborted = false;
       for (int t = blockIdx.x; t < ntiles && !aborted; t += gridDim.x)
         for (int c = 0; c < nchunks && !aborted; ++c)
-          for (int kb = 0; kb < num_kb; ++kb) {
+          for (int j = 0; j < num_kb; ++j) {
+            const int kb = kb_first + j < num_kb ? kb_first + j : kb_first + j - num_kb;
             if (!mbar_wait(bar(kRBarEmpty + s), ph ^ 1u, abort_flag)) { aborted = true; break; }
             mbar_expect_tx(bar(kRBarFull + s), RSTAGE_BYTES);
             tma_load_2d(sA + s * RA_BYTES, &args.tmX, kb * 64, t * RM, bar(kRBarFull + s));
@@ -167,14 +172,14 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(const __grid_co
           if (!mbar_wait(bar(kRBarTEmpty + acc), aph ^ 1u, abort_flag)) { aborted = true; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * RN);
-          for (int kb = 0; kb < num_kb; ++kb) {
+          for (int j = 0; j < num_kb; ++j) {  // k blocks in the producer's rotated order
             if (!mbar_wait(bar(kRBarFull + s), ph, abort_flag)) { aborted = true; break; }
             tc_fence_after();
             const uint32_t a0 = sA + s * RA_BYTES, b0 = sB + s * RB_BYTES;
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               tc_mma<false>(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), kRouterIdesc,
-                            (kb | k) != 0 ? 1u : 0u);
+                            (j | k) != 0 ? 1u : 0u);
             tc_commit(bar(kRBarEmpty + s));
             if (++s == RSTAGES) { s = 0; ph ^= 1u; }
           }
@@ -188,14 +193,13 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(const __grid_co
     // ---- epilogue: one token row per thread ----
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    const int K = args.K, E = args.E;
+    const int E = args.E;
+    const bool vec = (E & 3) == 0;
     int i = 0;
     bool aborted = false;
     for (int t = blockIdx.x; t < ntiles && !aborted; t += gridDim.x) {
-      float tv[9];
-      int te[9];
-#pragma unroll
-      for (int j = 0; j < 9; ++j) { tv[j] = -FLT_MAX; te[j] = INT_MAX; }
+      const long long tok = static_cast<long long>(t) * RM + row;
+      float* lrow = args.logits + tok * E;
       for (int c = 0; c < nchunks; ++c, ++i) {
         const int acc = i & 1;
         const uint32_t aph = (i >> 1) & 1;
@@ -217,58 +221,27 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(const __grid_co
           tmem_ld32(tb + REC + h, vm);
           tmem_ld32(tb + 2 * REC + h, vl);
           tmem_ld_wait();
+          float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int e = c * REC + h + j;
-            if (e < E) {
-              float v = (__uint_as_float(vh[j]) + __uint_as_float(vm[j])) + __uint_as_float(vl[j]);
-              if (args.bias) v += args.bias[e];
-              // insert, keeping (value desc, index asc): equal values do not
-              // overtake the earlier (lower-index) entry
-              float cv = v;
-              int ce = e;
+          for (int j = 0; j < 32; ++j)
+            v[j] = (__uint_as_float(vh[j]) + __uint_as_float(vm[j])) + __uint_as_float(vl[j]);
+          const int e0 = c * REC + h;
+          if (tok < args.N && e0 < E) {
+            if (vec && e0 + 32 <= E) {
+              float4* dst = reinterpret_cast<float4*>(lrow + e0);
 #pragma unroll
-              for (int s2 = 0; s2 < 9; ++s2) {
-                if (cv > tv[s2] || (cv == tv[s2] && te[s2] == INT_MAX)) {
-                  const float fv = tv[s2];
-                  const int fe = te[s2];
-                  tv[s2] = cv;
-                  te[s2] = ce;
-                  cv = fv;
-                  ce = fe;
-                }
-              }
+              for (int j = 0; j < 8; ++j)
+                dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (e0 + j < E) lrow[e0 + j] = v[j];
             }
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kRBarTEmpty + acc));
-      }
-      if (aborted) break;
-      const long long tok = static_cast<long long>(t) * RM + row;
-      if (tok < args.N) {
-        float z = 0.f, p[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          p[j] = 0.f;
-          if (j < K) {
-            p[j] = expf(tv[j] - tv[0]);
-            z += p[j];
-          }
-        }
-        float kth = tv[0], next = tv[0];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j < K) {
-            args.ids[tok * K + j] = te[j];
-            args.gates[tok * K + j] = p[j] / z;
-          }
-          if (j == K - 1) kth = tv[j];
-          if (j == K) next = tv[j];
-        }
-        if (K == 8) next = tv[8];
-        if (args.margin) args.margin[tok] = (K == E) ? __int_as_float(0x7f800000) : kth - next;
       }
     }
   }
@@ -286,9 +259,15 @@ __global__ void __launch_bounds__(kRThreads, 1) router_tc_kernel(const __grid_co
 
 }  // namespace
 
-size_t router_tc_scratch_bytes(int d, int E) {
+// scratch: the split weights (nchunks * 256 rows of d bf16), then the fp32
+// logits (N, E)
+static size_t split_weight_bytes(int d, int E) {
   const int nchunks = (E + REC - 1) / REC;
   return static_cast<size_t>(nchunks) * RN * d * sizeof(__nv_bfloat16);
+}
+
+size_t router_tc_scratch_bytes(int N, int d, int E) {
+  return split_weight_bytes(d, E) + static_cast<size_t>(N) * E * sizeof(float);
 }
 
 cudaError_t launch_router_tc(const void* x, const float* w_r, const float* bias, int N, int d,
@@ -314,12 +293,8 @@ cudaError_t launch_router_tc(const void* x, const float* w_r, const float* bias,
   a.N = N;
   a.d = d;
   a.E = E;
-  a.K = K;
   a.nchunks = nchunks;
-  a.bias = bias;
-  a.ids = ids;
-  a.gates = gates;
-  a.margin = margin;
+  a.logits = reinterpret_cast<float*>(static_cast<char*>(scratch) + split_weight_bytes(d, E));
   a.status = status;
   static int configured[64] = {0};
   int dev = 0;
@@ -332,8 +307,10 @@ cudaError_t launch_router_tc(const void* x, const float* w_r, const float* bias,
   }
   const int ntiles = (N + RM - 1) / RM;
   const int grid = ntiles < device_sm_count() ? ntiles : device_sm_count();
-  launch_pdl(router_tc_kernel, dim3(grid), dim3(kRThreads), kRSmemBytes, stream, a);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(router_tc_kernel, dim3(grid), dim3(kRThreads), kRSmemBytes, stream, a);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_logits_topk(a.logits, bias, N, E, K, ids, gates, margin, stream);
 }
 
 }  // namespace moe
