@@ -3,10 +3,11 @@
 // y[t*K+j] = y_perm[pos[t,j]] (aclnnQuantGroupedMatMulAlltoAllv formula:
 // unpermuteOut = Unpermute(gmmY), output (BSK, N1)).
 //
-// One warp per output token (gated) or per output row (reorder).  Each lane
-// moves 16-byte vectors; the K source rows of a token are read with
-// coalesced 512-byte warp accesses and accumulated in fp32 in slot order
-// j = 0..K-1, then rounded once to the output dtype.
+// WPT warps per output token (gated; more than one for small batches, the
+// row's 16-byte vectors split between them) or one warp per output row
+// (reorder).  The K source rows of a token are read with coalesced 512-byte
+// warp accesses and accumulated in fp32 in slot order j = 0..K-1, then
+// rounded once to the output dtype.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -38,7 +39,7 @@ template <> struct Vec<__nv_bfloat16> {
   }
 };
 
-template <typename T, int KMAX>
+template <typename T, int KMAX, int WPT>
 __global__ void __launch_bounds__(256)
 combine_kernel(const uint4* __restrict__ y_perm, int row_vecs, const int32_t* __restrict__ pos,
                const float* __restrict__ gates, int N, int K, int R, uint4* __restrict__ y,
@@ -46,8 +47,9 @@ combine_kernel(const uint4* __restrict__ y_perm, int row_vecs, const int32_t* __
   griddep_trigger();  // let the next kernel of the stream start launching
   griddep_wait();     // inputs written by the previous kernel are visible
 
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * (8 / WPT) + warp / WPT;
+  const int sub = warp % WPT;
   if (t >= N) return;
   int p[KMAX];
   float g[KMAX];
@@ -67,7 +69,7 @@ combine_kernel(const uint4* __restrict__ y_perm, int row_vecs, const int32_t* __
     g[j] = __shfl_sync(0xffffffffu, mine_g, j);
   }
   constexpr int n = Vec<T>::n;
-  for (int v = lane; v < row_vecs; v += 32) {
+  for (int v = sub * 32 + lane; v < row_vecs; v += 32 * WPT) {
     float acc[n];
 #pragma unroll
     for (int i = 0; i < n; ++i) acc[i] = 0.f;
@@ -112,16 +114,27 @@ unpermute_kernel(const uint4* __restrict__ y_perm, int row_vecs, const int32_t* 
   for (; v < row_vecs; v += 32) d[v] = s[v];
 }
 
+template <typename T, int KMAX>
+void launch_gated_k(const uint4* yp, int row_vecs, const int32_t* pos, const float* gates, int N,
+                    int K, int R, uint4* y, int* status, cudaStream_t stream) {
+  const int wpt = warps_per_token(N);
+  const dim3 grid((N + 8 / wpt - 1) / (8 / wpt));
+  if (wpt == 1)
+    launch_pdl(combine_kernel<T, KMAX, 1>, grid, dim3(256), 0, stream, yp, row_vecs, pos, gates, N, K, R, y, status);
+  else if (wpt == 2)
+    launch_pdl(combine_kernel<T, KMAX, 2>, grid, dim3(256), 0, stream, yp, row_vecs, pos, gates, N, K, R, y, status);
+  else if (wpt == 4)
+    launch_pdl(combine_kernel<T, KMAX, 4>, grid, dim3(256), 0, stream, yp, row_vecs, pos, gates, N, K, R, y, status);
+  else
+    launch_pdl(combine_kernel<T, KMAX, 8>, grid, dim3(256), 0, stream, yp, row_vecs, pos, gates, N, K, R, y, status);
+}
+
 template <typename T>
 void launch_gated(const uint4* yp, int row_vecs, const int32_t* pos, const float* gates, int N,
                   int K, int R, uint4* y, int* status, cudaStream_t stream) {
-  int grid = (N + 7) / 8;
-  if (K <= 2)
-    launch_pdl(combine_kernel<T, 2>, dim3(grid), dim3(256), 0, stream, yp, row_vecs, pos, gates, N, K, R, y, status);
-  else if (K <= 4)
-    launch_pdl(combine_kernel<T, 4>, dim3(grid), dim3(256), 0, stream, yp, row_vecs, pos, gates, N, K, R, y, status);
-  else
-    launch_pdl(combine_kernel<T, 8>, dim3(grid), dim3(256), 0, stream, yp, row_vecs, pos, gates, N, K, R, y, status);
+  if (K <= 2) launch_gated_k<T, 2>(yp, row_vecs, pos, gates, N, K, R, y, status, stream);
+  else if (K <= 4) launch_gated_k<T, 4>(yp, row_vecs, pos, gates, N, K, R, y, status, stream);
+  else launch_gated_k<T, 8>(yp, row_vecs, pos, gates, N, K, R, y, status, stream);
 }
 
 }  // namespace

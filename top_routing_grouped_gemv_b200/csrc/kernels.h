@@ -138,6 +138,16 @@ constexpr int kTcBlockN = 256;  // accumulator columns; SwiGLU: 128 gate + 128 u
 
 int device_sm_count();
 
+// Warps per token row for the row-copy kernels (gather, combine): the
+// smallest of 1, 2, 4, 8 that puts about 16 warps per SM in flight.
+inline int warps_per_token(int N) {
+  const long long want = 16LL * device_sm_count();
+  if (N >= want) return 1;
+  if (2LL * N >= want) return 2;
+  if (4LL * N >= want) return 4;
+  return 8;
+}
+
 // Shape of a plan for code outside the plan's translation unit: tokens,
 // token width, experts, experts per token and bytes per token row of x.
 // Returns false for a null plan.

@@ -7,10 +7,13 @@
 // Stable order: within expert e the rows appear in (token, slot) order, so
 //   pos[t,j] = offsets[e] + #{(t',j') before (t,j) with ids[t',j'] = e}.
 // Tokens are cut into chunks of kPermuteChunk (32).  Three launches:
-//   1. rank:   one warp per chunk ranks the chunk's (t, j) pairs with
-//              shuffles (no atomics in the ranks, so the order is fixed),
-//              writes each pair's rank within its chunk (into perm_pos) and
-//              the chunk's expert histogram (chunk_counts)
+//   1. rank:   one warp per chunk ranks the chunk's (t, j) pairs: each lane
+//              (token) sets its bit in a per-expert 32-bit mask, and the
+//              rank of (t, j) is the number of lower lanes in the mask of
+//              its expert (a token whose K experts are not distinct takes a
+//              shuffle-based count instead); writes each pair's rank within
+//              its chunk (into perm_pos) and the chunk's expert histogram
+//              (chunk_counts).  Either way the order is fixed.
 //   2. scan:   one CTA turns chunk_counts into per-(chunk, expert) bases
 //              (offsets[e] + rows of e in earlier chunks), counts, offsets
 //   3. gather: one warp per token turns its ranks into final positions and
@@ -36,11 +39,15 @@ permute_rank_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
   griddep_wait();     // inputs written by the previous kernel are visible
 
   __shared__ int hist[4][256];
+  __shared__ unsigned lanes_of[4][256];  // bit l: lane (token) l routes to the expert
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int c = blockIdx.x * 4 + warp;
   const int nchunks = (N + CH - 1) / CH;
   if (c >= nchunks) return;  // whole warp
-  for (int e = lane; e < E; e += 32) hist[warp][e] = 0;
+  for (int e = lane; e < E; e += 32) {
+    hist[warp][e] = 0;
+    lanes_of[warp][e] = 0u;
+  }
   __syncwarp();
   const int t = c * CH + lane;
   int my[KMAX];
@@ -55,23 +62,39 @@ permute_rank_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
   }
   // rank of (t, j): earlier slots of t with the same expert ...
   int rank[KMAX];
+  bool repeated = false;
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
     rank[j] = 0;
 #pragma unroll
     for (int jj = 0; jj < KMAX; ++jj)
-      if (jj < j && my[jj] == my[j]) rank[j]++;
+      if (jj < j && my[jj] == my[j] && my[j] >= 0) {
+        rank[j]++;
+        repeated = true;
+      }
   }
   // ... plus every slot of the earlier tokens of this chunk with that expert
+  if (!__any_sync(0xffffffffu, repeated)) {
+    // K distinct experts per token: one bit per (token, expert)
 #pragma unroll
-  for (int jj = 0; jj < KMAX; ++jj) {
-    if (jj >= K) break;
-    for (int sl = 0; sl < 31; ++sl) {
-      const int v = __shfl_sync(0xffffffffu, my[jj], sl);
-      if (sl < lane) {
+    for (int j = 0; j < KMAX; ++j)
+      if (my[j] >= 0) atomicOr(&lanes_of[warp][my[j]], 1u << lane);
+    __syncwarp();
+    const unsigned below = (1u << lane) - 1u;
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j)
-          if (v == my[j] && v >= 0) rank[j]++;
+    for (int j = 0; j < KMAX; ++j)
+      if (my[j] >= 0) rank[j] = __popc(lanes_of[warp][my[j]] & below);
+  } else {
+#pragma unroll
+    for (int jj = 0; jj < KMAX; ++jj) {
+      if (jj >= K) break;
+      for (int sl = 0; sl < 31; ++sl) {
+        const int v = __shfl_sync(0xffffffffu, my[jj], sl);
+        if (sl < lane) {
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j)
+            if (v == my[j] && v >= 0) rank[j]++;
+        }
       }
     }
   }
@@ -152,9 +175,12 @@ permute_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
   }
 }
 
-// One warp per token: final positions from the chunk bases and the ranks,
-// then one read of the token row and K writes.
-template <int KMAX>
+// WPT warps per token (8 / WPT tokens per CTA): final positions from the
+// chunk bases and the ranks (the token's first warp, shared through shared
+// memory), then one read of the token row and K writes, the row's 16-byte
+// vectors split over the token's warps.  WPT > 1 spreads a small batch over
+// more SMs.
+template <int KMAX, int WPT>
 __global__ void __launch_bounds__(256)
 permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* __restrict__ ids,
                       int N, int K, int E, const int32_t* __restrict__ chunk_base,
@@ -163,41 +189,66 @@ permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* 
   griddep_trigger();  // let the next kernel of the stream start launching
   griddep_wait();     // inputs written by the previous kernel are visible
 
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= N) return;
-  int mine = -1;
-  if (lane < K) {
-    const long long i = (long long)t * K + lane;
-    const int e = ids[i];
-    const int r = pos[i];  // rank within the chunk (written by the rank pass)
-    if (r >= 0 && e >= 0 && e < E) {
-      mine = chunk_base[(long long)(t / CH) * E + e] + r;
-      src[mine] = t;
-      if (slot) slot[mine] = static_cast<int32_t>(i);
+  __shared__ int sp[8 / WPT][KMAX];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tl = warp / WPT, sub = warp % WPT;
+  const int t = blockIdx.x * (8 / WPT) + tl;
+  if (t < N && sub == 0 && lane < KMAX) {
+    int mine = -1;
+    if (lane < K) {
+      const long long i = (long long)t * K + lane;
+      const int e = ids[i];
+      const int r = pos[i];  // rank within the chunk (written by the rank pass)
+      if (r >= 0 && e >= 0 && e < E) {
+        mine = chunk_base[(long long)(t / CH) * E + e] + r;
+        src[mine] = t;
+        if (slot) slot[mine] = static_cast<int32_t>(i);
+      }
+      pos[i] = mine;
     }
-    pos[i] = mine;
+    sp[tl][lane] = mine;
   }
+  if constexpr (WPT > 1) __syncthreads();
+  else __syncwarp();
+  if (t >= N) return;
   int p[KMAX];
 #pragma unroll
-  for (int j = 0; j < KMAX; ++j) p[j] = __shfl_sync(0xffffffffu, mine, j);
+  for (int j = 0; j < KMAX; ++j) p[j] = sp[tl][j];
   const uint4* srow = x + (long long)t * row_vecs;
-  int v = lane;
-  for (; v + 96 < row_vecs; v += 128) {
-    const uint4 a0 = srow[v], a1 = srow[v + 32], a2 = srow[v + 64], a3 = srow[v + 96];
+  constexpr int STEP = 32 * WPT;
+  int v = sub * 32 + lane;
+  for (; v + 3 * STEP < row_vecs; v += 4 * STEP) {
+    const uint4 a0 = srow[v], a1 = srow[v + STEP], a2 = srow[v + 2 * STEP], a3 = srow[v + 3 * STEP];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
       if (j >= K || p[j] < 0) continue;
       uint4* drow = x_perm + (long long)p[j] * row_vecs;
-      drow[v] = a0; drow[v + 32] = a1; drow[v + 64] = a2; drow[v + 96] = a3;
+      drow[v] = a0; drow[v + STEP] = a1; drow[v + 2 * STEP] = a2; drow[v + 3 * STEP] = a3;
     }
   }
-  for (; v < row_vecs; v += 32) {
+  for (; v < row_vecs; v += STEP) {
     const uint4 a0 = srow[v];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j)
       if (j < K && p[j] >= 0) x_perm[(long long)p[j] * row_vecs + v] = a0;
   }
+}
+
+template <int KMAX>
+void launch_gather_k(const uint4* xv, int row_vecs, const int32_t* ids, int N, int K, int E,
+                     const int32_t* chunk_base, int32_t* pos, int32_t* src, int32_t* slot,
+                     uint4* xp, cudaStream_t stream) {
+  const int wpt = warps_per_token(N);
+  const int tpc = 8 / wpt;
+  const dim3 grid((N + tpc - 1) / tpc);
+  if (wpt == 1)
+    launch_pdl(permute_gather_kernel<KMAX, 1>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp);
+  else if (wpt == 2)
+    launch_pdl(permute_gather_kernel<KMAX, 2>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp);
+  else if (wpt == 4)
+    launch_pdl(permute_gather_kernel<KMAX, 4>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp);
+  else
+    launch_pdl(permute_gather_kernel<KMAX, 8>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp);
 }
 
 }  // namespace
@@ -228,18 +279,14 @@ cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* i
   (void)status;  // bad ids were recorded by the rank pass
   if (N == 0) return cudaSuccess;
   const int row_vecs = row_bytes / 16;
-  const int grid = (N + 7) / 8;
   auto xv = static_cast<const uint4*>(x);
   auto xp = static_cast<uint4*>(x_perm);
   if (K <= 2)
-    launch_pdl(permute_gather_kernel<2>, dim3(grid), dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos,
-                                                       src, slot, xp);
+    launch_gather_k<2>(xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, stream);
   else if (K <= 4)
-    launch_pdl(permute_gather_kernel<4>, dim3(grid), dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos,
-                                                       src, slot, xp);
+    launch_gather_k<4>(xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, stream);
   else
-    launch_pdl(permute_gather_kernel<8>, dim3(grid), dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos,
-                                                       src, slot, xp);
+    launch_gather_k<8>(xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, stream);
   return cudaGetLastError();
 }
 
