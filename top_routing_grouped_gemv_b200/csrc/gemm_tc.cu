@@ -9,6 +9,10 @@
 //   kEpiStore : out = bf16(acc * scale)
 //   kEpiSwiglu: out = bf16(silu(acc_gate) * acc_up)  (the weight tile holds
 //               128 gate rows followed by 128 up rows of the same outputs)
+//   kEpiRouter: out = fp32 router logits (hi + mid) + lo  (the weight tile
+//               holds three bf16 parts of 64 experts' fp32 router weights
+//               and 64 zero rows: columns [0,64) hi, [64,128) mid,
+//               [128,192) lo; one group, rows = tokens)
 //
 // Structure (one persistent CTA per SM, 6 warps):
 //   warp 0      TMA producer: 128-byte-swizzled K-major tiles of A (128 rows)
@@ -312,7 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const TileCoord c = decode_tile<Gm::TILE_M>(T, s_pref, s_off, G);
       // lane quadrant q holds rows 32q.. of this CTA's 128 rows of the tile
       const int row = static_cast<int>(rank) * BM + q * 32 + lane;
-      constexpr int span = kEpi == kEpiSwiglu ? BN / 2 : BN;  // output columns of the tile
+      // output columns of the tile
+      constexpr int span = kEpi == kEpiSwiglu ? BN / 2 : kEpi == kEpiRouter ? BN / 4 : BN;
       const int col0 = c.n_tile * span;
       const long long grow = static_cast<long long>(c.m_row0) + row;
       const bool valid = grow < s_off[c.g + 1] && grow < args.m_total && grow >= 0;
@@ -321,7 +326,36 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       long long orow_i = grow;
       if (valid && args.out_rows != nullptr) orow_i = args.out_rows[grow];
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + orow_i * args.ldo;
-      if (kEpi == kEpiSwiglu) {
+      if constexpr (kEpi == kEpiRouter) {
+        float* frow = static_cast<float*>(args.out) + orow_i * args.ldo;
+        const bool vec4 = (args.ldo & 3) == 0;
+#pragma unroll 1
+        for (int cc = 0; cc < span; cc += 32) {
+          uint32_t vh[32], vm[32], vl[32];
+          __syncwarp();
+          tmem_ld32(tbase + cc, vh);             // hi part
+          tmem_ld32(tbase + span + cc, vm);      // mid part
+          tmem_ld32(tbase + 2 * span + cc, vl);  // lo part
+          tmem_ld_wait();
+          const int col = col0 + cc;
+          if (valid && col < args.n_out) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              v[j] = (__uint_as_float(vh[j]) + __uint_as_float(vm[j])) + __uint_as_float(vl[j]);
+            if (vec4 && col + 32 <= args.n_out) {
+              float4* dst = reinterpret_cast<float4*>(frow + col);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col + j < args.n_out) frow[col + j] = v[j];
+            }
+          }
+        }
+      } else if (kEpi == kEpiSwiglu) {
 #pragma unroll 1
         for (int cc = 0; cc < span; cc += 32) {
           uint32_t gr[32], ur[32];
@@ -505,6 +539,10 @@ cudaError_t launch_gemm_tc(const TcGemmArgs& args, int dtype, int epilogue, int 
   if (max_units <= 0) return cudaSuccess;
   const bool fp8 = dtype == kE4M3;
   const bool sw = epilogue == kEpiSwiglu;
+  if (epilogue == kEpiRouter) {
+    if (pair || fp8) return cudaErrorInvalidValue;
+    return launch_t<false, kEpiRouter, false>(args, max_units, stream);
+  }
   if (pair) {
     if (fp8) return sw ? launch_t<true, kEpiSwiglu, true>(args, max_units, stream)
                        : launch_t<true, kEpiStore, true>(args, max_units, stream);

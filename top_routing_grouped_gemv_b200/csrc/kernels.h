@@ -96,7 +96,9 @@ cudaError_t launch_gemm_simt_f32(const float* A, int kdim, const float* W, const
                                  int R, float* out, cudaStream_t stream);
 
 // ---- grouped GEMM on tcgen05 tensor cores -----------------------------------
-enum TcEpilogue { kEpiStore = 0, kEpiSwiglu = 1 };
+// kEpiRouter: fp32 logits from the three-part split router weights (bf16,
+// single-CTA tiles only).
+enum TcEpilogue { kEpiStore = 0, kEpiSwiglu = 1, kEpiRouter = 2 };
 
 struct TcGemmArgs {
   CUtensorMap tmA;   // activations: rows (R), cols kdim
@@ -108,7 +110,7 @@ struct TcGemmArgs {
   int kdim;
   int n_out;               // output columns per group
   int n_tiles;             // output column tiles per group
-  void* out;               // bf16 (rows, ldo)
+  void* out;               // bf16 (rows, ldo); fp32 for kEpiRouter
   long long ldo;           // elements
   float scale;             // multiplies the fp32 accumulator before rounding
   // finer scales (store epilogue): out = acc * scale * row_scale[row'] *

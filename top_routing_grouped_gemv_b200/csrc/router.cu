@@ -24,31 +24,41 @@ namespace {
 constexpr int kKC = 32;       // k rows per shared-memory chunk
 constexpr int kWarps = 8;
 
+// Order-preserving 32-bit key of a float (larger float -> larger key; -0
+// and +0 share the key of +0) and its inverse.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t b = __float_as_uint(f);
+  if ((b & 0x7fffffffu) == 0u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 // One round of the warp-wide argmax over the still-available logits of a
 // token (lane l holds experts l, l+32, ...): the larger value wins, equal
-// values go to the lower expert index.  Every lane returns the winner.
+// values go to the lower expert index.  Every lane returns the winner.  Two
+// warp reductions (redux.sync): the largest key, then the smallest expert
+// index among the lanes whose best entry carries that key.
 template <int EPL>
 __device__ __forceinline__ void warp_argmax(const float (&v)[EPL], const bool (&avail)[EPL],
                                             int lane, float& bv, int& be) {
-  bv = -FLT_MAX;
-  be = INT_MAX;
+  uint32_t mk = 0u;
+  int mi = INT_MAX;
 #pragma unroll
   for (int q = 0; q < EPL; ++q) {
-    const int e = lane + 32 * q;
-    if (avail[q] && (be == INT_MAX || v[q] > bv || (v[q] == bv && e < be))) {
-      bv = v[q];
-      be = e;
+    const uint32_t k = order_key(v[q]);
+    if (avail[q] && (mi == INT_MAX || k > mk)) {  // q ascending: ties keep the lower index
+      mk = k;
+      mi = lane + 32 * q;
     }
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-    if (oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be))) {
-      bv = ov;
-      be = oe;
-    }
-  }
+  const uint32_t wk = __reduce_max_sync(0xffffffffu, mi != INT_MAX ? mk : 0u);
+  const uint32_t wi =
+      __reduce_min_sync(0xffffffffu, (mi != INT_MAX && mk == wk) ? static_cast<uint32_t>(mi)
+                                                                 : 0xffffffffu);
+  be = wi == 0xffffffffu ? INT_MAX : static_cast<int>(wi);
+  bv = key_value(wk);
 }
 
 // Top-K of one token's logits held by a warp (lane l: experts l, l+32, ...;
