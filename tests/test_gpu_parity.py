@@ -49,6 +49,8 @@ SMALL = {
     "bf16_pair": synth.small_variant(synth.BF16_PREFILL, N=1024, d=256, E=4, K=2, F=384),
     "bf16_pair_ragged": synth.small_variant(synth.BF16_PREFILL, N=1300, d=320, E=4, K=2, F=200),
     "bf16_pair_zipf": synth.small_variant(synth.BF16_FINEGRAINED, N=2100, d=256, E=8, K=2, F=256),
+    # >= 2048 rows per expert: the SwiGLU gate/up GEMM pairs as well
+    "bf16_pair_swiglu": synth.MoEConfig("pair_sw", "bf16", 4100, 128, 2, 1, 256, "swiglu"),
     "e4m3_pair": synth.small_variant(synth.FP8_GMM, N=1100, d=256, E=4, K=2, F=392,
                                      shared=(256, 392)),
 }

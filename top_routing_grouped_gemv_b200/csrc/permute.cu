@@ -125,9 +125,19 @@ permute_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
   const int e = threadIdx.x % Ep, s = threadIdx.x / Ep;
   const int cs = (nchunks + S - 1) / S;
   const int c0 = s * cs, c1 = min(nchunks, c0 + cs);
+  // (chunk loops batched by 8 so that loads overlap)
   int sum = 0;
-  if (e < E)
-    for (int c = c0; c < c1; ++c) sum += chunk_counts[(long long)c * E + e];
+  if (e < E) {
+    int c = c0;
+    for (; c + 8 <= c1; c += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = chunk_counts[(long long)(c + u) * E + e];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sum += v[u];
+    }
+    for (; c < c1; ++c) sum += chunk_counts[(long long)c * E + e];
+  }
   part[threadIdx.x] = sum;
   __syncthreads();
   // exclusive scan over the slices of each expert
@@ -167,8 +177,19 @@ permute_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
   __syncthreads();
   if (e < E) {
     int run = total[e] + part[s * Ep + e];
-    for (int c = c0; c < c1; ++c) {
-      int v = chunk_counts[(long long)c * E + e];
+    int c = c0;
+    for (; c + 8 <= c1; c += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = chunk_counts[(long long)(c + u) * E + e];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        chunk_counts[(long long)(c + u) * E + e] = run;
+        run += v[u];
+      }
+    }
+    for (; c < c1; ++c) {
+      const int v = chunk_counts[(long long)c * E + e];
       chunk_counts[(long long)c * E + e] = run;
       run += v;
     }

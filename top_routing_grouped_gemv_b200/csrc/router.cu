@@ -207,17 +207,42 @@ router_smem_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
     const int c = (e * VEC + i) >> 2;
     wf[((long long)m * CPB + (c ^ (m & 7))) * 4 + (i & 3)] = v;
   };
+  // eight loads in flight per thread before their shared-memory stores
+  constexpr int kBatch = 8;
   if (E == E_T && (E & 3) == 0) {  // whole rows, 16-byte loads
     const float4* w4 = reinterpret_cast<const float4*>(w_r);
-    for (int idx = threadIdx.x; idx < d * E / 4; idx += blockDim.x) {
-      const float4 v = w4[idx];
-      const int k = idx * 4 / E, e = idx * 4 % E;
-      put(k, e, v.x); put(k, e + 1, v.y); put(k, e + 2, v.z); put(k, e + 3, v.w);
+    const int n4 = d * E / 4;
+    for (int base = threadIdx.x; base < n4; base += kBatch * blockDim.x) {
+      float4 v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = base + u * blockDim.x;
+        if (idx < n4) v[u] = w4[idx];
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = base + u * blockDim.x;
+        if (idx < n4) {
+          const int k = idx * 4 / E, e = idx * 4 % E;
+          put(k, e, v[u].x); put(k, e + 1, v[u].y); put(k, e + 2, v[u].z); put(k, e + 3, v[u].w);
+        }
+      }
     }
   } else {
-    for (int idx = threadIdx.x; idx < d * E_T; idx += blockDim.x) {
-      const int k = idx / E_T, e = idx % E_T;
-      put(k, e, e < E ? w_r[(long long)k * E + e] : 0.f);
+    const int n = d * E_T;
+    for (int base = threadIdx.x; base < n; base += kBatch * blockDim.x) {
+      float v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = base + u * blockDim.x;
+        const int k = idx / E_T, e = idx % E_T;
+        v[u] = (idx < n && e < E) ? w_r[(long long)k * E + e] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = base + u * blockDim.x;
+        if (idx < n) put(idx / E_T, idx % E_T, v[u]);
+      }
     }
   }
   __syncthreads();
