@@ -62,6 +62,7 @@ def lib():
                                          i, P, P, P, P]
         L.orc_dense_masked.argtypes = [i, i, i, i, P, P, i, i, i, P, P, P, d, d, P]
         L.orc_matmul.argtypes = [i, i, i, P, P, P]
+        L.orc_quantize_rows_dynamic.argtypes = [i, i, P, P, P]
         L.orc_bf16_to_f64.argtypes = [ctypes.c_uint16]
         L.orc_bf16_to_f64.restype = d
         L.orc_e4m3_to_f64.argtypes = [ctypes.c_uint8]
@@ -245,6 +246,18 @@ def dense_masked(x, x_dtype: int, G, act: str, w1, w3, w2, w_dtype: int, x_scale
     _check(lib().orc_dense_masked(N, din, E, x_dtype, _p(xn), _p(G), ACT[act], F, w_dtype, _p(w1n),
                                   _p(w3n), _p(w2n), x_scale, w_scale, _p(y)), "dense_masked")
     return y
+
+
+def quantize_rows_dynamic(x):
+    """Per-token dynamic e4m3 quantization of bf16 rows: (codes uint8 (n, d),
+    scales float32 (n,)), decisions in fp32 as the layer takes them."""
+    xn = _np(x)
+    n, d = xn.shape
+    codes = np.empty((n, d), np.uint8)
+    scales = np.empty(n, np.float32)
+    _check(lib().orc_quantize_rows_dynamic(n, d, _p(xn), _p(codes), _p(scales)),
+           "quantize_rows_dynamic")
+    return codes, scales
 
 
 def matmul(A, B):

@@ -369,6 +369,35 @@ int orc_expert_rows_scaled(int nrows, const int32_t* row_expert, int E, int din,
     return ORC_OK;
 }
 
+/* Per-token dynamic quantization (Ascend quant mode 7, "pertoken dynamic
+ * quantization", parameter section): each token row of bf16 activations gets
+ * its own scale amax(|row|) / 448 (448 = the largest e4m3 value; 1 for an
+ * all-zero row) and codes e4m3(x / scale), rounded to nearest even and
+ * saturated.  The page fixes no precision for this step; the layer takes it
+ * in fp32, and since the codes are integers decided by that arithmetic, the
+ * oracle takes the same decisions: the amax is exact, the two divisions are
+ * IEEE binary32 divisions (this file is compiled without fast-math or
+ * contraction), and the binary32 quotient is then rounded to e4m3 by the
+ * encoder above. */
+int orc_quantize_rows_dynamic(int n, int d, const uint16_t* x, uint8_t* codes, float* scales) {
+    if (n < 0 || d <= 0 || !x || !codes || !scales) return ORC_ERR_ARG;
+    for (int r = 0; r < n; ++r) {
+        const uint16_t* row = x + (int64_t)r * d;
+        float amax = 0.0f;
+        for (int k = 0; k < d; ++k) {
+            float v = fabsf((float)orc_bf16_to_f64(row[k]));
+            if (v > amax) amax = v;
+        }
+        volatile float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scales[r] = scale;
+        for (int k = 0; k < d; ++k) {
+            volatile float q = (float)orc_bf16_to_f64(row[k]) / scale;
+            codes[(int64_t)r * d + k] = orc_f64_to_e4m3((double)q);
+        }
+    }
+    return ORC_OK;
+}
+
 /* ------------------------------------------------------------------------ */
 /* unpermute / combine                                                      */
 /* ------------------------------------------------------------------------ */

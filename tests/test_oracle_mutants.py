@@ -51,6 +51,12 @@ MUTANTS = [
     ("fp8 scales divided instead of multiplied",
      "y[n] = dot_row(din, x, w1, w_dtype, (int64_t)e * F + n) * x_scale * w_scale;",
      "y[n] = dot_row(din, x, w1, w_dtype, (int64_t)e * F + n) / (x_scale * w_scale);"),
+    ("dynamic quantization scaled to the e4m3fnuz maximum 240",
+     "volatile float scale = amax > 0.0f ? amax / 448.0f : 1.0f;",
+     "volatile float scale = amax > 0.0f ? amax / 240.0f : 1.0f;"),
+    ("dynamic quantization multiplies by the scale",
+     "volatile float q = (float)orc_bf16_to_f64(row[k]) / scale;",
+     "volatile float q = (float)orc_bf16_to_f64(row[k]) * scale;"),
     ("e4m3 exponent bias 8 instead of 7",
      "v = ldexp(1.0 + m / 8.0, e - 7);",
      "v = ldexp(1.0 + m / 8.0, e - 8);"),

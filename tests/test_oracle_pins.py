@@ -343,6 +343,55 @@ def test_per_row_quantiser_round_trip():
     assert scale[3] == 1.0 and np.all(dec[3] == 0)
 
 
+# ------------------------------------------- per-token dynamic quantization
+
+def _bf16_rows(vals):
+    t = torch.tensor(vals, dtype=torch.float64).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def test_dynamic_quant_exact_when_row_is_scaled_e4m3(orc):
+    """A row that is e4m3 values (largest 448) times a power of two has scale
+    exactly that power of two and codes exactly the original ones."""
+    base = [448.0, 1.0, -2.0, 0.5, -0.0, 3.5, -448.0, 0.001953125]   # all e4m3 values
+    codes_ref = [orc.f64_to_e4m3(v) for v in base]
+    for p in (-7, -3, 0, 4):
+        row = _bf16_rows([[v * 2.0 ** p for v in base]])
+        codes, scales = orc.quantize_rows_dynamic(row)
+        assert scales[0] == np.float32(2.0 ** p)
+        assert [int(c) for c in codes[0]] == codes_ref
+
+
+def test_dynamic_quant_bounds_and_extremes(orc):
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((64, 96)) * np.exp(rng.uniform(-6, 6, (64, 1)))
+    rows = _bf16_rows(x)
+    xd = torch.from_numpy(rows.view(np.int16)).view(torch.bfloat16).double().numpy()
+    codes, scales = orc.quantize_rows_dynamic(rows)
+    for r in range(64):
+        amax = np.abs(xd[r]).max()
+        # scale = amax / 448 rounded once to fp32
+        assert scales[r] == np.float32(np.float32(amax) / np.float32(448.0))
+        deq = np.array([orc.e4m3_to_f64(int(c)) for c in codes[r]]) * float(scales[r])
+        # half an e4m3 step: 2^-4 relative for normals, 2^-10 * scale below
+        # 2^-6 * scale (subnormal codes); plus the fp32 quotient's rounding
+        bound = np.maximum(np.abs(xd[r]) * 2.0 ** -4, 2.0 ** -10 * float(scales[r])) * (1 + 1e-6)
+        assert np.all(np.abs(deq - xd[r]) <= bound)
+        k = int(np.argmax(np.abs(xd[r])))
+        assert codes[r, k] & 0x7F == 0x7E                     # the largest maps to 448
+    # negating a row flips every sign bit (zeros keep +0 vs -0 from the input)
+    c2, s2 = orc.quantize_rows_dynamic(_bf16_rows(-x))
+    assert np.array_equal(s2, scales)
+    nz = (codes & 0x7F) != 0
+    assert np.array_equal(c2[nz] ^ 0x80, codes[nz])
+
+
+def test_dynamic_quant_zero_row(orc):
+    codes, scales = orc.quantize_rows_dynamic(_bf16_rows([[0.0] * 16, [1.0] + [0.0] * 15]))
+    assert scales[0] == 1.0 and not codes[0].any()
+    assert scales[1] == np.float32(1.0 / 448.0) and codes[1, 0] == 0x7E and not codes[1, 1:].any()
+
+
 @pytest.mark.parametrize("act,dtype", [("relu", "f32"), ("swiglu", "bf16"), ("none", "e4m3")])
 def test_dense_masked_reference_equals_sparse(orc, act, dtype):
     """SpMM page: the dense product over the (N,E) gate matrix equals the sparse
