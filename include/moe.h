@@ -242,6 +242,28 @@ moe_status moe_forward_routed(moe_plan plan, const void* x, const int32_t* topk_
                               const float* x_token_scales_or_null, void* y, void* ws,
                               size_t ws_bytes, moe_stream_t stream);
 
+/* Permute with per-token dynamic quantization (Ascend quant mode 7,
+ * "pertoken dynamic quantization", parameter section): for an e4m3 plan, x is
+ * the bf16 activations (N, d) (16-byte aligned rows; d a multiple of 16).
+ * Each token row t gets token_scales[t] = amax(|x[t]|) / 448 (1 for an
+ * all-zero row, fp32) and its codes e4m3(x / scale) (fp32 division, round to
+ * nearest even, saturated to +-448) are written to its K destination rows of
+ * x_perm (N*K, d) e4m3.  counts, offsets, perm_pos, perm_src as moe_permute.
+ * MOE_ERR_UNSUPPORTED unless the plan dtype is e4m3. */
+moe_status moe_permute_quant(moe_plan plan, const void* x_bf16, const int32_t* topk_ids,
+                             int32_t* counts, int32_t* offsets, int32_t* perm_pos,
+                             int32_t* perm_src, void* x_perm, float* token_scales, void* ws,
+                             size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward_routed for bf16 activations of an e4m3 layer: permute with
+ * per-token dynamic quantization (as moe_permute_quant), the grouped fp8
+ * GEMM with each row's token scale (and the plan's weight scales), then
+ * unpermute (gates NULL, y (N*K, d_out), done by the GEMM's stores) or
+ * combine (y (N, d_out)). */
+moe_status moe_forward_routed_dynamic(moe_plan plan, const void* x_bf16, const int32_t* topk_ids,
+                                      const float* topk_gates_or_null, void* y, void* ws,
+                                      size_t ws_bytes, moe_stream_t stream);
+
 /* moe_forward from host buffers: copies x_host (N, d) in, runs the layer,
  * copies y back to y_host (N, d_out) and synchronises the stream.  Pinned
  * host memory gives asynchronous copies; pageable memory works too. */

@@ -167,3 +167,44 @@ def test_e4m3_gmm_unpermute_shared_n8192_h7168_e256_k8_n2048():
                               "none", inp.w_sh.reshape(1, N2, H2), None, None, oracle.E4M3,
                               inp.x_scale, inp.w_sh_scale)
     assert rel_err(f64(ysh[torch.from_numpy(srows).long().cuda()]), sref) <= TOL["e4m3"]
+
+
+def test_e4m3_gmm_dynamic_per_token_quant_n8192_h7168_e256_k8_n2048():
+    """The fp8 workload fed bf16 activations: per-token dynamic quantization
+    fused into the permute (codes, scales and permutation bit-exact in full),
+    then the grouped matmul with each row's token scale, unpermuted by its
+    stores (sampled tokens against the oracle)."""
+    cfg = synth.FP8_GMM
+    inp = synth.make_inputs(cfg)
+    plan, w = make_plan(inp)
+    c = cfg
+    R = c.N * c.K
+    rng = np.random.default_rng(31)
+    xb = torch.from_numpy(rng.standard_normal((c.N, c.d), dtype=np.float32)).to(torch.bfloat16)
+    ws = plan.new_workspace()
+    counts = torch.empty(c.E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(c.E + 1, dtype=torch.int32, device="cuda")
+    pos = torch.empty(R, dtype=torch.int32, device="cuda")
+    src = torch.empty(R, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty(R, c.d, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(c.N, dtype=torch.float32, device="cuda")
+    plan.permute_quant(xb.cuda(), inp.ids.cuda(), counts, offsets, pos, src, x_perm, scales, ws)
+    assert plan.read_device_status(ws) == 0
+    codes, rscale = oracle.quantize_rows_dynamic(xb)
+    rc, ro, rp, rs, rx = oracle.permute(inp.ids.numpy(), c.E, codes)
+    assert np.array_equal(scales.cpu().numpy(), rscale)
+    assert np.array_equal(pos.cpu().numpy(), rp) and np.array_equal(src.cpu().numpy(), rs)
+    assert np.array_equal(x_perm.cpu().numpy(), rx)
+
+    y = torch.empty(R, c.F, dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed_dynamic(xb.cuda(), inp.ids.cuda(), None, y, ws)
+    assert plan.read_device_status(ws) == 0
+    tok = np.array([0, 1, 4095, c.N - 1])
+    ids = inp.ids.numpy()
+    rows_tok = (tok[:, None] * c.K + np.arange(c.K)).reshape(-1)
+    row_e = ids.reshape(-1)[rows_tok].astype(np.int32)
+    ref = oracle.expert_rows_scaled(row_e, codes[np.repeat(tok, c.K)], oracle.E4M3, inp.w1,
+                                    oracle.E4M3, x_scale=1.0,
+                                    x_row_scales=rscale[np.repeat(tok, c.K)].astype(np.float64),
+                                    w_scale=inp.w_scale)
+    assert rel_err(f64(y[torch.from_numpy(rows_tok).long().cuda()]), ref) <= TOL["e4m3"]

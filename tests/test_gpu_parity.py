@@ -446,6 +446,72 @@ def test_fused_routed_with_gates_and_token_scales(name):
     assert rel_err(f64(y), ref) <= TOL["e4m3"]
 
 
+def _dyn_input(c, seed):
+    """bf16 activations for a dynamic-quantization case: rows of widely
+    different magnitudes and one all-zero row."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((c.N, c.d)) * np.exp(rng.uniform(-4, 4, (c.N, 1)))
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    xb[min(1, c.N - 1)] = 0
+    return xb
+
+
+DYN = ["e4m3_gmm", "e4m3_gmm_ragged", "e4m3_pair"]
+
+
+@pytest.mark.parametrize("name", DYN)
+def test_permute_quant_bit_exact(name):
+    """Per-token dynamic quantization fused into the permute: codes, scales
+    and the permutation bit-exact against the oracle (the codes are fp32
+    decisions on both sides)."""
+    inp, plan, w = case(name)
+    c = inp.cfg
+    xb = _dyn_input(c, 21)
+    R = c.N * c.K
+    counts = torch.empty(c.E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(c.E + 1, dtype=torch.int32, device="cuda")
+    pos = torch.empty(R, dtype=torch.int32, device="cuda")
+    src = torch.empty(R, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty(R, c.d, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(c.N, dtype=torch.float32, device="cuda")
+    ws = plan.new_workspace()
+    plan.permute_quant(xb.cuda(), inp.ids.cuda(), counts, offsets, pos, src, x_perm, scales, ws)
+    assert plan.read_device_status(ws) == 0
+    codes, rscale = oracle.quantize_rows_dynamic(xb)
+    rc, ro, rp, rs, rx = oracle.permute(inp.ids.numpy(), c.E, codes)
+    assert np.array_equal(scales.cpu().numpy(), rscale)
+    assert np.array_equal(counts.cpu().numpy(), rc) and np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(pos.cpu().numpy(), rp) and np.array_equal(src.cpu().numpy(), rs)
+    assert np.array_equal(x_perm.cpu().numpy(), rx)
+
+
+@pytest.mark.parametrize("name", DYN)
+@pytest.mark.parametrize("gated", [False, True])
+def test_forward_routed_dynamic(name, gated):
+    inp, plan, w = case(name)
+    c = inp.cfg
+    xb = _dyn_input(c, 22)
+    ws = plan.new_workspace()
+    ids = inp.ids.numpy()
+    g = None
+    if gated:
+        g = np.random.default_rng(9).random((c.N, c.K)).astype(np.float32)
+        y = torch.empty(c.N, c.d_out, dtype=torch.bfloat16, device="cuda")
+    else:
+        y = torch.full((c.N * c.K, c.d_out), float("nan"), dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed_dynamic(xb.cuda(), inp.ids.cuda(),
+                                None if g is None else torch.from_numpy(g).cuda(), y, ws)
+    assert plan.read_device_status(ws) == 0
+    codes, rscale = oracle.quantize_rows_dynamic(xb)
+    _, _, rp, rs, rx = oracle.permute(ids, c.E, codes)
+    row_e = np.repeat(np.arange(c.E, dtype=np.int32), np.bincount(ids.ravel(), minlength=c.E))
+    yp = oracle.expert_rows_scaled(row_e, rx, oracle.E4M3, inp.w1, oracle.E4M3, x_scale=1.0,
+                                   x_row_scales=rscale[rs].astype(np.float64),
+                                   w_scale=inp.w_scale)
+    ref = oracle.combine(rp, None if g is None else g.astype(np.float64), yp, c.N, c.K)
+    assert rel_err(f64(y), ref) <= TOL["e4m3"]
+
+
 def test_stage_profile_names():
     inp, plan, w = case("bf16_swiglu_ragged")
     c = inp.cfg

@@ -83,6 +83,8 @@ def load(path: str = LIB_PATH):
         "moe_shared_matmul": ([P, P, i32, i32, P, i32, f32, P, f32, P, P, P], ctypes.c_int),
         "moe_forward": ([P, P, P, P, sz, P], ctypes.c_int),
         "moe_forward_routed": ([P, P, P, P, f32, P, P, P, sz, P], ctypes.c_int),
+        "moe_permute_quant": ([P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_forward_routed_dynamic": ([P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_forward_host": ([P, P, P, P, sz, P], ctypes.c_int),
         "moe_forward_host_async": ([P, P, P, P, sz, P], ctypes.c_int),
         "moe_host_join": ([P, P], ctypes.c_int),
@@ -216,6 +218,18 @@ class Plan:
         _check(self.lib.moe_forward_routed(self.handle, _ptr(x), _ptr(ids), _ptr(gates), x_scale,
                                            _ptr(x_token_scales), _ptr(y), _ptr(ws), ws.numel(),
                                            _stream(stream)), "moe_forward_routed")
+
+    def permute_quant(self, x_bf16, ids, counts, offsets, pos, src, x_perm, token_scales, ws,
+                      stream=None):
+        _check(self.lib.moe_permute_quant(self.handle, _ptr(x_bf16), _ptr(ids), _ptr(counts),
+                                          _ptr(offsets), _ptr(pos), _ptr(src), _ptr(x_perm),
+                                          _ptr(token_scales), _ptr(ws), ws.numel(),
+                                          _stream(stream)), "moe_permute_quant")
+
+    def forward_routed_dynamic(self, x_bf16, ids, gates, y, ws, stream=None):
+        _check(self.lib.moe_forward_routed_dynamic(self.handle, _ptr(x_bf16), _ptr(ids),
+                                                   _ptr(gates), _ptr(y), _ptr(ws), ws.numel(),
+                                                   _stream(stream)), "moe_forward_routed_dynamic")
 
     def forward_host(self, x_host, y_host, ws, stream=None):
         _check(self.lib.moe_forward_host(self.handle, _ptr(x_host), _ptr(y_host), _ptr(ws),

@@ -27,7 +27,7 @@ constexpr int kHostEvents = 6;
 struct Layout {
   size_t status = 0, chunk_counts = 0, h = 0, h_end = 0;
   size_t ids = 0, gates = 0, pos = 0, src = 0, slot = 0, counts = 0, offsets = 0, x_perm = 0,
-         y_perm = 0;
+         y_perm = 0, tok_scale = 0;
   size_t fwd_end = 0, x_stage = 0, y_stage = 0, total = 0, x_stage_bytes = 0, y_stage_bytes = 0;
   size_t permute_end = 0, router_w3 = 0, router_end = 0;
 };
@@ -97,6 +97,7 @@ void layout(moe_plan p) {
   L.pos = off; off = align_up(off + static_cast<size_t>(R) * 4);
   L.src = off; off = align_up(off + static_cast<size_t>(R) * 4);
   L.slot = off; off = align_up(off + static_cast<size_t>(R) * 4);
+  L.tok_scale = off; off = align_up(off + static_cast<size_t>(d.N) * 4);
   L.counts = off; off = align_up(off + static_cast<size_t>(d.E) * 4);
   L.offsets = off; off = align_up(off + static_cast<size_t>(d.E + 1) * 4);
   L.x_perm = off; off = align_up(off + static_cast<size_t>(R) * d.d * p->ex);
@@ -161,6 +162,28 @@ moe_status run_permute(moe_plan p, int n, const void* x, const int32_t* ids, int
   mark(p, s, "permute_gather");
   if (launch_permute_gather(x, d.d * p->ex, ids, n, d.K, d.E, cc, pos, src, slot, x_perm, status,
                             s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  p->launches += 3;
+  return MOE_OK;
+}
+
+// run_permute with per-token dynamic quantization of bf16 x into e4m3 x_perm.
+moe_status run_permute_quant(moe_plan p, int n, const void* x_bf16, const int32_t* ids,
+                             int32_t* counts, int32_t* offsets, int32_t* pos, int32_t* src,
+                             void* x_perm, float* token_scales, void* ws, cudaStream_t s,
+                             int32_t* slot = nullptr) {
+  const moe_layer_desc& d = p->desc;
+  int* status = at<int>(ws, p->L.status);
+  int32_t* cc = at<int32_t>(ws, p->L.chunk_counts);
+  mark(p, s, "permute_count");
+  if (launch_permute_count(ids, n, d.K, d.E, cc, pos, status, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  mark(p, s, "permute_scan");
+  if (launch_permute_scan(cc, permute_chunks(n), d.E, counts, offsets, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  mark(p, s, "permute_quant");
+  if (launch_permute_quant(x_bf16, d.d, ids, n, d.K, d.E, cc, pos, src, slot, x_perm,
+                           token_scales, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   p->launches += 3;
   return MOE_OK;
@@ -492,6 +515,50 @@ moe_status moe_forward_routed(moe_plan p, const void* x, const int32_t* ids, con
   if (st == MOE_OK)
     st = run_ffn(p, n, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), x_scale,
                  x_token_scales, src, scatter ? y : at<void>(ws, L.y_perm), ws, stream, slot);
+  if (st == MOE_OK && !scatter)
+    st = run_combine(p, n, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_permute_quant(moe_plan p, const void* x_bf16, const int32_t* ids, int32_t* counts,
+                             int32_t* offsets, int32_t* pos, int32_t* src, void* x_perm,
+                             float* token_scales, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !x_bf16 || !ids || !counts || !offsets || !pos || !src || !x_perm || !token_scales)
+    return MOE_ERR_INVALID_ARG;
+  if (p->desc.dtype != MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x_bf16) || !aligned16(x_perm) || p->desc.d % 16) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.permute_end);
+  if (st != MOE_OK) return st;
+  begin(p);
+  st = run_permute_quant(p, p->desc.N, x_bf16, ids, counts, offsets, pos, src, x_perm,
+                         token_scales, ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_forward_routed_dynamic(moe_plan p, const void* x_bf16, const int32_t* ids,
+                                      const float* gates, void* y, void* ws, size_t ws_bytes,
+                                      moe_stream_t stream) {
+  if (!p || !x_bf16 || !ids || !y) return MOE_ERR_INVALID_ARG;
+  if (p->desc.dtype != MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x_bf16) || !aligned16(y) || p->desc.d % 16) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.fwd_end);
+  if (st != MOE_OK) return st;
+  const Layout& L = p->L;
+  begin(p);
+  const int n = p->desc.N;
+  int32_t* src = at<int32_t>(ws, L.src);
+  float* tok = at<float>(ws, L.tok_scale);
+  const bool scatter = p->desc.act == MOE_ACT_NONE && !gates;
+  int32_t* slot = scatter ? at<int32_t>(ws, L.slot) : nullptr;
+  st = run_permute_quant(p, n, x_bf16, ids, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
+                         at<int32_t>(ws, L.pos), src, at<void>(ws, L.x_perm), tok, ws, stream,
+                         slot);
+  // each permuted row takes its token's scale through the source-token index
+  if (st == MOE_OK)
+    st = run_ffn(p, n, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), 1.f, tok, src,
+                 scatter ? y : at<void>(ws, L.y_perm), ws, stream, slot);
   if (st == MOE_OK && !scatter)
     st = run_combine(p, n, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
   end(p, stream);

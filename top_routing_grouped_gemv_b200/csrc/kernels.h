@@ -82,6 +82,13 @@ cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* i
                                   int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
                                   int32_t* slot, void* x_perm, int* status, cudaStream_t stream);
 
+// The same with per-token dynamic quantization: x_bf16 (N, d) rows,
+// d % 16 == 0; x_perm gets e4m3 codes (N*K, d), token_scale (N) the scales.
+cudaError_t launch_permute_quant(const void* x_bf16, int d, const int32_t* ids, int N, int K,
+                                 int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
+                                 int32_t* slot, void* x_perm_e4m3, float* token_scale,
+                                 cudaStream_t stream);
+
 // ---- combine / unpermute ----------------------------------------------------
 // y_dtype: kF32 or kBF16 (the dtype of y_perm and y).
 cudaError_t launch_combine(const void* y_perm, int y_dtype, int dout, const int32_t* pos,

@@ -21,6 +21,8 @@
 //              rows with 16-byte vector loads/stores (and, on request, notes
 //              each position's flat slot t*K + j for an unpermute done by
 //              the grouped GEMM's stores).
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -255,6 +257,104 @@ permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* 
   }
 }
 
+// Per-token dynamic quantization fused into the gather (Ascend quant mode 7,
+// per-token dynamic): a bf16 token row gets the scale amax(|row|) / 448 (1
+// for an all-zero row) and e4m3 codes of x / scale (fp32 division, round to
+// nearest even, saturated to 448), written once per destination row; the
+// scale goes to token_scale[t].  WPT warps per token as in the gather; a lane
+// handles 16 elements (32 bytes in, 16 bytes out) at a time.
+template <int KMAX, int WPT>
+__global__ void __launch_bounds__(256)
+permute_quant_kernel(const uint4* __restrict__ x, int d, const int32_t* __restrict__ ids, int N,
+                     int K, int E, const int32_t* __restrict__ chunk_base,
+                     int32_t* __restrict__ pos, int32_t* __restrict__ src,
+                     int32_t* __restrict__ slot, uint4* __restrict__ x_perm,
+                     float* __restrict__ token_scale) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
+  __shared__ int sp[8 / WPT][KMAX];
+  __shared__ float wmax[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tl = warp / WPT, sub = warp % WPT;
+  const int t = blockIdx.x * (8 / WPT) + tl;
+  const bool active = t < N;
+  if (active && sub == 0 && lane < KMAX) {
+    int mine = -1;
+    if (lane < K) {
+      const long long i = (long long)t * K + lane;
+      const int e = ids[i];
+      const int r = pos[i];  // rank within the chunk (written by the rank pass)
+      if (r >= 0 && e >= 0 && e < E) {
+        mine = chunk_base[(long long)(t / CH) * E + e] + r;
+        src[mine] = t;
+        if (slot) slot[mine] = static_cast<int32_t>(i);
+      }
+      pos[i] = mine;
+    }
+    sp[tl][lane] = mine;
+  }
+  const int units = d / 16;               // 16 elements per unit
+  const uint4* srow = x + (long long)(active ? t : 0) * (d / 8);
+  constexpr int STEP = 32 * WPT;
+  float am = 0.f;
+  if (active)
+    for (int u = sub * 32 + lane; u < units; u += STEP) {
+      const uint4 a = srow[2 * u], b = srow[2 * u + 1];
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        am = fmaxf(am, fmaxf(fabsf(bf16lo(w[i])), fabsf(bf16hi(w[i]))));
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  if (lane == 0) wmax[warp] = am;
+  if constexpr (WPT > 1) __syncthreads();
+  else __syncwarp();
+  if (!active) return;
+  am = 0.f;
+#pragma unroll
+  for (int q = 0; q < WPT; ++q) am = fmaxf(am, wmax[tl * WPT + q]);
+  const float scale = am > 0.f ? am / 448.f : 1.f;
+  if (sub == 0 && lane == 0) token_scale[t] = scale;
+  int p[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) p[j] = sp[tl][j];
+  for (int u = sub * 32 + lane; u < units; u += STEP) {
+    const uint4 a = srow[2 * u], b = srow[2 * u + 1];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t packed[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t c0 = __nv_cvt_float_to_fp8(bf16lo(w[2 * i]) / scale, __NV_SATFINITE, __NV_E4M3);
+      const uint32_t c1 = __nv_cvt_float_to_fp8(bf16hi(w[2 * i]) / scale, __NV_SATFINITE, __NV_E4M3);
+      const uint32_t c2 = __nv_cvt_float_to_fp8(bf16lo(w[2 * i + 1]) / scale, __NV_SATFINITE, __NV_E4M3);
+      const uint32_t c3 = __nv_cvt_float_to_fp8(bf16hi(w[2 * i + 1]) / scale, __NV_SATFINITE, __NV_E4M3);
+      packed[i] = c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+    }
+    const uint4 out = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (j < K && p[j] >= 0) x_perm[(long long)p[j] * units + u] = out;
+  }
+}
+
+template <int KMAX>
+void launch_quant_k(const uint4* xv, int d, const int32_t* ids, int N, int K, int E,
+                    const int32_t* chunk_base, int32_t* pos, int32_t* src, int32_t* slot, uint4* xp,
+                    float* scales, cudaStream_t stream) {
+  const int wpt = warps_per_token(N);
+  const dim3 grid((N + 8 / wpt - 1) / (8 / wpt));
+  if (wpt == 1)
+    launch_pdl(permute_quant_kernel<KMAX, 1>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales);
+  else if (wpt == 2)
+    launch_pdl(permute_quant_kernel<KMAX, 2>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales);
+  else if (wpt == 4)
+    launch_pdl(permute_quant_kernel<KMAX, 4>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales);
+  else
+    launch_pdl(permute_quant_kernel<KMAX, 8>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales);
+}
+
 template <int KMAX>
 void launch_gather_k(const uint4* xv, int row_vecs, const int32_t* ids, int N, int K, int E,
                      const int32_t* chunk_base, int32_t* pos, int32_t* src, int32_t* slot,
@@ -308,6 +408,23 @@ cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* i
     launch_gather_k<4>(xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, stream);
   else
     launch_gather_k<8>(xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, stream);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_quant(const void* x_bf16, int d, const int32_t* ids, int N, int K,
+                                 int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
+                                 int32_t* slot, void* x_perm_e4m3, float* token_scale,
+                                 cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  if (d % 16) return cudaErrorInvalidValue;
+  auto xv = static_cast<const uint4*>(x_bf16);
+  auto xp = static_cast<uint4*>(x_perm_e4m3);
+  if (K <= 2)
+    launch_quant_k<2>(xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, token_scale, stream);
+  else if (K <= 4)
+    launch_quant_k<4>(xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, token_scale, stream);
+  else
+    launch_quant_k<8>(xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, token_scale, stream);
   return cudaGetLastError();
 }
 
