@@ -27,7 +27,7 @@ constexpr int kHostEvents = 6;
 struct Layout {
   size_t status = 0, chunk_counts = 0, h = 0, h_end = 0;
   size_t ids = 0, gates = 0, pos = 0, src = 0, slot = 0, counts = 0, offsets = 0, x_perm = 0,
-         y_perm = 0, tok_scale = 0;
+         y_perm = 0, tok_scale = 0, simt_part = 0;
   size_t fwd_end = 0, x_stage = 0, y_stage = 0, total = 0, x_stage_bytes = 0, y_stage_bytes = 0;
   size_t permute_end = 0, router_w3 = 0, router_end = 0;
 };
@@ -91,6 +91,11 @@ void layout(moe_plan p) {
   L.router_end = off;
   L.h = off;
   if (d.act != MOE_ACT_NONE) off = align_up(off + static_cast<size_t>(R) * d.F * p->eh);
+  // fp32 layers: split-K partial sums of the SIMT GEMMs (up to 8 slices,
+  // gate and up for SwiGLU), shared by the layer's GEMMs (they run in order)
+  L.simt_part = off;
+  if (!uses_tensor_cores(d))
+    off = align_up(off + static_cast<size_t>(8) * 2 * R * (d.F > d.d ? d.F : d.d) * sizeof(float));
   L.h_end = off;
   L.ids = off; off = align_up(off + static_cast<size_t>(R) * 4);
   L.gates = off; off = align_up(off + static_cast<size_t>(R) * 4);
@@ -202,24 +207,26 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
   void* h = at<void>(ws, p->L.h);
   if (!uses_tensor_cores(d)) {
     const float* A = static_cast<const float*>(x_perm);
+    float* part = at<float>(ws, p->L.simt_part);
+    auto launches = [&](int kdim, int ncols) { return simt_f32_splits(kdim, ncols, R, d.E) > 1 ? 2 : 1; };
     if (d.act == MOE_ACT_NONE) {
       mark(p, s, "ffn_simt_f32");
-      p->launches += 1;
+      p->launches += launches(d.d, d.F);
       return cuda_status(launch_gemm_simt_f32(A, d.d, static_cast<const float*>(p->w.w1), nullptr,
                                               d.F, kActNone, 1.f, offsets, d.E, R,
-                                              static_cast<float*>(y_perm), s));
+                                              static_cast<float*>(y_perm), part, s));
     }
     mark(p, s, "ffn1_simt_f32");
     if (launch_gemm_simt_f32(A, d.d, static_cast<const float*>(p->w.w1),
                              static_cast<const float*>(p->w.w3), d.F, d.act, 1.f, offsets, d.E, R,
-                             static_cast<float*>(h), s) != cudaSuccess)
+                             static_cast<float*>(h), part, s) != cudaSuccess)
       return MOE_ERR_CUDA;
     mark(p, s, "ffn2_simt_f32");
-    p->launches += 2;
+    p->launches += launches(d.d, d.F) + launches(d.F, d.d);
     return cuda_status(launch_gemm_simt_f32(static_cast<const float*>(h), d.F,
                                             static_cast<const float*>(p->w.w2), nullptr, d.d,
                                             kActNone, 1.f, offsets, d.E, R,
-                                            static_cast<float*>(y_perm), s));
+                                            static_cast<float*>(y_perm), part, s));
   }
   TcGemmArgs a;
   memset(&a, 0, sizeof(a));

@@ -98,9 +98,12 @@ cudaError_t launch_combine(const void* y_perm, int y_dtype, int dout, const int3
 // ---- grouped FFN, fp32 SIMT path --------------------------------------------
 // C[r, n] for rows of expert e: act(A[r,:] . W[e][n,:]) with A (R, kdim),
 // W (E, ncols, kdim); SwiGLU uses W3 as the up matrix.  out (R, ncols) fp32.
+// partial: split-K scratch of simt_f32_partial_bytes (NULL: no split).
 cudaError_t launch_gemm_simt_f32(const float* A, int kdim, const float* W, const float* W3,
                                  int ncols, int act, float scale, const int32_t* offsets, int E,
-                                 int R, float* out, cudaStream_t stream);
+                                 int R, float* out, float* partial, cudaStream_t stream);
+int simt_f32_splits(int kdim, int ncols, int R, int E);
+size_t simt_f32_partial_bytes(int kdim, int ncols, int R, int E, int act);
 
 // ---- grouped GEMM on tcgen05 tensor cores -----------------------------------
 // kEpiRouter: fp32 logits from the three-part split router weights (bf16,
