@@ -183,15 +183,16 @@ def oracle_sample_tokens(cfg, inp, target_s: float, max_tokens: int | None = Non
     import oracle
     threads = oracle.num_threads()
     n = max(1, threads)
+    gm = 0 if cfg.routing == "given" else 1   # given routing: the pure unpermute
     t0 = time.perf_counter()
-    oracle.forward_tokens(inp, np.arange(n))
+    oracle.forward_tokens(inp, np.arange(n), gates_mode=gm)
     dt = time.perf_counter() - t0
     n2 = int(min(max_tokens or cfg.N, max(n, n * target_s / max(dt, 1e-6))))
     n2 = max(threads, n2 // threads * threads) if n2 >= threads else n2
     rng = np.random.default_rng(17)
     tok = np.sort(rng.choice(cfg.N, size=min(n2, cfg.N), replace=False))
     t0 = time.perf_counter()
-    oracle.forward_tokens(inp, tok)
+    oracle.forward_tokens(inp, tok, gates_mode=gm)
     return len(tok), time.perf_counter() - t0, threads
 
 
@@ -207,11 +208,12 @@ def run_reference(args, rank: int):
     threads = oracle.num_threads()
     per = max(1, threads)
     rng = np.random.default_rng(23)
+    gm = 0 if cfg.routing == "given" else 1
     for _ in range(args.warmup):
-        oracle.forward_tokens(inp, rng.choice(cfg.N, size=per, replace=False))
+        oracle.forward_tokens(inp, rng.choice(cfg.N, size=per, replace=False), gates_mode=gm)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.forward_tokens(inp, rng.choice(cfg.N, size=per, replace=False))
+        oracle.forward_tokens(inp, rng.choice(cfg.N, size=per, replace=False), gates_mode=gm)
     dt = time.perf_counter() - t0
     value = per * args.steps / dt
     line = {
@@ -266,12 +268,26 @@ def main():
     ws = plan.new_workspace()
     x = inp.x.cuda()
     ydt = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
-    y = torch.empty(cfg.N, cfg.d_out, dtype=ydt, device="cuda")
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
+    given = cfg.routing == "given"
+    if given:
+        # fp8 grouped-matmul layer: the caller's routing, the pure unpermute
+        # done by the GEMM's stores, and the shared expert on a forked stream
+        ids = inp.ids.cuda()
+        y = torch.empty(cfg.N * cfg.K, cfg.d_out, dtype=ydt, device="cuda")
+        N2 = cfg.shared[1]
+        wsh = inp.w_sh.cuda()
+        ysh = torch.empty(cfg.N, N2, dtype=torch.bfloat16, device="cuda")
 
-    def step():
-        plan.forward(x, y, ws)
+        def step():
+            plan.forward_routed_shared(x, ids, None, y, wsh, inp.w_sh_scale, ysh, ws,
+                                       x_scale=inp.x_scale)
+    else:
+        y = torch.empty(cfg.N, cfg.d_out, dtype=ydt, device="cuda")
+
+        def step():
+            plan.forward(x, y, ws)
 
     # warm-up
     for _ in range(args.warmup):
@@ -279,7 +295,7 @@ def main():
         step()
     torch.cuda.synchronize()
     assert plan.read_device_status(ws) == 0, "device status after warm-up"
-    launches_per_step = plan.last_launch_count()
+    launches_per_step = plan.last_launch_count() + (1 if given else 0)  # + the shared matmul
 
     # timed region: K steps back to back (the host runs ahead of the GPU),
     # CUDA events around every step on the launching stream
@@ -320,7 +336,43 @@ def main():
     # its neighbours, as in a serving loop); device events from before the
     # first H2D to after the last D2H
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and given:
+        # fp8 layer: each step copies its x and routing in from pinned host
+        # memory, runs the routed layer and the shared expert, and copies both
+        # results back (no host-buffer entry point for this layer: the copies
+        # are queued on the compute stream)
+        xh = inp.x.clone().pin_memory()
+        idh = inp.ids.clone().pin_memory()
+        yh = torch.empty(tuple(y.shape), dtype=y.dtype).pin_memory()
+        yshh = torch.empty(tuple(ysh.shape), dtype=ysh.dtype).pin_memory()
+
+        def e2e_step():
+            x.copy_(xh, non_blocking=True)
+            ids.copy_(idh, non_blocking=True)
+            step()
+            yh.copy_(y, non_blocking=True)
+            yshh.copy_(ysh, non_blocking=True)
+
+        for _ in range(min(args.warmup, 3)):
+            e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(1, args.steps)
+        if dist:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        b.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b), dist)
+        assert plan.read_device_status(ws) == 0, "device status after the host-buffer loop"
+        e2e = {"value": replica_throughput(cfg.N, n_e2e, world, e_ms), "unit": "tokens/s",
+               "h2d_bytes_per_step": xh.numel() * xh.element_size() + idh.numel() * idh.element_size(),
+               "d2h_bytes_per_step": yh.numel() * yh.element_size() + yshh.numel() * yshh.element_size(),
+               "steps": n_e2e,
+               "api": "moe_forward_routed_shared with pinned host copies on the same stream"}
+    elif not args.no_e2e:
         xh = [inp.x.clone().pin_memory() for _ in range(2)]
         yh = [torch.empty(cfg.N, cfg.d_out, dtype=ydt).pin_memory() for _ in range(2)]
         for i in range(min(args.warmup, 3)):
@@ -358,17 +410,25 @@ def main():
     clk_summary = clk.summary()
     sustained = wall > 2.0 or "sw_power_cap" in clk_summary.get("reasons", [])
     peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    peak_note = ""
+    if cfg.dtype == "e4m3":
+        peak *= 2.0   # dense e4m3 = 2x bf16 (nominal ratio), no measured fp8 peak
+        peak_note = " x 2 (e4m3 nominal ratio)"
     t1 = stage_us.get(k1, float("nan")) * 1e-6
     achieved = f1 / t1 / 1e12
     traffic = profiled_traffic(cfg.name, k1)
     roofline = {"bound": "tensor", "kernel": k1, "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'}",
+                "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'}{peak_note}",
                 "algorithmic_flop_per_launch": f1}
     ffn_keys = [k for k in stage_us if k.startswith("ffn") or k.startswith("gmm")]
     ffn_s = sum(stage_us[k] for k in ffn_keys) * 1e-6
     gemm = {"tflops": (f1 + f2) / ffn_s / 1e12, "frac_of_peak": (f1 + f2) / ffn_s / 1e12 / peak,
             "flop_per_step": f1 + f2}
+
+    elem = {"f32": 4, "bf16": 2, "e4m3": 1}[cfg.dtype]
+    mats = {"swiglu": 3, "relu": 2, "none": 1}[cfg.act]
+    weight_mb = cfg.E * cfg.F * cfg.d * mats * elem / 1e6
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -386,10 +446,13 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic",
             "config": {"workload": cfg.name, "N": cfg.N, "d": cfg.d, "E": cfg.E, "K": cfg.K,
-                       "F": cfg.F, "act": cfg.act, "router": "fp32",
+                       "F": cfg.F, "act": cfg.act,
+                       "router": "given (top-K of seeded iid logits), shared expert "
+                                 f"{cfg.shared[0]}x{cfg.shared[1]} on a forked stream"
+                                 if given else "fp32",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "value: flushed (256 MiB write) before every step; e2e: inputs "
-                             "larger than L2 (805 MB of expert weights), no flush",
+                             f"larger than L2 ({weight_mb:.0f} MB of expert weights), no flush",
                        "inputs": "seeded synthetic, resident in HBM"},
             "roofline": roofline, "gemm": gemm,
             "stages_us": {k: round(v, 2) for k, v in stage_us.items()},

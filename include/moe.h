@@ -242,6 +242,21 @@ moe_status moe_forward_routed(moe_plan plan, const void* x, const int32_t* topk_
                               const float* x_token_scales_or_null, void* y, void* ws,
                               size_t ws_bytes, moe_stream_t stream);
 
+/* The routed fp8 layer and the shared expert "in parallel" (Ascend page,
+ * function section: the shared-expert matmul runs beside the routed grouped
+ * matmul): moe_shared_matmul(x, w_sh) on a stream owned by the plan, forked
+ * from `stream` at entry, concurrently with moe_forward_routed(...) on
+ * `stream`, joined back into `stream` before return (work queued on `stream`
+ * afterwards sees both y and y_sh).  x (N, d) e4m3; w_sh (N2, d) e4m3; y_sh
+ * (N, N2) bf16; scales as moe_shared_matmul (the activation scales are the
+ * routed call's).  The plan's side stream is created on first use. */
+moe_status moe_forward_routed_shared(moe_plan plan, const void* x, const int32_t* topk_ids,
+                                     const float* topk_gates_or_null, float x_scale,
+                                     const float* x_token_scales_or_null, void* y,
+                                     const void* w_sh, int32_t N2, float w_sh_scale,
+                                     const float* w_sh_channel_scales_or_null, void* y_sh,
+                                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Permute with per-token dynamic quantization (Ascend quant mode 7,
  * "pertoken dynamic quantization", parameter section): for an e4m3 plan, x is
  * the bf16 activations (N, d) (16-byte aligned rows; d a multiple of 16).

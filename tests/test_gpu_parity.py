@@ -446,6 +446,33 @@ def test_fused_routed_with_gates_and_token_scales(name):
     assert rel_err(f64(y), ref) <= TOL["e4m3"]
 
 
+@pytest.mark.parametrize("name", ["e4m3_gmm", "e4m3_pair"])
+@pytest.mark.parametrize("gated", [False, True])
+def test_forward_routed_shared_matches_separate_calls(name, gated):
+    """Routed layer and shared expert on forked streams: both outputs equal
+    the separate calls on one stream bit for bit."""
+    inp, plan, w = case(name)
+    c = inp.cfg
+    H2, N2 = c.shared
+    x, ids, wsh = inp.x.cuda(), inp.ids.cuda(), inp.w_sh.cuda()
+    g = None
+    rows = c.N * c.K
+    if gated:
+        g = torch.from_numpy(np.random.default_rng(4).random((c.N, c.K)).astype(np.float32)).cuda()
+        rows = c.N
+    ws = plan.new_workspace()
+    y1 = torch.empty(rows, c.d_out, dtype=torch.bfloat16, device="cuda")
+    s1 = torch.empty(c.N, N2, dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed(x, ids, g, y1, ws, x_scale=inp.x_scale)
+    plan.shared_matmul(x, wsh, inp.x_scale, inp.w_sh_scale, s1)
+    y2 = torch.empty_like(y1)
+    s2 = torch.empty_like(s1)
+    plan.forward_routed_shared(x, ids, g, y2, wsh, inp.w_sh_scale, s2, ws, x_scale=inp.x_scale)
+    assert plan.read_device_status(ws) == 0
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert torch.equal(s1.view(torch.int16), s2.view(torch.int16))
+
+
 def _dyn_input(c, seed):
     """bf16 activations for a dynamic-quantization case: rows of widely
     different magnitudes and one all-zero row."""

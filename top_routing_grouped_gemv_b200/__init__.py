@@ -84,6 +84,8 @@ def load(path: str = LIB_PATH):
         "moe_forward": ([P, P, P, P, sz, P], ctypes.c_int),
         "moe_forward_routed": ([P, P, P, P, f32, P, P, P, sz, P], ctypes.c_int),
         "moe_permute_quant": ([P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_forward_routed_shared": ([P, P, P, P, f32, P, P, P, i32, f32, P, P, P, sz, P],
+                                      ctypes.c_int),
         "moe_forward_routed_dynamic": ([P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_forward_host": ([P, P, P, P, sz, P], ctypes.c_int),
         "moe_forward_host_async": ([P, P, P, P, sz, P], ctypes.c_int),
@@ -230,6 +232,14 @@ class Plan:
         _check(self.lib.moe_forward_routed_dynamic(self.handle, _ptr(x_bf16), _ptr(ids),
                                                    _ptr(gates), _ptr(y), _ptr(ws), ws.numel(),
                                                    _stream(stream)), "moe_forward_routed_dynamic")
+
+    def forward_routed_shared(self, x, ids, gates, y, w_sh, w_sh_scale, y_sh, ws,
+                              x_scale: float = 1.0, x_token_scales=None,
+                              w_sh_channel_scales=None, stream=None):
+        _check(self.lib.moe_forward_routed_shared(
+            self.handle, _ptr(x), _ptr(ids), _ptr(gates), x_scale, _ptr(x_token_scales), _ptr(y),
+            _ptr(w_sh), w_sh.shape[0], w_sh_scale, _ptr(w_sh_channel_scales), _ptr(y_sh), _ptr(ws),
+            ws.numel(), _stream(stream)), "moe_forward_routed_shared")
 
     def forward_host(self, x_host, y_host, ws, stream=None):
         _check(self.lib.moe_forward_host(self.handle, _ptr(x_host), _ptr(y_host), _ptr(ws),

@@ -49,6 +49,8 @@ struct moe_plan_s {
   int nev;
   int launches;
   cudaStream_t h2d, d2h;  // host-buffer path copy streams (created on first use)
+  cudaStream_t side;      // shared-expert stream of moe_forward_routed_shared (first use)
+  cudaEvent_t sev[2];     // fork / join of that stream
   cudaEvent_t hev[kHostEvents];
   unsigned long long host_calls;  // host-buffer calls so far (selects the staging slot)
 };
@@ -401,6 +403,9 @@ moe_status moe_plan_destroy(moe_plan p) {
     if (p->hev[i]) cudaEventDestroy(p->hev[i]);
   if (p->h2d) cudaStreamDestroy(p->h2d);
   if (p->d2h) cudaStreamDestroy(p->d2h);
+  for (int i = 0; i < 2; ++i)
+    if (p->sev[i]) cudaEventDestroy(p->sev[i]);
+  if (p->side) cudaStreamDestroy(p->side);
   delete p;
   return MOE_OK;
 }
@@ -569,6 +574,37 @@ moe_status moe_forward_routed_dynamic(moe_plan p, const void* x_bf16, const int3
   if (st == MOE_OK && !scatter)
     st = run_combine(p, n, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
   end(p, stream);
+  return st;
+}
+
+moe_status moe_forward_routed_shared(moe_plan p, const void* x, const int32_t* ids,
+                                     const float* gates, float x_scale,
+                                     const float* x_token_scales, void* y, const void* w_sh,
+                                     int32_t N2, float w_sh_scale,
+                                     const float* w_sh_channel_scales, void* y_sh, void* ws,
+                                     size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !x || !ids || !y || !w_sh || !y_sh) return MOE_ERR_INVALID_ARG;
+  if (p->desc.dtype != MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(w_sh) || !aligned16(y_sh) || N2 < 1 || N2 >= 65536 || N2 % 8)
+    return MOE_ERR_INVALID_ARG;
+  if (!p->side) {
+    if (cudaStreamCreateWithFlags(&p->side, cudaStreamNonBlocking) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    for (int i = 0; i < 2; ++i)
+      if (cudaEventCreateWithFlags(&p->sev[i], cudaEventDisableTiming) != cudaSuccess)
+        return MOE_ERR_CUDA;
+  }
+  // fork: the shared expert on the plan's side stream, alongside the routed
+  // path on `stream`; join before returning
+  if (cudaEventRecord(p->sev[0], stream) != cudaSuccess ||
+      cudaStreamWaitEvent(p->side, p->sev[0], 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  moe_status st = moe_shared_matmul(p, x, p->desc.N, p->desc.d, w_sh, N2, x_scale, x_token_scales,
+                                    w_sh_scale, w_sh_channel_scales, y_sh, p->side);
+  if (st != MOE_OK) return st;
+  if (cudaEventRecord(p->sev[1], p->side) != cudaSuccess) return MOE_ERR_CUDA;
+  st = moe_forward_routed(p, x, ids, gates, x_scale, x_token_scales, y, ws, ws_bytes, stream);
+  if (cudaStreamWaitEvent(stream, p->sev[1], 0) != cudaSuccess) return MOE_ERR_CUDA;
   return st;
 }
 
