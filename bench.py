@@ -62,10 +62,18 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of what the grouped-GEMM kernel is compiled from: its own source,
+    the PTX helpers, the common helpers and its argument struct (the rest of
+    the launcher header does not change the kernel)."""
+    csrc = os.path.join(ROOT, "top_routing_grouped_gemv_b200", "csrc")
     h = hashlib.sha256()
-    for name in ("gemm_tc.cu", "tc_ptx.cuh", "kernels.h", "common.cuh"):
-        with open(os.path.join(ROOT, "top_routing_grouped_gemv_b200", "csrc", name), "rb") as f:
+    for name in ("gemm_tc.cu", "tc_ptx.cuh", "common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
+    with open(os.path.join(csrc, "kernels.h")) as f:
+        hdr = f.read()
+    m = re.search(r"struct TcGemmArgs \{.*?\n\};", hdr, re.S)
+    h.update((m.group(0) if m else hdr).encode())
     return h.hexdigest()[:16]
 
 
