@@ -45,6 +45,14 @@ SMALL = {
     "bf16_splitk_e100_k3": synth.MoEConfig("sk_e100", "bf16", 33, 1536, 100, 3, 64, "swiglu",
                                            zipf_bias=1.2),
     "f32_splitk_e16": synth.MoEConfig("sk_f32", "f32", 50, 1024, 16, 4, 64, "relu"),
+    # single-token batches (split-K router with one token; one row per expert tile)
+    "bf16_n1": synth.MoEConfig("n1_bf16", "bf16", 1, 1024, 8, 2, 128, "swiglu"),
+    "f32_n1": synth.MoEConfig("n1_f32", "f32", 1, 256, 4, 2, 64, "relu"),
+    "e4m3_n1": synth.small_variant(synth.FP8_GMM, N=1, d=256, E=16, K=8, F=128,
+                                   shared=(256, 64)),
+    # the largest expert count with the largest K, on the tensor-core router
+    "bf16_e256_k8": synth.MoEConfig("e256_k8", "bf16", 600, 256, 256, 8, 64, "swiglu",
+                                    zipf_bias=1.2),
     # >= 512 routed rows per expert on average: 256-row tiles on CTA pairs
     "bf16_pair": synth.small_variant(synth.BF16_PREFILL, N=1024, d=256, E=4, K=2, F=384),
     "bf16_pair_ragged": synth.small_variant(synth.BF16_PREFILL, N=1300, d=320, E=4, K=2, F=200),
