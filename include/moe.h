@@ -130,7 +130,11 @@ typedef struct moe_plan_s* moe_plan;
 
 /* Validates desc and weights, records the weight pointers (not owned: they
  * must stay valid while the plan is used) and encodes the TMA descriptors of
- * the weights for the current CUDA device.  Allocates host memory only. */
+ * the weights for the current CUDA device.  Allocates host memory only.
+ * With w1, w3 and w2 all NULL (and no per-channel scales) the plan is
+ * routing-only: router, permute and unpermute/combine work, the calls that
+ * run the experts return MOE_ERR_UNSUPPORTED (an expert-parallel rank's
+ * view of a layer whose experts live on several GPUs). */
 moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* weights,
                            moe_plan* out);
 moe_status moe_plan_destroy(moe_plan plan);
@@ -211,6 +215,22 @@ moe_status moe_grouped_ffn(moe_plan plan, const void* x_perm, const int32_t* off
 moe_status moe_unpermute_combine(moe_plan plan, const void* y_perm, const int32_t* perm_pos,
                                  const float* topk_gates_or_null, void* y, void* ws,
                                  size_t ws_bytes, moe_stream_t stream);
+
+/* The three stages above on the first n tokens of the plan's N (0 <= n <= N;
+ * rows = n*K), for a batch whose size changes per call, e.g. the rows an
+ * expert-parallel rank receives from the others (run with a plan of K = 1
+ * and N = the largest possible count; p1 section 1.2, p2 AlltoAllv).
+ * Otherwise as moe_permute / moe_grouped_ffn / moe_unpermute_combine. */
+moe_status moe_permute_n(moe_plan plan, int32_t n, const void* x, const int32_t* topk_ids,
+                         int32_t* counts, int32_t* offsets, int32_t* perm_pos, int32_t* perm_src,
+                         void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+moe_status moe_grouped_ffn_n(moe_plan plan, int32_t n, const void* x_perm, const int32_t* offsets,
+                             float x_scale, const float* x_row_scales_or_null, void* y_perm,
+                             void* ws, size_t ws_bytes, moe_stream_t stream);
+moe_status moe_unpermute_combine_n(moe_plan plan, int32_t n, const void* y_perm,
+                                   const int32_t* perm_pos, const float* topk_gates_or_null,
+                                   void* y, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 
 /* Shared-expert matmul run beside the routed experts (Ascend formula mmY =
  * (mmX @ mmWeight) * mmXScale * mmWeightScale).  x (M, H) e4m3, w (N2, H)

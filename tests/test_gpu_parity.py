@@ -630,3 +630,24 @@ def test_e4m3_per_channel_weights_per_token_activations(N, d, E, K, F):
                                       oracle.E4M3, x_row_scales=xs.astype(np.float64),
                                       w_channel_scales=shs.astype(np.float64).reshape(1, 136))
     assert rel_err(f64(ysh), ref_s) <= TOL["e4m3"]
+
+
+@pytest.mark.parametrize("name", ["bf16_swiglu_ragged", "bf16_zipf", "bf16_pair", "f32_relu_ragged"])
+def test_expert_parallel_stages_single_rank_equal_forward(name):
+    """The expert-parallel layer's GPU stages (a routing-only plan over all
+    experts, a K = 1 plan of the local experts on a variable row count) at
+    world size 1 reproduce moe_forward bit for bit."""
+    from top_routing_grouped_gemv_b200.ep import ExpertParallelMoE, LibraryStages
+    inp, plan, w = case(name)
+    c = inp.cfg
+    x = inp.x.cuda()
+    ydt = torch.float32 if c.dtype == "f32" else torch.bfloat16
+    y_ref = torch.empty(c.N, c.d, dtype=ydt, device="cuda")
+    ws = plan.new_workspace()
+    plan.forward(x, y_ref, ws)
+    stages = LibraryStages(c.N, c.d, c.E, c.K, c.F, c.dtype, c.act, 1, w["w_r"], w["w1"],
+                           w.get("w3"), w.get("w2"), bias=w.get("bias"))
+    y = ExpertParallelMoE(stages, c.E, c.K).forward(x)
+    assert stages.check() == 0
+    assert torch.equal(y.view(torch.int32 if c.dtype == "f32" else torch.int16),
+                       y_ref.view(torch.int32 if c.dtype == "f32" else torch.int16))

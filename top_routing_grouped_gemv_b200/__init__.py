@@ -87,6 +87,9 @@ def load(path: str = LIB_PATH):
         "moe_forward_routed_shared": ([P, P, P, P, f32, P, P, P, i32, f32, P, P, P, sz, P],
                                       ctypes.c_int),
         "moe_forward_routed_dynamic": ([P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_permute_n": ([P, i32, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_grouped_ffn_n": ([P, i32, P, P, f32, P, P, P, sz, P], ctypes.c_int),
+        "moe_unpermute_combine_n": ([P, i32, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_forward_host": ([P, P, P, P, sz, P], ctypes.c_int),
         "moe_forward_host_async": ([P, P, P, P, sz, P], ctypes.c_int),
         "moe_host_join": ([P, P], ctypes.c_int),
@@ -178,10 +181,16 @@ class Plan:
                                         _ptr(margin), _ptr(ws), ws.numel(), _stream(stream)),
                "moe_router_topk")
 
-    def permute(self, x, ids, counts, offsets, pos, src, x_perm, ws, stream=None):
-        _check(self.lib.moe_permute(self.handle, _ptr(x), _ptr(ids), _ptr(counts), _ptr(offsets),
-                                    _ptr(pos), _ptr(src), _ptr(x_perm), _ptr(ws), ws.numel(),
-                                    _stream(stream)), "moe_permute")
+    def permute(self, x, ids, counts, offsets, pos, src, x_perm, ws, stream=None, n=None):
+        """n: the number of tokens (default the plan's N)."""
+        if n is None:
+            _check(self.lib.moe_permute(self.handle, _ptr(x), _ptr(ids), _ptr(counts),
+                                        _ptr(offsets), _ptr(pos), _ptr(src), _ptr(x_perm),
+                                        _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
+        else:
+            _check(self.lib.moe_permute_n(self.handle, int(n), _ptr(x), _ptr(ids), _ptr(counts),
+                                          _ptr(offsets), _ptr(pos), _ptr(src), _ptr(x_perm),
+                                          _ptr(ws), ws.numel(), _stream(stream)), "moe_permute_n")
 
     def permute_noalloc(self, x, ids, counts, offsets, pos, src, x_perm, device_status=None,
                         stream=None):
@@ -193,15 +202,25 @@ class Plan:
                "moe_permute_noalloc")
 
     def grouped_ffn(self, x_perm, offsets, y_perm, ws, x_scale: float = 1.0, x_row_scales=None,
-                    stream=None):
-        _check(self.lib.moe_grouped_ffn(self.handle, _ptr(x_perm), _ptr(offsets), x_scale,
-                                        _ptr(x_row_scales), _ptr(y_perm), _ptr(ws), ws.numel(),
-                                        _stream(stream)), "moe_grouped_ffn")
+                    stream=None, n=None):
+        if n is None:
+            _check(self.lib.moe_grouped_ffn(self.handle, _ptr(x_perm), _ptr(offsets), x_scale,
+                                            _ptr(x_row_scales), _ptr(y_perm), _ptr(ws), ws.numel(),
+                                            _stream(stream)), "moe_grouped_ffn")
+        else:
+            _check(self.lib.moe_grouped_ffn_n(self.handle, int(n), _ptr(x_perm), _ptr(offsets),
+                                              x_scale, _ptr(x_row_scales), _ptr(y_perm), _ptr(ws),
+                                              ws.numel(), _stream(stream)), "moe_grouped_ffn_n")
 
-    def unpermute_combine(self, y_perm, pos, gates, y, ws, stream=None):
-        _check(self.lib.moe_unpermute_combine(self.handle, _ptr(y_perm), _ptr(pos), _ptr(gates),
-                                              _ptr(y), _ptr(ws), ws.numel(), _stream(stream)),
-               "moe_unpermute_combine")
+    def unpermute_combine(self, y_perm, pos, gates, y, ws, stream=None, n=None):
+        if n is None:
+            _check(self.lib.moe_unpermute_combine(self.handle, _ptr(y_perm), _ptr(pos),
+                                                  _ptr(gates), _ptr(y), _ptr(ws), ws.numel(),
+                                                  _stream(stream)), "moe_unpermute_combine")
+        else:
+            _check(self.lib.moe_unpermute_combine_n(self.handle, int(n), _ptr(y_perm), _ptr(pos),
+                                                    _ptr(gates), _ptr(y), _ptr(ws), ws.numel(),
+                                                    _stream(stream)), "moe_unpermute_combine_n")
 
     def shared_matmul(self, x, w, x_scale, w_scale, y, x_token_scales=None,
                       w_channel_scales=None, stream=None):

@@ -344,10 +344,14 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
     return MOE_ERR_INVALID_ARG;
   if (d.dtype == MOE_E4M3 && d.act != MOE_ACT_NONE) return MOE_ERR_UNSUPPORTED;
   if (d.dtype == MOE_BF16 && d.act == MOE_ACT_RELU) return MOE_ERR_UNSUPPORTED;
-  if (!w->w1 || (d.act == MOE_ACT_SWIGLU) != (w->w3 != nullptr) ||
-      (d.act != MOE_ACT_NONE) != (w->w2 != nullptr))
+  // a routing-only plan (no expert weights: router, permute and combine of
+  // an expert-parallel layer whose experts live on other GPUs) takes none of
+  // w1, w3, w2
+  const bool routing_only = !w->w1 && !w->w3 && !w->w2 && d.quant != MOE_QUANT_PER_CHANNEL;
+  if (!routing_only && (!w->w1 || (d.act == MOE_ACT_SWIGLU) != (w->w3 != nullptr) ||
+                        (d.act != MOE_ACT_NONE) != (w->w2 != nullptr)))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned16(w->w1) || (w->w3 && !aligned16(w->w3)) || (w->w2 && !aligned16(w->w2)) ||
+  if ((w->w1 && !aligned16(w->w1)) || (w->w3 && !aligned16(w->w3)) || (w->w2 && !aligned16(w->w2)) ||
       (w->w_r && !aligned16(w->w_r)))
     return MOE_ERR_INVALID_ARG;
 
@@ -371,7 +375,7 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
     delete p;
     return MOE_ERR_CUDA;
   }
-  if (uses_tensor_cores(d)) {
+  if (uses_tensor_cores(d) && !routing_only) {
     bool ok = true;
     const long long rows1 = static_cast<long long>(d.E) * d.F;
     if (d.act == MOE_ACT_NONE) {
@@ -436,15 +440,39 @@ moe_status moe_router_topk(moe_plan p, const void* x, int32_t* ids, float* gates
   return st;
 }
 
-moe_status moe_permute(moe_plan p, const void* x, const int32_t* ids, int32_t* counts,
-                       int32_t* offsets, int32_t* pos, int32_t* src, void* x_perm, void* ws,
-                       size_t ws_bytes, moe_stream_t stream) {
+moe_status moe_permute_n(moe_plan p, int32_t n, const void* x, const int32_t* ids,
+                         int32_t* counts, int32_t* offsets, int32_t* pos, int32_t* src,
+                         void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
   if (!p || !x || !ids || !counts || !offsets || !pos || !src || !x_perm) return MOE_ERR_INVALID_ARG;
+  if (n < 0 || n > p->desc.N) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
   moe_status st = check_ws(p, ws, ws_bytes, p->L.permute_end);
   if (st != MOE_OK) return st;
   begin(p);
-  st = run_permute(p, p->desc.N, x, ids, counts, offsets, pos, src, x_perm, ws, stream);
+  st = run_permute(p, n, x, ids, counts, offsets, pos, src, x_perm, ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_permute(moe_plan p, const void* x, const int32_t* ids, int32_t* counts,
+                       int32_t* offsets, int32_t* pos, int32_t* src, void* x_perm, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  return moe_permute_n(p, p->desc.N, x, ids, counts, offsets, pos, src, x_perm, ws, ws_bytes,
+                       stream);
+}
+
+moe_status moe_grouped_ffn_n(moe_plan p, int32_t n, const void* x_perm, const int32_t* offsets,
+                             float x_scale, const float* x_row_scales, void* y_perm, void* ws,
+                             size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !x_perm || !offsets || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (n < 0 || n > p->desc.N) return MOE_ERR_INVALID_ARG;
+  if (!p->w.w1) return MOE_ERR_UNSUPPORTED;  // routing-only plan
+  if (!aligned16(x_perm) || !aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.h_end);
+  if (st != MOE_OK) return st;
+  begin(p);
+  st = run_ffn(p, n, x_perm, offsets, x_scale, x_row_scales, nullptr, y_perm, ws, stream);
   end(p, stream);
   return st;
 }
@@ -452,12 +480,21 @@ moe_status moe_permute(moe_plan p, const void* x, const int32_t* ids, int32_t* c
 moe_status moe_grouped_ffn(moe_plan p, const void* x_perm, const int32_t* offsets, float x_scale,
                            const float* x_row_scales, void* y_perm, void* ws, size_t ws_bytes,
                            moe_stream_t stream) {
-  if (!p || !x_perm || !offsets || !y_perm) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x_perm) || !aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
-  moe_status st = check_ws(p, ws, ws_bytes, p->L.h_end);
+  if (!p) return MOE_ERR_INVALID_ARG;
+  return moe_grouped_ffn_n(p, p->desc.N, x_perm, offsets, x_scale, x_row_scales, y_perm, ws,
+                           ws_bytes, stream);
+}
+
+moe_status moe_unpermute_combine_n(moe_plan p, int32_t n, const void* y_perm,
+                                   const int32_t* pos, const float* gates, void* y, void* ws,
+                                   size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !y_perm || !pos || !y) return MOE_ERR_INVALID_ARG;
+  if (n < 0 || n > p->desc.N) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.chunk_counts);
   if (st != MOE_OK) return st;
   begin(p);
-  st = run_ffn(p, p->desc.N, x_perm, offsets, x_scale, x_row_scales, nullptr, y_perm, ws, stream);
+  st = run_combine(p, n, y_perm, pos, gates, y, ws, stream);
   end(p, stream);
   return st;
 }
@@ -465,14 +502,8 @@ moe_status moe_grouped_ffn(moe_plan p, const void* x_perm, const int32_t* offset
 moe_status moe_unpermute_combine(moe_plan p, const void* y_perm, const int32_t* pos,
                                  const float* gates, void* y, void* ws, size_t ws_bytes,
                                  moe_stream_t stream) {
-  if (!p || !y_perm || !pos || !y) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
-  moe_status st = check_ws(p, ws, ws_bytes, p->L.chunk_counts);
-  if (st != MOE_OK) return st;
-  begin(p);
-  st = run_combine(p, p->desc.N, y_perm, pos, gates, y, ws, stream);
-  end(p, stream);
-  return st;
+  if (!p) return MOE_ERR_INVALID_ARG;
+  return moe_unpermute_combine_n(p, p->desc.N, y_perm, pos, gates, y, ws, ws_bytes, stream);
 }
 
 moe_status moe_shared_matmul(moe_plan p, const void* x, int32_t M, int32_t H, const void* w,
@@ -510,6 +541,7 @@ moe_status moe_forward_routed(moe_plan p, const void* x, const int32_t* ids, con
                               float x_scale, const float* x_token_scales, void* y, void* ws,
                               size_t ws_bytes, moe_stream_t stream) {
   if (!p || !x || !ids || !y) return MOE_ERR_INVALID_ARG;
+  if (!p->w.w1) return MOE_ERR_UNSUPPORTED;  // routing-only plan
   if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   moe_status st = check_ws(p, ws, ws_bytes, p->L.fwd_end);
   if (st != MOE_OK) return st;
@@ -553,7 +585,7 @@ moe_status moe_forward_routed_dynamic(moe_plan p, const void* x_bf16, const int3
                                       const float* gates, void* y, void* ws, size_t ws_bytes,
                                       moe_stream_t stream) {
   if (!p || !x_bf16 || !ids || !y) return MOE_ERR_INVALID_ARG;
-  if (p->desc.dtype != MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (p->desc.dtype != MOE_E4M3 || !p->w.w1) return MOE_ERR_UNSUPPORTED;
   if (!aligned16(x_bf16) || !aligned16(y) || p->desc.d % 16) return MOE_ERR_INVALID_ARG;
   moe_status st = check_ws(p, ws, ws_bytes, p->L.fwd_end);
   if (st != MOE_OK) return st;
@@ -646,6 +678,7 @@ extern "C" {
 moe_status moe_forward(moe_plan p, const void* x, void* y, void* ws, size_t ws_bytes,
                        moe_stream_t stream) {
   if (!p || !x || !y || !p->w.w_r) return MOE_ERR_INVALID_ARG;
+  if (!p->w.w1) return MOE_ERR_UNSUPPORTED;  // routing-only plan
   if (p->desc.dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   moe_status st = check_ws(p, ws, ws_bytes, p->L.fwd_end);
@@ -665,7 +698,7 @@ moe_status moe_forward(moe_plan p, const void* x, void* y, void* ws, size_t ws_b
 moe_status moe_forward_host_async(moe_plan p, const void* x_host, void* y_host, void* ws,
                                   size_t ws_bytes, moe_stream_t stream) {
   if (!p || !x_host || !y_host || !p->w.w_r) return MOE_ERR_INVALID_ARG;
-  if (p->desc.dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (p->desc.dtype == MOE_E4M3 || !p->w.w1) return MOE_ERR_UNSUPPORTED;
   moe_status st = check_ws(p, ws, ws_bytes, p->L.total);
   if (st != MOE_OK) return st;
   if ((st = ensure_host_streams(p)) != MOE_OK) return st;

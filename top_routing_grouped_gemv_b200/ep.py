@@ -1,0 +1,176 @@
+"""Expert parallelism across GPUs: the experts of one layer are split over the
+ranks of a process group (rank r holds experts [r*E/G, (r+1)*E/G)), and each
+rank's tokens travel to the ranks that hold their experts and back
+("Advanced GPU Optimization ... Part 5", section 1.2 Expert Parallelism with
+All-to-All Communication: dispatch, local expert FFNs, combine;
+aclnnQuantGroupedMatMulAlltoAllv: AlltoAllv around the grouped matmul).
+
+One step on rank r (G ranks, E experts, E_loc = E / G):
+  1. route its N tokens over all E experts (router, top-K, gates);
+  2. permute the routed rows by expert: rows for rank q's experts are the
+     q-th contiguous block;
+  3. exchange the per-expert row counts (all-to-all of G x E_loc counts), so
+     that every rank knows how many rows it sends to and receives from each
+     rank (the host reads them: the split sizes of the next exchange);
+  4. all-to-all the rows (variable splits);
+  5. regroup the received rows by local expert (a permute with K = 1; rows
+     of one expert keep source-rank order), run the local experts on them,
+     and restore the received order (the pure reorder);
+  6. all-to-all the results back (the splits of step 4 swapped);
+  7. unpermute and combine with the gates.
+Every row is computed exactly as on one GPU, so the result equals the
+single-GPU layer's bit for bit.
+
+The per-step work is done by a `stages` object (the library's kernels on the
+GPU: `LibraryStages`); the exchanges use torch.distributed (NCCL on GPUs).
+Without an initialized process group the layer runs on one rank with no
+exchange.
+"""
+from __future__ import annotations
+
+import torch
+
+__all__ = ["ExpertParallelMoE", "LibraryStages"]
+
+
+def _dist():
+    import torch.distributed as dist
+    return dist if dist.is_available() and dist.is_initialized() else None
+
+
+class LibraryStages:
+    """The step's compute on this GPU through the C-ABI library: a
+    routing-only plan over all E experts for the rank's own tokens, and a
+    plan of the rank's E_loc experts (K = 1) for the rows it receives.
+
+    ``w_r`` (d, E) fp32 and optional ``bias`` route over all experts;
+    ``w1``/``w3``/``w2`` are this rank's experts only ((E_loc, F, d) etc.)."""
+
+    def __init__(self, N, d, E, K, F, dtype, act, world, w_r, w1, w3=None, w2=None, bias=None,
+                 w_scale=1.0):
+        from . import Plan
+        if E % world:
+            raise ValueError(f"{E} experts do not split over {world} ranks")
+        self.N, self.d, self.E, self.K, self.F = N, d, E, K, F
+        self.E_loc = E // world
+        self.d_out = F if act == "none" else d
+        self.dtype = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8}[dtype]
+        self.ydt = torch.float32 if dtype == "f32" else torch.bfloat16
+        route_w = {"w_r": w_r}
+        if bias is not None:
+            route_w["bias"] = bias
+        self.glob = Plan(N, d, E, K, F, dtype, act, route_w)
+        self.n_max = N * K * world  # every row of every rank may come here
+        local_w = {"w1": w1, "w_scale": w_scale}
+        if w3 is not None:
+            local_w["w3"] = w3
+        if w2 is not None:
+            local_w["w2"] = w2
+        self.loc = Plan(self.n_max, d, self.E_loc, 1, F, dtype, act, local_w)
+        self.ws_g = self.glob.new_workspace()
+        self.ws_l = self.loc.new_workspace()
+        dev = w_r.device
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.ids = torch.empty(N, K, **i32)
+        self.gates = torch.empty(N, K, dtype=torch.float32, device=dev)
+        self.counts = torch.empty(E, **i32)
+        self.offsets = torch.empty(E + 1, **i32)
+        self.pos = torch.empty(N * K, **i32)
+        self.src = torch.empty(N * K, **i32)
+        self.x_perm = torch.empty(N * K, d, dtype=self.dtype, device=dev)
+        self.counts_l = torch.empty(self.E_loc, **i32)
+        self.offsets_l = torch.empty(self.E_loc + 1, **i32)
+        self.pos_l = torch.empty(self.n_max, **i32)
+        self.src_l = torch.empty(self.n_max, **i32)
+        self.x_sorted = torch.empty(self.n_max, d, dtype=self.dtype, device=dev)
+        self.y_sorted = torch.empty(self.n_max, self.d_out, dtype=self.ydt, device=dev)
+
+    def route(self, x):
+        self.glob.router_topk(x, self.ids, self.gates, self.ws_g)
+        return self.ids, self.gates
+
+    def permute(self, x, ids):
+        self.glob.permute(x, ids, self.counts, self.offsets, self.pos, self.src, self.x_perm,
+                          self.ws_g)
+        return self.counts, self.offsets, self.pos, self.x_perm
+
+    def local_permute(self, n, x_recv, ids_recv):
+        self.loc.permute(x_recv, ids_recv, self.counts_l, self.offsets_l, self.pos_l, self.src_l,
+                         self.x_sorted, self.ws_l, n=n)
+        return self.offsets_l, self.pos_l, self.x_sorted
+
+    def local_ffn(self, n, x_sorted, offsets):
+        self.loc.grouped_ffn(x_sorted, offsets, self.y_sorted, self.ws_l, n=n)
+        return self.y_sorted
+
+    def local_unpermute(self, n, y_sorted, pos):
+        y_recv = torch.empty(max(n, 1), self.d_out, dtype=self.ydt, device=y_sorted.device)
+        self.loc.unpermute_combine(y_sorted, pos, None, y_recv, self.ws_l, n=n)
+        return y_recv[:n]
+
+    def combine(self, y_perm, pos, gates):
+        y = torch.empty(self.N, self.d_out, dtype=self.ydt, device=y_perm.device)
+        self.glob.unpermute_combine(y_perm, pos, gates, y, self.ws_g)
+        return y
+
+    def check(self):
+        """Sticky device status of both plans' workspaces (0 = clean)."""
+        return self.glob.read_device_status(self.ws_g) or self.loc.read_device_status(self.ws_l)
+
+
+class ExpertParallelMoE:
+    """The expert-parallel layer on this rank (see the module docstring)."""
+
+    def __init__(self, stages, E: int, K: int, group=None):
+        self.stages, self.E, self.K, self.group = stages, E, K, group
+
+    def _world(self):
+        dist = _dist()
+        if dist is None:
+            return None, 1, 0
+        return dist, dist.get_world_size(self.group), dist.get_rank(self.group)
+
+    def forward(self, x):
+        st = self.stages
+        dist, G, _ = self._world()
+        if self.E % G:
+            raise ValueError(f"{self.E} experts do not split over {G} ranks")
+        E_loc = self.E // G
+        ids, gates = st.route(x)
+        counts, offsets, pos, x_perm = st.permute(x, ids)
+
+        # per-expert row counts: block q of my counts goes to rank q
+        send_counts = counts.to(torch.int64).reshape(G, E_loc)
+        if dist is not None:
+            recv_counts = torch.empty_like(send_counts)
+            dist.all_to_all_single(recv_counts, send_counts, group=self.group)
+        else:
+            recv_counts = send_counts.clone()
+        send_h, recv_h = send_counts.cpu(), recv_counts.cpu()
+        send_rows = send_h.sum(1).tolist()
+        recv_rows = recv_h.sum(1).tolist()
+        n_send, n_recv = sum(send_rows), sum(recv_rows)
+
+        # dispatch: the rows, source-major, expert-minor within each source
+        if dist is not None:
+            x_recv = x_perm.new_empty((n_recv,) + tuple(x_perm.shape[1:]))
+            dist.all_to_all_single(x_recv, x_perm[:n_send].contiguous(), recv_rows, send_rows,
+                                   group=self.group)
+        else:
+            x_recv = x_perm[:n_send]
+        # regroup by local expert, run the local experts, restore the order
+        eids = torch.arange(E_loc, dtype=torch.int32).repeat(G)
+        ids_recv = torch.repeat_interleave(eids, recv_h.reshape(-1)).to(x_recv.device)
+        ids_recv = ids_recv.reshape(-1, 1).contiguous()
+        offsets_l, pos_l, x_sorted = st.local_permute(n_recv, x_recv, ids_recv)
+        y_sorted = st.local_ffn(n_recv, x_sorted, offsets_l)
+        y_recv = st.local_unpermute(n_recv, y_sorted, pos_l)
+
+        # return the results: the dispatch splits swapped
+        if dist is not None:
+            y_perm = y_recv.new_empty((n_send,) + tuple(y_recv.shape[1:]))
+            dist.all_to_all_single(y_perm, y_recv.contiguous(), send_rows, recv_rows,
+                                   group=self.group)
+        else:
+            y_perm = y_recv
+        return st.combine(y_perm, pos, gates)
