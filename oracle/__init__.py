@@ -63,6 +63,9 @@ def lib():
         L.orc_dense_masked.argtypes = [i, i, i, i, P, P, i, i, i, P, P, P, d, d, P]
         L.orc_matmul.argtypes = [i, i, i, P, P, P]
         L.orc_quantize_rows_dynamic.argtypes = [i, i, P, P, P]
+        L.orc_expert_rows_mx.argtypes = [i, P, i, i, P, P, i, P, P, P]
+        L.orc_e8m0_to_f64.argtypes = [ctypes.c_uint8]
+        L.orc_e8m0_to_f64.restype = d
         L.orc_bf16_to_f64.argtypes = [ctypes.c_uint16]
         L.orc_bf16_to_f64.restype = d
         L.orc_e4m3_to_f64.argtypes = [ctypes.c_uint8]
@@ -258,6 +261,24 @@ def quantize_rows_dynamic(x):
     _check(lib().orc_quantize_rows_dynamic(n, d, _p(xn), _p(codes), _p(scales)),
            "quantize_rows_dynamic")
     return codes, scales
+
+
+def e8m0_to_f64(s: int) -> float:
+    return lib().orc_e8m0_to_f64(s)
+
+
+def expert_rows_mx(row_expert, x, xs, w, ws):
+    """Single-matrix experts with MX block scales: x (n, din) e4m3 codes, xs
+    (n, din/32) E8M0, w (E, F, din) e4m3, ws (E, F, din/32) E8M0 -> y (n, F)
+    in double; rows with expert < 0 are left NaN."""
+    row_expert = np.ascontiguousarray(row_expert, np.int32)
+    xn, xsn = _np(x), _np(xs)
+    wn, wsn = _np(w), _np(ws)
+    E, F, din = wn.shape
+    y = np.full((len(row_expert), F), np.nan)
+    _check(lib().orc_expert_rows_mx(len(row_expert), _p(row_expert), E, din, _p(xn), _p(xsn), F,
+                                    _p(wn), _p(wsn), _p(y)), "expert_rows_mx")
+    return y
 
 
 def matmul(A, B):

@@ -23,6 +23,8 @@
  *    unpermuteOut = Unpermute(gmmY); shared expert
  *    mmY = (mmX @ mmWeight) * mmXScale * mmWeightScale; quant mode 1 =
  *    per-tensor; constraints: K in [2, 8], deterministic by default.
+ *    Quant mode 6 ("mx"): read as OCP MXFP8, e4m3 elements in blocks of 32
+ *    along the reduction dimension, each block with an E8M0 power-of-two scale.
  *  - zyxy.net "SpMM ... MoE inference", MoE structure: y = sum_i g_i(x)*E_i(x);
  *    expert selection: gating matrix (N, E), top-K index matrix (N, K),
  *    binary expert-activation matrix (N, E); SpMM section: C = A @ B.
@@ -362,6 +364,53 @@ int orc_expert_rows_scaled(int nrows, const int32_t* row_expert, int E, int din,
             for (int n = 0; n < F; ++n) {
                 double sw = ws ? ws[(int64_t)e * F + n] : w_scale;
                 y[(int64_t)r * F + n] = dot_row(din, xr, w1, w_dtype, (int64_t)e * F + n) * sx * sw;
+            }
+        }
+        free(xr);
+    }
+    return ORC_OK;
+}
+
+/* E8M0 (OCP Microscaling Formats v1.0, the shared block scale): eight
+ * exponent bits with bias 127, no sign and no mantissa; 0xFF encodes NaN. */
+double orc_e8m0_to_f64(uint8_t s) {
+    if (s == 0xFF) return NAN;
+    return ldexp(1.0, (int)s - 127);
+}
+
+/* Single-matrix experts with MX block scales (Ascend quant mode 6, "mx"; the
+ * block format is OCP MXFP8: 32 consecutive e4m3 elements along the
+ * reduction dimension share one E8M0 scale):
+ *   y[r][n] = sum_k (x[r][k] * 2^(xs[r][k/32] - 127)) * (W[e][n][k] * 2^(ws[e][n][k/32] - 127))
+ * with k ascending.  x (nrows, din) e4m3 codes, xs (nrows, din/32) E8M0;
+ * W (E, F, din) e4m3 (output-major), ws (E, F, din/32) E8M0; din a multiple
+ * of 32.  The page names the mode only; the block of 32 and E8M0 scales are
+ * the MX format's own definition. */
+int orc_expert_rows_mx(int nrows, const int32_t* row_expert, int E, int din, const uint8_t* x,
+                       const uint8_t* xs, int F, const uint8_t* w, const uint8_t* ws, double* y) {
+    if (nrows < 0 || !row_expert || !x || !xs || !w || !ws || !y || din <= 0 || F <= 0 ||
+        din % 32 != 0)
+        return ORC_ERR_ARG;
+    for (int r = 0; r < nrows; ++r)
+        if (row_expert[r] >= E) return ORC_ERR_INDEX;
+    const int nb = din / 32;
+#pragma omp parallel
+    {
+        double* xr = (double*)malloc(sizeof(double) * (size_t)din);
+#pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < nrows; ++r) {
+            int e = row_expert[r];
+            if (e < 0) continue;
+            for (int k = 0; k < din; ++k)
+                xr[k] = orc_e4m3_to_f64(x[(int64_t)r * din + k]) *
+                        orc_e8m0_to_f64(xs[(int64_t)r * nb + k / 32]);
+            for (int n = 0; n < F; ++n) {
+                int64_t wrow = (int64_t)e * F + n;
+                double acc = 0.0;
+                for (int k = 0; k < din; ++k)
+                    acc += xr[k] * (orc_e4m3_to_f64(w[wrow * din + k]) *
+                                    orc_e8m0_to_f64(ws[wrow * nb + k / 32]));
+                y[(int64_t)r * F + n] = acc;
             }
         }
         free(xr);

@@ -14,11 +14,14 @@ Workloads (the five shapes the layer is measured and checked on):
   router bias 1.2*ln(1/rank) (Zipf-like skew, some experts empty)
 * ``e4m3_n8192_h7168_e256_k8_n2048_gmm``    fp8 e4m3 per-tensor grouped matmul
   + token-major unpermute, plus a shared-expert matmul (8192x7168)@(7168x2048)
+* ``e4m3mx_n8192_h7168_e256_k8_n2048_gmm``  the same grouped matmul with MX block
+  scales (OCP MXFP8: one E8M0 scale per 32 consecutive elements along H1)
 
 Value recipe: x ~ N(0,1); router and expert weights ~ N(0, 1/fan_in)
 (fan_in = d for the router and the first FFN matrices, F for the second);
 for the fp8 workload x and W ~ N(0,1) quantised with one amax scale per
-tensor (scale = amax/448, e4m3 round-to-nearest-even, saturating).  Routing
+tensor (scale = amax/448, e4m3 round-to-nearest-even, saturating), or, for
+the MX workload, per block of 32 (scale 2^(floor(log2 amax) - 8)).  Routing
 for the fp8 workload is an ordered set of K distinct experts per token, drawn
 uniformly (the same law as the top-K of iid N(0,1) logits).
 
@@ -74,6 +77,7 @@ class MoEConfig:
     zipf_bias: float = 0.0          # router bias b_e = zipf_bias * ln(1/(e+1)); 0 = no bias
     shared: tuple | None = None     # (H2, N2) shared-expert matmul, fp8 workload only
     routing: str = "router"         # "router" (logits from x @ W_r) or "given" (drawn ids)
+    quant: str = "tensor"           # fp8 scales: "tensor" (one per tensor) or "mx" (E8M0 per 32)
 
     @property
     def d_out(self) -> int:
@@ -105,6 +109,8 @@ BF16_FINEGRAINED = _reg(MoEConfig("bf16_n16384_d2048_e128_k8_f768_swiglu_zipf", 
                                   2048, 128, 8, 768, ACT_SWIGLU, index=3, zipf_bias=1.2))
 FP8_GMM = _reg(MoEConfig("e4m3_n8192_h7168_e256_k8_n2048_gmm", DTYPE_E4M3, 8192, 7168, 256, 8, 2048,
                          ACT_NONE, index=4, shared=(7168, 2048), routing="given"))
+MX_GMM = _reg(MoEConfig("e4m3mx_n8192_h7168_e256_k8_n2048_gmm", DTYPE_E4M3, 8192, 7168, 256, 8,
+                        2048, ACT_NONE, index=5, routing="given", quant="mx"))
 
 
 # ----------------------------------------------------------------------------
@@ -239,6 +245,44 @@ def normal_e4m3(seed: int, stream: int, n: int) -> tuple[np.ndarray, float]:
     return out, scale
 
 
+def quantize_mx(a: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """OCP MXFP8 (E4M3) quantisation along the last axis (a multiple of 32):
+    each block of 32 gets the E8M0 scale 2^X, X = floor(log2(amax)) - 8 (8 =
+    the exponent of e4m3's largest normal, 448 = 1.75 * 2^8), clamped to
+    [-127, 127]; its elements become e4m3(v / 2^X), round to nearest even,
+    saturating.  An all-zero block gets X = -127 (scale code 0).  Returns
+    (codes uint8, same shape; scales uint8, last axis / 32)."""
+    a = np.asarray(a, np.float64)
+    d = a.shape[-1]
+    assert d % 32 == 0, "MX blocks are 32 elements"
+    b = a.reshape(-1, d // 32, 32)
+    amax = np.max(np.abs(b), axis=2)
+    _, ex = np.frexp(amax)                  # amax = m * 2^ex, m in [0.5, 1): floor(log2) = ex - 1
+    X = np.where(amax > 0, ex.astype(np.int64) - 1 - 8, -127)
+    X = np.clip(X, -127, 127)
+    codes = e4m3_encode(b / np.ldexp(1.0, X)[..., None])
+    return codes.reshape(a.shape), (X + 127).astype(np.uint8).reshape(a.shape[:-1] + (d // 32,))
+
+
+def normal_mx(seed: int, stream: int, rows: int, cols: int) -> tuple[np.ndarray, np.ndarray]:
+    """rows x cols iid N(0,1) draws quantised to MXFP8 (quantize_mx), chunk by
+    chunk of whole rows: (codes (rows, cols) uint8, scales (rows, cols/32))."""
+    rows_per = max(1, _CHUNK // cols)
+    nchunks = max(1, (rows + rows_per - 1) // rows_per)
+    children = np.random.SeedSequence([seed, stream]).spawn(nchunks)
+    codes = np.empty((rows, cols), np.uint8)
+    scales = np.empty((rows, cols // 32), np.uint8)
+
+    def work(i):
+        lo, hi = i * rows_per, min(rows, (i + 1) * rows_per)
+        v = np.random.Generator(np.random.Philox(children[i])).standard_normal(
+            (hi - lo) * cols, dtype=np.float32).reshape(hi - lo, cols)
+        codes[lo:hi], scales[lo:hi] = quantize_mx(v)
+
+    _run(work, nchunks)
+    return codes, scales
+
+
 def _run(fn, nchunks):
     if nchunks == 1:
         fn(0)
@@ -277,6 +321,8 @@ class MoEInputs:
     w_scale: float = 1.0
     w_sh: torch.Tensor | None = None
     w_sh_scale: float = 1.0
+    x_sf: torch.Tensor | None = None    # (N, d/32) uint8 E8M0, MX workload
+    w_sf: torch.Tensor | None = None    # (E, F, d/32) uint8 E8M0, MX workload
     extra: dict = field(default_factory=dict)
 
 
@@ -307,6 +353,14 @@ def make_inputs(cfg: MoEConfig, seed: int | None = None) -> MoEInputs:
     if seed is None:
         seed = SEED_BASE + cfg.index
     N, d, E, K, F = cfg.N, cfg.d, cfg.E, cfg.K, cfg.F
+    if cfg.dtype == DTYPE_E4M3 and cfg.quant == "mx":
+        xq, xsf = normal_mx(seed, 1, N, d)
+        wq, wsf = normal_mx(seed, 2, E * F, d)
+        return MoEInputs(cfg, torch.from_numpy(xq), None, None,
+                         torch.from_numpy(wq.reshape(E, F, d)), None, None,
+                         ids=torch.from_numpy(given_routing(seed, N, E, K)),
+                         x_sf=torch.from_numpy(xsf),
+                         w_sf=torch.from_numpy(wsf.reshape(E, F, d // 32)))
     if cfg.dtype == DTYPE_E4M3:
         xq, xs = normal_e4m3(seed, 1, N * d)
         wq, ws = normal_e4m3(seed, 2, E * F * d)

@@ -63,6 +63,15 @@ MUTANTS = [
     ("e4m3 subnormals scaled like normals",
      "v = ldexp((double)m, -9);              /* m/8 * 2^(1-7) */",
      "v = ldexp((double)m, -10);"),
+    ("MX scale taken from the next block",
+     "orc_e8m0_to_f64(xs[(int64_t)r * nb + k / 32]);",
+     "orc_e8m0_to_f64(xs[(int64_t)r * nb + (k / 32 + 1) % nb]);"),
+    ("MX weight scales of expert 0 for every expert",
+     "orc_e8m0_to_f64(ws[wrow * nb + k / 32]));",
+     "orc_e8m0_to_f64(ws[(int64_t)n * nb + k / 32]));"),
+    ("E8M0 bias 128 instead of 127",
+     "return ldexp(1.0, (int)s - 127);",
+     "return ldexp(1.0, (int)s - 128);"),
     ("bf16 widened from the wrong half",
      "uint32_t u = (uint32_t)b << 16;",
      "uint32_t u = ((uint32_t)b << 16) | 0x8000u;"),

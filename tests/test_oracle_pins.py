@@ -327,6 +327,132 @@ def test_fp8_per_channel_and_per_token_scales_exact(orc):
     assert np.array_equal(y0, y1)
 
 
+def test_e8m0_decode_definition(orc):
+    """OCP MX E8M0 scale: 2^(code - 127), code 255 is NaN."""
+    assert orc.e8m0_to_f64(127) == 1.0
+    assert orc.e8m0_to_f64(128) == 2.0
+    assert orc.e8m0_to_f64(120) == 2.0 ** -7
+    assert orc.e8m0_to_f64(0) == 2.0 ** -127
+    assert orc.e8m0_to_f64(254) == 2.0 ** 127
+    assert math.isnan(orc.e8m0_to_f64(255))
+
+
+def _mx_ones(*shape):
+    return np.full(shape, 0x38, np.uint8)   # e4m3 1.0
+
+
+def test_mx_block_scales_closed_form(orc):
+    """Quant mode 6 (MX): with every element 1.0 and scales xs[r][b] =
+    127 + r + b, ws[e][n][b] = 127 - n + 2b + e, each block of 32 adds
+    32 * 2^(r + b) * 2^(2b - n + e), so y[r][n] = 32 * 2^(r - n + e) *
+    (8^nb - 1) / 7 with nb = din / 32 blocks.  A block size other than 32,
+    a transposed scale index or another expert's scales all change it."""
+    E, F, nb, R = 3, 5, 4, 6
+    din = 32 * nb
+    xs = np.array([[127 + r + b for b in range(nb)] for r in range(R)], np.uint8)
+    ws = np.array([[[127 - n + 2 * b + e for b in range(nb)] for n in range(F)] for e in range(E)],
+                  np.uint8)
+    rexp = np.array([0, 1, 2, 2, 1, 0], np.int32)
+    y = orc.expert_rows_mx(rexp, _mx_ones(R, din), xs, _mx_ones(E, F, din), ws)
+    for r in range(R):
+        e = int(rexp[r])
+        for n in range(F):
+            assert y[r, n] == 32 * 2.0 ** (r - n + e) * (8 ** nb - 1) / 7
+
+
+def test_mx_exact_integers_random_block_scales(orc):
+    """Small integer codes and random power-of-two block scales: every product
+    and partial sum is exact in fp64, so y equals the exact value
+    sum_b 2^(xs + ws - 254) * sum_{k in block b} X*W from Python integers."""
+    rng = np.random.default_rng(21)
+    E, F, nb, R = 3, 4, 3, 7
+    din = 32 * nb
+    Xi = rng.integers(-8, 9, size=(R, din))
+    Wi = rng.integers(-8, 9, size=(E, F, din))
+    enc = np.vectorize(orc.f64_to_e4m3, otypes=[np.uint8])
+    Xq, Wq = enc(Xi.astype(np.float64)), enc(Wi.astype(np.float64))
+    xs = rng.integers(120, 135, size=(R, nb)).astype(np.uint8)
+    ws = rng.integers(120, 135, size=(E, F, nb)).astype(np.uint8)
+    rexp = rng.integers(0, E, size=R).astype(np.int32)
+    rexp[2] = -1
+    y = orc.expert_rows_mx(rexp, Xq, xs, Wq, ws)
+    assert np.isnan(y[2]).all()
+    for r in range(R):
+        e = int(rexp[r])
+        if e < 0:
+            continue
+        for n in range(F):
+            exact = 0.0
+            for b in range(nb):
+                blk = sum(int(Xi[r, k]) * int(Wi[e, n, k]) for k in range(32 * b, 32 * b + 32))
+                exact += blk * 2.0 ** (int(xs[r, b]) + int(ws[e, n, b]) - 254)
+            assert y[r, n] == exact
+
+
+def test_mx_unit_scales_equal_plain_fp8(orc):
+    """With every block scale 1 (code 127) the MX matmul is the per-tensor fp8
+    matmul with unit scales, bit for bit (same products, same order)."""
+    cfg = synth.MoEConfig("mx1", "e4m3", 12, 64, 4, 2, 24, "none", routing="given", quant="mx")
+    inp = synth.make_inputs(cfg, 7)
+    rexp = np.arange(12, dtype=np.int32) % 4
+    ones_x = np.full((12, 2), 127, np.uint8)
+    ones_w = np.full((4, 24, 2), 127, np.uint8)
+    y = orc.expert_rows_mx(rexp, inp.x, ones_x, inp.w1, ones_w)
+    y0 = orc.expert_rows(rexp, inp.x, orc.E4M3, "none", inp.w1, None, None, orc.E4M3, 1.0, 1.0)
+    assert np.array_equal(y, y0)
+
+
+def test_mx_row_and_column_constant_scales_reduce_to_matmul(orc):
+    """When a row's blocks share one scale 2^a[r] and an output column's blocks
+    share 2^c[n], y = diag(2^a) (Xd W_e^T) diag(2^c): the library matmul (fp64)
+    of the decoded codes, per expert."""
+    rng = np.random.default_rng(4)
+    cfg = synth.MoEConfig("mx2", "e4m3", 10, 96, 2, 1, 16, "none", routing="given", quant="mx")
+    inp = synth.make_inputs(cfg, 11)
+    a = rng.integers(118, 136, size=10)
+    c = rng.integers(118, 136, size=(2, 16))
+    xs = np.repeat(a[:, None], 3, axis=1).astype(np.uint8)
+    ws = np.repeat(c[:, :, None], 3, axis=2).astype(np.uint8)
+    rexp = np.array([0, 1] * 5, np.int32)
+    y = orc.expert_rows_mx(rexp, inp.x, xs, inp.w1, ws)
+    dec = np.array([orc.e4m3_to_f64(v) for v in range(256)])
+    Xd = torch.from_numpy(dec[inp.x.numpy()])
+    for e in range(2):
+        rows = np.nonzero(rexp == e)[0]
+        Wd = torch.from_numpy(dec[inp.w1[e].numpy()])
+        ref = (Xd[rows] @ Wd.T).numpy() * 2.0 ** (a[rows, None] - 127) * 2.0 ** (c[e][None, :] - 127)
+        assert np.abs(y[rows] - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_mx_quantiser_blocks(orc):
+    """The MX input quantiser (OCP MXFP8): a block of e4m3 values whose largest
+    magnitude is in [256, 448], times 2^p, gets scale code 127 + p and its
+    codes back exactly; an all-zero block gets scale code 0; every block's
+    largest element lands in [256, 448] times its scale."""
+    base = [448.0, 1.0, -2.0, 0.5, -300.0, 3.5, -448.0, 0.001953125] * 4
+    codes_ref = [orc.f64_to_e4m3(v) for v in base]
+    for p in (-9, -1, 0, 5):
+        c, s = synth.quantize_mx(np.array([[v * 2.0 ** p for v in base]]))
+        assert int(s[0, 0]) == 127 + p
+        assert [int(v) for v in c[0]] == codes_ref
+    c, s = synth.quantize_mx(np.zeros((1, 64)))
+    assert not s.any() and not c.any()
+    rng = np.random.default_rng(2)
+    v = rng.standard_normal((8, 128)) * np.exp(rng.uniform(-5, 5, (8, 1)))
+    c, s = synth.quantize_mx(v)
+    dec = np.array([orc.e4m3_to_f64(int(q)) for q in c.ravel()]).reshape(c.shape)
+    for r in range(8):
+        for b in range(4):
+            blk = np.abs(dec[r, 32 * b:32 * b + 32])
+            assert 256.0 <= blk.max() <= 448.0
+            scale = 2.0 ** (int(s[r, b]) - 127)
+            err = np.abs(dec[r, 32 * b:32 * b + 32] * scale - v[r, 32 * b:32 * b + 32])
+            # half an e4m3 step (2^-4 relative) or the saturation at 448
+            big = np.abs(v[r, 32 * b:32 * b + 32]) / scale > 448.0
+            assert np.all((err <= np.abs(v[r, 32 * b:32 * b + 32]) * 2.0 ** -4 + 2.0 ** -10 * scale)
+                          | big)
+
+
 def test_per_row_quantiser_round_trip():
     rng = np.random.default_rng(2)
     a = rng.standard_normal((50, 64)) * rng.uniform(0.01, 100, size=(50, 1))
