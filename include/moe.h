@@ -94,13 +94,20 @@ typedef enum { MOE_ACT_NONE = 0, MOE_ACT_RELU = 1, MOE_ACT_SWIGLU = 2 } moe_act;
 
 /* Scale granularity of the expert weights; values equal the Ascend page's
  * quant-mode enumeration (0 = not quantised, 1 = per-tensor, 2 =
- * per-channel: one scale per output column of each expert).  Per-token
- * activation scales (mode 3) are a per-call argument (x_token_scales).
- * Group, block and mx modes are not built. */
+ * per-channel: one scale per output column of each expert, 6 = mx).
+ * Per-token activation scales (mode 3) are a per-call argument
+ * (x_token_scales); per-token dynamic quantization (mode 7) is
+ * moe_permute_quant.  MX is read as OCP MXFP8: e4m3 elements in blocks of
+ * 32 consecutive values along the reduction dimension (d), each block with
+ * one E8M0 scale byte 2^(s - 127) (255 = NaN), for the weights
+ * (w_mx_scales) and the activations (the _mx calls' x_mx_scales); the
+ * single-matrix layer only.  Group and block modes (4, 5) are not built
+ * (MOE_ERR_UNSUPPORTED). */
 typedef enum {
   MOE_QUANT_NONE = 0,
   MOE_QUANT_PER_TENSOR = 1,
-  MOE_QUANT_PER_CHANNEL = 2
+  MOE_QUANT_PER_CHANNEL = 2,
+  MOE_QUANT_MX = 6
 } moe_quant;
 
 typedef struct {
@@ -122,6 +129,8 @@ typedef struct {
   const void* w2;           /* (E, d, F) for RELU / SWIGLU, else NULL */
   float w_scale;            /* per-tensor weight scale (gmmWeightScale), e4m3 PER_TENSOR */
   const float* w_channel_scales; /* (E, F) fp32 per output channel, e4m3 PER_CHANNEL, else NULL */
+  const uint8_t* w_mx_scales;    /* (E, F, d/32) E8M0 of w1, MOE_QUANT_MX, else NULL; read
+                                    once by moe_plan_create (may be freed afterwards) */
 } moe_layer_weights;
 
 typedef struct moe_plan_s* moe_plan;
@@ -130,7 +139,11 @@ typedef struct moe_plan_s* moe_plan;
 
 /* Validates desc and weights, records the weight pointers (not owned: they
  * must stay valid while the plan is used) and encodes the TMA descriptors of
- * the weights for the current CUDA device.  Allocates host memory only.
+ * the weights for the current CUDA device.  Allocates host memory only,
+ * except for MOE_QUANT_MX: the plan then also holds a device copy of the
+ * weight scales in the layout of the block-scaled tensor-core MMA (the same
+ * bytes as w_mx_scales, rearranged; about E*F*d/32 bytes), made here
+ * (synchronously) and freed by moe_plan_destroy.
  * With w1, w3 and w2 all NULL (and no per-channel scales) the plan is
  * routing-only: router, permute and unpermute/combine work, the calls that
  * run the experts return MOE_ERR_UNSUPPORTED (an expert-parallel rank's
@@ -276,6 +289,31 @@ moe_status moe_forward_routed_shared(moe_plan plan, const void* x, const int32_t
                                      const void* w_sh, int32_t N2, float w_sh_scale,
                                      const float* w_sh_channel_scales_or_null, void* y_sh,
                                      void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* MX layer (MOE_QUANT_MX, act NONE): x (N, d) e4m3 codes with x_mx_scales
+ * (N, d/32) E8M0, one per 32 consecutive elements of a row.  Computes, per
+ * routed row of expert e,
+ *   gmmY[r][n] = sum_k (x[r][k] * 2^(xs[r][k/32] - 127)) * (W[e][n][k] * 2^(ws[e][n][k/32] - 127))
+ * in fp32 on the tensor cores (block-scaled tcgen05 MMA), rounded once to
+ * bf16.  moe_forward_routed_mx: permute, the scales of every permuted row
+ * rearranged for the MMA (in ws), the grouped matmul, then pure unpermute
+ * (gates NULL: y (N*K, F), done by the GEMM's stores) or combine (y (N, F)).
+ * moe_permute_mx: moe_permute plus x_perm_mx_scales (N*K, d/32), row r the
+ * scales of x row perm_src[r].  moe_grouped_ffn_mx: the grouped matmul of
+ * permuted rows x_perm with their scales x_perm_mx_scales (N*K, d/32).
+ * MOE_ERR_UNSUPPORTED for a plan that is not MX; the other FFN calls return
+ * MOE_ERR_UNSUPPORTED for an MX plan. */
+moe_status moe_forward_routed_mx(moe_plan plan, const void* x, const uint8_t* x_mx_scales,
+                                 const int32_t* topk_ids, const float* topk_gates_or_null,
+                                 void* y, void* ws, size_t ws_bytes, moe_stream_t stream);
+moe_status moe_permute_mx(moe_plan plan, const void* x, const uint8_t* x_mx_scales,
+                          const int32_t* topk_ids, int32_t* counts, int32_t* offsets,
+                          int32_t* perm_pos, int32_t* perm_src, void* x_perm,
+                          uint8_t* x_perm_mx_scales, void* ws, size_t ws_bytes,
+                          moe_stream_t stream);
+moe_status moe_grouped_ffn_mx(moe_plan plan, const void* x_perm, const uint8_t* x_perm_mx_scales,
+                              const int32_t* offsets, void* y_perm, void* ws, size_t ws_bytes,
+                              moe_stream_t stream);
 
 /* Permute with per-token dynamic quantization (Ascend quant mode 7,
  * "pertoken dynamic quantization", parameter section): for an e4m3 plan, x is

@@ -28,7 +28,7 @@ def test_library_exports_every_header_symbol(lib):
 
 def test_struct_layouts_match_header():
     assert ctypes.sizeof(moe.LayerDesc) == 32
-    assert ctypes.sizeof(moe.LayerWeights) == 56
+    assert ctypes.sizeof(moe.LayerWeights) == 64
 
 
 def test_status_strings(lib):
@@ -37,9 +37,9 @@ def test_status_strings(lib):
 
 
 def _create(lib, N=64, d=64, E=8, K=2, F=64, dtype=moe.MOE_BF16, act=moe.ACT_SWIGLU,
-            quant=moe.QUANT_NONE, w1=0x1000, w3=0x2000, w2=0x3000, w_r=0x4000):
+            quant=moe.QUANT_NONE, w1=0x1000, w3=0x2000, w2=0x3000, w_r=0x4000, w_mx=None):
     desc = moe.LayerDesc(N, d, E, K, F, dtype, act, quant)
-    w = moe.LayerWeights(w_r, None, w1, w3, w2, 1.0, None)
+    w = moe.LayerWeights(w_r, None, w1, w3, w2, 1.0, None, w_mx)
     h = ctypes.c_void_p()
     rc = lib.moe_plan_create(ctypes.byref(desc), ctypes.byref(w), ctypes.byref(h))
     if rc == 0:
@@ -54,7 +54,16 @@ def _create(lib, N=64, d=64, E=8, K=2, F=64, dtype=moe.MOE_BF16, act=moe.ACT_SWI
     (dict(quant=moe.QUANT_PER_TENSOR), 2),                                 # per-tensor needs e4m3
     (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None,
           quant=moe.QUANT_PER_CHANNEL), 1),                                # per-channel needs scales
-    (dict(quant=7), 1),                                                    # mode not built
+    (dict(quant=7), 1),                                                    # mode 7 is per call
+    (dict(quant=4), 2), (dict(quant=5), 2),                                # group, block: not built
+    (dict(quant=3), 2),                                                    # per-token is per call
+    (dict(quant=moe.QUANT_MX, w_mx=0x5000), 2),                            # MX needs e4m3
+    (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None,
+          quant=moe.QUANT_MX), 1),                                         # MX needs its scales
+    (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None, d=48,
+          quant=moe.QUANT_MX, w_mx=0x5000), 1),                            # d not a multiple of 32
+    (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None,
+          quant=moe.QUANT_PER_TENSOR, w_mx=0x5000), 1),                    # scales without MX
     (dict(dtype=moe.MOE_E4M3, act=moe.ACT_SWIGLU, quant=moe.QUANT_PER_TENSOR), 2),
     (dict(dtype=moe.MOE_BF16, act=moe.ACT_RELU, w3=None), 2),
     (dict(w3=None), 1),                                                    # SwiGLU needs w3

@@ -651,3 +651,141 @@ def test_expert_parallel_stages_single_rank_equal_forward(name):
     assert stages.check() == 0
     assert torch.equal(y.view(torch.int32 if c.dtype == "f32" else torch.int16),
                        y_ref.view(torch.int32 if c.dtype == "f32" else torch.int16))
+
+
+# ---------------------------------------------------------------- MX (quant mode 6)
+
+MX = {
+    # two K stages, two column tiles (the second ragged), ~75 rows per expert
+    "mx_small": synth.MoEConfig("mx_small", "e4m3", 300, 256, 8, 2, 384, "none",
+                                routing="given", quant="mx"),
+    # K = 160: one full 128-element stage and a 32-element tail; ragged rows
+    "mx_ragged": synth.MoEConfig("mx_ragged", "e4m3", 257, 160, 5, 3, 200, "none",
+                                 routing="given", quant="mx"),
+    # many small experts (K = 8 of 64, ~16 rows each), several row tiles
+    "mx_fine": synth.MoEConfig("mx_fine", "e4m3", 128, 512, 64, 8, 256, "none",
+                               routing="given", quant="mx"),
+    # empty experts, single-row groups
+    "mx_sparse": synth.MoEConfig("mx_sparse", "e4m3", 20, 128, 16, 1, 64, "none",
+                                 routing="given", quant="mx"),
+    # an expert with more than one 128-row tile (500 rows over 2 experts)
+    "mx_tall": synth.MoEConfig("mx_tall", "e4m3", 500, 384, 2, 1, 512, "none",
+                               routing="given", quant="mx"),
+}
+_mx_cache = {}
+
+
+def mx_case(name, wide=True):
+    """Inputs of an MX case; wide=True replaces the quantiser's scales (which
+    are nearly equal for N(0,1) data) by independent random E8M0 codes in
+    [117, 137] for every block of x and W, so that any misplaced scale shows."""
+    key = (name, wide)
+    if key not in _mx_cache:
+        import top_routing_grouped_gemv_b200 as moe
+        c = MX[name]
+        inp = synth.make_inputs(c, 31 + sum(map(ord, name)))
+        xs, ws = inp.x_sf.numpy(), inp.w_sf.numpy()
+        if wide:
+            rng = np.random.default_rng(sum(map(ord, name)))
+            xs = rng.integers(117, 138, size=xs.shape).astype(np.uint8)
+            ws = rng.integers(117, 138, size=ws.shape).astype(np.uint8)
+        w = {"w1": inp.w1.cuda(), "w_mx_scales": torch.from_numpy(ws).cuda()}
+        plan = moe.Plan(c.N, c.d, c.E, c.K, c.F, "e4m3", "none", w)
+        _mx_cache[key] = (inp, plan, w, xs, ws)
+    return _mx_cache[key]
+
+
+def mx_ref(inp, xs, ws, gates):
+    """Oracle: permute, MX experts on the permuted rows, unpermute/combine."""
+    c = inp.cfg
+    ids = inp.ids.numpy()
+    _, _, rp, rs, rx = oracle.permute(ids, c.E, inp.x.numpy())
+    row_e = np.repeat(np.arange(c.E, dtype=np.int32), np.bincount(ids.ravel(), minlength=c.E))
+    yp = oracle.expert_rows_mx(row_e, rx, xs[rs], inp.w1, ws)
+    return oracle.combine(rp, gates, yp, c.N, c.K), yp
+
+
+@pytest.mark.parametrize("name", list(MX))
+@pytest.mark.parametrize("gated", [False, True])
+def test_forward_routed_mx(name, gated):
+    inp, plan, w, xs, ws = mx_case(name)
+    c = inp.cfg
+    wsp = plan.new_workspace()
+    g = None
+    if gated:
+        g = np.random.default_rng(3).random((c.N, c.K)).astype(np.float32)
+        y = torch.empty(c.N, c.F, dtype=torch.bfloat16, device="cuda")
+    else:
+        y = torch.full((c.N * c.K, c.F), float("nan"), dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed_mx(inp.x.cuda(), torch.from_numpy(xs).cuda(), inp.ids.cuda(),
+                           None if g is None else torch.from_numpy(g).cuda(), y, wsp)
+    assert plan.read_device_status(wsp) == 0
+    ref, _ = mx_ref(inp, xs, ws, None if g is None else g.astype(np.float64))
+    err = rel_err(f64(y), ref)
+    assert err <= TOL["e4m3"], err
+    # fp32 accumulation of exact e4m3 x E8M0 products, one bf16 rounding: far
+    # inside the fp8 bar; a misplaced scale (a factor 2^1..2^20) is not
+    assert err <= 1e-2, err
+
+
+@pytest.mark.parametrize("name", ["mx_small", "mx_ragged", "mx_sparse"])
+def test_mx_stage_calls_and_fused_path_agree(name):
+    """moe_permute_mx (codes and scale rows bit-exact), moe_grouped_ffn_mx
+    (against the oracle), and the fused call's unpermuted rows equal to the
+    stage composition bit for bit."""
+    inp, plan, w, xs, ws = mx_case(name)
+    c = inp.cfg
+    R = c.N * c.K
+    wsp = plan.new_workspace()
+    i32 = dict(dtype=torch.int32, device="cuda")
+    counts, offsets = torch.empty(c.E, **i32), torch.empty(c.E + 1, **i32)
+    pos, src = torch.empty(R, **i32), torch.empty(R, **i32)
+    x_perm = torch.empty(R, c.d, dtype=torch.uint8, device="cuda")
+    sf_perm = torch.empty(R, c.d // 32, dtype=torch.uint8, device="cuda")
+    plan.permute_mx(inp.x.cuda(), torch.from_numpy(xs).cuda(), inp.ids.cuda(), counts, offsets,
+                    pos, src, x_perm, sf_perm, wsp)
+    assert plan.read_device_status(wsp) == 0
+    _, ro, rp, rs, rx = oracle.permute(inp.ids.numpy(), c.E, inp.x.numpy())
+    assert np.array_equal(offsets.cpu().numpy(), ro) and np.array_equal(pos.cpu().numpy(), rp)
+    assert np.array_equal(x_perm.cpu().numpy(), rx)
+    assert np.array_equal(sf_perm.cpu().numpy(), xs[rs])
+    y_perm = torch.empty(R, c.F, dtype=torch.bfloat16, device="cuda")
+    plan.grouped_ffn_mx(x_perm, sf_perm, offsets, y_perm, wsp)
+    assert plan.read_device_status(wsp) == 0
+    _, yp_ref = mx_ref(inp, xs, ws, None)
+    assert rel_err(f64(y_perm), yp_ref) <= 1e-2
+    y = torch.empty(R, c.F, dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed_mx(inp.x.cuda(), torch.from_numpy(xs).cuda(), inp.ids.cuda(), None, y, wsp)
+    yp = y_perm.cpu().view(torch.int16).numpy()
+    assert np.array_equal(y.cpu().view(torch.int16).numpy(), yp[rp])
+
+
+def test_mx_with_quantiser_scales():
+    """The same path on the MX quantiser's own scales (OCP MXFP8 of N(0,1))."""
+    inp, plan, w, xs, ws = mx_case("mx_small", wide=False)
+    c = inp.cfg
+    wsp = plan.new_workspace()
+    y = torch.empty(c.N * c.K, c.F, dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed_mx(inp.x.cuda(), torch.from_numpy(xs).cuda(), inp.ids.cuda(), None, y, wsp)
+    assert plan.read_device_status(wsp) == 0
+    ref, _ = mx_ref(inp, xs, ws, None)
+    assert rel_err(f64(y), ref) <= 1e-2
+
+
+def test_mx_and_per_tensor_calls_are_not_mixed():
+    import top_routing_grouped_gemv_b200 as moe
+    inp, plan, w, xs, ws = mx_case("mx_sparse")
+    c = inp.cfg
+    wsp = plan.new_workspace()
+    y = torch.empty(c.N * c.K, c.F, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(moe.MoEError) as e:
+        plan.forward_routed(inp.x.cuda(), inp.ids.cuda(), None, y, wsp)
+    assert e.value.code == 2
+    inp8, plan8, _ = case("e4m3_gmm")
+    ws8 = plan8.new_workspace()
+    y8 = torch.empty(inp8.cfg.N * inp8.cfg.K, inp8.cfg.F, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(moe.MoEError) as e:
+        plan8.forward_routed_mx(inp8.x.cuda(), torch.zeros(inp8.cfg.N, inp8.cfg.d // 32,
+                                                           dtype=torch.uint8, device="cuda"),
+                                inp8.ids.cuda(), None, y8, ws8)
+    assert e.value.code == 2

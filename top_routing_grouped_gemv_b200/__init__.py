@@ -20,7 +20,7 @@ HEADER = os.path.join(ROOT, "include", "moe.h")
 
 MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
 ACT_NONE, ACT_RELU, ACT_SWIGLU = 0, 1, 2
-QUANT_NONE, QUANT_PER_TENSOR, QUANT_PER_CHANNEL = 0, 1, 2
+QUANT_NONE, QUANT_PER_TENSOR, QUANT_PER_CHANNEL, QUANT_MX = 0, 1, 2, 6
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
           3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_BAD_INDEX",
@@ -44,7 +44,8 @@ class LayerDesc(ctypes.Structure):
 class LayerWeights(ctypes.Structure):
     _fields_ = [("w_r", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
                 ("w1", ctypes.c_void_p), ("w3", ctypes.c_void_p), ("w2", ctypes.c_void_p),
-                ("w_scale", ctypes.c_float), ("w_channel_scales", ctypes.c_void_p)]
+                ("w_scale", ctypes.c_float), ("w_channel_scales", ctypes.c_void_p),
+                ("w_mx_scales", ctypes.c_void_p)]
 
 
 _lib = None
@@ -87,6 +88,9 @@ def load(path: str = LIB_PATH):
         "moe_forward_routed_shared": ([P, P, P, P, f32, P, P, P, i32, f32, P, P, P, sz, P],
                                       ctypes.c_int),
         "moe_forward_routed_dynamic": ([P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_forward_routed_mx": ([P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_permute_mx": ([P, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_grouped_ffn_mx": ([P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_permute_n": ([P, i32, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_grouped_ffn_n": ([P, i32, P, P, f32, P, P, P, sz, P], ctypes.c_int),
         "moe_unpermute_combine_n": ([P, i32, P, P, P, P, P, sz, P], ctypes.c_int),
@@ -129,8 +133,10 @@ class Plan:
 
     ``weights``: dict with torch CUDA tensors ``w_r`` (d, E) fp32, optional
     ``bias`` (E,), ``w1`` (E, F, d), ``w3`` (E, F, d) for SwiGLU, ``w2``
-    (E, d, F), and float ``w_scale`` (e4m3).  The tensors are kept alive by
-    the plan (the library only records their addresses).
+    (E, d, F), and float ``w_scale`` (e4m3); for e4m3, optional
+    ``w_channel_scales`` (E, F) fp32 (per-channel) or ``w_mx_scales`` (E, F,
+    d/32) uint8 E8M0 (MX).  The tensors are kept alive by the plan (the
+    library only records their addresses).
     """
 
     def __init__(self, N, d, E, K, F, dtype: str, act: str, weights: dict):
@@ -142,12 +148,12 @@ class Plan:
         quant = QUANT_NONE
         if dtype == "e4m3":
             quant = QUANT_PER_CHANNEL if weights.get("w_channel_scales") is not None \
-                else QUANT_PER_TENSOR
+                else QUANT_MX if weights.get("w_mx_scales") is not None else QUANT_PER_TENSOR
         desc = LayerDesc(N, d, E, K, F, DTYPE_CODE[dtype], ACT_CODE[act], quant)
         w = LayerWeights(_ptr(weights.get("w_r")), _ptr(weights.get("bias")),
                          _ptr(weights.get("w1")), _ptr(weights.get("w3")),
                          _ptr(weights.get("w2")), float(weights.get("w_scale", 1.0)),
-                         _ptr(weights.get("w_channel_scales")))
+                         _ptr(weights.get("w_channel_scales")), _ptr(weights.get("w_mx_scales")))
         h = ctypes.c_void_p()
         _check(self.lib.moe_plan_create(ctypes.byref(desc), ctypes.byref(w), ctypes.byref(h)),
                "moe_plan_create")
@@ -246,6 +252,23 @@ class Plan:
                                           _ptr(offsets), _ptr(pos), _ptr(src), _ptr(x_perm),
                                           _ptr(token_scales), _ptr(ws), ws.numel(),
                                           _stream(stream)), "moe_permute_quant")
+
+    def forward_routed_mx(self, x, x_mx_scales, ids, gates, y, ws, stream=None):
+        _check(self.lib.moe_forward_routed_mx(self.handle, _ptr(x), _ptr(x_mx_scales), _ptr(ids),
+                                              _ptr(gates), _ptr(y), _ptr(ws), ws.numel(),
+                                              _stream(stream)), "moe_forward_routed_mx")
+
+    def permute_mx(self, x, x_mx_scales, ids, counts, offsets, pos, src, x_perm,
+                   x_perm_mx_scales, ws, stream=None):
+        _check(self.lib.moe_permute_mx(self.handle, _ptr(x), _ptr(x_mx_scales), _ptr(ids),
+                                       _ptr(counts), _ptr(offsets), _ptr(pos), _ptr(src),
+                                       _ptr(x_perm), _ptr(x_perm_mx_scales), _ptr(ws), ws.numel(),
+                                       _stream(stream)), "moe_permute_mx")
+
+    def grouped_ffn_mx(self, x_perm, x_perm_mx_scales, offsets, y_perm, ws, stream=None):
+        _check(self.lib.moe_grouped_ffn_mx(self.handle, _ptr(x_perm), _ptr(x_perm_mx_scales),
+                                           _ptr(offsets), _ptr(y_perm), _ptr(ws), ws.numel(),
+                                           _stream(stream)), "moe_grouped_ffn_mx")
 
     def forward_routed_dynamic(self, x_bf16, ids, gates, y, ws, stream=None):
         _check(self.lib.moe_forward_routed_dynamic(self.handle, _ptr(x_bf16), _ptr(ids),

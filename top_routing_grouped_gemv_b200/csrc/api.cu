@@ -30,6 +30,7 @@ struct Layout {
          y_perm = 0, tok_scale = 0, simt_part = 0;
   size_t fwd_end = 0, x_stage = 0, y_stage = 0, total = 0, x_stage_bytes = 0, y_stage_bytes = 0;
   size_t permute_end = 0, router_w3 = 0, router_end = 0;
+  size_t sfa = 0, sfa_end = 0;  // MX plans: activation scale atoms of the permuted rows
 };
 
 }  // namespace
@@ -53,6 +54,7 @@ struct moe_plan_s {
   cudaEvent_t sev[2];     // fork / join of that stream
   cudaEvent_t hev[kHostEvents];
   unsigned long long host_calls;  // host-buffer calls so far (selects the staging slot)
+  uint8_t* sfb;  // MX plans: the weight scales in the tensor-core layout (owned)
 };
 
 namespace {
@@ -109,6 +111,9 @@ void layout(moe_plan p) {
   L.offsets = off; off = align_up(off + static_cast<size_t>(d.E + 1) * 4);
   L.x_perm = off; off = align_up(off + static_cast<size_t>(R) * d.d * p->ex);
   L.y_perm = off; off = align_up(off + static_cast<size_t>(R) * p->dout * p->ey);
+  L.sfa = off;
+  if (d.quant == MOE_QUANT_MX) off = align_up(off + mx_act_sf_bytes(R, d.E, d.d));
+  L.sfa_end = off;
   L.fwd_end = off;
   // two staging slots for x and y: consecutive host-buffer calls alternate
   const size_t xbytes = align_up(static_cast<size_t>(d.N) * d.d * p->ex);
@@ -204,6 +209,7 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
                    const float* x_rows, const int32_t* row_index, void* y_perm, void* ws,
                    cudaStream_t s, const int32_t* out_rows = nullptr) {
   const moe_layer_desc& d = p->desc;
+  if (d.quant == MOE_QUANT_MX) return MOE_ERR_UNSUPPORTED;  // the _mx calls carry the scales
   const int R = n * d.K;
   int* status = at<int>(ws, p->L.status);
   void* h = at<void>(ws, p->L.h);
@@ -292,6 +298,35 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
   return cuda_status(launch_gemm_tc(b, d.dtype, kEpiStore, R, pair, s));
 }
 
+// MX grouped matmul: the activation scales of the permuted rows are already
+// in ws at L.sfa (tensor-core layout); out_rows as run_ffn.
+moe_status run_ffn_mx(moe_plan p, int n, const void* x_perm, const int32_t* offsets, void* y_perm,
+                      void* ws, cudaStream_t s, const int32_t* out_rows = nullptr) {
+  const moe_layer_desc& d = p->desc;
+  const int R = n * d.K;
+  TcGemmArgs a;
+  memset(&a, 0, sizeof(a));
+  if (!encode_kmajor_map(&a.tmA, x_perm, 1, R > 0 ? R : 1, d.d, kTcBlockM)) return MOE_ERR_CUDA;
+  a.tmB0 = p->tmW1;
+  a.tmB1 = a.tmB0;
+  a.offsets = offsets;
+  a.groups = d.E;
+  a.m_total = R;
+  a.kdim = d.d;
+  a.n_out = d.F;
+  a.n_tiles = (d.F + kTcBlockN - 1) / kTcBlockN;
+  a.out = y_perm;
+  a.out_rows = out_rows;
+  a.ldo = d.F;
+  a.scale = 1.f;
+  a.status = at<int>(ws, p->L.status);
+  a.sfa = at<uint8_t>(ws, p->L.sfa);
+  a.sfb = p->sfb;
+  mark(p, s, "gmm_mx_tc");
+  p->launches += 1;
+  return cuda_status(launch_gemm_tc(a, kGemmMxE4M3, kEpiStore, R, false, s));
+}
+
 moe_status run_combine(moe_plan p, int n, const void* y_perm, const int32_t* pos,
                        const float* gates, void* y, void* ws, cudaStream_t s) {
   const moe_layer_desc& d = p->desc;
@@ -336,18 +371,23 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
     return MOE_ERR_INVALID_ARG;
   if (static_cast<long long>(d.N) * d.K >= (1LL << 31)) return MOE_ERR_INVALID_ARG;
   if (d.dtype < MOE_F32 || d.dtype > MOE_E4M3 || d.act < MOE_ACT_NONE || d.act > MOE_ACT_SWIGLU ||
-      d.quant < MOE_QUANT_NONE || d.quant > MOE_QUANT_PER_CHANNEL)
+      d.quant < MOE_QUANT_NONE || d.quant > MOE_QUANT_MX)
     return MOE_ERR_INVALID_ARG;
-  if (d.quant < MOE_QUANT_NONE || d.quant > MOE_QUANT_PER_CHANNEL) return MOE_ERR_INVALID_ARG;
+  // modes 3 (per-token) and 7 (dynamic) are per-call; 4 and 5 are not built
+  if (d.quant == 3 || d.quant == 4 || d.quant == 5) return MOE_ERR_UNSUPPORTED;
   if ((d.quant != MOE_QUANT_NONE) != (d.dtype == MOE_E4M3)) return MOE_ERR_UNSUPPORTED;
   if ((d.quant == MOE_QUANT_PER_CHANNEL) != (w->w_channel_scales != nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (d.quant != MOE_QUANT_MX && w->w_mx_scales) return MOE_ERR_INVALID_ARG;
+  if (d.quant == MOE_QUANT_MX && (d.d % kMxBlock || (w->w1 && !w->w_mx_scales)))
     return MOE_ERR_INVALID_ARG;
   if (d.dtype == MOE_E4M3 && d.act != MOE_ACT_NONE) return MOE_ERR_UNSUPPORTED;
   if (d.dtype == MOE_BF16 && d.act == MOE_ACT_RELU) return MOE_ERR_UNSUPPORTED;
   // a routing-only plan (no expert weights: router, permute and combine of
   // an expert-parallel layer whose experts live on other GPUs) takes none of
   // w1, w3, w2
-  const bool routing_only = !w->w1 && !w->w3 && !w->w2 && d.quant != MOE_QUANT_PER_CHANNEL;
+  const bool routing_only = !w->w1 && !w->w3 && !w->w2 && d.quant != MOE_QUANT_PER_CHANNEL &&
+                            !w->w_mx_scales;
   if (!routing_only && (!w->w1 || (d.act == MOE_ACT_SWIGLU) != (w->w3 != nullptr) ||
                         (d.act != MOE_ACT_NONE) != (w->w2 != nullptr)))
     return MOE_ERR_INVALID_ARG;
@@ -393,6 +433,21 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
       return MOE_ERR_CUDA;
     }
   }
+  if (d.quant == MOE_QUANT_MX && !routing_only) {
+    // the weight scales, once, in the layout the block-scaled GEMM reads
+    cudaStream_t cs = nullptr;
+    const size_t bytes = mx_weight_sf_bytes(d.E, d.F, d.d);
+    bool ok = cudaMalloc(reinterpret_cast<void**>(&p->sfb), bytes) == cudaSuccess;
+    ok = ok && cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) == cudaSuccess;
+    ok = ok && launch_mx_weight_sf(w->w_mx_scales, d.E, d.F, d.d, p->sfb, cs) == cudaSuccess;
+    ok = ok && cudaStreamSynchronize(cs) == cudaSuccess;
+    if (cs) cudaStreamDestroy(cs);
+    if (!ok) {
+      if (p->sfb) cudaFree(p->sfb);
+      delete p;
+      return MOE_ERR_CUDA;
+    }
+  }
   for (int i = 0; i < kMaxEvents; ++i) p->ev[i] = nullptr;
   layout(p);
   *out = p;
@@ -410,6 +465,7 @@ moe_status moe_plan_destroy(moe_plan p) {
   for (int i = 0; i < 2; ++i)
     if (p->sev[i]) cudaEventDestroy(p->sev[i]);
   if (p->side) cudaStreamDestroy(p->side);
+  if (p->sfb) cudaFree(p->sfb);
   delete p;
   return MOE_OK;
 }
@@ -561,6 +617,84 @@ moe_status moe_forward_routed(moe_plan p, const void* x, const int32_t* ids, con
                  x_token_scales, src, scatter ? y : at<void>(ws, L.y_perm), ws, stream, slot);
   if (st == MOE_OK && !scatter)
     st = run_combine(p, n, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_permute_mx(moe_plan p, const void* x, const uint8_t* x_mx_scales,
+                          const int32_t* ids, int32_t* counts, int32_t* offsets, int32_t* pos,
+                          int32_t* src, void* x_perm, uint8_t* x_perm_mx_scales, void* ws,
+                          size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !x || !x_mx_scales || !ids || !counts || !offsets || !pos || !src || !x_perm ||
+      !x_perm_mx_scales)
+    return MOE_ERR_INVALID_ARG;
+  if (p->desc.quant != MOE_QUANT_MX) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.permute_end);
+  if (st != MOE_OK) return st;
+  const moe_layer_desc& d = p->desc;
+  begin(p);
+  st = run_permute(p, d.N, x, ids, counts, offsets, pos, src, x_perm, ws, stream);
+  if (st == MOE_OK) {
+    mark(p, stream, "mx_sf_gather");
+    p->launches += 1;
+    st = cuda_status(launch_mx_sf_gather(x_mx_scales, src, offsets, d.E, d.N * d.K,
+                                         d.d / kMxBlock, x_perm_mx_scales, stream));
+  }
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_grouped_ffn_mx(moe_plan p, const void* x_perm, const uint8_t* x_perm_mx_scales,
+                              const int32_t* offsets, void* y_perm, void* ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+  if (!p || !x_perm || !x_perm_mx_scales || !offsets || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (p->desc.quant != MOE_QUANT_MX) return MOE_ERR_UNSUPPORTED;
+  if (!p->w.w1) return MOE_ERR_UNSUPPORTED;  // routing-only plan
+  if (!aligned16(x_perm) || !aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.sfa_end);
+  if (st != MOE_OK) return st;
+  const moe_layer_desc& d = p->desc;
+  const int R = d.N * d.K;
+  begin(p);
+  mark(p, stream, "mx_act_sf");
+  p->launches += 1;
+  st = cuda_status(launch_mx_act_sf(x_perm_mx_scales, nullptr, offsets, d.E, R, d.d,
+                                    at<uint8_t>(ws, p->L.sfa), stream));
+  if (st == MOE_OK) st = run_ffn_mx(p, d.N, x_perm, offsets, y_perm, ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_forward_routed_mx(moe_plan p, const void* x, const uint8_t* x_mx_scales,
+                                 const int32_t* ids, const float* gates, void* y, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !x || !x_mx_scales || !ids || !y) return MOE_ERR_INVALID_ARG;
+  if (p->desc.quant != MOE_QUANT_MX) return MOE_ERR_UNSUPPORTED;
+  if (!p->w.w1) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.fwd_end);
+  if (st != MOE_OK) return st;
+  const moe_layer_desc& d = p->desc;
+  const Layout& L = p->L;
+  begin(p);
+  int32_t* src = at<int32_t>(ws, L.src);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* slot = gates ? nullptr : at<int32_t>(ws, L.slot);  // unpermute by the GEMM's stores
+  st = run_permute(p, d.N, x, ids, at<int32_t>(ws, L.counts), offsets, at<int32_t>(ws, L.pos), src,
+                   at<void>(ws, L.x_perm), ws, stream, slot);
+  if (st == MOE_OK) {
+    // each permuted row's scales come from its source token's row
+    mark(p, stream, "mx_act_sf");
+    p->launches += 1;
+    st = cuda_status(launch_mx_act_sf(x_mx_scales, src, offsets, d.E, d.N * d.K, d.d,
+                                      at<uint8_t>(ws, L.sfa), stream));
+  }
+  if (st == MOE_OK)
+    st = run_ffn_mx(p, d.N, at<void>(ws, L.x_perm), offsets, gates ? at<void>(ws, L.y_perm) : y, ws,
+                    stream, slot);
+  if (st == MOE_OK && gates)
+    st = run_combine(p, d.N, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
   end(p, stream);
   return st;
 }

@@ -32,6 +32,16 @@
 // Optional row scatter: result row r is stored at row out_rows[r] (the pure
 // unpermute of the single-matrix layer done by the stores).
 //
+// MX variant (Ascend quant mode 6, read as OCP MXFP8: e4m3 operands, one
+// E8M0 scale per 32 elements of K for every row of A and of W): each stage
+// also brings the stage's scale atoms (512 bytes per 128 rows) by untiled
+// bulk copies; the MMA thread copies them into TMEM (tcgen05.cp, four scale
+// columns for A, eight for the 256 weight rows) ahead of the stage's four
+// block-scaled MMAs (tcgen05.mma kind::mxf8f6f4.block_scale, scale byte k
+// for the k-th MMA).  The scale columns take the place of the second
+// accumulator, so the MX kernel has one accumulator and its epilogue does
+// not overlap the next tile's MMAs.
+//
 // Every mbarrier wait is bounded (1 s): on expiry the CTA records
 // MOE_ERR_DEVICE_TIMEOUT, the other roles leave their loops, in-flight
 // copies and MMAs are drained (bounded) and TMEM is freed before exit.
@@ -57,11 +67,12 @@ constexpr int kMaxGroups = 256;
 // Per-mode geometry.  Single CTA: B tile 256 rows, 4 stages of 48 KB.  CTA
 // pair (tcgen05 cta_group::2): each CTA holds its 128 A rows and half of the
 // 256 B rows, 6 stages of 32 KB.
-template <bool kPair>
+template <bool kPair, bool kMx = false>
 struct Geo {
   static constexpr int B_ROWS = kPair ? BN / 2 : BN;
   static constexpr int B_BYTES = B_ROWS * ROWB;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SF_BYTES = kMx ? 3 * kMxAtomBytes : 0;  // A atom + two B atoms
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES;
   static constexpr int STAGES = kPair ? 6 : 4;
   static constexpr int TILE_M = kPair ? 2 * BM : BM;
   static constexpr int kBarFull = 0, kBarEmpty = STAGES, kBarTFull = 2 * STAGES,
@@ -73,11 +84,12 @@ struct Geo {
 
 struct TileCoord {
   int g, m_row0, n_tile;
+  int m_tile;  // row tile counted over all groups' (padded) row tiles
 };
 
 template <int TILE_M>
 __device__ __forceinline__ TileCoord decode_tile(int T, const int* s_pref, const int* s_off,
-                                                 int G) {
+                                                 int G, int n_tiles) {
   int lo = 0, hi = G - 1;
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
@@ -89,6 +101,7 @@ __device__ __forceinline__ TileCoord decode_tile(int T, const int* s_pref, const
   const int mt = (s_off[lo + 1] - s_off[lo] + TILE_M - 1) / TILE_M;
   c.n_tile = local / mt;
   c.m_row0 = s_off[lo] + (local - c.n_tile * mt) * TILE_M;
+  c.m_tile = s_pref[lo] / n_tiles + (local - c.n_tile * mt);
   return c;
 }
 
@@ -101,21 +114,32 @@ constexpr uint32_t make_idesc_mode() {
          (static_cast<uint32_t>((kPair ? 2 * BM : BM) >> 4) << 24);
 }
 
+// Block-scaled (MX) instruction descriptor: e4m3 A and B (format 0), E8M0
+// scales (bit 23), N >> 3 at [17,23), M >> 4 at [24,29); the scale byte of
+// B goes to [4,6) and of A to [29,31) per MMA (mx_sf_ids).
+constexpr uint32_t make_idesc_mx() {
+  return (1u << 23) | (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+}
+__device__ __forceinline__ uint32_t mx_sf_ids(uint32_t k) { return (k << 29) | (k << 4); }
+
 // kPair: a cluster of 2 CTAs computes 256-row tiles with tcgen05 cta_group::2;
 // CTA rank r holds rows [128r, 128r+128) of the tile and B rows [128r, 128r+128)
 // of the 256-row weight tile; the leader (rank 0) issues the MMAs.
-template <bool kFp8, int kEpi, bool kPair>
+template <bool kFp8, int kEpi, bool kPair, bool kMx>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ TcGemmArgs args) {
   griddep_trigger();  // let the next kernel of the stream start launching
   griddep_wait();     // inputs written by the previous kernel are visible
 
-  using Gm = Geo<kPair>;
+  static_assert(!kMx || (kFp8 && !kPair && kEpi == kEpiStore), "MX: e4m3, single CTA, store");
+  using Gm = Geo<kPair, kMx>;
   constexpr int STAGES = Gm::STAGES;
+  constexpr int kAcc = kMx ? 1 : 2;  // accumulators in TMEM
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + STAGES * A_BYTES;
+  const uint32_t sSF = sB + STAGES * Gm::B_BYTES;  // MX scale atoms (kMx only)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Gm::STAGE_BYTES);
   const uint32_t bar0 = smem_u32(bars);
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
@@ -215,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       uint32_t issued = 0, issued_ph = 0;  // per-stage bits: loaded at least once / its parity
       const CUtensorMap* mapB = (kEpi == kEpiSwiglu && kPair && rank == 1) ? &args.tmB1 : &args.tmB0;
       for (int T = unit; T < total && !aborted; T += nunits) {
-        const TileCoord c = decode_tile<Gm::TILE_M>(T, s_pref, s_off, G);
+        const TileCoord c = decode_tile<Gm::TILE_M>(T, s_pref, s_off, G, args.n_tiles);
         const int arow = c.m_row0 + static_cast<int>(rank) * BM;
         int brow;
         if constexpr (kEpi == kEpiSwiglu)
@@ -240,6 +264,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             } else {
               tma_load_2d(sB + s * Gm::B_BYTES, &args.tmB0, kx, brow, bar(Gm::kBarFull + s));
             }
+            if constexpr (kMx) {
+              const uint32_t sf = sSF + s * Gm::SF_BYTES;
+              bulk_load(sf, args.sfa + (static_cast<size_t>(c.m_tile) * num_kb + kb) * kMxAtomBytes,
+                        kMxAtomBytes, bar(Gm::kBarFull + s));
+              bulk_load(sf + kMxAtomBytes,
+                        args.sfb + ((static_cast<size_t>(c.g) * args.n_tiles + c.n_tile) * num_kb + kb) *
+                                       (2 * kMxAtomBytes),
+                        2 * kMxAtomBytes, bar(Gm::kBarFull + s));
+            }
           }
           issued |= 1u << s;
           issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
@@ -258,14 +291,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   } else if (warp == 1) {
     // ---------------- MMA issuer (the pair leader issues for both CTAs) ----------------
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = make_idesc_mode<kFp8, kPair>();
+      constexpr uint32_t idesc = kMx ? make_idesc_mx() : make_idesc_mode<kFp8, kPair>();
+      // MX scale columns (after the single accumulator): A at BN, B at BN + 4
+      const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(BN);
+      const uint32_t sfb_t = sfa_t + 4u;
       int s = 0;
       uint32_t ph = 0;
       bool aborted = false;
       int i = 0;
       for (int T = unit; T < total; T += nunits, ++i) {
-        const int acc = i & 1;
-        const uint32_t aph = (i >> 1) & 1;
+        const int acc = i % kAcc;
+        const uint32_t aph = (i / kAcc) & 1;
         if (!mbar_wait(bar(Gm::kBarTEmpty + acc), aph ^ 1u, abort_flag)) { aborted = true; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -273,10 +309,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           if (!mbar_wait(bar(Gm::kBarFull + s), ph, abort_flag)) { aborted = true; break; }
           tc_fence_after();
           const uint32_t a0 = sA + s * A_BYTES, b0 = sB + s * Gm::B_BYTES;
+          if constexpr (kMx) {
+            // the stage's scales into TMEM; tcgen05 operations of this thread
+            // run in issue order, so the MMAs below read them, and the next
+            // stage's copies wait for those MMAs
+            const uint32_t sf = sSF + s * Gm::SF_BYTES;
+            tc_cp_32x128b_x4(sfa_t, rows16_desc(sf));
+            tc_cp_32x128b_x4(sfb_t, rows16_desc(sf + kMxAtomBytes));
+            tc_cp_32x128b_x4(sfb_t + 4u, rows16_desc(sf + 2 * kMxAtomBytes));
+          }
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
-            if constexpr (kPair)
+            if constexpr (kMx)
+              tc_mma_mx(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k),
+                        idesc | mx_sf_ids(k), sfa_t | (static_cast<uint32_t>(k) << 30),
+                        sfb_t | (static_cast<uint32_t>(k) << 30), accum);
+            else if constexpr (kPair)
               tc_mma_pair<kFp8>(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, accum);
             else
               tc_mma<kFp8>(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, accum);
@@ -303,8 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     int i = 0;
     for (int T = unit; T < total; T += nunits, ++i) {
-      const int acc = i & 1;
-      const uint32_t aph = (i >> 1) & 1;
+      const int acc = i % kAcc;
+      const uint32_t aph = (i / kAcc) & 1;
       // every lane polls; lane 0's answer is taken by all (and converges the warp
       // before the .sync.aligned TMEM loads)
       const bool ok = __shfl_sync(0xffffffffu, mbar_wait(bar(Gm::kBarTFull + acc), aph, abort_flag), 0);
@@ -313,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         break;
       }
       tc_fence_after();
-      const TileCoord c = decode_tile<Gm::TILE_M>(T, s_pref, s_off, G);
+      const TileCoord c = decode_tile<Gm::TILE_M>(T, s_pref, s_off, G, args.n_tiles);
       // lane quadrant q holds rows 32q.. of this CTA's 128 rows of the tile
       const int row = static_cast<int>(rank) * BM + q * 32 + lane;
       // output columns of the tile
@@ -468,10 +517,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <bool kFp8, int kEpi, bool kPair>
+template <bool kFp8, int kEpi, bool kPair, bool kMx = false>
 cudaError_t launch_t(const TcGemmArgs& args, long long max_units, cudaStream_t stream) {
-  using Gm = Geo<kPair>;
-  auto kern = gemm_tc_kernel<kFp8, kEpi, kPair>;
+  using Gm = Geo<kPair, kMx>;
+  auto kern = gemm_tc_kernel<kFp8, kEpi, kPair, kMx>;
   static int configured[64] = {0};
   static int max_clusters[64] = {0};
   int dev = 0;
@@ -537,6 +586,10 @@ cudaError_t launch_gemm_tc(const TcGemmArgs& args, int dtype, int epilogue, int 
   const long long max_units =
       (static_cast<long long>(rows_upper) / tile_m + args.groups) * args.n_tiles;
   if (max_units <= 0) return cudaSuccess;
+  if (dtype == kGemmMxE4M3) {
+    if (pair || epilogue != kEpiStore || !args.sfa || !args.sfb) return cudaErrorInvalidValue;
+    return launch_t<true, kEpiStore, false, true>(args, max_units, stream);
+  }
   const bool fp8 = dtype == kE4M3;
   const bool sw = epilogue == kEpiSwiglu;
   if (epilogue == kEpiRouter) {

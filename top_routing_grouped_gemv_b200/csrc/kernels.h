@@ -132,6 +132,12 @@ struct TcGemmArgs {
   // Row scatter (unpermute fused into the store): when set, row r of the
   // result is stored at row out_rows[r] of out.
   const int32_t* out_rows;
+  // MX block scales (GEMM dtype kGemmMxE4M3), in the tensor-core scale
+  // layout below: sfa per 128-row tile of A counted over the groups' padded
+  // tiles (group g's tiles follow those of groups < g, each group starting
+  // a new tile), sfb per (group, 256-row weight tile).
+  const uint8_t* sfa;
+  const uint8_t* sfb;
 };
 
 // Host: encode a 2-D K-major tile map over a (rows, kdim) row-major matrix of
@@ -143,10 +149,50 @@ bool encode_kmajor_map(CUtensorMap* map, const void* base, int elem_bytes, long 
 // number of A rows (to size the grid).  pair: 256-row tiles on CTA pairs
 // (tcgen05 cta_group::2); the B maps then have 128-row boxes for the store
 // epilogue (each CTA loads half of the 256 weight rows).
+// dtype kGemmMxE4M3: e4m3 operands with MX block scales (args.sfa, args.sfb),
+// single CTA, store epilogue only.
 cudaError_t launch_gemm_tc(const TcGemmArgs& args, int dtype, int epilogue, int rows_upper,
                            bool pair, cudaStream_t stream);
 constexpr int kTcBlockM = 128;
 constexpr int kTcBlockN = 256;  // accumulator columns; SwiGLU: 128 gate + 128 up
+constexpr int kGemmMxE4M3 = 3;
+
+// ---- MX (OCP MXFP8) block scales in the tensor-core layout ----------------
+// One E8M0 byte scales 32 consecutive elements of K.  The GEMM consumes them
+// per 128-element K stage as 512-byte atoms of 128 rows x 4 scales: the
+// scale j (0..3) of row i (0..127) sits at byte (i % 32) * 16 + (i / 32) * 4
+// + j, the order in which tcgen05.cp 32x128b.warpx4 fills the scale columns
+// of the block-scaled MMA.  Scales past the end of K or of the rows are 127
+// (1.0; their operands are zero or never stored).
+//   weights: atom ((g * n_tiles + nt) * num_kb + kb) * 2 + h covers weight
+//            rows nt * 256 + h * 128 + i of group g, n_tiles = ceil(n_out / 256)
+//   activations: atom (pt * num_kb + kb) covers padded row 128 * pt + i
+// with num_kb = ceil(kdim / 128).
+constexpr int kMxBlock = 32;
+constexpr int kMxAtomBytes = 512;
+__host__ __device__ inline int mx_num_kb(int kdim) { return (kdim + 127) / 128; }
+inline size_t mx_weight_sf_bytes(int groups, int n_out, int kdim) {
+  return static_cast<size_t>(groups) * ((n_out + kTcBlockN - 1) / kTcBlockN) * mx_num_kb(kdim) * 2 *
+         kMxAtomBytes;
+}
+// upper bound of the padded activation tiles of `rows` rows over `groups`
+inline size_t mx_act_sf_bytes(long long rows, int groups, int kdim) {
+  return static_cast<size_t>(rows / kTcBlockM + groups + 1) * mx_num_kb(kdim) * kMxAtomBytes;
+}
+// w_sf (groups, n_out, kdim / 32) row-major -> the weight atoms.
+cudaError_t launch_mx_weight_sf(const uint8_t* w_sf, int groups, int n_out, int kdim, uint8_t* out,
+                                cudaStream_t stream);
+// Activation atoms of the permuted rows r < offsets[groups] (at most
+// rows_upper): the scales of row r are row src_rows[r] (or r when NULL) of
+// x_sf (*, kdim / 32) row-major.
+cudaError_t launch_mx_act_sf(const uint8_t* x_sf, const int32_t* src_rows, const int32_t* offsets,
+                             int groups, int rows_upper, int kdim, uint8_t* out,
+                             cudaStream_t stream);
+// Row gather of scales: out row r = x_sf row src_rows[r], for r <
+// offsets[groups] (at most rows_upper); nsf bytes per row.
+cudaError_t launch_mx_sf_gather(const uint8_t* x_sf, const int32_t* src_rows,
+                                const int32_t* offsets, int groups, int rows_upper, int nsf,
+                                uint8_t* out, cudaStream_t stream);
 
 int device_sm_count();
 

@@ -73,6 +73,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+// Untiled bulk copy of `bytes` from global into this CTA's shared memory,
+// completing on `bar` (no multicast).  Both addresses 16-byte aligned,
+// bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -106,6 +117,35 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
         : "memory");
   }
 }
+// Block-scaled MMA (MXFP8: e4m3 operands, one E8M0 scale per 32 elements of
+// K per row of A and per row of B).  The scale operands are TMEM addresses
+// whose bits 30-31 select the byte of each 32-bit scale cell (the k-th MMA
+// of a 128-element stage uses byte k).
+__device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+// Shared memory -> TMEM copy of 32 rows x 128 bits, written to lanes
+// [0,32) of every lane quadrant (the scale-factor layout of the block-scaled
+// MMA: lane i of each quadrant receives row i, four 32-bit columns).
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+// Shared-memory descriptor of 32 contiguous rows of 16 bytes, no swizzle:
+// 8-row core matrices of 128 bytes, 128 bytes apart (stride offset); the
+// leading offset (16 B) is unused with a single 16-byte column.
+__device__ __forceinline__ uint64_t rows16_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (1ull << 16) |
+         (static_cast<uint64_t>(128 >> 4) << 32) | (1ull << 46);
+}
+
 // 32 lanes x 32 consecutive fp32 columns: thread i of the warp gets row
 // (quadrant*32 + i), columns [col, col+32).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
