@@ -184,6 +184,21 @@ def gemm_flops(cfg, rows: int):
     return 2.0 * rows * cfg.d * cfg.F, 0.0
 
 
+def oracle_tokens(inp, tok):
+    """The oracle's layer on tokens `tok`: the whole forward, or for the MX
+    layer its K rows per token through the MX experts (pure unpermute)."""
+    import numpy as np
+    import oracle
+    cfg = inp.cfg
+    if cfg.quant == "mx":
+        rows = np.repeat(np.asarray(tok), cfg.K)
+        row_e = inp.ids.numpy()[tok].reshape(-1).astype(np.int32)
+        return oracle.expert_rows_mx(row_e, inp.x.numpy()[rows], inp.x_sf.numpy()[rows], inp.w1,
+                                     inp.w_sf)
+    gm = 0 if cfg.routing == "given" else 1   # given routing: the pure unpermute
+    return oracle.forward_tokens(inp, tok, gates_mode=gm)
+
+
 def oracle_sample_tokens(cfg, inp, target_s: float, max_tokens: int | None = None):
     """Time the oracle's whole-layer forward on a token sample sized to take
     about target_s seconds; returns (tokens, seconds, threads)."""
@@ -191,16 +206,15 @@ def oracle_sample_tokens(cfg, inp, target_s: float, max_tokens: int | None = Non
     import oracle
     threads = oracle.num_threads()
     n = max(1, threads)
-    gm = 0 if cfg.routing == "given" else 1   # given routing: the pure unpermute
     t0 = time.perf_counter()
-    oracle.forward_tokens(inp, np.arange(n), gates_mode=gm)
+    oracle_tokens(inp, np.arange(n))
     dt = time.perf_counter() - t0
     n2 = int(min(max_tokens or cfg.N, max(n, n * target_s / max(dt, 1e-6))))
     n2 = max(threads, n2 // threads * threads) if n2 >= threads else n2
     rng = np.random.default_rng(17)
     tok = np.sort(rng.choice(cfg.N, size=min(n2, cfg.N), replace=False))
     t0 = time.perf_counter()
-    oracle.forward_tokens(inp, tok, gates_mode=gm)
+    oracle_tokens(inp, tok)
     return len(tok), time.perf_counter() - t0, threads
 
 
@@ -216,12 +230,11 @@ def run_reference(args, rank: int):
     threads = oracle.num_threads()
     per = max(1, threads)
     rng = np.random.default_rng(23)
-    gm = 0 if cfg.routing == "given" else 1
     for _ in range(args.warmup):
-        oracle.forward_tokens(inp, rng.choice(cfg.N, size=per, replace=False), gates_mode=gm)
+        oracle_tokens(inp, rng.choice(cfg.N, size=per, replace=False))
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.forward_tokens(inp, rng.choice(cfg.N, size=per, replace=False), gates_mode=gm)
+        oracle_tokens(inp, rng.choice(cfg.N, size=per, replace=False))
     dt = time.perf_counter() - t0
     value = per * args.steps / dt
     line = {
@@ -269,7 +282,8 @@ def main():
     cfg = synth.CONFIGS[args.workload]
     inp = synth.make_inputs(cfg)
     w = {"w1": inp.w1.cuda(), "w_scale": inp.w_scale}
-    for k, t in (("w3", inp.w3), ("w2", inp.w2), ("w_r", inp.w_r), ("bias", inp.bias)):
+    for k, t in (("w3", inp.w3), ("w2", inp.w2), ("w_r", inp.w_r), ("bias", inp.bias),
+                 ("w_mx_scales", inp.w_sf)):
         if t is not None:
             w[k] = t.cuda()
     plan = moe.Plan(cfg.N, cfg.d, cfg.E, cfg.K, cfg.F, cfg.dtype, cfg.act, w)
@@ -279,7 +293,19 @@ def main():
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     given = cfg.routing == "given"
-    if given:
+    mx = cfg.quant == "mx"
+    shared = cfg.shared is not None
+    ysh = xsf = None
+    if given and mx:
+        # MX grouped-matmul layer: the caller's routing and block scales, the
+        # pure unpermute done by the GEMM's stores
+        ids = inp.ids.cuda()
+        xsf = inp.x_sf.cuda()
+        y = torch.empty(cfg.N * cfg.K, cfg.d_out, dtype=ydt, device="cuda")
+
+        def step():
+            plan.forward_routed_mx(x, xsf, ids, None, y, ws)
+    elif given:
         # fp8 grouped-matmul layer: the caller's routing, the pure unpermute
         # done by the GEMM's stores, and the shared expert on a forked stream
         ids = inp.ids.cuda()
@@ -303,7 +329,7 @@ def main():
         step()
     torch.cuda.synchronize()
     assert plan.read_device_status(ws) == 0, "device status after warm-up"
-    launches_per_step = plan.last_launch_count() + (1 if given else 0)  # + the shared matmul
+    launches_per_step = plan.last_launch_count() + (1 if shared else 0)  # + the shared matmul
 
     # timed region: K steps back to back (the host runs ahead of the GPU),
     # CUDA events around every step on the launching stream
@@ -345,21 +371,23 @@ def main():
     # first H2D to after the last D2H
     e2e = None
     if not args.no_e2e and given:
-        # fp8 layer: each step copies its x and routing in from pinned host
-        # memory, runs the routed layer and the shared expert, and copies both
-        # results back (no host-buffer entry point for this layer: the copies
-        # are queued on the compute stream)
-        xh = inp.x.clone().pin_memory()
-        idh = inp.ids.clone().pin_memory()
-        yh = torch.empty(tuple(y.shape), dtype=y.dtype).pin_memory()
-        yshh = torch.empty(tuple(ysh.shape), dtype=ysh.dtype).pin_memory()
+        # fp8 layers: each step copies its x (and MX scales) and routing in
+        # from pinned host memory, runs the routed layer (and the shared
+        # expert), and copies the results back (no host-buffer entry point
+        # for these layers: the copies are queued on the compute stream)
+        ins = [(x, inp.x.clone().pin_memory()), (ids, inp.ids.clone().pin_memory())]
+        if mx:
+            ins.append((xsf, inp.x_sf.clone().pin_memory()))
+        outs = [(y, torch.empty(tuple(y.shape), dtype=y.dtype).pin_memory())]
+        if shared:
+            outs.append((ysh, torch.empty(tuple(ysh.shape), dtype=ysh.dtype).pin_memory()))
 
         def e2e_step():
-            x.copy_(xh, non_blocking=True)
-            ids.copy_(idh, non_blocking=True)
+            for dev, host in ins:
+                dev.copy_(host, non_blocking=True)
             step()
-            yh.copy_(y, non_blocking=True)
-            yshh.copy_(ysh, non_blocking=True)
+            for dev, host in outs:
+                host.copy_(dev, non_blocking=True)
 
         for _ in range(min(args.warmup, 3)):
             e2e_step()
@@ -376,10 +404,11 @@ def main():
         e_ms = max_over_ranks(a.elapsed_time(b), dist)
         assert plan.read_device_status(ws) == 0, "device status after the host-buffer loop"
         e2e = {"value": replica_throughput(cfg.N, n_e2e, world, e_ms), "unit": "tokens/s",
-               "h2d_bytes_per_step": xh.numel() * xh.element_size() + idh.numel() * idh.element_size(),
-               "d2h_bytes_per_step": yh.numel() * yh.element_size() + yshh.numel() * yshh.element_size(),
+               "h2d_bytes_per_step": sum(h.numel() * h.element_size() for _, h in ins),
+               "d2h_bytes_per_step": sum(h.numel() * h.element_size() for _, h in outs),
                "steps": n_e2e,
-               "api": "moe_forward_routed_shared with pinned host copies on the same stream"}
+               "api": ("moe_forward_routed_mx" if mx else "moe_forward_routed_shared")
+                      + " with pinned host copies on the same stream"}
     elif not args.no_e2e:
         xh = [inp.x.clone().pin_memory() for _ in range(2)]
         yh = [torch.empty(cfg.N, cfg.d_out, dtype=ydt).pin_memory() for _ in range(2)]
@@ -411,7 +440,8 @@ def main():
     peaks, peak_src = load_peaks()
     R = cfg.N * cfg.K
     f1, f2 = gemm_flops(cfg, R)
-    k1 = "ffn1_swiglu_tc" if cfg.act == "swiglu" else ("gmm_tc" if cfg.act == "none" else "ffn1_simt_f32")
+    k1 = "ffn1_swiglu_tc" if cfg.act == "swiglu" else (
+        ("gmm_mx_tc" if mx else "gmm_tc") if cfg.act == "none" else "ffn1_simt_f32")
     stage_us = {k: 1e3 * statistics.mean(v) for k, v in per_kernel.items()}
     # the sustained (power-capped) peak applies to a kernel timed inside a long
     # loop or while the power cap throttles the clock; the burst one otherwise
@@ -455,8 +485,10 @@ def main():
             "dtype": cfg.dtype, "data": "synthetic",
             "config": {"workload": cfg.name, "N": cfg.N, "d": cfg.d, "E": cfg.E, "K": cfg.K,
                        "F": cfg.F, "act": cfg.act,
-                       "router": "given (top-K of seeded iid logits), shared expert "
-                                 f"{cfg.shared[0]}x{cfg.shared[1]} on a forked stream"
+                       "router": ("given (top-K of seeded iid logits), OCP MXFP8 block scales "
+                                  "(E8M0 per 32 elements)" if mx else
+                                  "given (top-K of seeded iid logits), shared expert "
+                                  f"{cfg.shared[0]}x{cfg.shared[1]} on a forked stream")
                                  if given else "fp32",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "value: flushed (256 MiB write) before every step; e2e: inputs "

@@ -16,6 +16,8 @@ Workloads (the five shapes the layer is measured and checked on):
   + token-major unpermute, plus a shared-expert matmul (8192x7168)@(7168x2048)
 * ``e4m3mx_n8192_h7168_e256_k8_n2048_gmm``  the same grouped matmul with MX block
   scales (OCP MXFP8: one E8M0 scale per 32 consecutive elements along H1)
+* ``e4m3_n2048_h7168_e64_k8_n2048_gmm``, ``e4m3mx_n2048_h7168_e64_k8_n2048_gmm``
+  reduced copies of the two fp8 layers for kernel profiling
 
 Value recipe: x ~ N(0,1); router and expert weights ~ N(0, 1/fan_in)
 (fan_in = d for the router and the first FFN matrices, F for the second);
@@ -111,6 +113,14 @@ FP8_GMM = _reg(MoEConfig("e4m3_n8192_h7168_e256_k8_n2048_gmm", DTYPE_E4M3, 8192,
                          ACT_NONE, index=4, shared=(7168, 2048), routing="given"))
 MX_GMM = _reg(MoEConfig("e4m3mx_n8192_h7168_e256_k8_n2048_gmm", DTYPE_E4M3, 8192, 7168, 256, 8,
                         2048, ACT_NONE, index=5, routing="given", quant="mx"))
+# Reduced copies of the two fp8 layers (a quarter of the tokens, E = 64, the
+# same per-expert shape and ~256 rows per expert): small enough for kernel
+# captures that replay every launch many times, weights (0.94 GB) still far
+# larger than L2.
+FP8_GMM_PROFILE = _reg(MoEConfig("e4m3_n2048_h7168_e64_k8_n2048_gmm", DTYPE_E4M3, 2048, 7168, 64, 8,
+                                 2048, ACT_NONE, index=6, shared=(7168, 2048), routing="given"))
+MX_GMM_PROFILE = _reg(MoEConfig("e4m3mx_n2048_h7168_e64_k8_n2048_gmm", DTYPE_E4M3, 2048, 7168, 64,
+                                8, 2048, ACT_NONE, index=7, routing="given", quant="mx"))
 
 
 # ----------------------------------------------------------------------------

@@ -208,3 +208,51 @@ def test_e4m3_gmm_dynamic_per_token_quant_n8192_h7168_e256_k8_n2048():
                                     x_row_scales=rscale[np.repeat(tok, c.K)].astype(np.float64),
                                     w_scale=inp.w_scale)
     assert rel_err(f64(y[torch.from_numpy(rows_tok).long().cuda()]), ref) <= TOL["e4m3"]
+
+
+def test_e4m3_mx_gmm_unpermute_n8192_h7168_e256_k8_n2048():
+    """The grouped matmul with MX block scales (quant mode 6) at full size:
+    permute and permuted scale rows bit-exact in full, the grouped matmul on
+    sampled rows against the oracle, the fused call (unpermute by the GEMM's
+    stores) equal to the stage composition bit for bit, sampled tokens of the
+    fused result against the oracle."""
+    import top_routing_grouped_gemv_b200 as moe
+    c = synth.MX_GMM
+    inp = synth.make_inputs(c)
+    R = c.N * c.K
+    w = {"w1": inp.w1.cuda(), "w_mx_scales": inp.w_sf.cuda()}
+    plan = moe.Plan(c.N, c.d, c.E, c.K, c.F, "e4m3", "none", w)
+    x, xsf, ids = inp.x.cuda(), inp.x_sf.cuda(), inp.ids.cuda()
+    xs = inp.x_sf.numpy()
+    ws = plan.new_workspace()
+    i32 = dict(dtype=torch.int32, device="cuda")
+    counts, offsets = torch.empty(c.E, **i32), torch.empty(c.E + 1, **i32)
+    pos, src = torch.empty(R, **i32), torch.empty(R, **i32)
+    x_perm = torch.empty(R, c.d, dtype=torch.uint8, device="cuda")
+    sf_perm = torch.empty(R, c.d // 32, dtype=torch.uint8, device="cuda")
+    plan.permute_mx(x, xsf, ids, counts, offsets, pos, src, x_perm, sf_perm, ws)
+    assert plan.read_device_status(ws) == 0
+    rc, ro, rp, rs, rx = oracle.permute(inp.ids.numpy(), c.E, inp.x)
+    assert np.array_equal(offsets.cpu().numpy(), ro) and np.array_equal(pos.cpu().numpy(), rp)
+    assert torch.equal(x_perm.cpu(), torch.from_numpy(rx))
+    assert np.array_equal(sf_perm.cpu().numpy(), xs[rs])
+
+    y_perm = torch.empty(R, c.F, dtype=torch.bfloat16, device="cuda")
+    plan.grouped_ffn_mx(x_perm, sf_perm, offsets, y_perm, ws)
+    assert plan.read_device_status(ws) == 0
+    rows = sample_rows(ro, R, 48, 9)
+    row_e = (np.searchsorted(ro, rows, side="right") - 1).astype(np.int32)
+    ref = oracle.expert_rows_mx(row_e, rx[rows], xs[rs[rows]], inp.w1, inp.w_sf)
+    assert rel_err(f64(y_perm[torch.from_numpy(rows).long().cuda()]), ref) <= 1e-2
+
+    y = torch.empty(R, c.F, dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed_mx(x, xsf, ids, None, y, ws)
+    assert plan.read_device_status(ws) == 0
+    yp = y_perm.cpu().view(torch.int16).numpy()
+    assert np.array_equal(y.cpu().view(torch.int16).numpy(), yp[rp])
+    tok = np.array([0, 1, 4095, c.N - 1])
+    rows_tok = (tok[:, None] * c.K + np.arange(c.K)).reshape(-1)
+    row_e = inp.ids.numpy().reshape(-1)[rows_tok].astype(np.int32)
+    tr = np.repeat(tok, c.K)
+    yref = oracle.expert_rows_mx(row_e, inp.x.numpy()[tr], xs[tr], inp.w1, inp.w_sf)
+    assert rel_err(f64(y[torch.from_numpy(rows_tok).long().cuda()]), yref) <= 1e-2
