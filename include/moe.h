@@ -101,7 +101,7 @@ typedef enum { MOE_ACT_NONE = 0, MOE_ACT_RELU = 1, MOE_ACT_SWIGLU = 2 } moe_act;
  * 32 consecutive values along the reduction dimension (d), each block with
  * one E8M0 scale byte 2^(s - 127) (255 = NaN), for the weights
  * (w_mx_scales) and the activations (the _mx calls' x_mx_scales); the
- * single-matrix layer only.  Group and block modes (4, 5) are not built
+ * single-matrix layer only, d a multiple of 32 and at most 32768.  Group and block modes (4, 5) are not built
  * (MOE_ERR_UNSUPPORTED). */
 typedef enum {
   MOE_QUANT_NONE = 0,

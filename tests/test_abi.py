@@ -62,6 +62,8 @@ def _create(lib, N=64, d=64, E=8, K=2, F=64, dtype=moe.MOE_BF16, act=moe.ACT_SWI
           quant=moe.QUANT_MX), 1),                                         # MX needs its scales
     (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None, d=48,
           quant=moe.QUANT_MX, w_mx=0x5000), 1),                            # d not a multiple of 32
+    (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None, d=32800,
+          quant=moe.QUANT_MX, w_mx=0x5000), 1),                            # d above 32768
     (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None,
           quant=moe.QUANT_PER_TENSOR, w_mx=0x5000), 1),                    # scales without MX
     (dict(dtype=moe.MOE_E4M3, act=moe.ACT_SWIGLU, quant=moe.QUANT_PER_TENSOR), 2),

@@ -379,7 +379,7 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
   if ((d.quant == MOE_QUANT_PER_CHANNEL) != (w->w_channel_scales != nullptr))
     return MOE_ERR_INVALID_ARG;
   if (d.quant != MOE_QUANT_MX && w->w_mx_scales) return MOE_ERR_INVALID_ARG;
-  if (d.quant == MOE_QUANT_MX && (d.d % kMxBlock || (w->w1 && !w->w_mx_scales)))
+  if (d.quant == MOE_QUANT_MX && (d.d % kMxBlock || d.d > kMxMaxKdim || (w->w1 && !w->w_mx_scales)))
     return MOE_ERR_INVALID_ARG;
   if (d.dtype == MOE_E4M3 && d.act != MOE_ACT_NONE) return MOE_ERR_UNSUPPORTED;
   if (d.dtype == MOE_BF16 && d.act == MOE_ACT_RELU) return MOE_ERR_UNSUPPORTED;

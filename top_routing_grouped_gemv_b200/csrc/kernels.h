@@ -169,6 +169,7 @@ constexpr int kGemmMxE4M3 = 3;
 //   activations: atom (pt * num_kb + kb) covers padded row 128 * pt + i
 // with num_kb = ceil(kdim / 128).
 constexpr int kMxBlock = 32;
+constexpr int kMxMaxKdim = 32768;  // MX layers: d <= 32768 (one 128-row tile's scales in 128 KB)
 constexpr int kMxAtomBytes = 512;
 __host__ __device__ inline int mx_num_kb(int kdim) { return (kdim + 127) / 128; }
 inline size_t mx_weight_sf_bytes(int groups, int n_out, int kdim) {

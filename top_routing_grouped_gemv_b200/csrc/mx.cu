@@ -87,34 +87,70 @@ __device__ void tile_prefix(const int32_t* offsets, int G, int* s_off, int* s_tp
   }
 }
 
-// One thread per (permuted row, K stage).
-__global__ void mx_act_sf_kernel(const uint8_t* __restrict__ x_sf, const int32_t* __restrict__ src,
-                                 const int32_t* __restrict__ offsets, int G, int rows_upper,
-                                 int kdim, uint8_t* __restrict__ out) {
+// One block per padded 128-row tile: the scale rows of the tile's permuted
+// rows are gathered into shared memory, then the tile's num_kb atoms (one
+// contiguous region) are written with 16-byte stores.  Rows past the
+// group's end and scales past the end of K get 127.
+constexpr int kActThreads = 256;
+
+__global__ void __launch_bounds__(kActThreads) mx_act_sf_kernel(
+    const uint8_t* __restrict__ x_sf, const int32_t* __restrict__ src,
+    const int32_t* __restrict__ offsets, int G, int kdim, uint8_t* __restrict__ out) {
+  extern __shared__ uint8_t s_rows[];  // (128, row_bytes): the tile's scale rows
   __shared__ int s_off[257], s_tp[257];
   griddep_trigger();
   griddep_wait();
   if (threadIdx.x < 32) tile_prefix(offsets, G, s_off, s_tp);
   __syncthreads();
-  const int rows = min(s_off[G], rows_upper);
+  const int pt = blockIdx.x;
+  if (pt >= s_tp[G]) return;
+  int lo = 0, hi = G - 1;  // the group owning padded tile pt: last g with s_tp[g] <= pt
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_tp[mid] <= pt) lo = mid; else hi = mid - 1;
+  }
+  const int r0 = s_off[lo] + (pt - s_tp[lo]) * kTcBlockM;  // first permuted row of the tile
+  const int nrow = min(kTcBlockM, s_off[lo + 1] - r0);
   const int nsf = kdim / kMxBlock;
   const int num_kb = mx_num_kb(kdim);
-  const long long total = static_cast<long long>(rows) * num_kb;
-  for (long long t = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; t < total;
-       t += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int kb = static_cast<int>(t % num_kb);
-    const int r = static_cast<int>(t / num_kb);
-    int lo = 0, hi = G - 1;  // the group holding row r: last g with s_off[g] <= r
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_off[mid] <= r) lo = mid; else hi = mid - 1;
+  const int row_bytes = num_kb * 4;
+  // gather: row i of the tile <- scale row src[r0 + i] (127 past the end)
+  if (nsf % 16 == 0 && (reinterpret_cast<uintptr_t>(x_sf) & 15) == 0) {
+    // rows of whole, aligned 16-byte chunks (row_bytes == nsf): unrolled vector loads
+    const int vpr = nsf / 16;
+    const uint4 unit = make_uint4(kUnitScales, kUnitScales, kUnitScales, kUnitScales);
+#pragma unroll 8
+    for (int t = threadIdx.x; t < kTcBlockM * vpr; t += kActThreads) {
+      const int i = t / vpr, v = t - i * vpr;
+      uint4 val = unit;
+      if (i < nrow) {
+        const long long sr = src ? src[r0 + i] : r0 + i;
+        val = reinterpret_cast<const uint4*>(x_sf + sr * nsf)[v];
+      }
+      reinterpret_cast<uint4*>(s_rows)[t] = val;
     }
-    const int local = r - s_off[lo];
-    const int pt = s_tp[lo] + local / kTcBlockM;
-    const long long sr = src ? src[r] : r;
-    const uint32_t v = stage_scales(x_sf + sr * nsf, nsf, kb);
-    uint8_t* atom = out + (static_cast<long long>(pt) * num_kb + kb) * kMxAtomBytes;
-    *reinterpret_cast<uint32_t*>(atom + atom_offset(local & (kTcBlockM - 1))) = v;
+  } else {
+#pragma unroll 8
+    for (int t = threadIdx.x; t < kTcBlockM * row_bytes; t += kActThreads) {
+      const int i = t / row_bytes, b = t - i * row_bytes;
+      uint8_t v = 0x7F;
+      if (i < nrow && b < nsf) {
+        const long long sr = src ? src[r0 + i] : r0 + i;
+        v = x_sf[sr * nsf + b];
+      }
+      s_rows[t] = v;
+    }
+  }
+  __syncthreads();
+  // atoms: line m of atom kb = scales 4kb..4kb+3 of rows m, m+32, m+64, m+96
+  uint4* dst = reinterpret_cast<uint4*>(out + static_cast<long long>(pt) * num_kb * kMxAtomBytes);
+  for (int t = threadIdx.x; t < num_kb * 32; t += kActThreads) {
+    const int kb = t >> 5, m = t & 31;
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      w[q] = *reinterpret_cast<const uint32_t*>(s_rows + (m + 32 * q) * row_bytes + 4 * kb);
+    dst[t] = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -154,11 +190,22 @@ cudaError_t launch_mx_weight_sf(const uint8_t* w_sf, int groups, int n_out, int 
 cudaError_t launch_mx_act_sf(const uint8_t* x_sf, const int32_t* src_rows, const int32_t* offsets,
                              int groups, int rows_upper, int kdim, uint8_t* out,
                              cudaStream_t stream) {
-  if (groups < 1 || groups > 256 || kdim < kMxBlock || kdim % kMxBlock) return cudaErrorInvalidValue;
+  if (groups < 1 || groups > 256 || kdim < kMxBlock || kdim % kMxBlock || kdim > kMxMaxKdim)
+    return cudaErrorInvalidValue;
   if (rows_upper <= 0) return cudaSuccess;
-  const long long work = static_cast<long long>(rows_upper) * mx_num_kb(kdim);
-  return launch_pdl(mx_act_sf_kernel, dim3(grid_for(work, 256)), dim3(256), 0, stream, x_sf,
-                    src_rows, offsets, groups, rows_upper, kdim, out);
+  // one block per padded tile; at most rows_upper / 128 + groups tiles exist
+  const int tiles = rows_upper / kTcBlockM + groups;
+  const size_t smem = static_cast<size_t>(kTcBlockM) * mx_num_kb(kdim) * 4;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(mx_act_sf_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kTcBlockM * mx_num_kb(kMxMaxKdim) * 4);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  return launch_pdl(mx_act_sf_kernel, dim3(tiles), dim3(kActThreads), smem, stream, x_sf, src_rows,
+                    offsets, groups, kdim, out);
 }
 
 cudaError_t launch_mx_sf_gather(const uint8_t* x_sf, const int32_t* src_rows,
