@@ -64,6 +64,7 @@ def lib():
         L.orc_matmul.argtypes = [i, i, i, P, P, P]
         L.orc_quantize_rows_dynamic.argtypes = [i, i, P, P, P]
         L.orc_expert_rows_mx.argtypes = [i, P, i, i, P, P, i, P, P, P]
+        L.orc_expert_rows_kscaled.argtypes = [i, P, i, i, i, P, P, d, i, i, P, P, P]
         L.orc_e8m0_to_f64.argtypes = [ctypes.c_uint8]
         L.orc_e8m0_to_f64.restype = d
         L.orc_bf16_to_f64.argtypes = [ctypes.c_uint16]
@@ -279,6 +280,30 @@ def expert_rows_mx(row_expert, x, xs, w, ws):
     _check(lib().orc_expert_rows_mx(len(row_expert), _p(row_expert), E, din, _p(xn), _p(xsn), F,
                                     _p(wn), _p(wsn), _p(y)), "expert_rows_mx")
     return y
+
+
+def expert_rows_kscaled(row_expert, xrows, x_dtype: int, w1, w_dtype: int, w_group_scales,
+                        x_group_scales=None, x_scale: float = 1.0):
+    """Single-matrix experts with fp32 scales per 128-element group of K:
+    w_group_scales (E, F, din/128), x_group_scales (n, din/128) or the scalar
+    x_scale; rows with expert < 0 are left NaN."""
+    row_expert = np.ascontiguousarray(row_expert, np.int32)
+    xr, w1n = _np(xrows), _np(w1)
+    E, F, din = w1n.shape
+    ws = np.ascontiguousarray(w_group_scales, np.float64)
+    xs = None if x_group_scales is None else np.ascontiguousarray(x_group_scales, np.float64)
+    y = np.full((len(row_expert), F), np.nan)
+    _check(lib().orc_expert_rows_kscaled(len(row_expert), _p(row_expert), E, din, x_dtype, _p(xr),
+                                         _p(xs), x_scale, F, w_dtype, _p(w1n), _p(ws), _p(y)),
+           "expert_rows_kscaled")
+    return y
+
+
+def block_to_group_scales(w_block_scales, F: int):
+    """128 x 128 weight-block scales (E, ceil(F/128), G) -> per-channel group
+    scales (E, F, G): channel n takes block n // 128."""
+    wb = np.asarray(w_block_scales, np.float64)
+    return np.ascontiguousarray(np.repeat(wb, 128, axis=1)[:, :F])
 
 
 def matmul(A, B):

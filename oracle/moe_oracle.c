@@ -23,6 +23,9 @@
  *    unpermuteOut = Unpermute(gmmY); shared expert
  *    mmY = (mmX @ mmWeight) * mmXScale * mmWeightScale; quant mode 1 =
  *    per-tensor; constraints: K in [2, 8], deterministic by default.
+ *    Quant modes 4 (pergroup) and 5 (perblock): read as fp32 scales per
+ *    group of 128 elements of K (per output channel, or per 128 x 128 weight
+ *    block, with per-token-per-group activation scales).
  *    Quant mode 6 ("mx"): read as OCP MXFP8, e4m3 elements in blocks of 32
  *    along the reduction dimension, each block with an E8M0 power-of-two scale.
  *  - zyxy.net "SpMM ... MoE inference", MoE structure: y = sum_i g_i(x)*E_i(x);
@@ -410,6 +413,51 @@ int orc_expert_rows_mx(int nrows, const int32_t* row_expert, int E, int din, con
                 for (int k = 0; k < din; ++k)
                     acc += xr[k] * (orc_e4m3_to_f64(w[wrow * din + k]) *
                                     orc_e8m0_to_f64(ws[wrow * nb + k / 32]));
+                y[(int64_t)r * F + n] = acc;
+            }
+        }
+        free(xr);
+    }
+    return ORC_OK;
+}
+
+/* Single-matrix experts with fp32 scales per group of 128 elements of K
+ * (Ascend quant modes 4 "pergroup" and 5 "perblock"; the page names the
+ * modes only, the group of 128 along the reduction dimension is this
+ * layer's reading):
+ *   y[r][n] = sum_g xs[r][g] * ws[e][n][g] * (sum_{k in group g} x[r][k] * W[e][n][k])
+ * groups g = 0 .. din/128 - 1 ascending, k ascending inside a group.
+ * xs (nrows, din/128): the activation scale of each row and group (NULL:
+ * x_scale for all); ws (E, F, din/128): the weight scale of each output
+ * channel and group.  Per-group weights (mode 4) give ws directly; 128 x 128
+ * weight blocks (mode 5) repeat one scale over the 128 channels of a block. */
+int orc_expert_rows_kscaled(int nrows, const int32_t* row_expert, int E, int din, int x_dtype,
+                            const void* xrows, const double* xs, double x_scale, int F,
+                            int w_dtype, const void* w1, const double* ws, double* y) {
+    if (nrows < 0 || !row_expert || !xrows || !w1 || !ws || !y || din <= 0 || F <= 0 ||
+        din % 128 != 0)
+        return ORC_ERR_ARG;
+    for (int r = 0; r < nrows; ++r)
+        if (row_expert[r] >= E) return ORC_ERR_INDEX;
+    const int ng = din / 128;
+#pragma omp parallel
+    {
+        double* xr = (double*)malloc(sizeof(double) * (size_t)din);
+#pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < nrows; ++r) {
+            int e = row_expert[r];
+            if (e < 0) continue;
+            orc_to_f64(xrows, x_dtype, (int64_t)r * din, din, xr);
+            for (int n = 0; n < F; ++n) {
+                int64_t wrow = (int64_t)e * F + n;
+                double acc = 0.0;
+                for (int g = 0; g < ng; ++g) {
+                    double part = 0.0;
+                    for (int k = 128 * g; k < 128 * g + 128; ++k)
+                        part += xr[k] * load_elem(w1, w_dtype, wrow * din + k);
+                    double sx = xs ? xs[(int64_t)r * ng + g] : x_scale;
+                    acc += sx * ws[wrow * ng + g] * part;
+                }
                 y[(int64_t)r * F + n] = acc;
             }
         }

@@ -16,6 +16,8 @@ Workloads (the five shapes the layer is measured and checked on):
   + token-major unpermute, plus a shared-expert matmul (8192x7168)@(7168x2048)
 * ``e4m3mx_n8192_h7168_e256_k8_n2048_gmm``  the same grouped matmul with MX block
   scales (OCP MXFP8: one E8M0 scale per 32 consecutive elements along H1)
+* ``e4m3blk_n8192_h7168_e256_k8_n2048_gmm``  the same grouped matmul with fp32 scales per
+  128 x 128 weight block and per token and 128-element group of the activations
 * ``e4m3_n2048_h7168_e64_k8_n2048_gmm``, ``e4m3mx_n2048_h7168_e64_k8_n2048_gmm``
   reduced copies of the two fp8 layers for kernel profiling
 
@@ -79,7 +81,8 @@ class MoEConfig:
     zipf_bias: float = 0.0          # router bias b_e = zipf_bias * ln(1/(e+1)); 0 = no bias
     shared: tuple | None = None     # (H2, N2) shared-expert matmul, fp8 workload only
     routing: str = "router"         # "router" (logits from x @ W_r) or "given" (drawn ids)
-    quant: str = "tensor"           # fp8 scales: "tensor" (one per tensor) or "mx" (E8M0 per 32)
+    quant: str = "tensor"           # fp8 scales: "tensor" (one per tensor), "mx" (E8M0 per 32),
+                                    # "group" (fp32 per 128 of K and channel), "block" (128 x 128)
 
     @property
     def d_out(self) -> int:
@@ -113,6 +116,8 @@ FP8_GMM = _reg(MoEConfig("e4m3_n8192_h7168_e256_k8_n2048_gmm", DTYPE_E4M3, 8192,
                          ACT_NONE, index=4, shared=(7168, 2048), routing="given"))
 MX_GMM = _reg(MoEConfig("e4m3mx_n8192_h7168_e256_k8_n2048_gmm", DTYPE_E4M3, 8192, 7168, 256, 8,
                         2048, ACT_NONE, index=5, routing="given", quant="mx"))
+BLOCK_GMM = _reg(MoEConfig("e4m3blk_n8192_h7168_e256_k8_n2048_gmm", DTYPE_E4M3, 8192, 7168, 256, 8,
+                           2048, ACT_NONE, index=8, routing="given", quant="block"))
 # Reduced copies of the two fp8 layers (a quarter of the tokens, E = 64, the
 # same per-expert shape and ~256 rows per expert): small enough for kernel
 # captures that replay every launch many times, weights (0.94 GB) still far
@@ -274,6 +279,37 @@ def quantize_mx(a: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     return codes.reshape(a.shape), (X + 127).astype(np.uint8).reshape(a.shape[:-1] + (d // 32,))
 
 
+def quantize_groups(a: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """e4m3 quantisation with one fp32 scale per 128 consecutive elements of
+    the last axis: scale = amax/448 (1 for an all-zero group), codes
+    e4m3(v / scale) rounded to nearest even, saturating."""
+    a = np.asarray(a, np.float64)
+    d = a.shape[-1]
+    assert d % 128 == 0, "groups are 128 elements"
+    b = a.reshape(-1, d // 128, 128)
+    amax = np.max(np.abs(b), axis=2)
+    scale = np.where(amax > 0, amax / 448.0, 1.0).astype(np.float32)
+    codes = e4m3_encode(b / scale.astype(np.float64)[..., None])
+    return codes.reshape(a.shape), scale.reshape(a.shape[:-1] + (d // 128,))
+
+
+def quantize_blocks(w: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """e4m3 quantisation of (E, F, d) weights with one fp32 scale per 128 x 128
+    block (128 output channels x 128 elements of K; the last channel block may
+    be ragged): scale = amax/448 (1 for an all-zero block)."""
+    w = np.asarray(w, np.float64)
+    E, F, d = w.shape
+    assert d % 128 == 0
+    fb = (F + 127) // 128
+    pad = np.zeros((E, fb * 128, d))
+    pad[:, :F] = w
+    b = pad.reshape(E, fb, 128, d // 128, 128)
+    amax = np.max(np.abs(b), axis=(2, 4))
+    scale = np.where(amax > 0, amax / 448.0, 1.0).astype(np.float32)
+    codes = e4m3_encode(b / scale.astype(np.float64)[:, :, None, :, None])
+    return codes.reshape(E, fb * 128, d)[:, :F], scale
+
+
 def normal_mx(seed: int, stream: int, rows: int, cols: int) -> tuple[np.ndarray, np.ndarray]:
     """rows x cols iid N(0,1) draws quantised to MXFP8 (quantize_mx), chunk by
     chunk of whole rows: (codes (rows, cols) uint8, scales (rows, cols/32))."""
@@ -333,6 +369,8 @@ class MoEInputs:
     w_sh_scale: float = 1.0
     x_sf: torch.Tensor | None = None    # (N, d/32) uint8 E8M0, MX workload
     w_sf: torch.Tensor | None = None    # (E, F, d/32) uint8 E8M0, MX workload
+    x_gs: torch.Tensor | None = None    # (N, d/128) fp32, group / block workloads
+    w_gs: torch.Tensor | None = None    # (E, F, d/128) fp32 (group) or (E, F/128, d/128) (block)
     extra: dict = field(default_factory=dict)
 
 
@@ -363,6 +401,23 @@ def make_inputs(cfg: MoEConfig, seed: int | None = None) -> MoEInputs:
     if seed is None:
         seed = SEED_BASE + cfg.index
     N, d, E, K, F = cfg.N, cfg.d, cfg.E, cfg.K, cfg.F
+    if cfg.dtype == DTYPE_E4M3 and cfg.quant in ("group", "block"):
+        xv = normal_f32(seed, 1, N * d).reshape(N, d)
+        xq, xgs = quantize_groups(xv)
+        wq = np.empty((E, F, d), np.uint8)
+        wgs = np.empty((E, F, d // 128) if cfg.quant == "group" else (E, (F + 127) // 128, d // 128),
+                       np.float32)
+        for e in range(E):   # expert by expert (bounded memory)
+            wv = normal_f32(seed, 100 + e, F * d).reshape(1, F, d)
+            if cfg.quant == "group":
+                c, sc = quantize_groups(wv[0])
+                wq[e], wgs[e] = c, sc
+            else:
+                c, sc = quantize_blocks(wv)
+                wq[e], wgs[e] = c[0], sc[0]
+        return MoEInputs(cfg, torch.from_numpy(xq), None, None, torch.from_numpy(wq), None, None,
+                         ids=torch.from_numpy(given_routing(seed, N, E, K)),
+                         x_gs=torch.from_numpy(xgs), w_gs=torch.from_numpy(wgs))
     if cfg.dtype == DTYPE_E4M3 and cfg.quant == "mx":
         xq, xsf = normal_mx(seed, 1, N, d)
         wq, wsf = normal_mx(seed, 2, E * F, d)

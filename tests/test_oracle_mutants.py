@@ -72,6 +72,15 @@ MUTANTS = [
     ("E8M0 bias 128 instead of 127",
      "return ldexp(1.0, (int)s - 127);",
      "return ldexp(1.0, (int)s - 128);"),
+    ("group of 64 instead of 128 elements",
+     "for (int k = 128 * g; k < 128 * g + 128; ++k)",
+     "for (int k = 64 * g; k < 64 * g + 128; ++k)"),
+    ("group scale of the activations taken from the first group",
+     "double sx = xs ? xs[(int64_t)r * ng + g] : x_scale;",
+     "double sx = xs ? xs[(int64_t)r * ng] : x_scale;"),
+    ("group weight scales indexed group-major",
+     "acc += sx * ws[wrow * ng + g] * part;",
+     "acc += sx * ws[((int64_t)e * ng + g) * F + n] * part;"),
     ("bf16 widened from the wrong half",
      "uint32_t u = (uint32_t)b << 16;",
      "uint32_t u = ((uint32_t)b << 16) | 0x8000u;"),

@@ -453,6 +453,83 @@ def test_mx_quantiser_blocks(orc):
                           | big)
 
 
+def test_group_scales_closed_form(orc):
+    """Quant modes 4/5 (fp32 scales per 128-element group of K): with every
+    element 1.0, xs[r][g] = 2^(r + g) and ws[e][n][g] = 2^(2g - n + e), each
+    group adds 128 * 2^(r - n + e) * 8^g: y = 128 * 2^(r - n + e) * (8^G - 1) / 7.
+    A group size other than 128, a transposed index or another expert's
+    scales change it."""
+    E, F, G, R = 3, 5, 3, 6
+    din = 128 * G
+    xs = np.array([[2.0 ** (r + g) for g in range(G)] for r in range(R)])
+    ws = np.array([[[2.0 ** (2 * g - n + e) for g in range(G)] for n in range(F)] for e in range(E)])
+    rexp = np.array([0, 1, 2, 2, 1, 0], np.int32)
+    y = orc.expert_rows_kscaled(rexp, _mx_ones(R, din), orc.E4M3, _mx_ones(E, F, din), orc.E4M3,
+                                ws, x_group_scales=xs)
+    for r in range(R):
+        e = int(rexp[r])
+        for n in range(F):
+            assert y[r, n] == 128 * 2.0 ** (r - n + e) * (8 ** G - 1) / 7
+
+
+def test_group_scales_exact_integers(orc):
+    """Small integer codes, random power-of-two group scales: exact in fp64,
+    so y equals sum_g xs * ws * (sum_{k in g} X*W) from Python integers; the
+    scalar x_scale replaces missing activation scales."""
+    rng = np.random.default_rng(17)
+    E, F, G, R = 3, 4, 2, 7
+    din = 128 * G
+    Xi = rng.integers(-8, 9, size=(R, din))
+    Wi = rng.integers(-8, 9, size=(E, F, din))
+    enc = np.vectorize(orc.f64_to_e4m3, otypes=[np.uint8])
+    Xq, Wq = enc(Xi.astype(np.float64)), enc(Wi.astype(np.float64))
+    xs = 2.0 ** rng.integers(-5, 4, size=(R, G))
+    ws = 2.0 ** rng.integers(-5, 4, size=(E, F, G))
+    rexp = rng.integers(0, E, size=R).astype(np.int32)
+    y = orc.expert_rows_kscaled(rexp, Xq, orc.E4M3, Wq, orc.E4M3, ws, x_group_scales=xs)
+    y2 = orc.expert_rows_kscaled(rexp, Xq, orc.E4M3, Wq, orc.E4M3, ws, x_scale=0.5)
+    for r in range(R):
+        e = int(rexp[r])
+        for n in range(F):
+            parts = [sum(int(Xi[r, k]) * int(Wi[e, n, k]) for k in range(128 * g, 128 * g + 128))
+                     for g in range(G)]
+            assert y[r, n] == sum(p * xs[r, g] * ws[e, n, g] for g, p in enumerate(parts))
+            assert y2[r, n] == sum(p * 0.5 * ws[e, n, g] for g, p in enumerate(parts))
+
+
+def test_group_scales_constant_over_groups_reduce_to_channel_scales(orc):
+    """Scales that do not change along K reduce modes 4/5 to per-channel
+    weights times per-token activations (modes 2/3), exactly on integer data."""
+    rng = np.random.default_rng(19)
+    E, F, G, R = 2, 6, 3, 5
+    din = 128 * G
+    enc = np.vectorize(orc.f64_to_e4m3, otypes=[np.uint8])
+    Xq = enc(rng.integers(-6, 7, size=(R, din)).astype(np.float64))
+    Wq = enc(rng.integers(-6, 7, size=(E, F, din)).astype(np.float64))
+    a = 2.0 ** rng.integers(-4, 4, size=R)
+    c = 2.0 ** rng.integers(-4, 4, size=(E, F))
+    rexp = np.array([0, 1, 1, 0, 1], np.int32)
+    y = orc.expert_rows_kscaled(rexp, Xq, orc.E4M3, Wq, orc.E4M3,
+                                np.repeat(c[:, :, None], G, axis=2),
+                                x_group_scales=np.repeat(a[:, None], G, axis=1))
+    y0 = orc.expert_rows_scaled(rexp, Xq, orc.E4M3, Wq, orc.E4M3, x_row_scales=a,
+                                w_channel_scales=c)
+    assert np.array_equal(y, y0)
+
+
+def test_block_scales_expand_to_channels(orc):
+    """A 128 x 128 weight block's scale applies to its 128 output channels:
+    channel n of a 300-channel expert takes block n // 128 (the last block
+    ragged)."""
+    E, F, G = 2, 300, 3
+    wb = np.arange(E * 3 * G, dtype=np.float64).reshape(E, 3, G) + 1.0
+    wg = orc.block_to_group_scales(wb, F)
+    assert wg.shape == (E, F, G)
+    for e in range(E):
+        for n in (0, 127, 128, 255, 256, 299):
+            assert np.array_equal(wg[e, n], wb[e, n // 128])
+
+
 def test_per_row_quantiser_round_trip():
     rng = np.random.default_rng(2)
     a = rng.standard_normal((50, 64)) * rng.uniform(0.01, 100, size=(50, 1))
