@@ -94,19 +94,27 @@ typedef enum { MOE_ACT_NONE = 0, MOE_ACT_RELU = 1, MOE_ACT_SWIGLU = 2 } moe_act;
 
 /* Scale granularity of the expert weights; values equal the Ascend page's
  * quant-mode enumeration (0 = not quantised, 1 = per-tensor, 2 =
- * per-channel: one scale per output column of each expert, 6 = mx).
+ * per-channel: one scale per output column of each expert, 4 = per-group,
+ * 5 = per-block, 6 = mx).
  * Per-token activation scales (mode 3) are a per-call argument
  * (x_token_scales); per-token dynamic quantization (mode 7) is
  * moe_permute_quant.  MX is read as OCP MXFP8: e4m3 elements in blocks of
  * 32 consecutive values along the reduction dimension (d), each block with
  * one E8M0 scale byte 2^(s - 127) (255 = NaN), for the weights
  * (w_mx_scales) and the activations (the _mx calls' x_mx_scales); the
- * single-matrix layer only, d a multiple of 32 and at most 32768.  Group and block modes (4, 5) are not built
- * (MOE_ERR_UNSUPPORTED). */
+ * single-matrix layer only, d a multiple of 32 and at most 32768.
+ * PER_GROUP and PER_BLOCK are read as fp32 weight scales per group of 128
+ * consecutive elements of d: one per output channel and group (PER_GROUP,
+ * w_group_scales (E, F, d/128)) or one per block of 128 output channels x
+ * 128 elements (PER_BLOCK, w_group_scales (E, ceil(F/128), d/128)); the
+ * activations take a scalar, per-token, or per-token-and-group scales (the
+ * _group_scales calls); the single-matrix layer only, d a multiple of 128. */
 typedef enum {
   MOE_QUANT_NONE = 0,
   MOE_QUANT_PER_TENSOR = 1,
   MOE_QUANT_PER_CHANNEL = 2,
+  MOE_QUANT_PER_GROUP = 4,
+  MOE_QUANT_PER_BLOCK = 5,
   MOE_QUANT_MX = 6
 } moe_quant;
 
@@ -118,7 +126,8 @@ typedef struct {
   int32_t F;      /* FFN inner width; for MOE_ACT_NONE the output width N1; < 65536 */
   moe_dtype dtype;/* of x and the expert weights */
   moe_act act;
-  moe_quant quant;/* PER_TENSOR or PER_CHANNEL for dtype MOE_E4M3; NONE otherwise */
+  moe_quant quant;/* PER_TENSOR, PER_CHANNEL, PER_GROUP, PER_BLOCK or MX for dtype
+                     MOE_E4M3; NONE otherwise */
 } moe_layer_desc;
 
 typedef struct {
@@ -131,6 +140,8 @@ typedef struct {
   const float* w_channel_scales; /* (E, F) fp32 per output channel, e4m3 PER_CHANNEL, else NULL */
   const uint8_t* w_mx_scales;    /* (E, F, d/32) E8M0 of w1, MOE_QUANT_MX, else NULL; read
                                     once by moe_plan_create (may be freed afterwards) */
+  const float* w_group_scales;   /* fp32 of w1: (E, F, d/128) PER_GROUP, (E, ceil(F/128),
+                                    d/128) PER_BLOCK, else NULL; read once by moe_plan_create */
 } moe_layer_weights;
 
 typedef struct moe_plan_s* moe_plan;
@@ -143,7 +154,8 @@ typedef struct moe_plan_s* moe_plan;
  * except for MOE_QUANT_MX: the plan then also holds a device copy of the
  * weight scales in the layout of the block-scaled tensor-core MMA (the same
  * bytes as w_mx_scales, rearranged; about E*F*d/32 bytes), made here
- * (synchronously) and freed by moe_plan_destroy.
+ * (synchronously) and freed by moe_plan_destroy; likewise for PER_GROUP /
+ * PER_BLOCK a transposed copy of w_group_scales (E, d/128, columns).
  * With w1, w3 and w2 all NULL (and no per-channel scales) the plan is
  * routing-only: router, permute and unpermute/combine work, the calls that
  * run the experts return MOE_ERR_UNSUPPORTED (an expert-parallel rank's
@@ -314,6 +326,31 @@ moe_status moe_permute_mx(moe_plan plan, const void* x, const uint8_t* x_mx_scal
 moe_status moe_grouped_ffn_mx(moe_plan plan, const void* x_perm, const uint8_t* x_perm_mx_scales,
                               const int32_t* offsets, void* y_perm, void* ws, size_t ws_bytes,
                               moe_stream_t stream);
+
+/* Group / block-scaled layer (MOE_QUANT_PER_GROUP or PER_BLOCK, act NONE):
+ *   gmmY[r][n] = sum_g xs[r][g] * ws[e][n][g] * (sum_{k in group g} x[r][k] * W[e][n][k])
+ * groups of 128 elements of d; ws the plan's weight scales (for PER_BLOCK
+ * the scale of channel n's block n/128); xs per row and group from
+ * x_group_scales (N, d/128), else per token from x_token_scales (N), else
+ * x_scale.  Every K stage of 128 is accumulated alone on the tensor cores
+ * (fp32) and added to fp32 sums with its scales; the result is rounded
+ * once to bf16.  moe_forward_routed_group_scales: permute, the grouped
+ * matmul, pure unpermute by its stores (gates NULL, y (N*K, F)) or combine
+ * (y (N, F)); the activation scales are indexed by token.
+ * moe_grouped_ffn_group_scales: permuted rows, their scales per permuted
+ * row (x_row_scales (N*K) or x_group_scales (N*K, d/128)).
+ * MOE_ERR_UNSUPPORTED for other plans. */
+moe_status moe_forward_routed_group_scales(moe_plan plan, const void* x, float x_scale,
+                                           const float* x_token_scales_or_null,
+                                           const float* x_group_scales_or_null,
+                                           const int32_t* topk_ids,
+                                           const float* topk_gates_or_null, void* y, void* ws,
+                                           size_t ws_bytes, moe_stream_t stream);
+moe_status moe_grouped_ffn_group_scales(moe_plan plan, const void* x_perm, float x_scale,
+                                        const float* x_row_scales_or_null,
+                                        const float* x_group_scales_or_null,
+                                        const int32_t* offsets, void* y_perm, void* ws,
+                                        size_t ws_bytes, moe_stream_t stream);
 
 /* Permute with per-token dynamic quantization (Ascend quant mode 7,
  * "pertoken dynamic quantization", parameter section): for an e4m3 plan, x is

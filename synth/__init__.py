@@ -407,14 +407,17 @@ def make_inputs(cfg: MoEConfig, seed: int | None = None) -> MoEInputs:
         wq = np.empty((E, F, d), np.uint8)
         wgs = np.empty((E, F, d // 128) if cfg.quant == "group" else (E, (F + 127) // 128, d // 128),
                        np.float32)
-        for e in range(E):   # expert by expert (bounded memory)
-            wv = normal_f32(seed, 100 + e, F * d).reshape(1, F, d)
+        def expert(e):   # expert by expert (bounded memory), experts in parallel
+            wv = np.random.Generator(np.random.Philox(np.random.SeedSequence([seed, 100, e]))) \
+                .standard_normal(F * d, dtype=np.float32).reshape(1, F, d)
             if cfg.quant == "group":
                 c, sc = quantize_groups(wv[0])
                 wq[e], wgs[e] = c, sc
             else:
                 c, sc = quantize_blocks(wv)
                 wq[e], wgs[e] = c[0], sc[0]
+
+        _run(expert, E)
         return MoEInputs(cfg, torch.from_numpy(xq), None, None, torch.from_numpy(wq), None, None,
                          ids=torch.from_numpy(given_routing(seed, N, E, K)),
                          x_gs=torch.from_numpy(xgs), w_gs=torch.from_numpy(wgs))

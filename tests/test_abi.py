@@ -28,7 +28,7 @@ def test_library_exports_every_header_symbol(lib):
 
 def test_struct_layouts_match_header():
     assert ctypes.sizeof(moe.LayerDesc) == 32
-    assert ctypes.sizeof(moe.LayerWeights) == 64
+    assert ctypes.sizeof(moe.LayerWeights) == 72
 
 
 def test_status_strings(lib):
@@ -37,9 +37,10 @@ def test_status_strings(lib):
 
 
 def _create(lib, N=64, d=64, E=8, K=2, F=64, dtype=moe.MOE_BF16, act=moe.ACT_SWIGLU,
-            quant=moe.QUANT_NONE, w1=0x1000, w3=0x2000, w2=0x3000, w_r=0x4000, w_mx=None):
+            quant=moe.QUANT_NONE, w1=0x1000, w3=0x2000, w2=0x3000, w_r=0x4000, w_mx=None,
+            w_gs=None):
     desc = moe.LayerDesc(N, d, E, K, F, dtype, act, quant)
-    w = moe.LayerWeights(w_r, None, w1, w3, w2, 1.0, None, w_mx)
+    w = moe.LayerWeights(w_r, None, w1, w3, w2, 1.0, None, w_mx, w_gs)
     h = ctypes.c_void_p()
     rc = lib.moe_plan_create(ctypes.byref(desc), ctypes.byref(w), ctypes.byref(h))
     if rc == 0:
@@ -55,7 +56,13 @@ def _create(lib, N=64, d=64, E=8, K=2, F=64, dtype=moe.MOE_BF16, act=moe.ACT_SWI
     (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None,
           quant=moe.QUANT_PER_CHANNEL), 1),                                # per-channel needs scales
     (dict(quant=7), 1),                                                    # mode 7 is per call
-    (dict(quant=4), 2), (dict(quant=5), 2),                                # group, block: not built
+    (dict(quant=4, w_gs=0x6000), 2), (dict(quant=5, w_gs=0x6000), 2),      # group, block need e4m3
+    (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None,
+          quant=moe.QUANT_PER_GROUP), 1),                                  # group needs its scales
+    (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None, d=192,
+          quant=moe.QUANT_PER_BLOCK, w_gs=0x6000), 1),                     # d not a multiple of 128
+    (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None,
+          quant=moe.QUANT_PER_TENSOR, w_gs=0x6000), 1),                    # scales without the mode
     (dict(quant=3), 2),                                                    # per-token is per call
     (dict(quant=moe.QUANT_MX, w_mx=0x5000), 2),                            # MX needs e4m3
     (dict(dtype=moe.MOE_E4M3, act=moe.ACT_NONE, w3=None, w2=None,

@@ -789,3 +789,121 @@ def test_mx_and_per_tensor_calls_are_not_mixed():
                                                            dtype=torch.uint8, device="cuda"),
                                 inp8.ids.cuda(), None, y8, ws8)
     assert e.value.code == 2
+
+
+# ------------------------------------------------- group / block scales (quant modes 4, 5)
+
+GS = {
+    # two 128-element groups, two column tiles (the second ragged)
+    "gs_small": synth.MoEConfig("gs_small", "e4m3", 300, 256, 8, 2, 384, "none", routing="given"),
+    # many small experts, four groups
+    "gs_fine": synth.MoEConfig("gs_fine", "e4m3", 128, 512, 64, 8, 256, "none", routing="given"),
+    # empty experts, one group, F below one 128-channel block
+    "gs_sparse": synth.MoEConfig("gs_sparse", "e4m3", 20, 128, 16, 1, 72, "none", routing="given"),
+    # an expert with several 128-row tiles, three groups
+    "gs_tall": synth.MoEConfig("gs_tall", "e4m3", 500, 384, 2, 1, 512, "none", routing="given"),
+}
+_gs_cache = {}
+
+
+def gs_case(name, quant):
+    """Inputs of a group/block case with independent random fp32 scales in
+    [0.25, 4) per weight group (or block) and per token and group."""
+    key = (name, quant)
+    if key not in _gs_cache:
+        import top_routing_grouped_gemv_b200 as moe
+        c = GS[name].scaled(quant=quant)
+        inp = synth.make_inputs(c, 77 + sum(map(ord, name)))
+        rng = np.random.default_rng(sum(map(ord, name)) + (0 if quant == "group" else 1))
+        G = c.d // 128
+        wshape = (c.E, c.F, G) if quant == "group" else (c.E, (c.F + 127) // 128, G)
+        ws = rng.uniform(0.25, 4.0, size=wshape).astype(np.float32)
+        xs = rng.uniform(0.25, 4.0, size=(c.N, G)).astype(np.float32)
+        wkey = "w_group_scales" if quant == "group" else "w_block_scales"
+        w = {"w1": inp.w1.cuda(), wkey: torch.from_numpy(ws).cuda()}
+        plan = moe.Plan(c.N, c.d, c.E, c.K, c.F, "e4m3", "none", w)
+        ws_full = ws.astype(np.float64) if quant == "group" else \
+            oracle.block_to_group_scales(ws, c.F)
+        _gs_cache[key] = (inp, plan, w, xs, ws_full)
+    return _gs_cache[key]
+
+
+def gs_ref(inp, ws_full, x_group=None, x_tok=None, x_scale=1.0, gates=None):
+    c = inp.cfg
+    ids = inp.ids.numpy()
+    _, _, rp, rs, rx = oracle.permute(ids, c.E, inp.x.numpy())
+    row_e = np.repeat(np.arange(c.E, dtype=np.int32), np.bincount(ids.ravel(), minlength=c.E))
+    G = c.d // 128
+    xg = None
+    if x_group is not None:
+        xg = x_group[rs].astype(np.float64)
+    elif x_tok is not None:
+        xg = np.repeat(x_tok[rs].astype(np.float64)[:, None], G, axis=1)
+    yp = oracle.expert_rows_kscaled(row_e, rx, oracle.E4M3, inp.w1, oracle.E4M3, ws_full,
+                                    x_group_scales=xg, x_scale=x_scale)
+    return oracle.combine(rp, gates, yp, c.N, c.K), yp, rp, rs
+
+
+@pytest.mark.parametrize("name", list(GS))
+@pytest.mark.parametrize("quant", ["group", "block"])
+@pytest.mark.parametrize("gated", [False, True])
+def test_forward_routed_group_scales(name, quant, gated):
+    inp, plan, w, xs, ws_full = gs_case(name, quant)
+    c = inp.cfg
+    wsp = plan.new_workspace()
+    g = None
+    if gated:
+        g = np.random.default_rng(4).random((c.N, c.K)).astype(np.float32)
+        y = torch.empty(c.N, c.F, dtype=torch.bfloat16, device="cuda")
+    else:
+        y = torch.full((c.N * c.K, c.F), float("nan"), dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed_group_scales(inp.x.cuda(), inp.ids.cuda(),
+                                     None if g is None else torch.from_numpy(g).cuda(), y, wsp,
+                                     x_group_scales=torch.from_numpy(xs).cuda())
+    assert plan.read_device_status(wsp) == 0
+    ref, _, _, _ = gs_ref(inp, ws_full, x_group=xs,
+                          gates=None if g is None else g.astype(np.float64))
+    err = rel_err(f64(y), ref)
+    assert err <= TOL["e4m3"], err
+    assert err <= 1e-2, err   # fp32 stage sums and promotion, one bf16 rounding
+
+
+@pytest.mark.parametrize("quant", ["group", "block"])
+def test_group_scales_with_token_and_scalar_activation_scales(quant):
+    inp, plan, w, xs, ws_full = gs_case("gs_small", quant)
+    c = inp.cfg
+    wsp = plan.new_workspace()
+    tok = np.random.default_rng(8).uniform(0.5, 2.0, size=c.N).astype(np.float32)
+    y = torch.empty(c.N * c.K, c.F, dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed_group_scales(inp.x.cuda(), inp.ids.cuda(), None, y, wsp,
+                                     x_token_scales=torch.from_numpy(tok).cuda())
+    assert plan.read_device_status(wsp) == 0
+    ref, _, _, _ = gs_ref(inp, ws_full, x_tok=tok)
+    assert rel_err(f64(y), ref) <= 1e-2
+    plan.forward_routed_group_scales(inp.x.cuda(), inp.ids.cuda(), None, y, wsp, x_scale=0.375)
+    ref, _, _, _ = gs_ref(inp, ws_full, x_scale=0.375)
+    assert rel_err(f64(y), ref) <= 1e-2
+
+
+@pytest.mark.parametrize("name", ["gs_small", "gs_sparse", "gs_tall"])
+@pytest.mark.parametrize("quant", ["group", "block"])
+def test_group_scales_stage_call_equals_fused(name, quant):
+    """moe_grouped_ffn_group_scales on the permuted rows (scales per permuted
+    row) against the oracle, and the fused call's unpermuted rows equal to it
+    bit for bit."""
+    inp, plan, w, xs, ws_full = gs_case(name, quant)
+    c = inp.cfg
+    R = c.N * c.K
+    wsp = plan.new_workspace()
+    ref, yp_ref, rp, rs = gs_ref(inp, ws_full, x_group=xs)
+    _, ro, _, _, rx = oracle.permute(inp.ids.numpy(), c.E, inp.x.numpy())
+    y_perm = torch.empty(R, c.F, dtype=torch.bfloat16, device="cuda")
+    plan.grouped_ffn_group_scales(torch.from_numpy(rx).cuda(), torch.from_numpy(ro).cuda(), y_perm,
+                                  wsp, x_group_scales=torch.from_numpy(xs[rs]).cuda())
+    assert plan.read_device_status(wsp) == 0
+    assert rel_err(f64(y_perm), yp_ref) <= 1e-2
+    y = torch.empty(R, c.F, dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed_group_scales(inp.x.cuda(), inp.ids.cuda(), None, y, wsp,
+                                     x_group_scales=torch.from_numpy(xs).cuda())
+    yp = y_perm.cpu().view(torch.int16).numpy()
+    assert np.array_equal(y.cpu().view(torch.int16).numpy(), yp[rp])

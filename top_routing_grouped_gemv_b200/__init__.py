@@ -21,6 +21,7 @@ HEADER = os.path.join(ROOT, "include", "moe.h")
 MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
 ACT_NONE, ACT_RELU, ACT_SWIGLU = 0, 1, 2
 QUANT_NONE, QUANT_PER_TENSOR, QUANT_PER_CHANNEL, QUANT_MX = 0, 1, 2, 6
+QUANT_PER_GROUP, QUANT_PER_BLOCK = 4, 5
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
           3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_BAD_INDEX",
@@ -45,7 +46,7 @@ class LayerWeights(ctypes.Structure):
     _fields_ = [("w_r", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
                 ("w1", ctypes.c_void_p), ("w3", ctypes.c_void_p), ("w2", ctypes.c_void_p),
                 ("w_scale", ctypes.c_float), ("w_channel_scales", ctypes.c_void_p),
-                ("w_mx_scales", ctypes.c_void_p)]
+                ("w_mx_scales", ctypes.c_void_p), ("w_group_scales", ctypes.c_void_p)]
 
 
 _lib = None
@@ -91,6 +92,8 @@ def load(path: str = LIB_PATH):
         "moe_forward_routed_mx": ([P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_permute_mx": ([P, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_grouped_ffn_mx": ([P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_forward_routed_group_scales": ([P, P, f32, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "moe_grouped_ffn_group_scales": ([P, P, f32, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_permute_n": ([P, i32, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "moe_grouped_ffn_n": ([P, i32, P, P, f32, P, P, P, sz, P], ctypes.c_int),
         "moe_unpermute_combine_n": ([P, i32, P, P, P, P, P, sz, P], ctypes.c_int),
@@ -134,8 +137,9 @@ class Plan:
     ``weights``: dict with torch CUDA tensors ``w_r`` (d, E) fp32, optional
     ``bias`` (E,), ``w1`` (E, F, d), ``w3`` (E, F, d) for SwiGLU, ``w2``
     (E, d, F), and float ``w_scale`` (e4m3); for e4m3, optional
-    ``w_channel_scales`` (E, F) fp32 (per-channel) or ``w_mx_scales`` (E, F,
-    d/32) uint8 E8M0 (MX).  The tensors are kept alive by the plan (the
+    ``w_channel_scales`` (E, F) fp32 (per-channel), ``w_group_scales`` (E, F,
+    d/128) fp32 (per-group), ``w_block_scales`` (E, ceil(F/128), d/128) fp32
+    (per-block) or ``w_mx_scales`` (E, F, d/32) uint8 E8M0 (MX).  The tensors are kept alive by the plan (the
     library only records their addresses).
     """
 
@@ -147,13 +151,18 @@ class Plan:
         self._keep = dict(weights)
         quant = QUANT_NONE
         if dtype == "e4m3":
-            quant = QUANT_PER_CHANNEL if weights.get("w_channel_scales") is not None \
-                else QUANT_MX if weights.get("w_mx_scales") is not None else QUANT_PER_TENSOR
+            quant = QUANT_PER_TENSOR
+            for key, code in (("w_channel_scales", QUANT_PER_CHANNEL), ("w_mx_scales", QUANT_MX),
+                              ("w_group_scales", QUANT_PER_GROUP),
+                              ("w_block_scales", QUANT_PER_BLOCK)):
+                if weights.get(key) is not None:
+                    quant = code
         desc = LayerDesc(N, d, E, K, F, DTYPE_CODE[dtype], ACT_CODE[act], quant)
         w = LayerWeights(_ptr(weights.get("w_r")), _ptr(weights.get("bias")),
                          _ptr(weights.get("w1")), _ptr(weights.get("w3")),
                          _ptr(weights.get("w2")), float(weights.get("w_scale", 1.0)),
-                         _ptr(weights.get("w_channel_scales")), _ptr(weights.get("w_mx_scales")))
+                         _ptr(weights.get("w_channel_scales")), _ptr(weights.get("w_mx_scales")),
+                         _ptr(weights.get("w_group_scales", weights.get("w_block_scales"))))
         h = ctypes.c_void_p()
         _check(self.lib.moe_plan_create(ctypes.byref(desc), ctypes.byref(w), ctypes.byref(h)),
                "moe_plan_create")
@@ -269,6 +278,20 @@ class Plan:
         _check(self.lib.moe_grouped_ffn_mx(self.handle, _ptr(x_perm), _ptr(x_perm_mx_scales),
                                            _ptr(offsets), _ptr(y_perm), _ptr(ws), ws.numel(),
                                            _stream(stream)), "moe_grouped_ffn_mx")
+
+    def forward_routed_group_scales(self, x, ids, gates, y, ws, x_scale: float = 1.0,
+                                    x_token_scales=None, x_group_scales=None, stream=None):
+        _check(self.lib.moe_forward_routed_group_scales(
+            self.handle, _ptr(x), x_scale, _ptr(x_token_scales), _ptr(x_group_scales), _ptr(ids),
+            _ptr(gates), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)),
+            "moe_forward_routed_group_scales")
+
+    def grouped_ffn_group_scales(self, x_perm, offsets, y_perm, ws, x_scale: float = 1.0,
+                                 x_row_scales=None, x_group_scales=None, stream=None):
+        _check(self.lib.moe_grouped_ffn_group_scales(
+            self.handle, _ptr(x_perm), x_scale, _ptr(x_row_scales), _ptr(x_group_scales),
+            _ptr(offsets), _ptr(y_perm), _ptr(ws), ws.numel(), _stream(stream)),
+            "moe_grouped_ffn_group_scales")
 
     def forward_routed_dynamic(self, x_bf16, ids, gates, y, ws, stream=None):
         _check(self.lib.moe_forward_routed_dynamic(self.handle, _ptr(x_bf16), _ptr(ids),

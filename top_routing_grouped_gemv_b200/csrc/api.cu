@@ -55,6 +55,7 @@ struct moe_plan_s {
   cudaEvent_t hev[kHostEvents];
   unsigned long long host_calls;  // host-buffer calls so far (selects the staging slot)
   uint8_t* sfb;  // MX plans: the weight scales in the tensor-core layout (owned)
+  float* wgs;    // group / block plans: the weight scales, (E, d/128, F or F/128) (owned)
 };
 
 namespace {
@@ -209,7 +210,8 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
                    const float* x_rows, const int32_t* row_index, void* y_perm, void* ws,
                    cudaStream_t s, const int32_t* out_rows = nullptr) {
   const moe_layer_desc& d = p->desc;
-  if (d.quant == MOE_QUANT_MX) return MOE_ERR_UNSUPPORTED;  // the _mx calls carry the scales
+  if (d.quant == MOE_QUANT_MX || d.quant == MOE_QUANT_PER_GROUP || d.quant == MOE_QUANT_PER_BLOCK)
+    return MOE_ERR_UNSUPPORTED;  // the _mx / _group_scales calls carry the scales
   const int R = n * d.K;
   int* status = at<int>(ws, p->L.status);
   void* h = at<void>(ws, p->L.h);
@@ -327,6 +329,40 @@ moe_status run_ffn_mx(moe_plan p, int n, const void* x_perm, const int32_t* offs
   return cuda_status(launch_gemm_tc(a, kGemmMxE4M3, kEpiStore, R, false, s));
 }
 
+// Group / block-scaled grouped matmul (quant modes 4, 5).  Activation
+// scales: x_group (per row and 128-element group, indexed through
+// row_index), else x_rows (per row), else x_scale.
+moe_status run_ffn_gs(moe_plan p, int n, const void* x_perm, const int32_t* offsets, float x_scale,
+                      const float* x_rows, const float* x_group, const int32_t* row_index,
+                      void* y_perm, void* ws, cudaStream_t s, const int32_t* out_rows = nullptr) {
+  const moe_layer_desc& d = p->desc;
+  const int R = n * d.K;
+  TcGemmArgs a;
+  memset(&a, 0, sizeof(a));
+  if (!encode_kmajor_map(&a.tmA, x_perm, 1, R > 0 ? R : 1, d.d, kTcBlockM)) return MOE_ERR_CUDA;
+  a.tmB0 = p->tmW1;
+  a.tmB1 = a.tmB0;
+  a.offsets = offsets;
+  a.groups = d.E;
+  a.m_total = R;
+  a.kdim = d.d;
+  a.n_out = d.F;
+  a.n_tiles = (d.F + kTcBlockN - 1) / kTcBlockN;
+  a.out = y_perm;
+  a.out_rows = out_rows;
+  a.ldo = d.F;
+  a.scale = x_group || x_rows ? 1.f : x_scale;
+  a.row_scale = x_group ? nullptr : x_rows;
+  a.row_index = row_index;
+  a.xgs = x_group;
+  a.wgs = p->wgs;
+  a.status = at<int>(ws, p->L.status);
+  const bool blocks = d.quant == MOE_QUANT_PER_BLOCK;
+  mark(p, s, blocks ? "gmm_block_tc" : "gmm_group_tc");
+  p->launches += 1;
+  return cuda_status(launch_gemm_tc(a, kE4M3, blocks ? kEpiBlockScale : kEpiGroupScale, R, false, s));
+}
+
 moe_status run_combine(moe_plan p, int n, const void* y_perm, const int32_t* pos,
                        const float* gates, void* y, void* ws, cudaStream_t s) {
   const moe_layer_desc& d = p->desc;
@@ -373,12 +409,15 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
   if (d.dtype < MOE_F32 || d.dtype > MOE_E4M3 || d.act < MOE_ACT_NONE || d.act > MOE_ACT_SWIGLU ||
       d.quant < MOE_QUANT_NONE || d.quant > MOE_QUANT_MX)
     return MOE_ERR_INVALID_ARG;
-  // modes 3 (per-token) and 7 (dynamic) are per-call; 4 and 5 are not built
-  if (d.quant == 3 || d.quant == 4 || d.quant == 5) return MOE_ERR_UNSUPPORTED;
+  // modes 3 (per-token) and 7 (dynamic) are per-call arguments
+  if (d.quant == 3) return MOE_ERR_UNSUPPORTED;
+  const bool gs = d.quant == MOE_QUANT_PER_GROUP || d.quant == MOE_QUANT_PER_BLOCK;
   if ((d.quant != MOE_QUANT_NONE) != (d.dtype == MOE_E4M3)) return MOE_ERR_UNSUPPORTED;
   if ((d.quant == MOE_QUANT_PER_CHANNEL) != (w->w_channel_scales != nullptr))
     return MOE_ERR_INVALID_ARG;
   if (d.quant != MOE_QUANT_MX && w->w_mx_scales) return MOE_ERR_INVALID_ARG;
+  if (!gs && w->w_group_scales) return MOE_ERR_INVALID_ARG;
+  if (gs && (d.d % 128 || (w->w1 && !w->w_group_scales))) return MOE_ERR_INVALID_ARG;
   if (d.quant == MOE_QUANT_MX && (d.d % kMxBlock || d.d > kMxMaxKdim || (w->w1 && !w->w_mx_scales)))
     return MOE_ERR_INVALID_ARG;
   if (d.dtype == MOE_E4M3 && d.act != MOE_ACT_NONE) return MOE_ERR_UNSUPPORTED;
@@ -387,7 +426,7 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
   // an expert-parallel layer whose experts live on other GPUs) takes none of
   // w1, w3, w2
   const bool routing_only = !w->w1 && !w->w3 && !w->w2 && d.quant != MOE_QUANT_PER_CHANNEL &&
-                            !w->w_mx_scales;
+                            !w->w_mx_scales && !w->w_group_scales;
   if (!routing_only && (!w->w1 || (d.act == MOE_ACT_SWIGLU) != (w->w3 != nullptr) ||
                         (d.act != MOE_ACT_NONE) != (w->w2 != nullptr)))
     return MOE_ERR_INVALID_ARG;
@@ -448,6 +487,26 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
       return MOE_ERR_CUDA;
     }
   }
+  if (gs && !routing_only) {
+    // the weight scales, once, transposed to (E, d/128, columns): a stage's
+    // scales are contiguous for the epilogue (256 floats of slack at the end
+    // for its vector loads past the last column)
+    const int ng = d.d / 128;
+    const int cols = d.quant == MOE_QUANT_PER_BLOCK ? (d.F + 127) / 128 : d.F;
+    const size_t bytes = (static_cast<size_t>(d.E) * ng * cols + 256) * sizeof(float);
+    cudaStream_t cs = nullptr;
+    bool ok = cudaMalloc(reinterpret_cast<void**>(&p->wgs), bytes) == cudaSuccess;
+    ok = ok && cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) == cudaSuccess;
+    ok = ok && cudaMemsetAsync(p->wgs, 0, bytes, cs) == cudaSuccess;
+    ok = ok && launch_group_scales_t(w->w_group_scales, d.E, cols, ng, p->wgs, cs) == cudaSuccess;
+    ok = ok && cudaStreamSynchronize(cs) == cudaSuccess;
+    if (cs) cudaStreamDestroy(cs);
+    if (!ok) {
+      if (p->wgs) cudaFree(p->wgs);
+      delete p;
+      return MOE_ERR_CUDA;
+    }
+  }
   for (int i = 0; i < kMaxEvents; ++i) p->ev[i] = nullptr;
   layout(p);
   *out = p;
@@ -466,6 +525,7 @@ moe_status moe_plan_destroy(moe_plan p) {
     if (p->sev[i]) cudaEventDestroy(p->sev[i]);
   if (p->side) cudaStreamDestroy(p->side);
   if (p->sfb) cudaFree(p->sfb);
+  if (p->wgs) cudaFree(p->wgs);
   delete p;
   return MOE_OK;
 }
@@ -693,6 +753,54 @@ moe_status moe_forward_routed_mx(moe_plan p, const void* x, const uint8_t* x_mx_
   if (st == MOE_OK)
     st = run_ffn_mx(p, d.N, at<void>(ws, L.x_perm), offsets, gates ? at<void>(ws, L.y_perm) : y, ws,
                     stream, slot);
+  if (st == MOE_OK && gates)
+    st = run_combine(p, d.N, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_grouped_ffn_group_scales(moe_plan p, const void* x_perm, float x_scale,
+                                        const float* x_row_scales, const float* x_group_scales,
+                                        const int32_t* offsets, void* y_perm, void* ws,
+                                        size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !x_perm || !offsets || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (p->desc.quant != MOE_QUANT_PER_GROUP && p->desc.quant != MOE_QUANT_PER_BLOCK)
+    return MOE_ERR_UNSUPPORTED;
+  if (!p->w.w1) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x_perm) || !aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.permute_end);
+  if (st != MOE_OK) return st;
+  begin(p);
+  st = run_ffn_gs(p, p->desc.N, x_perm, offsets, x_scale, x_row_scales, x_group_scales, nullptr,
+                  y_perm, ws, stream);
+  end(p, stream);
+  return st;
+}
+
+moe_status moe_forward_routed_group_scales(moe_plan p, const void* x, float x_scale,
+                                           const float* x_token_scales,
+                                           const float* x_group_scales, const int32_t* ids,
+                                           const float* gates, void* y, void* ws,
+                                           size_t ws_bytes, moe_stream_t stream) {
+  if (!p || !x || !ids || !y) return MOE_ERR_INVALID_ARG;
+  if (p->desc.quant != MOE_QUANT_PER_GROUP && p->desc.quant != MOE_QUANT_PER_BLOCK)
+    return MOE_ERR_UNSUPPORTED;
+  if (!p->w.w1) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_ws(p, ws, ws_bytes, p->L.fwd_end);
+  if (st != MOE_OK) return st;
+  const moe_layer_desc& d = p->desc;
+  const Layout& L = p->L;
+  begin(p);
+  int32_t* src = at<int32_t>(ws, L.src);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* slot = gates ? nullptr : at<int32_t>(ws, L.slot);  // unpermute by the GEMM's stores
+  st = run_permute(p, d.N, x, ids, at<int32_t>(ws, L.counts), offsets, at<int32_t>(ws, L.pos), src,
+                   at<void>(ws, L.x_perm), ws, stream, slot);
+  // the activation scales reach the permuted rows through the source token
+  if (st == MOE_OK)
+    st = run_ffn_gs(p, d.N, at<void>(ws, L.x_perm), offsets, x_scale, x_token_scales,
+                    x_group_scales, src, gates ? at<void>(ws, L.y_perm) : y, ws, stream, slot);
   if (st == MOE_OK && gates)
     st = run_combine(p, d.N, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), gates, y, ws, stream);
   end(p, stream);

@@ -60,7 +60,14 @@ constexpr int BM = kTcBlockM;     // 128 rows per CTA (256 per CTA pair)
 constexpr int BN = kTcBlockN;     // 256 accumulator columns per tile
 constexpr int ROWB = 128;         // bytes of K per row per stage (one swizzle atom)
 constexpr int A_BYTES = BM * ROWB;
-constexpr int kThreads = 192;
+// producer warp, MMA warp, epilogue warps: four (one per TMEM lane
+// quadrant), eight for the group-scaled epilogues (two per quadrant, 128
+// columns each, whose fp32 sums live in registers)
+constexpr int kGsEpiWarps = 8;
+template <int kEpi>
+constexpr int threads_of() {
+  return kEpi == kEpiGroupScale || kEpi == kEpiBlockScale ? 32 * (2 + kGsEpiWarps) : 192;
+}
 constexpr uint32_t kTmemCols = 2 * BN;
 constexpr int kMaxGroups = 256;
 
@@ -126,11 +133,13 @@ __device__ __forceinline__ uint32_t mx_sf_ids(uint32_t k) { return (k << 29) | (
 // CTA rank r holds rows [128r, 128r+128) of the tile and B rows [128r, 128r+128)
 // of the 256-row weight tile; the leader (rank 0) issues the MMAs.
 template <bool kFp8, int kEpi, bool kPair, bool kMx>
-__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ TcGemmArgs args) {
+__global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __grid_constant__ TcGemmArgs args) {
   griddep_trigger();  // let the next kernel of the stream start launching
   griddep_wait();     // inputs written by the previous kernel are visible
 
   static_assert(!kMx || (kFp8 && !kPair && kEpi == kEpiStore), "MX: e4m3, single CTA, store");
+  constexpr bool kGs = kEpi == kEpiGroupScale || kEpi == kEpiBlockScale;
+  static_assert(!kGs || (kFp8 && !kPair && !kMx), "group scales: e4m3, single CTA");
   using Gm = Geo<kPair, kMx>;
   constexpr int STAGES = Gm::STAGES;
   constexpr int kAcc = kMx ? 1 : 2;  // accumulators in TMEM
@@ -193,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar(Gm::kBarTFull + a), 1);
-      mbar_init(bar(Gm::kBarTEmpty + a), kPair ? 8 : 4);
+      mbar_init(bar(Gm::kBarTEmpty + a), kGs ? kGsEpiWarps : kPair ? 8 : 4);
     }
     mbar_init(bar(Gm::kBarDrain), 1);
     *abort_flag = 0;
@@ -290,7 +299,36 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     __syncwarp();
   } else if (warp == 1) {
     // ---------------- MMA issuer (the pair leader issues for both CTAs) ----------------
-    if (lane == 0 && leader) {
+    if (kGs && lane == 0) {
+      // every K stage into a fresh accumulator (the two alternate); the
+      // epilogue adds it to its fp32 sums with the stage's scales
+      constexpr uint32_t idesc = make_idesc_mode<true, false>();
+      int s = 0;
+      uint32_t ph = 0, j = 0;
+      bool aborted = false;
+      for (int T = unit; T < total && !aborted; T += nunits) {
+        for (int kb = 0; kb < num_kb; ++kb, ++j) {
+          const uint32_t acc = j & 1u, aph = (j >> 1) & 1u;
+          if (!mbar_wait(bar(Gm::kBarTEmpty + acc), aph ^ 1u, abort_flag)) { aborted = true; break; }
+          if (!mbar_wait(bar(Gm::kBarFull + s), ph, abort_flag)) { aborted = true; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * static_cast<uint32_t>(BN);
+          const uint32_t a0 = sA + s * A_BYTES, b0 = sB + s * Gm::B_BYTES;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma<true>(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc,
+                         k != 0 ? 1u : 0u);
+          tc_commit(bar(Gm::kBarEmpty + s));
+          tc_commit(bar(Gm::kBarTFull + acc));
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (aborted) {
+        set_status(args.status, kStatusTimeout);
+        tc_commit(bar(Gm::kBarDrain));
+        mbar_wait_drain(bar(Gm::kBarDrain), 0);
+      }
+    } else if (!kGs && lane == 0 && leader) {
       constexpr uint32_t idesc = kMx ? make_idesc_mx() : make_idesc_mode<kFp8, kPair>();
       // MX scale columns (after the single accumulator): A at BN, B at BN + 4
       const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(BN);
@@ -348,10 +386,101 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5 of every CTA) ----------------
+    // ---------------- epilogue (warps 2..5 of every CTA; 2..17 group-scaled) ----------------
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     int i = 0;
-    for (int T = unit; T < total; T += nunits, ++i) {
+    if constexpr (kGs) {
+      constexpr int kCols = BN / (kGsEpiWarps / 4);  // columns of this warp
+      const int half = (warp - 2) >> 2;               // its column slice
+      const int nblk = (args.n_out + 127) / 128;
+      uint32_t j = 0;
+      for (int T = unit; T < total; T += nunits) {
+        const TileCoord c = decode_tile<Gm::TILE_M>(T, s_pref, s_off, G, args.n_tiles);
+        const int row = q * 32 + lane;
+        const long long grow = static_cast<long long>(c.m_row0) + row;
+        const bool valid = grow < s_off[c.g + 1] && grow < args.m_total && grow >= 0;
+        const long long srow = valid && args.row_index != nullptr ? args.row_index[grow] : grow;
+        const int col0 = c.n_tile * BN + half * kCols;
+        const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                            static_cast<uint32_t>(half * kCols);
+        float sum[kCols];
+#pragma unroll
+        for (int cc = 0; cc < kCols; ++cc) sum[cc] = 0.f;
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb, ++j) {
+          const uint32_t a = j & 1u, aph = (j >> 1) & 1u;
+          ok = __shfl_sync(0xffffffffu, mbar_wait(bar(Gm::kBarTFull + a), aph, abort_flag), 0);
+          if (!ok) break;
+          tc_fence_after();
+          const float sx = valid && args.xgs != nullptr ? args.xgs[srow * num_kb + kb] : 1.f;
+          const long long wk = static_cast<long long>(c.g) * num_kb + kb;
+          if constexpr (kEpi == kEpiBlockScale) {
+            // one 128 x 128 weight block covers this warp's columns
+            const float f = sx * args.wgs[wk * nblk + col0 / 128];
+#pragma unroll
+            for (int cc = 0; cc < kCols; cc += 16) {
+              uint32_t v[16];
+              __syncwarp();
+              tmem_ld16(tq + a * BN + cc, v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) sum[cc + jj] = fmaf(__uint_as_float(v[jj]), f, sum[cc + jj]);
+            }
+          } else {
+            // per-column scales: eight columns at a time (registers: the 128
+            // sums stay live across the stages)
+            const float4* w4 = reinterpret_cast<const float4*>(args.wgs + wk * args.n_out + col0);
+#pragma unroll
+            for (int cc = 0; cc < kCols; cc += 8) {
+              uint32_t v[8];
+              __syncwarp();
+              tmem_ld8(tq + a * BN + cc, v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int jj = 0; jj < 8; jj += 4) {
+                const float4 w = __ldg(w4 + (cc + jj) / 4);
+                sum[cc + jj] = fmaf(__uint_as_float(v[jj]), sx * w.x, sum[cc + jj]);
+                sum[cc + jj + 1] = fmaf(__uint_as_float(v[jj + 1]), sx * w.y, sum[cc + jj + 1]);
+                sum[cc + jj + 2] = fmaf(__uint_as_float(v[jj + 2]), sx * w.z, sum[cc + jj + 2]);
+                sum[cc + jj + 3] = fmaf(__uint_as_float(v[jj + 3]), sx * w.w, sum[cc + jj + 3]);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(Gm::kBarTEmpty + a));
+        }
+        if (!ok) {
+          set_status(args.status, kStatusTimeout);
+          break;
+        }
+        if (valid) {
+          float sc = args.scale;
+          if (args.row_scale != nullptr)
+            sc *= args.row_scale[args.row_index != nullptr ? args.row_index[grow] : grow];
+          const long long orow_i = args.out_rows != nullptr ? args.out_rows[grow] : grow;
+          __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + orow_i * args.ldo;
+#pragma unroll
+          for (int cc = 0; cc < kCols; cc += 32) {
+            const int col = col0 + cc;
+            if (col + 32 <= args.n_out) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4)
+                dst[q4] = make_uint4(pack_bf16x2(sum[cc + 8 * q4] * sc, sum[cc + 8 * q4 + 1] * sc),
+                                     pack_bf16x2(sum[cc + 8 * q4 + 2] * sc, sum[cc + 8 * q4 + 3] * sc),
+                                     pack_bf16x2(sum[cc + 8 * q4 + 4] * sc, sum[cc + 8 * q4 + 5] * sc),
+                                     pack_bf16x2(sum[cc + 8 * q4 + 6] * sc, sum[cc + 8 * q4 + 7] * sc));
+            } else if (col < args.n_out) {
+#pragma unroll
+              for (int jj = 0; jj < 32; ++jj)
+                if (col + jj < args.n_out) orow[col + jj] = __float2bfloat16_rn(sum[cc + jj] * sc);
+            }
+          }
+        }
+      }
+    }
+    for (int T = unit; !kGs && T < total; T += nunits, ++i) {
       const int acc = i % kAcc;
       const uint32_t aph = (i / kAcc) & 1;
       // every lane polls; lane 0's answer is taken by all (and converges the warp
@@ -528,7 +657,7 @@ cudaError_t launch_t(const TcGemmArgs& args, long long max_units, cudaStream_t s
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(threads_of<kEpi>(), 1, 1);
   cfg.dynamicSmemBytes = Gm::kSmemBytes;
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -589,6 +718,11 @@ cudaError_t launch_gemm_tc(const TcGemmArgs& args, int dtype, int epilogue, int 
   if (dtype == kGemmMxE4M3) {
     if (pair || epilogue != kEpiStore || !args.sfa || !args.sfb) return cudaErrorInvalidValue;
     return launch_t<true, kEpiStore, false, true>(args, max_units, stream);
+  }
+  if (epilogue == kEpiGroupScale || epilogue == kEpiBlockScale) {
+    if (pair || dtype != kE4M3 || !args.wgs || args.kdim % 128) return cudaErrorInvalidValue;
+    return epilogue == kEpiGroupScale ? launch_t<true, kEpiGroupScale, false>(args, max_units, stream)
+                                      : launch_t<true, kEpiBlockScale, false>(args, max_units, stream);
   }
   const bool fp8 = dtype == kE4M3;
   const bool sw = epilogue == kEpiSwiglu;

@@ -108,7 +108,13 @@ size_t simt_f32_partial_bytes(int kdim, int ncols, int R, int E, int act);
 // ---- grouped GEMM on tcgen05 tensor cores -----------------------------------
 // kEpiRouter: fp32 logits from the three-part split router weights (bf16,
 // single-CTA tiles only).
-enum TcEpilogue { kEpiStore = 0, kEpiSwiglu = 1, kEpiRouter = 2 };
+// kEpiGroupScale: e4m3 store epilogue with fp32 scales per 128-element K
+// stage (group / block quantization): every stage is accumulated alone and
+// the epilogue adds it to fp32 registers times the stage's scales.
+// kEpiGroupScale takes one weight scale per output column and stage,
+// kEpiBlockScale one per 128 x 128 weight block.
+enum TcEpilogue { kEpiStore = 0, kEpiSwiglu = 1, kEpiRouter = 2, kEpiGroupScale = 3,
+                  kEpiBlockScale = 4 };
 
 struct TcGemmArgs {
   CUtensorMap tmA;   // activations: rows (R), cols kdim
@@ -138,6 +144,16 @@ struct TcGemmArgs {
   // a new tile), sfb per (group, 256-row weight tile).
   const uint8_t* sfa;
   const uint8_t* sfb;
+  // Group scales (kEpiGroupScale, kEpiBlockScale), one per 128-element K
+  // stage kb:
+  //   out = sum_kb (xgs[row'][kb] (1 if NULL) * w) * acc_kb, then * scale * row_scale
+  // w = wgs[(g * num_kb + kb) * n_out + col] (kEpiGroupScale, per output
+  // column; the buffer holds 256 floats of slack past its end), or
+  // wgs[(g * num_kb + kb) * ceil(n_out / 128) + col / 128] (kEpiBlockScale,
+  // 128 x 128 weight blocks).  row' = row_index[row] (or row); num_kb =
+  // kdim / 128.
+  const float* xgs;
+  const float* wgs;
 };
 
 // Host: encode a 2-D K-major tile map over a (rows, kdim) row-major matrix of
@@ -189,6 +205,10 @@ cudaError_t launch_mx_weight_sf(const uint8_t* w_sf, int groups, int n_out, int 
 cudaError_t launch_mx_act_sf(const uint8_t* x_sf, const int32_t* src_rows, const int32_t* offsets,
                              int groups, int rows_upper, int kdim, uint8_t* out,
                              cudaStream_t stream);
+// Group / block scales of the weights, (E, rows, ng) fp32 -> the kernel's
+// (E, ng, rows) layout (rows = F per output column, or ceil(F / 128) blocks).
+cudaError_t launch_group_scales_t(const float* src, int groups, int rows, int ng, float* dst,
+                                  cudaStream_t stream);
 // Row gather of scales: out row r = x_sf row src_rows[r], for r <
 // offsets[groups] (at most rows_upper); nsf bytes per row.
 cudaError_t launch_mx_sf_gather(const uint8_t* x_sf, const int32_t* src_rows,

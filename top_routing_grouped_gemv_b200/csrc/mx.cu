@@ -1,6 +1,8 @@
 // MX block scales: from the row-major E8M0 scale matrices the caller holds
 // to the 512-byte atoms the block-scaled grouped GEMM reads (layout in
-// kernels.h), and the row gather of scales that goes with the permute.
+// kernels.h), and the row gather of scales that goes with the permute; the
+// transposition of fp32 group / block weight scales for the group-scaled
+// GEMM (quant modes 4 and 5).
 //
 // Quant mode 6 ("mx") of the Ascend grouped-matmul page
 // ("aclnnQuantGroupedMatMulAlltoAllv", parameter section, quant-mode
@@ -170,6 +172,19 @@ __global__ void mx_sf_gather_kernel(const uint8_t* __restrict__ x_sf, const int3
   }
 }
 
+__global__ void group_scales_t_kernel(const float* __restrict__ src, int groups, int rows, int ng,
+                                      float* __restrict__ dst) {
+  const long long total = static_cast<long long>(groups) * rows * ng;
+  for (long long t = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; t < total;
+       t += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int n = static_cast<int>(t % rows);          // destination order: (g, kb, n)
+    const long long gk = t / rows;
+    const int kb = static_cast<int>(gk % ng);
+    const long long g = gk / ng;
+    dst[t] = src[(g * rows + n) * ng + kb];
+  }
+}
+
 int grid_for(long long work, int threads) {
   const long long b = (work + threads - 1) / threads;
   const long long cap = 8LL * device_sm_count();
@@ -184,6 +199,14 @@ cudaError_t launch_mx_weight_sf(const uint8_t* w_sf, int groups, int n_out, int 
   const long long work = static_cast<long long>(groups) * ((n_out + kTcBlockN - 1) / kTcBlockN) *
                          kTcBlockN * mx_num_kb(kdim);
   mx_weight_sf_kernel<<<grid_for(work, 256), 256, 0, stream>>>(w_sf, groups, n_out, kdim, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_group_scales_t(const float* src, int groups, int rows, int ng, float* dst,
+                                  cudaStream_t stream) {
+  if (groups < 1 || rows < 1 || ng < 1) return cudaErrorInvalidValue;
+  const long long work = static_cast<long long>(groups) * rows * ng;
+  group_scales_t_kernel<<<grid_for(work, 256), 256, 0, stream>>>(src, groups, rows, ng, dst);
   return cudaGetLastError();
 }
 
