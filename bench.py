@@ -190,11 +190,18 @@ def oracle_tokens(inp, tok):
     import numpy as np
     import oracle
     cfg = inp.cfg
-    if cfg.quant == "mx":
+    if cfg.quant in ("mx", "group", "block"):
         rows = np.repeat(np.asarray(tok), cfg.K)
         row_e = inp.ids.numpy()[tok].reshape(-1).astype(np.int32)
-        return oracle.expert_rows_mx(row_e, inp.x.numpy()[rows], inp.x_sf.numpy()[rows], inp.w1,
-                                     inp.w_sf)
+        if cfg.quant == "mx":
+            return oracle.expert_rows_mx(row_e, inp.x.numpy()[rows], inp.x_sf.numpy()[rows],
+                                         inp.w1, inp.w_sf)
+        ws = inp.w_gs.numpy().astype(np.float64)
+        if cfg.quant == "block":
+            ws = oracle.block_to_group_scales(ws, cfg.F)
+        return oracle.expert_rows_kscaled(row_e, inp.x.numpy()[rows], oracle.E4M3, inp.w1,
+                                          oracle.E4M3, ws,
+                                          x_group_scales=inp.x_gs.numpy()[rows])
     gm = 0 if cfg.routing == "given" else 1   # given routing: the pure unpermute
     return oracle.forward_tokens(inp, tok, gates_mode=gm)
 
@@ -282,8 +289,9 @@ def main():
     cfg = synth.CONFIGS[args.workload]
     inp = synth.make_inputs(cfg)
     w = {"w1": inp.w1.cuda(), "w_scale": inp.w_scale}
+    gkey = "w_block_scales" if cfg.quant == "block" else "w_group_scales"
     for k, t in (("w3", inp.w3), ("w2", inp.w2), ("w_r", inp.w_r), ("bias", inp.bias),
-                 ("w_mx_scales", inp.w_sf)):
+                 ("w_mx_scales", inp.w_sf), (gkey, inp.w_gs)):
         if t is not None:
             w[k] = t.cuda()
     plan = moe.Plan(cfg.N, cfg.d, cfg.E, cfg.K, cfg.F, cfg.dtype, cfg.act, w)
@@ -294,9 +302,19 @@ def main():
     stream = torch.cuda.current_stream()
     given = cfg.routing == "given"
     mx = cfg.quant == "mx"
+    gsq = cfg.quant in ("group", "block")
     shared = cfg.shared is not None
     ysh = xsf = None
-    if given and mx:
+    if given and gsq:
+        # group / block-scaled grouped-matmul layer: the caller's routing and
+        # per-token-and-group activation scales, unpermute in the GEMM's stores
+        ids = inp.ids.cuda()
+        xsf = inp.x_gs.cuda()
+        y = torch.empty(cfg.N * cfg.K, cfg.d_out, dtype=ydt, device="cuda")
+
+        def step():
+            plan.forward_routed_group_scales(x, ids, None, y, ws, x_group_scales=xsf)
+    elif given and mx:
         # MX grouped-matmul layer: the caller's routing and block scales, the
         # pure unpermute done by the GEMM's stores
         ids = inp.ids.cuda()
@@ -376,8 +394,8 @@ def main():
         # expert), and copies the results back (no host-buffer entry point
         # for these layers: the copies are queued on the compute stream)
         ins = [(x, inp.x.clone().pin_memory()), (ids, inp.ids.clone().pin_memory())]
-        if mx:
-            ins.append((xsf, inp.x_sf.clone().pin_memory()))
+        if mx or gsq:
+            ins.append((xsf, (inp.x_sf if mx else inp.x_gs).clone().pin_memory()))
         outs = [(y, torch.empty(tuple(y.shape), dtype=y.dtype).pin_memory())]
         if shared:
             outs.append((ysh, torch.empty(tuple(ysh.shape), dtype=ysh.dtype).pin_memory()))
@@ -407,7 +425,8 @@ def main():
                "h2d_bytes_per_step": sum(h.numel() * h.element_size() for _, h in ins),
                "d2h_bytes_per_step": sum(h.numel() * h.element_size() for _, h in outs),
                "steps": n_e2e,
-               "api": ("moe_forward_routed_mx" if mx else "moe_forward_routed_shared")
+               "api": ("moe_forward_routed_mx" if mx else "moe_forward_routed_group_scales" if gsq
+                       else "moe_forward_routed_shared")
                       + " with pinned host copies on the same stream"}
     elif not args.no_e2e:
         xh = [inp.x.clone().pin_memory() for _ in range(2)]
@@ -441,7 +460,8 @@ def main():
     R = cfg.N * cfg.K
     f1, f2 = gemm_flops(cfg, R)
     k1 = "ffn1_swiglu_tc" if cfg.act == "swiglu" else (
-        ("gmm_mx_tc" if mx else "gmm_tc") if cfg.act == "none" else "ffn1_simt_f32")
+        ("gmm_mx_tc" if mx else f"gmm_{cfg.quant}_tc" if gsq else "gmm_tc")
+        if cfg.act == "none" else "ffn1_simt_f32")
     stage_us = {k: 1e3 * statistics.mean(v) for k, v in per_kernel.items()}
     # the sustained (power-capped) peak applies to a kernel timed inside a long
     # loop or while the power cap throttles the clock; the burst one otherwise
@@ -487,6 +507,8 @@ def main():
                        "F": cfg.F, "act": cfg.act,
                        "router": ("given (top-K of seeded iid logits), OCP MXFP8 block scales "
                                   "(E8M0 per 32 elements)" if mx else
+                                  f"given (top-K of seeded iid logits), fp32 {cfg.quant} scales "
+                                  "(128-element groups of K)" if gsq else
                                   "given (top-K of seeded iid logits), shared expert "
                                   f"{cfg.shared[0]}x{cfg.shared[1]} on a forked stream")
                                  if given else "fp32",

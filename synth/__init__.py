@@ -18,8 +18,8 @@ Workloads (the five shapes the layer is measured and checked on):
   scales (OCP MXFP8: one E8M0 scale per 32 consecutive elements along H1)
 * ``e4m3blk_n8192_h7168_e256_k8_n2048_gmm``  the same grouped matmul with fp32 scales per
   128 x 128 weight block and per token and 128-element group of the activations
-* ``e4m3_n2048_h7168_e64_k8_n2048_gmm``, ``e4m3mx_n2048_h7168_e64_k8_n2048_gmm``
-  reduced copies of the two fp8 layers for kernel profiling
+* ``e4m3_n2048_h7168_e64_k8_n2048_gmm``, ``e4m3mx_n2048_h7168_e64_k8_n2048_gmm``,
+  ``e4m3blk_n2048_h7168_e64_k8_n2048_gmm`` reduced copies of the fp8 layers for kernel profiling
 
 Value recipe: x ~ N(0,1); router and expert weights ~ N(0, 1/fan_in)
 (fan_in = d for the router and the first FFN matrices, F for the second);
@@ -126,6 +126,8 @@ FP8_GMM_PROFILE = _reg(MoEConfig("e4m3_n2048_h7168_e64_k8_n2048_gmm", DTYPE_E4M3
                                  2048, ACT_NONE, index=6, shared=(7168, 2048), routing="given"))
 MX_GMM_PROFILE = _reg(MoEConfig("e4m3mx_n2048_h7168_e64_k8_n2048_gmm", DTYPE_E4M3, 2048, 7168, 64,
                                 8, 2048, ACT_NONE, index=7, routing="given", quant="mx"))
+BLOCK_GMM_PROFILE = _reg(MoEConfig("e4m3blk_n2048_h7168_e64_k8_n2048_gmm", DTYPE_E4M3, 2048, 7168,
+                                   64, 8, 2048, ACT_NONE, index=9, routing="given", quant="block"))
 
 
 # ----------------------------------------------------------------------------

@@ -256,3 +256,35 @@ def test_e4m3_mx_gmm_unpermute_n8192_h7168_e256_k8_n2048():
     tr = np.repeat(tok, c.K)
     yref = oracle.expert_rows_mx(row_e, inp.x.numpy()[tr], xs[tr], inp.w1, inp.w_sf)
     assert rel_err(f64(y[torch.from_numpy(rows_tok).long().cuda()]), yref) <= 1e-2
+
+
+def test_e4m3_block_scales_gmm_unpermute_n8192_h7168_e256_k8_n2048():
+    """The grouped matmul with fp32 scales per 128 x 128 weight block and per
+    token and 128-element group (quant mode 5) at full size: sampled rows of
+    the stage call against the oracle, the fused call (unpermute by the
+    GEMM's stores) equal to the stage composition bit for bit."""
+    import top_routing_grouped_gemv_b200 as moe
+    c = synth.BLOCK_GMM
+    inp = synth.make_inputs(c)
+    R = c.N * c.K
+    w = {"w1": inp.w1.cuda(), "w_block_scales": inp.w_gs.cuda()}
+    plan = moe.Plan(c.N, c.d, c.E, c.K, c.F, "e4m3", "none", w)
+    ws = plan.new_workspace()
+    xg = inp.x_gs.numpy()
+    rc, ro, rp, rs, rx = oracle.permute(inp.ids.numpy(), c.E, inp.x)
+    y_perm = torch.empty(R, c.F, dtype=torch.bfloat16, device="cuda")
+    plan.grouped_ffn_group_scales(torch.from_numpy(rx).cuda(), torch.from_numpy(ro).cuda(), y_perm,
+                                  ws, x_group_scales=torch.from_numpy(xg[rs]).cuda())
+    assert plan.read_device_status(ws) == 0
+    rows = sample_rows(ro, R, 48, 13)
+    row_e = (np.searchsorted(ro, rows, side="right") - 1).astype(np.int32)
+    wfull = oracle.block_to_group_scales(inp.w_gs.numpy(), c.F)
+    ref = oracle.expert_rows_kscaled(row_e, rx[rows], oracle.E4M3, inp.w1, oracle.E4M3, wfull,
+                                     x_group_scales=xg[rs[rows]])
+    assert rel_err(f64(y_perm[torch.from_numpy(rows).long().cuda()]), ref) <= 1e-2
+    y = torch.empty(R, c.F, dtype=torch.bfloat16, device="cuda")
+    plan.forward_routed_group_scales(inp.x.cuda(), inp.ids.cuda(), None, y, ws,
+                                     x_group_scales=inp.x_gs.cuda())
+    assert plan.read_device_status(ws) == 0
+    yp = y_perm.cpu().view(torch.int16).numpy()
+    assert np.array_equal(y.cpu().view(torch.int16).numpy(), yp[rp])

@@ -61,12 +61,16 @@ constexpr int BN = kTcBlockN;     // 256 accumulator columns per tile
 constexpr int ROWB = 128;         // bytes of K per row per stage (one swizzle atom)
 constexpr int A_BYTES = BM * ROWB;
 // producer warp, MMA warp, epilogue warps: four (one per TMEM lane
-// quadrant), eight for the group-scaled epilogues (two per quadrant, 128
-// columns each, whose fp32 sums live in registers)
-constexpr int kGsEpiWarps = 8;
+// quadrant); for the group-scaled epilogues, whose fp32 sums live in
+// registers, eight with block scales (two per quadrant, 128 columns each)
+// and sixteen with per-column scales (four per quadrant, 64 columns each:
+// twice the warps to overlap the per-column work; measured 4.3 -> 3.4 ms on
+// the full fp8 workload, while block scales ran 1.6 -> 2.6 ms with sixteen)
+template <int kEpi>
+constexpr int gs_epi_warps() { return kEpi == kEpiGroupScale ? 16 : 8; }
 template <int kEpi>
 constexpr int threads_of() {
-  return kEpi == kEpiGroupScale || kEpi == kEpiBlockScale ? 32 * (2 + kGsEpiWarps) : 192;
+  return kEpi == kEpiGroupScale || kEpi == kEpiBlockScale ? 32 * (2 + gs_epi_warps<kEpi>()) : 192;
 }
 constexpr uint32_t kTmemCols = 2 * BN;
 constexpr int kMaxGroups = 256;
@@ -202,7 +206,7 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar(Gm::kBarTFull + a), 1);
-      mbar_init(bar(Gm::kBarTEmpty + a), kGs ? kGsEpiWarps : kPair ? 8 : 4);
+      mbar_init(bar(Gm::kBarTEmpty + a), kGs ? gs_epi_warps<kEpi>() : kPair ? 8 : 4);
     }
     mbar_init(bar(Gm::kBarDrain), 1);
     *abort_flag = 0;
@@ -386,11 +390,11 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5 of every CTA; 2..17 group-scaled) ----------------
+    // ---------------- epilogue (warps 2..5; 2..9 or 2..17 group-scaled) ----------------
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     int i = 0;
     if constexpr (kGs) {
-      constexpr int kCols = BN / (kGsEpiWarps / 4);  // columns of this warp
+      constexpr int kCols = BN / (gs_epi_warps<kEpi>() / 4);  // columns of this warp
       const int half = (warp - 2) >> 2;               // its column slice
       const int nblk = (args.n_out + 127) / 128;
       uint32_t j = 0;
@@ -406,17 +410,36 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
         float sum[kCols];
 #pragma unroll
         for (int cc = 0; cc < kCols; ++cc) sum[cc] = 0.f;
+        // the stage's row scale (and block scale) are loaded one stage ahead,
+        // so their latency is not on the path from TFull to TEmpty
+        const float* xrow = valid && args.xgs != nullptr ? args.xgs + srow * num_kb : nullptr;
+        const float* wblk = args.wgs + static_cast<long long>(c.g) * num_kb * nblk + col0 / 128;
+        float sx_next = xrow ? xrow[0] : 1.f;
+        float wb_next = kEpi == kEpiBlockScale ? wblk[0] : 0.f;
+        // per-column scales of the stage: four per lane (128 columns from col0)
+        const float4* wcol = reinterpret_cast<const float4*>(
+                                 args.wgs + static_cast<long long>(c.g) * num_kb * args.n_out + col0) +
+                             lane;
+        float4 wc_next = kEpi == kEpiGroupScale ? __ldg(wcol) : make_float4(0.f, 0.f, 0.f, 0.f);
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb, ++j) {
           const uint32_t a = j & 1u, aph = (j >> 1) & 1u;
+          const float sx = sx_next, wb = wb_next;
+          const float4 wc = wc_next;
+          if (kb + 1 < num_kb) {
+            if (xrow) sx_next = xrow[kb + 1];
+            if (kEpi == kEpiBlockScale) wb_next = wblk[static_cast<long long>(kb + 1) * nblk];
+            if (kEpi == kEpiGroupScale)
+              wc_next = __ldg(reinterpret_cast<const float4*>(
+                                  reinterpret_cast<const float*>(wcol) +
+                                  static_cast<long long>(kb + 1) * args.n_out));
+          }
           ok = __shfl_sync(0xffffffffu, mbar_wait(bar(Gm::kBarTFull + a), aph, abort_flag), 0);
           if (!ok) break;
           tc_fence_after();
-          const float sx = valid && args.xgs != nullptr ? args.xgs[srow * num_kb + kb] : 1.f;
-          const long long wk = static_cast<long long>(c.g) * num_kb + kb;
           if constexpr (kEpi == kEpiBlockScale) {
             // one 128 x 128 weight block covers this warp's columns
-            const float f = sx * args.wgs[wk * nblk + col0 / 128];
+            const float f = sx * wb;
 #pragma unroll
             for (int cc = 0; cc < kCols; cc += 16) {
               uint32_t v[16];
@@ -427,9 +450,11 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
               for (int jj = 0; jj < 16; ++jj) sum[cc + jj] = fmaf(__uint_as_float(v[jj]), f, sum[cc + jj]);
             }
           } else {
-            // per-column scales: eight columns at a time (registers: the 128
-            // sums stay live across the stages)
-            const float4* w4 = reinterpret_cast<const float4*>(args.wgs + wk * args.n_out + col0);
+            // per-column scales: lane l holds those of columns 4l..4l+3 from
+            // this warp's first column (the warp uses the first kCols / 4
+            // lanes'), loaded a stage ahead; each column takes its scale
+            // from that lane by a shuffle (sx is this lane's own row's)
+            const float4 w = wc;
 #pragma unroll
             for (int cc = 0; cc < kCols; cc += 8) {
               uint32_t v[8];
@@ -437,12 +462,11 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
               tmem_ld8(tq + a * BN + cc, v);
               tmem_ld_wait();
 #pragma unroll
-              for (int jj = 0; jj < 8; jj += 4) {
-                const float4 w = __ldg(w4 + (cc + jj) / 4);
-                sum[cc + jj] = fmaf(__uint_as_float(v[jj]), sx * w.x, sum[cc + jj]);
-                sum[cc + jj + 1] = fmaf(__uint_as_float(v[jj + 1]), sx * w.y, sum[cc + jj + 1]);
-                sum[cc + jj + 2] = fmaf(__uint_as_float(v[jj + 2]), sx * w.z, sum[cc + jj + 2]);
-                sum[cc + jj + 3] = fmaf(__uint_as_float(v[jj + 3]), sx * w.w, sum[cc + jj + 3]);
+              for (int jj = 0; jj < 8; ++jj) {
+                const int col = cc + jj;
+                const float part = (col & 3) == 0 ? w.x : (col & 3) == 1 ? w.y : (col & 3) == 2 ? w.z : w.w;
+                const float f = __shfl_sync(0xffffffffu, part, col >> 2) * sx;
+                sum[col] = fmaf(__uint_as_float(v[jj]), f, sum[col]);
               }
             }
           }
