@@ -219,13 +219,17 @@ cudaError_t launch_mx_act_sf(const uint8_t* x_sf, const int32_t* src_rows, const
   // one block per padded tile; at most rows_upper / 128 + groups tiles exist
   const int tiles = rows_upper / kTcBlockM + groups;
   const size_t smem = static_cast<size_t>(kTcBlockM) * mx_num_kb(kdim) * 4;
-  static bool configured = false;
-  if (!configured) {
+  // the shared-memory opt-in is a per-device function attribute
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(mx_act_sf_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kTcBlockM * mx_num_kb(kMxMaxKdim) * 4);
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured[dev] = true;
   }
   return launch_pdl(mx_act_sf_kernel, dim3(tiles), dim3(kActThreads), smem, stream, x_sf, src_rows,
                     offsets, groups, kdim, out);
