@@ -69,7 +69,38 @@ combine_kernel(const uint4* __restrict__ y_perm, int row_vecs, const int32_t* __
     g[j] = __shfl_sync(0xffffffffu, mine_g, j);
   }
   constexpr int n = Vec<T>::n;
-  for (int v = sub * 32 + lane; v < row_vecs; v += 32 * WPT) {
+  constexpr int STEP = 32 * WPT;
+  // several vectors of the row per lane at once (about eight 16-byte loads
+  // in flight per lane: KMAX rows x kBatch vectors)
+  constexpr int kBatch = KMAX <= 2 ? 4 : KMAX <= 4 ? 2 : 1;
+  int v = sub * 32 + lane;
+  if constexpr (kBatch > 1) {
+    for (; v + (kBatch - 1) * STEP < row_vecs; v += kBatch * STEP) {
+      uint4 raw[kBatch][KMAX];
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b)
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+          if (j < K && p[j] >= 0) raw[b][j] = y_perm[(long long)p[j] * row_vecs + v + b * STEP];
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        float acc[n];
+#pragma unroll
+        for (int i = 0; i < n; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          if (j < K && p[j] >= 0) {
+            float f[n];
+            Vec<T>::load(raw[b][j], f);
+#pragma unroll
+            for (int i = 0; i < n; ++i) acc[i] = fmaf(g[j], f[i], acc[i]);
+          }
+        }
+        y[(long long)t * row_vecs + v + b * STEP] = Vec<T>::store(acc);
+      }
+    }
+  }
+  for (; v < row_vecs; v += STEP) {
     float acc[n];
 #pragma unroll
     for (int i = 0; i < n; ++i) acc[i] = 0.f;

@@ -240,6 +240,19 @@ permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* 
   const uint4* srow = x + (long long)t * row_vecs;
   constexpr int STEP = 32 * WPT;
   int v = sub * 32 + lane;
+  // eight 16-byte loads in flight per lane where the row allows, then four
+  for (; v + 7 * STEP < row_vecs; v += 8 * STEP) {
+    uint4 a[8];
+#pragma unroll
+    for (int b = 0; b < 8; ++b) a[b] = srow[v + b * STEP];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j >= K || p[j] < 0) continue;
+      uint4* drow = x_perm + (long long)p[j] * row_vecs;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) drow[v + b * STEP] = a[b];
+    }
+  }
   for (; v + 3 * STEP < row_vecs; v += 4 * STEP) {
     const uint4 a0 = srow[v], a1 = srow[v + STEP], a2 = srow[v + 2 * STEP], a3 = srow[v + 3 * STEP];
 #pragma unroll
