@@ -74,7 +74,7 @@ def _free_port():
     return port
 
 
-def _worker(rank, world, port, name, q):
+def _worker(rank, world, port, name, q, host_exchange=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import datetime
     dist.init_process_group("gloo", rank=rank, world_size=world,
@@ -84,7 +84,8 @@ def _worker(rank, world, port, name, q):
         inp = synth.make_inputs(cfg, seed=99)
         n_loc = cfg.N // world
         x = inp.x[rank * n_loc:(rank + 1) * n_loc].contiguous()
-        layer = ExpertParallelMoE(OracleStages(inp, rank, world, n_loc), cfg.E, cfg.K)
+        layer = ExpertParallelMoE(OracleStages(inp, rank, world, n_loc), cfg.E, cfg.K,
+                                  host_exchange=host_exchange)
         y = layer.forward(x).numpy()
         ref, _, _, _ = oracle.forward_tokens(inp, np.arange(rank * n_loc, (rank + 1) * n_loc))
         q.put((rank, float(np.abs(y - ref).max()), float(np.abs(ref).max())))
@@ -93,13 +94,15 @@ def _worker(rank, world, port, name, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("world,host_exchange", [(2, False), (4, False), (2, True)])
 @pytest.mark.parametrize("name", list(CFGS))
-def test_expert_parallel_matches_single_rank_oracle(name, world):
+def test_expert_parallel_matches_single_rank_oracle(name, world, host_exchange):
+    """host_exchange: the rows travel as byte views of host copies."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, name, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, name, q, host_exchange))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:

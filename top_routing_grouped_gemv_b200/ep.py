@@ -23,8 +23,10 @@ single-GPU layer's bit for bit.
 
 The per-step work is done by a `stages` object (the library's kernels on the
 GPU: `LibraryStages`); the exchanges use torch.distributed (NCCL on GPUs).
-Without an initialized process group the layer runs on one rank with no
-exchange.
+With `host_exchange=True` the exchanged tensors travel as host copies (byte
+views of the rows), for process groups whose backend moves only host memory
+(gloo).  Without an initialized process group the layer runs on one rank
+with no exchange.
 """
 from __future__ import annotations
 
@@ -121,8 +123,24 @@ class LibraryStages:
 class ExpertParallelMoE:
     """The expert-parallel layer on this rank (see the module docstring)."""
 
-    def __init__(self, stages, E: int, K: int, group=None):
+    def __init__(self, stages, E: int, K: int, group=None, host_exchange: bool = False):
         self.stages, self.E, self.K, self.group = stages, E, K, group
+        self.host_exchange = host_exchange
+
+    def _all_to_all(self, dist, t, out_rows, out_splits=None, in_splits=None):
+        """all_to_all_single of the rows of t (variable splits if given)."""
+        shape = (out_rows,) + tuple(t.shape[1:])
+        if not self.host_exchange:
+            out = t.new_empty(shape)
+            dist.all_to_all_single(out, t.contiguous(), out_splits, in_splits, group=self.group)
+            return out
+        # host copies, rows as bytes (the backend may not know the dtype)
+        src = t.contiguous().cpu()
+        src_b = src.view(torch.uint8).reshape(src.shape[0], -1) if src.dim() > 1 else src
+        out_b = torch.empty((out_rows,) + tuple(src_b.shape[1:]), dtype=src_b.dtype)
+        dist.all_to_all_single(out_b, src_b, out_splits, in_splits, group=self.group)
+        out = out_b.view(t.dtype).reshape(shape) if src.dim() > 1 else out_b
+        return out.to(t.device)
 
     def _world(self):
         dist = _dist()
@@ -142,8 +160,7 @@ class ExpertParallelMoE:
         # per-expert row counts: block q of my counts goes to rank q
         send_counts = counts.to(torch.int64).reshape(G, E_loc)
         if dist is not None:
-            recv_counts = torch.empty_like(send_counts)
-            dist.all_to_all_single(recv_counts, send_counts, group=self.group)
+            recv_counts = self._all_to_all(dist, send_counts, G)
         else:
             recv_counts = send_counts.clone()
         send_h, recv_h = send_counts.cpu(), recv_counts.cpu()
@@ -153,9 +170,7 @@ class ExpertParallelMoE:
 
         # dispatch: the rows, source-major, expert-minor within each source
         if dist is not None:
-            x_recv = x_perm.new_empty((n_recv,) + tuple(x_perm.shape[1:]))
-            dist.all_to_all_single(x_recv, x_perm[:n_send].contiguous(), recv_rows, send_rows,
-                                   group=self.group)
+            x_recv = self._all_to_all(dist, x_perm[:n_send], n_recv, recv_rows, send_rows)
         else:
             x_recv = x_perm[:n_send]
         # regroup by local expert, run the local experts, restore the order
@@ -168,9 +183,7 @@ class ExpertParallelMoE:
 
         # return the results: the dispatch splits swapped
         if dist is not None:
-            y_perm = y_recv.new_empty((n_send,) + tuple(y_recv.shape[1:]))
-            dist.all_to_all_single(y_perm, y_recv.contiguous(), send_rows, recv_rows,
-                                   group=self.group)
+            y_perm = self._all_to_all(dist, y_recv, n_send, send_rows, recv_rows)
         else:
             y_perm = y_recv
         return st.combine(y_perm, pos, gates)
