@@ -21,6 +21,10 @@ CFGS = {
     "bf16_zipf_k4": synth.MoEConfig("ep_zipf", "bf16", 384, 256, 16, 4, 256, "swiglu",
                                     zipf_bias=1.2),
     "f32_relu": synth.MoEConfig("ep_f32", "f32", 192, 128, 8, 2, 256, "relu"),
+    # a router bias of 50 ln(1/rank) sends every token to experts 0 and 1:
+    # rank 1 (experts 2, 3) receives no rows and returns none
+    "bf16_rank_empty": synth.MoEConfig("ep_empty", "bf16", 128, 256, 4, 2, 256, "swiglu",
+                                       zipf_bias=50.0),
 }
 
 

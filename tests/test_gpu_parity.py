@@ -907,3 +907,30 @@ def test_group_scales_stage_call_equals_fused(name, quant):
                                      x_group_scales=torch.from_numpy(xs).cuda())
     yp = y_perm.cpu().view(torch.int16).numpy()
     assert np.array_equal(y.cpu().view(torch.int16).numpy(), yp[rp])
+
+
+@pytest.mark.parametrize("name", ["bf16_swiglu_ragged", "f32_relu_n256", "e4m3_gmm"])
+def test_stage_calls_with_zero_rows(name):
+    """n = 0 (an expert-parallel rank that receives no rows): the row-count
+    stage calls succeed, give all-zero counts and offsets and write nothing."""
+    inp, plan, w = case(name)
+    c = inp.cfg
+    ws = plan.new_workspace()
+    i32 = dict(dtype=torch.int32, device="cuda")
+    counts = torch.full((c.E,), -7, **i32)
+    offsets = torch.full((c.E + 1,), -7, **i32)
+    pos = torch.full((c.N * c.K,), -7, **i32)
+    src = torch.full((c.N * c.K,), -7, **i32)
+    xdt = inp.x.dtype
+    x_perm = torch.zeros(c.N * c.K, c.d, dtype=xdt, device="cuda")
+    plan.permute(inp.x.cuda(), torch.zeros(c.N, c.K, **i32), counts, offsets, pos, src, x_perm, ws,
+                 n=0)
+    assert plan.read_device_status(ws) == 0
+    assert not counts.cpu().any() and not offsets.cpu().any()
+    ydt = torch.float32 if c.dtype == "f32" else torch.bfloat16
+    y_perm = torch.full((c.N * c.K, c.d_out), 3.0, dtype=ydt, device="cuda")
+    plan.grouped_ffn(x_perm, offsets, y_perm, ws, n=0, x_scale=inp.x_scale)
+    y = torch.full((c.N, c.d_out), 5.0, dtype=ydt, device="cuda")
+    plan.unpermute_combine(y_perm, pos, torch.ones(c.N, c.K, device="cuda"), y, ws, n=0)
+    assert plan.read_device_status(ws) == 0
+    assert bool((y_perm == 3.0).all()) and bool((y == 5.0).all())

@@ -252,7 +252,9 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
   // the down GEMM was 6-9 % faster paired (measured on one B200).
   const bool pair = R >= 512 * d.E;
   const bool pair_swiglu = R >= 2048 * d.E;
-  if (!encode_kmajor_map(&a.tmA, x_perm, p->ex, R, d.d, kTcBlockM)) return MOE_ERR_CUDA;
+  // with no rows the GEMM schedules no tile; a map of one row keeps it valid
+  const int map_rows = R > 0 ? R : 1;
+  if (!encode_kmajor_map(&a.tmA, x_perm, p->ex, map_rows, d.d, kTcBlockM)) return MOE_ERR_CUDA;
   if (d.act == MOE_ACT_NONE) {
     a.tmB0 = pair ? p->tmW1h : p->tmW1;
     a.tmB1 = a.tmB0;
@@ -287,7 +289,7 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
   mark(p, s, "ffn1_swiglu_tc");
   if (launch_gemm_tc(a, d.dtype, kEpiSwiglu, R, pair_swiglu, s) != cudaSuccess) return MOE_ERR_CUDA;
   TcGemmArgs b = a;
-  if (!encode_kmajor_map(&b.tmA, h, p->eh, R, d.F, kTcBlockM)) return MOE_ERR_CUDA;
+  if (!encode_kmajor_map(&b.tmA, h, p->eh, map_rows, d.F, kTcBlockM)) return MOE_ERR_CUDA;
   b.tmB0 = pair ? p->tmW2h : p->tmW2;
   b.tmB1 = b.tmB0;
   b.kdim = d.F;

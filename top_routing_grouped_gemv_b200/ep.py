@@ -97,18 +97,25 @@ class LibraryStages:
         return self.counts, self.offsets, self.pos, self.x_perm
 
     def local_permute(self, n, x_recv, ids_recv):
+        if n == 0:  # nothing received: no launches (an empty tensor may have no address)
+            self.offsets_l.zero_()
+            return self.offsets_l, self.pos_l[:0], self.x_sorted[:0]
         self.loc.permute(x_recv, ids_recv, self.counts_l, self.offsets_l, self.pos_l, self.src_l,
                          self.x_sorted, self.ws_l, n=n)
         return self.offsets_l, self.pos_l, self.x_sorted
 
     def local_ffn(self, n, x_sorted, offsets):
+        if n == 0:
+            return self.y_sorted[:0]
         self.loc.grouped_ffn(x_sorted, offsets, self.y_sorted, self.ws_l, n=n)
         return self.y_sorted
 
     def local_unpermute(self, n, y_sorted, pos):
-        y_recv = torch.empty(max(n, 1), self.d_out, dtype=self.ydt, device=y_sorted.device)
+        if n == 0:
+            return torch.empty(0, self.d_out, dtype=self.ydt, device=y_sorted.device)
+        y_recv = torch.empty(n, self.d_out, dtype=self.ydt, device=y_sorted.device)
         self.loc.unpermute_combine(y_sorted, pos, None, y_recv, self.ws_l, n=n)
-        return y_recv[:n]
+        return y_recv
 
     def combine(self, y_perm, pos, gates):
         y = torch.empty(self.N, self.d_out, dtype=self.ydt, device=y_perm.device)
@@ -136,11 +143,13 @@ class ExpertParallelMoE:
             return out
         # host copies, rows as bytes (the backend may not know the dtype)
         src = t.contiguous().cpu()
-        src_b = src.view(torch.uint8).reshape(src.shape[0], -1) if src.dim() > 1 else src
-        out_b = torch.empty((out_rows,) + tuple(src_b.shape[1:]), dtype=src_b.dtype)
+        row_bytes = t.element_size()
+        for s in t.shape[1:]:
+            row_bytes *= s
+        src_b = src.view(torch.uint8).reshape(src.shape[0], row_bytes)
+        out_b = torch.empty((out_rows, row_bytes), dtype=torch.uint8)
         dist.all_to_all_single(out_b, src_b, out_splits, in_splits, group=self.group)
-        out = out_b.view(t.dtype).reshape(shape) if src.dim() > 1 else out_b
-        return out.to(t.device)
+        return out_b.view(t.dtype).reshape(shape).to(t.device)
 
     def _world(self):
         dist = _dist()
