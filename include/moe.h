@@ -138,10 +138,12 @@ typedef struct {
   const void* w2;           /* (E, d, F) for RELU / SWIGLU, else NULL */
   float w_scale;            /* per-tensor weight scale (gmmWeightScale), e4m3 PER_TENSOR */
   const float* w_channel_scales; /* (E, F) fp32 per output channel, e4m3 PER_CHANNEL, else NULL */
-  const uint8_t* w_mx_scales;    /* (E, F, d/32) E8M0 of w1, MOE_QUANT_MX, else NULL; read
-                                    once by moe_plan_create (may be freed afterwards) */
+  const uint8_t* w_mx_scales;    /* (E, F, d/32) E8M0 of w1, MOE_QUANT_MX, else NULL; device
+                                    memory (MOE_ERR_INVALID_ARG otherwise), read once by
+                                    moe_plan_create (may be freed afterwards) */
   const float* w_group_scales;   /* fp32 of w1: (E, F, d/128) PER_GROUP, (E, ceil(F/128),
-                                    d/128) PER_BLOCK, else NULL; read once by moe_plan_create */
+                                    d/128) PER_BLOCK, else NULL; device memory, read once by
+                                    moe_plan_create */
 } moe_layer_weights;
 
 typedef struct moe_plan_s* moe_plan;

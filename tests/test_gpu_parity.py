@@ -934,3 +934,21 @@ def test_stage_calls_with_zero_rows(name):
     plan.unpermute_combine(y_perm, pos, torch.ones(c.N, c.K, device="cuda"), y, ws, n=0)
     assert plan.read_device_status(ws) == 0
     assert bool((y_perm == 3.0).all()) and bool((y == 5.0).all())
+
+
+def test_plan_refuses_host_scale_tables():
+    """The plan-time kernels read the MX and group scale tables: a host
+    pointer is refused with MOE_ERR_INVALID_ARG before any launch."""
+    import top_routing_grouped_gemv_b200 as moe
+    c = MX["mx_sparse"]
+    inp = synth.make_inputs(c, 1)
+    with pytest.raises(moe.MoEError) as e:
+        moe.Plan(c.N, c.d, c.E, c.K, c.F, "e4m3", "none",
+                 {"w1": inp.w1.cuda(), "w_mx_scales": inp.w_sf})   # host tensor
+    assert e.value.code == 1
+    g = GS["gs_sparse"].scaled(quant="block")
+    ginp = synth.make_inputs(g, 1)
+    with pytest.raises(moe.MoEError) as e:
+        moe.Plan(g.N, g.d, g.E, g.K, g.F, "e4m3", "none",
+                 {"w1": ginp.w1.cuda(), "w_block_scales": ginp.w_gs})
+    assert e.value.code == 1

@@ -64,6 +64,17 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Device or managed memory (a kernel may read it); host or unknown pointers
+// are refused before any launch.
+bool device_accessible(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the error of an unregistered host pointer
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
 // Stage boundary marker for the optional per-kernel timing.
 void mark(moe_plan p, cudaStream_t s, const char* name_of_next) {
   if (!p->profile || p->nev >= kMaxEvents) return;
@@ -473,6 +484,12 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
       delete p;
       return MOE_ERR_CUDA;
     }
+  }
+  // the plan-time kernels below read the scale tables: refuse host pointers
+  if ((d.quant == MOE_QUANT_MX && !routing_only && !device_accessible(w->w_mx_scales)) ||
+      (gs && !routing_only && !device_accessible(w->w_group_scales))) {
+    delete p;
+    return MOE_ERR_INVALID_ARG;
   }
   if (d.quant == MOE_QUANT_MX && !routing_only) {
     // the weight scales, once, in the layout the block-scaled GEMM reads
