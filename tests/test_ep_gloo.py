@@ -48,21 +48,25 @@ class OracleStages:
     def local_ffn(self, n, x_sorted, offsets):
         row_e = np.repeat(np.arange(self.E_loc, dtype=np.int32), np.diff(offsets.numpy()))
         y = oracle.expert_rows(row_e, x_sorted.numpy(), self.dt, self.c.act, self.w1, self.w3,
-                               self.w2, self.dt)
+                               self.w2, self.dt, self.inp.x_scale, self.inp.w_scale)
         return torch.from_numpy(y)
 
     def local_unpermute(self, n, y_sorted, pos):
         return torch.from_numpy(oracle.combine(pos.numpy(), None, y_sorted.numpy(), n, 1))
 
     def combine(self, y_perm, pos, gates):
-        return torch.from_numpy(oracle.combine(pos.numpy(), gates.numpy(), y_perm.numpy(),
-                                               self.n_loc, self.c.K))
+        g = None if gates is None else gates.numpy()
+        return torch.from_numpy(oracle.combine(pos.numpy(), g, y_perm.numpy(), self.n_loc,
+                                               self.c.K))
 
 
 CFGS = {
     # fp32 (gloo moves float32 rows), ReLU and SwiGLU, uneven routing
     "relu": synth.MoEConfig("ep_relu", "f32", 96, 64, 8, 2, 48, "relu"),
     "swiglu_zipf": synth.MoEConfig("ep_sw", "f32", 120, 32, 8, 3, 40, "swiglu", zipf_bias=1.2),
+    # the fp8 single-matrix layer with given routing and the pure unpermute:
+    # fp8 codes cross the exchange
+    "e4m3_given": synth.MoEConfig("ep_e4m3", "e4m3", 96, 64, 8, 4, 48, "none", routing="given"),
 }
 
 
@@ -86,8 +90,13 @@ def _worker(rank, world, port, name, q, host_exchange=False):
         x = inp.x[rank * n_loc:(rank + 1) * n_loc].contiguous()
         layer = ExpertParallelMoE(OracleStages(inp, rank, world, n_loc), cfg.E, cfg.K,
                                   host_exchange=host_exchange)
-        y = layer.forward(x).numpy()
-        ref, _, _, _ = oracle.forward_tokens(inp, np.arange(rank * n_loc, (rank + 1) * n_loc))
+        tok = np.arange(rank * n_loc, (rank + 1) * n_loc)
+        if cfg.routing == "given":
+            y = layer.forward(x, ids=inp.ids[rank * n_loc:(rank + 1) * n_loc].contiguous()).numpy()
+            ref, _, _, _ = oracle.forward_tokens(inp, tok, gates_mode=0)
+        else:
+            y = layer.forward(x).numpy()
+            ref, _, _, _ = oracle.forward_tokens(inp, tok)
         q.put((rank, float(np.abs(y - ref).max()), float(np.abs(ref).max())))
         dist.barrier()
     finally:

@@ -25,6 +25,10 @@ CFGS = {
     # rank 1 (experts 2, 3) receives no rows and returns none
     "bf16_rank_empty": synth.MoEConfig("ep_empty", "bf16", 128, 256, 4, 2, 256, "swiglu",
                                        zipf_bias=50.0),
+    # the fp8 grouped matmul with given routing and the pure unpermute (fp8
+    # codes cross the exchange), against moe_forward_routed
+    "e4m3_given": synth.MoEConfig("ep_e4m3", "e4m3", 256, 512, 8, 4, 384, "none",
+                                  routing="given"),
 }
 
 
@@ -57,15 +61,24 @@ def _worker(rank, world, port, name, q):
         x_all = inp.x.cuda()
         x = x_all[rank * n_loc:(rank + 1) * n_loc].contiguous()
         sl = lambda t: None if t is None else t[e0:e0 + E_loc].contiguous()
-        stages = LibraryStages(n_loc, c.d, c.E, c.K, c.F, c.dtype, c.act, world, w["w_r"],
-                               sl(w["w1"]), sl(w.get("w3")), sl(w.get("w2")), bias=w.get("bias"))
-        y = ExpertParallelMoE(stages, c.E, c.K, host_exchange=True).forward(x)
-        torch.cuda.synchronize()
+        stages = LibraryStages(n_loc, c.d, c.E, c.K, c.F, c.dtype, c.act, world, w.get("w_r"),
+                               sl(w["w1"]), sl(w.get("w3")), sl(w.get("w2")), bias=w.get("bias"),
+                               w_scale=inp.w_scale, x_scale=inp.x_scale)
+        layer = ExpertParallelMoE(stages, c.E, c.K, host_exchange=True)
         # the whole layer on one GPU, all experts, this rank's tokens
         plan = moe.Plan(n_loc, c.d, c.E, c.K, c.F, c.dtype, c.act, w)
         ws = plan.new_workspace()
-        y_ref = torch.empty_like(y)
-        plan.forward(x, y_ref, ws)
+        if c.routing == "given":
+            ids = inp.ids[rank * n_loc:(rank + 1) * n_loc].contiguous().cuda()
+            y = layer.forward(x, ids=ids)
+            torch.cuda.synchronize()
+            y_ref = torch.empty_like(y)
+            plan.forward_routed(x, ids, None, y_ref, ws, x_scale=inp.x_scale)
+        else:
+            y = layer.forward(x)
+            torch.cuda.synchronize()
+            y_ref = torch.empty_like(y)
+            plan.forward(x, y_ref, ws)
         torch.cuda.synchronize()
         iv = torch.int32 if c.dtype == "f32" else torch.int16
         q.put((rank, stages.check(), plan.read_device_status(ws),

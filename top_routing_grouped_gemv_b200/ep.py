@@ -45,11 +45,14 @@ class LibraryStages:
     routing-only plan over all E experts for the rank's own tokens, and a
     plan of the rank's E_loc experts (K = 1) for the rows it receives.
 
-    ``w_r`` (d, E) fp32 and optional ``bias`` route over all experts;
-    ``w1``/``w3``/``w2`` are this rank's experts only ((E_loc, F, d) etc.)."""
+    ``w_r`` (d, E) fp32 and optional ``bias`` route over all experts (None:
+    the caller gives the routing to ExpertParallelMoE.forward);
+    ``w1``/``w3``/``w2`` are this rank's experts only ((E_loc, F, d) etc.).
+    e4m3 layers take the per-tensor ``w_scale`` and ``x_scale``: the rows
+    cross the exchange as fp8 codes."""
 
     def __init__(self, N, d, E, K, F, dtype, act, world, w_r, w1, w3=None, w2=None, bias=None,
-                 w_scale=1.0):
+                 w_scale=1.0, x_scale=1.0):
         from . import Plan
         if E % world:
             raise ValueError(f"{E} experts do not split over {world} ranks")
@@ -58,7 +61,10 @@ class LibraryStages:
         self.d_out = F if act == "none" else d
         self.dtype = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8}[dtype]
         self.ydt = torch.float32 if dtype == "f32" else torch.bfloat16
-        route_w = {"w_r": w_r}
+        self.x_scale = x_scale
+        route_w = {}
+        if w_r is not None:
+            route_w["w_r"] = w_r
         if bias is not None:
             route_w["bias"] = bias
         self.glob = Plan(N, d, E, K, F, dtype, act, route_w)
@@ -71,7 +77,7 @@ class LibraryStages:
         self.loc = Plan(self.n_max, d, self.E_loc, 1, F, dtype, act, local_w)
         self.ws_g = self.glob.new_workspace()
         self.ws_l = self.loc.new_workspace()
-        dev = w_r.device
+        dev = w1.device
         i32 = dict(dtype=torch.int32, device=dev)
         self.ids = torch.empty(N, K, **i32)
         self.gates = torch.empty(N, K, dtype=torch.float32, device=dev)
@@ -107,7 +113,7 @@ class LibraryStages:
     def local_ffn(self, n, x_sorted, offsets):
         if n == 0:
             return self.y_sorted[:0]
-        self.loc.grouped_ffn(x_sorted, offsets, self.y_sorted, self.ws_l, n=n)
+        self.loc.grouped_ffn(x_sorted, offsets, self.y_sorted, self.ws_l, n=n, x_scale=self.x_scale)
         return self.y_sorted
 
     def local_unpermute(self, n, y_sorted, pos):
@@ -118,7 +124,9 @@ class LibraryStages:
         return y_recv
 
     def combine(self, y_perm, pos, gates):
-        y = torch.empty(self.N, self.d_out, dtype=self.ydt, device=y_perm.device)
+        """gates None: the pure unpermute, y (N*K, d_out) token-major."""
+        rows = self.N if gates is not None else self.N * self.K
+        y = torch.empty(rows, self.d_out, dtype=self.ydt, device=y_perm.device)
         self.glob.unpermute_combine(y_perm, pos, gates, y, self.ws_g)
         return y
 
@@ -157,13 +165,17 @@ class ExpertParallelMoE:
             return None, 1, 0
         return dist, dist.get_world_size(self.group), dist.get_rank(self.group)
 
-    def forward(self, x):
+    def forward(self, x, ids=None, gates=None):
+        """ids (N, K) int32 / gates (N, K) fp32: routing given by the caller
+        (default: the stages' router); with given ids and no gates the result
+        is the pure unpermute (N*K, d_out), as the single-GPU routed layer."""
         st = self.stages
         dist, G, _ = self._world()
         if self.E % G:
             raise ValueError(f"{self.E} experts do not split over {G} ranks")
         E_loc = self.E // G
-        ids, gates = st.route(x)
+        if ids is None:
+            ids, gates = st.route(x)
         counts, offsets, pos, x_perm = st.permute(x, ids)
 
         # per-expert row counts: block q of my counts goes to rank q
