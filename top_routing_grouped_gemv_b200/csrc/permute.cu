@@ -113,7 +113,12 @@ permute_rank_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
 // One CTA of 1024 threads.  Thread (e, s) owns expert e and a contiguous
 // slice s of the chunks.  Afterwards chunk_counts[c][e] holds the first
 // destination row of chunk c's rows of expert e.
-__global__ void __launch_bounds__(1024)
+// At most 40 registers a thread: the 1024 threads (eight warps on each SM
+// sub-partition, 10 K of its 16 K registers) then fit on an SM beside one CTA
+// of a persistent tensor-core GEMM (the shared expert running on a forked
+// stream, two warps of 72 registers on a sub-partition), instead of waiting
+// for that GEMM to end.
+__global__ void __maxnreg__(40)
 permute_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
   griddep_trigger();  // let the next kernel of the stream start launching
