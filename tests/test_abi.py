@@ -90,3 +90,12 @@ def test_null_arguments(lib):
     assert lib.moe_workspace_size(None, None) == 1
     assert lib.moe_forward(None, None, None, None, 0, None) == 1
     assert lib.moe_last_launch_count(None) == -1
+    # the quant-mode calls refuse a null plan before anything else
+    assert lib.moe_forward_routed_mx(None, None, None, None, None, None, None, 0, None) == 1
+    assert lib.moe_permute_mx(None, None, None, None, None, None, None, None, None, None, None, 0,
+                              None) == 1
+    assert lib.moe_grouped_ffn_mx(None, None, None, None, None, None, 0, None) == 1
+    assert lib.moe_forward_routed_group_scales(None, None, 1.0, None, None, None, None, None, None,
+                                               0, None) == 1
+    assert lib.moe_grouped_ffn_group_scales(None, None, 1.0, None, None, None, None, None, 0,
+                                            None) == 1

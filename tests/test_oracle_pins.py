@@ -530,6 +530,33 @@ def test_block_scales_expand_to_channels(orc):
             assert np.array_equal(wg[e, n], wb[e, n // 128])
 
 
+def test_group_and_block_quantisers(orc):
+    """The per-group and per-block input quantisers: a group (or 128 x 128
+    block) of e4m3 values whose largest magnitude is 448, times p, gets scale
+    p (amax / 448) and its codes back exactly; an all-zero group gets scale
+    1 and zero codes; every dequantised group lies within half an e4m3 step."""
+    base = np.array([448.0, 1.0, -2.0, 0.5, -300.0, 3.5, -448.0, 0.001953125] * 16)
+    codes_ref = [orc.f64_to_e4m3(v) for v in base]
+    for p in (0.25, 1.0, 8.0):
+        c, s = synth.quantize_groups(np.stack([base * p, np.zeros(128)]))
+        assert s[0, 0] == np.float32(p) and s[1, 0] == 1.0
+        assert [int(v) for v in c[0]] == codes_ref and not c[1].any()
+    rng = np.random.default_rng(6)
+    w = rng.standard_normal((2, 200, 256)) * np.exp(rng.uniform(-4, 4, (2, 1, 1)))
+    c, s = synth.quantize_blocks(w)
+    assert c.shape == w.shape and s.shape == (2, 2, 2)
+    dec = np.array([orc.e4m3_to_f64(int(q)) for q in c.ravel()]).reshape(c.shape)
+    for e in range(2):
+        for nb in range(2):
+            for g in range(2):
+                blk = np.s_[e, 128 * nb:128 * nb + 128, 128 * g:128 * g + 128]
+                amax = np.abs(w[blk]).max()
+                assert s[e, nb, g] == np.float32(amax / 448.0)
+                err = np.abs(dec[blk] * float(s[e, nb, g]) - w[blk])
+                assert np.all(err <= np.abs(w[blk]) * 2.0 ** -4 * (1 + 1e-6)
+                              + 2.0 ** -10 * float(s[e, nb, g]))
+
+
 def test_per_row_quantiser_round_trip():
     rng = np.random.default_rng(2)
     a = rng.standard_normal((50, 64)) * rng.uniform(0.01, 100, size=(50, 1))
