@@ -81,6 +81,15 @@ MUTANTS = [
     ("group weight scales indexed group-major",
      "acc += sx * ws[wrow * ng + g] * part;",
      "acc += sx * ws[((int64_t)e * ng + g) * F + n] * part;"),
+    ("source token of a permuted row off by one",
+     "if (src) src[p] = t;",
+     "if (src) src[p] = t + (t + 1 < N);"),
+    ("pure unpermute writes slot j from the next slot's row",
+     "                       y_perm + (int64_t)pos[(int64_t)t * K + j] * dout, sizeof(double) * (size_t)dout);",
+     "                       y_perm + (int64_t)pos[(int64_t)t * K + (j + 1) % K] * dout, sizeof(double) * (size_t)dout);"),
+    ("E8M0 code 255 decoded as a number instead of NaN",
+     "    if (s == 0xFF) return NAN;\n    return ldexp(1.0, (int)s - 127);",
+     "    return ldexp(1.0, (int)s - 127);"),
     ("bf16 widened from the wrong half",
      "uint32_t u = (uint32_t)b << 16;",
      "uint32_t u = ((uint32_t)b << 16) | 0x8000u;"),

@@ -235,6 +235,20 @@ def test_unpermute_of_permute_is_identity(orc):
     assert np.allclose(y, x, rtol=0, atol=1e-13)
 
 
+def test_pure_unpermute_returns_each_slot_its_own_expert(orc):
+    """Label every permuted row with the expert whose segment (from the
+    offsets) holds it: the pure reorder must put label ids[t][j] in slot
+    t*K + j -- each slot gets its own expert's result, whatever the order of
+    the slots (identity experts cannot tell slots of one token apart)."""
+    rng = np.random.default_rng(12)
+    N, E, K = 50, 9, 4
+    ids = np.stack([rng.permutation(E)[:K] for _ in range(N)]).astype(np.int32)
+    _, offsets, pos, _, _ = orc.permute(ids, E)
+    labels = np.repeat(np.arange(E, dtype=np.float64), np.diff(offsets))[:, None]
+    y = orc.combine(pos, None, labels, N, K)
+    assert np.array_equal(y[:, 0], ids.reshape(-1).astype(np.float64))
+
+
 # ---------------------------------------------------------------- experts
 
 def _scaled_identity_experts(E, D, c, dtype):
