@@ -31,6 +31,8 @@ class OracleStages:
         self.w1 = inp.w1[e0:e0 + self.E_loc]
         self.w3 = None if inp.w3 is None else inp.w3[e0:e0 + self.E_loc]
         self.w2 = None if inp.w2 is None else inp.w2[e0:e0 + self.E_loc]
+        self.d_out = c.d_out
+        self.ydt = torch.float64
 
     def route(self, x):
         ids, gates, _, _ = oracle.router(x.numpy(), self.dt, self.inp.w_r, self.inp.bias, self.c.K)
@@ -67,6 +69,10 @@ CFGS = {
     # the fp8 single-matrix layer with given routing and the pure unpermute:
     # fp8 codes cross the exchange
     "e4m3_given": synth.MoEConfig("ep_e4m3", "e4m3", 96, 64, 8, 4, 48, "none", routing="given"),
+    # a bias of 50 ln(1/rank) sends every token to experts 0 and 1: the ranks
+    # holding experts 2 and 3 receive no rows
+    "relu_ranks_empty": synth.MoEConfig("ep_empty", "f32", 64, 32, 4, 2, 16, "relu",
+                                        zipf_bias=50.0),
 }
 
 
@@ -78,7 +84,7 @@ def _free_port():
     return port
 
 
-def _worker(rank, world, port, name, q, host_exchange=False):
+def _worker(rank, world, port, name, q, host_exchange=False, overlap=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import datetime
     dist.init_process_group("gloo", rank=rank, world_size=world,
@@ -89,7 +95,7 @@ def _worker(rank, world, port, name, q, host_exchange=False):
         n_loc = cfg.N // world
         x = inp.x[rank * n_loc:(rank + 1) * n_loc].contiguous()
         layer = ExpertParallelMoE(OracleStages(inp, rank, world, n_loc), cfg.E, cfg.K,
-                                  host_exchange=host_exchange)
+                                  host_exchange=host_exchange, overlap=overlap)
         tok = np.arange(rank * n_loc, (rank + 1) * n_loc)
         if cfg.routing == "given":
             y = layer.forward(x, ids=inp.ids[rank * n_loc:(rank + 1) * n_loc].contiguous()).numpy()
@@ -103,14 +109,17 @@ def _worker(rank, world, port, name, q, host_exchange=False):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,host_exchange", [(2, False), (4, False), (2, True)])
+@pytest.mark.parametrize("world,host_exchange,overlap",
+                         [(2, False, False), (4, False, False), (2, True, False),
+                          (2, False, True), (4, True, True)])
 @pytest.mark.parametrize("name", list(CFGS))
-def test_expert_parallel_matches_single_rank_oracle(name, world, host_exchange):
-    """host_exchange: the rows travel as byte views of host copies."""
+def test_expert_parallel_matches_single_rank_oracle(name, world, host_exchange, overlap):
+    """host_exchange: the rows travel as byte views of host copies; overlap:
+    peer-to-peer blocks, own rows computed while the others travel."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, name, q, host_exchange))
+    procs = [ctx.Process(target=_worker, args=(r, world, port, name, q, host_exchange, overlap))
              for r in range(world)]
     for p in procs:
         p.start()

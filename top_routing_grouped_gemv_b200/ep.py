@@ -25,8 +25,12 @@ The per-step work is done by a `stages` object (the library's kernels on the
 GPU: `LibraryStages`); the exchanges use torch.distributed (NCCL on GPUs).
 With `host_exchange=True` the exchanged tensors travel as host copies (byte
 views of the rows), for process groups whose backend moves only host memory
-(gloo).  Without an initialized process group the layer runs on one rank
-with no exchange.
+(gloo).  With `overlap=True` the rows travel peer to peer (isend / irecv):
+the rank's rows for its own experts are computed while the others are in
+flight, then every peer's rows as they arrive, each block's results sent
+straight back (computing and communicating overlap; more, smaller expert
+launches).  Every row is still computed as on one GPU.  Without an
+initialized process group the layer runs on one rank with no exchange.
 """
 from __future__ import annotations
 
@@ -138,9 +142,11 @@ class LibraryStages:
 class ExpertParallelMoE:
     """The expert-parallel layer on this rank (see the module docstring)."""
 
-    def __init__(self, stages, E: int, K: int, group=None, host_exchange: bool = False):
+    def __init__(self, stages, E: int, K: int, group=None, host_exchange: bool = False,
+                 overlap: bool = False):
         self.stages, self.E, self.K, self.group = stages, E, K, group
         self.host_exchange = host_exchange
+        self.overlap = overlap
 
     def _all_to_all(self, dist, t, out_rows, out_splits=None, in_splits=None):
         """all_to_all_single of the rows of t (variable splits if given)."""
@@ -150,11 +156,8 @@ class ExpertParallelMoE:
             dist.all_to_all_single(out, t.contiguous(), out_splits, in_splits, group=self.group)
             return out
         # host copies, rows as bytes (the backend may not know the dtype)
-        src = t.contiguous().cpu()
-        row_bytes = t.element_size()
-        for s in t.shape[1:]:
-            row_bytes *= s
-        src_b = src.view(torch.uint8).reshape(src.shape[0], row_bytes)
+        src_b = self._wire_host(t)
+        row_bytes = src_b.shape[1]
         out_b = torch.empty((out_rows, row_bytes), dtype=torch.uint8)
         dist.all_to_all_single(out_b, src_b, out_splits, in_splits, group=self.group)
         return out_b.view(t.dtype).reshape(shape).to(t.device)
@@ -189,6 +192,10 @@ class ExpertParallelMoE:
         recv_rows = recv_h.sum(1).tolist()
         n_send, n_recv = sum(send_rows), sum(recv_rows)
 
+        if self.overlap and dist is not None and G > 1:
+            y_perm = self._exchange_overlapped(dist, G, x_perm, send_h, recv_h)
+            return st.combine(y_perm, pos, gates)
+
         # dispatch: the rows, source-major, expert-minor within each source
         if dist is not None:
             x_recv = self._all_to_all(dist, x_perm[:n_send], n_recv, recv_rows, send_rows)
@@ -208,3 +215,114 @@ class ExpertParallelMoE:
         else:
             y_perm = y_recv
         return st.combine(y_perm, pos, gates)
+
+    # ---- peer-to-peer exchange overlapped with the local experts -------------
+
+    @staticmethod
+    def _wire_host(t):
+        """Host byte view of the rows of t (rows, row bytes); a zero-row tensor
+        (whose strides may not allow a view) gives an empty byte tensor."""
+        row_bytes = t.element_size()
+        for n in t.shape[1:]:
+            row_bytes *= n
+        if t.shape[0] == 0:
+            return torch.empty((0, row_bytes), dtype=torch.uint8)
+        return t.contiguous().cpu().view(torch.uint8).reshape(t.shape[0], row_bytes)
+
+    def _wire(self, t):
+        """The tensor as it travels: itself, or a host byte view."""
+        if not self.host_exchange:
+            return t.contiguous()
+        return self._wire_host(t)
+
+    def _wire_buffer(self, rows, like):
+        shape = (rows,) + tuple(like.shape[1:])
+        if not self.host_exchange:
+            return like.new_empty(shape)
+        row_bytes = like.element_size()
+        for n in like.shape[1:]:
+            row_bytes *= n
+        return torch.empty((rows, row_bytes), dtype=torch.uint8)
+
+    def _unwire(self, buf, like, rows):
+        if not self.host_exchange:
+            return buf
+        return buf.view(like.dtype).reshape((rows,) + tuple(like.shape[1:])).to(like.device)
+
+    def _compute_block(self, rows, x_rows, counts_q):
+        """This rank's experts on rows received from one source (expert-
+        contiguous, counts_q rows per local expert): regroup, FFN, restore."""
+        st = self.stages
+        E_loc = counts_q.numel()
+        ids_q = torch.repeat_interleave(torch.arange(E_loc, dtype=torch.int32), counts_q)
+        ids_q = ids_q.to(x_rows.device).reshape(-1, 1).contiguous()
+        offsets_l, pos_l, x_sorted = st.local_permute(rows, x_rows, ids_q)
+        y_sorted = st.local_ffn(rows, x_sorted, offsets_l)
+        return st.local_unpermute(rows, y_sorted, pos_l)
+
+    def _exchange_overlapped(self, dist, G, x_perm, send_h, recv_h):
+        rank = dist.get_rank(self.group)
+        send_rows = send_h.sum(1).tolist()
+        recv_rows = recv_h.sum(1).tolist()
+        send_off = [0] * G
+        for q in range(1, G):
+            send_off[q] = send_off[q - 1] + send_rows[q - 1]
+        peer = (lambda q: dist.get_global_rank(self.group, q)) if self.group is not None else \
+            (lambda q: q)
+        # post every dispatch receive and send (tag 1); empty blocks are not sent
+        recv_buf, reqs, sends = {}, [], []
+        for q in range(G):
+            if q == rank:
+                continue
+            if recv_rows[q]:
+                recv_buf[q] = self._wire_buffer(recv_rows[q], x_perm)
+                reqs.append((q, dist.irecv(recv_buf[q], src=peer(q), group=self.group, tag=1)))
+            if send_rows[q]:
+                blk = self._wire(x_perm[send_off[q]:send_off[q] + send_rows[q]])
+                recv_buf[("send", q)] = blk   # alive until its send completes
+                sends.append(dist.isend(blk, dst=peer(q), group=self.group, tag=1))
+        y_parts = {}
+        # my own rows first, while the others travel
+        if send_rows[rank]:
+            own = x_perm[send_off[rank]:send_off[rank] + send_rows[rank]]
+            y_parts[rank] = self._compute_block(send_rows[rank], own, recv_h[rank])
+        # then each peer's rows as they arrive; the results go straight back (tag 2)
+        back_recv, back_keep = {}, []
+        y_like = None
+        for q, req in reqs:
+            req.wait()
+            x_q = self._unwire(recv_buf[q], x_perm, recv_rows[q])
+            y_q = self._compute_block(recv_rows[q], x_q, recv_h[q])
+            y_like = y_q
+            w = self._wire(y_q)
+            back_keep.append(w)
+            sends.append(dist.isend(w, dst=peer(q), group=self.group, tag=2))
+        if y_like is None and rank in y_parts:
+            y_like = y_parts[rank]
+        # collect my rows' results from every peer
+        pending = []
+        for q in range(G):
+            if q != rank and send_rows[q]:
+                like = y_like if y_like is not None else self._result_like(x_perm)
+                back_recv[q] = self._wire_buffer(send_rows[q], like)
+                pending.append((q, like, dist.irecv(back_recv[q], src=peer(q), group=self.group,
+                                                    tag=2)))
+        for q, like, req in pending:
+            req.wait()
+            y_parts[q] = self._unwire(back_recv[q], like, send_rows[q])
+        for w in sends:
+            w.wait()
+        # the results in the permuted order (rank blocks in rank order)
+        blocks = [y_parts[q] for q in range(G) if send_rows[q]]
+        if not blocks:
+            return self._result_like(x_perm)[:0]
+        return torch.cat(blocks, dim=0)
+
+    def _result_like(self, x_perm):
+        """An empty result-shaped tensor (rows, d_out) of the stages' output dtype."""
+        st = self.stages
+        d_out = getattr(st, "d_out", None)
+        ydt = getattr(st, "ydt", None)
+        if d_out is None or ydt is None:
+            raise ValueError("the stages give no result shape")
+        return torch.empty(1, d_out, dtype=ydt, device=x_perm.device)
