@@ -40,7 +40,7 @@ def _free_port():
     return port
 
 
-def _worker(rank, world, port, name, q):
+def _worker(rank, world, port, name, q, overlap=False):
     import datetime
     import torch.distributed as dist
     import top_routing_grouped_gemv_b200 as moe
@@ -64,7 +64,7 @@ def _worker(rank, world, port, name, q):
         stages = LibraryStages(n_loc, c.d, c.E, c.K, c.F, c.dtype, c.act, world, w.get("w_r"),
                                sl(w["w1"]), sl(w.get("w3")), sl(w.get("w2")), bias=w.get("bias"),
                                w_scale=inp.w_scale, x_scale=inp.x_scale)
-        layer = ExpertParallelMoE(stages, c.E, c.K, host_exchange=True)
+        layer = ExpertParallelMoE(stages, c.E, c.K, host_exchange=True, overlap=overlap)
         # the whole layer on one GPU, all experts, this rank's tokens
         plan = moe.Plan(n_loc, c.d, c.E, c.K, c.F, c.dtype, c.act, w)
         ws = plan.new_workspace()
@@ -88,13 +88,19 @@ def _worker(rank, world, port, name, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("name", list(CFGS))
-def test_expert_parallel_two_ranks_on_gpu_equal_single_gpu(name):
+CASES = [(n, False) for n in CFGS] + [("bf16_zipf_k4", True), ("bf16_rank_empty", True),
+                                      ("e4m3_given", True)]
+
+
+@pytest.mark.parametrize("name,overlap", CASES)
+def test_expert_parallel_two_ranks_on_gpu_equal_single_gpu(name, overlap):
+    """overlap: peer-to-peer blocks, own rows computed while the others travel."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
     world = 2
-    procs = [ctx.Process(target=_worker, args=(r, world, port, name, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, name, q, overlap))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
