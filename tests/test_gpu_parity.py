@@ -13,7 +13,7 @@ import torch
 
 import oracle
 import synth
-from tests._util import TOL, check_routing, f64, make_plan, near_tie_tokens, rel_err, to_gpu
+from tests._util import TOL, check_routing, f64, make_plan, rel_err
 
 pytestmark = pytest.mark.gpu
 

@@ -5,7 +5,6 @@ worked by hand (tests/golden), closed forms, invariants, brute force on tiny
 inputs, or a library routine (numpy / torch fp64) on a special case.  None of
 these needs a GPU.
 """
-import itertools
 import json
 import math
 import os
