@@ -99,3 +99,12 @@ def test_null_arguments(lib):
                                                0, None) == 1
     assert lib.moe_grouped_ffn_group_scales(None, None, 1.0, None, None, None, None, None, 0,
                                             None) == 1
+
+
+def test_binding_refuses_two_weight_scale_modes():
+    """The Python plan takes one weight scale mode (the C ABI has one quant
+    field): two kinds of scales in the weights dict are an error before the
+    library is asked."""
+    with pytest.raises(ValueError, match="one weight scale mode"):
+        moe.Plan(16, 64, 4, 2, 32, "e4m3", "none",
+                 {"w1": None, "w_mx_scales": object(), "w_group_scales": object()})

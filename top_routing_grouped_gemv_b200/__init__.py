@@ -152,11 +152,16 @@ class Plan:
         quant = QUANT_NONE
         if dtype == "e4m3":
             quant = QUANT_PER_TENSOR
-            for key, code in (("w_channel_scales", QUANT_PER_CHANNEL), ("w_mx_scales", QUANT_MX),
-                              ("w_group_scales", QUANT_PER_GROUP),
-                              ("w_block_scales", QUANT_PER_BLOCK)):
-                if weights.get(key) is not None:
-                    quant = code
+            given = [(key, code) for key, code in (("w_channel_scales", QUANT_PER_CHANNEL),
+                                                   ("w_mx_scales", QUANT_MX),
+                                                   ("w_group_scales", QUANT_PER_GROUP),
+                                                   ("w_block_scales", QUANT_PER_BLOCK))
+                     if weights.get(key) is not None]
+            if len(given) > 1:
+                raise ValueError("one weight scale mode per plan, got "
+                                 + ", ".join(k for k, _ in given))
+            if given:
+                quant = given[0][1]
         desc = LayerDesc(N, d, E, K, F, DTYPE_CODE[dtype], ACT_CODE[act], quant)
         w = LayerWeights(_ptr(weights.get("w_r")), _ptr(weights.get("bias")),
                          _ptr(weights.get("w1")), _ptr(weights.get("w3")),
