@@ -304,7 +304,9 @@ moe_status moe_forward_routed_shared(moe_plan plan, const void* x, const int32_t
                                      const float* w_sh_channel_scales_or_null, void* y_sh,
                                      void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* MX layer (MOE_QUANT_MX, act NONE): x (N, d) e4m3 codes with x_mx_scales
+/* MX layer ("aclnnQuantGroupedMatMulAlltoAllv", parameter section, quant
+ * mode 6 "mx", read as OCP MXFP8; the formula section's gmmY with the block
+ * scales inside the sum).  MOE_QUANT_MX, act NONE: x (N, d) e4m3 codes with x_mx_scales
  * (N, d/32) E8M0, one per 32 consecutive elements of a row.  Computes, per
  * routed row of expert e,
  *   gmmY[r][n] = sum_k (x[r][k] * 2^(xs[r][k/32] - 127)) * (W[e][n][k] * 2^(ws[e][n][k/32] - 127))
@@ -316,7 +318,9 @@ moe_status moe_forward_routed_shared(moe_plan plan, const void* x, const int32_t
  * scales of x row perm_src[r].  moe_grouped_ffn_mx: the grouped matmul of
  * permuted rows x_perm with their scales x_perm_mx_scales (N*K, d/32).
  * MOE_ERR_UNSUPPORTED for a plan that is not MX; the other FFN calls return
- * MOE_ERR_UNSUPPORTED for an MX plan. */
+ * MOE_ERR_UNSUPPORTED for an MX plan.  MOE_ERR_INVALID_ARG for null or
+ * misaligned pointers; device errors go to the workspace status word.  All
+ * buffers are the caller's. */
 moe_status moe_forward_routed_mx(moe_plan plan, const void* x, const uint8_t* x_mx_scales,
                                  const int32_t* topk_ids, const float* topk_gates_or_null,
                                  void* y, void* ws, size_t ws_bytes, moe_stream_t stream);
@@ -329,7 +333,10 @@ moe_status moe_grouped_ffn_mx(moe_plan plan, const void* x_perm, const uint8_t* 
                               const int32_t* offsets, void* y_perm, void* ws, size_t ws_bytes,
                               moe_stream_t stream);
 
-/* Group / block-scaled layer (MOE_QUANT_PER_GROUP or PER_BLOCK, act NONE):
+/* Group / block-scaled layer ("aclnnQuantGroupedMatMulAlltoAllv", parameter
+ * section, quant modes 4 "pergroup" and 5 "perblock", read as fp32 scales per
+ * 128 elements of K; the formula section's gmmY with the scales inside the
+ * sum).  MOE_QUANT_PER_GROUP or PER_BLOCK, act NONE:
  *   gmmY[r][n] = sum_g xs[r][g] * ws[e][n][g] * (sum_{k in group g} x[r][k] * W[e][n][k])
  * groups of 128 elements of d; ws the plan's weight scales (for PER_BLOCK
  * the scale of channel n's block n/128); xs per row and group from
@@ -341,7 +348,10 @@ moe_status moe_grouped_ffn_mx(moe_plan plan, const void* x_perm, const uint8_t* 
  * (y (N, F)); the activation scales are indexed by token.
  * moe_grouped_ffn_group_scales: permuted rows, their scales per permuted
  * row (x_row_scales (N*K) or x_group_scales (N*K, d/128)).
- * MOE_ERR_UNSUPPORTED for other plans. */
+ * MOE_ERR_UNSUPPORTED for other plans; MOE_ERR_INVALID_ARG for null or
+ * misaligned pointers (x, y, x_perm, y_perm: 16-byte aligned rows); device
+ * errors (bad expert ids, a pipeline wait that ran out) go to the workspace
+ * status word.  All buffers are the caller's. */
 moe_status moe_forward_routed_group_scales(moe_plan plan, const void* x, float x_scale,
                                            const float* x_token_scales_or_null,
                                            const float* x_group_scales_or_null,
