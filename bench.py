@@ -1,8 +1,11 @@
 """Benchmark of the one-GPU MoE layer forward (router -> permute -> grouped
-FFN -> combine) on the bf16 prefill workload: N=4096 tokens, d=2048, E=8
-experts, top-2, SwiGLU FFN d->8192->d, fp32 router; seeded synthetic inputs.
+FFN -> combine).  Default workload: the fine-grained bf16 prefill layer,
+N=16384 tokens, d=2048, E=128 experts, top-8, SwiGLU FFN d->768->d, fp32
+router with a Zipf-like per-expert bias 1.2*ln(1/rank) (skewed expert loads,
+some experts empty); seeded synthetic inputs.  --workload picks another one.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --measure-peak      # dense e4m3 / bf16 matmul peaks of this GPU
 
 One JSON line on rank 0.  ``value`` is whole-job tokens/s from CUDA events on
 the launching stream (max over ranks), inputs resident in HBM, L2 flushed
@@ -36,6 +39,8 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE layer tokens/s and grouped-GEMM TFLOP/s (% of tensor/HBM roofline), 1 B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
+DEFAULT_WORKLOAD = "bf16_n16384_d2048_e128_k8_f768_swiglu_zipf"
+E4M3_PEAK_FILE = os.path.join(ROOT, "profiles", "peak_e4m3_matmul_8192.md")
 
 
 def parse():
@@ -44,7 +49,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="bf16_n4096_d2048_e8_k2_f8192_swiglu")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--measure-peak", action="store_true",
+                    help="time dense 8192^3 e4m3 and bf16 matmuls (cuBLASLt through torch) "
+                         "and write the e4m3 peak file that the fp8 rooflines divide by")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -59,6 +67,91 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_e4m3_peak():
+    """The measured dense e4m3 matmul peaks (burst, sustained) in TFLOP/s from
+    the committed peak file, or None."""
+    if not os.path.exists(E4M3_PEAK_FILE):
+        return None
+    text = open(E4M3_PEAK_FILE).read()
+    vals = {}
+    for key in ("e4m3_tflops", "e4m3_tflops_sustained"):
+        m = re.search(rf"^{key}:\s*([0-9.eE+]+)\s*$", text, re.M)
+        if not m:
+            return None
+        vals[key] = float(m.group(1))
+    return vals
+
+
+def measure_peak(steps_burst: int = 10, sustain_s: float = 4.0):
+    """Dense matmul peaks of this GPU through torch (cuBLASLt): e4m3 x e4m3 ->
+    bf16 with unit fp32 scales (torch._scaled_mm) and bf16 x bf16, both
+    8192^3 (2 * 8192^3 FLOP).  Burst = the best of `steps_burst` single runs
+    (CUDA events, after warm-up); sustained = the mean over back-to-back runs
+    for `sustain_s` seconds, under the power cap.  SM clocks are sampled
+    meanwhile.  Writes E4M3_PEAK_FILE and prints one JSON line."""
+    import torch
+    n = 8192
+    flop = 2.0 * n * n * n
+    torch.manual_seed(0)
+    a8 = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+    b8 = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()  # column-major operand
+    one = torch.ones((), device="cuda")
+    a16 = torch.randn(n, n, device="cuda", dtype=torch.bfloat16)
+    b16 = torch.randn(n, n, device="cuda", dtype=torch.bfloat16)
+    runs = {
+        "e4m3": lambda: torch._scaled_mm(a8, b8, scale_a=one, scale_b=one, out_dtype=torch.bfloat16),
+        "bf16": lambda: torch.matmul(a16, b16),
+    }
+    out = {}
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for name, f in runs.items():
+            for _ in range(5):
+                f()
+            torch.cuda.synchronize()
+            best = float("inf")
+            for _ in range(steps_burst):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                f()
+                e1.record()
+                e1.synchronize()
+                best = min(best, e0.elapsed_time(e1))
+            # sustained: launch in batches of 20 until sustain_s has passed
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            count = 0
+            t0 = time.perf_counter()
+            e0.record()
+            while time.perf_counter() - t0 < sustain_s:
+                for _ in range(20):
+                    f()
+                count += 20
+                torch.cuda.synchronize()
+            e1.record()
+            e1.synchronize()
+            out[name] = {"burst_tflops": flop / (best * 1e-3) / 1e12,
+                         "sustained_tflops": flop * count / (e0.elapsed_time(e1) * 1e-3) / 1e12}
+    clocks = clk.summary()
+    line = {"peaks": out, "clocks": clocks, "n": n}
+    text = (
+        "# Dense e4m3 matmul peak of this B200 (the denominator of the fp8 rooflines)\n\n"
+        "Command (one GPU, no profiler): `python bench.py --measure-peak`\n\n"
+        f"8192^3 matmuls through torch (cuBLASLt): e4m3 x e4m3 -> bf16 with unit fp32 scales "
+        f"(torch._scaled_mm) and bf16 x bf16 (torch.matmul); burst = best of {steps_burst} "
+        f"single runs, sustained = back-to-back runs for {sustain_s:.0f} s under the power cap; "
+        "CUDA events.\n\n"
+        f"e4m3_tflops: {out['e4m3']['burst_tflops']:.1f}\n"
+        f"e4m3_tflops_sustained: {out['e4m3']['sustained_tflops']:.1f}\n"
+        f"bf16_tflops_same_run: {out['bf16']['burst_tflops']:.1f}\n"
+        f"bf16_tflops_sustained_same_run: {out['bf16']['sustained_tflops']:.1f}\n"
+        f"sm_mhz_median: {clocks.get('sm_mhz')}\n"
+        f"sm_max_mhz: {clocks.get('sm_max_mhz')}\n"
+        f"throttle_reasons: {', '.join(clocks.get('reasons') or []) or 'none'}\n"
+    )
+    with open(E4M3_PEAK_FILE, "w") as f:
+        f.write(text)
+    print(json.dumps(line), flush=True)
 
 
 def kernel_source_hash() -> str:
@@ -269,6 +362,10 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank)
         return
+    if args.measure_peak:
+        if rank == 0:
+            measure_peak()
+        return
 
     import numpy as np
     import torch
@@ -468,16 +565,22 @@ def main():
     clk_summary = clk.summary()
     sustained = wall > 2.0 or "sw_power_cap" in clk_summary.get("reasons", [])
     peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
-    peak_note = ""
+    peak_desc = f"{peak_src} bf16 {'sustained' if sustained else 'burst'}"
     if cfg.dtype == "e4m3":
-        peak *= 2.0   # dense e4m3 = 2x bf16 (nominal ratio), no measured fp8 peak
-        peak_note = " x 2 (e4m3 nominal ratio)"
+        p8 = load_e4m3_peak()
+        if p8 is not None:   # the measured dense e4m3 matmul peak of this machine's B200s
+            peak = p8["e4m3_tflops_sustained" if sustained else "e4m3_tflops"]
+            peak_desc = (f"measured e4m3 {'sustained' if sustained else 'burst'} "
+                         f"({os.path.relpath(E4M3_PEAK_FILE, ROOT)})")
+        else:                # no measurement: 2x bf16, the nominal ratio
+            peak *= 2.0
+            peak_desc += " x 2 (e4m3 nominal ratio)"
     t1 = stage_us.get(k1, float("nan")) * 1e-6
     achieved = f1 / t1 / 1e12
     traffic = profiled_traffic(cfg.name, k1)
     roofline = {"bound": "tensor", "kernel": k1, "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'}{peak_note}",
+                "peak_source": peak_desc,
                 "algorithmic_flop_per_launch": f1}
     ffn_keys = [k for k in stage_us if k.startswith("ffn") or k.startswith("gmm")]
     ffn_s = sum(stage_us[k] for k in ffn_keys) * 1e-6

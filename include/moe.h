@@ -24,10 +24,15 @@
  * Conventions for every call
  *  - Pointers named *_host are host memory; every other data pointer is
  *    device memory of the plan's device.  The caller allocates and frees all
- *    of them.  The library allocates no device memory (not in
- *    moe_plan_create either); it never frees caller memory.  Its only
- *    device memory of its own is the static scratch array of
- *    moe_permute_noalloc.
+ *    of them; the library never frees caller memory.
+ *  - Device memory of the library's own: moe_plan_create allocates, once,
+ *    plan-owned copies of weight data in the layout the kernels read, and
+ *    moe_plan_destroy frees them: the router weights split into three bf16
+ *    parts (plans whose router runs on the tensor cores), the MX weight
+ *    scales (MOE_QUANT_MX) and the transposed group / block weight scales
+ *    (MOE_QUANT_PER_GROUP, MOE_QUANT_PER_BLOCK).  No call allocates device
+ *    memory after moe_plan_create.  The only other device memory of the
+ *    library is the static scratch array of moe_permute_noalloc.
  *  - Launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *    default stream).  Only moe_read_device_status, moe_forward_host and
  *    moe_profile_read synchronise.
@@ -210,9 +215,12 @@ moe_status moe_permute(moe_plan plan, const void* x, const int32_t* topk_ids, in
  * NULL; the caller zeroes it) receives MOE_ERR_DEVICE_BAD_INDEX if an id is
  * outside [0, E).  Limit: ceil(N/32) * E * 4 bytes <= 1 MiB (e.g. N = 32768
  * with E = 256); a larger plan is refused with MOE_ERR_WORKSPACE_TOO_SMALL
- * and nothing is launched.  The first call on each device looks up the
- * array's device address (with that device current), so make that first
- * call before any stream capture.  All calls share the one array: calls
+ * and nothing is launched.  Every call looks up the array's device address
+ * on the current device (cudaGetSymbolAddress, which allocates nothing and
+ * is not cached, so it stays valid after a cudaDeviceReset); the first call
+ * on a device also loads the library's module there, so make that first
+ * call before any stream capture.  Like moe_permute it sets the plan's
+ * launch count and stage events.  All calls share the one array: calls
  * whose kernels overlap on the GPU (different streams, or several threads)
  * race on it; serialise them. */
 moe_status moe_permute_noalloc(moe_plan plan, const void* x, const int32_t* topk_ids,

@@ -7,19 +7,45 @@ import torch
 
 import synth
 
-# Float tolerances (normwise: max|gpu - ref| / max|ref| over a tensor) against
-# the fp64 oracle: fp32 1e-5, bf16 2e-2, fp8 6e-2.
+# Float tolerances against the fp64 oracle: fp32 1e-5, bf16 2e-2, fp8 6e-2.
+# Each bounds both the normwise error (max|gpu - ref| / max|ref| over the
+# tensor) and the worst row's error relative to that row's own max|ref|
+# (floored at ROW_FLOOR of the tensor's max|ref|, so that a row of near-zero
+# values is judged on absolute error): a small-valued row cannot hide behind
+# large rows elsewhere.
 TOL = {"f32": 1e-5, "bf16": 2e-2, "e4m3": 6e-2}
 NEAR_TIE = 1e-5
+ROW_FLOOR = 1e-3
 
 
-def rel_err(gpu: np.ndarray, ref: np.ndarray) -> float:
+def normwise_err(gpu: np.ndarray, ref: np.ndarray) -> float:
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
     den = np.abs(ref).max() if ref.size else 0.0
     if den == 0.0:
         return float(np.abs(gpu).max()) if gpu.size else 0.0
     return float(np.abs(gpu - ref).max() / den)
+
+
+def row_err(gpu: np.ndarray, ref: np.ndarray) -> float:
+    """Worst row of |gpu - ref| / max(max|ref row|, ROW_FLOOR * max|ref|)
+    (rows = the last axis; a 1-D array is one row)."""
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    if not ref.size:
+        return 0.0
+    g2 = gpu.reshape(-1, ref.shape[-1]) if ref.ndim > 1 else gpu.reshape(1, -1)
+    r2 = ref.reshape(-1, ref.shape[-1]) if ref.ndim > 1 else ref.reshape(1, -1)
+    top = np.abs(r2).max()
+    if top == 0.0:
+        return float(np.abs(g2).max())
+    den = np.maximum(np.abs(r2).max(axis=1), ROW_FLOOR * top)
+    return float((np.abs(g2 - r2).max(axis=1) / den).max())
+
+
+def rel_err(gpu: np.ndarray, ref: np.ndarray) -> float:
+    """The larger of the normwise and the worst-row relative error."""
+    return max(normwise_err(gpu, ref), row_err(gpu, ref))
 
 
 def to_gpu(inp: synth.MoEInputs) -> dict:

@@ -7,8 +7,9 @@ library's static device memory instead of a caller workspace.
 Checked through the C ABI against moe_permute on two calls in a row with
 different routings, so a stale scratch array from the first call would
 show up in the second.  Collected last so that a run stopping at the first
-failure has already run every other test; it also runs alone in a fresh
-process (it builds and loads the library itself).
+failure has already run every other test.  It needs no state from other
+tests (it builds and loads the library itself), so it passes both after the
+rest of the suite and on its own (pytest tests/test_zz_no_alloc.py).
 """
 import numpy as np
 import pytest
@@ -49,6 +50,7 @@ def test_noalloc_permute_matches_workspace_permute_twice():
         got = bufs()
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
         plan.permute_noalloc(x, ids, *got, device_status=status)
+        assert plan.last_launch_count() == 3  # rank, scan, gather, as moe_permute
         torch.cuda.synchronize()
         assert int(status.item()) == 0, f"call {call}: device status {int(status.item())}"
         for a, b in zip(got, ref):

@@ -1052,6 +1052,15 @@ int moe_last_launch_count(moe_plan p) { return p ? p->launches : -1; }
 
 }  // extern "C"
 
+void moe::plan_call_begin(moe_plan_s* p) { begin(p); }
+void moe::plan_call_mark(moe_plan_s* p, cudaStream_t s, const char* name_of_next) {
+  mark(p, s, name_of_next);
+}
+void moe::plan_call_end(moe_plan_s* p, cudaStream_t s, int launches) {
+  p->launches += launches;
+  end(p, s);
+}
+
 bool moe::plan_permute_shape(const moe_plan_s* p, int* N, int* d, int* E, int* K,
                              int* row_bytes) {
   if (!p) return false;

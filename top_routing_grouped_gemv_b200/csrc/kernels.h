@@ -233,4 +233,13 @@ inline int warps_per_token(int N) {
 bool plan_permute_shape(const ::moe_plan_s* plan, int* N, int* d, int* E, int* K,
                         int* row_bytes);
 
+// Per-call bookkeeping of a plan for entry points outside the plan's
+// translation unit: begin() clears the launch count and the stage events,
+// mark() records the boundary before the named stage (when per-stage timing
+// is on), end() records the last boundary and adds the call's launches to
+// the count that moe_last_launch_count reports.
+void plan_call_begin(::moe_plan_s* plan);
+void plan_call_mark(::moe_plan_s* plan, cudaStream_t s, const char* name_of_next);
+void plan_call_end(::moe_plan_s* plan, cudaStream_t s, int launches);
+
 }  // namespace moe

@@ -9,12 +9,12 @@
 //
 // The array is a module-scope __device__ variable: every GPU that loads the
 // library holds its 1 MiB until the process exits.  Its host-side name is
-// only a stand-in for the symbol, so the device address is looked up with
-// cudaGetSymbolAddress once per device (on the first call made with that
-// device current) and cached.
+// only a stand-in for the symbol, so every call looks the device address up
+// with cudaGetSymbolAddress on the current device (a host-side query that
+// allocates nothing; on a device's first call it also loads the module
+// there).  Nothing is cached, so the address stays right after a
+// cudaDeviceReset or a reload of the library.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "moe.h"
 #include "kernels.h"
@@ -22,28 +22,20 @@
 namespace {
 
 constexpr size_t kScratchBytes = size_t(1) << 20;
-constexpr int kMaxDevices = 64;
 
 // Per-chunk expert counts, then (after the scan) per-chunk expert bases.
 // Every call writes all ceil(N/32)*E entries it later reads, so no entry has
 // to start at zero.
 static __device__ __align__(256) int32_t g_permute_scratch[kScratchBytes / sizeof(int32_t)];
 
-std::mutex g_mutex;
-int32_t* g_scratch_ptr[kMaxDevices] = {nullptr};
-
 // Device address of g_permute_scratch on the current device.
 moe_status scratch_on_current_device(int32_t** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr)
-      return MOE_ERR_CUDA;
-    g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) {
+    cudaGetLastError();  // leave no sticky error behind for the caller
+    return MOE_ERR_CUDA;
   }
-  *out = g_scratch_ptr[dev];
+  *out = static_cast<int32_t*>(p);
   return MOE_OK;
 }
 
@@ -68,10 +60,16 @@ extern "C" moe_status moe_permute_noalloc(moe_plan plan, const void* x, const in
   if (st != MOE_OK) return st;
   cudaStream_t s = stream;
   int* status = device_status_or_null;
-  if (moe::launch_permute_count(topk_ids, N, K, E, scratch, perm_pos, status, s) != cudaSuccess ||
-      moe::launch_permute_scan(scratch, nchunks, E, counts, offsets, s) != cudaSuccess ||
-      moe::launch_permute_gather(x, row_bytes, topk_ids, N, K, E, scratch, perm_pos, perm_src, nullptr,
-                                 x_perm, status, s) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  return MOE_OK;
+  // the same three kernels as moe_permute, recorded in the plan's launch
+  // count and stage events like that call
+  moe::plan_call_begin(plan);
+  moe::plan_call_mark(plan, s, "permute_count");
+  bool ok = moe::launch_permute_count(topk_ids, N, K, E, scratch, perm_pos, status, s) == cudaSuccess;
+  moe::plan_call_mark(plan, s, "permute_scan");
+  ok = ok && moe::launch_permute_scan(scratch, nchunks, E, counts, offsets, s) == cudaSuccess;
+  moe::plan_call_mark(plan, s, "permute_gather");
+  ok = ok && moe::launch_permute_gather(x, row_bytes, topk_ids, N, K, E, scratch, perm_pos, perm_src,
+                                        nullptr, x_perm, status, s) == cudaSuccess;
+  moe::plan_call_end(plan, s, 3);
+  return ok ? MOE_OK : MOE_ERR_CUDA;
 }
