@@ -463,13 +463,16 @@ def main():
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
         # per-kernel durations: the same loop with the library recording
-        # events between its kernels (the L2 flush before each step gives the
-        # host a head start, so the GEMMs are enqueued before the GPU reaches
-        # them and no launch gap lands inside their spans)
+        # events between its kernels.  Each iteration waits for its events, so
+        # the host starts every step from idle: a GPU sleep after the L2 flush
+        # (about 0.5 ms) gives it the head start it has in the timed loop, so
+        # every launch is queued before the GPU reaches it and no host launch
+        # delay lands inside a kernel's span (the first kernel's included)
         plan.profile(True)
         per_kernel: dict[str, list[float]] = {}
         for i in range(min(args.steps, 100)):
             flush.zero_()
+            torch.cuda._sleep(1_000_000)
             step()
             for name, ms in plan.profile_read():
                 per_kernel.setdefault(name, []).append(ms)

@@ -157,12 +157,19 @@ typedef struct moe_plan_s* moe_plan;
 
 /* Validates desc and weights, records the weight pointers (not owned: they
  * must stay valid while the plan is used) and encodes the TMA descriptors of
- * the weights for the current CUDA device.  Allocates host memory only,
- * except for MOE_QUANT_MX: the plan then also holds a device copy of the
- * weight scales in the layout of the block-scaled tensor-core MMA (the same
- * bytes as w_mx_scales, rearranged; about E*F*d/32 bytes), made here
- * (synchronously) and freed by moe_plan_destroy; likewise for PER_GROUP /
- * PER_BLOCK a transposed copy of w_group_scales (E, d/128, columns).
+ * the weights for the current CUDA device.  Some plans also hold device
+ * copies of weight data in the layout their kernels read, made here
+ * (synchronously, on a private stream) and freed by moe_plan_destroy:
+ *  - a router on the tensor cores (bf16 x with at most 16 experts, unless
+ *    the split-K router applies): w_r split into three bf16 parts, 6*d*E
+ *    bytes rounded up to whole 32 x 8 tiles; w_r must be device memory
+ *    (MOE_ERR_INVALID_ARG otherwise).  The split is taken from w_r now:
+ *    after changing w_r in place call moe_plan_refresh_router;
+ *  - MOE_QUANT_MX: the weight scales in the layout of the block-scaled
+ *    tensor-core MMA (the same bytes as w_mx_scales, rearranged; about
+ *    E*F*d/32 bytes);
+ *  - PER_GROUP / PER_BLOCK: a transposed copy of w_group_scales (E, d/128,
+ *    columns).
  * With w1, w3 and w2 all NULL (and no per-channel scales) the plan is
  * routing-only: router, permute and unpermute/combine work, the calls that
  * run the experts return MOE_ERR_UNSUPPORTED (an expert-parallel rank's
@@ -170,6 +177,13 @@ typedef struct moe_plan_s* moe_plan;
 moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* weights,
                            moe_plan* out);
 moe_status moe_plan_destroy(moe_plan plan);
+
+/* Re-derives the plan's copy of the router weights from weights.w_r (after
+ * the caller changed w_r in place), stream-ordered on `stream`; no-op for
+ * plans whose router reads w_r directly.  Not part of the pages' interface:
+ * the plan-time copy is this library's choice (the router weights change
+ * rarely, the split need not run on every call). */
+moe_status moe_plan_refresh_router(moe_plan plan, moe_stream_t stream);
 
 /* Bytes of device workspace that every call below accepts (the largest
  * need, that of moe_forward_host).  Workspace base must be 256-byte aligned. */
@@ -185,10 +199,11 @@ moe_status moe_workspace_init(moe_plan plan, void* ws, size_t ws_bytes, moe_stre
  * accuracy; keep the K largest (descending, equal logits -> lower expert
  * index); gates = softmax over the kept K only.  margin_or_null (N)
  * receives l_(K) - l_(K+1) (+inf when K == E).  x dtype fp32 or bf16.
- * Needs plan weights.w_r.  bf16 layers with more than 32 experts compute the
- * logits on the tensor cores from an exact three-part bf16 split of w_r,
- * written to workspace scratch on every call (so w_r may change between
- * calls). */
+ * Needs plan weights.w_r.  bf16 layers with at most 16 experts compute the
+ * logits on the warp-level tensor-core MMA from the plan's exact three-part
+ * bf16 split of w_r (moe_plan_create, moe_plan_refresh_router); bf16 layers
+ * with more than 32 experts on tcgen05 from the same split, written to
+ * workspace scratch on every call; the others, and fp32 x, with fp32 FMA. */
 moe_status moe_router_topk(moe_plan plan, const void* x, int32_t* topk_ids, float* topk_gates,
                            float* margin_or_null, void* ws, size_t ws_bytes, moe_stream_t stream);
 
@@ -208,13 +223,16 @@ moe_status moe_permute(moe_plan plan, const void* x, const int32_t* topk_ids, in
  * allocation and passes an operator only its inputs and outputs (a plugin
  * of an inference engine), or latency-critical code that must not risk the
  * device-wide synchronisation a cudaMalloc / cudaFree can cause.  This
- * variant takes no workspace and allocates nothing: its scratch (the
- * per-chunk expert counts) is a 1 MiB array in the library's static device
- * memory, held by every GPU that loads the library until the process exits.
+ * variant takes no workspace and allocates nothing: its scratch (a counter
+ * and the per-256-token-block expert counts) is a 1 MiB array in the
+ * library's static device memory, held by every GPU that loads the library
+ * until the process exits; the counter starts at zero when the library is
+ * loaded on a device and every call leaves it at zero.
  * Same outputs as moe_permute.  device_status_or_null (device int32, may be
  * NULL; the caller zeroes it) receives MOE_ERR_DEVICE_BAD_INDEX if an id is
- * outside [0, E).  Limit: ceil(N/32) * E * 4 bytes <= 1 MiB (e.g. N = 32768
- * with E = 256); a larger plan is refused with MOE_ERR_WORKSPACE_TOO_SMALL
+ * outside [0, E).  Limit: 256 + ceil(N/256) * E * 4 bytes <= 1 MiB (e.g.
+ * N = 262144 with E = 255, or N = 261888 with E = 256); a larger plan is
+ * refused with MOE_ERR_WORKSPACE_TOO_SMALL
  * and nothing is launched.  Every call looks up the array's device address
  * on the current device (cudaGetSymbolAddress, which allocates nothing and
  * is not cached, so it stays valid after a cudaDeviceReset); the first call

@@ -84,7 +84,7 @@ def _free_port():
     return port
 
 
-def _worker(rank, world, port, name, q, host_exchange=False, overlap=False):
+def _worker(rank, world, port, name, q, host_exchange=False, overlap=False, capacity=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import datetime
     dist.init_process_group("gloo", rank=rank, world_size=world,
@@ -95,7 +95,8 @@ def _worker(rank, world, port, name, q, host_exchange=False, overlap=False):
         n_loc = cfg.N // world
         x = inp.x[rank * n_loc:(rank + 1) * n_loc].contiguous()
         layer = ExpertParallelMoE(OracleStages(inp, rank, world, n_loc), cfg.E, cfg.K,
-                                  host_exchange=host_exchange, overlap=overlap)
+                                  host_exchange=host_exchange, overlap=overlap,
+                                  capacity=capacity)
         tok = np.arange(rank * n_loc, (rank + 1) * n_loc)
         if cfg.routing == "given":
             y = layer.forward(x, ids=inp.ids[rank * n_loc:(rank + 1) * n_loc].contiguous()).numpy()
@@ -109,17 +110,22 @@ def _worker(rank, world, port, name, q, host_exchange=False, overlap=False):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,host_exchange,overlap",
-                         [(2, False, False), (4, False, False), (2, True, False),
-                          (2, False, True), (4, True, True)])
+@pytest.mark.parametrize("world,host_exchange,overlap,capacity",
+                         [(2, False, False, False), (4, False, False, False),
+                          (2, True, False, False), (2, False, True, False), (4, True, True, False),
+                          (2, False, False, True), (4, True, False, True)])
 @pytest.mark.parametrize("name", list(CFGS))
-def test_expert_parallel_matches_single_rank_oracle(name, world, host_exchange, overlap):
+def test_expert_parallel_matches_single_rank_oracle(name, world, host_exchange, overlap,
+                                                    capacity):
     """host_exchange: the rows travel as byte views of host copies; overlap:
-    peer-to-peer blocks, own rows computed while the others travel."""
+    peer-to-peer blocks, own rows computed while the others travel;
+    capacity: fixed-size padded blocks with the counts inside, no host read
+    of the counts."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, name, q, host_exchange, overlap))
+    procs = [ctx.Process(target=_worker,
+                         args=(r, world, port, name, q, host_exchange, overlap, capacity))
              for r in range(world)]
     for p in procs:
         p.start()
@@ -133,10 +139,33 @@ def test_expert_parallel_matches_single_rank_oracle(name, world, host_exchange, 
         assert err == 0.0, (rank, err)
 
 
-def test_single_rank_without_process_group():
+@pytest.mark.parametrize("capacity", [False, True])
+def test_single_rank_without_process_group(capacity):
     cfg = CFGS["relu"]
     inp = synth.make_inputs(cfg, seed=3)
-    layer = ExpertParallelMoE(OracleStages(inp, 0, 1, cfg.N), cfg.E, cfg.K)
+    layer = ExpertParallelMoE(OracleStages(inp, 0, 1, cfg.N), cfg.E, cfg.K, capacity=capacity)
     y = layer.forward(inp.x).numpy()
     ref, _, _, _ = oracle.forward_tokens(inp, np.arange(cfg.N))
     assert np.abs(y - ref).max() == 0.0
+
+
+def test_capacity_exchange_reads_no_counts_on_the_host(monkeypatch):
+    """The fixed-capacity exchange never moves a tensor's values to the host:
+    every Tensor.cpu / .item / .tolist / bool / int / float during its
+    exchange fails the test."""
+    cfg = CFGS["swiglu_zipf"]
+    inp = synth.make_inputs(cfg, seed=4)
+    st = OracleStages(inp, 0, 1, cfg.N)
+    layer = ExpertParallelMoE(st, cfg.E, cfg.K, capacity=True)
+    x = inp.x
+    ids, gates = st.route(x)
+    counts, offsets, pos, x_perm = st.permute(x, ids)
+    calls = []
+    for name in ("cpu", "item", "tolist", "__bool__", "__int__", "__float__"):
+        monkeypatch.setattr(torch.Tensor, name, lambda self, *a, _n=name, **k: calls.append(_n))
+    monkeypatch.setattr(st, "local_ffn",
+                        lambda n, xs, offs: torch.zeros(n, st.d_out, dtype=torch.float64))
+    y_perm = layer._exchange_capacity(None, 1, cfg.E, x_perm, counts, offsets)
+    monkeypatch.undo()
+    assert calls == []
+    assert tuple(y_perm.shape) == (cfg.N * cfg.K, st.d_out)

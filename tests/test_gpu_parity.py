@@ -61,6 +61,13 @@ SMALL = {
     "bf16_pair_swiglu": synth.MoEConfig("pair_sw", "bf16", 4100, 128, 2, 1, 256, "swiglu"),
     "e4m3_pair": synth.small_variant(synth.FP8_GMM, N=1100, d=256, E=4, K=2, F=392,
                                      shared=(256, 392)),
+    # bf16, at most 16 experts: router on the warp-level MMA; rows not a whole
+    # number of 32-element blocks, two expert tiles, a ragged 16-token group
+    "bf16_mma_router_e13": synth.MoEConfig("mma_e13", "bf16", 333, 424, 13, 3, 64, "swiglu"),
+    # enough 16-token groups for two per CTA (one and two expert tiles)
+    "bf16_mma_router_g2_e8": synth.MoEConfig("mma_g2_e8", "bf16", 4801, 256, 8, 2, 64, "swiglu"),
+    "bf16_mma_router_g2_e16": synth.MoEConfig("mma_g2_e16", "bf16", 4900, 160, 16, 4, 64,
+                                              "swiglu", zipf_bias=1.2),
 }
 
 _cache = {}
@@ -557,10 +564,10 @@ def test_stage_profile_names():
     prof = plan.profile_read()
     plan.profile(False)
     names = [n for n, _ in prof]
-    assert names == ["router_topk", "permute_count", "permute_scan", "permute_gather",
-                     "ffn1_swiglu_tc", "ffn2_tc", "combine"]
+    assert names == ["router_mma", "permute_rank", "permute_gather", "ffn1_swiglu_tc",
+                     "ffn2_tc", "combine"]
     assert all(ms >= 0 for _, ms in prof)
-    assert plan.last_launch_count() == 7
+    assert plan.last_launch_count() == 6
 
 
 def test_bounded_wait_timeout_sets_status_and_context_survives():
@@ -952,3 +959,34 @@ def test_plan_refuses_host_scale_tables():
         moe.Plan(g.N, g.d, g.E, g.K, g.F, "e4m3", "none",
                  {"w1": ginp.w1.cuda(), "w_block_scales": ginp.w_gs})
     assert e.value.code == 1
+
+
+def test_refresh_router_after_weights_change():
+    """A bf16 plan with at most 16 experts routes from its own split copy of
+    w_r, taken at plan creation: changing w_r in place leaves the routing as it
+    was until moe_plan_refresh_router, after which it follows the new weights
+    (checked against the oracle)."""
+    cfg = synth.MoEConfig("refresh", "bf16", 600, 256, 8, 2, 64, "swiglu")
+    inp = synth.make_inputs(cfg, seed=5)
+    plan, w = make_plan(inp)
+    x = inp.x.cuda()
+    ws = plan.new_workspace()
+
+    def route():
+        ids = torch.empty(cfg.N, cfg.K, dtype=torch.int32, device="cuda")
+        gates = torch.empty(cfg.N, cfg.K, dtype=torch.float32, device="cuda")
+        plan.router_topk(x, ids, gates, ws)
+        torch.cuda.synchronize()
+        return ids.cpu().numpy(), gates.cpu().double().numpy()
+
+    ids0, _ = route()
+    new_wr = torch.flip(inp.w_r, dims=[1]).contiguous()   # the experts in reverse order
+    w["w_r"].copy_(new_wr.cuda())
+    ids_stale, _ = route()
+    assert np.array_equal(ids_stale, ids0)
+    plan.refresh_router()
+    ids1, g1 = route()
+    rid, rg, _, logits = oracle.router(inp.x, oracle.DTYPE["bf16"], new_wr, None, cfg.K,
+                                       want_logits=True)
+    check_routing(ids1, g1, logits, rid, rg)
+    assert not np.array_equal(ids1, ids0)

@@ -75,6 +75,7 @@ def load(path: str = LIB_PATH):
         "moe_plan_create": ([ctypes.POINTER(LayerDesc), ctypes.POINTER(LayerWeights),
                              ctypes.POINTER(P)], ctypes.c_int),
         "moe_plan_destroy": ([P], ctypes.c_int),
+        "moe_plan_refresh_router": ([P, P], ctypes.c_int),
         "moe_workspace_size": ([P, ctypes.POINTER(sz)], ctypes.c_int),
         "moe_workspace_init": ([P, P, sz, P], ctypes.c_int),
         "moe_router_topk": ([P, P, P, P, P, P, sz, P], ctypes.c_int),
@@ -186,6 +187,12 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+    def refresh_router(self, stream=None):
+        """Re-derive the plan's copy of the router weights after w_r changed
+        in place (moe_plan_refresh_router)."""
+        _check(self.lib.moe_plan_refresh_router(self.handle, _stream(stream)),
+               "moe_plan_refresh_router")
 
     # -- workspace ---------------------------------------------------------
     def new_workspace(self, device=None):

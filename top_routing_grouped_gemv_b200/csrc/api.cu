@@ -25,7 +25,7 @@ constexpr int kMaxEvents = 16;
 constexpr int kHostEvents = 6;
 
 struct Layout {
-  size_t status = 0, chunk_counts = 0, h = 0, h_end = 0;
+  size_t status = 0, counter = 0, chunk_counts = 0, h = 0, h_end = 0;
   size_t ids = 0, gates = 0, pos = 0, src = 0, slot = 0, counts = 0, offsets = 0, x_perm = 0,
          y_perm = 0, tok_scale = 0, simt_part = 0;
   size_t fwd_end = 0, x_stage = 0, y_stage = 0, total = 0, x_stage_bytes = 0, y_stage_bytes = 0;
@@ -56,6 +56,9 @@ struct moe_plan_s {
   unsigned long long host_calls;  // host-buffer calls so far (selects the staging slot)
   uint8_t* sfb;  // MX plans: the weight scales in the tensor-core layout (owned)
   float* wgs;    // group / block plans: the weight scales, (E, d/128, F or F/128) (owned)
+  void* router_w;  // the router weights split for the tensor-core routers (owned), or NULL
+  int router_kind; // kRouterSimt, kRouterMma, kRouterTc
+  CUtensorMap tmRouterW;  // kRouterTc: TMA map of the split router weights
 };
 
 namespace {
@@ -85,12 +88,16 @@ void mark(moe_plan p, cudaStream_t s, const char* name_of_next) {
 
 bool uses_tensor_cores(const moe_layer_desc& d) { return d.dtype != MOE_F32; }
 
-// Router flavour of a plan: split-K SIMT for few tokens with long rows,
-// else tensor cores for bf16 tokens and many experts, else the per-token
-// SIMT kernels.
+enum RouterKind { kRouterSimt = 0, kRouterMma = 1, kRouterTc = 2 };
+
+// Router flavour of a plan: split-K SIMT for few tokens with long rows;
+// else, for bf16 tokens, the warp-MMA router (E <= 16) or the fused tcgen05
+// router (33..128 experts), both on the plan's split copy of w_r, or the
+// tcgen05 logits GEMM + top-K kernel on a per-call split in workspace
+// scratch (more than 128 experts); else the per-token SIMT kernels.
 bool router_splitk(const moe_layer_desc& d) { return router_uses_splitk(d.N, d.d); }
 bool router_on_tensor_cores(const moe_layer_desc& d) {
-  return !router_splitk(d) && d.dtype == MOE_BF16 && d.E >= kRouterTcMinExperts;
+  return !router_splitk(d) && d.dtype == MOE_BF16 && d.E > kRouterFusedMaxExperts;
 }
 
 void layout(moe_plan p) {
@@ -99,7 +106,9 @@ void layout(moe_plan p) {
   Layout L;
   size_t off = 0;
   L.status = off; off = align_up(off + 4);
-  L.chunk_counts = off; off = align_up(off + static_cast<size_t>(permute_chunks(d.N)) * d.E * 4);
+  L.counter = off; off = align_up(off + 4);  // the permute rank pass's last-CTA counter
+  // the rank pass's per-block expert histograms, then block bases
+  L.chunk_counts = off; off = align_up(off + permute_block_counts_bytes(d.N, d.E));
   L.permute_end = off;
   L.router_w3 = off;
   if (router_on_tensor_cores(d)) off = align_up(off + router_tc_scratch_bytes(d.N, d.d, d.E));
@@ -155,6 +164,18 @@ moe_status check_ws(moe_plan p, void* ws, size_t ws_bytes, size_t need) {
 moe_status run_router(moe_plan p, int n, const void* x, int32_t* ids, float* gates, float* margin,
                       void* ws, cudaStream_t s) {
   const moe_layer_desc& d = p->desc;
+  if (p->router_kind == kRouterMma) {
+    mark(p, s, "router_mma");
+    p->launches += 1;
+    return cuda_status(launch_router_mma(x, p->router_w, p->w.router_bias, n, d.d, d.E, d.K, ids,
+                                         gates, margin, s));
+  }
+  if (p->router_kind == kRouterTc) {
+    mark(p, s, "router_tc");
+    p->launches += 1;  // logits and top-K in one kernel
+    return cuda_status(launch_router_fused(x, p->tmRouterW, p->w.router_bias, n, d.d, d.E, d.K,
+                                           ids, gates, margin, at<int>(ws, p->L.status), s));
+  }
   if (router_on_tensor_cores(d)) {
     mark(p, s, "router_tc");
     p->launches += 3;  // weight split + logits + top-K
@@ -177,17 +198,15 @@ moe_status run_permute(moe_plan p, int n, const void* x, const int32_t* ids, int
   const moe_layer_desc& d = p->desc;
   int* status = at<int>(ws, p->L.status);
   int32_t* cc = at<int32_t>(ws, p->L.chunk_counts);
-  mark(p, s, "permute_count");
-  if (launch_permute_count(ids, n, d.K, d.E, cc, pos, status, s) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  mark(p, s, "permute_scan");
-  if (launch_permute_scan(cc, permute_chunks(n), d.E, counts, offsets, s) != cudaSuccess)
+  mark(p, s, "permute_rank");
+  if (launch_permute_rank(ids, n, d.K, d.E, cc, at<unsigned>(ws, p->L.counter), pos, counts,
+                          offsets, status, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   mark(p, s, "permute_gather");
   if (launch_permute_gather(x, d.d * p->ex, ids, n, d.K, d.E, cc, pos, src, slot, x_perm, status,
                             s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  p->launches += 3;
+  p->launches += 2;
   return MOE_OK;
 }
 
@@ -199,17 +218,15 @@ moe_status run_permute_quant(moe_plan p, int n, const void* x_bf16, const int32_
   const moe_layer_desc& d = p->desc;
   int* status = at<int>(ws, p->L.status);
   int32_t* cc = at<int32_t>(ws, p->L.chunk_counts);
-  mark(p, s, "permute_count");
-  if (launch_permute_count(ids, n, d.K, d.E, cc, pos, status, s) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  mark(p, s, "permute_scan");
-  if (launch_permute_scan(cc, permute_chunks(n), d.E, counts, offsets, s) != cudaSuccess)
+  mark(p, s, "permute_rank");
+  if (launch_permute_rank(ids, n, d.K, d.E, cc, at<unsigned>(ws, p->L.counter), pos, counts,
+                          offsets, status, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   mark(p, s, "permute_quant");
   if (launch_permute_quant(x_bf16, d.d, ids, n, d.K, d.E, cc, pos, src, slot, x_perm,
-                           token_scales, s) != cudaSuccess)
+                           token_scales, status, s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  p->launches += 3;
+  p->launches += 2;
   return MOE_OK;
 }
 
@@ -528,8 +545,41 @@ moe_status moe_plan_create(const moe_layer_desc* desc, const moe_layer_weights* 
   }
   for (int i = 0; i < kMaxEvents; ++i) p->ev[i] = nullptr;
   layout(p);
+  // the router weights, once, in the layout of the plan's tensor-core router
+  p->router_kind = kRouterSimt;
+  if (w->w_r && router_uses_mma(d.N, d.d, d.E, d.dtype)) p->router_kind = kRouterMma;
+  if (w->w_r && router_uses_fused_tc(d.N, d.d, d.E, d.dtype)) p->router_kind = kRouterTc;
+  if (p->router_kind != kRouterSimt) {
+    if (!device_accessible(w->w_r)) {
+      moe_plan_destroy(p);
+      return MOE_ERR_INVALID_ARG;
+    }
+    const size_t bytes = p->router_kind == kRouterMma ? router_mma_frag_bytes(d.d, d.E)
+                                                      : router_fused_weight_bytes(d.d, d.E);
+    cudaStream_t cs = nullptr;
+    bool ok = cudaMalloc(&p->router_w, bytes) == cudaSuccess;
+    ok = ok && (p->router_kind != kRouterTc ||
+                encode_router_fused_weights(&p->tmRouterW, p->router_w, d.d, d.E));
+    ok = ok && cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) == cudaSuccess;
+    ok = ok && moe_plan_refresh_router(p, cs) == MOE_OK;
+    ok = ok && cudaStreamSynchronize(cs) == cudaSuccess;
+    if (cs) cudaStreamDestroy(cs);
+    if (!ok) {
+      moe_plan_destroy(p);
+      return MOE_ERR_CUDA;
+    }
+  }
   *out = p;
   return MOE_OK;
+}
+
+moe_status moe_plan_refresh_router(moe_plan p, moe_stream_t stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (p->router_kind == kRouterSimt || !p->w.w_r) return MOE_OK;  // reads w_r on every call
+  const moe_layer_desc& d = p->desc;
+  if (p->router_kind == kRouterMma)
+    return cuda_status(launch_router_mma_frag(p->w.w_r, d.d, d.E, p->router_w, stream));
+  return cuda_status(launch_router_fused_split(p->w.w_r, d.d, d.E, p->router_w, stream));
 }
 
 moe_status moe_plan_destroy(moe_plan p) {
@@ -545,6 +595,7 @@ moe_status moe_plan_destroy(moe_plan p) {
   if (p->side) cudaStreamDestroy(p->side);
   if (p->sfb) cudaFree(p->sfb);
   if (p->wgs) cudaFree(p->wgs);
+  if (p->router_w) cudaFree(p->router_w);
   delete p;
   return MOE_OK;
 }
@@ -559,7 +610,8 @@ moe_status moe_workspace_init(moe_plan p, void* ws, size_t ws_bytes, moe_stream_
   if (!p) return MOE_ERR_INVALID_ARG;
   moe_status st = check_ws(p, ws, ws_bytes, p->L.chunk_counts);
   if (st != MOE_OK) return st;
-  return cuda_status(cudaMemsetAsync(ws, 0, 4, stream));
+  // the status word and the permute's counter
+  return cuda_status(cudaMemsetAsync(ws, 0, p->L.chunk_counts, stream));
 }
 
 moe_status moe_router_topk(moe_plan p, const void* x, int32_t* ids, float* gates, float* margin,

@@ -50,6 +50,18 @@ bool router_uses_splitk(int N, int d);
 int router_splitk_rows(int d, int E);
 size_t router_splitk_scratch_bytes(int N, int d, int E);
 
+// bf16 tokens and at most kRouterMmaMaxExperts experts (and not split-K):
+// logits on the warp-level tensor-core MMA from a fragment-ordered three-part
+// bf16 split of w_r made once per plan (launch_router_mma_frag, into
+// router_mma_frag_bytes of device memory).
+constexpr int kRouterMmaMaxExperts = 16;
+bool router_uses_mma(int N, int d, int E, int x_dtype);
+size_t router_mma_frag_bytes(int d, int E);
+cudaError_t launch_router_mma_frag(const float* w_r, int d, int E, void* frag, cudaStream_t stream);
+cudaError_t launch_router_mma(const void* x, const void* frag, const float* bias, int N, int d,
+                              int E, int K, int32_t* ids, float* gates, float* margin,
+                              cudaStream_t stream);
+
 // Top-K, softmax and margin of fp32 logits (N, E) in memory, plus bias.
 cudaError_t launch_logits_topk(const float* logits, const float* bias, int N, int E, int K,
                               int32_t* ids, float* gates, float* margin, cudaStream_t stream);
@@ -63,21 +75,44 @@ cudaError_t launch_router_tc(const void* x, const float* w_r, const float* bias,
                              void* scratch, int* status, cudaStream_t stream);
 // Experts above which bf16 routers run on the tensor cores.
 constexpr int kRouterTcMinExperts = 33;
+// bf16 tokens with 33..kRouterFusedMaxExperts experts (and not split-K): one
+// kernel computes the logits on tcgen05 from the plan's split router weights
+// (launch_router_fused_split into router_fused_weight_bytes of device memory,
+// TMA map from encode_router_fused_weights) and takes the top-K in its
+// epilogue.  More experts use launch_router_tc.
+constexpr int kRouterFusedMaxExperts = 128;
+bool router_uses_fused_tc(int N, int d, int E, int x_dtype);
+size_t router_fused_weight_bytes(int d, int E);
+cudaError_t launch_router_fused_split(const float* w_r, int d, int E, void* out,
+                                      cudaStream_t stream);
+bool encode_router_fused_weights(CUtensorMap* map, const void* split, int d, int E);
+cudaError_t launch_router_fused(const void* x, const CUtensorMap& tmW, const float* bias, int N,
+                                int d, int E, int K, int32_t* ids, float* gates, float* margin,
+                                int* status, cudaStream_t stream);
 
 // ---- permute ----------------------------------------------------------------
-constexpr int kPermuteChunk = 32;  // tokens per chunk of the stable counting pass
-inline int permute_chunks(int N) { return (N + kPermuteChunk - 1) / kPermuteChunk; }
+constexpr int kPermuteChunk = 32;   // tokens ranked by one warp (lane = token)
+constexpr int kPermuteBlock = 256;  // tokens per rank CTA: its expert histogram is one row
+inline int permute_blocks(int N) { return (N + kPermuteBlock - 1) / kPermuteBlock; }
+// Device scratch of the rank pass: the block histograms (then bases) and the
+// last-CTA counter (one unsigned, zero between calls).
+inline size_t permute_block_counts_bytes(int N, int E) {
+  return static_cast<size_t>(permute_blocks(N) > 0 ? permute_blocks(N) : 1) * E * 4;
+}
 
-// Writes each (t, j)'s rank within its 32-token chunk to local_rank (the
-// perm_pos buffer; the gather turns it into the final position) and the
-// chunk's expert histogram to chunk_counts.
-cudaError_t launch_permute_count(const int32_t* ids, int N, int K, int E, int32_t* chunk_counts,
-                                 int32_t* local_rank, int* status, cudaStream_t stream);
-cudaError_t launch_permute_scan(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
-                                int32_t* offsets, cudaStream_t stream);
-// pos holds the ranks from launch_permute_count on entry, the final
+// Writes each (t, j)'s rank within its 256-token block to local_rank (the
+// perm_pos buffer; the gather turns it into the final position), the blocks'
+// expert histograms to block_counts, and -- in the last CTA to finish, found
+// through *counter, which must be zero on entry and is zero again on exit --
+// the per-(block, expert) first destination rows (over block_counts), the
+// expert counts and the offsets (E + 1).
+cudaError_t launch_permute_rank(const int32_t* ids, int N, int K, int E, int32_t* block_counts,
+                                unsigned* counter, int32_t* local_rank, int32_t* counts,
+                                int32_t* offsets, int* status, cudaStream_t stream);
+// pos holds the ranks from launch_permute_rank on entry, the final
 // positions on exit; src[pos] = t and, when slot is non-null,
-// slot[pos] = t*K + j.
+// slot[pos] = t*K + j.  chunk_base = the block bases from the rank pass; a
+// position outside [0, N*K) is recorded in status and skipped.
 cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* ids, int N, int K,
                                   int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
                                   int32_t* slot, void* x_perm, int* status, cudaStream_t stream);
@@ -86,7 +121,7 @@ cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* i
 // d % 16 == 0; x_perm gets e4m3 codes (N*K, d), token_scale (N) the scales.
 cudaError_t launch_permute_quant(const void* x_bf16, int d, const int32_t* ids, int N, int K,
                                  int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
-                                 int32_t* slot, void* x_perm_e4m3, float* token_scale,
+                                 int32_t* slot, void* x_perm_e4m3, float* token_scale, int* status,
                                  cudaStream_t stream);
 
 // ---- combine / unpermute ----------------------------------------------------

@@ -6,21 +6,25 @@
 //
 // Stable order: within expert e the rows appear in (token, slot) order, so
 //   pos[t,j] = offsets[e] + #{(t',j') before (t,j) with ids[t',j'] = e}.
-// Tokens are cut into chunks of kPermuteChunk (32).  Three launches:
-//   1. rank:   one warp per chunk ranks the chunk's (t, j) pairs: each lane
-//              (token) sets its bit in a per-expert 32-bit mask, and the
-//              rank of (t, j) is the number of lower lanes in the mask of
-//              its expert (a token whose K experts are not distinct takes a
-//              shuffle-based count instead); writes each pair's rank within
-//              its chunk (into perm_pos) and the chunk's expert histogram
-//              (chunk_counts).  Either way the order is fixed.
-//   2. scan:   one CTA turns chunk_counts into per-(chunk, expert) bases
-//              (offsets[e] + rows of e in earlier chunks), counts, offsets
-//   3. gather: one warp per token turns its ranks into final positions and
-//              copies the token row once from HBM into its K destination
-//              rows with 16-byte vector loads/stores (and, on request, notes
-//              each position's flat slot t*K + j for an unpermute done by
-//              the grouped GEMM's stores).
+// Tokens are cut into chunks of kPermuteChunk (32) and blocks of
+// kPermuteBlock (256 = eight chunks).  Two launches:
+//   1. rank:   one CTA of eight warps per block, one warp per chunk: each
+//              lane (token) sets its bit in a per-expert 32-bit mask of its
+//              warp, and the rank of (t, j) within the chunk is the number of
+//              lower lanes in the mask of its expert (a token whose K experts
+//              are not distinct takes a shuffle-based count instead); the
+//              chunks' histograms are scanned over the block's eight chunks,
+//              so each pair's rank within its block goes to perm_pos and the
+//              block's expert histogram to block_counts.  The last CTA to
+//              finish (an atomic counter, reset for the next call) scans the
+//              block histograms into per-(block, expert) bases (offsets[e] +
+//              rows of e in earlier blocks), counts and offsets.  Either way
+//              the order is fixed.
+//   2. gather: one warp per token turns its ranks into final positions
+//              (checked against N*K) and copies the token row once from HBM
+//              into its K destination rows with 16-byte vector loads/stores
+//              (and, on request, notes each position's flat slot t*K + j for
+//              an unpermute done by the grouped GEMM's stores).
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -30,39 +34,133 @@ namespace moe {
 namespace {
 
 constexpr int CH = kPermuteChunk;
+constexpr int BT = kPermuteBlock;
+constexpr int kRankWarps = BT / CH;  // chunks (warps) per block
+static_assert(kRankWarps * 32 == 256, "one rank CTA = 256 threads");
 
-// One warp per chunk of 32 tokens; lane = token.
+// Exclusive scan of the block histograms bc (nblk, E) over blocks, per
+// expert, by the 256 threads of one CTA; afterwards bc[b][e] holds the first
+// destination row of block b's rows of expert e, and counts / offsets the
+// expert totals and their exclusive scan (offsets[E] = the rows).  Thread
+// (e, s) owns expert e and a contiguous slice s of the blocks; part and
+// total are 256 and 257 ints of shared memory.  bc is read through L2 (it
+// was written by other CTAs).
+__device__ __forceinline__ void scan_block_counts(int32_t* __restrict__ bc, int nblk, int E,
+                                                  int32_t* __restrict__ counts,
+                                                  int32_t* __restrict__ offsets, int* part,
+                                                  int* total) {
+  int Ep = 1;
+  while (Ep < E) Ep <<= 1;
+  const int S = 256 / Ep;  // slices per expert (>= 1 for E <= 256)
+  const int e = threadIdx.x % Ep, sl = threadIdx.x / Ep;
+  const int cs = (nblk + S - 1) / S;
+  const int c0 = sl * cs, c1 = min(nblk, c0 + cs);
+  int sum = 0;
+  if (e < E) {
+    int c = c0;
+    for (; c + 8 <= c1; c += 8) {  // eight loads in flight
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(bc + (long long)(c + u) * E + e);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sum += v[u];
+    }
+    for (; c < c1; ++c) sum += __ldcg(bc + (long long)c * E + e);
+  }
+  part[threadIdx.x] = sum;
+  __syncthreads();
+  if (threadIdx.x < E) {  // over the slices of each expert
+    int run = 0;
+    for (int q = 0; q < S; ++q) {
+      const int v = part[q * Ep + threadIdx.x];
+      part[q * Ep + threadIdx.x] = run;
+      run += v;
+    }
+    total[threadIdx.x] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {  // over the experts (E <= 256: up to 8 per lane)
+    const int lane = threadIdx.x;
+    const int per = (E + 31) / 32;
+    const int b0 = min(E, lane * per), b1 = min(E, b0 + per);
+    int local = 0;
+    for (int q = b0; q < b1; ++q) local += total[q];
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int run = incl - local;
+    for (int q = b0; q < b1; ++q) {
+      const int c = total[q];
+      counts[q] = c;
+      offsets[q] = run;
+      total[q] = run;
+      run += c;
+    }
+    if (lane == 31) offsets[E] = incl;
+  }
+  __syncthreads();
+  if (e < E) {
+    int run = total[e] + part[sl * Ep + e];
+    int c = c0;
+    for (; c + 8 <= c1; c += 8) {  // eight loads in flight, then the eight bases
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(bc + (long long)(c + u) * E + e);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        bc[(long long)(c + u) * E + e] = run;
+        run += v[u];
+      }
+    }
+    for (; c < c1; ++c) {
+      int32_t* q = bc + (long long)c * E + e;
+      const int v = __ldcg(q);
+      *q = run;
+      run += v;
+    }
+  }
+}
+
+// One CTA per block of 256 tokens, one warp per 32-token chunk (lane =
+// token); the last CTA also runs the scan.  At most 40 registers a thread:
+// a CTA (8 warps, 10 K registers, 18 KB of shared memory) then fits on an SM
+// beside one CTA of a persistent tensor-core GEMM (the shared expert running
+// on a forked stream) instead of waiting for that GEMM to end.
 template <int KMAX>
-__global__ void __launch_bounds__(128)
+__global__ void __maxnreg__(40)
 permute_rank_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
-                    int32_t* __restrict__ chunk_counts, int32_t* __restrict__ local_rank,
-                    int* status) {
+                    int32_t* __restrict__ block_counts, unsigned* __restrict__ counter,
+                    int32_t* __restrict__ local_rank, int32_t* __restrict__ counts,
+                    int32_t* __restrict__ offsets, int* status) {
   griddep_trigger();  // let the next kernel of the stream start launching
   griddep_wait();     // inputs written by the previous kernel are visible
 
-  __shared__ int hist[4][256];
-  __shared__ unsigned lanes_of[4][256];  // bit l: lane (token) l routes to the expert
+  __shared__ int hist[kRankWarps][256];
+  __shared__ unsigned lanes_of[kRankWarps][256];  // bit l: lane (token) l routes to the expert
+  __shared__ int s_part[256];
+  __shared__ int s_total[257];
+  __shared__ int s_last;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int c = blockIdx.x * 4 + warp;
-  const int nchunks = (N + CH - 1) / CH;
-  if (c >= nchunks) return;  // whole warp
   for (int e = lane; e < E; e += 32) {
     hist[warp][e] = 0;
     lanes_of[warp][e] = 0u;
   }
   __syncwarp();
-  const int t = c * CH + lane;
+  const long long t = (static_cast<long long>(blockIdx.x) * kRankWarps + warp) * CH + lane;
   int my[KMAX];
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
     my[j] = -1;
     if (j < K && t < N) {
-      const int e = ids[(long long)t * K + j];
+      const int e = ids[t * K + j];
       if (e >= 0 && e < E) my[j] = e;
       else set_status(status, kStatusBadIndex);
     }
   }
-  // rank of (t, j): earlier slots of t with the same expert ...
+  // rank of (t, j) in its chunk: earlier slots of t with the same expert ...
   int rank[KMAX];
   bool repeated = false;
 #pragma unroll
@@ -101,106 +199,35 @@ permute_rank_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
     }
   }
 #pragma unroll
+  for (int j = 0; j < KMAX; ++j)
+    if (j < K && my[j] >= 0) atomicAdd(&hist[warp][my[j]], 1);  // integer counts: order-independent
+  __syncthreads();
+  // the chunks' histograms -> exclusive prefix over the block's chunks
+  for (int e = threadIdx.x; e < E; e += 256) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kRankWarps; ++w) {
+      const int v = hist[w][e];
+      hist[w][e] = run;
+      run += v;
+    }
+    block_counts[static_cast<long long>(blockIdx.x) * E + e] = run;
+  }
+  __syncthreads();
+#pragma unroll
   for (int j = 0; j < KMAX; ++j) {
     if (j >= K) break;
-    if (t < N) local_rank[(long long)t * K + j] = my[j] >= 0 ? rank[j] : -1;
-    if (my[j] >= 0) atomicAdd(&hist[warp][my[j]], 1);  // integer counts: order-independent
+    if (t < N) local_rank[t * K + j] = my[j] >= 0 ? hist[warp][my[j]] + rank[j] : -1;
   }
-  __syncwarp();
-  for (int e = lane; e < E; e += 32) chunk_counts[(long long)c * E + e] = hist[warp][e];
-}
-
-// One CTA of 1024 threads.  Thread (e, s) owns expert e and a contiguous
-// slice s of the chunks.  Afterwards chunk_counts[c][e] holds the first
-// destination row of chunk c's rows of expert e.
-// At most 40 registers a thread: the 1024 threads (eight warps on each SM
-// sub-partition, 10 K of its 16 K registers) then fit on an SM beside one CTA
-// of a persistent tensor-core GEMM (the shared expert running on a forked
-// stream, two warps of 72 registers on a sub-partition), instead of waiting
-// for that GEMM to end.
-__global__ void __maxnreg__(40)
-permute_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
-                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
-  griddep_trigger();  // let the next kernel of the stream start launching
-  griddep_wait();     // inputs written by the previous kernel are visible
-
-  __shared__ int part[1024];
-  __shared__ int total[257];
-  int Ep = 1;
-  while (Ep < E) Ep <<= 1;
-  const int S = 1024 / Ep;                 // slices per expert (>= 4 for E <= 256)
-  const int e = threadIdx.x % Ep, s = threadIdx.x / Ep;
-  const int cs = (nchunks + S - 1) / S;
-  const int c0 = s * cs, c1 = min(nchunks, c0 + cs);
-  // (chunk loops batched by 8 so that loads overlap)
-  int sum = 0;
-  if (e < E) {
-    int c = c0;
-    for (; c + 8 <= c1; c += 8) {
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = chunk_counts[(long long)(c + u) * E + e];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) sum += v[u];
-    }
-    for (; c < c1; ++c) sum += chunk_counts[(long long)c * E + e];
-  }
-  part[threadIdx.x] = sum;
+  // the last CTA to get here scans every block's histogram
+  __threadfence();
   __syncthreads();
-  // exclusive scan over the slices of each expert
-  if (threadIdx.x < E) {
-    int run = 0;
-    for (int q = 0; q < S; ++q) {
-      int v = part[q * Ep + threadIdx.x];
-      part[q * Ep + threadIdx.x] = run;
-      run += v;
-    }
-    total[threadIdx.x] = run;
-  }
+  if (threadIdx.x == 0) s_last = atomicAdd(counter, 1u) == gridDim.x - 1;
   __syncthreads();
-  // exclusive scan over experts (warp 0; E <= 256 -> up to 8 per lane)
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    const int per = (E + 31) / 32;
-    const int b0 = lane * per, b1 = min(E, b0 + per);
-    int local = 0;
-    for (int q = b0; q < b1; ++q) local += total[q];
-    int incl = local;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    int run = incl - local;
-    for (int q = b0; q < b1; ++q) {
-      int c = total[q];
-      counts[q] = c;
-      offsets[q] = run;
-      total[q] = run;
-      run += c;
-    }
-    if (lane == 31) offsets[E] = incl;
-  }
-  __syncthreads();
-  if (e < E) {
-    int run = total[e] + part[s * Ep + e];
-    int c = c0;
-    for (; c + 8 <= c1; c += 8) {
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = chunk_counts[(long long)(c + u) * E + e];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        chunk_counts[(long long)(c + u) * E + e] = run;
-        run += v[u];
-      }
-    }
-    for (; c < c1; ++c) {
-      const int v = chunk_counts[(long long)c * E + e];
-      chunk_counts[(long long)c * E + e] = run;
-      run += v;
-    }
-  }
+  if (!s_last) return;
+  __threadfence();
+  scan_block_counts(block_counts, static_cast<int>(gridDim.x), E, counts, offsets, s_part, s_total);
+  if (threadIdx.x == 0) *counter = 0u;  // ready for the next call (stream-ordered)
 }
 
 // WPT warps per token (8 / WPT tokens per CTA): final positions from the
@@ -213,7 +240,7 @@ __global__ void __launch_bounds__(256)
 permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* __restrict__ ids,
                       int N, int K, int E, const int32_t* __restrict__ chunk_base,
                       int32_t* __restrict__ pos, int32_t* __restrict__ src,
-                      int32_t* __restrict__ slot, uint4* __restrict__ x_perm) {
+                      int32_t* __restrict__ slot, uint4* __restrict__ x_perm, int* status) {
   griddep_trigger();  // let the next kernel of the stream start launching
   griddep_wait();     // inputs written by the previous kernel are visible
 
@@ -226,11 +253,16 @@ permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* 
     if (lane < K) {
       const long long i = (long long)t * K + lane;
       const int e = ids[i];
-      const int r = pos[i];  // rank within the chunk (written by the rank pass)
+      const int r = pos[i];  // rank within the block (written by the rank pass)
       if (r >= 0 && e >= 0 && e < E) {
-        mine = chunk_base[(long long)(t / CH) * E + e] + r;
-        src[mine] = t;
-        if (slot) slot[mine] = static_cast<int32_t>(i);
+        mine = chunk_base[(long long)(t / BT) * E + e] + r;
+        if (mine < 0 || mine >= N * K) {  // only a damaged workspace gets here
+          set_status(status, kStatusBadIndex);
+          mine = -1;
+        } else {
+          src[mine] = t;
+          if (slot) slot[mine] = static_cast<int32_t>(i);
+        }
       }
       pos[i] = mine;
     }
@@ -287,7 +319,7 @@ permute_quant_kernel(const uint4* __restrict__ x, int d, const int32_t* __restri
                      int K, int E, const int32_t* __restrict__ chunk_base,
                      int32_t* __restrict__ pos, int32_t* __restrict__ src,
                      int32_t* __restrict__ slot, uint4* __restrict__ x_perm,
-                     float* __restrict__ token_scale) {
+                     float* __restrict__ token_scale, int* status) {
   griddep_trigger();  // let the next kernel of the stream start launching
   griddep_wait();     // inputs written by the previous kernel are visible
 
@@ -302,11 +334,16 @@ permute_quant_kernel(const uint4* __restrict__ x, int d, const int32_t* __restri
     if (lane < K) {
       const long long i = (long long)t * K + lane;
       const int e = ids[i];
-      const int r = pos[i];  // rank within the chunk (written by the rank pass)
+      const int r = pos[i];  // rank within the block (written by the rank pass)
       if (r >= 0 && e >= 0 && e < E) {
-        mine = chunk_base[(long long)(t / CH) * E + e] + r;
-        src[mine] = t;
-        if (slot) slot[mine] = static_cast<int32_t>(i);
+        mine = chunk_base[(long long)(t / BT) * E + e] + r;
+        if (mine < 0 || mine >= N * K) {  // only a damaged workspace gets here
+          set_status(status, kStatusBadIndex);
+          mine = -1;
+        } else {
+          src[mine] = t;
+          if (slot) slot[mine] = static_cast<int32_t>(i);
+        }
       }
       pos[i] = mine;
     }
@@ -360,89 +397,83 @@ permute_quant_kernel(const uint4* __restrict__ x, int d, const int32_t* __restri
 template <int KMAX>
 void launch_quant_k(const uint4* xv, int d, const int32_t* ids, int N, int K, int E,
                     const int32_t* chunk_base, int32_t* pos, int32_t* src, int32_t* slot, uint4* xp,
-                    float* scales, cudaStream_t stream) {
+                    float* scales, int* status, cudaStream_t stream) {
   const int wpt = warps_per_token(N);
   const dim3 grid((N + 8 / wpt - 1) / (8 / wpt));
   if (wpt == 1)
-    launch_pdl(permute_quant_kernel<KMAX, 1>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales);
+    launch_pdl(permute_quant_kernel<KMAX, 1>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales, status);
   else if (wpt == 2)
-    launch_pdl(permute_quant_kernel<KMAX, 2>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales);
+    launch_pdl(permute_quant_kernel<KMAX, 2>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales, status);
   else if (wpt == 4)
-    launch_pdl(permute_quant_kernel<KMAX, 4>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales);
+    launch_pdl(permute_quant_kernel<KMAX, 4>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales, status);
   else
-    launch_pdl(permute_quant_kernel<KMAX, 8>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales);
+    launch_pdl(permute_quant_kernel<KMAX, 8>, grid, dim3(256), 0, stream, xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, scales, status);
 }
 
 template <int KMAX>
 void launch_gather_k(const uint4* xv, int row_vecs, const int32_t* ids, int N, int K, int E,
                      const int32_t* chunk_base, int32_t* pos, int32_t* src, int32_t* slot,
-                     uint4* xp, cudaStream_t stream) {
+                     uint4* xp, int* status, cudaStream_t stream) {
   const int wpt = warps_per_token(N);
   const int tpc = 8 / wpt;
   const dim3 grid((N + tpc - 1) / tpc);
   if (wpt == 1)
-    launch_pdl(permute_gather_kernel<KMAX, 1>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp);
+    launch_pdl(permute_gather_kernel<KMAX, 1>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, status);
   else if (wpt == 2)
-    launch_pdl(permute_gather_kernel<KMAX, 2>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp);
+    launch_pdl(permute_gather_kernel<KMAX, 2>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, status);
   else if (wpt == 4)
-    launch_pdl(permute_gather_kernel<KMAX, 4>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp);
+    launch_pdl(permute_gather_kernel<KMAX, 4>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, status);
   else
-    launch_pdl(permute_gather_kernel<KMAX, 8>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp);
+    launch_pdl(permute_gather_kernel<KMAX, 8>, grid, dim3(256), 0, stream, xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, status);
 }
 
 }  // namespace
 
-cudaError_t launch_permute_count(const int32_t* ids, int N, int K, int E, int32_t* chunk_counts,
-                                 int32_t* local_rank, int* status, cudaStream_t stream) {
-  const int nchunks = permute_chunks(N);
-  if (nchunks == 0) return cudaSuccess;
-  const int grid = (nchunks + 3) / 4;
+cudaError_t launch_permute_rank(const int32_t* ids, int N, int K, int E, int32_t* block_counts,
+                                unsigned* counter, int32_t* local_rank, int32_t* counts,
+                                int32_t* offsets, int* status, cudaStream_t stream) {
+  // at least one CTA, so that counts and offsets are written for zero tokens
+  const int grid = permute_blocks(N) > 0 ? permute_blocks(N) : 1;
   if (K <= 2)
-    launch_pdl(permute_rank_kernel<2>, dim3(grid), dim3(128), 0, stream, ids, N, K, E, chunk_counts, local_rank, status);
-  else if (K <= 4)
-    launch_pdl(permute_rank_kernel<4>, dim3(grid), dim3(128), 0, stream, ids, N, K, E, chunk_counts, local_rank, status);
-  else
-    launch_pdl(permute_rank_kernel<8>, dim3(grid), dim3(128), 0, stream, ids, N, K, E, chunk_counts, local_rank, status);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_permute_scan(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
-                                int32_t* offsets, cudaStream_t stream) {
-  launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, stream, chunk_counts, nchunks, E, counts, offsets);
-  return cudaGetLastError();
+    return launch_pdl(permute_rank_kernel<2>, dim3(grid), dim3(256), 0, stream, ids, N, K, E,
+                      block_counts, counter, local_rank, counts, offsets, status);
+  if (K <= 4)
+    return launch_pdl(permute_rank_kernel<4>, dim3(grid), dim3(256), 0, stream, ids, N, K, E,
+                      block_counts, counter, local_rank, counts, offsets, status);
+  return launch_pdl(permute_rank_kernel<8>, dim3(grid), dim3(256), 0, stream, ids, N, K, E,
+                    block_counts, counter, local_rank, counts, offsets, status);
 }
 
 cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* ids, int N, int K,
                                   int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
                                   int32_t* slot, void* x_perm, int* status, cudaStream_t stream) {
-  (void)status;  // bad ids were recorded by the rank pass
   if (N == 0) return cudaSuccess;
   const int row_vecs = row_bytes / 16;
   auto xv = static_cast<const uint4*>(x);
   auto xp = static_cast<uint4*>(x_perm);
   if (K <= 2)
-    launch_gather_k<2>(xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, stream);
+    launch_gather_k<2>(xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, status, stream);
   else if (K <= 4)
-    launch_gather_k<4>(xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, stream);
+    launch_gather_k<4>(xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, status, stream);
   else
-    launch_gather_k<8>(xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, stream);
+    launch_gather_k<8>(xv, row_vecs, ids, N, K, E, chunk_base, pos, src, slot, xp, status, stream);
   return cudaGetLastError();
 }
 
 cudaError_t launch_permute_quant(const void* x_bf16, int d, const int32_t* ids, int N, int K,
                                  int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
-                                 int32_t* slot, void* x_perm_e4m3, float* token_scale,
+                                 int32_t* slot, void* x_perm_e4m3, float* token_scale, int* status,
                                  cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
   if (d % 16) return cudaErrorInvalidValue;
   auto xv = static_cast<const uint4*>(x_bf16);
   auto xp = static_cast<uint4*>(x_perm_e4m3);
   if (K <= 2)
-    launch_quant_k<2>(xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, token_scale, stream);
+    launch_quant_k<2>(xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, token_scale, status, stream);
   else if (K <= 4)
-    launch_quant_k<4>(xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, token_scale, stream);
+    launch_quant_k<4>(xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, token_scale, status, stream);
   else
-    launch_quant_k<8>(xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, token_scale, stream);
+    launch_quant_k<8>(xv, d, ids, N, K, E, chunk_base, pos, src, slot, xp, token_scale, status, stream);
   return cudaGetLastError();
 }
 

@@ -23,9 +23,14 @@ namespace {
 
 constexpr size_t kScratchBytes = size_t(1) << 20;
 
-// Per-chunk expert counts, then (after the scan) per-chunk expert bases.
-// Every call writes all ceil(N/32)*E entries it later reads, so no entry has
-// to start at zero.
+constexpr size_t kCounterBytes = 256;  // the counter, alone in the array's first 256 bytes
+
+// First 256 bytes: the rank pass's last-CTA counter, which must be zero when
+// a call starts.  A __device__ array starts zeroed when the module loads, and
+// every call's last CTA sets the counter back to zero.  Then the per-block
+// expert counts, and after the scan the per-block expert bases: every call
+// writes all ceil(N/256)*E entries that it later reads, so these need no
+// clearing.
 static __device__ __align__(256) int32_t g_permute_scratch[kScratchBytes / sizeof(int32_t)];
 
 // Device address of g_permute_scratch on the current device.
@@ -52,24 +57,24 @@ extern "C" moe_status moe_permute_noalloc(moe_plan plan, const void* x, const in
   if (!x || !topk_ids || !counts || !offsets || !perm_pos || !perm_src || !x_perm)
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
-  const int nchunks = moe::permute_chunks(N);
-  if (static_cast<size_t>(nchunks) * E * sizeof(int32_t) > kScratchBytes)
+  if (kCounterBytes + moe::permute_block_counts_bytes(N, E) > kScratchBytes)
     return MOE_ERR_WORKSPACE_TOO_SMALL;
   int32_t* scratch = nullptr;
   moe_status st = scratch_on_current_device(&scratch);
   if (st != MOE_OK) return st;
   cudaStream_t s = stream;
   int* status = device_status_or_null;
-  // the same three kernels as moe_permute, recorded in the plan's launch
-  // count and stage events like that call
+  // the same two kernels as moe_permute, recorded in the plan's launch count
+  // and stage events like that call
+  unsigned* counter = reinterpret_cast<unsigned*>(scratch);
+  int32_t* block_counts = scratch + kCounterBytes / sizeof(int32_t);
   moe::plan_call_begin(plan);
-  moe::plan_call_mark(plan, s, "permute_count");
-  bool ok = moe::launch_permute_count(topk_ids, N, K, E, scratch, perm_pos, status, s) == cudaSuccess;
-  moe::plan_call_mark(plan, s, "permute_scan");
-  ok = ok && moe::launch_permute_scan(scratch, nchunks, E, counts, offsets, s) == cudaSuccess;
+  moe::plan_call_mark(plan, s, "permute_rank");
+  bool ok = moe::launch_permute_rank(topk_ids, N, K, E, block_counts, counter, perm_pos, counts,
+                                     offsets, status, s) == cudaSuccess;
   moe::plan_call_mark(plan, s, "permute_gather");
-  ok = ok && moe::launch_permute_gather(x, row_bytes, topk_ids, N, K, E, scratch, perm_pos, perm_src,
-                                        nullptr, x_perm, status, s) == cudaSuccess;
-  moe::plan_call_end(plan, s, 3);
+  ok = ok && moe::launch_permute_gather(x, row_bytes, topk_ids, N, K, E, block_counts, perm_pos,
+                                        perm_src, nullptr, x_perm, status, s) == cudaSuccess;
+  moe::plan_call_end(plan, s, 2);
   return ok ? MOE_OK : MOE_ERR_CUDA;
 }

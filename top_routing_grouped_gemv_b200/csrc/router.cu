@@ -561,6 +561,172 @@ cudaError_t launch_t(const TX* x, const float* w_r, const float* bias, int N, in
   return launch_epl<TX, 8>(x, w_r, bias, N, d, E, K, ids, gates, margin, stream);
 }
 
+// ---- bf16 tokens, few experts: the logits on the warp-level tensor-core MMA ----
+//
+// For a handful of experts (E <= 16) the router reads N*d*2 bytes of tokens
+// and does 8 FLOP per byte: the fp32 FMA form above spends more issue slots
+// on its multiply-adds and weight loads than the tokens take to stream from
+// HBM.  Here the contraction runs on mma.sync m16n8k16 (bf16 in, fp32
+// accumulate), one instruction per 16 tokens x 8 experts x 16 k, so the
+// kernel is bound by the token stream.  fp32-level logits come from the same
+// exact three-part split as the tcgen05 router:
+//   w = hi + mid + lo,  hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid),
+// each part in its own fp32 accumulator (bf16 x bf16 products are exact in
+// fp32), logit = (hi + mid) + lo.
+//
+// Work split: a CTA owns G groups of 16 tokens; its 8G warps are (group,
+// k-slice) pairs, the reduction dimension cut into 8 slices of 32-element
+// blocks, so every warp issues all the 16-byte token loads of its slice at
+// once (16 rows x 256 elements for d = 2048).  The slices' partial logits
+// meet in shared memory and are added in slice order (fixed: deterministic);
+// then one warp per token takes the top-K as in the other routers.
+//
+// k order inside a 32-element block.  Thread (g, c) of a warp (g = lane / 4,
+// c = lane % 4) loads 8 consecutive elements 8c..8c+7 of token rows g and
+// g+8 as one 16-byte vector each.  The MMA's A fragment wants that thread to
+// hold logical k positions {2c, 2c+1, 2c+8, 2c+9}; the sum over k does not
+// depend on which physical k sits at which logical position as long as A and
+// B agree, so the first MMA of a block takes physical k = 8c + {0,1,2,3} and
+// the second 8c + {4,5,6,7}.  The weights are stored in exactly that order
+// (router_frag_kernel): entry ((b * NT + nt) * 3 + part) * 32 + lane is the
+// 16-byte vector W_part[32b + 8c + i][8nt + g], i = 0..7.
+
+constexpr int kMmaSlices = 8;   // warps (k slices) per 16-token group
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Token rows are read once: keep them out of L1 so the weights stay there.
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// w_r (d, E) fp32 -> fragment-ordered three-part bf16 split (see above), for
+// nb = ceil(d / 32) blocks and NT = ceil(E / 8) expert tiles; entries past d
+// or E are zero.  One thread per 16-byte entry.
+__global__ void __launch_bounds__(256)
+router_frag_kernel(const float* __restrict__ w_r, int d, int E, int nb, int NT,
+                   uint4* __restrict__ frag) {
+  const long long n = static_cast<long long>(nb) * NT * 3 * 32;
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int lane = static_cast<int>(i % 32);
+  const int part = static_cast<int>((i / 32) % 3);
+  const int nt = static_cast<int>((i / 96) % NT);
+  const int b = static_cast<int>(i / (96LL * NT));
+  const int g = lane >> 2, c = lane & 3;
+  const int e = 8 * nt + g;
+  uint32_t h[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int k = 32 * b + 8 * c + q;
+    const float w = (k < d && e < E) ? w_r[static_cast<long long>(k) * E + e] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    const __nv_bfloat16 v = part == 0 ? hi : part == 1 ? mid : lo;
+    h[q] = static_cast<uint32_t>(__bfloat16_as_ushort(v));
+  }
+  frag[i] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
+                       h[6] | (h[7] << 16));
+}
+
+// XB: 32-element blocks whose token vectors are loaded before their MMAs
+// (2 * XB 16-byte loads in flight per thread; fewer for two expert tiles,
+// whose accumulators take the registers).
+template <int NT, int G, int XB = (NT == 1 ? 8 : 4)>
+__global__ void __launch_bounds__(32 * kMmaSlices * G)
+router_mma_kernel(const __nv_bfloat16* __restrict__ x, const uint4* __restrict__ frag,
+                  const float* __restrict__ bias, int N, int d, int E, int K, int nb, int bps,
+                  int32_t* __restrict__ ids, float* __restrict__ gates,
+                  float* __restrict__ margin) {
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
+  constexpr int EW = 8 * NT;  // expert columns
+  __shared__ float part_s[G][kMmaSlices][16][EW];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gi = warp / kMmaSlices, ks = warp % kMmaSlices;
+  const int g = lane >> 2, c = lane & 3;
+  const long long t0 = (static_cast<long long>(blockIdx.x) * G + gi) * 16;
+  const long long ta = t0 + g, tb = t0 + g + 8;
+  const int rv = d / 8;  // 16-byte vectors per token row (d % 8 == 0)
+  const uint4* xa = reinterpret_cast<const uint4*>(x) + (ta < N ? ta : 0) * rv;
+  const uint4* xb = reinterpret_cast<const uint4*>(x) + (tb < N ? tb : 0) * rv;
+
+  float acc[3][NT][4];
+#pragma unroll
+  for (int p = 0; p < 3; ++p)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[p][nt][q] = 0.f;
+
+  const int b0 = ks * bps, b1 = min(nb, b0 + bps);
+  for (int bb = b0; bb < b1; bb += XB) {
+    // the token vectors of up to XB blocks in flight before any MMA
+    uint4 ua[XB], ub[XB];
+#pragma unroll
+    for (int i = 0; i < XB; ++i) {
+      const int v = 4 * (bb + i) + c;  // vector index of elements 32(bb+i) + 8c ..
+      const bool in = bb + i < b1 && v < rv;
+      ua[i] = (in && ta < N) ? ld_stream(xa + v) : make_uint4(0u, 0u, 0u, 0u);
+      ub[i] = (in && tb < N) ? ld_stream(xb + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < XB; ++i) {
+      const int b = bb + i;
+      if (b >= b1) break;  // warp-uniform
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint4* wp = frag + (static_cast<long long>(b) * NT + nt) * 96 + lane;
+#pragma unroll
+        for (int p = 0; p < 3; ++p) {
+          const uint4 w = __ldg(wp + 32 * p);
+          mma_bf16_16816(acc[p][nt], ua[i].x, ub[i].x, ua[i].y, ub[i].y, w.x, w.y);
+          mma_bf16_16816(acc[p][nt], ua[i].z, ub[i].z, ua[i].w, ub[i].w, w.z, w.w);
+        }
+      }
+    }
+  }
+  // this slice's partial logits: rows g, g+8; columns 8nt + 2c, 2c+1
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int row = g + (q >> 1) * 8, col = 8 * nt + 2 * c + (q & 1);
+      part_s[gi][ks][row][col] = (acc[0][nt][q] + acc[1][nt][q]) + acc[2][nt][q];
+    }
+  __syncthreads();
+  // top-K: one warp per token, lane e holds expert e's logit (slices added in order)
+  for (int tl = warp; tl < 16 * G; tl += kMmaSlices * G) {
+    const long long t = static_cast<long long>(blockIdx.x) * 16 * G + tl;
+    if (t >= N) break;  // warp-uniform
+    float v[1];
+    bool avail[1];
+    float sum = 0.f;
+    if (lane < EW) {
+#pragma unroll
+      for (int s = 0; s < kMmaSlices; ++s) sum += part_s[tl / 16][s][tl % 16][lane];
+    }
+    avail[0] = lane < E;
+    v[0] = avail[0] ? sum + (bias != nullptr ? bias[lane] : 0.f) : 0.f;
+    write_topk<1>(v, avail, lane, K, E, t, ids, gates, margin);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_logits_topk(const float* logits, const float* bias, int N, int E, int K,
@@ -613,6 +779,53 @@ cudaError_t launch_router(const void* x, int x_dtype, const float* w_r, const fl
                     stream);
   return launch_t(static_cast<const __nv_bfloat16*>(x), w_r, bias, N, d, E, K, ids, gates, margin,
                   stream);
+}
+
+
+// ---- the warp-MMA router (bf16 tokens, E <= 16) ----------------------------
+
+bool router_uses_mma(int N, int d, int E, int x_dtype) {
+  return x_dtype == kBF16 && E <= kRouterMmaMaxExperts && !router_uses_splitk(N, d);
+}
+
+size_t router_mma_frag_bytes(int d, int E) {
+  const int nb = (d + 31) / 32, NT = (E + 7) / 8;
+  return static_cast<size_t>(nb) * NT * 3 * 32 * sizeof(uint4);
+}
+
+cudaError_t launch_router_mma_frag(const float* w_r, int d, int E, void* frag, cudaStream_t stream) {
+  const int nb = (d + 31) / 32, NT = (E + 7) / 8;
+  const long long n = static_cast<long long>(nb) * NT * 96;
+  router_frag_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+      w_r, d, E, nb, NT, static_cast<uint4*>(frag));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_mma(const void* x, const void* frag, const float* bias, int N, int d,
+                              int E, int K, int32_t* ids, float* gates, float* margin,
+                              cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  if (E > kRouterMmaMaxExperts || d % 8) return cudaErrorInvalidValue;
+  const int nb = (d + 31) / 32;
+  const int bps = (nb + kMmaSlices - 1) / kMmaSlices;  // 32-element blocks per slice
+  auto xb = static_cast<const __nv_bfloat16*>(x);
+  auto fr = static_cast<const uint4*>(frag);
+  // two 16-token groups per CTA when that still gives every SM a CTA
+  const long long groups = (N + 15) / 16;
+  const bool two = groups >= 2LL * device_sm_count();
+  const unsigned grid = static_cast<unsigned>(two ? (groups + 1) / 2 : groups);
+  if (E <= 8) {
+    if (two)
+      return launch_pdl(router_mma_kernel<1, 2>, dim3(grid), dim3(512), 0, stream, xb, fr, bias,
+                        N, d, E, K, nb, bps, ids, gates, margin);
+    return launch_pdl(router_mma_kernel<1, 1>, dim3(grid), dim3(256), 0, stream, xb, fr, bias, N,
+                      d, E, K, nb, bps, ids, gates, margin);
+  }
+  if (two)
+    return launch_pdl(router_mma_kernel<2, 2>, dim3(grid), dim3(512), 0, stream, xb, fr, bias, N,
+                      d, E, K, nb, bps, ids, gates, margin);
+  return launch_pdl(router_mma_kernel<2, 1>, dim3(grid), dim3(256), 0, stream, xb, fr, bias, N, d,
+                    E, K, nb, bps, ids, gates, margin);
 }
 
 }  // namespace moe

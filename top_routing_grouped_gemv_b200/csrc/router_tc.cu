@@ -23,10 +23,12 @@
 // (A dedicated kernel with one CTA per 128-token tile that kept a running
 // top-9 list per thread in its epilogue was bound by that epilogue: 116 us
 // against 44 us without it for 16384 tokens x 128 experts.)
+#include <math.h>
 #include <string.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace moe {
 namespace {
@@ -68,6 +70,356 @@ router_split_kernel(const float* __restrict__ w_r, int d, int E, __nv_bfloat16* 
   }
 }
 
+
+// ---- fused router: logits on tcgen05, top-K in the epilogue (33..128 experts) ----
+//
+// One CTA per 128-token tile.  The plan holds w_r split into its three bf16
+// parts as 3*EP K-major rows [hi(EP) | mid(EP) | lo(EP)] (EP = E rounded up
+// to 32, rows past E zero), made once (router_split3_kernel).  Per 64-element
+// K stage the producer loads the tile's 128 token rows and the three parts'
+// EP rows by TMA (128-byte swizzle); the MMA thread issues, per K=16 step,
+// one M=128, N=EP tcgen05.mma per part into its own fp32 accumulator (TMEM
+// columns [0,EP) hi, [EP,2EP) mid, [2EP,3EP) lo: bf16 x bf16 products are
+// exact in fp32, each part keeps its own rounding scale).  The four
+// epilogue warps then own one token row each per lane (TMEM lane = token):
+//   logit[e] = ((hi + mid) + lo) + bias[e]
+// and the top-K (value descending, equal values to the lower expert) in
+// three passes over the row:
+//   1. tau = min over KMAX+1 disjoint expert groups of the group maximum: at
+//      least KMAX+1 logits are >= tau, so every member of the top K+1 is;
+//   2. the logits >= tau (usually a dozen or two) are appended, in expert
+//      order, to the thread's list in shared memory (the pipeline buffers,
+//      free once the accumulators are final);
+//   3. they are inserted into a sorted K+1 list held in registers (an
+//      unrolled compare-and-shift; ties keep the earlier, lower expert).
+// This touches each logit with a few instructions instead of a full
+// insertion, which matters because the four epilogue warps have the SM to
+// themselves (one tile per CTA) and are bound by instruction issue.
+// Softmax over the kept K, margin = K-th minus (K+1)-th logit.
+
+constexpr int kFrBM = 128;      // tokens per tile
+constexpr int kFrKE = 64;       // K elements per stage (128 bytes of bf16)
+
+template <int EP>
+struct FrGeo {
+  static constexpr int A_BYTES = kFrBM * 128;
+  static constexpr int B_BYTES = 3 * EP * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = EP <= 64 ? 5 : EP <= 96 ? 4 : 3;
+  static constexpr int kBarFull = 0, kBarEmpty = STAGES, kBarTFull = 2 * STAGES,
+                       kNumBars = 2 * STAGES + 1;
+  // ring | barriers | TMEM slot + abort flag (16 B) | bias (EP floats)
+  static constexpr int kSmemBytes = 1024 + STAGES * STAGE_BYTES + kNumBars * 8 + 16 + EP * 4;
+  // candidate lists of the epilogue: EP entries of (value, expert) per token
+  static_assert(kFrBM * EP * 8 <= STAGES * STAGE_BYTES, "candidate lists fit the ring");
+};
+
+__device__ __forceinline__ void fr_insert(float v, int e, float* val, int* idx, int L) {
+  // descending list of L entries (L <= 9, unrolled to 9; entries past L
+  // are never read); v goes after entries equal to it
+#pragma unroll
+  for (int j = 8; j > 0; --j) {
+    if (j < L) {
+      const bool up = v > val[j - 1];
+      const bool here = v > val[j];
+      const float nv = up ? val[j - 1] : (here ? v : val[j]);
+      const int ni = up ? idx[j - 1] : (here ? e : idx[j]);
+      val[j] = nv;
+      idx[j] = ni;
+    }
+  }
+  if (v > val[0]) {
+    val[0] = v;
+    idx[0] = e;
+  }
+}
+
+template <int EP, int KMAX>
+__global__ void __launch_bounds__(192, 1)
+router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                    const float* __restrict__ bias, int N, int d, int E, int K,
+                    int32_t* __restrict__ ids, float* __restrict__ gates,
+                    float* __restrict__ margin, int* status) {
+  using namespace tc;
+  griddep_trigger();  // let the next kernel of the stream start launching
+  griddep_wait();     // inputs written by the previous kernel are visible
+
+  using Gm = FrGeo<EP>;
+  constexpr int STAGES = Gm::STAGES;
+  extern __shared__ uint8_t fr_smem_raw[];
+  const uint32_t raw = smem_u32(fr_smem_raw);
+  uint8_t* smem = fr_smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + STAGES * Gm::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Gm::STAGE_BYTES);
+  const uint32_t bar0 = smem_u32(bars);
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Gm::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_bias = reinterpret_cast<float*>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = blockIdx.x * kFrBM;
+  for (int e = threadIdx.x; e < EP; e += blockDim.x)
+    s_bias[e] = (bias != nullptr && e < E) ? bias[e] : 0.f;
+  const int num_kb = (d + kFrKE - 1) / kFrKE;
+
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar(Gm::kBarFull + s), 1);
+      mbar_init(bar(Gm::kBarEmpty + s), 1);
+    }
+    mbar_init(bar(Gm::kBarTFull), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- TMA producer ----
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_ph = 0;
+      bool aborted = false;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(bar(Gm::kBarEmpty + s), ph ^ 1u, abort_flag)) { aborted = true; break; }
+        const int kx = kb * kFrKE;
+        mbar_expect_tx(bar(Gm::kBarFull + s), Gm::STAGE_BYTES);
+        tma_load_2d(sA + s * Gm::A_BYTES, &tmX, kx, row0, bar(Gm::kBarFull + s));
+#pragma unroll
+        for (int p = 0; p < 3; ++p)
+          tma_load_2d(sB + s * Gm::B_BYTES + p * EP * 128, &tmW, kx, p * EP, bar(Gm::kBarFull + s));
+        issued |= 1u << s;
+        issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
+        if (++s == STAGES) { s = 0; ph ^= 1u; }
+      }
+      if (aborted) {
+        set_status(status, kStatusTimeout);
+        for (int i = 0; i < STAGES; ++i)
+          if ((issued >> i) & 1u) mbar_wait_drain(bar(Gm::kBarFull + i), (issued_ph >> i) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer: three parts, each into its own accumulator ----
+      constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                                 (static_cast<uint32_t>(EP >> 3) << 17) |
+                                 (static_cast<uint32_t>(kFrBM >> 4) << 24);
+      int s = 0;
+      uint32_t ph = 0;
+      bool aborted = false;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(bar(Gm::kBarFull + s), ph, abort_flag)) { aborted = true; break; }
+        tc_fence_after();
+        const uint32_t a0 = sA + s * Gm::A_BYTES, b0 = sB + s * Gm::B_BYTES;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int p = 0; p < 3; ++p)
+            tc_mma<false>(tmem_base + static_cast<uint32_t>(p * EP), sw128_desc(a0 + 32 * k),
+                          sw128_desc(b0 + p * EP * 128 + 32 * k), idesc, (kb | k) != 0 ? 1u : 0u);
+        tc_commit(bar(Gm::kBarEmpty + s));
+        if (++s == STAGES) { s = 0; ph ^= 1u; }
+      }
+      if (aborted) set_status(status, kStatusTimeout);
+      // arrives once every MMA issued so far has finished (the epilogue
+      // leaves through the abort flag when the loop gave up)
+      tc_commit(bar(Gm::kBarTFull));
+      if (aborted) mbar_wait_drain(bar(Gm::kBarTFull), 0);
+    }
+    __syncwarp();
+  } else {
+    // ---- epilogue: one token per lane ----
+    const int q = warp & 3;  // TMEM lane quadrant of this warp
+    const bool ok = __shfl_sync(0xffffffffu, mbar_wait(bar(Gm::kBarTFull), 0, abort_flag), 0);
+    if (!ok) {
+      set_status(status, kStatusTimeout);
+    } else {
+      tc_fence_after();
+      const int r = q * 32 + lane;  // row of the tile
+      const long long t = static_cast<long long>(row0) + r;
+      const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      constexpr int G = KMAX + 1;  // disjoint expert groups for the threshold
+      // pass 1: the group maxima -> tau
+      float gmax[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) gmax[g] = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < EP; cc += 32) {
+        uint32_t vh[32], vm[32], vl[32];
+        __syncwarp();
+        tmem_ld32(tq + cc, vh);
+        tmem_ld32(tq + EP + cc, vm);
+        tmem_ld32(tq + 2 * EP + cc, vl);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int e = cc + j;
+          if (e < E) {
+            const float v = ((__uint_as_float(vh[j]) + __uint_as_float(vm[j])) +
+                             __uint_as_float(vl[j])) + s_bias[e];
+            gmax[e % G] = fmaxf(gmax[e % G], v);
+          }
+        }
+      }
+      float tau = gmax[0];
+#pragma unroll
+      for (int g = 1; g < G; ++g) tau = fminf(tau, gmax[g]);
+      // pass 2: the candidates >= tau, in expert order, to this thread's list
+      // (entry i of row r at float2 index i * 128 + r of the ring)
+      float2* cand = reinterpret_cast<float2*>(smem);
+      int cnt = 0;
+#pragma unroll
+      for (int cc = 0; cc < EP; cc += 32) {
+        uint32_t vh[32], vm[32], vl[32];
+        __syncwarp();
+        tmem_ld32(tq + cc, vh);
+        tmem_ld32(tq + EP + cc, vm);
+        tmem_ld32(tq + 2 * EP + cc, vl);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int e = cc + j;
+          if (e < E) {
+            const float v = ((__uint_as_float(vh[j]) + __uint_as_float(vm[j])) +
+                             __uint_as_float(vl[j])) + s_bias[e];
+            if (v >= tau) {
+              cand[cnt * kFrBM + r] = make_float2(v, __int_as_float(e));
+              ++cnt;
+            }
+          }
+        }
+      }
+      // pass 3: sorted top K+1 of the candidates
+      const int L = K + 1 <= E ? K + 1 : K;
+      float val[9];
+      int idx[9];
+#pragma unroll
+      for (int j = 0; j < 9; ++j) {
+        val[j] = -INFINITY;
+        idx[j] = 0x7fffffff;
+      }
+      for (int i = 0; i < cnt; ++i) {
+        const float2 c = cand[i * kFrBM + r];
+        fr_insert(c.x, __float_as_int(c.y), val, idx, L);
+      }
+      if (t < N) {
+        float z = 0.f;
+        float p[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          p[j] = 0.f;
+          if (j < K) {
+            p[j] = expf(val[j] - val[0]);
+            z += p[j];
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < K) {
+            ids[t * K + j] = idx[j];
+            gates[t * K + j] = p[j] / z;
+          }
+        if (margin != nullptr) {
+          float kth = val[0], next = val[0];
+#pragma unroll
+          for (int j = 0; j < 9; ++j) {
+            if (j == K - 1) kth = val[j];
+            if (j == K) next = val[j];
+          }
+          margin[t] = (K == E) ? INFINITY : kth - next;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512)
+                 : "memory");
+  }
+}
+
+// w_r (d, E) fp32 -> out (3 * EP, d) bf16 rows [hi | mid | lo], rows e >= E
+// zero; through a 32 x 32 shared tile (reads along e, writes along k).
+// Block (32, 8); grid (EP / 32, ceil(d / 32)).
+__global__ void __launch_bounds__(256)
+router_split3_kernel(const float* __restrict__ w_r, int d, int E, int EP,
+                     __nv_bfloat16* __restrict__ out) {
+  __shared__ float tile[32][33];
+  const int e0 = blockIdx.x * 32, k0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int r = ty; r < 32; r += 8) {
+    const int k = k0 + r, e = e0 + tx;
+    tile[r][tx] = (k < d && e < E) ? w_r[static_cast<long long>(k) * E + e] : 0.f;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int e = e0 + r, k = k0 + tx;
+    if (k >= d) continue;
+    const float w = tile[tx][r];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    out[static_cast<long long>(e) * d + k] = hi;
+    out[static_cast<long long>(EP + e) * d + k] = mid;
+    out[static_cast<long long>(2 * EP + e) * d + k] = lo;
+  }
+}
+
+template <int EP, int KMAX>
+cudaError_t launch_fused_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias,
+                           int N, int d, int E, int K, int32_t* ids, float* gates, float* margin,
+                           int* status, cudaStream_t stream) {
+  auto kern = router_fused_kernel<EP, KMAX>;
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         FrGeo<EP>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const dim3 grid(static_cast<unsigned>((N + kFrBM - 1) / kFrBM));
+  return launch_pdl(kern, grid, dim3(192), FrGeo<EP>::kSmemBytes, stream, tmX, tmW, bias, N, d,
+                    E, K, ids, gates, margin, status);
+}
+
+template <int EP>
+cudaError_t launch_fused_k(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias,
+                           int N, int d, int E, int K, int32_t* ids, float* gates, float* margin,
+                           int* status, cudaStream_t stream) {
+  if (K <= 2)
+    return launch_fused_t<EP, 2>(tmX, tmW, bias, N, d, E, K, ids, gates, margin, status, stream);
+  if (K <= 4)
+    return launch_fused_t<EP, 4>(tmX, tmW, bias, N, d, E, K, ids, gates, margin, status, stream);
+  return launch_fused_t<EP, 8>(tmX, tmW, bias, N, d, E, K, ids, gates, margin, status, stream);
+}
+
+int fused_ep(int E) { return (E + 31) / 32 * 32; }
 }  // namespace
 
 // scratch: the split weights (nchunks * 256 rows of d bf16), then the fp32
@@ -113,6 +465,51 @@ cudaError_t launch_router_tc(const void* x, const float* w_r, const float* bias,
   cudaError_t e = launch_gemm_tc(a, kBF16, kEpiRouter, N, false, stream);
   if (e != cudaSuccess) return e;
   return launch_logits_topk(logits, bias, N, E, K, ids, gates, margin, stream);
+}
+
+}  // namespace moe
+
+namespace moe {
+
+bool router_uses_fused_tc(int N, int d, int E, int x_dtype) {
+  return x_dtype == kBF16 && E >= kRouterTcMinExperts && E <= kRouterFusedMaxExperts &&
+         !router_uses_splitk(N, d);
+}
+
+size_t router_fused_weight_bytes(int d, int E) {
+  return static_cast<size_t>(3) * fused_ep(E) * d * sizeof(__nv_bfloat16);
+}
+
+cudaError_t launch_router_fused_split(const float* w_r, int d, int E, void* out,
+                                      cudaStream_t stream) {
+  const int EP = fused_ep(E);
+  const dim3 grid(static_cast<unsigned>(EP / 32), static_cast<unsigned>((d + 31) / 32));
+  router_split3_kernel<<<grid, dim3(32, 8), 0, stream>>>(w_r, d, E, EP,
+                                                          static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+bool encode_router_fused_weights(CUtensorMap* map, const void* split, int d, int E) {
+  const int EP = fused_ep(E);
+  return encode_kmajor_map(map, split, 2, 3LL * EP, d, EP);
+}
+
+cudaError_t launch_router_fused(const void* x, const CUtensorMap& tmW, const float* bias, int N,
+                                int d, int E, int K, int32_t* ids, float* gates, float* margin,
+                                int* status, cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  CUtensorMap tmX;
+  if (!encode_kmajor_map(&tmX, x, 2, N, d, kFrBM)) return cudaErrorInvalidValue;
+  switch (fused_ep(E)) {
+    case 64:
+      return launch_fused_k<64>(tmX, tmW, bias, N, d, E, K, ids, gates, margin, status, stream);
+    case 96:
+      return launch_fused_k<96>(tmX, tmW, bias, N, d, E, K, ids, gates, margin, status, stream);
+    case 128:
+      return launch_fused_k<128>(tmX, tmW, bias, N, d, E, K, ids, gates, margin, status, stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace moe

@@ -31,6 +31,18 @@ flight, then every peer's rows as they arrive, each block's results sent
 straight back (computing and communicating overlap; more, smaller expert
 launches).  Every row is still computed as on one GPU.  Without an
 initialized process group the layer runs on one rank with no exchange.
+
+With `capacity=True` the host never reads the counts: every per-peer block
+has a fixed capacity of N*K rows (all of a rank's routed rows could go to one
+peer), the block's per-expert counts travel in header rows at its start, and
+both exchanges are all-to-alls of equal, fixed splits.  The sender fills its
+blocks, and the receiver regroups the rows by local expert and returns the
+results into the same padded layout, by index arithmetic on the device
+(cumulative counts, searchsorted, row gathers), so a step has no device to
+host synchronisation.  The price is bytes on the wire: G * (header + N*K)
+rows per rank and direction against the about N*K rows of the variable-split
+exchange, i.e. about G times as many.  Every rank must hold the same number
+of tokens (the capacity is the same on all ranks).
 """
 from __future__ import annotations
 
@@ -143,10 +155,13 @@ class ExpertParallelMoE:
     """The expert-parallel layer on this rank (see the module docstring)."""
 
     def __init__(self, stages, E: int, K: int, group=None, host_exchange: bool = False,
-                 overlap: bool = False):
+                 overlap: bool = False, capacity: bool = False):
+        if overlap and capacity:
+            raise ValueError("choose one exchange: overlap or capacity")
         self.stages, self.E, self.K, self.group = stages, E, K, group
         self.host_exchange = host_exchange
         self.overlap = overlap
+        self.capacity = capacity
 
     def _all_to_all(self, dist, t, out_rows, out_splits=None, in_splits=None):
         """all_to_all_single of the rows of t (variable splits if given)."""
@@ -180,6 +195,9 @@ class ExpertParallelMoE:
         if ids is None:
             ids, gates = st.route(x)
         counts, offsets, pos, x_perm = st.permute(x, ids)
+        if self.capacity:
+            y_perm = self._exchange_capacity(dist, G, E_loc, x_perm, counts, offsets)
+            return st.combine(y_perm, pos, gates)
 
         # per-expert row counts: block q of my counts goes to rank q
         send_counts = counts.to(torch.int64).reshape(G, E_loc)
@@ -215,6 +233,90 @@ class ExpertParallelMoE:
         else:
             y_perm = y_recv
         return st.combine(y_perm, pos, gates)
+
+    # ---- fixed-capacity exchange: no host read of the counts ------------------
+
+    @staticmethod
+    def _bytes(t):
+        """(rows, row bytes) uint8 view of a contiguous row tensor."""
+        t = t.contiguous()
+        row_bytes = t.element_size()
+        for n in t.shape[1:]:
+            row_bytes *= n
+        return t.view(torch.uint8).reshape(t.shape[0], row_bytes)
+
+    def _exchange_capacity(self, dist, G, E_loc, x_perm, counts, offsets):
+        st = self.stages
+        dev = x_perm.device
+        i64 = dict(dtype=torch.int64, device=dev)
+        NK = x_perm.shape[0]
+        C = NK                                   # rows per peer block
+        xb = self._bytes(x_perm)                 # (NK, rb)
+        rb = xb.shape[1]
+        H = -(-4 * E_loc // rb)                  # header rows holding E_loc int32 counts
+        cnt = counts.to(**i64).reshape(G, E_loc)
+        send_rows = cnt.sum(1)                                   # rows for rank q
+        send_off = offsets.to(**i64)[torch.arange(G, device=dev) * E_loc]
+        # my blocks: rows [send_off[q], send_off[q] + send_rows[q]) of x_perm
+        slot = torch.arange(C, **i64)
+        src = send_off[:, None] + slot[None, :]
+        src = torch.where(slot[None, :] < send_rows[:, None], src, torch.zeros_like(src))
+        hdr = torch.zeros(G, H * rb, dtype=torch.uint8, device=dev)
+        hdr[:, :4 * E_loc] = cnt.to(torch.int32).contiguous().view(torch.uint8)
+        send = torch.cat([hdr.reshape(G, H, rb), xb[src.reshape(-1)].reshape(G, C, rb)], dim=1)
+        recv = self._fixed_all_to_all(dist, G, send)             # (G, H + C, rb)
+        # counts of the rows from rank q for my local expert l
+        rcnt = recv[:, :H].reshape(G, H * rb)[:, :4 * E_loc].contiguous().view(torch.int32)
+        rcnt = rcnt.to(torch.int64)                              # (G, E_loc)
+        tot = rcnt.sum(0)
+        offs_l = torch.zeros(E_loc + 1, **i64)
+        offs_l[1:] = torch.cumsum(tot, 0)
+        sstart = torch.cumsum(rcnt, 1) - rcnt                    # start of (q, l) in block q
+        dstart = offs_l[:-1][None, :] + (torch.cumsum(rcnt, 0) - rcnt)  # start of (q, l) sorted
+        # sorted row j <- its (expert l, source q) segment, expert-major, source-minor
+        flat_cnt = rcnt.t().reshape(-1)
+        flat_end = torch.cumsum(flat_cnt, 0)
+        j = torch.arange(G * C, **i64)
+        k = torch.searchsorted(flat_end, j, right=True)
+        kk = k.clamp(max=E_loc * G - 1)
+        l, q = kk // G, kk % G
+        i = j - (flat_end[kk] - flat_cnt[kk])
+        rows_src = q * (H + C) + H + sstart[q, l] + i
+        rows_src = torch.where(k < E_loc * G, rows_src, torch.zeros_like(rows_src))
+        x_sorted = recv.reshape(-1, rb)[rows_src].contiguous().view(x_perm.dtype)
+        x_sorted = x_sorted.reshape((G * C,) + tuple(x_perm.shape[1:]))
+        y_sorted = st.local_ffn(G * C, x_sorted, offs_l.to(torch.int32))
+        # results into the padded blocks: block q row H + sstart[q, l] + i <- y_sorted[dstart + i]
+        rc_end = torch.cumsum(rcnt, 1)
+        r = torch.arange(C, **i64).expand(G, C).contiguous()
+        lq = torch.searchsorted(rc_end, r, right=True)
+        lq_c = lq.clamp(max=E_loc - 1)
+        i2 = r - (rc_end.gather(1, lq_c) - rcnt.gather(1, lq_c))
+        ysrc = dstart.gather(1, lq_c) + i2
+        ysrc = torch.where(lq < E_loc, ysrc, torch.zeros_like(ysrc))
+        if y_sorted.shape[0] == 0:       # no rows anywhere on this rank's experts
+            like = self._result_like(x_perm)
+            yb = torch.zeros(G * C, self._bytes(like).shape[1], dtype=torch.uint8, device=dev)
+            ydt, tail = like.dtype, tuple(like.shape[1:])
+        else:
+            yb = self._bytes(y_sorted)[ysrc.reshape(-1)]
+            ydt, tail = y_sorted.dtype, tuple(y_sorted.shape[1:])
+        ret = self._fixed_all_to_all(dist, G, yb.reshape(G, C, -1))   # my rows' results
+        # back in my permuted order: row r of x_perm was row r - send_off[q] of block q
+        send_end = torch.cumsum(send_rows, 0)
+        rr = torch.arange(NK, **i64)
+        rq = torch.searchsorted(send_end, rr, right=True).clamp(max=G - 1)
+        yrow = rq * C + (rr - send_off[rq])
+        yrow = torch.where(rr < send_end[-1], yrow, torch.zeros_like(yrow))
+        return ret.reshape(G * C, -1)[yrow].contiguous().view(ydt).reshape((NK,) + tail)
+
+    def _fixed_all_to_all(self, dist, G, t):
+        """all_to_all_single of G equal blocks of a (G, rows, bytes) uint8 tensor."""
+        if dist is None:
+            return t
+        flat = t.reshape(t.shape[0] * t.shape[1], t.shape[2])
+        out = self._all_to_all(dist, flat, flat.shape[0])
+        return out.reshape(t.shape)
 
     # ---- peer-to-peer exchange overlapped with the local experts -------------
 
