@@ -168,7 +168,7 @@ moe_status run_router(moe_plan p, int n, const void* x, int32_t* ids, float* gat
     mark(p, s, "router_mma");
     p->launches += 1;
     return cuda_status(launch_router_mma(x, p->router_w, p->w.router_bias, n, d.d, d.E, d.K, ids,
-                                         gates, margin, s));
+                                         gates, margin, at<int>(ws, p->L.status), s));
   }
   if (p->router_kind == kRouterTc) {
     mark(p, s, "router_tc");

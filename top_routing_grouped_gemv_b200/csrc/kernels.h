@@ -58,8 +58,10 @@ constexpr int kRouterMmaMaxExperts = 16;
 bool router_uses_mma(int N, int d, int E, int x_dtype);
 size_t router_mma_frag_bytes(int d, int E);
 cudaError_t launch_router_mma_frag(const float* w_r, int d, int E, void* frag, cudaStream_t stream);
+// Split weights up to this size are staged in shared memory by each CTA.
+constexpr size_t kRouterMmaSmemMax = 96 * 1024;
 cudaError_t launch_router_mma(const void* x, const void* frag, const float* bias, int N, int d,
-                              int E, int K, int32_t* ids, float* gates, float* margin,
+                              int E, int K, int32_t* ids, float* gates, float* margin, int* status,
                               cudaStream_t stream);
 
 // Top-K, softmax and margin of fp32 logits (N, E) in memory, plus bias.

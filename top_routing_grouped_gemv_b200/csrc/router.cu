@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace moe {
 namespace {
@@ -646,17 +647,30 @@ router_frag_kernel(const float* __restrict__ w_r, int d, int E, int nb, int NT,
 // XB: 32-element blocks whose token vectors are loaded before their MMAs
 // (2 * XB 16-byte loads in flight per thread; fewer for two expert tiles,
 // whose accumulators take the registers).
-template <int NT, int G, int XB = (NT == 1 ? 8 : 4)>
+//
+// kSmemW: the CTA first copies the split weights into shared memory, one
+// bulk copy (cp.async.bulk, no multicast) per k slice onto that slice's
+// mbarrier, issued in an order rotated by the CTA index; each warp issues its
+// token loads, then waits for its own slice only.  Every CTA reads the same
+// weights: rotating the order spreads those reads over the weight lines
+// instead of every SM asking for the same lines at once.  Without kSmemW
+// (weights too large for shared memory) the fragments are read straight
+// from global memory, the slice's blocks in the same rotated order.
+template <int NT, int G, bool kSmemW, int XB = (NT == 1 ? 8 : 4)>
 __global__ void __launch_bounds__(32 * kMmaSlices * G)
 router_mma_kernel(const __nv_bfloat16* __restrict__ x, const uint4* __restrict__ frag,
                   const float* __restrict__ bias, int N, int d, int E, int K, int nb, int bps,
                   int32_t* __restrict__ ids, float* __restrict__ gates,
-                  float* __restrict__ margin) {
+                  float* __restrict__ margin, int* status) {
   griddep_trigger();  // let the next kernel of the stream start launching
   griddep_wait();     // inputs written by the previous kernel are visible
 
   constexpr int EW = 8 * NT;  // expert columns
+  constexpr int kBlockU4 = NT * 96;  // 16-byte entries of one 32-element block
   __shared__ float part_s[G][kMmaSlices][16][EW];
+  __shared__ __align__(8) uint64_t wbar[kMmaSlices];
+  __shared__ int abort_s;
+  extern __shared__ uint4 mma_wsm[];  // kSmemW: the split weights, nb blocks
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gi = warp / kMmaSlices, ks = warp % kMmaSlices;
   const int g = lane >> 2, c = lane & 3;
@@ -665,6 +679,31 @@ router_mma_kernel(const __nv_bfloat16* __restrict__ x, const uint4* __restrict__
   const int rv = d / 8;  // 16-byte vectors per token row (d % 8 == 0)
   const uint4* xa = reinterpret_cast<const uint4*>(x) + (ta < N ? ta : 0) * rv;
   const uint4* xb = reinterpret_cast<const uint4*>(x) + (tb < N ? tb : 0) * rv;
+  const int b0 = ks * bps, b1 = min(nb, b0 + bps);
+
+  if constexpr (kSmemW) {
+    if (threadIdx.x == 0) {
+      for (int q = 0; q < kMmaSlices; ++q) tc::mbar_init(tc::smem_u32(&wbar[q]), 1);
+      abort_s = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int i = 0; i < kMmaSlices; ++i) {
+        const int q = static_cast<int>((i + blockIdx.x) % kMmaSlices);
+        const int q0 = q * bps, q1 = min(nb, q0 + bps);
+        const uint32_t bar = tc::smem_u32(&wbar[q]);
+        if (q1 > q0) {
+          const uint32_t bytes = static_cast<uint32_t>((q1 - q0) * kBlockU4 * 16);
+          tc::mbar_expect_tx(bar, bytes);
+          tc::bulk_load(tc::smem_u32(mma_wsm + static_cast<long long>(q0) * kBlockU4),
+                        frag + static_cast<long long>(q0) * kBlockU4, bytes, bar);
+        } else {
+          tc::mbar_arrive(bar);  // an empty slice: its phase completes at once
+        }
+      }
+    }
+  }
 
   float acc[3][NT][4];
 #pragma unroll
@@ -674,32 +713,43 @@ router_mma_kernel(const __nv_bfloat16* __restrict__ x, const uint4* __restrict__
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[p][nt][q] = 0.f;
 
-  const int b0 = ks * bps, b1 = min(nb, b0 + bps);
-  for (int bb = b0; bb < b1; bb += XB) {
+  bool waited = !kSmemW;
+  const int nblk = b1 > b0 ? b1 - b0 : 0;
+  const int rot = kSmemW ? 0 : static_cast<int>(blockIdx.x % static_cast<unsigned>(nblk > 0 ? nblk : 1));
+  for (int bb = 0; bb < nblk; bb += XB) {
     // the token vectors of up to XB blocks in flight before any MMA
     uint4 ua[XB], ub[XB];
 #pragma unroll
     for (int i = 0; i < XB; ++i) {
-      const int v = 4 * (bb + i) + c;  // vector index of elements 32(bb+i) + 8c ..
-      const bool in = bb + i < b1 && v < rv;
+      const int bi = bb + i < nblk ? b0 + (bb + i + rot) % nblk : b0;
+      const int v = 4 * bi + c;  // vector index of elements 32 bi + 8c ..
+      const bool in = bb + i < nblk && v < rv;
       ua[i] = (in && ta < N) ? ld_stream(xa + v) : make_uint4(0u, 0u, 0u, 0u);
       ub[i] = (in && tb < N) ? ld_stream(xb + v) : make_uint4(0u, 0u, 0u, 0u);
     }
+    if (!waited) {  // this slice's weights in shared memory
+      waited = true;
+      const bool ok = tc::mbar_wait(tc::smem_u32(&wbar[ks]), 0, &abort_s);
+      if (!ok) set_status(status, kStatusTimeout);
+    }
 #pragma unroll
     for (int i = 0; i < XB; ++i) {
-      const int b = bb + i;
-      if (b >= b1) break;  // warp-uniform
+      if (bb + i >= nblk) break;  // warp-uniform
+      const int b = b0 + (bb + i + rot) % nblk;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const uint4* wp = frag + (static_cast<long long>(b) * NT + nt) * 96 + lane;
+        const long long wi = static_cast<long long>(b) * kBlockU4 + nt * 96 + lane;
 #pragma unroll
         for (int p = 0; p < 3; ++p) {
-          const uint4 w = __ldg(wp + 32 * p);
+          const uint4 w = kSmemW ? mma_wsm[wi + 32 * p] : __ldg(frag + wi + 32 * p);
           mma_bf16_16816(acc[p][nt], ua[i].x, ub[i].x, ua[i].y, ub[i].y, w.x, w.y);
           mma_bf16_16816(acc[p][nt], ua[i].z, ub[i].z, ua[i].w, ub[i].w, w.z, w.w);
         }
       }
     }
+  }
+  if (kSmemW && !waited) {  // a slice with no blocks still consumes its phase
+    if (!tc::mbar_wait(tc::smem_u32(&wbar[ks]), 0, &abort_s)) set_status(status, kStatusTimeout);
   }
   // this slice's partial logits: rows g, g+8; columns 8nt + 2c, 2c+1
 #pragma unroll
@@ -802,7 +852,7 @@ cudaError_t launch_router_mma_frag(const float* w_r, int d, int E, void* frag, c
 }
 
 cudaError_t launch_router_mma(const void* x, const void* frag, const float* bias, int N, int d,
-                              int E, int K, int32_t* ids, float* gates, float* margin,
+                              int E, int K, int32_t* ids, float* gates, float* margin, int* status,
                               cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
   if (E > kRouterMmaMaxExperts || d % 8) return cudaErrorInvalidValue;
@@ -810,22 +860,48 @@ cudaError_t launch_router_mma(const void* x, const void* frag, const float* bias
   const int bps = (nb + kMmaSlices - 1) / kMmaSlices;  // 32-element blocks per slice
   auto xb = static_cast<const __nv_bfloat16*>(x);
   auto fr = static_cast<const uint4*>(frag);
-  // two 16-token groups per CTA when that still gives every SM a CTA
+  // two 16-token groups per CTA (sixteen warps) once there are more groups
+  // than SMs: the same per-SM work as two one-group CTAs, half the weight reads
   const long long groups = (N + 15) / 16;
-  const bool two = groups >= 2LL * device_sm_count();
+  const bool two = groups > device_sm_count();
   const unsigned grid = static_cast<unsigned>(two ? (groups + 1) / 2 : groups);
+  const size_t wbytes = router_mma_frag_bytes(d, E);
+  const bool smem_w = wbytes <= kRouterMmaSmemMax;
+  const size_t smem = smem_w ? wbytes : 0;
+  const dim3 block(two ? 512 : 256);
+#define MOE_ROUTER_MMA_LAUNCH(NT_, G_, S_)                                                       \
+  do {                                                                                           \
+    auto kern = router_mma_kernel<NT_, G_, S_>;                                                  \
+    if (S_) {                                                                                    \
+      static bool configured[64] = {false};                                                      \
+      int dev = 0;                                                                               \
+      cudaGetDevice(&dev);                                                                       \
+      if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;                                   \
+      if (!configured[dev]) {                                                                    \
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                             static_cast<int>(kRouterMmaSmemMax));               \
+        if (e != cudaSuccess) return e;                                                          \
+        configured[dev] = true;                                                                  \
+      }                                                                                          \
+    }                                                                                            \
+    return launch_pdl(kern, dim3(grid), block, smem, stream, xb, fr, bias, N, d, E, K, nb, bps,  \
+                      ids, gates, margin, status);                                               \
+  } while (0)
   if (E <= 8) {
-    if (two)
-      return launch_pdl(router_mma_kernel<1, 2>, dim3(grid), dim3(512), 0, stream, xb, fr, bias,
-                        N, d, E, K, nb, bps, ids, gates, margin);
-    return launch_pdl(router_mma_kernel<1, 1>, dim3(grid), dim3(256), 0, stream, xb, fr, bias, N,
-                      d, E, K, nb, bps, ids, gates, margin);
+    if (two) {
+      if (smem_w) MOE_ROUTER_MMA_LAUNCH(1, 2, true);
+      MOE_ROUTER_MMA_LAUNCH(1, 2, false);
+    }
+    if (smem_w) MOE_ROUTER_MMA_LAUNCH(1, 1, true);
+    MOE_ROUTER_MMA_LAUNCH(1, 1, false);
   }
-  if (two)
-    return launch_pdl(router_mma_kernel<2, 2>, dim3(grid), dim3(512), 0, stream, xb, fr, bias, N,
-                      d, E, K, nb, bps, ids, gates, margin);
-  return launch_pdl(router_mma_kernel<2, 1>, dim3(grid), dim3(256), 0, stream, xb, fr, bias, N, d,
-                    E, K, nb, bps, ids, gates, margin);
+  if (two) {
+    if (smem_w) MOE_ROUTER_MMA_LAUNCH(2, 2, true);
+    MOE_ROUTER_MMA_LAUNCH(2, 2, false);
+  }
+  if (smem_w) MOE_ROUTER_MMA_LAUNCH(2, 1, true);
+  MOE_ROUTER_MMA_LAUNCH(2, 1, false);
+#undef MOE_ROUTER_MMA_LAUNCH
 }
 
 }  // namespace moe

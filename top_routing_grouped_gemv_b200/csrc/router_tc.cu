@@ -163,6 +163,12 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
   for (int e = threadIdx.x; e < EP; e += blockDim.x)
     s_bias[e] = (bias != nullptr && e < E) ? bias[e] : 0.f;
   const int num_kb = (d + kFrKE - 1) / kFrKE;
+  // Every CTA reads the same router weights.  Starting each CTA's k loop at
+  // a different stage spreads those reads over the weight tiles, instead of
+  // every SM asking for the same L2 lines at the same moment (a hot spot
+  // that made the stages several times slower than their MMAs).  Only the
+  // order of the fp32 accumulation over k changes, fixed per CTA.
+  const int kb0 = static_cast<int>(blockIdx.x % static_cast<unsigned>(num_kb));
 
   if (threadIdx.x == 32) {
     for (int s = 0; s < STAGES; ++s) {
@@ -197,8 +203,9 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_ph = 0;
       bool aborted = false;
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int it = 0; it < num_kb; ++it) {
         if (!mbar_wait(bar(Gm::kBarEmpty + s), ph ^ 1u, abort_flag)) { aborted = true; break; }
+        const int kb = it + kb0 < num_kb ? it + kb0 : it + kb0 - num_kb;
         const int kx = kb * kFrKE;
         mbar_expect_tx(bar(Gm::kBarFull + s), Gm::STAGE_BYTES);
         tma_load_2d(sA + s * Gm::A_BYTES, &tmX, kx, row0, bar(Gm::kBarFull + s));
@@ -225,7 +232,7 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
       int s = 0;
       uint32_t ph = 0;
       bool aborted = false;
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int it = 0; it < num_kb; ++it) {
         if (!mbar_wait(bar(Gm::kBarFull + s), ph, abort_flag)) { aborted = true; break; }
         tc_fence_after();
         const uint32_t a0 = sA + s * Gm::A_BYTES, b0 = sB + s * Gm::B_BYTES;
@@ -234,7 +241,7 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 #pragma unroll
           for (int p = 0; p < 3; ++p)
             tc_mma<false>(tmem_base + static_cast<uint32_t>(p * EP), sw128_desc(a0 + 32 * k),
-                          sw128_desc(b0 + p * EP * 128 + 32 * k), idesc, (kb | k) != 0 ? 1u : 0u);
+                          sw128_desc(b0 + p * EP * 128 + 32 * k), idesc, (it | k) != 0 ? 1u : 0u);
         tc_commit(bar(Gm::kBarEmpty + s));
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
