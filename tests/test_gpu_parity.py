@@ -68,6 +68,13 @@ SMALL = {
     "bf16_mma_router_g2_e8": synth.MoEConfig("mma_g2_e8", "bf16", 4801, 256, 8, 2, 64, "swiglu"),
     "bf16_mma_router_g2_e16": synth.MoEConfig("mma_g2_e16", "bf16", 4900, 160, 16, 4, 64,
                                               "swiglu", zipf_bias=1.2),
+    # at most 16 routed rows per expert on average: the whole-layer call's
+    # gate/up GEMM gathers its rows from x (tile::gather4), the permute copies
+    # no rows; ragged row counts, and a skewed router that gives one expert
+    # more than a full 128-row tile
+    "bf16_decode_ragged": synth.MoEConfig("dec_rag", "bf16", 37, 520, 32, 4, 192, "swiglu"),
+    "bf16_decode_zipf": synth.MoEConfig("dec_zipf", "bf16", 200, 256, 64, 4, 128, "swiglu",
+                                        zipf_bias=1.2),
 }
 
 _cache = {}

@@ -198,11 +198,19 @@ moe_status run_permute(moe_plan p, int n, const void* x, const int32_t* ids, int
   const moe_layer_desc& d = p->desc;
   int* status = at<int>(ws, p->L.status);
   int32_t* cc = at<int32_t>(ws, p->L.chunk_counts);
+  // no rows to copy and a small batch: the rank pass also makes the positions
+  const bool positions_in_rank =
+      x_perm == nullptr && slot == nullptr &&
+      static_cast<long long>(n) * d.K <= kRankPositionsMaxRows;
   mark(p, s, "permute_rank");
   if (launch_permute_rank(ids, n, d.K, d.E, cc, at<unsigned>(ws, p->L.counter), pos, counts,
-                          offsets, status, s) != cudaSuccess)
+                          offsets, status, s, positions_in_rank ? src : nullptr) != cudaSuccess)
     return MOE_ERR_CUDA;
-  mark(p, s, "permute_gather");
+  if (positions_in_rank) {
+    p->launches += 1;
+    return MOE_OK;
+  }
+  mark(p, s, x_perm ? "permute_gather" : "permute_positions");
   if (launch_permute_gather(x, d.d * p->ex, ids, n, d.K, d.E, cc, pos, src, slot, x_perm, status,
                             s) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -230,13 +238,28 @@ moe_status run_permute_quant(moe_plan p, int n, const void* x_bf16, const int32_
   return MOE_OK;
 }
 
+// Whether the whole-layer call of a bf16 SwiGLU plan gathers the gate/up
+// GEMM's A rows straight from the tokens (no row copy in the permute): for
+// decode-shaped batches, at most kGatherRowsPerExpert routed rows per expert
+// on average, where each stage's A tile is a few rows beside 256 weight rows
+// (for larger batches a 128-row A box per stage, copied once by the permute,
+// is cheaper than re-gathering it for every column tile).
+constexpr int kGatherRowsPerExpert = 16;
+bool gather_fused(const moe_layer_desc& d, int n) {
+  return d.dtype == MOE_BF16 && d.act == MOE_ACT_SWIGLU &&
+         static_cast<long long>(n) * d.K <= static_cast<long long>(kGatherRowsPerExpert) * d.E;
+}
+
 // x_rows: per-token activation scales indexed by row_index[row] (or by the
 // permuted row itself when row_index is NULL); NULL = the scalar x_scale.
 // out_rows (tensor cores, single-matrix layer): result row r goes to row
 // out_rows[r] of y_perm (the pure unpermute done by the GEMM's stores).
+// x_tokens, a_rows (bf16 SwiGLU): the gate/up GEMM takes its A rows from the
+// token rows, row r = x_tokens[a_rows[r]], instead of x_perm.
 moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets, float x_scale,
                    const float* x_rows, const int32_t* row_index, void* y_perm, void* ws,
-                   cudaStream_t s, const int32_t* out_rows = nullptr) {
+                   cudaStream_t s, const int32_t* out_rows = nullptr,
+                   const void* x_tokens = nullptr, const int32_t* a_rows = nullptr) {
   const moe_layer_desc& d = p->desc;
   if (d.quant == MOE_QUANT_MX || d.quant == MOE_QUANT_PER_GROUP || d.quant == MOE_QUANT_PER_BLOCK)
     return MOE_ERR_UNSUPPORTED;  // the _mx / _group_scales calls carry the scales
@@ -306,6 +329,10 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
     return cuda_status(launch_gemm_tc(a, d.dtype, kEpiStore, R, pair, s));
   }
   // SwiGLU: gate/up GEMM with the activation fused into its epilogue, then down
+  if (x_tokens != nullptr && a_rows != nullptr && !pair_swiglu) {
+    if (!encode_kmajor_map(&a.tmAg, x_tokens, p->ex, n > 0 ? n : 1, d.d, 1)) return MOE_ERR_CUDA;
+    a.a_rows = a_rows;
+  }
   a.tmB0 = p->tmW1;
   a.tmB1 = p->tmW3;
   a.kdim = d.d;
@@ -314,9 +341,10 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
   a.out = h;
   a.ldo = d.F;
   a.scale = 1.f;
-  mark(p, s, "ffn1_swiglu_tc");
+  mark(p, s, a.a_rows ? "ffn1_swiglu_tc_gather" : "ffn1_swiglu_tc");
   if (launch_gemm_tc(a, d.dtype, kEpiSwiglu, R, pair_swiglu, s) != cudaSuccess) return MOE_ERR_CUDA;
   TcGemmArgs b = a;
+  b.a_rows = nullptr;
   if (!encode_kmajor_map(&b.tmA, h, p->eh, map_rows, d.F, kTcBlockM)) return MOE_ERR_CUDA;
   b.tmB0 = pair ? p->tmW2h : p->tmW2;
   b.tmB1 = b.tmB0;
@@ -959,15 +987,19 @@ namespace {
 // The whole layer on n <= N tokens; every intermediate lives in the workspace.
 moe_status forward_tokens(moe_plan p, int n, const void* x, void* y, void* ws, cudaStream_t stream) {
   const Layout& L = p->L;
+  // decode-shaped bf16 SwiGLU batches: the gate/up GEMM gathers its rows from
+  // x, the permute only makes the positions
+  const bool gather = gather_fused(p->desc, n);
   moe_status st = run_router(p, n, x, at<int32_t>(ws, L.ids), at<float>(ws, L.gates), nullptr,
                              ws, stream);
   if (st == MOE_OK)
     st = run_permute(p, n, x, at<int32_t>(ws, L.ids), at<int32_t>(ws, L.counts),
                      at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.pos), at<int32_t>(ws, L.src),
-                     at<void>(ws, L.x_perm), ws, stream);
+                     gather ? nullptr : at<void>(ws, L.x_perm), ws, stream);
   if (st == MOE_OK)
     st = run_ffn(p, n, at<void>(ws, L.x_perm), at<int32_t>(ws, L.offsets), 1.f, nullptr, nullptr,
-                 at<void>(ws, L.y_perm), ws, stream);
+                 at<void>(ws, L.y_perm), ws, stream, nullptr, gather ? x : nullptr,
+                 gather ? at<int32_t>(ws, L.src) : nullptr);
   if (st == MOE_OK)
     st = run_combine(p, n, at<void>(ws, L.y_perm), at<int32_t>(ws, L.pos), at<float>(ws, L.gates),
                      y, ws, stream);

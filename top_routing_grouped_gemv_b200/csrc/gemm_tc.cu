@@ -42,6 +42,15 @@
 // accumulator, so the MX kernel has one accumulator and its epilogue does
 // not overlap the next tile's MMAs.
 //
+// Gathered A (kGather, bf16 SwiGLU gate/up GEMM on single CTAs): instead of
+// a 128-row box of the permuted rows, each stage's A tile is gathered from the
+// token rows themselves (args.tmAg over x, a box one row high;
+// args.a_rows[r] = the token of permuted row r) by TMA tile::gather4, four
+// rows per instruction and only as many as the tile has rows of its expert;
+// the tile's other rows keep stale data, are computed and never stored.  It
+// lets small batches skip the permute's row copy: with a few rows per expert
+// the A tile is a sliver of the stage next to the 256 weight rows.
+//
 // Every mbarrier wait is bounded (1 s): on expiry the CTA records
 // MOE_ERR_DEVICE_TIMEOUT, the other roles leave their loops, in-flight
 // copies and MMAs are drained (bounded) and TMEM is freed before exit.
@@ -136,12 +145,14 @@ __device__ __forceinline__ uint32_t mx_sf_ids(uint32_t k) { return (k << 29) | (
 // kPair: a cluster of 2 CTAs computes 256-row tiles with tcgen05 cta_group::2;
 // CTA rank r holds rows [128r, 128r+128) of the tile and B rows [128r, 128r+128)
 // of the 256-row weight tile; the leader (rank 0) issues the MMAs.
-template <bool kFp8, int kEpi, bool kPair, bool kMx>
+template <bool kFp8, int kEpi, bool kPair, bool kMx, bool kGather = false>
 __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __grid_constant__ TcGemmArgs args) {
   griddep_trigger();  // let the next kernel of the stream start launching
   griddep_wait();     // inputs written by the previous kernel are visible
 
   static_assert(!kMx || (kFp8 && !kPair && kEpi == kEpiStore), "MX: e4m3, single CTA, store");
+  static_assert(!kGather || (!kFp8 && !kPair && !kMx && kEpi == kEpiSwiglu),
+                "gathered A: bf16 SwiGLU, single CTA");
   constexpr bool kGs = kEpi == kEpiGroupScale || kEpi == kEpiBlockScale;
   static_assert(!kGs || (kFp8 && !kPair && !kMx), "group scales: e4m3, single CTA");
   using Gm = Geo<kPair, kMx>;
@@ -214,7 +225,8 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&args.tmA);
+    if constexpr (kGather) tma_prefetch_desc(&args.tmAg);
+    else tma_prefetch_desc(&args.tmA);
     tma_prefetch_desc(&args.tmB0);
     if (kEpi == kEpiSwiglu) tma_prefetch_desc(&args.tmB1);
   }
@@ -254,6 +266,16 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
       for (int T = unit; T < total && !aborted; T += nunits) {
         const TileCoord c = decode_tile<Gm::TILE_M>(T, s_pref, s_off, G, args.n_tiles);
         const int arow = c.m_row0 + static_cast<int>(rank) * BM;
+        // gathered A: the tile's rows of its expert and, for a tile of at most
+        // 16 rows, their token indices once for all its stages
+        int g_rows = 0, g_idx[16];
+        if constexpr (kGather) {
+          g_rows = min(BM, s_off[c.g + 1] - c.m_row0);
+          if (g_rows <= 16) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) g_idx[u] = args.a_rows[c.m_row0 + min(u, g_rows - 1)];
+          }
+        }
         int brow;
         if constexpr (kEpi == kEpiSwiglu)
           brow = c.g * args.n_out + c.n_tile * (BN / 2);  // gate (and up) rows of 128 outputs
@@ -268,8 +290,32 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
             tma_load_2d_pair(sA + s * A_BYTES, &args.tmA, kx, arow, full_leader);
             tma_load_2d_pair(sB + s * Gm::B_BYTES, mapB, kx, brow, full_leader);
           } else {
-            mbar_expect_tx(bar(Gm::kBarFull + s), Gm::STAGE_BYTES);
-            tma_load_2d(sA + s * A_BYTES, &args.tmA, kx, arow, bar(Gm::kBarFull + s));
+            if constexpr (kGather) {
+              // the tile's rows of its expert, four per gather (the last
+              // group padded with the last row)
+              const int rows = g_rows;
+              const int ng4 = (rows + 3) >> 2;
+              mbar_expect_tx(bar(Gm::kBarFull + s), ng4 * 512 + Gm::B_BYTES);
+              if (rows <= 16) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  if (q < ng4)
+                    tma_gather4(sA + s * A_BYTES + 512 * q, &args.tmAg, kx, g_idx[4 * q],
+                                g_idx[4 * q + 1], g_idx[4 * q + 2], g_idx[4 * q + 3],
+                                bar(Gm::kBarFull + s));
+              } else {
+                const int32_t* src = args.a_rows + c.m_row0;
+                for (int q = 0; q < ng4; ++q) {
+                  const int i = 4 * q;
+                  tma_gather4(sA + s * A_BYTES + 512 * q, &args.tmAg, kx, src[i],
+                              src[min(i + 1, rows - 1)], src[min(i + 2, rows - 1)],
+                              src[min(i + 3, rows - 1)], bar(Gm::kBarFull + s));
+                }
+              }
+            } else {
+              mbar_expect_tx(bar(Gm::kBarFull + s), Gm::STAGE_BYTES);
+              tma_load_2d(sA + s * A_BYTES, &args.tmA, kx, arow, bar(Gm::kBarFull + s));
+            }
             if (kEpi == kEpiSwiglu) {
               tma_load_2d(sB + s * Gm::B_BYTES, &args.tmB0, kx, brow, bar(Gm::kBarFull + s));
               tma_load_2d(sB + s * Gm::B_BYTES + (BN / 2) * ROWB, &args.tmB1, kx, brow,
@@ -670,10 +716,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <bool kFp8, int kEpi, bool kPair, bool kMx = false>
+template <bool kFp8, int kEpi, bool kPair, bool kMx = false, bool kGather = false>
 cudaError_t launch_t(const TcGemmArgs& args, long long max_units, cudaStream_t stream) {
   using Gm = Geo<kPair, kMx>;
-  auto kern = gemm_tc_kernel<kFp8, kEpi, kPair, kMx>;
+  auto kern = gemm_tc_kernel<kFp8, kEpi, kPair, kMx, kGather>;
   static int configured[64] = {0};
   static int max_clusters[64] = {0};
   int dev = 0;
@@ -750,6 +796,10 @@ cudaError_t launch_gemm_tc(const TcGemmArgs& args, int dtype, int epilogue, int 
   }
   const bool fp8 = dtype == kE4M3;
   const bool sw = epilogue == kEpiSwiglu;
+  if (args.a_rows != nullptr) {
+    if (pair || fp8 || !sw) return cudaErrorInvalidValue;
+    return launch_t<false, kEpiSwiglu, false, false, true>(args, max_units, stream);
+  }
   if (epilogue == kEpiRouter) {
     if (pair || fp8) return cudaErrorInvalidValue;
     return launch_t<false, kEpiRouter, false>(args, max_units, stream);

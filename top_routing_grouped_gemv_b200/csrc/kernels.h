@@ -108,13 +108,18 @@ inline size_t permute_block_counts_bytes(int N, int E) {
 // through *counter, which must be zero on entry and is zero again on exit --
 // the per-(block, expert) first destination rows (over block_counts), the
 // expert counts and the offsets (E + 1).
+// With src non-null (N*K <= kRankPositionsMaxRows) the last CTA also makes
+// the final positions (local_rank -> pos, src[pos] = t), as the gather would.
+constexpr long long kRankPositionsMaxRows = 8192;
 cudaError_t launch_permute_rank(const int32_t* ids, int N, int K, int E, int32_t* block_counts,
                                 unsigned* counter, int32_t* local_rank, int32_t* counts,
-                                int32_t* offsets, int* status, cudaStream_t stream);
+                                int32_t* offsets, int* status, cudaStream_t stream,
+                                int32_t* src = nullptr);
 // pos holds the ranks from launch_permute_rank on entry, the final
 // positions on exit; src[pos] = t and, when slot is non-null,
 // slot[pos] = t*K + j.  chunk_base = the block bases from the rank pass; a
-// position outside [0, N*K) is recorded in status and skipped.
+// position outside [0, N*K) is recorded in status and skipped.  With x_perm
+// NULL only the positions are made (no row is copied).
 cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* ids, int N, int K,
                                   int E, const int32_t* chunk_base, int32_t* pos, int32_t* src,
                                   int32_t* slot, void* x_perm, int* status, cudaStream_t stream);
@@ -191,6 +196,11 @@ struct TcGemmArgs {
   // kdim / 128.
   const float* xgs;
   const float* wgs;
+  // Gathered A (bf16 SwiGLU gate/up GEMM, single CTA): when a_rows is set,
+  // row r of A is row a_rows[r] of the matrix under tmAg (a box one row
+  // high, 128 bytes of K); tmA is not read.
+  const int32_t* a_rows;
+  CUtensorMap tmAg;
 };
 
 // Host: encode a 2-D K-major tile map over a (rows, kdim) row-major matrix of

@@ -129,12 +129,16 @@ __device__ __forceinline__ void scan_block_counts(int32_t* __restrict__ bc, int 
 // a CTA (8 warps, 10 K registers, 18 KB of shared memory) then fits on an SM
 // beside one CTA of a persistent tensor-core GEMM (the shared expert running
 // on a forked stream) instead of waiting for that GEMM to end.
+//
+// With src non-null (small batches) the last CTA also turns every rank into
+// its final position (pos = block base + rank, src[pos] = t), so that a
+// permute that copies no rows needs no second launch.
 template <int KMAX>
 __global__ void __maxnreg__(40)
 permute_rank_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
                     int32_t* __restrict__ block_counts, unsigned* __restrict__ counter,
                     int32_t* __restrict__ local_rank, int32_t* __restrict__ counts,
-                    int32_t* __restrict__ offsets, int* status) {
+                    int32_t* __restrict__ offsets, int32_t* __restrict__ src, int* status) {
   griddep_trigger();  // let the next kernel of the stream start launching
   griddep_wait();     // inputs written by the previous kernel are visible
 
@@ -228,6 +232,26 @@ permute_rank_kernel(const int32_t* __restrict__ ids, int N, int K, int E,
   __threadfence();
   scan_block_counts(block_counts, static_cast<int>(gridDim.x), E, counts, offsets, s_part, s_total);
   if (threadIdx.x == 0) *counter = 0u;  // ready for the next call (stream-ordered)
+  if (src != nullptr) {
+    __syncthreads();  // the block bases are in block_counts
+    const long long R = static_cast<long long>(N) * K;
+    for (long long i = threadIdx.x; i < R; i += blockDim.x) {
+      const long long tt = i / K;
+      const int e = __ldcg(ids + i);
+      const int r = __ldcg(local_rank + i);  // written by every CTA
+      int mine = -1;
+      if (r >= 0 && e >= 0 && e < E) {
+        mine = __ldcg(block_counts + (tt / BT) * E + e) + r;
+        if (mine < 0 || mine >= R) {  // only a damaged workspace gets here
+          set_status(status, kStatusBadIndex);
+          mine = -1;
+        } else {
+          src[mine] = static_cast<int32_t>(tt);
+        }
+      }
+      local_rank[i] = mine;
+    }
+  }
 }
 
 // WPT warps per token (8 / WPT tokens per CTA): final positions from the
@@ -270,7 +294,7 @@ permute_gather_kernel(const uint4* __restrict__ x, int row_vecs, const int32_t* 
   }
   if constexpr (WPT > 1) __syncthreads();
   else __syncwarp();
-  if (t >= N) return;
+  if (t >= N || x_perm == nullptr) return;  // no x_perm: positions only
   int p[KMAX];
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) p[j] = sp[tl][j];
@@ -431,17 +455,20 @@ void launch_gather_k(const uint4* xv, int row_vecs, const int32_t* ids, int N, i
 
 cudaError_t launch_permute_rank(const int32_t* ids, int N, int K, int E, int32_t* block_counts,
                                 unsigned* counter, int32_t* local_rank, int32_t* counts,
-                                int32_t* offsets, int* status, cudaStream_t stream) {
+                                int32_t* offsets, int* status, cudaStream_t stream,
+                                int32_t* src) {
+  if (src != nullptr && static_cast<long long>(N) * K > kRankPositionsMaxRows)
+    return cudaErrorInvalidValue;
   // at least one CTA, so that counts and offsets are written for zero tokens
   const int grid = permute_blocks(N) > 0 ? permute_blocks(N) : 1;
   if (K <= 2)
     return launch_pdl(permute_rank_kernel<2>, dim3(grid), dim3(256), 0, stream, ids, N, K, E,
-                      block_counts, counter, local_rank, counts, offsets, status);
+                      block_counts, counter, local_rank, counts, offsets, src, status);
   if (K <= 4)
     return launch_pdl(permute_rank_kernel<4>, dim3(grid), dim3(256), 0, stream, ids, N, K, E,
-                      block_counts, counter, local_rank, counts, offsets, status);
+                      block_counts, counter, local_rank, counts, offsets, src, status);
   return launch_pdl(permute_rank_kernel<8>, dim3(grid), dim3(256), 0, stream, ids, N, K, E,
-                    block_counts, counter, local_rank, counts, offsets, status);
+                    block_counts, counter, local_rank, counts, offsets, src, status);
 }
 
 cudaError_t launch_permute_gather(const void* x, int row_bytes, const int32_t* ids, int N, int K,

@@ -99,6 +99,7 @@ router_split_kernel(const float* __restrict__ w_r, int d, int E, __nv_bfloat16* 
 
 constexpr int kFrBM = 128;      // tokens per tile
 constexpr int kFrKE = 64;       // K elements per stage (128 bytes of bf16)
+constexpr int kFrPrefetch = 8;  // stages of token rows prefetched into L2 ahead
 
 template <int EP>
 struct FrGeo {
@@ -203,9 +204,17 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_ph = 0;
       bool aborted = false;
+      // The token rows come from HBM, once; the ring holds only a few stages
+      // of them beside the three weight parts, so their DRAM latency would
+      // set the pace.  Prefetch the token box kFrPrefetch stages ahead into
+      // L2 (the weights are L2-resident: every CTA reads them).
+      auto kb_of = [&](int it) { return it + kb0 < num_kb ? it + kb0 : it + kb0 - num_kb; };
+      for (int it = 0; it < kFrPrefetch && it < num_kb; ++it)
+        tma_prefetch_l2(&tmX, kb_of(it) * kFrKE, row0);
       for (int it = 0; it < num_kb; ++it) {
         if (!mbar_wait(bar(Gm::kBarEmpty + s), ph ^ 1u, abort_flag)) { aborted = true; break; }
-        const int kb = it + kb0 < num_kb ? it + kb0 : it + kb0 - num_kb;
+        if (it + kFrPrefetch < num_kb) tma_prefetch_l2(&tmX, kb_of(it + kFrPrefetch) * kFrKE, row0);
+        const int kb = kb_of(it);
         const int kx = kb * kFrKE;
         mbar_expect_tx(bar(Gm::kBarFull + s), Gm::STAGE_BYTES);
         tma_load_2d(sA + s * Gm::A_BYTES, &tmX, kx, row0, bar(Gm::kBarFull + s));
