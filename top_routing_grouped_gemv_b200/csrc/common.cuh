@@ -31,6 +31,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// c ? a : b as one PTX select.  A chain of such selects over a small array
+// with constant indices (pick element K-1, element `lane`, ...) would
+// otherwise be folded by the compiler into one runtime-indexed load, which
+// moves the whole array to local memory.
+__device__ __forceinline__ float sel_f(bool c, float a, float b) {
+  float r;
+  asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\tselp.f32 %0, %1, %2, p;\n\t}"
+      : "=f"(r)
+      : "f"(a), "f"(b), "r"(static_cast<int>(c)));
+  return r;
+}
+__device__ __forceinline__ int sel_i(bool c, int a, int b) {
+  int r;
+  asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\tselp.b32 %0, %1, %2, p;\n\t}"
+      : "=r"(r)
+      : "r"(a), "r"(b), "r"(static_cast<int>(c)));
+  return r;
+}
+
 __device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 

@@ -86,6 +86,7 @@ __device__ __forceinline__ void write_topk(const float (&v)[EPL], bool (&avail)[
     warp_argmax<EPL>(v, avail, lane, next_v, next_e);
   }
   // softmax over the kept logits, largest first (sel_v[0] is the max)
+  // (selections by sel_f / sel_i: sel_v and sel_e stay in registers)
   float z = 0.f, my_g = 0.f;
   int my_e = 0;
 #pragma unroll
@@ -93,7 +94,8 @@ __device__ __forceinline__ void write_topk(const float (&v)[EPL], bool (&avail)[
     if (j < K) {
       const float p = expf(sel_v[j] - sel_v[0]);
       z += p;
-      if (j == lane) { my_g = p; my_e = sel_e[j]; }
+      my_g = sel_f(j == lane, p, my_g);
+      my_e = sel_i(j == lane, sel_e[j], my_e);
     }
   }
   if (lane < K) {
@@ -103,8 +105,7 @@ __device__ __forceinline__ void write_topk(const float (&v)[EPL], bool (&avail)[
   if (margin != nullptr && lane == 0) {
     float kth = sel_v[0];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j == K - 1) kth = sel_v[j];
+    for (int j = 0; j < 8; ++j) kth = sel_f(j == K - 1, sel_v[j], kth);
     margin[t] = (K == E) ? __int_as_float(0x7f800000) : kth - next_v;
   }
 }

@@ -85,8 +85,9 @@ router_split_kernel(const float* __restrict__ w_r, int d, int E, __nv_bfloat16* 
 //   logit[e] = ((hi + mid) + lo) + bias[e]
 // and the top-K (value descending, equal values to the lower expert) in
 // three passes over the row:
-//   1. tau = min over KMAX+1 disjoint expert groups of the group maximum: at
-//      least KMAX+1 logits are >= tau, so every member of the top K+1 is;
+//   1. tau = min over KMAX+1 disjoint expert groups (group (e mod 32) mod
+//      (KMAX+1)) of the group maximum: at least KMAX+1 logits are >= tau,
+//      so every member of the top K+1 is;
 //   2. the logits >= tau (usually a dozen or two) are appended, in expert
 //      order, to the thread's list in shared memory (the pipeline buffers,
 //      free once the accumulators are final);
@@ -99,7 +100,6 @@ router_split_kernel(const float* __restrict__ w_r, int d, int E, __nv_bfloat16* 
 
 constexpr int kFrBM = 128;      // tokens per tile
 constexpr int kFrKE = 64;       // K elements per stage (128 bytes of bf16)
-constexpr int kFrPrefetch = 8;  // stages of token rows prefetched into L2 ahead
 
 template <int EP>
 struct FrGeo {
@@ -115,19 +115,17 @@ struct FrGeo {
   static_assert(kFrBM * EP * 8 <= STAGES * STAGE_BYTES, "candidate lists fit the ring");
 };
 
-__device__ __forceinline__ void fr_insert(float v, int e, float* val, int* idx, int L) {
-  // descending list of L entries (L <= 9, unrolled to 9; entries past L
-  // are never read); v goes after entries equal to it
+// Inserts (v, e) into a descending list of L entries held in registers (L
+// a compile-time size, every index a constant); v goes after entries equal
+// to it, so with e ascending equal values keep the lower expert first.
+template <int L>
+__device__ __forceinline__ void fr_insert(float v, int e, float (&val)[L], int (&idx)[L]) {
 #pragma unroll
-  for (int j = 8; j > 0; --j) {
-    if (j < L) {
-      const bool up = v > val[j - 1];
-      const bool here = v > val[j];
-      const float nv = up ? val[j - 1] : (here ? v : val[j]);
-      const int ni = up ? idx[j - 1] : (here ? e : idx[j]);
-      val[j] = nv;
-      idx[j] = ni;
-    }
+  for (int j = L - 1; j > 0; --j) {
+    const bool up = v > val[j - 1];
+    const bool here = v > val[j];
+    val[j] = up ? val[j - 1] : (here ? v : val[j]);
+    idx[j] = up ? idx[j - 1] : (here ? e : idx[j]);
   }
   if (v > val[0]) {
     val[0] = v;
@@ -204,16 +202,9 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_ph = 0;
       bool aborted = false;
-      // The token rows come from HBM, once; the ring holds only a few stages
-      // of them beside the three weight parts, so their DRAM latency would
-      // set the pace.  Prefetch the token box kFrPrefetch stages ahead into
-      // L2 (the weights are L2-resident: every CTA reads them).
       auto kb_of = [&](int it) { return it + kb0 < num_kb ? it + kb0 : it + kb0 - num_kb; };
-      for (int it = 0; it < kFrPrefetch && it < num_kb; ++it)
-        tma_prefetch_l2(&tmX, kb_of(it) * kFrKE, row0);
       for (int it = 0; it < num_kb; ++it) {
         if (!mbar_wait(bar(Gm::kBarEmpty + s), ph ^ 1u, abort_flag)) { aborted = true; break; }
-        if (it + kFrPrefetch < num_kb) tma_prefetch_l2(&tmX, kb_of(it + kFrPrefetch) * kFrKE, row0);
         const int kb = kb_of(it);
         const int kx = kb * kFrKE;
         mbar_expect_tx(bar(Gm::kBarFull + s), Gm::STAGE_BYTES);
@@ -291,7 +282,7 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
           if (e < E) {
             const float v = ((__uint_as_float(vh[j]) + __uint_as_float(vm[j])) +
                              __uint_as_float(vl[j])) + s_bias[e];
-            gmax[e % G] = fmaxf(gmax[e % G], v);
+            gmax[j % G] = fmaxf(gmax[j % G], v);  // group (e mod 32) mod G: a constant index
           }
         }
       }
@@ -323,24 +314,26 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
           }
         }
       }
-      // pass 3: sorted top K+1 of the candidates
-      const int L = K + 1 <= E ? K + 1 : K;
-      float val[9];
-      int idx[9];
+      // pass 3: sorted top KMAX+1 of the candidates (K <= KMAX reads the
+      // first K+1: the list keeps a superset of what it needs)
+      float val[G];
+      int idx[G];
 #pragma unroll
-      for (int j = 0; j < 9; ++j) {
+      for (int j = 0; j < G; ++j) {
         val[j] = -INFINITY;
         idx[j] = 0x7fffffff;
       }
       for (int i = 0; i < cnt; ++i) {
         const float2 c = cand[i * kFrBM + r];
-        fr_insert(c.x, __float_as_int(c.y), val, idx, L);
+        fr_insert<G>(c.x, __float_as_int(c.y), val, idx);
       }
       if (t < N) {
+        // every index below is a constant within the list (j < KMAX < G), so
+        // the list stays in registers
         float z = 0.f;
-        float p[8];
+        float p[KMAX];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < KMAX; ++j) {
           p[j] = 0.f;
           if (j < K) {
             p[j] = expf(val[j] - val[0]);
@@ -348,7 +341,7 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
           }
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < KMAX; ++j)
           if (j < K) {
             ids[t * K + j] = idx[j];
             gates[t * K + j] = p[j] / z;
@@ -356,9 +349,9 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         if (margin != nullptr) {
           float kth = val[0], next = val[0];
 #pragma unroll
-          for (int j = 0; j < 9; ++j) {
-            if (j == K - 1) kth = val[j];
-            if (j == K) next = val[j];
+          for (int j = 0; j < G; ++j) {
+            kth = sel_f(j == K - 1, val[j], kth);
+            next = sel_f(j == K, val[j], next);
           }
           margin[t] = (K == E) ? INFINITY : kth - next;
         }
