@@ -268,6 +268,11 @@ def replica_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms
     return world * tokens_per_rank_step * steps / (max_ms / 1e3)
 
 
+def R_rows(cfg) -> int:
+    """Routed rows of a layer (tokens x experts per token)."""
+    return cfg.N * cfg.K
+
+
 def gemm_flops(cfg, rows: int):
     """Algorithmic FLOPs of the grouped FFN over the actual routed rows."""
     if cfg.act == "swiglu":
@@ -563,6 +568,11 @@ def main():
         ("gmm_mx_tc" if mx else f"gmm_{cfg.quant}_tc" if gsq else "gmm_tc")
         if cfg.act == "none" else "ffn1_simt_f32")
     stage_us = {k: 1e3 * statistics.mean(v) for k, v in per_kernel.items()}
+    if k1 not in stage_us and k1 + "_gather" in stage_us:
+        k1 += "_gather"   # decode-shaped batches: the gate/up GEMM gathers its rows from x
+    # decode-shaped layers (a few rows per expert) stream their weights: the
+    # gate/up GEMM's bound is HBM, not the tensor pipe
+    decode = cfg.dtype == "bf16" and cfg.act == "swiglu" and R_rows(cfg) <= 16 * cfg.E
     # the sustained (power-capped) peak applies to a kernel timed inside a long
     # loop or while the power cap throttles the clock; the burst one otherwise
     clk_summary = clk.summary()
@@ -579,12 +589,22 @@ def main():
             peak *= 2.0
             peak_desc += " x 2 (e4m3 nominal ratio)"
     t1 = stage_us.get(k1, float("nan")) * 1e-6
-    achieved = f1 / t1 / 1e12
     traffic = profiled_traffic(cfg.name, k1)
-    roofline = {"bound": "tensor", "kernel": k1, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "peak_source": peak_desc,
-                "algorithmic_flop_per_launch": f1}
+    if decode:
+        # every expert's gate and up weights (R >= 4E: all experts are routed
+        # to, but for a vanishing chance), the routed rows in, h out
+        bytes1 = cfg.E * 2 * cfg.F * cfg.d * 2 + R * cfg.d * 2 + R * cfg.F * 2
+        achieved = bytes1 / t1 / 1e9
+        roofline = {"bound": "hbm", "kernel": k1, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                    "peak_source": f"{peak_src} HBM copy bandwidth",
+                    "algorithmic_bytes_per_launch": bytes1}
+    else:
+        achieved = f1 / t1 / 1e12
+        roofline = {"bound": "tensor", "kernel": k1, "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                    "peak_source": peak_desc,
+                    "algorithmic_flop_per_launch": f1}
     ffn_keys = [k for k in stage_us if k.startswith("ffn") or k.startswith("gmm")]
     ffn_s = sum(stage_us[k] for k in ffn_keys) * 1e-6
     gemm = {"tflops": (f1 + f2) / ffn_s / 1e12, "frac_of_peak": (f1 + f2) / ffn_s / 1e12 / peak,

@@ -73,12 +73,17 @@ router_split_kernel(const float* __restrict__ w_r, int d, int E, __nv_bfloat16* 
 
 // ---- fused router: logits on tcgen05, top-K in the epilogue (33..128 experts) ----
 //
-// One CTA per 128-token tile.  The plan holds w_r split into its three bf16
+// One CTA pair (a cluster of two, tcgen05 cta_group::2) per 256-token tile:
+// each CTA loads its 128 token rows and half of every weight part, the
+// leader issues M=256 MMAs over both CTAs' shared memory, and each CTA's
+// accumulators hold its own 128 tokens -- half the weight bytes per CTA and
+// stage of a single-CTA tile, which is what sets the pace (the weights are
+// read by every tile).  The plan holds w_r split into its three bf16
 // parts as 3*EP K-major rows [hi(EP) | mid(EP) | lo(EP)] (EP = E rounded up
 // to 32, rows past E zero), made once (router_split3_kernel).  Per 64-element
-// K stage the producer loads the tile's 128 token rows and the three parts'
-// EP rows by TMA (128-byte swizzle); the MMA thread issues, per K=16 step,
-// one M=128, N=EP tcgen05.mma per part into its own fp32 accumulator (TMEM
+// K stage each CTA loads its 128 token rows and its EP/2 rows of each part by
+// TMA (128-byte swizzle); the leader's MMA thread issues, per K=16 step, one
+// M=256, N=EP tcgen05.mma per part into its own fp32 accumulator (TMEM
 // columns [0,EP) hi, [EP,2EP) mid, [2EP,3EP) lo: bf16 x bf16 products are
 // exact in fp32, each part keeps its own rounding scale).  The four
 // epilogue warps then own one token row each per lane (TMEM lane = token):
@@ -104,9 +109,9 @@ constexpr int kFrKE = 64;       // K elements per stage (128 bytes of bf16)
 template <int EP>
 struct FrGeo {
   static constexpr int A_BYTES = kFrBM * 128;
-  static constexpr int B_BYTES = 3 * EP * 128;
+  static constexpr int B_BYTES = 3 * (EP / 2) * 128;  // this CTA's half of each part
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = EP <= 64 ? 5 : EP <= 96 ? 4 : 3;
+  static constexpr int STAGES = EP <= 64 ? 7 : EP <= 96 ? 6 : 5;
   static constexpr int kBarFull = 0, kBarEmpty = STAGES, kBarTFull = 2 * STAGES,
                        kNumBars = 2 * STAGES + 1;
   // ring | barriers | TMEM slot + abort flag (16 B) | bias (EP floats)
@@ -158,16 +163,18 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
   float* s_bias = reinterpret_cast<float*>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row0 = blockIdx.x * kFrBM;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int row0 = pair * 2 * kFrBM + static_cast<int>(rank) * kFrBM;
   for (int e = threadIdx.x; e < EP; e += blockDim.x)
     s_bias[e] = (bias != nullptr && e < E) ? bias[e] : 0.f;
   const int num_kb = (d + kFrKE - 1) / kFrKE;
-  // Every CTA reads the same router weights.  Starting each CTA's k loop at
-  // a different stage spreads those reads over the weight tiles, instead of
-  // every SM asking for the same L2 lines at the same moment (a hot spot
-  // that made the stages several times slower than their MMAs).  Only the
-  // order of the fp32 accumulation over k changes, fixed per CTA.
-  const int kb0 = static_cast<int>(blockIdx.x % static_cast<unsigned>(num_kb));
+  // Every tile reads the same router weights; each pair starts its k loop
+  // at a different stage (the same in both CTAs), so the weight tiles in
+  // flight differ between pairs.  Only the order of the fp32 accumulation
+  // over k changes, fixed per pair.
+  const int kb0 = static_cast<int>(static_cast<unsigned>(pair) % static_cast<unsigned>(num_kb));
 
   if (threadIdx.x == 32) {
     for (int s = 0; s < STAGES; ++s) {
@@ -185,14 +192,15 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
   }
   if (warp == 1) {
     __syncwarp();
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
                  "r"(512)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // the leader's barriers exist before the peer's copies signal them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -207,28 +215,33 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         if (!mbar_wait(bar(Gm::kBarEmpty + s), ph ^ 1u, abort_flag)) { aborted = true; break; }
         const int kb = kb_of(it);
         const int kx = kb * kFrKE;
-        mbar_expect_tx(bar(Gm::kBarFull + s), Gm::STAGE_BYTES);
-        tma_load_2d(sA + s * Gm::A_BYTES, &tmX, kx, row0, bar(Gm::kBarFull + s));
+        // both CTAs' copies complete on the leader's barrier
+        const uint32_t full_leader = map_to_rank(bar(Gm::kBarFull + s), 0);
+        if (leader) mbar_expect_tx(bar(Gm::kBarFull + s), 2 * Gm::STAGE_BYTES);
+        tma_load_2d_pair(sA + s * Gm::A_BYTES, &tmX, kx, row0, full_leader);
 #pragma unroll
         for (int p = 0; p < 3; ++p)
-          tma_load_2d(sB + s * Gm::B_BYTES + p * EP * 128, &tmW, kx, p * EP, bar(Gm::kBarFull + s));
+          tma_load_2d_pair(sB + s * Gm::B_BYTES + p * (EP / 2) * 128, &tmW, kx,
+                           p * EP + static_cast<int>(rank) * (EP / 2), full_leader);
         issued |= 1u << s;
         issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
       if (aborted) {
         set_status(status, kStatusTimeout);
-        for (int i = 0; i < STAGES; ++i)
-          if ((issued >> i) & 1u) mbar_wait_drain(bar(Gm::kBarFull + i), (issued_ph >> i) & 1u);
+        // let copies already in flight land before the CTA pair's memory is reused
+        if (leader)
+          for (int i = 0; i < STAGES; ++i)
+            if ((issued >> i) & 1u) mbar_wait_drain(bar(Gm::kBarFull + i), (issued_ph >> i) & 1u);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---- MMA issuer: three parts, each into its own accumulator ----
+    if (lane == 0 && leader) {
+      // ---- MMA issuer (the pair's leader): three parts, each into its own accumulator ----
       constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
                                  (static_cast<uint32_t>(EP >> 3) << 17) |
-                                 (static_cast<uint32_t>(kFrBM >> 4) << 24);
+                                 (static_cast<uint32_t>((2 * kFrBM) >> 4) << 24);
       int s = 0;
       uint32_t ph = 0;
       bool aborted = false;
@@ -240,15 +253,16 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         for (int k = 0; k < 4; ++k)
 #pragma unroll
           for (int p = 0; p < 3; ++p)
-            tc_mma<false>(tmem_base + static_cast<uint32_t>(p * EP), sw128_desc(a0 + 32 * k),
-                          sw128_desc(b0 + p * EP * 128 + 32 * k), idesc, (it | k) != 0 ? 1u : 0u);
-        tc_commit(bar(Gm::kBarEmpty + s));
+            tc_mma_pair<false>(tmem_base + static_cast<uint32_t>(p * EP), sw128_desc(a0 + 32 * k),
+                               sw128_desc(b0 + p * (EP / 2) * 128 + 32 * k), idesc,
+                               (it | k) != 0 ? 1u : 0u);
+        tc_commit_pair_both(bar(Gm::kBarEmpty + s));  // frees the stage in both CTAs
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
       if (aborted) set_status(status, kStatusTimeout);
-      // arrives once every MMA issued so far has finished (the epilogue
-      // leaves through the abort flag when the loop gave up)
-      tc_commit(bar(Gm::kBarTFull));
+      // arrives (in both CTAs) once every MMA issued so far has finished;
+      // the epilogues leave through the abort flag when the loop gave up
+      tc_commit_pair_both(bar(Gm::kBarTFull));
       if (aborted) mbar_wait_drain(bar(Gm::kBarTFull), 0);
     }
     __syncwarp();
@@ -361,10 +375,11 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // the peer is done with this CTA's shared memory and TMEM
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512)
                  : "memory");
   }
 }
@@ -412,9 +427,22 @@ cudaError_t launch_fused_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  const dim3 grid(static_cast<unsigned>((N + kFrBM - 1) / kFrBM));
-  return launch_pdl(kern, grid, dim3(192), FrGeo<EP>::kSmemBytes, stream, tmX, tmW, bias, N, d,
-                    E, K, ids, gates, margin, status);
+  // a cluster of two CTAs per 256 tokens
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * ((N + 2 * kFrBM - 1) / (2 * kFrBM))));
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = FrGeo<EP>::kSmemBytes;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, tmX, tmW, bias, N, d, E, K, ids, gates, margin, status);
 }
 
 template <int EP>
@@ -500,7 +528,7 @@ cudaError_t launch_router_fused_split(const float* w_r, int d, int E, void* out,
 
 bool encode_router_fused_weights(CUtensorMap* map, const void* split, int d, int E) {
   const int EP = fused_ep(E);
-  return encode_kmajor_map(map, split, 2, 3LL * EP, d, EP);
+  return encode_kmajor_map(map, split, 2, 3LL * EP, d, EP / 2);  // a CTA's half of a part
 }
 
 cudaError_t launch_router_fused(const void* x, const CUtensorMap& tmW, const float* bias, int N,
