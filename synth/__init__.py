@@ -18,6 +18,8 @@ Workloads (the five shapes the layer is measured and checked on):
   scales (OCP MXFP8: one E8M0 scale per 32 consecutive elements along H1)
 * ``e4m3blk_n8192_h7168_e256_k8_n2048_gmm``  the same grouped matmul with fp32 scales per
   128 x 128 weight block and per token and 128-element group of the activations
+* ``e4m3grp_n8192_h7168_e256_k8_n2048_gmm``  the same with fp32 scales per output column and
+  128-element group of K for the weights (per token and group for the activations)
 * ``e4m3_n2048_h7168_e64_k8_n2048_gmm``, ``e4m3mx_n2048_h7168_e64_k8_n2048_gmm``,
   ``e4m3blk_n2048_h7168_e64_k8_n2048_gmm`` reduced copies of the fp8 layers for kernel profiling
 
@@ -118,6 +120,8 @@ MX_GMM = _reg(MoEConfig("e4m3mx_n8192_h7168_e256_k8_n2048_gmm", DTYPE_E4M3, 8192
                         2048, ACT_NONE, index=5, routing="given", quant="mx"))
 BLOCK_GMM = _reg(MoEConfig("e4m3blk_n8192_h7168_e256_k8_n2048_gmm", DTYPE_E4M3, 8192, 7168, 256, 8,
                            2048, ACT_NONE, index=8, routing="given", quant="block"))
+GROUP_GMM = _reg(MoEConfig("e4m3grp_n8192_h7168_e256_k8_n2048_gmm", DTYPE_E4M3, 8192, 7168, 256, 8,
+                           2048, ACT_NONE, index=10, routing="given", quant="group"))
 # Reduced copies of the two fp8 layers (a quarter of the tokens, E = 64, the
 # same per-expert shape and ~256 rows per expert): small enough for kernel
 # captures that replay every launch many times, weights (0.94 GB) still far

@@ -398,14 +398,18 @@ moe_status run_ffn_gs(moe_plan p, int n, const void* x_perm, const int32_t* offs
   TcGemmArgs a;
   memset(&a, 0, sizeof(a));
   if (!encode_kmajor_map(&a.tmA, x_perm, 1, R > 0 ? R : 1, d.d, kTcBlockM)) return MOE_ERR_CUDA;
-  a.tmB0 = p->tmW1;
+  const bool blocks = d.quant == MOE_QUANT_PER_BLOCK;
+  // per-column scales: 128 x 128 tiles (128-row weight boxes); block scales:
+  // 128 x 256 tiles
+  a.tmB0 = blocks ? p->tmW1 : p->tmW1h;
   a.tmB1 = a.tmB0;
   a.offsets = offsets;
   a.groups = d.E;
   a.m_total = R;
   a.kdim = d.d;
   a.n_out = d.F;
-  a.n_tiles = (d.F + kTcBlockN - 1) / kTcBlockN;
+  const int tile_n = blocks ? kTcBlockN : kGsTileN;
+  a.n_tiles = (d.F + tile_n - 1) / tile_n;
   a.out = y_perm;
   a.out_rows = out_rows;
   a.ldo = d.F;
@@ -415,10 +419,10 @@ moe_status run_ffn_gs(moe_plan p, int n, const void* x_perm, const int32_t* offs
   a.xgs = x_group;
   a.wgs = p->wgs;
   a.status = at<int>(ws, p->L.status);
-  const bool blocks = d.quant == MOE_QUANT_PER_BLOCK;
   mark(p, s, blocks ? "gmm_block_tc" : "gmm_group_tc");
   p->launches += 1;
-  return cuda_status(launch_gemm_tc(a, kE4M3, blocks ? kEpiBlockScale : kEpiGroupScale, R, false, s));
+  return cuda_status(blocks ? launch_gemm_tc(a, kE4M3, kEpiBlockScale, R, false, s)
+                            : launch_gemm_gs(a, R, s));
 }
 
 moe_status run_combine(moe_plan p, int n, const void* y_perm, const int32_t* pos,

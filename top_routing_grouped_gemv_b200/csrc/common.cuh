@@ -42,6 +42,17 @@ __device__ __forceinline__ float sel_f(bool c, float a, float b) {
       : "f"(a), "f"(b), "r"(static_cast<int>(c)));
   return r;
 }
+// Two fp32 fused multiply-adds in one instruction (sm_100 packed f32x2),
+// each rounded exactly as the scalar fmaf.
+__device__ __forceinline__ void fma_f32x2(float& d0, float& d1, float a0, float a1, float b0,
+                                          float b1) {
+  uint64_t d, a, b, c;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(c) : "f"(d0), "f"(d1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
 __device__ __forceinline__ int sel_i(bool c, int a, int b) {
   int r;
   asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\tselp.b32 %0, %1, %2, p;\n\t}"

@@ -57,6 +57,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "grouped_tiles.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
 
@@ -70,16 +71,13 @@ constexpr int BN = kTcBlockN;     // 256 accumulator columns per tile
 constexpr int ROWB = 128;         // bytes of K per row per stage (one swizzle atom)
 constexpr int A_BYTES = BM * ROWB;
 // producer warp, MMA warp, epilogue warps: four (one per TMEM lane
-// quadrant); for the group-scaled epilogues, whose fp32 sums live in
-// registers, eight with block scales (two per quadrant, 128 columns each)
-// and sixteen with per-column scales (four per quadrant, 64 columns each:
-// twice the warps to overlap the per-column work; measured 4.3 -> 3.4 ms on
-// the full fp8 workload, while block scales ran 1.6 -> 2.6 ms with sixteen)
-template <int kEpi>
-constexpr int gs_epi_warps() { return kEpi == kEpiGroupScale ? 16 : 8; }
+// quadrant); eight for the block-scaled epilogue, whose fp32 sums live in
+// registers (two per quadrant, 128 columns each; sixteen ran 1.6 -> 2.6 ms
+// on the full fp8 workload)
+constexpr int kBsEpiWarps = 8;
 template <int kEpi>
 constexpr int threads_of() {
-  return kEpi == kEpiGroupScale || kEpi == kEpiBlockScale ? 32 * (2 + gs_epi_warps<kEpi>()) : 192;
+  return kEpi == kEpiBlockScale ? 32 * (2 + kBsEpiWarps) : 192;
 }
 constexpr uint32_t kTmemCols = 2 * BN;
 constexpr int kMaxGroups = 256;
@@ -101,29 +99,6 @@ struct Geo {
   static constexpr int kSmemBytes = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES +
                                     kNumBars * 8 + 16 + 2 * (kMaxGroups + 1) * 4;
 };
-
-struct TileCoord {
-  int g, m_row0, n_tile;
-  int m_tile;  // row tile counted over all groups' (padded) row tiles
-};
-
-template <int TILE_M>
-__device__ __forceinline__ TileCoord decode_tile(int T, const int* s_pref, const int* s_off,
-                                                 int G, int n_tiles) {
-  int lo = 0, hi = G - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (s_pref[mid] <= T) lo = mid; else hi = mid - 1;
-  }
-  TileCoord c;
-  c.g = lo;
-  const int local = T - s_pref[lo];
-  const int mt = (s_off[lo + 1] - s_off[lo] + TILE_M - 1) / TILE_M;
-  c.n_tile = local / mt;
-  c.m_row0 = s_off[lo] + (local - c.n_tile * mt) * TILE_M;
-  c.m_tile = s_pref[lo] / n_tiles + (local - c.n_tile * mt);
-  return c;
-}
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.f + __expf(-g)) * u; }
 
@@ -153,8 +128,10 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
   static_assert(!kMx || (kFp8 && !kPair && kEpi == kEpiStore), "MX: e4m3, single CTA, store");
   static_assert(!kGather || (!kFp8 && !kPair && !kMx && kEpi == kEpiSwiglu),
                 "gathered A: bf16 SwiGLU, single CTA");
-  constexpr bool kGs = kEpi == kEpiGroupScale || kEpi == kEpiBlockScale;
-  static_assert(!kGs || (kFp8 && !kPair && !kMx), "group scales: e4m3, single CTA");
+  // per-column group scales run in gemm_gs.cu; block scales here
+  constexpr bool kGs = kEpi == kEpiBlockScale;
+  static_assert(kEpi != kEpiGroupScale, "per-column group scales: gemm_gs_kernel");
+  static_assert(!kGs || (kFp8 && !kPair && !kMx), "block scales: e4m3, single CTA");
   using Gm = Geo<kPair, kMx>;
   constexpr int STAGES = Gm::STAGES;
   constexpr int kAcc = kMx ? 1 : 2;  // accumulators in TMEM
@@ -180,36 +157,8 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
   const int nunits = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   // Per-group tile counts -> exclusive prefix (warp 0), group row offsets.
-  if (warp == 0) {
-    const int per = (G + 31) / 32;
-    const int b0 = min(G, lane * per), b1 = min(G, b0 + per);
-    int local = 0;
-    for (int q = b0; q < b1; ++q) {
-      int o0 = args.offsets ? args.offsets[q] : 0;
-      int o1 = args.offsets ? args.offsets[q + 1] : args.m_total;
-      s_off[q] = o0;
-      int cnt = max(0, o1 - o0);
-      int t = (cnt + Gm::TILE_M - 1) / Gm::TILE_M * args.n_tiles;
-      s_pref[q] = t;
-      local += t;
-    }
-    int incl = local;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    int run = incl - local;
-    for (int q = b0; q < b1; ++q) {
-      int t = s_pref[q];
-      s_pref[q] = run;
-      run += t;
-    }
-    if (lane == 31) {
-      s_pref[G] = incl;
-      s_off[G] = args.offsets ? args.offsets[G] : args.m_total;
-    }
-  }
+  if (warp == 0)
+    build_tile_prefix<Gm::TILE_M>(args.offsets, G, args.m_total, args.n_tiles, lane, s_pref, s_off);
   if (threadIdx.x == 32) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar(Gm::kBarFull + s), 1);
@@ -217,7 +166,7 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar(Gm::kBarTFull + a), 1);
-      mbar_init(bar(Gm::kBarTEmpty + a), kGs ? gs_epi_warps<kEpi>() : kPair ? 8 : 4);
+      mbar_init(bar(Gm::kBarTEmpty + a), kGs ? kBsEpiWarps : kPair ? 8 : 4);
     }
     mbar_init(bar(Gm::kBarDrain), 1);
     *abort_flag = 0;
@@ -436,11 +385,11 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5; 2..9 or 2..17 group-scaled) ----------------
+    // ---------------- epilogue (warps 2..5; 2..9 block-scaled) ----------------
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     int i = 0;
     if constexpr (kGs) {
-      constexpr int kCols = BN / (gs_epi_warps<kEpi>() / 4);  // columns of this warp
+      constexpr int kCols = BN / (kBsEpiWarps / 4);  // columns of this warp
       const int half = (warp - 2) >> 2;               // its column slice
       const int nblk = (args.n_out + 127) / 128;
       uint32_t j = 0;
@@ -456,34 +405,24 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
         float sum[kCols];
 #pragma unroll
         for (int cc = 0; cc < kCols; ++cc) sum[cc] = 0.f;
-        // the stage's row scale (and block scale) are loaded one stage ahead,
+        // the stage's row scale and block scale are loaded one stage ahead,
         // so their latency is not on the path from TFull to TEmpty
         const float* xrow = valid && args.xgs != nullptr ? args.xgs + srow * num_kb : nullptr;
         const float* wblk = args.wgs + static_cast<long long>(c.g) * num_kb * nblk + col0 / 128;
         float sx_next = xrow ? xrow[0] : 1.f;
-        float wb_next = kEpi == kEpiBlockScale ? wblk[0] : 0.f;
-        // per-column scales of the stage: four per lane (128 columns from col0)
-        const float4* wcol = reinterpret_cast<const float4*>(
-                                 args.wgs + static_cast<long long>(c.g) * num_kb * args.n_out + col0) +
-                             lane;
-        float4 wc_next = kEpi == kEpiGroupScale ? __ldg(wcol) : make_float4(0.f, 0.f, 0.f, 0.f);
+        float wb_next = wblk[0];
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb, ++j) {
           const uint32_t a = j & 1u, aph = (j >> 1) & 1u;
           const float sx = sx_next, wb = wb_next;
-          const float4 wc = wc_next;
           if (kb + 1 < num_kb) {
             if (xrow) sx_next = xrow[kb + 1];
-            if (kEpi == kEpiBlockScale) wb_next = wblk[static_cast<long long>(kb + 1) * nblk];
-            if (kEpi == kEpiGroupScale)
-              wc_next = __ldg(reinterpret_cast<const float4*>(
-                                  reinterpret_cast<const float*>(wcol) +
-                                  static_cast<long long>(kb + 1) * args.n_out));
+            wb_next = wblk[static_cast<long long>(kb + 1) * nblk];
           }
           ok = __shfl_sync(0xffffffffu, mbar_wait(bar(Gm::kBarTFull + a), aph, abort_flag), 0);
           if (!ok) break;
           tc_fence_after();
-          if constexpr (kEpi == kEpiBlockScale) {
+          {
             // one 128 x 128 weight block covers this warp's columns
             const float f = sx * wb;
 #pragma unroll
@@ -493,27 +432,9 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
               tmem_ld16(tq + a * BN + cc, v);
               tmem_ld_wait();
 #pragma unroll
-              for (int jj = 0; jj < 16; ++jj) sum[cc + jj] = fmaf(__uint_as_float(v[jj]), f, sum[cc + jj]);
-            }
-          } else {
-            // per-column scales: lane l holds those of columns 4l..4l+3 from
-            // this warp's first column (the warp uses the first kCols / 4
-            // lanes'), loaded a stage ahead; each column takes its scale
-            // from that lane by a shuffle (sx is this lane's own row's)
-            const float4 w = wc;
-#pragma unroll
-            for (int cc = 0; cc < kCols; cc += 8) {
-              uint32_t v[8];
-              __syncwarp();
-              tmem_ld8(tq + a * BN + cc, v);
-              tmem_ld_wait();
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj) {
-                const int col = cc + jj;
-                const float part = (col & 3) == 0 ? w.x : (col & 3) == 1 ? w.y : (col & 3) == 2 ? w.z : w.w;
-                const float f = __shfl_sync(0xffffffffu, part, col >> 2) * sx;
-                sum[col] = fmaf(__uint_as_float(v[jj]), f, sum[col]);
-              }
+              for (int jj = 0; jj < 16; jj += 2)
+                fma_f32x2(sum[cc + jj], sum[cc + jj + 1], __uint_as_float(v[jj]),
+                          __uint_as_float(v[jj + 1]), f, f);
             }
           }
           tc_fence_before();
@@ -789,10 +710,10 @@ cudaError_t launch_gemm_tc(const TcGemmArgs& args, int dtype, int epilogue, int 
     if (pair || epilogue != kEpiStore || !args.sfa || !args.sfb) return cudaErrorInvalidValue;
     return launch_t<true, kEpiStore, false, true>(args, max_units, stream);
   }
-  if (epilogue == kEpiGroupScale || epilogue == kEpiBlockScale) {
+  if (epilogue == kEpiGroupScale) return cudaErrorInvalidValue;  // launch_gemm_gs
+  if (epilogue == kEpiBlockScale) {
     if (pair || dtype != kE4M3 || !args.wgs || args.kdim % 128) return cudaErrorInvalidValue;
-    return epilogue == kEpiGroupScale ? launch_t<true, kEpiGroupScale, false>(args, max_units, stream)
-                                      : launch_t<true, kEpiBlockScale, false>(args, max_units, stream);
+    return launch_t<true, kEpiBlockScale, false>(args, max_units, stream);
   }
   const bool fp8 = dtype == kE4M3;
   const bool sw = epilogue == kEpiSwiglu;

@@ -218,6 +218,13 @@ cudaError_t launch_gemm_tc(const TcGemmArgs& args, int dtype, int epilogue, int 
                            bool pair, cudaStream_t stream);
 constexpr int kTcBlockM = 128;
 constexpr int kTcBlockN = 256;  // accumulator columns; SwiGLU: 128 gate + 128 up
+
+// e4m3 GEMM with per-column group scales (the kEpiGroupScale arithmetic;
+// launch_gemm_tc refuses that epilogue): 128 x 128 tiles, so args.n_tiles =
+// ceil(n_out / kGsTileN) and tmB0 has 128-row boxes; the other fields as for
+// launch_gemm_tc's block-scaled epilogue.
+constexpr int kGsTileN = 128;
+cudaError_t launch_gemm_gs(const TcGemmArgs& args, int rows_upper, cudaStream_t stream);
 constexpr int kGemmMxE4M3 = 3;
 
 // ---- MX (OCP MXFP8) block scales in the tensor-core layout ----------------
