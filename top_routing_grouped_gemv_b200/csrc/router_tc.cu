@@ -74,18 +74,21 @@ router_split_kernel(const float* __restrict__ w_r, int d, int E, __nv_bfloat16* 
 // ---- fused router: logits on tcgen05, top-K in the epilogue (33..128 experts) ----
 //
 // One CTA pair (a cluster of two, tcgen05 cta_group::2) per 256-token tile:
-// each CTA loads its 128 token rows and half of every weight part, the
-// leader issues M=256 MMAs over both CTAs' shared memory, and each CTA's
+// each CTA loads its 128 token rows and half of the weight rows, the leader
+// issues M=256 MMAs over both CTAs' shared memory, and each CTA's
 // accumulators hold its own 128 tokens -- half the weight bytes per CTA and
-// stage of a single-CTA tile, which is what sets the pace (the weights are
-// read by every tile).  The plan holds w_r split into its three bf16
-// parts as 3*EP K-major rows [hi(EP) | mid(EP) | lo(EP)] (EP = E rounded up
-// to 32, rows past E zero), made once (router_split3_kernel).  Per 64-element
-// K stage each CTA loads its 128 token rows and its EP/2 rows of each part by
-// TMA (128-byte swizzle); the leader's MMA thread issues, per K=16 step, one
-// M=256, N=EP tcgen05.mma per part into its own fp32 accumulator (TMEM
-// columns [0,EP) hi, [EP,2EP) mid, [2EP,3EP) lo: bf16 x bf16 products are
-// exact in fp32, each part keeps its own rounding scale).  The four
+// stage of a single-CTA tile (the weights are read by every tile).  The
+// plan holds w_r split into its three bf16 parts as 3*EP K-major rows
+// [hi(EP) | mid(EP) | lo(EP)] (EP = E rounded up to 32, rows past E zero),
+// made once (router_split3_kernel).  Per 64-element K stage each CTA loads
+// its 128 token rows and its half of the weight rows by TMA (128-byte
+// swizzle); the leader's MMA thread issues, per K=16 step, one M=256 MMA of
+// N = 3*EP (EP = 64) or two, of N = 2*EP and N = EP (FrGeo), whose output
+// columns are the parts' fp32 accumulators (TMEM columns [0,EP) hi,
+// [EP,2EP) mid, [2EP,3EP) lo: bf16 x bf16 products are exact in fp32, each
+// part keeps its own rounding scale).  Wide MMAs matter: with one N=EP MMA
+// per part the MMAs alone took 37 us for a tile's 32 stages, three times
+// their tensor-pipe time.  The four
 // epilogue warps then own one token row each per lane (TMEM lane = token):
 //   logit[e] = ((hi + mid) + lo) + bias[e]
 // and the top-K (value descending, equal values to the lower expert) in
@@ -108,8 +111,17 @@ constexpr int kFrKE = 64;       // K elements per stage (128 bytes of bf16)
 
 template <int EP>
 struct FrGeo {
+  // The 3*EP weight rows [hi | mid | lo] go to the tensor core as one MMA
+  // of N = 3*EP columns when that fits (N <= 256: EP = 64), else as one of
+  // the first two parts (N = 2*EP) and one of the third (N = EP): few wide
+  // MMAs, each reading the token tile once, instead of one narrow MMA per
+  // part.  In a CTA pair each MMA's weight rows are split in halves, the
+  // first half in the leader's shared memory and the second in the peer's;
+  // a CTA's halves of the chunks sit back to back, as PARTS0 + (PARTS0 ==
+  // 2) boxes of EP/2 rows.
+  static constexpr int PARTS0 = 3 * EP <= 256 ? 3 : 2;  // parts in the first MMA
   static constexpr int A_BYTES = kFrBM * 128;
-  static constexpr int B_BYTES = 3 * (EP / 2) * 128;  // this CTA's half of each part
+  static constexpr int B_BYTES = 3 * (EP / 2) * 128;  // this CTA's halves of the chunks
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = EP <= 64 ? 7 : EP <= 96 ? 6 : 5;
   static constexpr int kBarFull = 0, kBarEmpty = STAGES, kBarTFull = 2 * STAGES,
@@ -220,9 +232,14 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         if (leader) mbar_expect_tx(bar(Gm::kBarFull + s), 2 * Gm::STAGE_BYTES);
         tma_load_2d_pair(sA + s * Gm::A_BYTES, &tmX, kx, row0, full_leader);
 #pragma unroll
-        for (int p = 0; p < 3; ++p)
-          tma_load_2d_pair(sB + s * Gm::B_BYTES + p * (EP / 2) * 128, &tmW, kx,
-                           p * EP + static_cast<int>(rank) * (EP / 2), full_leader);
+        for (int b = 0; b < 3; ++b) {
+          // box b: weight rows of the first MMA's half (b < PARTS0) or of
+          // the second's
+          const int wrow = b < Gm::PARTS0
+                               ? static_cast<int>(rank) * (Gm::PARTS0 * EP / 2) + b * (EP / 2)
+                               : Gm::PARTS0 * EP + static_cast<int>(rank) * (EP / 2);
+          tma_load_2d_pair(sB + s * Gm::B_BYTES + b * (EP / 2) * 128, &tmW, kx, wrow, full_leader);
+        }
         issued |= 1u << s;
         issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
         if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -238,10 +255,12 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && leader) {
-      // ---- MMA issuer (the pair's leader): three parts, each into its own accumulator ----
-      constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                                 (static_cast<uint32_t>(EP >> 3) << 17) |
-                                 (static_cast<uint32_t>((2 * kFrBM) >> 4) << 24);
+      // ---- MMA issuer (the pair's leader): each part into its own TMEM columns ----
+      // bf16 x bf16 -> fp32, M = 256 (the pair), N = the chunk's rows
+      constexpr uint32_t idesc_base = (1u << 4) | (1u << 7) | (1u << 10) |
+                                      (static_cast<uint32_t>((2 * kFrBM) >> 4) << 24);
+      constexpr uint32_t idesc0 = idesc_base | (static_cast<uint32_t>((Gm::PARTS0 * EP) >> 3) << 17);
+      constexpr uint32_t idesc1 = idesc_base | (static_cast<uint32_t>(EP >> 3) << 17);
       int s = 0;
       uint32_t ph = 0;
       bool aborted = false;
@@ -250,12 +269,14 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         tc_fence_after();
         const uint32_t a0 = sA + s * Gm::A_BYTES, b0 = sB + s * Gm::B_BYTES;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-#pragma unroll
-          for (int p = 0; p < 3; ++p)
-            tc_mma_pair<false>(tmem_base + static_cast<uint32_t>(p * EP), sw128_desc(a0 + 32 * k),
-                               sw128_desc(b0 + p * (EP / 2) * 128 + 32 * k), idesc,
-                               (it | k) != 0 ? 1u : 0u);
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t acc = (it | k) != 0 ? 1u : 0u;
+          tc_mma_pair<false>(tmem_base, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc0,
+                             acc);
+          if constexpr (Gm::PARTS0 == 2)
+            tc_mma_pair<false>(tmem_base + static_cast<uint32_t>(2 * EP), sw128_desc(a0 + 32 * k),
+                               sw128_desc(b0 + 2 * (EP / 2) * 128 + 32 * k), idesc1, acc);
+        }
         tc_commit_pair_both(bar(Gm::kBarEmpty + s));  // frees the stage in both CTAs
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
