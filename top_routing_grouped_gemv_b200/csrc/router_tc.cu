@@ -93,17 +93,19 @@ router_split_kernel(const float* __restrict__ w_r, int d, int E, __nv_bfloat16* 
 //   logit[e] = ((hi + mid) + lo) + bias[e]
 // and the top-K (value descending, equal values to the lower expert) in
 // three passes over the row:
-//   1. tau = min over KMAX+1 disjoint expert groups (group (e mod 32) mod
-//      (KMAX+1)) of the group maximum: at least KMAX+1 logits are >= tau,
-//      so every member of the top K+1 is;
-//   2. the logits >= tau (usually a dozen or two) are appended, in expert
-//      order, to the thread's list in shared memory (the pipeline buffers,
-//      free once the accumulators are final);
-//   3. they are inserted into a sorted K+1 list held in registers (an
-//      unrolled compare-and-shift; ties keep the earlier, lower expert).
+//   1. the logits go to shared memory (the pipeline buffers, free once the
+//      accumulators are final), and tau = min over KMAX+1 disjoint expert
+//      groups (group (e mod 32) mod (KMAX+1)) of the group maximum: at
+//      least KMAX+1 logits are >= tau, so every member of the top K+1 is;
+//   2. a bit per expert marks the logits >= tau (usually a dozen or two);
+//   3. the marked ones are inserted, in expert order, into a sorted K+1
+//      list held in registers (an unrolled compare-and-shift; ties keep the
+//      earlier, lower expert).
 // This touches each logit with a few instructions instead of a full
 // insertion, which matters because the four epilogue warps have the SM to
-// themselves (one tile per CTA) and are bound by instruction issue.
+// themselves (one tile per CTA) and are bound by instruction issue.  An
+// earlier pass 2 appended each candidate to a per-thread list in shared
+// memory: its data-dependent store per logit cost ~7 us of the tile.
 // Softmax over the kept K, margin = K-th minus (K+1)-th logit.
 
 constexpr int kFrBM = 128;      // tokens per tile
@@ -128,8 +130,8 @@ struct FrGeo {
                        kNumBars = 2 * STAGES + 1;
   // ring | barriers | TMEM slot + abort flag (16 B) | bias (EP floats)
   static constexpr int kSmemBytes = 1024 + STAGES * STAGE_BYTES + kNumBars * 8 + 16 + EP * 4;
-  // candidate lists of the epilogue: EP entries of (value, expert) per token
-  static_assert(kFrBM * EP * 8 <= STAGES * STAGE_BYTES, "candidate lists fit the ring");
+  // the epilogue's logits: EP floats per token
+  static_assert(kFrBM * EP * 4 <= STAGES * STAGE_BYTES, "the tile's logits fit the ring");
 };
 
 // Inserts (v, e) into a descending list of L entries held in registers (L
@@ -299,11 +301,18 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
       const long long t = static_cast<long long>(row0) + r;
       const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       constexpr int G = KMAX + 1;  // disjoint expert groups for the threshold
-      // pass 1: the group maxima -> tau
+      // The passes run chunk by chunk (32 experts unrolled, the chunks in a
+      // loop): fully unrolled over all EP experts the epilogue is thousands
+      // of instructions executed once, and fetching them cost more than
+      // running them.
+      // pass 1: the logits, into the ring (logit e of row r at float index
+      // e * 128 + r: a warp's 32 rows are 32 consecutive words), and the
+      // group maxima -> tau
+      float* lg = reinterpret_cast<float*>(smem);
       float gmax[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) gmax[g] = -INFINITY;
-#pragma unroll
+#pragma unroll 1
       for (int cc = 0; cc < EP; cc += 32) {
         uint32_t vh[32], vm[32], vl[32];
         __syncwarp();
@@ -317,6 +326,7 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
           if (e < E) {
             const float v = ((__uint_as_float(vh[j]) + __uint_as_float(vm[j])) +
                              __uint_as_float(vl[j])) + s_bias[e];
+            lg[e * kFrBM + r] = v;
             gmax[j % G] = fmaxf(gmax[j % G], v);  // group (e mod 32) mod G: a constant index
           }
         }
@@ -324,33 +334,10 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
       float tau = gmax[0];
 #pragma unroll
       for (int g = 1; g < G; ++g) tau = fminf(tau, gmax[g]);
-      // pass 2: the candidates >= tau, in expert order, to this thread's list
-      // (entry i of row r at float2 index i * 128 + r of the ring)
-      float2* cand = reinterpret_cast<float2*>(smem);
-      int cnt = 0;
-#pragma unroll
-      for (int cc = 0; cc < EP; cc += 32) {
-        uint32_t vh[32], vm[32], vl[32];
-        __syncwarp();
-        tmem_ld32(tq + cc, vh);
-        tmem_ld32(tq + EP + cc, vm);
-        tmem_ld32(tq + 2 * EP + cc, vl);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int e = cc + j;
-          if (e < E) {
-            const float v = ((__uint_as_float(vh[j]) + __uint_as_float(vm[j])) +
-                             __uint_as_float(vl[j])) + s_bias[e];
-            if (v >= tau) {
-              cand[cnt * kFrBM + r] = make_float2(v, __int_as_float(e));
-              ++cnt;
-            }
-          }
-        }
-      }
-      // pass 3: sorted top KMAX+1 of the candidates (K <= KMAX reads the
-      // first K+1: the list keeps a superset of what it needs)
+      // passes 2 and 3, per chunk: a bit per expert whose logit is >= tau
+      // (no branches, no data-dependent addresses), then those inserted in
+      // expert order into a sorted top KMAX+1 (K <= KMAX reads the first
+      // K+1: the list keeps a superset of what it needs)
       float val[G];
       int idx[G];
 #pragma unroll
@@ -358,9 +345,17 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         val[j] = -INFINITY;
         idx[j] = 0x7fffffff;
       }
-      for (int i = 0; i < cnt; ++i) {
-        const float2 c = cand[i * kFrBM + r];
-        fr_insert<G>(c.x, __float_as_int(c.y), val, idx);
+#pragma unroll 1
+      for (int cc = 0; cc < EP; cc += 32) {
+        uint32_t m = 0u;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (cc + j < E) m |= static_cast<uint32_t>(lg[(cc + j) * kFrBM + r] >= tau) << j;
+        while (m != 0u) {
+          const int e = cc + __ffs(m) - 1;
+          m &= m - 1u;
+          fr_insert<G>(lg[e * kFrBM + r], e, val, idx);
+        }
       }
       if (t < N) {
         // every index below is a constant within the list (j < KMAX < G), so
