@@ -155,12 +155,13 @@ def measure_peak(steps_burst: int = 10, sustain_s: float = 4.0):
 
 
 def kernel_source_hash() -> str:
-    """Hash of what the grouped-GEMM kernel is compiled from: its own source,
-    the PTX helpers, the common helpers and its argument struct (the rest of
-    the launcher header does not change the kernel)."""
+    """Hash of what the grouped-GEMM kernels are compiled from: their sources
+    (the 128 x 256 kernel and the per-group-scale one), the shared tile
+    schedule, the PTX helpers, the common helpers and their argument struct
+    (the rest of the launcher header does not change the kernels)."""
     csrc = os.path.join(ROOT, "top_routing_grouped_gemv_b200", "csrc")
     h = hashlib.sha256()
-    for name in ("gemm_tc.cu", "tc_ptx.cuh", "common.cuh"):
+    for name in ("gemm_tc.cu", "gemm_gs.cu", "grouped_tiles.cuh", "tc_ptx.cuh", "common.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     with open(os.path.join(csrc, "kernels.h")) as f:

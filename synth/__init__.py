@@ -21,7 +21,8 @@ Workloads (the five shapes the layer is measured and checked on):
 * ``e4m3grp_n8192_h7168_e256_k8_n2048_gmm``  the same with fp32 scales per output column and
   128-element group of K for the weights (per token and group for the activations)
 * ``e4m3_n2048_h7168_e64_k8_n2048_gmm``, ``e4m3mx_n2048_h7168_e64_k8_n2048_gmm``,
-  ``e4m3blk_n2048_h7168_e64_k8_n2048_gmm`` reduced copies of the fp8 layers for kernel profiling
+  ``e4m3blk_n2048_h7168_e64_k8_n2048_gmm``, ``e4m3grp_n2048_h7168_e64_k8_n2048_gmm`` reduced copies of
+  the fp8 layers for kernel profiling
 
 Value recipe: x ~ N(0,1); router and expert weights ~ N(0, 1/fan_in)
 (fan_in = d for the router and the first FFN matrices, F for the second);
@@ -132,6 +133,8 @@ MX_GMM_PROFILE = _reg(MoEConfig("e4m3mx_n2048_h7168_e64_k8_n2048_gmm", DTYPE_E4M
                                 8, 2048, ACT_NONE, index=7, routing="given", quant="mx"))
 BLOCK_GMM_PROFILE = _reg(MoEConfig("e4m3blk_n2048_h7168_e64_k8_n2048_gmm", DTYPE_E4M3, 2048, 7168,
                                    64, 8, 2048, ACT_NONE, index=9, routing="given", quant="block"))
+GROUP_GMM_PROFILE = _reg(MoEConfig("e4m3grp_n2048_h7168_e64_k8_n2048_gmm", DTYPE_E4M3, 2048, 7168,
+                                   64, 8, 2048, ACT_NONE, index=11, routing="given", quant="group"))
 
 
 # ----------------------------------------------------------------------------
