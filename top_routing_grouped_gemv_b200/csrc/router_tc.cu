@@ -128,10 +128,12 @@ struct FrGeo {
   static constexpr int STAGES = EP <= 64 ? 7 : EP <= 96 ? 6 : 5;
   static constexpr int kBarFull = 0, kBarEmpty = STAGES, kBarTFull = 2 * STAGES,
                        kNumBars = 2 * STAGES + 1;
-  // ring | barriers | TMEM slot + abort flag (16 B) | bias (EP floats)
-  static constexpr int kSmemBytes = 1024 + STAGES * STAGE_BYTES + kNumBars * 8 + 16 + EP * 4;
-  // the epilogue's logits: EP floats per token
-  static_assert(kFrBM * EP * 4 <= STAGES * STAGE_BYTES, "the tile's logits fit the ring");
+  // ring | barriers | TMEM slot + abort flag (16 B) | bias (EP floats) |
+  // the epilogue warp pairs' go-ahead flags (8 ints)
+  static constexpr int kSmemBytes = 1024 + STAGES * STAGE_BYTES + kNumBars * 8 + 16 + EP * 4 + 32;
+  // the epilogue's logits (EP floats per token), the exchanged group maxima
+  // (2 * (KMAX + 1) floats per token) and half lists ((KMAX + 1) float2)
+  static_assert(kFrBM * (EP + 4 * 9) * 4 <= STAGES * STAGE_BYTES, "the epilogue's data fit the ring");
 };
 
 // Inserts (v, e) into a descending list of L entries held in registers (L
@@ -152,8 +154,17 @@ __device__ __forceinline__ void fr_insert(float v, int e, float (&val)[L], int (
   }
 }
 
+// Threads: warp 0 TMA producer, warp 1 MMA issuer, warps 2..9 epilogue (two
+// per TMEM lane quadrant, each selecting over half of the experts).
+constexpr int kFrThreads = 320;
+
+__device__ __forceinline__ void fr_pair_bar(int q) {
+  // the two epilogue warps of lane quadrant q (named barrier 1 + q)
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(64) : "memory");
+}
+
 template <int EP, int KMAX>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kFrThreads, 1)
 router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                     const float* __restrict__ bias, int N, int d, int E, int K,
                     int32_t* __restrict__ ids, float* __restrict__ gates,
@@ -175,6 +186,7 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Gm::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* s_bias = reinterpret_cast<float*>(tmem_slot + 4);
+  int* s_pair_ok = reinterpret_cast<int*>(s_bias + EP);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -290,54 +302,70 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     }
     __syncwarp();
   } else {
-    // ---- epilogue: one token per lane ----
-    const int q = warp & 3;  // TMEM lane quadrant of this warp
-    const bool ok = __shfl_sync(0xffffffffu, mbar_wait(bar(Gm::kBarTFull), 0, abort_flag), 0);
+    // ---- epilogue: one token per lane, two warps per token row ----
+    const int q = warp & 3;            // TMEM lane quadrant of this warp
+    const int h = (warp - 2) >> 2;     // its half of the experts
+    const bool ok_self =
+        __shfl_sync(0xffffffffu, mbar_wait(bar(Gm::kBarTFull), 0, abort_flag), 0);
+    // the pair goes on only if both of its warps saw the accumulators final
+    // (every barrier below is shared by the pair)
+    if (lane == 0) s_pair_ok[2 * q + h] = ok_self ? 1 : 0;
+    fr_pair_bar(q);
+    const bool ok = ok_self && s_pair_ok[2 * q + (1 - h)] != 0;
     if (!ok) {
-      set_status(status, kStatusTimeout);
+      if (!ok_self) set_status(status, kStatusTimeout);
     } else {
       tc_fence_after();
       const int r = q * 32 + lane;  // row of the tile
       const long long t = static_cast<long long>(row0) + r;
       const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      constexpr int G = KMAX + 1;  // disjoint expert groups for the threshold
-      // The passes run chunk by chunk (32 experts unrolled, the chunks in a
-      // loop): fully unrolled over all EP experts the epilogue is thousands
-      // of instructions executed once, and fetching them cost more than
-      // running them.
-      // pass 1: the logits, into the ring (logit e of row r at float index
-      // e * 128 + r: a warp's 32 rows are 32 consecutive words), and the
-      // group maxima -> tau
+      constexpr int G = KMAX + 1;   // disjoint expert groups for the threshold
+      constexpr int HALF = EP / 2;  // experts per warp of the pair
+      const int e0 = h * HALF;
+      // Per 16-expert chunk (the chunks in a loop: fully unrolled over the
+      // experts the epilogue is thousands of instructions executed once,
+      // and fetching them cost more than running them).
+      // pass 1: this half's logits, into the ring (logit e of row r at float
+      // index e * 128 + r: a warp's 32 rows are 32 consecutive words), and
+      // its group maxima (group = position in the chunk mod G)
       float* lg = reinterpret_cast<float*>(smem);
       float gmax[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) gmax[g] = -INFINITY;
 #pragma unroll 1
-      for (int cc = 0; cc < EP; cc += 32) {
-        uint32_t vh[32], vm[32], vl[32];
+      for (int cc = 0; cc < HALF; cc += 16) {
+        uint32_t vh[16], vm[16], vl[16];
         __syncwarp();
-        tmem_ld32(tq + cc, vh);
-        tmem_ld32(tq + EP + cc, vm);
-        tmem_ld32(tq + 2 * EP + cc, vl);
+        tmem_ld16(tq + e0 + cc, vh);
+        tmem_ld16(tq + EP + e0 + cc, vm);
+        tmem_ld16(tq + 2 * EP + e0 + cc, vl);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int e = cc + j;
+        for (int j = 0; j < 16; ++j) {
+          const int e = e0 + cc + j;
           if (e < E) {
             const float v = ((__uint_as_float(vh[j]) + __uint_as_float(vm[j])) +
                              __uint_as_float(vl[j])) + s_bias[e];
             lg[e * kFrBM + r] = v;
-            gmax[j % G] = fmaxf(gmax[j % G], v);  // group (e mod 32) mod G: a constant index
+            gmax[j % G] = fmaxf(gmax[j % G], v);  // a constant index
           }
         }
       }
-      float tau = gmax[0];
+      // the pair's group maxima -> tau: at least KMAX+1 logits (one per
+      // group; experts 0..31 fill every position, so no group is empty) are
+      // >= tau, so every member of the top K+1 is
+      float* xg = lg + EP * kFrBM;
 #pragma unroll
-      for (int g = 1; g < G; ++g) tau = fminf(tau, gmax[g]);
+      for (int g = 0; g < G; ++g) xg[(h * G + g) * kFrBM + r] = gmax[g];
+      fr_pair_bar(q);
+      float tau = INFINITY;
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+        tau = fminf(tau, fmaxf(gmax[g], xg[((1 - h) * G + g) * kFrBM + r]));
       // passes 2 and 3, per chunk: a bit per expert whose logit is >= tau
       // (no branches, no data-dependent addresses), then those inserted in
-      // expert order into a sorted top KMAX+1 (K <= KMAX reads the first
-      // K+1: the list keeps a superset of what it needs)
+      // expert order into a sorted top KMAX+1 of this half (K <= KMAX reads
+      // the first K+1: the list keeps a superset of what it needs)
       float val[G];
       int idx[G];
 #pragma unroll
@@ -346,18 +374,36 @@ router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         idx[j] = 0x7fffffff;
       }
 #pragma unroll 1
-      for (int cc = 0; cc < EP; cc += 32) {
+      for (int cc = 0; cc < HALF; cc += 16) {
         uint32_t m = 0u;
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (cc + j < E) m |= static_cast<uint32_t>(lg[(cc + j) * kFrBM + r] >= tau) << j;
+        for (int j = 0; j < 16; ++j) {
+          const int e = e0 + cc + j;
+          if (e < E) m |= static_cast<uint32_t>(lg[e * kFrBM + r] >= tau) << j;
+        }
         while (m != 0u) {
-          const int e = cc + __ffs(m) - 1;
+          const int e = e0 + cc + __ffs(m) - 1;
           m &= m - 1u;
           fr_insert<G>(lg[e * kFrBM + r], e, val, idx);
         }
       }
-      if (t < N) {
+      // merge: the upper half's list into the lower half's; its experts are
+      // all higher, so inserting after equal values keeps ties on the lower
+      // expert
+      float2* xl = reinterpret_cast<float2*>(xg + 2 * G * kFrBM);
+      if (h == 1) {
+#pragma unroll
+        for (int j = 0; j < G; ++j) xl[j * kFrBM + r] = make_float2(val[j], __int_as_float(idx[j]));
+      }
+      fr_pair_bar(q);
+      if (h == 0) {
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          const float2 c = xl[j * kFrBM + r];
+          fr_insert<G>(c.x, __float_as_int(c.y), val, idx);
+        }
+      }
+      if (h == 0 && t < N) {
         // every index below is a constant within the list (j < KMAX < G), so
         // the list stays in registers
         float z = 0.f;
@@ -447,7 +493,7 @@ cudaError_t launch_fused_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   cfg.gridDim = dim3(static_cast<unsigned>(2 * ((N + 2 * kFrBM - 1) / (2 * kFrBM))));
-  cfg.blockDim = dim3(192);
+  cfg.blockDim = dim3(kFrThreads);
   cfg.dynamicSmemBytes = FrGeo<EP>::kSmemBytes;
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
