@@ -39,6 +39,13 @@ SMALL = {
     "bf16_tc_router_e100_k3": synth.MoEConfig("tc_e100", "bf16", 333, 256, 100, 3, 128, "swiglu",
                                               zipf_bias=1.2),
     "bf16_tc_router_e256_k1": synth.MoEConfig("tc_e256", "bf16", 130, 128, 256, 1, 64, "swiglu"),
+    # the fused router's expert splits: 33 experts (the upper half of the
+    # 64-column tile holds one), 96 (48-expert halves, two MMAs of N = 192
+    # and 96), 127 (one padding column); ragged token counts, K from 1 to 8
+    "bf16_tc_router_e33_k2": synth.MoEConfig("tc_e33", "bf16", 300, 256, 33, 2, 64, "swiglu"),
+    "bf16_tc_router_e96_k8": synth.MoEConfig("tc_e96", "bf16", 520, 384, 96, 8, 64, "swiglu",
+                                             zipf_bias=1.2),
+    "bf16_tc_router_e127_k1": synth.MoEConfig("tc_e127", "bf16", 777, 192, 127, 1, 64, "swiglu"),
     # few tokens with long rows: split-K router (partial logits per slice of d)
     "bf16_splitk_e8": synth.MoEConfig("sk_e8", "bf16", 40, 2048, 8, 2, 128, "swiglu"),
     "bf16_splitk_e256_k8": synth.MoEConfig("sk_e256", "bf16", 130, 1024, 256, 8, 64, "swiglu"),
