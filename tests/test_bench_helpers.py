@@ -32,10 +32,10 @@ def test_profiled_traffic_follows_the_kernel_source_hash(tmp_path, monkeypatch):
     h = bench.kernel_source_hash()
     assert re.fullmatch(r"[0-9a-f]{16}", h)
     prof = os.path.join(bench.ROOT, "profiles",
-                        "ffn1_swiglu_tc_bf16_n4096_d2048_e8_k2_f8192_swiglu.md")
+                        "ffn1_swiglu_tc_bf16_n16384_d2048_e128_k8_f768_swiglu_zipf.md")
     text = open(prof).read()
     committed = re.search(r"kernel_source_sha256_16: ([0-9a-f]+)", text).group(1)
-    value = bench.profiled_traffic("bf16_n4096_d2048_e8_k2_f8192_swiglu", "ffn1_swiglu_tc")
+    value = bench.profiled_traffic("bf16_n16384_d2048_e128_k8_f768_swiglu_zipf", "ffn1_swiglu_tc")
     if committed == h:
         assert value == float(re.search(r"dram_bytes_per_launch: ([0-9]+)", text).group(1))
     else:
