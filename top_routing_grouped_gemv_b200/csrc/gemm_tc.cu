@@ -14,7 +14,7 @@
 //               and 64 zero rows: columns [0,64) hi, [64,128) mid,
 //               [128,192) lo; one group, rows = tokens)
 //
-// Structure (one persistent CTA per SM, 6 warps):
+// Structure (one persistent CTA per SM, 10 warps):
 //   warp 0      TMA producer: 128-byte-swizzled K-major tiles of A (128 rows)
 //               and W (256 rows) into a 4-stage shared-memory ring (6
 //               stages of 128 + 128 rows per CTA in the CTA-pair mode)
@@ -22,8 +22,9 @@
 //               (M=128, N=256, K=16 bf16 / K=32 e4m3 per instruction) into
 //               one of two fp32 accumulators, and tcgen05.commit releases
 //               ring slots and hands finished accumulators to the epilogue
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows of their TMEM
-//               lane quadrant, activation/scale, bf16, 16-byte stores;
+//   warps 2..9  epilogue, two per TMEM lane quadrant, each taking half of
+//               the tile's columns: tcgen05.ld of the accumulator rows of
+//               their quadrant, activation/scale, bf16, 16-byte stores;
 //               overlaps the next tile's MMAs (double-buffered TMEM)
 // The tile list (group, row tile, column tile) is derived on the device
 // from the offsets, so no host synchronisation is needed; empty groups own
@@ -70,14 +71,18 @@ constexpr int BM = kTcBlockM;     // 128 rows per CTA (256 per CTA pair)
 constexpr int BN = kTcBlockN;     // 256 accumulator columns per tile
 constexpr int ROWB = 128;         // bytes of K per row per stage (one swizzle atom)
 constexpr int A_BYTES = BM * ROWB;
-// producer warp, MMA warp, epilogue warps: four (one per TMEM lane
-// quadrant); eight for the block-scaled epilogue, whose fp32 sums live in
-// registers (two per quadrant, 128 columns each; sixteen ran 1.6 -> 2.6 ms
-// on the full fp8 workload)
-constexpr int kBsEpiWarps = 8;
+// producer warp, MMA warp, eight epilogue warps: two per TMEM lane
+// quadrant, each draining half of the tile's columns (with one warp per
+// quadrant the epilogue's stores held back the next tiles' MMAs: the
+// fine-grained workload's down GEMM ran 420 us with its stores, 320 us
+// without).  The block-scaled epilogue, whose fp32 sums live in
+// registers, splits the columns the same way (sixteen warps ran 1.6 ->
+// 2.6 ms on the full fp8 workload).
+constexpr int kEpiWarps = 8;
+constexpr int kBsEpiWarps = kEpiWarps;
 template <int kEpi>
 constexpr int threads_of() {
-  return kEpi == kEpiBlockScale ? 32 * (2 + kBsEpiWarps) : 192;
+  return 32 * (2 + kEpiWarps);
 }
 constexpr uint32_t kTmemCols = 2 * BN;
 constexpr int kMaxGroups = 256;
@@ -96,11 +101,42 @@ struct Geo {
   static constexpr int kBarFull = 0, kBarEmpty = STAGES, kBarTFull = 2 * STAGES,
                        kBarTEmpty = 2 * STAGES + 2, kBarDrain = 2 * STAGES + 4,
                        kNumBars = 2 * STAGES + 5;
+  // ring | barriers | TMEM slot + abort flag | tile prefix and group offsets |
+  // the epilogue warps' 2 KB staging buffers for their stores (16-byte aligned)
   static constexpr int kSmemBytes = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES +
-                                    kNumBars * 8 + 16 + 2 * (kMaxGroups + 1) * 4;
+                                    kNumBars * 8 + 16 + 2 * (kMaxGroups + 1) * 4 + 16 +
+                                    kEpiWarps * 2048;
 };
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.f + __expf(-g)) * u; }
+
+// Stores a warp's chunk of 32 rows x 32 bf16 columns (lane l holds row l's
+// 16 packed words; dst: this lane's row at the chunk's first column, or
+// nullptr when the row is not stored) through the warp's 2 KB of shared
+// memory: lane l writes its row's four 16-byte units (unit u to slot
+// u ^ ((l >> 1) & 3): conflict-free), then each store instruction writes
+// 64 contiguous bytes into each of 8 rows -- whole 32-byte sectors, where a
+// store straight from the row-per-lane registers writes 16 bytes into each
+// of 32 rows 4 KB apart.
+__device__ __forceinline__ void store_chunk_rows(uint8_t* stage, int lane, const uint32_t (&pk)[16],
+                                                 __nv_bfloat16* dst) {
+  uint4* srow = reinterpret_cast<uint4*>(stage + lane * 64);
+  const int f = (lane >> 1) & 3;
+  __syncwarp();  // the previous chunk's reads are done
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    srow[u ^ f] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+  __syncwarp();
+  const int U = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int R = 8 * i + (lane >> 2);
+    const uint4 v = reinterpret_cast<const uint4*>(stage + R * 64)[U ^ ((R >> 1) & 3)];
+    const unsigned long long p =
+        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst), R);
+    if (p != 0ull) reinterpret_cast<uint4*>(p)[U] = v;
+  }
+}
 
 template <bool kFp8, bool kPair>
 constexpr uint32_t make_idesc_mode() {
@@ -148,6 +184,8 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_pref = reinterpret_cast<int*>(tmem_slot + 4);
   int* s_off = s_pref + (kMaxGroups + 1);
+  uint8_t* s_ostage = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(s_off + kMaxGroups + 1) + 15) & ~static_cast<uintptr_t>(15));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.groups;
@@ -166,7 +204,7 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar(Gm::kBarTFull + a), 1);
-      mbar_init(bar(Gm::kBarTEmpty + a), kGs ? kBsEpiWarps : kPair ? 8 : 4);
+      mbar_init(bar(Gm::kBarTEmpty + a), kPair ? 2 * kEpiWarps : kEpiWarps);
     }
     mbar_init(bar(Gm::kBarDrain), 1);
     *abort_flag = 0;
@@ -385,7 +423,7 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5; 2..9 block-scaled) ----------------
+    // ---------------- epilogue (warps 2..9, two per TMEM lane quadrant) ----------------
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     int i = 0;
     if constexpr (kGs) {
@@ -485,21 +523,29 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
       const TileCoord c = decode_tile<Gm::TILE_M>(T, s_pref, s_off, G, args.n_tiles);
       // lane quadrant q holds rows 32q.. of this CTA's 128 rows of the tile
       const int row = static_cast<int>(rank) * BM + q * 32 + lane;
-      // output columns of the tile
+      // output columns of the tile, and this warp's half of them
       constexpr int span = kEpi == kEpiSwiglu ? BN / 2 : kEpi == kEpiRouter ? BN / 4 : BN;
-      const int col0 = c.n_tile * span;
+      constexpr int hspan = span / 2;
+      const int hh = (warp - 2) >> 2;
+      const int col0 = c.n_tile * span + hh * hspan;
       const long long grow = static_cast<long long>(c.m_row0) + row;
       const bool valid = grow < s_off[c.g + 1] && grow < args.m_total && grow >= 0;
-      const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      // TMEM columns of the accumulator (and of its gate / up or hi / mid /
+      // lo parts) from this warp's first column
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN + hh * hspan);
       long long orow_i = grow;
       if (valid && args.out_rows != nullptr) orow_i = args.out_rows[grow];
+      // staged stores where the warp stores most of its 32 rows; a warp of a
+      // short tile (an expert's last rows, decode-shaped batches) stores
+      // its few rows directly
+      const bool staged = __popc(__ballot_sync(0xffffffffu, valid)) > 16;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + orow_i * args.ldo;
       if constexpr (kEpi == kEpiRouter) {
         float* frow = static_cast<float*>(args.out) + orow_i * args.ldo;
         const bool vec4 = (args.ldo & 3) == 0;
 #pragma unroll 1
-        for (int cc = 0; cc < span; cc += 32) {
+        for (int cc = 0; cc < hspan; cc += 32) {
           uint32_t vh[32], vm[32], vl[32];
           __syncwarp();
           tmem_ld32(tbase + cc, vh);             // hi part
@@ -526,26 +572,31 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
         }
       } else if (kEpi == kEpiSwiglu) {
 #pragma unroll 1
-        for (int cc = 0; cc < span; cc += 32) {
+        for (int cc = 0; cc < hspan; cc += 32) {
           uint32_t gr[32], ur[32];
           __syncwarp();
           tmem_ld32(tbase + cc, gr);          // gate columns
           tmem_ld32(tbase + span + cc, ur);   // up columns of the same outputs
           tmem_ld_wait();
           const int col = col0 + cc;
-          if (valid && col < args.n_out) {
+          const bool whole = col + 32 <= args.n_out;  // the same for the whole warp
+          if (whole && (staged || valid)) {
             uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j)
               pk[j] = pack_bf16x2(silu_mul(__uint_as_float(gr[2 * j]), __uint_as_float(ur[2 * j])),
                                   silu_mul(__uint_as_float(gr[2 * j + 1]),
                                            __uint_as_float(ur[2 * j + 1])));
-            if (col + 32 <= args.n_out) {
+            if (staged) {
+              store_chunk_rows(s_ostage + (warp - 2) * 2048, lane, pk, valid ? orow + col : nullptr);
+            } else {
               uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
               for (int j = 0; j < 4; ++j)
                 dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-            } else {
+            }
+          } else if (!whole && valid && col < args.n_out) {
+            {
 #pragma unroll
               for (int j = 0; j < 32; ++j)
                 if (col + j < args.n_out)
@@ -559,31 +610,41 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
         if (valid && args.row_scale != nullptr)
           rsc *= args.row_scale[args.row_index != nullptr ? args.row_index[grow] : grow];
 #pragma unroll 1
-        for (int cc = 0; cc < span; cc += 32) {
+        for (int cc = 0; cc < hspan; cc += 32) {
           uint32_t v[32];
           __syncwarp();
           tmem_ld32(tbase + cc, v);
           tmem_ld_wait();
           const int col = col0 + cc;
-          if (valid && col < args.n_out) {
-            const float sc = rsc;
+          const float sc = rsc;
+          const bool whole = col + 32 <= args.n_out;  // the same for the whole warp
+          if (whole && (staged || valid)) {
             if (args.col_scale != nullptr) {
               // per output channel: fold the channel scale into the values
+              const float* cs = args.col_scale + static_cast<long long>(c.g) * args.n_out + col;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * cs[j]);
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * sc, __uint_as_float(v[2 * j + 1]) * sc);
+            if (staged) {
+              store_chunk_rows(s_ostage + (warp - 2) * 2048, lane, pk, valid ? orow + col : nullptr);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            }
+          } else if (!whole && valid && col < args.n_out) {
+            if (args.col_scale != nullptr) {
               const float* cs = args.col_scale + static_cast<long long>(c.g) * args.n_out + col;
 #pragma unroll
               for (int j = 0; j < 32; ++j)
                 if (col + j < args.n_out) v[j] = __float_as_uint(__uint_as_float(v[j]) * cs[j]);
             }
-            if (col + 32 <= args.n_out) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + col);
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                dst[j] = make_uint4(
-                    pack_bf16x2(__uint_as_float(v[8 * j + 0]) * sc, __uint_as_float(v[8 * j + 1]) * sc),
-                    pack_bf16x2(__uint_as_float(v[8 * j + 2]) * sc, __uint_as_float(v[8 * j + 3]) * sc),
-                    pack_bf16x2(__uint_as_float(v[8 * j + 4]) * sc, __uint_as_float(v[8 * j + 5]) * sc),
-                    pack_bf16x2(__uint_as_float(v[8 * j + 6]) * sc, __uint_as_float(v[8 * j + 7]) * sc));
-            } else {
+            {
 #pragma unroll
               for (int j = 0; j < 32; ++j)
                 if (col + j < args.n_out) orow[col + j] = __float2bfloat16_rn(__uint_as_float(v[j]) * sc);
