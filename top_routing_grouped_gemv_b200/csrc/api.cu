@@ -340,6 +340,7 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
   a.n_tiles = (d.F + kTcBlockN / 2 - 1) / (kTcBlockN / 2);
   a.out = h;
   a.ldo = d.F;
+  a.out_tma = R > 0 && encode_out_map(&a.tmOut, h, R, d.F, d.F) ? 1 : 0;
   a.scale = 1.f;
   mark(p, s, a.a_rows ? "ffn1_swiglu_tc_gather" : "ffn1_swiglu_tc");
   if (launch_gemm_tc(a, d.dtype, kEpiSwiglu, R, pair_swiglu, s) != cudaSuccess) return MOE_ERR_CUDA;
@@ -353,6 +354,7 @@ moe_status run_ffn(moe_plan p, int n, const void* x_perm, const int32_t* offsets
   b.n_tiles = (d.d + kTcBlockN - 1) / kTcBlockN;
   b.out = y_perm;
   b.ldo = d.d;
+  b.out_tma = R > 0 && encode_out_map(&b.tmOut, y_perm, R, d.d, d.d) ? 1 : 0;
   mark(p, s, "ffn2_tc");
   p->launches += 2;
   return cuda_status(launch_gemm_tc(b, d.dtype, kEpiStore, R, pair, s));

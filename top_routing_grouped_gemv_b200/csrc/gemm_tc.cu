@@ -102,9 +102,10 @@ struct Geo {
                        kBarTEmpty = 2 * STAGES + 2, kBarDrain = 2 * STAGES + 4,
                        kNumBars = 2 * STAGES + 5;
   // ring | barriers | TMEM slot + abort flag | tile prefix and group offsets |
-  // the epilogue warps' 2 KB staging buffers for their stores (16-byte aligned)
+  // the epilogue warps' 2 KB staging buffers for their stores (1024-byte
+  // aligned: a buffer is also a TMA store's 64-byte-swizzled source)
   static constexpr int kSmemBytes = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES +
-                                    kNumBars * 8 + 16 + 2 * (kMaxGroups + 1) * 4 + 16 +
+                                    kNumBars * 8 + 16 + 2 * (kMaxGroups + 1) * 4 + 1024 +
                                     kEpiWarps * 2048;
 };
 
@@ -122,6 +123,7 @@ __device__ __forceinline__ void store_chunk_rows(uint8_t* stage, int lane, const
                                                  __nv_bfloat16* dst) {
   uint4* srow = reinterpret_cast<uint4*>(stage + lane * 64);
   const int f = (lane >> 1) & 3;
+  if (lane == 0) tc::bulk_wait_read0();  // a TMA store of the buffer has read it
   __syncwarp();  // the previous chunk's reads are done
 #pragma unroll
   for (int u = 0; u < 4; ++u)
@@ -135,6 +137,28 @@ __device__ __forceinline__ void store_chunk_rows(uint8_t* stage, int lane, const
     const unsigned long long p =
         __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst), R);
     if (p != 0ull) reinterpret_cast<uint4*>(p)[U] = v;
+  }
+}
+
+// The same chunk when all 32 rows are stored and are consecutive rows of
+// out: written to the buffer in the layout of a 32 x 32 box with 64-byte
+// swizzle (16-byte unit u of row r at unit u ^ ((r >> 1) & 3), the layout
+// above), then stored by one TMA instruction; the warp goes on without
+// waiting for the store.
+__device__ __forceinline__ void store_chunk_tma(uint8_t* stage, int lane, const uint32_t (&pk)[16],
+                                                const CUtensorMap* map, int col, int row) {
+  uint4* srow = reinterpret_cast<uint4*>(stage + lane * 64);
+  const int f = (lane >> 1) & 3;
+  if (lane == 0) tc::bulk_wait_read0();  // the previous store has read the buffer
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    srow[u ^ f] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+  tc::fence_proxy_async_smem();  // this lane's writes, visible to the TMA engine
+  __syncwarp();
+  if (lane == 0) {
+    tc::tma_store_2d(map, tc::smem_u32(stage), col, row);
+    tc::bulk_commit();
   }
 }
 
@@ -185,7 +209,7 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
   int* s_pref = reinterpret_cast<int*>(tmem_slot + 4);
   int* s_off = s_pref + (kMaxGroups + 1);
   uint8_t* s_ostage = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(s_off + kMaxGroups + 1) + 15) & ~static_cast<uintptr_t>(15));
+      (reinterpret_cast<uintptr_t>(s_off + kMaxGroups + 1) + 1023) & ~static_cast<uintptr_t>(1023));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.groups;
@@ -539,7 +563,11 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
       // staged stores where the warp stores most of its 32 rows; a warp of a
       // short tile (an expert's last rows, decode-shaped batches) stores
       // its few rows directly
-      const bool staged = __popc(__ballot_sync(0xffffffffu, valid)) > 16;
+      const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+      const bool staged = __popc(vmask) > 16;
+      // all 32 rows stored, consecutive in out: TMA tile stores
+      const bool tma_rows = args.out_tma != 0 && vmask == 0xffffffffu;
+      const int warp_row0 = static_cast<int>(c.m_row0) + static_cast<int>(rank) * BM + q * 32;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + orow_i * args.ldo;
       if constexpr (kEpi == kEpiRouter) {
         float* frow = static_cast<float*>(args.out) + orow_i * args.ldo;
@@ -588,7 +616,10 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
                                   silu_mul(__uint_as_float(gr[2 * j + 1]),
                                            __uint_as_float(ur[2 * j + 1])));
             if (staged) {
-              store_chunk_rows(s_ostage + (warp - 2) * 2048, lane, pk, valid ? orow + col : nullptr);
+              if (tma_rows)
+                store_chunk_tma(s_ostage + (warp - 2) * 2048, lane, pk, &args.tmOut, col, warp_row0);
+              else
+                store_chunk_rows(s_ostage + (warp - 2) * 2048, lane, pk, valid ? orow + col : nullptr);
             } else {
               uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
@@ -630,7 +661,10 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
             for (int j = 0; j < 16; ++j)
               pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * sc, __uint_as_float(v[2 * j + 1]) * sc);
             if (staged) {
-              store_chunk_rows(s_ostage + (warp - 2) * 2048, lane, pk, valid ? orow + col : nullptr);
+              if (tma_rows)
+                store_chunk_tma(s_ostage + (warp - 2) * 2048, lane, pk, &args.tmOut, col, warp_row0);
+              else
+                store_chunk_rows(s_ostage + (warp - 2) * 2048, lane, pk, valid ? orow + col : nullptr);
             } else {
               uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
@@ -659,6 +693,7 @@ __global__ void __launch_bounds__(threads_of<kEpi>(), 1) gemm_tc_kernel(const __
         else mbar_arrive(bar(Gm::kBarTEmpty + acc));
       }
     }
+    if (lane == 0) bulk_wait0();  // the warp's TMA tile stores have completed
   }
 
   tc_fence_before();
@@ -743,6 +778,19 @@ cudaError_t launch_t(const TcGemmArgs& args, long long max_units, cudaStream_t s
 }
 
 }  // namespace
+
+bool encode_out_map(CUtensorMap* map, void* base, long long rows, long long cols, long long ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows <= 0 || cols <= 0 || (ld * 2) % 16 != 0) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {32, 32};  // 64 bytes x 32 rows: one warp's chunk
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 bool encode_kmajor_map(CUtensorMap* map, const void* base, int elem_bytes, long long rows,
                        long long kdim, int box_rows) {

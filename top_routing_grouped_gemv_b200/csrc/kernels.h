@@ -201,7 +201,16 @@ struct TcGemmArgs {
   // high, 128 bytes of K); tmA is not read.
   const int32_t* a_rows;
   CUtensorMap tmAg;
+  // Tile stores by TMA (bf16 out with contiguous rows, out_rows NULL): when
+  // out_tma is set, tmOut covers out as m_total rows of n_out columns, ldo
+  // apart (encode_out_map: 32 x 32 boxes, 64-byte swizzle); a warp whose 32
+  // rows are all stored hands each 32-column chunk to the TMA engine.
+  CUtensorMap tmOut;
+  int out_tma;
 };
+
+// Host: the tile-store map of a bf16 (rows, cols) matrix, ld elements apart.
+bool encode_out_map(CUtensorMap* map, void* base, long long rows, long long cols, long long ld);
 
 // Host: encode a 2-D K-major tile map over a (rows, kdim) row-major matrix of
 // elem_bytes-wide elements; box = (128 bytes of K) x box_rows, 128-B swizzle.
